@@ -1,0 +1,145 @@
+"""Python binding of the seeded synthetic-input generator (``csrc/synth.c``).
+
+Every array returned is in the canonical (interchange) layout:
+
+* q4 weights: ``uint8 [N][K/2]``, element k in byte k/2, low nibble for even k,
+  4-bit two's complement (values -8..7);
+* q8 weights: ``int8 [N][K]``;
+* group scales: ``uint16 [N][K/32]`` holding fp16 bits;
+* activations: ``uint16 [M][K]`` holding bf16 bits.
+
+Streams identify tensors: one (seed, stream) pair per weight tensor, a separate
+stream for its scales and one per activation block, so any row of any tensor
+can be regenerated on its own.
+"""
+from __future__ import annotations
+
+import ctypes
+
+import numpy as np
+
+from . import build as _build
+
+_lib = None
+
+SCALE_STD = 0.02
+
+
+def lib() -> ctypes.CDLL:
+    global _lib
+    if _lib is None:
+        path = _build.build_synth()
+        L = ctypes.CDLL(path)
+        i64, u64 = ctypes.c_int64, ctypes.c_uint64
+        vp = ctypes.c_void_p
+        L.synth_q4.argtypes = [u64, u64, i64, i64, i64, vp]
+        L.synth_q8.argtypes = [u64, u64, i64, i64, i64, vp]
+        L.synth_scales.argtypes = [u64, u64, i64, i64, i64, ctypes.c_double, vp]
+        L.synth_bf16_normals.argtypes = [u64, u64, i64, i64, vp]
+        L.synth_normals_f64.argtypes = [u64, u64, i64, i64, vp]
+        L.synth_f64_to_f16_array.argtypes = [vp, i64, vp]
+        L.synth_f64_to_bf16_array.argtypes = [vp, i64, vp]
+        L.synth_words.argtypes = [u64, u64, i64, i64, vp]
+        for f in (L.synth_q4, L.synth_q8, L.synth_scales, L.synth_bf16_normals, L.synth_normals_f64):
+            f.restype = ctypes.c_int
+        L.synth_f64_to_f16_array.restype = None
+        L.synth_f64_to_bf16_array.restype = None
+        L.synth_words.restype = None
+        _lib = L
+    return _lib
+
+
+def _ptr(a: np.ndarray) -> int:
+    return a.ctypes.data
+
+
+def weights(bits: int, seed: int, stream: int, K: int, row0: int, nrows: int) -> np.ndarray:
+    """Canonical quantised weights for rows [row0, row0+nrows) of a tensor with K columns."""
+    if bits == 4:
+        out = np.empty((nrows, K // 2), dtype=np.uint8)
+        rc = lib().synth_q4(seed, stream, K, row0, nrows, _ptr(out))
+    elif bits == 8:
+        out = np.empty((nrows, K), dtype=np.int8)
+        rc = lib().synth_q8(seed, stream, K, row0, nrows, _ptr(out))
+    else:
+        raise ValueError("bits must be 4 or 8")
+    if rc != 0:
+        raise ValueError(f"synth: bad shape K={K} row0={row0} nrows={nrows}")
+    return out
+
+
+def scales(seed: int, stream: int, K: int, row0: int, nrows: int, std: float = SCALE_STD) -> np.ndarray:
+    """fp16 bits of the group scales |std * N(0,1)|, shape [nrows][K/32]."""
+    out = np.empty((nrows, K // 32), dtype=np.uint16)
+    if lib().synth_scales(seed, stream, K, row0, nrows, float(std), _ptr(out)) != 0:
+        raise ValueError(f"synth: bad shape K={K}")
+    return out
+
+
+def activations(seed: int, stream: int, M: int, K: int) -> np.ndarray:
+    """bf16 bits of M activation rows of N(0,1), shape [M][K]."""
+    out = np.empty((M, K), dtype=np.uint16)
+    if lib().synth_bf16_normals(seed, stream, 0, M * K, _ptr(out)) != 0:
+        raise ValueError("synth: bad activation shape")
+    return out
+
+
+def normals_f64(seed: int, stream: int, i0: int, count: int) -> np.ndarray:
+    out = np.empty(count, dtype=np.float64)
+    lib().synth_normals_f64(seed, stream, i0, count, _ptr(out))
+    return out
+
+
+def words(seed: int, stream: int, i0: int, count: int) -> np.ndarray:
+    out = np.empty(count, dtype=np.uint64)
+    lib().synth_words(seed, stream, i0, count, _ptr(out))
+    return out
+
+
+def f64_to_f16_bits(a: np.ndarray) -> np.ndarray:
+    a = np.ascontiguousarray(a, dtype=np.float64)
+    out = np.empty(a.shape, dtype=np.uint16)
+    lib().synth_f64_to_f16_array(_ptr(a), a.size, _ptr(out))
+    return out
+
+
+def f64_to_bf16_bits(a: np.ndarray) -> np.ndarray:
+    a = np.ascontiguousarray(a, dtype=np.float64)
+    out = np.empty(a.shape, dtype=np.uint16)
+    lib().synth_f64_to_bf16_array(_ptr(a), a.size, _ptr(out))
+    return out
+
+
+# ----------------------------------------------------------------------------
+# Stream identifiers of the workloads.  Each weight tensor has one id t; its
+# quantised values use stream 2t and its scales stream 2t+1.  Activations use
+# streams from ACT_STREAM_BASE up.
+# ----------------------------------------------------------------------------
+ACT_STREAM_BASE = 1 << 20
+
+
+def weight_stream(tensor_id: int) -> int:
+    return 2 * tensor_id
+
+
+def scale_stream(tensor_id: int) -> int:
+    return 2 * tensor_id + 1
+
+
+def act_stream(k_id: int) -> int:
+    return ACT_STREAM_BASE + k_id
+
+
+def tensor(bits: int, seed: int, tensor_id: int, N: int, K: int, row0: int = 0, nrows: int | None = None):
+    """(canonical q, fp16 scale bits) of one synthetic weight tensor (or a row slice of it)."""
+    if nrows is None:
+        nrows = N - row0
+    q = weights(bits, seed, weight_stream(tensor_id), K, row0, nrows)
+    s = scales(seed, scale_stream(tensor_id), K, row0, nrows)
+    return q, s
+
+
+__all__ = [
+    "weights", "scales", "activations", "normals_f64", "words", "f64_to_f16_bits", "f64_to_bf16_bits",
+    "tensor", "weight_stream", "scale_stream", "act_stream", "SCALE_STD", "lib",
+]

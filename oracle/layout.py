@@ -1,0 +1,87 @@
+"""Decoder of the kernel-native packed layout -- TEST INFRASTRUCTURE.
+
+Written from the layout's specification (the "Kernel-native packed layout"
+block of include/q4gemv.h), in the opposite direction to the library's packer:
+for every canonical element (n, k) it computes where the specification puts it
+and reads it back.  It shares no code with the library.  The pages describe no
+packed layout (the bs178.com llamAmpere post, "Why it is this fast", part one,
+only says the fork "fixed the reads" and staged them with async copies); the
+layout is this library's own design.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+ROWS = 16
+
+
+def _geometry(bits: int, N: int, K: int):
+    kc = 64 if bits == 4 else 32
+    T = -(-N // ROWS)
+    C = -(-K // kc)
+    CB = 576 if bits == 4 else 544
+    return T, C, CB
+
+
+def decode(bits: int, packed: np.ndarray, N: int, K: int) -> tuple[np.ndarray, np.ndarray]:
+    """Integer weights q [N][K] (int64) and fp16 scale bits [N][K/32] from packed bytes."""
+    T, C, CB = _geometry(bits, N, K)
+    packed = np.asarray(packed, dtype=np.uint8)
+    assert packed.size >= T * C * CB
+    n = np.arange(N, dtype=np.int64)[:, None]
+    k = np.arange(K, dtype=np.int64)[None, :]
+    t = n // ROWS
+    rr = n % ROWS
+    gi = rr % 8
+    upper = rr // 8  # 1 for the row R + 8 of the slot
+    if bits == 4:
+        c = k // 64
+        kk = k % 64
+        h = kk // 32
+        within = kk % 32
+        ti = within // 8
+        e = (within % 8) // 4
+        r4 = within % 4  # = 2*((i>>1)&1) + (i>>2)
+        i = 4 * (r4 % 2) + 2 * (r4 // 2) + upper
+        j = 2 * h + e
+        off = (t * C + c) * CB + 16 * (4 * gi + ti) + 4 * j
+        word = _word(packed, off)
+        u = (word >> (4 * i).astype(np.uint32)) & 0xF
+        q = u.astype(np.int64) - 8
+    else:
+        c = k // 32
+        within = k % 32
+        ti = within // 8
+        e = (within % 8) // 4
+        r4 = within % 4  # = 2f + (b>>1)
+        f = r4 // 2
+        b = 2 * (r4 % 2) + upper
+        j = 2 * e + f
+        off = (t * C + c) * CB + 16 * (4 * gi + ti) + 4 * j
+        word = _word(packed, off)
+        u = (word >> (8 * b).astype(np.uint32)) & 0xFF
+        q = u.astype(np.int64) - 128
+    G = K // 32
+    g = np.arange(G, dtype=np.int64)[None, :]
+    if bits == 4:
+        cs = g // 2
+        half = 2 * upper + (g % 2)
+        soff = (t * C + cs) * CB + 512 + 8 * gi + 2 * half
+    else:
+        soff = (t * C + g) * CB + 512 + 4 * gi + 2 * upper
+    s = packed[soff].astype(np.uint16) | (packed[soff + 1].astype(np.uint16) << 8)
+    return q, s
+
+
+def _word(packed: np.ndarray, off: np.ndarray) -> np.ndarray:
+    b = [packed[off + m].astype(np.uint32) for m in range(4)]
+    return b[0] | (b[1] << 8) | (b[2] << 16) | (b[3] << 24)
+
+
+def padding_is_zero(bits: int, packed: np.ndarray, N: int, K: int) -> bool:
+    """Rows >= N and groups >= K/32 of the padded tiles decode to q = 0, scale 0."""
+    T, C, CB = _geometry(bits, N, K)
+    Np = T * ROWS
+    Kp = C * (64 if bits == 4 else 32)
+    q, s = decode(bits, packed, Np, Kp)
+    return bool(np.all(q[N:, :] == 0) and np.all(q[:, K:] == 0) and np.all(s[N:, :] == 0) and np.all(s[:, K // 32:] == 0))

@@ -1,0 +1,508 @@
+"""Benchmark of the 64-layer decode weight stream on B200.
+
+One step = one pass of the whole hot path over one decode token's weights:
+the 257 group-quantised products of a dense 27B-shaped hybrid model (64 layers
+of fused q|k|v, o, gate|up, down; the 16 attention layers' q|k|v|o and the
+output head in q8 g32, everything else q4 g32), replayed as one captured
+layer stack.  13.7 GB of packed weights are resident in HBM; x and y are small.
+
+Metric: weight-stream GB/s (algorithmic weight bytes / device time per step)
+at M = 1, with % of the measured HBM peak and the implied decode tok/s; the
+same at M = 4 (one verification pass of 3 drafted tokens + 1) in "m4".
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+With N > 1 it runs under torch.distributed (one process per GPU): every rank
+streams its own replica of the weights (the single-token stream has no data
+exchange to shard: replicas only), the device time is the max over ranks, and
+the value is the bytes of all ranks over that time.  `--impl reference` times
+the CPU oracle on a bounded sample of the same workload (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import re
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "weight-stream GB/s & % of HBM peak (M=1,4); implied decode tok/s, 64 layers"
+UNIT = "GB/s"
+WORKLOAD = "64-layer decode weight stream + q8 output head (27B dense hybrid, 16 attn q8 / 48 DeltaNet q4, g32), M=1"
+
+
+# ----------------------------------------------------------------------------
+# helpers
+# ----------------------------------------------------------------------------
+def measured_peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return 6650.0, "fallback"
+
+
+def kernel_source_sha() -> str:
+    h = hashlib.sha256()
+    for rel in ("bit_weight_gemv_q4_b200/csrc/q4gemv_kernels.cuh", "bit_weight_gemv_q4_b200/csrc/q4gemv.cu"):
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic():
+    """DRAM bytes per launch of the dominant kernel from the committed ncu
+    summary, if it was taken on the current kernel source; else None."""
+    path = os.path.join(ROOT, "profiles", "gemv_q4_traffic.md")
+    try:
+        text = open(path).read()
+    except OSError:
+        return None
+    sha = re.search(r"kernel_source_sha:\s*([0-9a-f]+)", text)
+    per = re.search(r"dram_bytes_per_full_launch:\s*([0-9]+)", text)
+    if not sha or not per or sha.group(1) != kernel_source_sha():
+        return None
+    return int(per.group(1))
+
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons through NVML while running."""
+
+    REASONS = {
+        0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap", 0x8: "hw_slowdown",
+        0x10: "sync_boost", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+        0x100: "display_clock_setting",
+    }
+
+    def __init__(self, device_index: int, period_s: float = 0.02):
+        self.period = period_s
+        self.samples: list[int] = []
+        self.reasons: set[str] = set()
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._thread = None
+        self.error = None
+        try:
+            import pynvml
+
+            pynvml.nvmlInit()
+            self.nvml = pynvml
+            self.handle = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.handle, pynvml.NVML_CLOCK_SM)
+        except Exception as exc:  # clocks are reported as unavailable
+            self.nvml = None
+            self.error = str(exc)
+
+    def _run(self):
+        nv = self.nvml
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self.handle, nv.NVML_CLOCK_SM))
+                mask = nv.nvmlDeviceGetCurrentClocksEventReasons(self.handle)
+                for bit, name in self.REASONS.items():
+                    if mask & bit and name != "gpu_idle":
+                        self.reasons.add(name)
+            except Exception as exc:
+                self.error = str(exc)
+                return
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.nvml is not None:
+            self._thread = threading.Thread(target=self._run, daemon=True)
+            self._thread.start()
+        return self
+
+    def __exit__(self, *exc):
+        self._stop.set()
+        if self._thread is not None:
+            self._thread.join()
+        return False
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
+                    "samples": 0, "note": self.error or "no samples"}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+def nvml_index(local_rank: int) -> int:
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+    if vis:
+        ids = [v.strip() for v in vis.split(",") if v.strip()]
+        if local_rank < len(ids) and ids[local_rank].isdigit():
+            return int(ids[local_rank])
+    return local_rank
+
+
+# ----------------------------------------------------------------------------
+# CPU oracle on a bounded sample of the workload
+# ----------------------------------------------------------------------------
+def oracle_sample_rate(target_s: float = 12.0, seed: int = 0):
+    """Times the CPU oracle on whole rows spread over every tensor of the decode
+    stream; returns (GB/s of weights, threads, sample description, seconds)."""
+    import numpy as np
+
+    import oracle
+    from bit_weight_gemv_q4_b200 import synth, workloads
+
+    tensors = workloads.decode_stream(fused=True)
+    x = {K: synth.activations(seed, synth.act_stream(workloads.activation_stream_id(K)), 1, K)
+         for K in workloads.distinct_k(tensors)}
+
+    def run(rows_per_tensor):
+        inputs = []
+        for t in tensors:
+            stride = max(1, t.N // rows_per_tensor)
+            r0 = (seed * 7919) % stride
+            rows = list(range(r0, t.N, stride))[:rows_per_tensor]
+            # contiguous blocks of 1 row each: generate them on the host
+            qs = [synth.tensor(t.bits, seed, t.tensor_id, t.N, t.K, row0=r, nrows=1) for r in rows]
+            q = np.concatenate([a for a, _ in qs])
+            s = np.concatenate([b for _, b in qs])
+            inputs.append((t, q, s))
+        nbytes = sum(workloads.weight_bytes(t.bits, q.shape[0], t.K) for t, q, _ in inputs)
+        t0 = time.perf_counter()
+        for t, q, s in inputs:
+            oracle.gemv(t.bits, q, s, x[t.K])
+        return nbytes, time.perf_counter() - t0
+
+    nb, dt = run(2)
+    rows = max(2, min(4096, int(2 * target_s / max(dt, 1e-3))))
+    nb, dt = run(rows)
+    desc = (f"{rows} whole rows (evenly strided) of each of the 257 tensors of the M=1 decode stream, "
+            f"{nb / 1e6:.1f} MB of weights, fp64 oracle, {dt:.1f} s")
+    return nb / dt / 1e9, oracle.threads(), desc, dt
+
+
+# ----------------------------------------------------------------------------
+# distributed plumbing
+# ----------------------------------------------------------------------------
+class Dist:
+    def __init__(self, gpus: int):
+        self.world = int(os.environ.get("WORLD_SIZE", "1"))
+        self.rank = int(os.environ.get("RANK", "0"))
+        self.local = int(os.environ.get("LOCAL_RANK", "0"))
+        self.pg = False
+        if self.world != gpus and not (self.world == 1 and gpus == 1):
+            if self.world == 1:
+                raise SystemExit(f"--gpus {gpus} needs torch.distributed.run with {gpus} processes")
+        if self.world > 1:
+            import torch
+            import torch.distributed as dist
+
+            torch.cuda.set_device(self.local)
+            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                    device_id=torch.device("cuda", self.local))
+            self.pg = True
+
+    @classmethod
+    def single(cls):
+        """Rank 0 of a multi-process launch doing host-only work: no process group."""
+        d = cls.__new__(cls)
+        d.world, d.rank, d.local, d.pg = 1, 0, int(os.environ.get("LOCAL_RANK", "0")), False
+        return d
+
+    def barrier(self):
+        if self.pg:
+            import torch.distributed as dist
+
+            dist.barrier()
+
+    def max(self, v: float) -> float:
+        if not self.pg:
+            return v
+        import torch
+        import torch.distributed as dist
+
+        t = torch.tensor([v], dtype=torch.float64, device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    def close(self):
+        if self.pg:
+            import torch.distributed as dist
+
+            dist.destroy_process_group()
+
+
+# ----------------------------------------------------------------------------
+# our arm
+# ----------------------------------------------------------------------------
+def time_region(torch, fn, steps, stream):
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(steps):
+        fn()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1)  # ms
+
+
+def run_ours(args, d: Dist):
+    import torch
+
+    import bit_weight_gemv_q4_b200 as q4
+    from bit_weight_gemv_q4_b200 import workloads
+
+    torch.cuda.set_device(d.local)
+    stream = torch.cuda.current_stream()
+    tensors = workloads.decode_stream(fused=True)
+    peak, peak_kind = measured_peaks()
+
+    st = workloads.DeviceStream(tensors, 1, seed=args.seed)
+    n_launch = st.stack.launches()
+    wbytes = st.weight_bytes
+
+    for _ in range(args.warmup):
+        st.run()
+    torch.cuda.synchronize()
+    st.check()
+
+    sampler = ClockSampler(nvml_index(d.local))
+    d.barrier()
+    torch.cuda.synchronize()
+    with sampler:
+        ms = time_region(torch, st.run, args.steps, stream)
+    d.barrier()
+    st.check()
+    ms_step = d.max(ms / args.steps)
+    value = wbytes * d.world / (ms_step * 1e6)  # GB/s over all ranks
+
+    # dominant kernel: the q4 instantiation (82% of the bytes), timed as the
+    # sequence of its launches in the stream (same buffers, own captured stack)
+    q4_idx = [i for i, t in enumerate(tensors) if t.bits == 4]
+    q4_entries = [(4, tensors[i].N, tensors[i].K, st.packed[i], st.x[tensors[i].K], st.y[i]) for i in q4_idx]
+    q4_stack = q4.layer_stack_create(q4_entries, 1)
+    q4_bytes = sum(tensors[i].bytes for i in q4_idx)
+    for _ in range(max(3, args.warmup)):
+        q4.layer_stack_run(q4_stack)
+    q4_steps = max(3, args.steps // 2)
+    ms_q4 = time_region(torch, lambda: q4.layer_stack_run(q4_stack), q4_steps, stream) / q4_steps
+    q4.layer_stack_check(q4_stack)
+    launch_us = ms_q4 * 1e3 / len(q4_idx)
+    achieved = q4_bytes / len(q4_idx) / (launch_us * 1e-6) / 1e9
+    q4_stack.close()
+
+    # e2e through the public API: activations from pinned host memory in,
+    # the stack, the logits (head output) back to pinned host memory
+    x_host = {K: xb.cpu().pin_memory() for K, xb in st.x.items()}
+    logits = st.y[-1]
+    logits_host = torch.empty(logits.shape, dtype=logits.dtype, pin_memory=True)
+
+    def e2e_step():
+        for K, xb in st.x.items():
+            xb.copy_(x_host[K], non_blocking=True)
+        st.run()
+        logits_host.copy_(logits, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    d.barrier()
+    ms_e2e = d.max(time_region(torch, e2e_step, args.steps, stream) / args.steps)
+    h2d = sum(v.numel() * v.element_size() for v in x_host.values())
+    d2h = logits_host.numel() * logits_host.element_size()
+    st.check()
+    st.close()
+    del st
+    torch.cuda.empty_cache()
+
+    # M = 4: one verification pass of three drafted tokens plus one
+    st4 = workloads.DeviceStream(tensors, 4, seed=args.seed)
+    for _ in range(args.warmup):
+        st4.run()
+    d.barrier()
+    ms4 = d.max(time_region(torch, st4.run, args.steps, stream) / args.steps)
+    st4.check()
+    st4.close()
+    del st4
+    torch.cuda.empty_cache()
+
+    cpu = None
+    if d.rank == 0 and not args.no_cpu_baseline:
+        rate, threads, desc, _ = oracle_sample_rate(args.cpu_seconds, args.seed)
+        cpu = {"value": round(rate, 4), "unit": UNIT, "cores": threads, "kind": "oracle", "sample": desc}
+
+    traffic = profiled_traffic()
+    clocks = sampler.summary()
+    gbs1 = wbytes / (ms_step * 1e6)
+    line = {
+        "metric": METRIC,
+        "value": round(value, 1),
+        "unit": UNIT,
+        "n_gpus": d.world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms_step, 5),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "q4/q8 g32 weights, bf16 x, fp32 accumulate",
+        "data": "synthetic (seeded generator: q uniform, fp16 scales |N(0,0.02)|, bf16 x N(0,1))",
+        "config": {
+            "workload": WORKLOAD,
+            "tensors": len(tensors),
+            "weight_bytes_per_step": wbytes,
+            "M": 1,
+            "parallelism": "replicas" if d.world > 1 else "single GPU",
+            "l2": "inputs larger than L2 (13.7 GB of weights per step vs 126 MB L2); no flush",
+        },
+        "pct_of_hbm_peak": round(100 * gbs1 / peak, 2),
+        "hbm_peak_gbs": peak,
+        "hbm_peak_kind": peak_kind,
+        "tok_per_s": round(1000.0 / ms_step, 1),
+        "m4": {
+            "value": round(wbytes * d.world / (ms4 * 1e6), 1),
+            "unit": UNIT,
+            "ms_per_step": round(ms4, 5),
+            "pct_of_hbm_peak": round(100 * wbytes / (ms4 * 1e6) / peak, 2),
+            "verify_passes_per_s": round(1000.0 / ms4, 1),
+        },
+        "roofline": {
+            "bound": "hbm",
+            "kernel": "q4gemv gemv_kernel<4,1> (q4 products of the stream)",
+            "achieved": round(achieved, 1),
+            "peak": peak,
+            "unit": "GB/s",
+            "frac": round(achieved / peak, 4),
+            "traffic": traffic,
+            "bytes_per_launch": q4_bytes // len(q4_idx),
+            "launch_us": round(launch_us, 3),
+            "launches": len(q4_idx),
+            "peak_kind": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs, copy burst)" if peak_kind == "measured" else peak_kind,
+        },
+        "cpu_baseline": cpu,
+        "e2e": {
+            "value": round(wbytes * d.world / (ms_e2e * 1e6), 1),
+            "unit": UNIT,
+            "ms_per_step": round(ms_e2e, 5),
+            "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h,
+        },
+        "gpu_launches": n_launch * args.steps,
+        "clocks": clocks,
+    }
+    return line
+
+
+def run_reference(args, d: Dist):
+    """The CPU oracle on the host cores: each step is a bounded sample of the
+    same workload; value = sampled weight bytes / time, same metric."""
+    if d.rank != 0:
+        return None
+    import numpy as np
+
+    import oracle
+    from bit_weight_gemv_q4_b200 import synth, workloads
+
+    tensors = workloads.decode_stream(fused=True)
+    x = {K: synth.activations(args.seed, synth.act_stream(workloads.activation_stream_id(K)), 1, K)
+         for K in workloads.distinct_k(tensors)}
+    rows = args.reference_rows
+    inputs = []
+    for t in tensors:
+        stride = max(1, t.N // rows)
+        qs = [synth.tensor(t.bits, args.seed, t.tensor_id, t.N, t.K, row0=r, nrows=1) for r in range(0, t.N, stride)[:rows]]
+        inputs.append((t, np.concatenate([a for a, _ in qs]), np.concatenate([b for _, b in qs])))
+    nbytes = sum(workloads.weight_bytes(t.bits, q.shape[0], t.K) for t, q, _ in inputs)
+
+    def step():
+        for t, q, s in inputs:
+            oracle.gemv(t.bits, q, s, x[t.K])
+
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    dt = (time.perf_counter() - t0) / args.steps
+    value = nbytes / dt / 1e9
+    desc = (f"{rows} whole rows (evenly strided) of each of the 257 tensors of the M=1 decode stream per step, "
+            f"{nbytes / 1e6:.1f} MB of weights")
+    return {
+        "impl": "reference",
+        "metric": METRIC,
+        "value": round(value, 4),
+        "unit": UNIT,
+        "n_gpus": d.world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(dt * 1e3, 3),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "fp64 accumulate (oracle)",
+        "data": "synthetic (seeded generator)",
+        "config": {"workload": WORKLOAD, "tensors": len(tensors), "M": 1},
+        "cpu_baseline": {"value": round(value, 4), "unit": UNIT, "cores": oracle.threads(), "kind": "oracle",
+                         "sample": desc},
+        "e2e": {"value": round(value, 4), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def run_profile_case(args):
+    """A small single-product case for ncu: a q4 65536 x 5120 tensor (189 MB,
+    larger than L2), `--profile-launches` launches at M = args.m."""
+    import torch
+
+    from bit_weight_gemv_q4_b200 import workloads
+
+    t = workloads.Tensor("profile.q4", 4 if args.profile_bits == 4 else 8, 65536, 5120, 900)
+    st = workloads.DeviceStream([t], args.m, seed=args.seed)
+    for _ in range(args.profile_launches):
+        st.run()
+    torch.cuda.synchronize()
+    st.check()
+    print(json.dumps({"profile_case": t.name, "bits": t.bits, "N": t.N, "K": t.K, "M": args.m,
+                      "launches": args.profile_launches, "weight_bytes": t.bytes,
+                      "kernel_source_sha": kernel_source_sha()}))
+    st.close()
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU time of the oracle sample")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--reference-rows", type=int, default=8, help="rows per tensor per reference step")
+    ap.add_argument("--profile-case", action="store_true", help="run the small ncu case and exit")
+    ap.add_argument("--profile-bits", type=int, default=4)
+    ap.add_argument("--profile-launches", type=int, default=3)
+    ap.add_argument("--m", type=int, default=1)
+    args = ap.parse_args()
+    if args.warmup < 3 and not args.profile_case:
+        raise SystemExit("--warmup must be at least 3")
+
+    if args.profile_case:
+        run_profile_case(args)
+        return
+
+    if args.impl == "reference" and int(os.environ.get("RANK", "0")) != 0:
+        return  # the CPU oracle arm runs on rank 0 alone
+    d = Dist(args.gpus) if args.impl == "ours" else Dist.single()
+    try:
+        line = run_reference(args, d) if args.impl == "reference" else run_ours(args, d)
+        if d.rank == 0 and line is not None:
+            print(json.dumps(line), flush=True)
+    finally:
+        d.close()
+
+
+if __name__ == "__main__":
+    main()

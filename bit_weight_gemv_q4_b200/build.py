@@ -2,8 +2,9 @@
 
 * ``libq4gemv.so``  -- the C-ABI product library: the host packer and the
   sm_100a CUDA kernels (``csrc/pack.cpp``, ``csrc/q4gemv.cu``).
-* ``libq4synth.so`` -- the seeded synthetic-input generator (``csrc/synth.c``),
-  host C only.
+* ``libq4synth.so`` -- the seeded synthetic-input generator (``csrc/synth.cu``,
+  one definition in ``csrc/synth_core.h`` compiled for host and device,
+  without floating-point contraction so both give identical bits).
 
 Run ``python -m bit_weight_gemv_q4_b200.build`` or call :func:`build_all`.
 A library is rebuilt only when one of its sources is newer than it.
@@ -24,7 +25,8 @@ SYNTH_LIB = os.path.join(HERE, "libq4synth.so")
 
 GEMV_SOURCES = [os.path.join(CSRC, "q4gemv.cu"), os.path.join(CSRC, "pack.cpp")]
 GEMV_DEPS = GEMV_SOURCES + [os.path.join(INCLUDE, "q4gemv.h"), os.path.join(CSRC, "q4gemv_kernels.cuh")]
-SYNTH_SOURCES = [os.path.join(CSRC, "synth.c")]
+SYNTH_SOURCES = [os.path.join(CSRC, "synth.cu")]
+SYNTH_DEPS = SYNTH_SOURCES + [os.path.join(CSRC, "synth_core.h")]
 
 NVCC_ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
@@ -50,10 +52,11 @@ def _run(cmd: list[str]) -> None:
 
 
 def build_synth(force: bool = False) -> str:
-    if force or _stale(SYNTH_LIB, SYNTH_SOURCES):
+    if force or _stale(SYNTH_LIB, SYNTH_DEPS):
         tmp = SYNTH_LIB + ".tmp"
-        _run(["gcc", "-O2", "-std=c11", "-ffp-contract=off", "-fopenmp", "-fPIC", "-shared",
-              *SYNTH_SOURCES, "-o", tmp, "-lm"])
+        _run([_nvcc(), *NVCC_ARCH, "-O3", "-std=c++17", "-shared", "-fmad=false",
+              "-Xcompiler", "-fPIC", "-Xcompiler", "-ffp-contract=off", "-Xcompiler", "-fopenmp",
+              "-Xcompiler", "-fvisibility=hidden", "-cudart", "static", *SYNTH_SOURCES, "-o", tmp, "-lgomp"])
         os.replace(tmp, SYNTH_LIB)
     return SYNTH_LIB
 

@@ -1,0 +1,240 @@
+// Offline repack of canonical group-quantised weights into the kernel-native
+// chunk layout, and its exact inverse.  Host code, run once per tensor (the
+// weights of a decode model are packed when they are loaded, not per token).
+//
+// The layout itself is specified in include/q4gemv.h; in short, the tensor is a
+// sequence of 32-row x (64 or 32)-column chunks in memory order (tile, chunk),
+// each chunk holding the tensor-core A fragments of one warp for its two
+// 16-row halves, followed by the fp16 scales of its groups.  Streaming a tile
+// is streaming one contiguous run.
+#include <cstdint>
+#include <cstring>
+#include <string>
+
+#include "q4gemv.h"
+
+namespace q4 {
+void set_error(const std::string& msg);
+}  // namespace q4
+
+namespace {
+
+constexpr int kTileRows = 32;
+
+struct Geometry {
+  int bits;
+  int64_t N, K, T, C, chunk_bytes, k_per_chunk;
+};
+
+bool geometry(int bits, int64_t N, int64_t K, Geometry* g) {
+  if ((bits != 4 && bits != 8) || N < 0 || K < 0 || K % 32 != 0) return false;
+  // keep every offset and index comfortably inside int64 / int32 tile counts
+  if (N > (int64_t(1) << 34) || K > (int64_t(1) << 30)) return false;
+  g->bits = bits;
+  g->N = N;
+  g->K = K;
+  g->T = (N + kTileRows - 1) / kTileRows;
+  g->k_per_chunk = bits == 4 ? 64 : 32;
+  g->C = (K + g->k_per_chunk - 1) / g->k_per_chunk;
+  g->chunk_bytes = bits == 4 ? 1152 : 1088;
+  return true;
+}
+
+// Row and column of nibble i of word j in slot (gi, ti) of half h of q4
+// chunk (t, c).
+inline void q4_coord(int64_t t, int64_t c, int h, int gi, int ti, int j, int i, int64_t* row, int64_t* col) {
+  const int G = j >> 1, e = j & 1;
+  *row = kTileRows * t + 16 * h + gi + 8 * (i & 1);
+  *col = 64 * c + 32 * G + 8 * ti + 4 * e + 2 * ((i >> 1) & 1) + (i >> 2);
+}
+
+// Row and column of byte b of word j in slot (gi, ti) of half h of q8 chunk (t, c).
+inline void q8_coord(int64_t t, int64_t c, int h, int gi, int ti, int j, int b, int64_t* row, int64_t* col) {
+  const int e = j >> 1, f = j & 1;
+  *row = kTileRows * t + 16 * h + gi + 8 * (b & 1);
+  *col = 32 * c + 8 * ti + 4 * e + 2 * f + (b >> 1);
+}
+
+// Row of scale slot (h, up) of entry gi in tile t: 16h + gi + 8up.
+inline int64_t scale_row(int64_t t, int h, int gi, int up) { return kTileRows * t + 16 * h + gi + 8 * up; }
+
+inline int canon_q4(const uint8_t* q, int64_t K, int64_t row, int64_t col) {
+  const uint8_t byte = q[row * (K / 2) + col / 2];
+  const int nib = (col & 1) ? (byte >> 4) : (byte & 0xF);
+  return nib >= 8 ? nib - 16 : nib;
+}
+
+}  // namespace
+
+extern "C" Q4_API size_t q4_packed_bytes(int bits, int64_t N, int64_t K) {
+  Geometry g;
+  if (!geometry(bits, N, K, &g)) return 0;
+  return static_cast<size_t>(g.T * g.C * g.chunk_bytes);
+}
+
+extern "C" Q4_API int q4_pack_weights(int bits, const void* canon_q, const uint16_t* scales, int64_t N, int64_t K,
+                                      void* out, size_t out_bytes) {
+  Geometry g;
+  if (bits != 4 && bits != 8) {
+    q4::set_error("q4_pack_weights: bits must be 4 or 8");
+    return Q4_ERR_INVALID_ARG;
+  }
+  if (!geometry(bits, N, K, &g)) {
+    q4::set_error("q4_pack_weights: need N >= 0, K >= 0, K % 32 == 0 (and sizes below 2^34 x 2^30)");
+    return Q4_ERR_SHAPE;
+  }
+  const size_t need = static_cast<size_t>(g.T * g.C * g.chunk_bytes);
+  if (need == 0) return Q4_OK;
+  if (!canon_q || !scales || !out) {
+    q4::set_error("q4_pack_weights: null pointer");
+    return Q4_ERR_INVALID_ARG;
+  }
+  if (out_bytes < need) {
+    q4::set_error("q4_pack_weights: out_bytes " + std::to_string(out_bytes) + " < " + std::to_string(need));
+    return Q4_ERR_BUFFER_TOO_SMALL;
+  }
+  const int64_t G = K / 32;
+  uint8_t* dst = static_cast<uint8_t*>(out);
+#pragma omp parallel for schedule(static)
+  for (int64_t t = 0; t < g.T; ++t) {
+    for (int64_t c = 0; c < g.C; ++c) {
+      uint8_t* chunk = dst + (t * g.C + c) * g.chunk_bytes;
+      for (int h = 0; h < 2; ++h) {
+        for (int gi = 0; gi < 8; ++gi) {
+          for (int ti = 0; ti < 4; ++ti) {
+            uint32_t words[4];
+            for (int j = 0; j < 4; ++j) {
+              uint32_t w = 0;
+              if (bits == 4) {
+                for (int i = 0; i < 8; ++i) {
+                  int64_t row, col;
+                  q4_coord(t, c, h, gi, ti, j, i, &row, &col);
+                  int q = 0;
+                  if (row < N && col < K) q = canon_q4(static_cast<const uint8_t*>(canon_q), K, row, col);
+                  w |= static_cast<uint32_t>(q + 8) << (4 * i);
+                }
+              } else {
+                for (int b = 0; b < 4; ++b) {
+                  int64_t row, col;
+                  q8_coord(t, c, h, gi, ti, j, b, &row, &col);
+                  int q = 0;
+                  if (row < N && col < K) q = static_cast<const int8_t*>(canon_q)[row * K + col];
+                  w |= static_cast<uint32_t>(q + 128) << (8 * b);
+                }
+              }
+              words[j] = w;
+            }
+            std::memcpy(chunk + 512 * h + 16 * (4 * gi + ti), words, 16);
+          }
+        }
+      }
+      // scales: entry gi lists rows 16h + gi + 8up for h, up in {0, 1}
+      for (int gi = 0; gi < 8; ++gi) {
+        if (bits == 4) {
+          uint16_t s8[8];
+          for (int h = 0; h < 2; ++h)
+            for (int up = 0; up < 2; ++up)
+              for (int gg = 0; gg < 2; ++gg) {
+                const int64_t row = scale_row(t, h, gi, up), grp = 2 * c + gg;
+                s8[4 * h + 2 * up + gg] = (row < N && grp < G) ? scales[row * G + grp] : 0;
+              }
+          std::memcpy(chunk + 1024 + 16 * gi, s8, 16);
+        } else {
+          uint16_t s4[4];
+          for (int h = 0; h < 2; ++h)
+            for (int up = 0; up < 2; ++up) {
+              const int64_t row = scale_row(t, h, gi, up);
+              s4[2 * h + up] = row < N ? scales[row * G + c] : 0;
+            }
+          std::memcpy(chunk + 1024 + 8 * gi, s4, 8);
+        }
+      }
+    }
+  }
+  return Q4_OK;
+}
+
+extern "C" Q4_API int q4_unpack_weights(int bits, const void* packed, size_t packed_bytes, int64_t N, int64_t K,
+                                        void* canon_q_out, uint16_t* scales_out) {
+  Geometry g;
+  if (bits != 4 && bits != 8) {
+    q4::set_error("q4_unpack_weights: bits must be 4 or 8");
+    return Q4_ERR_INVALID_ARG;
+  }
+  if (!geometry(bits, N, K, &g)) {
+    q4::set_error("q4_unpack_weights: need N >= 0, K >= 0, K % 32 == 0");
+    return Q4_ERR_SHAPE;
+  }
+  const size_t need = static_cast<size_t>(g.T * g.C * g.chunk_bytes);
+  if (need == 0) return Q4_OK;
+  if (!packed || !canon_q_out || !scales_out) {
+    q4::set_error("q4_unpack_weights: null pointer");
+    return Q4_ERR_INVALID_ARG;
+  }
+  if (packed_bytes < need) {
+    q4::set_error("q4_unpack_weights: packed_bytes too small");
+    return Q4_ERR_BUFFER_TOO_SMALL;
+  }
+  const int64_t G = K / 32;
+  const uint8_t* src = static_cast<const uint8_t*>(packed);
+  if (bits == 4) std::memset(canon_q_out, 0, static_cast<size_t>(N * (K / 2)));
+#pragma omp parallel for schedule(static)
+  for (int64_t t = 0; t < g.T; ++t) {
+    for (int64_t c = 0; c < g.C; ++c) {
+      const uint8_t* chunk = src + (t * g.C + c) * g.chunk_bytes;
+      for (int h = 0; h < 2; ++h) {
+        for (int gi = 0; gi < 8; ++gi) {
+          for (int ti = 0; ti < 4; ++ti) {
+            uint32_t words[4];
+            std::memcpy(words, chunk + 512 * h + 16 * (4 * gi + ti), 16);
+            for (int j = 0; j < 4; ++j) {
+              if (bits == 4) {
+                for (int i = 0; i < 8; ++i) {
+                  int64_t row, col;
+                  q4_coord(t, c, h, gi, ti, j, i, &row, &col);
+                  if (row >= N || col >= K) continue;
+                  const int q = static_cast<int>((words[j] >> (4 * i)) & 0xF) - 8;
+                  uint8_t* byte = static_cast<uint8_t*>(canon_q_out) + row * (K / 2) + col / 2;
+                  const uint8_t nib = static_cast<uint8_t>(q & 0xF);
+                  // each (row, col) is visited once and the two nibbles of a
+                  // byte belong to the same tile, so this thread owns the byte
+                  *byte = (col & 1) ? static_cast<uint8_t>((*byte & 0x0F) | (nib << 4))
+                                    : static_cast<uint8_t>((*byte & 0xF0) | nib);
+                }
+              } else {
+                for (int b = 0; b < 4; ++b) {
+                  int64_t row, col;
+                  q8_coord(t, c, h, gi, ti, j, b, &row, &col);
+                  if (row >= N || col >= K) continue;
+                  static_cast<int8_t*>(canon_q_out)[row * K + col] =
+                      static_cast<int8_t>(static_cast<int>((words[j] >> (8 * b)) & 0xFF) - 128);
+                }
+              }
+            }
+          }
+        }
+      }
+      for (int gi = 0; gi < 8; ++gi) {
+        if (bits == 4) {
+          uint16_t s8[8];
+          std::memcpy(s8, chunk + 1024 + 16 * gi, 16);
+          for (int h = 0; h < 2; ++h)
+            for (int up = 0; up < 2; ++up)
+              for (int gg = 0; gg < 2; ++gg) {
+                const int64_t row = scale_row(t, h, gi, up), grp = 2 * c + gg;
+                if (row < N && grp < G) scales_out[row * G + grp] = s8[4 * h + 2 * up + gg];
+              }
+        } else {
+          uint16_t s4[4];
+          std::memcpy(s4, chunk + 1024 + 8 * gi, 8);
+          for (int h = 0; h < 2; ++h)
+            for (int up = 0; up < 2; ++up) {
+              const int64_t row = scale_row(t, h, gi, up);
+              if (row < N) scales_out[row * G + c] = s4[2 * h + up];
+            }
+        }
+      }
+    }
+  }
+  return Q4_OK;
+}

@@ -1,0 +1,539 @@
+// C-ABI of the group-quantised weight x activation product on B200 (sm_100a).
+// Host side: argument validation, launch-shape selection, the workspace
+// contract, and the CUDA-graph-captured layer stack.  Device code lives in
+// q4gemv_kernels.cuh.
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <string>
+#include <vector>
+
+#include "q4gemv.h"
+#include "q4gemv_kernels.cuh"
+
+namespace q4 {
+
+thread_local std::string g_last_error;
+
+void set_error(const std::string& msg) { g_last_error = msg; }
+
+namespace {
+
+constexpr unsigned long long kDefaultTimeoutNs = 2000000000ULL;
+std::atomic<unsigned long long> g_timeout_ns{kDefaultTimeoutNs};
+
+// Launch shape of the product kernel: one persistent CTA of NW warps per SM;
+// per warp a ring of kRingChunks chunks cut into D = kRingChunks / U stages of
+// U chunks (U = 2 when it divides the chunks per tile, else 1).  Measured on
+// B200: bulk-copy streaming holds ~7 TB/s with 16 warps per SM and 32-64
+// copies in flight per SM, and falls off sharply beyond that.  The defaults
+// can be changed at compile time for tuning sweeps.
+#ifndef Q4_TUNE_NW
+#define Q4_TUNE_NW 16
+#endif
+#ifndef Q4_TUNE_CTAS_PER_SM
+#define Q4_TUNE_CTAS_PER_SM 1
+#endif
+#ifndef Q4_TUNE_RING_CHUNKS
+#define Q4_TUNE_RING_CHUNKS 4
+#endif
+#ifndef Q4_TUNE_MAX_U
+#define Q4_TUNE_MAX_U 2
+#endif
+constexpr int kNW = Q4_TUNE_NW;
+constexpr int kCtasPerSm = Q4_TUNE_CTAS_PER_SM;
+constexpr int kRingChunks = Q4_TUNE_RING_CHUNKS;
+constexpr int kMaxU = Q4_TUNE_MAX_U;
+static_assert(kRingChunks % 2 == 0 && kRingChunks >= 4, "ring must hold two stages of two chunks");
+// shared memory a CTA may use (B200: 227 KB per CTA)
+constexpr int kSmemLimit = 227 * 1024 / kCtasPerSm;
+constexpr size_t kWsHeader = 256;
+
+int fail(int code, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return code;
+}
+
+int cuda_fail(cudaError_t err, const char* what) {
+  return fail(Q4_ERR_CUDA, "%s: %s (%s)", what, cudaGetErrorString(err), cudaGetErrorName(err));
+}
+
+struct DeviceInfo {
+  int sms = 0;
+  bool ok = false;
+  std::string why;
+};
+
+std::mutex g_dev_mutex;
+std::vector<DeviceInfo> g_devices;
+
+// Per-device facts, checked once: an sm_100 device and its SM count.
+int device_info(DeviceInfo* out) {
+  int dev = 0;
+  cudaError_t err = cudaGetDevice(&dev);
+  if (err != cudaSuccess) return cuda_fail(err, "cudaGetDevice");
+  std::lock_guard<std::mutex> lock(g_dev_mutex);
+  if (static_cast<int>(g_devices.size()) <= dev) g_devices.resize(dev + 1);
+  DeviceInfo& info = g_devices[dev];
+  if (!info.ok && info.why.empty()) {
+    int major = 0, minor = 0, sms = 0;
+    if ((err = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev)) != cudaSuccess ||
+        (err = cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev)) != cudaSuccess ||
+        (err = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
+      return cuda_fail(err, "cudaDeviceGetAttribute");
+    if (major != 10 || minor != 0) {
+      info.why = "device " + std::to_string(dev) + " is sm_" + std::to_string(major) + std::to_string(minor) +
+                 "; this library is built for sm_100a only";
+    } else {
+      info.sms = sms;
+      info.ok = true;
+    }
+  }
+  if (!info.ok) return fail(Q4_ERR_UNSUPPORTED, "%s", info.why.c_str());
+  *out = info;
+  return Q4_OK;
+}
+
+struct Shape {
+  int bits;
+  long long N, K;
+  int T, C;
+  long long TC;
+};
+
+int make_shape(int bits, int64_t N, int64_t K, Shape* s, const char* who) {
+  if (bits != 4 && bits != 8) return fail(Q4_ERR_INVALID_ARG, "%s: bits must be 4 or 8", who);
+  if (N < 0 || K < 0 || K % 32 != 0)
+    return fail(Q4_ERR_SHAPE, "%s: need N >= 0, K >= 0 and K %% 32 == 0 (N=%lld K=%lld)", who, (long long)N,
+                (long long)K);
+  if (N > (int64_t(1) << 34) || K > (int64_t(1) << 30))
+    return fail(Q4_ERR_SHAPE, "%s: N or K too large", who);
+  s->bits = bits;
+  s->N = N;
+  s->K = K;
+  s->T = static_cast<int>((N + q4k::kTileRows - 1) / q4k::kTileRows);
+  const int kc = bits == 4 ? 64 : 32;
+  s->C = static_cast<int>((K + kc - 1) / kc);
+  s->TC = static_cast<long long>(s->T) * s->C;
+  return Q4_OK;
+}
+
+long long max_warps(const DeviceInfo& dev) { return static_cast<long long>(dev.sms) * kCtasPerSm * kNW; }
+
+// Workspace layout: [status word | partial sums | tile counters].  The
+// partial-sum region has one fixed size per device (M = 4 worst case), so the
+// counters sit at the same offset for every shape and M: one zero-filled
+// workspace serves any sequence of products, each leaving its counters zero.
+size_t partials_bytes(const DeviceInfo& dev) {
+  return static_cast<size_t>(max_warps(dev)) * 2 * 4 * q4k::kTileRows * sizeof(float);
+}
+
+size_t workspace_bytes(const Shape& s, int M, const DeviceInfo& dev) {
+  (void)M;
+  const size_t counters = (static_cast<size_t>(s.T) * 4 + 255) / 256 * 256;
+  return kWsHeader + partials_bytes(dev) + counters;
+}
+
+template <int BITS, int M, int U, bool XS>
+void* kernel_ptr() {
+  return reinterpret_cast<void*>(&q4k::gemv_kernel<BITS, M, kNW, kRingChunks / U, U, XS>);
+}
+
+template <int BITS, int U>
+int smem_base() {
+  using Cfg = q4k::GemvConfig<BITS, kNW, kRingChunks / U, U>;
+  return Cfg::kXOffset;
+}
+
+int pick_u(int C) { return (kMaxU >= 2 && C % 2 == 0) ? 2 : 1; }
+
+void* select_kernel(int bits, int M, int U, bool xs) {
+#define Q4_ROW(B, M_) \
+  {{kernel_ptr<B, M_, 1, false>(), kernel_ptr<B, M_, 1, true>()}, {kernel_ptr<B, M_, 2, false>(), kernel_ptr<B, M_, 2, true>()}}
+  static void* const table[2][4][2][2] = {
+      {Q4_ROW(4, 1), Q4_ROW(4, 2), Q4_ROW(4, 3), Q4_ROW(4, 4)},
+      {Q4_ROW(8, 1), Q4_ROW(8, 2), Q4_ROW(8, 3), Q4_ROW(8, 4)},
+  };
+#undef Q4_ROW
+  return table[bits == 4 ? 0 : 1][M - 1][U - 1][xs ? 1 : 0];
+}
+
+// Dynamic shared memory of a launch: the rings, the barriers and, with the
+// activations staged, M padded rows.
+int smem_bytes(int bits, int U, int M, long long K, bool xs) {
+  const int base = bits == 4 ? (U == 2 ? smem_base<4, 2>() : smem_base<4, 1>())
+                             : (U == 2 ? smem_base<8, 2>() : smem_base<8, 1>());
+  return base + (xs ? static_cast<int>(M * q4k::x_row_stride_bytes(K)) : 0);
+}
+
+bool stage_x(int bits, int U, int M, long long K) {
+  return static_cast<long long>(smem_bytes(bits, U, M, 0, false)) + M * q4k::x_row_stride_bytes(K) <= kSmemLimit;
+}
+
+struct Launch {
+  void* fn = nullptr;
+  dim3 grid, block;
+  int smem = 0;
+  q4k::GemvParams params{};
+  bool zero_fill = false;  // K == 0: y = 0
+  size_t zero_bytes = 0;
+  bool noop = false;
+};
+
+int prepare(int bits, const void* packed, int64_t N, int64_t K, const uint16_t* x, int M, float* y, void* workspace,
+            size_t workspace_bytes_given, const char* who, Launch* L) {
+  Shape s;
+  int rc = make_shape(bits, N, K, &s, who);
+  if (rc) return rc;
+  if (M < 0 || M > 4) return fail(Q4_ERR_INVALID_ARG, "%s: M must be in 0..4 (got %d)", who, M);
+  if (N == 0 || M == 0) {
+    L->noop = true;
+    return Q4_OK;
+  }
+  if (!y) return fail(Q4_ERR_INVALID_ARG, "%s: y is null", who);
+  if (reinterpret_cast<uintptr_t>(y) % 4) return fail(Q4_ERR_ALIGN, "%s: y must be 4-byte aligned", who);
+  if (K == 0) {
+    L->zero_fill = true;
+    L->zero_bytes = static_cast<size_t>(M) * static_cast<size_t>(N) * sizeof(float);
+    return Q4_OK;
+  }
+  if (!packed || !x || !workspace) return fail(Q4_ERR_INVALID_ARG, "%s: null device pointer", who);
+  if (reinterpret_cast<uintptr_t>(packed) % 16) return fail(Q4_ERR_ALIGN, "%s: packed must be 16-byte aligned", who);
+  if (reinterpret_cast<uintptr_t>(x) % 16) return fail(Q4_ERR_ALIGN, "%s: x must be 16-byte aligned", who);
+  if (reinterpret_cast<uintptr_t>(workspace) % 16)
+    return fail(Q4_ERR_ALIGN, "%s: workspace must be 16-byte aligned", who);
+  DeviceInfo dev;
+  if ((rc = device_info(&dev))) return rc;
+  const size_t need = workspace_bytes(s, M, dev);
+  if (workspace_bytes_given < need)
+    return fail(Q4_ERR_BUFFER_TOO_SMALL, "%s: workspace %zu bytes < %zu required", who, workspace_bytes_given, need);
+
+  const int U = pick_u(s.C);
+  const bool xs = stage_x(bits, U, M, s.K);
+  long long P = max_warps(dev);
+  if (P > s.TC / U) P = s.TC / U;
+  const int G = static_cast<int>((P + kNW - 1) / kNW);
+  unsigned char* ws = static_cast<unsigned char*>(workspace);
+
+  q4k::GemvParams& p = L->params;
+  p.packed = static_cast<const uint8_t*>(packed);
+  p.x = x;
+  p.y = y;
+  p.status = reinterpret_cast<unsigned*>(ws);
+  p.partials = reinterpret_cast<float*>(ws + kWsHeader);
+  p.counters = reinterpret_cast<unsigned*>(ws + kWsHeader + partials_bytes(dev));
+  p.N = s.N;
+  p.K = s.K;
+  p.TC = s.TC;
+  p.T = s.T;
+  p.C = s.C;
+  p.P = static_cast<int>(P);
+  p.khalf = (bits == 4 && K % 64 == 32) ? 1 : 0;
+  p.timeout_ns = g_timeout_ns.load();
+  L->fn = select_kernel(bits, M, U, xs);
+  L->grid = dim3(G);
+  L->block = dim3(kNW * 32);
+  L->smem = smem_bytes(bits, U, M, s.K, xs);
+  return Q4_OK;
+}
+
+int launch(Launch& L, cudaStream_t stream, bool pdl) {
+  cudaError_t err;
+  if (L.noop) return Q4_OK;
+  if (L.zero_fill) {
+    err = cudaMemsetAsync(L.params.y, 0, L.zero_bytes, stream);
+    return err == cudaSuccess ? Q4_OK : cuda_fail(err, "cudaMemsetAsync(y)");
+  }
+  static std::once_flag smem_once;
+  static cudaError_t smem_err = cudaSuccess;
+  std::call_once(smem_once, [] {
+    for (int bits : {4, 8})
+      for (int M = 1; M <= 4; ++M)
+        for (int U : {1, 2})
+          for (bool xs : {false, true}) {
+            cudaError_t e = cudaFuncSetAttribute(select_kernel(bits, M, U, xs),
+                                                 cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemLimit);
+            if (e != cudaSuccess) smem_err = e;
+          }
+  });
+  if (smem_err != cudaSuccess) return cuda_fail(smem_err, "cudaFuncSetAttribute");
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = L.grid;
+  cfg.blockDim = L.block;
+  cfg.dynamicSmemBytes = static_cast<size_t>(L.smem);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  void* args[] = {&L.params};
+  err = cudaLaunchKernelExC(&cfg, L.fn, args);
+  if (err != cudaSuccess) return cuda_fail(err, "kernel launch");
+  return Q4_OK;
+}
+
+int gemv_entry(int bits, const void* packed, int64_t N, int64_t K, const uint16_t* x, int M, float* y,
+               void* workspace, size_t workspace_bytes_given, void* stream, const char* who) {
+  Launch L;
+  // the zero-fill path needs y in params
+  int rc = prepare(bits, packed, N, K, x, M, y, workspace, workspace_bytes_given, who, &L);
+  if (rc) return rc;
+  L.params.y = y;
+  return launch(L, static_cast<cudaStream_t>(stream), true);
+}
+
+}  // namespace
+}  // namespace q4
+
+using namespace q4;
+
+extern "C" Q4_API const char* q4_last_error(void) { return g_last_error.c_str(); }
+
+extern "C" Q4_API size_t q4_gemv_workspace_bytes(int bits, int64_t N, int64_t K, int M) {
+  Shape s;
+  if (make_shape(bits, N, K, &s, "q4_gemv_workspace_bytes")) return 0;
+  if (M < 0 || M > 4) {
+    fail(Q4_ERR_INVALID_ARG, "q4_gemv_workspace_bytes: M must be in 0..4");
+    return 0;
+  }
+  DeviceInfo dev;
+  if (device_info(&dev)) return 0;
+  return workspace_bytes(s, M, dev);
+}
+
+extern "C" Q4_API int q4_gemv(const void* packed, int64_t N, int64_t K, const uint16_t* x, int M, float* y,
+                              void* workspace, size_t workspace_bytes_given, void* stream) {
+  return gemv_entry(4, packed, N, K, x, M, y, workspace, workspace_bytes_given, stream, "q4_gemv");
+}
+
+extern "C" Q4_API int q8_gemv(const void* packed, int64_t N, int64_t K, const uint16_t* x, int M, float* y,
+                              void* workspace, size_t workspace_bytes_given, void* stream) {
+  return gemv_entry(8, packed, N, K, x, M, y, workspace, workspace_bytes_given, stream, "q8_gemv");
+}
+
+extern "C" Q4_API int q4_workspace_check(void* workspace, size_t workspace_bytes_given, void* stream) {
+  if (!workspace) return fail(Q4_ERR_INVALID_ARG, "q4_workspace_check: workspace is null");
+  if (workspace_bytes_given < kWsHeader)
+    return fail(Q4_ERR_BUFFER_TOO_SMALL, "q4_workspace_check: workspace smaller than its header");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t err = cudaStreamSynchronize(s);
+  if (err != cudaSuccess) return cuda_fail(err, "cudaStreamSynchronize");
+  unsigned status = 0;
+  err = cudaMemcpy(&status, workspace, sizeof(status), cudaMemcpyDeviceToHost);
+  if (err != cudaSuccess) return cuda_fail(err, "cudaMemcpy(status)");
+  if (status == 0) return Q4_OK;
+  err = cudaMemset(workspace, 0, workspace_bytes_given);
+  if (err != cudaSuccess) return cuda_fail(err, "cudaMemset(workspace)");
+  return fail(Q4_ERR_TIMEOUT, "a device wait gave up after %llu ns; the affected outputs are undefined",
+              static_cast<unsigned long long>(g_timeout_ns.load()));
+}
+
+extern "C" Q4_API int q4_set_wait_timeout_ns(uint64_t ns) {
+  g_timeout_ns.store(ns == 0 ? kDefaultTimeoutNs : ns);
+  return Q4_OK;
+}
+
+extern "C" Q4_API int q4_unpack_device(int bits, const void* packed, int64_t N, int64_t K, int8_t* q_out,
+                                       uint16_t* scales_out, void* stream) {
+  Shape s;
+  int rc = make_shape(bits, N, K, &s, "q4_unpack_device");
+  if (rc) return rc;
+  if (s.TC == 0) return Q4_OK;
+  if (!packed || !q_out || !scales_out) return fail(Q4_ERR_INVALID_ARG, "q4_unpack_device: null pointer");
+  if (reinterpret_cast<uintptr_t>(packed) % 16)
+    return fail(Q4_ERR_ALIGN, "q4_unpack_device: packed must be 16-byte aligned");
+  DeviceInfo dev;
+  if ((rc = device_info(&dev))) return rc;
+  const int warps = 8;
+  const long long blocks = (s.TC + warps - 1) / warps;
+  if (blocks > 0x7FFFFFFFLL) return fail(Q4_ERR_SHAPE, "q4_unpack_device: tensor too large");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (bits == 4)
+    q4k::unpack_kernel<4><<<static_cast<unsigned>(blocks), warps * 32, 0, st>>>(
+        static_cast<const uint8_t*>(packed), s.N, s.K, s.T, s.C, q_out, scales_out);
+  else
+    q4k::unpack_kernel<8><<<static_cast<unsigned>(blocks), warps * 32, 0, st>>>(
+        static_cast<const uint8_t*>(packed), s.N, s.K, s.T, s.C, q_out, scales_out);
+  cudaError_t err = cudaGetLastError();
+  return err == cudaSuccess ? Q4_OK : cuda_fail(err, "unpack kernel launch");
+}
+
+extern "C" Q4_API int q4_pack_weights_device(int bits, const void* canon_q, const uint16_t* scales_fp16, int64_t N,
+                                             int64_t K, void* out, size_t out_bytes, void* stream) {
+  Shape s;
+  int rc = make_shape(bits, N, K, &s, "q4_pack_weights_device");
+  if (rc) return rc;
+  const size_t need = static_cast<size_t>(s.TC) * (bits == 4 ? q4k::Format<4>::kChunkBytes : q4k::Format<8>::kChunkBytes);
+  if (need == 0) return Q4_OK;
+  if (!canon_q || !scales_fp16 || !out) return fail(Q4_ERR_INVALID_ARG, "q4_pack_weights_device: null pointer");
+  if (reinterpret_cast<uintptr_t>(out) % 16)
+    return fail(Q4_ERR_ALIGN, "q4_pack_weights_device: out must be 16-byte aligned");
+  if (reinterpret_cast<uintptr_t>(scales_fp16) % 2)
+    return fail(Q4_ERR_ALIGN, "q4_pack_weights_device: scales must be 2-byte aligned");
+  if (out_bytes < need)
+    return fail(Q4_ERR_BUFFER_TOO_SMALL, "q4_pack_weights_device: out_bytes %zu < %zu", out_bytes, need);
+  DeviceInfo dev;
+  if ((rc = device_info(&dev))) return rc;
+  const long long threads = s.TC * 64;
+  const long long blocks = (threads + 255) / 256;
+  if (blocks > 0x7FFFFFFFLL) return fail(Q4_ERR_SHAPE, "q4_pack_weights_device: tensor too large");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const uint8_t* q = static_cast<const uint8_t*>(canon_q);
+  if (bits == 4)
+    q4k::pack_kernel<4><<<static_cast<unsigned>(blocks), 256, 0, st>>>(q, scales_fp16, s.N, s.K, s.T, s.C,
+                                                                        static_cast<uint8_t*>(out));
+  else
+    q4k::pack_kernel<8><<<static_cast<unsigned>(blocks), 256, 0, st>>>(q, scales_fp16, s.N, s.K, s.T, s.C,
+                                                                        static_cast<uint8_t*>(out));
+  cudaError_t err = cudaGetLastError();
+  return err == cudaSuccess ? Q4_OK : cuda_fail(err, "pack kernel launch");
+}
+
+extern "C" Q4_API int q4_selftest_wait_timeout(uint64_t timeout_ns, int* status_out) {
+  if (!status_out) return fail(Q4_ERR_INVALID_ARG, "q4_selftest_wait_timeout: status_out is null");
+  DeviceInfo dev;
+  int rc = device_info(&dev);
+  if (rc) return rc;
+  int* d_result = nullptr;
+  cudaError_t err = cudaMalloc(&d_result, sizeof(int));
+  if (err != cudaSuccess) return cuda_fail(err, "cudaMalloc");
+  err = cudaMemset(d_result, 0xFF, sizeof(int));
+  if (err == cudaSuccess) {
+    q4k::wait_selftest_kernel<<<1, 32>>>(static_cast<unsigned long long>(timeout_ns), d_result);
+    err = cudaGetLastError();
+  }
+  if (err == cudaSuccess) err = cudaDeviceSynchronize();
+  int h = -1;
+  if (err == cudaSuccess) err = cudaMemcpy(&h, d_result, sizeof(int), cudaMemcpyDeviceToHost);
+  cudaFree(d_result);
+  if (err != cudaSuccess) return cuda_fail(err, "wait self-test");
+  *status_out = h;
+  return Q4_OK;
+}
+
+// ----------------------------------------------------------------------------
+// Layer stack: the ordered products of one decode step, captured once.
+// ----------------------------------------------------------------------------
+struct q4_stack {
+  cudaGraph_t graph = nullptr;
+  cudaGraphExec_t exec = nullptr;
+  void* workspace = nullptr;
+  size_t workspace_bytes = 0;
+  int launches = 0;
+  int device = 0;
+};
+
+extern "C" Q4_API int layer_stack_create(const q4_stack_entry* entries, int n_entries, int M, int flags,
+                                         q4_stack** out) {
+  if (!out) return fail(Q4_ERR_INVALID_ARG, "layer_stack_create: out is null");
+  *out = nullptr;
+  if (n_entries < 0 || (n_entries > 0 && !entries))
+    return fail(Q4_ERR_INVALID_ARG, "layer_stack_create: bad entry list");
+  if (M < 1 || M > 4) return fail(Q4_ERR_INVALID_ARG, "layer_stack_create: M must be in 1..4");
+  DeviceInfo dev;
+  int rc = device_info(&dev);
+  if (rc) return rc;
+  // workspace sized for the largest entry; all entries run in stream order
+  size_t ws = kWsHeader;
+  for (int i = 0; i < n_entries; ++i) {
+    Shape s;
+    char who[64];
+    snprintf(who, sizeof(who), "layer_stack_create entry %d", i);
+    if ((rc = make_shape(entries[i].bits, entries[i].N, entries[i].K, &s, who))) return rc;
+    const size_t need = workspace_bytes(s, M, dev);
+    if (need > ws) ws = need;
+  }
+  q4_stack* st = new q4_stack();
+  cudaGetDevice(&st->device);
+  cudaError_t err = cudaMalloc(&st->workspace, ws);
+  if (err != cudaSuccess) {
+    delete st;
+    return cuda_fail(err, "layer_stack_create: cudaMalloc(workspace)");
+  }
+  st->workspace_bytes = ws;
+  err = cudaMemset(st->workspace, 0, ws);
+  std::vector<Launch> launches(static_cast<size_t>(n_entries));
+  for (int i = 0; i < n_entries && err == cudaSuccess; ++i) {
+    const q4_stack_entry& en = entries[i];
+    char who[64];
+    snprintf(who, sizeof(who), "layer_stack_create entry %d", i);
+    rc = prepare(en.bits, en.packed, en.N, en.K, en.x, M, en.y, st->workspace, ws, who, &launches[i]);
+    if (rc) {
+      cudaFree(st->workspace);
+      delete st;
+      return rc;
+    }
+    launches[i].params.y = en.y;
+  }
+  if (err != cudaSuccess) {
+    cudaFree(st->workspace);
+    delete st;
+    return cuda_fail(err, "layer_stack_create: cudaMemset(workspace)");
+  }
+  cudaStream_t cs = nullptr;
+  err = cudaStreamCreateWithFlags(&cs, cudaStreamNonBlocking);
+  if (err == cudaSuccess) err = cudaStreamBeginCapture(cs, cudaStreamCaptureModeThreadLocal);
+  if (err != cudaSuccess) {
+    if (cs) cudaStreamDestroy(cs);
+    cudaFree(st->workspace);
+    delete st;
+    return cuda_fail(err, "layer_stack_create: begin capture");
+  }
+  const bool pdl = (flags & Q4_STACK_NO_PDL) == 0;
+  for (auto& L : launches) {
+    if (L.noop) continue;
+    rc = launch(L, cs, pdl);
+    if (rc) break;
+    ++st->launches;
+  }
+  cudaGraph_t graph = nullptr;
+  cudaError_t end_err = cudaStreamEndCapture(cs, &graph);
+  cudaStreamDestroy(cs);
+  if (rc || end_err != cudaSuccess) {
+    if (graph) cudaGraphDestroy(graph);
+    cudaFree(st->workspace);
+    delete st;
+    return rc ? rc : cuda_fail(end_err, "layer_stack_create: end capture");
+  }
+  st->graph = graph;
+  err = cudaGraphInstantiate(&st->exec, graph, 0);
+  if (err != cudaSuccess) {
+    cudaGraphDestroy(graph);
+    cudaFree(st->workspace);
+    delete st;
+    return cuda_fail(err, "layer_stack_create: cudaGraphInstantiate");
+  }
+  *out = st;
+  return Q4_OK;
+}
+
+extern "C" Q4_API int layer_stack_run(q4_stack* st, void* stream) {
+  if (!st || !st->exec) return fail(Q4_ERR_INVALID_ARG, "layer_stack_run: null stack");
+  cudaError_t err = cudaGraphLaunch(st->exec, static_cast<cudaStream_t>(stream));
+  return err == cudaSuccess ? Q4_OK : cuda_fail(err, "cudaGraphLaunch");
+}
+
+extern "C" Q4_API int layer_stack_check(q4_stack* st, void* stream) {
+  if (!st) return fail(Q4_ERR_INVALID_ARG, "layer_stack_check: null stack");
+  return q4_workspace_check(st->workspace, st->workspace_bytes, stream);
+}
+
+extern "C" Q4_API int layer_stack_launches(const q4_stack* st) { return st ? st->launches : 0; }
+
+extern "C" Q4_API void layer_stack_destroy(q4_stack* st) {
+  if (!st) return;
+  if (st->exec) cudaGraphExecDestroy(st->exec);
+  if (st->graph) cudaGraphDestroy(st->graph);
+  if (st->workspace) cudaFree(st->workspace);
+  delete st;
+}

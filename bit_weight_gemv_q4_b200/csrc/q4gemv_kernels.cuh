@@ -1,0 +1,745 @@
+// sm_100a kernels of the group-quantised weight x activation product
+// y[m][n] = sum_k s[n][k/32] q[n][k] x[m][k], M <= 4 activation rows.
+//
+// Design (B200):
+//  * The product is bound by HBM: each weight byte is read once and the work
+//    is a byte stream, not a dense contraction.  Every warp streams ONE
+//    contiguous byte range of the packed tensor: the flat sequence of chunks
+//    (32 rows x 64 or 32 columns, in memory order) is cut into equal ranges,
+//    one per warp of a grid sized to the SMs ("stream-K"), so all warps finish
+//    together whatever N and K are.
+//  * Bytes move HBM -> shared memory with 1-D bulk async copies
+//    (cp.async.bulk, the non-tensor TMA path) into a per-warp ring of D
+//    stages completed on mbarriers, with an L2 evict-first hint (the weights
+//    are read once).  Lane 0 of each warp is that warp's producer.
+//  * Dequantisation happens in registers.  A 32-bit word of codes decodes to
+//    four bf16 pairs with one mask-and-or each: the code u becomes the
+//    mantissa of 128 + u, an exact integer q + c (c = 136 for q4; for q8 the
+//    byte is split into a (2048 + 16 u_hi) and a (128 + u_lo) part, summing
+//    to q + 2304).  The pairs are already the A fragments of mma.sync
+//    m16n8k16 (bf16 in, fp32 accumulate) and the activations are its B
+//    fragments (columns >= M are never stored).  The offset c is removed
+//    inside the tensor core: each group's accumulator starts from (-c) * x,
+//    one product of a constant matrix with the same B fragment, shared by the
+//    two 16-row halves of the chunk.  Every product of a <= 12-bit integer
+//    and a bf16 is exact; each group's fp32 sum is scaled by its fp16 scale
+//    with one fp32 FMA per output.
+//  * Tiles split between warps are finished deterministically: each warp
+//    writes its partial sums to the workspace, and the last of the tile's
+//    warps to arrive (an integer counter) adds them in fixed warp order,
+//    writes y and re-zeroes the counter.  No float atomics: y is bitwise
+//    reproducible.
+//  * Programmatic dependent launch: a kernel issues its first weight copies,
+//    waits for its predecessor (griddepcontrol.wait) before touching x, y or
+//    the workspace, then lets its successor launch.
+//  * Every wait on an mbarrier is bounded by a %globaltimer limit; on expiry
+//    the warp records kStatusTimeout in the workspace, waits (bounded) for its
+//    own copies in flight and returns.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <stdint.h>
+
+namespace q4k {
+
+constexpr int kTileRows = 32;        // rows per tile: two m16 tensor-core tiles
+constexpr int kHalfBytes = 512;      // integer codes of one 16-row half (32 lanes x 16 B)
+constexpr int kCodeBytes = 1024;     // integer codes of a chunk
+constexpr unsigned kStatusTimeout = 1u;
+
+template <int BITS>
+struct Format;
+template <>
+struct Format<4> {
+  static constexpr int kKPerChunk = 64;    // two groups of 32
+  static constexpr int kChunkBytes = 1152; // 1024 code bytes + 32 rows x 2 groups x fp16
+};
+template <>
+struct Format<8> {
+  static constexpr int kKPerChunk = 32;    // one group
+  static constexpr int kChunkBytes = 1088; // 1024 code bytes + 32 rows x fp16
+};
+
+struct GemvParams {
+  const uint8_t* packed;     // packed chunks, 16-byte aligned
+  const uint16_t* x;         // bf16 bits [M][K]
+  float* y;                  // [M][N]
+  float* partials;           // [P][2][M][32] split-tile partial sums
+  unsigned* counters;        // [T] arrival counters, zero between launches
+  unsigned* status;          // status word
+  long long N, K;
+  long long TC;              // T * C, the number of chunks
+  int T, C;                  // tiles, chunks per tile
+  int P;                     // warps with work (P <= TC / U)
+  int khalf;                 // q4 with K % 64 == 32: the last chunk of a tile holds one group
+  unsigned long long timeout_ns;
+};
+
+// ----------------------------------------------------------------------------
+// PTX wrappers
+// ----------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t smem_addr(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void fence_barrier_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+__device__ __forceinline__ unsigned long long global_timer_ns() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+// Polls until the phase with the given parity completes or timeout_ns passes.
+__device__ __noinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity, unsigned long long timeout_ns) {
+  const unsigned long long t0 = global_timer_ns();
+  bool ok;
+  while (!(ok = mbar_try_wait(bar, parity))) {
+    if (global_timer_ns() - t0 > timeout_ns) break;
+  }
+  return ok;
+}
+
+// Waits for the phase with the given parity to complete, for at most
+// timeout_ns.  Returns false when the limit was reached.  Every lane of the
+// warp calls it; the result is uniform across the warp.
+__device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity, unsigned long long timeout_ns) {
+  bool ok = mbar_try_wait(bar, parity);
+  if (!__all_sync(0xFFFFFFFFu, ok)) {
+    if (!ok) ok = mbar_wait_slow(bar, parity, timeout_ns);
+    ok = __all_sync(0xFFFFFFFFu, ok);
+  }
+  return ok;
+}
+
+__device__ __forceinline__ uint64_t l2_evict_first_policy() {
+  uint64_t policy;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(policy));
+  return policy;
+}
+
+// 1-D bulk copy global -> this CTA's shared memory, completing on `bar`.
+__device__ __forceinline__ void bulk_copy_g2s(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar,
+                                              uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1], %2, [%3], %4;" ::
+          "r"(dst),
+      "l"(src), "r"(bytes), "r"(bar), "l"(policy)
+      : "memory");
+}
+
+__device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void grid_dependents_launch() { asm volatile("griddepcontrol.launch_dependents;"); }
+
+__device__ __forceinline__ uint4 lds128(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
+  return v;
+}
+__device__ __forceinline__ uint2 lds64(uint32_t addr) {
+  uint2 v;
+  asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(addr));
+  return v;
+}
+
+// 16-byte activation load done only by the lanes whose B column is a real
+// token (pred); the other lanes keep their register values, which only feed
+// output columns >= M that are never stored.
+__device__ __forceinline__ void ldg128_pred(uint4& v, const uint16_t* ptr, bool pred) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %5, 0;\n\t"
+      "@p ld.global.v4.u32 {%0, %1, %2, %3}, [%4];\n\t}"
+      : "+r"(v.x), "+r"(v.y), "+r"(v.z), "+r"(v.w)
+      : "l"(ptr), "r"(static_cast<int>(pred))
+      : "memory");
+}
+
+__device__ __forceinline__ uint32_t lop3_and_or(uint32_t a, uint32_t mask, uint32_t bits) {
+  uint32_t d;
+  asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(d) : "r"(a), "r"(mask), "r"(bits));  // (a & mask) | bits
+  return d;
+}
+
+// D += A (16x16, bf16, row) * B (16x8, bf16, col), fp32 accumulators.
+__device__ __forceinline__ void mma_bf16_m16n8k16(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 "
+      "{%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// D = A * B + C with separate C registers (no copies of C into D).
+__device__ __forceinline__ void mma_bf16_m16n8k16_c(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1,
+                                                    const float (&c)[4]) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 "
+      "{%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, {%10, %11, %12, %13};"
+      : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1), "f"(c[0]), "f"(c[1]), "f"(c[2]), "f"(c[3]));
+}
+
+__device__ __forceinline__ float2 half2_bits_to_float2(uint32_t h2) {
+  return __half22float2(*reinterpret_cast<const __half2*>(&h2));
+}
+
+// ----------------------------------------------------------------------------
+// In-register dequantisation (shared by the product and the debug decoder)
+// ----------------------------------------------------------------------------
+constexpr uint32_t kNibbleMask = 0x000F000Fu;
+constexpr uint32_t kBf16_128 = 0x43004300u;    // bf16 pair (128, 128): mantissa LSB = 1
+constexpr uint32_t kBf16_2048 = 0x45004500u;   // (2048, 2048): mantissa LSB = 16
+constexpr uint32_t kBf16_m136 = 0xC308C308u;   // (-136, -136): removes the q4 offset 128 + 8
+constexpr uint32_t kBf16_m2304 = 0xC510C510u;  // (-2304, -2304): removes the q8 offset 2048 + 128 + 128
+constexpr int kQ4Offset = 136;
+constexpr int kQ8Offset = 2304;
+
+// One q4 word -> A fragment registers a[0..3] holding exact integers q + 136.
+// a[i] takes nibbles i and i + 4 (bits 4i and 16 + 4i).
+__device__ __forceinline__ void dequant_q4_word(uint32_t w, uint32_t (&a)[4]) {
+  a[0] = lop3_and_or(w, kNibbleMask, kBf16_128);
+  a[1] = lop3_and_or(w >> 4, kNibbleMask, kBf16_128);
+  a[2] = lop3_and_or(w >> 8, kNibbleMask, kBf16_128);
+  a[3] = lop3_and_or(w >> 12, kNibbleMask, kBf16_128);
+}
+
+// Two q8 words (one m16n8k16 block) -> A fragments hi, lo with
+// hi + lo = q + 2304 exactly: hi = 2048 + 16 u_hi, lo = 128 + u_lo, u = q + 128.
+__device__ __forceinline__ void dequant_q8_block(uint32_t w0, uint32_t w1, uint32_t (&hi)[4], uint32_t (&lo)[4]) {
+  lo[0] = lop3_and_or(w0, kNibbleMask, kBf16_128);
+  lo[1] = lop3_and_or(w0 >> 8, kNibbleMask, kBf16_128);
+  lo[2] = lop3_and_or(w1, kNibbleMask, kBf16_128);
+  lo[3] = lop3_and_or(w1 >> 8, kNibbleMask, kBf16_128);
+  hi[0] = lop3_and_or(w0 >> 4, kNibbleMask, kBf16_2048);
+  hi[1] = lop3_and_or(w0 >> 12, kNibbleMask, kBf16_2048);
+  hi[2] = lop3_and_or(w1 >> 4, kNibbleMask, kBf16_2048);
+  hi[3] = lop3_and_or(w1 >> 12, kNibbleMask, kBf16_2048);
+}
+
+// ----------------------------------------------------------------------------
+// One chunk's contribution to this lane's accumulators acc[h][0..3]
+// (half h: rows 16h + gi and 16h + gi + 8 of the tile; columns 2ti, 2ti + 1).
+// ----------------------------------------------------------------------------
+struct ChunkRegs {
+  uint4 codes[2];  // this lane's 16 code bytes of each half
+  uint4 scales;    // q4: (R0: 2c, 2c+1) (R0+8) (R1) (R1+8);  q8: .x = (R0, R0+8), .y = (R1, R1+8)
+};
+
+__device__ __forceinline__ void q4_chunk_mac(float (&acc)[2][4], const ChunkRegs& r, const uint4& xa,
+                                             const uint4& xb) {
+  const uint32_t cst[4] = {kBf16_m136, kBf16_m136, kBf16_m136, kBf16_m136};
+  const uint32_t sc[4] = {r.scales.x, r.scales.y, r.scales.z, r.scales.w};
+#pragma unroll
+  for (int G = 0; G < 2; ++G) {
+    const uint4& xg = G ? xb : xa;
+    float corr[4] = {0.f, 0.f, 0.f, 0.f};  // -136 * (sum of x over the group), every row
+    mma_bf16_m16n8k16(corr, cst, xg.x, xg.y);
+    mma_bf16_m16n8k16(corr, cst, xg.z, xg.w);
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const uint4& w = r.codes[h];
+      float d[4];
+      uint32_t a[4];
+      dequant_q4_word(G ? w.z : w.x, a);
+      mma_bf16_m16n8k16_c(d, a, xg.x, xg.y, corr);
+      dequant_q4_word(G ? w.w : w.y, a);
+      mma_bf16_m16n8k16(d, a, xg.z, xg.w);
+      const float2 s_r = half2_bits_to_float2(sc[2 * h]);       // row 16h + gi: groups 2c, 2c+1
+      const float2 s_r8 = half2_bits_to_float2(sc[2 * h + 1]);  // row 16h + gi + 8
+      const float sr = G ? s_r.y : s_r.x;
+      const float sr8 = G ? s_r8.y : s_r8.x;
+      acc[h][0] = fmaf(sr, d[0], acc[h][0]);
+      acc[h][1] = fmaf(sr, d[1], acc[h][1]);
+      acc[h][2] = fmaf(sr8, d[2], acc[h][2]);
+      acc[h][3] = fmaf(sr8, d[3], acc[h][3]);
+    }
+  }
+}
+
+__device__ __forceinline__ void q8_chunk_mac(float (&acc)[2][4], const ChunkRegs& r, const uint4& xa) {
+  const uint32_t cst[4] = {kBf16_m2304, kBf16_m2304, kBf16_m2304, kBf16_m2304};
+  float corr[4] = {0.f, 0.f, 0.f, 0.f};  // -2304 * (sum of x over the group), every row
+  mma_bf16_m16n8k16(corr, cst, xa.x, xa.y);
+  mma_bf16_m16n8k16(corr, cst, xa.z, xa.w);
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    const uint4& w = r.codes[h];
+    float d[4];
+    uint32_t hi[4], lo[4];
+    dequant_q8_block(w.x, w.y, hi, lo);
+    mma_bf16_m16n8k16_c(d, hi, xa.x, xa.y, corr);
+    mma_bf16_m16n8k16(d, lo, xa.x, xa.y);
+    dequant_q8_block(w.z, w.w, hi, lo);
+    mma_bf16_m16n8k16(d, hi, xa.z, xa.w);
+    mma_bf16_m16n8k16(d, lo, xa.z, xa.w);
+    const float2 s = half2_bits_to_float2(h ? r.scales.y : r.scales.x);  // rows 16h + gi, 16h + gi + 8
+    acc[h][0] = fmaf(s.x, d[0], acc[h][0]);
+    acc[h][1] = fmaf(s.x, d[1], acc[h][1]);
+    acc[h][2] = fmaf(s.y, d[2], acc[h][2]);
+    acc[h][3] = fmaf(s.y, d[3], acc[h][3]);
+  }
+}
+
+// The flat sequence of TB blocks (U chunks each) is cut into P ranges,
+// range p = [floor(p*TB/P), floor((p+1)*TB/P)); P <= TB, so none is empty.
+// owner_of(i) is the range holding block i: the largest p with begin <= i.
+__device__ __forceinline__ int owner_of(long long i, long long TB, int P) {
+  return static_cast<int>(((i + 1) * P - 1) / TB);
+}
+__device__ __forceinline__ long long range_begin(int p, long long TB, int P) {
+  return static_cast<long long>(p) * TB / P;
+}
+
+template <int M>
+__device__ __forceinline__ void store_tile(const GemvParams& p, int r, const float (&v)[2][4], int lane) {
+  const int gi = lane >> 2, ti = lane & 3;
+  const int m0 = 2 * ti, m1 = 2 * ti + 1;
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    const long long row0 = static_cast<long long>(r) * kTileRows + 16 * h + gi;
+    const long long row1 = row0 + 8;
+    if (m0 < M) {
+      if (row0 < p.N) p.y[m0 * p.N + row0] = v[h][0];
+      if (row1 < p.N) p.y[m0 * p.N + row1] = v[h][2];
+    }
+    if (m1 < M) {
+      if (row0 < p.N) p.y[m1 * p.N + row0] = v[h][1];
+      if (row1 < p.N) p.y[m1 * p.N + row1] = v[h][3];
+    }
+  }
+}
+
+// Writes a finished tile's sums, or hands a split tile's partial sums to the
+// deterministic fix-up.
+template <int M, int U>
+__device__ __forceinline__ void finish_tile(const GemvParams& p, int pw, long long b, long long e, int r,
+                                         const float (&acc)[2][4], int lane) {
+  const int gi = lane >> 2, ti = lane & 3;
+  const int m0 = 2 * ti, m1 = 2 * ti + 1;
+  const long long tile_lo = static_cast<long long>(r) * p.C;
+  const long long tile_hi = tile_lo + p.C;
+  if (tile_lo >= b && tile_hi <= e) {
+    store_tile<M>(p, r, acc, lane);
+    return;
+  }
+  // split tile: this warp's partial goes to slot 0 (its first tile) or 1
+  const int slot = (tile_lo <= b) ? 0 : 1;
+  float* mine = p.partials + (static_cast<long long>(pw) * 2 + slot) * (M * kTileRows);
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    const int row0 = 16 * h + gi, row1 = row0 + 8;
+    if (m0 < M) {
+      mine[m0 * kTileRows + row0] = acc[h][0];
+      mine[m0 * kTileRows + row1] = acc[h][2];
+    }
+    if (m1 < M) {
+      mine[m1 * kTileRows + row0] = acc[h][1];
+      mine[m1 * kTileRows + row1] = acc[h][3];
+    }
+  }
+  __threadfence();
+  __syncwarp();
+  unsigned arrived = 0;
+  if (lane == 0) arrived = atomicAdd(p.counters + r, 1u);
+  arrived = __shfl_sync(0xFFFFFFFFu, arrived, 0);
+  const long long TB = p.TC / U;
+  const int p_lo = owner_of(tile_lo / U, TB, p.P);
+  const int p_hi = owner_of(tile_hi / U - 1, TB, p.P);
+  if (arrived != static_cast<unsigned>(p_hi - p_lo)) return;
+  // last arrival: add the partial sums in fixed warp order
+  __threadfence();
+  float s[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+  for (int q = p_lo; q <= p_hi; ++q) {
+    const int qslot = (tile_lo <= range_begin(q, TB, p.P) * U) ? 0 : 1;
+    const float* part = p.partials + (static_cast<long long>(q) * 2 + qslot) * (M * kTileRows);
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int row0 = 16 * h + gi, row1 = row0 + 8;
+      if (m0 < M) {
+        s[h][0] += __ldcg(part + m0 * kTileRows + row0);
+        s[h][2] += __ldcg(part + m0 * kTileRows + row1);
+      }
+      if (m1 < M) {
+        s[h][1] += __ldcg(part + m1 * kTileRows + row0);
+        s[h][3] += __ldcg(part + m1 * kTileRows + row1);
+      }
+    }
+  }
+  store_tile<M>(p, r, s, lane);
+  if (lane == 0) p.counters[r] = 0u;
+}
+
+// ----------------------------------------------------------------------------
+// The product kernel.  NW warps per CTA, each with a ring of D stages of U
+// chunks in shared memory.  Warp ranges are whole blocks of U chunks and U
+// divides C, so a stage never straddles two tiles: the tile bookkeeping runs
+// once per stage.  With XS the activations are staged once per CTA in shared
+// memory (one bulk copy per row, rows padded with 64 zero bytes so the empty
+// half of a last q4 chunk reads zeros); otherwise they are read from global
+// memory through L1.
+// ----------------------------------------------------------------------------
+constexpr int kXPadBytes = 64;
+
+template <int BITS, int NW, int D, int U>
+struct GemvConfig {
+  static constexpr int kChunkBytes = Format<BITS>::kChunkBytes;
+  static constexpr int kStageBytes = U * kChunkBytes;
+  static constexpr int kRingBytes = D * kStageBytes;
+  static constexpr int kBarOffset = NW * kRingBytes;
+  static constexpr int kXBarOffset = kBarOffset + NW * D * 8;
+  static constexpr int kXOffset = (kXBarOffset + 8 + 127) / 128 * 128;  // activations (XS)
+  static constexpr int kThreads = NW * 32;
+};
+
+__host__ __device__ constexpr long long x_row_stride_bytes(long long K) { return 2 * K + kXPadBytes; }
+
+template <int BITS, int M, int NW, int D, int U, bool XS>
+__global__ void __launch_bounds__(NW * 32, 1) gemv_kernel(const GemvParams p) {
+  using Cfg = GemvConfig<BITS, NW, D, U>;
+  constexpr int CB = Cfg::kChunkBytes;
+  constexpr int KC = Format<BITS>::kKPerChunk;
+  extern __shared__ __align__(128) unsigned char smem[];
+
+  const int lane = threadIdx.x & 31;
+  const int warp = threadIdx.x >> 5;
+  const int gi = lane >> 2, ti = lane & 3;
+  const int pw = blockIdx.x * NW + warp;
+
+  const uint32_t ring = smem_addr(smem + warp * Cfg::kRingBytes);
+  const uint32_t bars = smem_addr(smem + Cfg::kBarOffset) + warp * D * 8;
+  const uint32_t xbar = smem_addr(smem + Cfg::kXBarOffset);
+  const uint32_t xsm = smem_addr(smem + Cfg::kXOffset);
+  const uint32_t xstride = static_cast<uint32_t>(x_row_stride_bytes(p.K));
+
+  // this warp's range of chunks: whole blocks of U chunks
+  const long long TB = p.TC / U;
+  long long b = 0, e = 0;
+  if (pw < p.P) {
+    b = range_begin(pw, TB, p.P) * U;
+    e = range_begin(pw + 1, TB, p.P) * U;
+  }
+  const int nst = static_cast<int>((e - b) / U);
+
+  if (lane == 0) {
+    for (int s = 0; s < D; ++s) mbar_init(bars + 8 * s, 1);
+    if (XS && warp == 0) mbar_init(xbar, 1);
+    fence_barrier_init();
+  }
+  if (XS) {
+    // zero the pad after each activation row (bytes the bulk copies never write)
+    for (int i = threadIdx.x; i < M * (kXPadBytes / 16); i += NW * 32) {
+      const int m = i / (kXPadBytes / 16), q = i % (kXPadBytes / 16);
+      const uint32_t addr = xsm + m * xstride + static_cast<uint32_t>(2 * p.K) + 16 * q;
+      asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(addr), "r"(0) : "memory");
+    }
+  }
+  __syncthreads();
+
+  const uint64_t policy = l2_evict_first_policy();
+  const uint8_t* src = p.packed + b * CB;
+  if (lane == 0) {
+    const int first = nst < D ? nst : D;
+    for (int s = 0; s < first; ++s) {
+      mbar_arrive_expect_tx(bars + 8 * s, Cfg::kStageBytes);
+      bulk_copy_g2s(ring + s * Cfg::kStageBytes, src + static_cast<long long>(s) * Cfg::kStageBytes,
+                    Cfg::kStageBytes, bars + 8 * s, policy);
+    }
+  }
+  int issued = nst < D ? nst : D;
+
+  // The weights do not depend on the previous kernel; x, y and the workspace may.
+  grid_dependency_wait();
+  grid_dependents_launch();
+
+  if (XS && threadIdx.x == 0) {
+    mbar_arrive_expect_tx(xbar, static_cast<uint32_t>(M * 2 * p.K));
+    for (int m = 0; m < M; ++m) {
+      asm volatile(
+          "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+              xsm + m * xstride),
+          "l"(p.x + static_cast<long long>(m) * p.K), "r"(static_cast<uint32_t>(2 * p.K)), "r"(xbar)
+          : "memory");
+    }
+  }
+
+  int r = static_cast<int>(b / p.C);
+  int c = static_cast<int>(b - static_cast<long long>(r) * p.C);
+  const bool x_lane = gi < M;
+  // shared-memory activations: lanes whose column is not a token read row 0
+  const uint32_t xs_lane = xsm + (x_lane ? gi : 0) * xstride + 16 * ti;
+  const uint16_t* xrow = p.x + static_cast<long long>(x_lane ? gi : 0) * p.K + 8 * ti;
+  float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+  uint4 xa = make_uint4(0, 0, 0, 0), xb = make_uint4(0, 0, 0, 0);
+
+  bool ok = true;
+  if (XS) ok = mbar_wait_bounded(xbar, 0, p.timeout_ns);
+  int slot = 0;
+  uint32_t phase = 0;
+  int i = 0;
+  for (; ok && i < nst; ++i) {
+    if (!mbar_wait_bounded(bars + 8 * slot, phase, p.timeout_ns)) {
+      ok = false;
+      break;
+    }
+    const uint32_t stage = ring + slot * Cfg::kStageBytes;
+    ChunkRegs regs[U];
+#pragma unroll
+    for (int j = 0; j < U; ++j) {
+      regs[j].codes[0] = lds128(stage + j * CB + 16 * lane);
+      regs[j].codes[1] = lds128(stage + j * CB + kHalfBytes + 16 * lane);
+      if (BITS == 4) {
+        regs[j].scales = lds128(stage + j * CB + kCodeBytes + 16 * gi);
+      } else {
+        const uint2 s2 = lds64(stage + j * CB + kCodeBytes + 8 * gi);
+        regs[j].scales = make_uint4(s2.x, s2.y, 0u, 0u);
+      }
+    }
+    // Every lane has read the stage (warp-synchronous order, as an mbarrier
+    // release would give a separate consumer); lane 0 refills the slot.
+    __syncwarp();
+    if (i + D < nst) {
+      if (lane == 0) {
+        mbar_arrive_expect_tx(bars + 8 * slot, Cfg::kStageBytes);
+        bulk_copy_g2s(stage, src + static_cast<long long>(i + D) * Cfg::kStageBytes, Cfg::kStageBytes,
+                      bars + 8 * slot, policy);
+      }
+      issued = i + D + 1;
+    }
+#pragma unroll
+    for (int j = 0; j < U; ++j) {
+      if (XS) {
+        const uint32_t xo = xs_lane + 2 * KC * (c + j);
+        xa = lds128(xo);
+        if (BITS == 4) xb = lds128(xo + 64);
+      } else {
+        const uint16_t* xs = xrow + static_cast<long long>(c + j) * KC;
+        ldg128_pred(xa, xs, x_lane);
+        if (BITS == 4) {
+          // a K that is an odd multiple of 32 leaves the last chunk half empty
+          const bool half_empty = p.khalf && c + j == p.C - 1;
+          ldg128_pred(xb, xs + 32, x_lane && !half_empty);
+          if (half_empty) xb = make_uint4(0, 0, 0, 0);
+        }
+      }
+      if (BITS == 4)
+        q4_chunk_mac(acc, regs[j], xa, xb);
+      else
+        q8_chunk_mac(acc, regs[j], xa);
+    }
+    c += U;
+    if (c == p.C) {
+      finish_tile<M, U>(p, pw, b, e, r, acc, lane);
+      ++r;
+      c = 0;
+#pragma unroll
+      for (int h = 0; h < 2; ++h) acc[h][0] = acc[h][1] = acc[h][2] = acc[h][3] = 0.f;
+    }
+    if (++slot == D) {
+      slot = 0;
+      phase ^= 1u;
+    }
+  }
+  if (!ok) {
+    if (lane == 0) atomicOr(p.status, kStatusTimeout);
+    // wait (bounded) for this warp's own copies still in flight, then leave
+    for (int s = i; s < issued; ++s) {
+      if (!mbar_wait_bounded(bars + 8 * (s % D), (s / D) & 1, p.timeout_ns)) break;
+    }
+    if (XS) (void)mbar_wait_bounded(xbar, 0, p.timeout_ns);
+    return;
+  }
+  if (nst > 0 && c != 0) finish_tile<M, U>(p, pw, b, e, r, acc, lane);
+}
+
+// ----------------------------------------------------------------------------
+// Debug decoder: one warp per chunk, using the same in-register dequantisation
+// as the product kernel; writes int8 q [N][K] and fp16 scales [N][K/32].
+// ----------------------------------------------------------------------------
+__device__ __forceinline__ int bf16_bits_to_int(uint32_t h) {
+  const uint16_t b = static_cast<uint16_t>(h & 0xFFFF);
+  return static_cast<int>(__bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(&b)));
+}
+
+template <int BITS>
+__global__ void unpack_kernel(const uint8_t* packed, long long N, long long K, int T, int C, int8_t* q_out,
+                              uint16_t* s_out) {
+  constexpr int CB = Format<BITS>::kChunkBytes;
+  const int lane = threadIdx.x & 31;
+  const long long chunk = static_cast<long long>(blockIdx.x) * (blockDim.x / 32) + (threadIdx.x >> 5);
+  if (chunk >= static_cast<long long>(T) * C) return;
+  const int t = static_cast<int>(chunk / C), c = static_cast<int>(chunk % C);
+  const int gi = lane >> 2, ti = lane & 3;
+  const uint8_t* base = packed + chunk * CB;
+  const long long G = K / 32;
+  auto put = [&](long long row, long long col, int q) {
+    if (row < N && col < K) q_out[row * K + col] = static_cast<int8_t>(q);
+  };
+  for (int h = 0; h < 2; ++h) {
+    const uint4 codes = *reinterpret_cast<const uint4*>(base + kHalfBytes * h + 16 * lane);
+    const uint32_t w[4] = {codes.x, codes.y, codes.z, codes.w};
+    const long long R = static_cast<long long>(t) * kTileRows + 16 * h + gi;
+    if (BITS == 4) {
+      for (int j = 0; j < 4; ++j) {
+        uint32_t a[4];
+        dequant_q4_word(w[j], a);
+        const long long kb = 64LL * c + 32 * (j >> 1) + 8 * ti + 4 * (j & 1);
+        // a[0]: row R, k kb, kb+1; a[1]: row R+8; a[2]: row R, kb+2, kb+3; a[3]: row R+8
+        for (int reg = 0; reg < 4; ++reg) {
+          const long long row = R + 8 * (reg & 1);
+          const long long col = kb + 2 * (reg >> 1);
+          put(row, col, bf16_bits_to_int(a[reg]) - kQ4Offset);
+          put(row, col + 1, bf16_bits_to_int(a[reg] >> 16) - kQ4Offset);
+        }
+      }
+    } else {
+      for (int blk = 0; blk < 2; ++blk) {
+        uint32_t hi[4], lo[4];
+        dequant_q8_block(w[2 * blk], w[2 * blk + 1], hi, lo);
+        const long long kb = 32LL * c + 8 * ti + 4 * blk;
+        for (int reg = 0; reg < 4; ++reg) {
+          const long long row = R + 8 * (reg & 1);
+          const long long col = kb + 2 * (reg >> 1);
+          put(row, col, bf16_bits_to_int(hi[reg]) + bf16_bits_to_int(lo[reg]) - kQ8Offset);
+          put(row, col + 1, bf16_bits_to_int(hi[reg] >> 16) + bf16_bits_to_int(lo[reg] >> 16) - kQ8Offset);
+        }
+      }
+    }
+  }
+  if (ti == 0) {
+    const uint16_t* s = reinterpret_cast<const uint16_t*>(base + kCodeBytes + (BITS == 4 ? 16 : 8) * gi);
+    for (int h = 0; h < 2; ++h) {
+      for (int up = 0; up < 2; ++up) {
+        const long long row = static_cast<long long>(t) * kTileRows + 16 * h + gi + 8 * up;
+        if (row >= N) continue;
+        if (BITS == 4) {
+          for (int g = 0; g < 2; ++g) {
+            const long long grp = 2LL * c + g;
+            if (grp < G) s_out[row * G + grp] = s[4 * h + 2 * up + g];
+          }
+        } else {
+          s_out[row * G + c] = s[2 * h + up];
+        }
+      }
+    }
+  }
+}
+
+// ----------------------------------------------------------------------------
+// Device repack: canonical q and scales -> packed chunks, one thread per
+// 16-byte code slot (the same placement as the host packer).
+// ----------------------------------------------------------------------------
+template <int BITS>
+__global__ void pack_kernel(const uint8_t* q, const uint16_t* s, long long N, long long K, int T, int C,
+                            uint8_t* out) {
+  constexpr int CB = Format<BITS>::kChunkBytes;
+  const long long idx = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (idx >= static_cast<long long>(T) * C * 64) return;
+  const long long chunk = idx >> 6;
+  const int h = static_cast<int>((idx >> 5) & 1);
+  const int slot = static_cast<int>(idx & 31);
+  const int gi = slot >> 2, ti = slot & 3;
+  const long long t = chunk / C, c = chunk % C;
+  const long long R = t * kTileRows + 16 * h + gi;
+  uint32_t w[4];
+  for (int j = 0; j < 4; ++j) {
+    uint32_t word = 0;
+    if (BITS == 4) {
+      const int G = j >> 1, e = j & 1;
+      for (int i = 0; i < 8; ++i) {
+        const long long row = R + 8 * (i & 1);
+        const long long col = 64 * c + 32 * G + 8 * ti + 4 * e + 2 * ((i >> 1) & 1) + (i >> 2);
+        int v = 0;
+        if (row < N && col < K) {
+          const int byte = q[row * (K / 2) + col / 2];
+          const int nib = (col & 1) ? (byte >> 4) : (byte & 0xF);
+          v = nib >= 8 ? nib - 16 : nib;
+        }
+        word |= static_cast<uint32_t>(v + 8) << (4 * i);
+      }
+    } else {
+      const int e = j >> 1, f = j & 1;
+      for (int b = 0; b < 4; ++b) {
+        const long long row = R + 8 * (b & 1);
+        const long long col = 32 * c + 8 * ti + 4 * e + 2 * f + (b >> 1);
+        int v = 0;
+        if (row < N && col < K) v = static_cast<int8_t>(q[row * K + col]);
+        word |= static_cast<uint32_t>(v + 128) << (8 * b);
+      }
+    }
+    w[j] = word;
+  }
+  uint8_t* dst = out + chunk * CB;
+  *reinterpret_cast<uint4*>(dst + kHalfBytes * h + 16 * slot) = make_uint4(w[0], w[1], w[2], w[3]);
+  if (ti == 0 && h == 0) {
+    const long long G = K / 32;
+    uint16_t v[8];
+    for (int hh = 0; hh < 2; ++hh) {
+      for (int up = 0; up < 2; ++up) {
+        const long long row = t * kTileRows + 16 * hh + gi + 8 * up;
+        if (BITS == 4) {
+          for (int g = 0; g < 2; ++g) {
+            const long long grp = 2 * c + g;
+            v[4 * hh + 2 * up + g] = (row < N && grp < G) ? s[row * G + grp] : 0;
+          }
+        } else {
+          v[2 * hh + up] = row < N ? s[row * G + c] : 0;
+        }
+      }
+    }
+    if (BITS == 4) {
+      *reinterpret_cast<uint4*>(dst + kCodeBytes + 16 * gi) =
+          make_uint4(v[0] | (static_cast<uint32_t>(v[1]) << 16), v[2] | (static_cast<uint32_t>(v[3]) << 16),
+                     v[4] | (static_cast<uint32_t>(v[5]) << 16), v[6] | (static_cast<uint32_t>(v[7]) << 16));
+    } else {
+      *reinterpret_cast<uint2*>(dst + kCodeBytes + 8 * gi) =
+          make_uint2(v[0] | (static_cast<uint32_t>(v[1]) << 16), v[2] | (static_cast<uint32_t>(v[3]) << 16));
+    }
+  }
+}
+
+// ----------------------------------------------------------------------------
+// Self-test of the bounded wait: a barrier expecting two arrivals gets one.
+// ----------------------------------------------------------------------------
+__global__ void wait_selftest_kernel(unsigned long long timeout_ns, int* result) {
+  __shared__ __align__(8) unsigned long long bar_storage;
+  const uint32_t bar = smem_addr(&bar_storage);
+  if (threadIdx.x == 0) {
+    mbar_init(bar, 2);
+    fence_barrier_init();
+  }
+  __syncwarp();
+  if (threadIdx.x == 0) mbar_arrive(bar);
+  __syncwarp();
+  const bool ok = mbar_wait_bounded(bar, 0, timeout_ns);
+  if (threadIdx.x == 0) *result = ok ? 0 : 1;
+}
+
+}  // namespace q4k

@@ -1,0 +1,276 @@
+"""Python binding of the q4gemv C-ABI library (``libq4gemv.so``).
+
+Argument marshalling only: every step of the product runs in the library's
+CUDA kernels, and the functions here carry the C names.  Device buffers are
+torch CUDA tensors (or raw integer device addresses); host buffers are numpy
+arrays.  There is no CPU fallback: if the library cannot be loaded, importing
+this package raises, and GPU calls without a usable sm_100 device raise
+:class:`Q4Error`.
+
+See ``include/q4gemv.h`` for the operation, the layouts and the error codes.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import numpy as np
+
+from . import build as _build
+
+Q4_OK = 0
+Q4_ERR_INVALID_ARG = -1
+Q4_ERR_SHAPE = -2
+Q4_ERR_ALIGN = -3
+Q4_ERR_BUFFER_TOO_SMALL = -4
+Q4_ERR_CUDA = -5
+Q4_ERR_TIMEOUT = -6
+Q4_ERR_UNSUPPORTED = -7
+Q4_STACK_NO_PDL = 1
+
+ERROR_NAMES = {
+    Q4_ERR_INVALID_ARG: "INVALID_ARG",
+    Q4_ERR_SHAPE: "SHAPE",
+    Q4_ERR_ALIGN: "ALIGN",
+    Q4_ERR_BUFFER_TOO_SMALL: "BUFFER_TOO_SMALL",
+    Q4_ERR_CUDA: "CUDA",
+    Q4_ERR_TIMEOUT: "TIMEOUT",
+    Q4_ERR_UNSUPPORTED: "UNSUPPORTED",
+}
+
+# Symbols include/q4gemv.h declares (checked by the tests against the header).
+EXPORTED = [
+    "q4_last_error", "q4_packed_bytes", "q4_pack_weights", "q4_pack_weights_device", "q4_unpack_weights",
+    "q4_gemv_workspace_bytes",
+    "q4_gemv", "q8_gemv", "q4_workspace_check", "q4_set_wait_timeout_ns", "q4_unpack_device",
+    "q4_selftest_wait_timeout", "layer_stack_create", "layer_stack_run", "layer_stack_check",
+    "layer_stack_launches", "layer_stack_destroy",
+]
+
+
+class Q4Error(RuntimeError):
+    def __init__(self, code: int, message: str):
+        super().__init__(f"{ERROR_NAMES.get(code, code)}: {message}")
+        self.code = code
+
+
+class StackEntry(ctypes.Structure):
+    _fields_ = [
+        ("bits", ctypes.c_int),
+        ("N", ctypes.c_int64),
+        ("K", ctypes.c_int64),
+        ("packed", ctypes.c_void_p),
+        ("x", ctypes.c_void_p),
+        ("y", ctypes.c_void_p),
+    ]
+
+
+def _load() -> ctypes.CDLL:
+    path = _build.GEMV_LIB
+    if not os.path.exists(path) or _build._stale(path, _build.GEMV_DEPS):
+        try:
+            _build.build_gemv()
+        except Exception as exc:  # no silent fallback: the product needs its CUDA library
+            raise ImportError(f"libq4gemv.so is missing and could not be built: {exc}") from exc
+    L = ctypes.CDLL(path)
+    i32, i64, u64, sz, vp = ctypes.c_int, ctypes.c_int64, ctypes.c_uint64, ctypes.c_size_t, ctypes.c_void_p
+    sig = {
+        "q4_last_error": ([], ctypes.c_char_p),
+        "q4_packed_bytes": ([i32, i64, i64], sz),
+        "q4_pack_weights": ([i32, vp, vp, i64, i64, vp, sz], i32),
+        "q4_pack_weights_device": ([i32, vp, vp, i64, i64, vp, sz, vp], i32),
+        "q4_unpack_weights": ([i32, vp, sz, i64, i64, vp, vp], i32),
+        "q4_gemv_workspace_bytes": ([i32, i64, i64, i32], sz),
+        "q4_gemv": ([vp, i64, i64, vp, i32, vp, vp, sz, vp], i32),
+        "q8_gemv": ([vp, i64, i64, vp, i32, vp, vp, sz, vp], i32),
+        "q4_workspace_check": ([vp, sz, vp], i32),
+        "q4_set_wait_timeout_ns": ([u64], i32),
+        "q4_unpack_device": ([i32, vp, i64, i64, vp, vp, vp], i32),
+        "q4_selftest_wait_timeout": ([u64, ctypes.POINTER(i32)], i32),
+        "layer_stack_create": ([ctypes.POINTER(StackEntry), i32, i32, i32, ctypes.POINTER(vp)], i32),
+        "layer_stack_run": ([vp, vp], i32),
+        "layer_stack_check": ([vp, vp], i32),
+        "layer_stack_launches": ([vp], i32),
+        "layer_stack_destroy": ([vp], None),
+    }
+    for name, (args, res) in sig.items():
+        f = getattr(L, name)
+        f.argtypes = args
+        f.restype = res
+    return L
+
+
+_lib = _load()
+
+
+def lib() -> ctypes.CDLL:
+    return _lib
+
+
+def q4_last_error() -> str:
+    return _lib.q4_last_error().decode()
+
+
+def _check(rc: int) -> None:
+    if rc != Q4_OK:
+        raise Q4Error(rc, q4_last_error())
+
+
+def _dev_ptr(t) -> int:
+    """Device address of a torch CUDA tensor (or an int address, or None -> 0)."""
+    if t is None:
+        return 0
+    if isinstance(t, int):
+        return t
+    if not getattr(t, "is_cuda", False):
+        raise Q4Error(Q4_ERR_INVALID_ARG, "expected a CUDA tensor")
+    return t.data_ptr()
+
+
+def _nbytes(t) -> int:
+    return t.numel() * t.element_size()
+
+
+def _stream(stream) -> int:
+    if stream is None:
+        import torch
+
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+# ----------------------------------------------------------------------------
+# host-side packing
+# ----------------------------------------------------------------------------
+def q4_packed_bytes(bits: int, N: int, K: int) -> int:
+    return int(_lib.q4_packed_bytes(bits, N, K))
+
+
+def q4_pack_weights(bits: int, canon_q: np.ndarray, scales_fp16: np.ndarray, N: int, K: int) -> np.ndarray:
+    """Canonical q and fp16 scale bits (numpy, host) -> packed bytes (numpy uint8)."""
+    q = np.ascontiguousarray(canon_q, dtype=np.uint8 if bits == 4 else np.int8)
+    s = np.ascontiguousarray(scales_fp16, dtype=np.uint16)
+    expect_q = (N, K // 2) if bits == 4 else (N, K)
+    if q.size != expect_q[0] * expect_q[1] or s.size != N * (K // 32):
+        raise Q4Error(Q4_ERR_SHAPE, f"canonical arrays do not match N={N} K={K}")
+    out = np.zeros(max(q4_packed_bytes(bits, N, K), 1), dtype=np.uint8)
+    _check(_lib.q4_pack_weights(bits, q.ctypes.data, s.ctypes.data, N, K, out.ctypes.data, out.size))
+    return out[: q4_packed_bytes(bits, N, K)]
+
+
+def q4_pack_weights_device(bits: int, canon_q, scales_fp16, N: int, K: int, out, stream=None) -> None:
+    """Canonical q and fp16 scale bits (device tensors) -> packed bytes in `out` (device)."""
+    _check(_lib.q4_pack_weights_device(bits, _dev_ptr(canon_q), _dev_ptr(scales_fp16), N, K, _dev_ptr(out),
+                                       _nbytes(out), _stream(stream)))
+
+
+def q4_unpack_weights(bits: int, packed: np.ndarray, N: int, K: int) -> tuple[np.ndarray, np.ndarray]:
+    packed = np.ascontiguousarray(packed, dtype=np.uint8)
+    q = np.zeros((N, K // 2) if bits == 4 else (N, K), dtype=np.uint8 if bits == 4 else np.int8)
+    s = np.zeros((N, K // 32), dtype=np.uint16)
+    _check(_lib.q4_unpack_weights(bits, packed.ctypes.data, packed.size, N, K, q.ctypes.data, s.ctypes.data))
+    return q, s
+
+
+# ----------------------------------------------------------------------------
+# device-side product
+# ----------------------------------------------------------------------------
+def q4_gemv_workspace_bytes(bits: int, N: int, K: int, M: int) -> int:
+    n = int(_lib.q4_gemv_workspace_bytes(bits, N, K, M))
+    if n == 0:
+        raise Q4Error(Q4_ERR_INVALID_ARG, q4_last_error())
+    return n
+
+
+def _gemv(fn, packed, N, K, x, M, y, workspace, stream):
+    _check(fn(_dev_ptr(packed), N, K, _dev_ptr(x), M, _dev_ptr(y), _dev_ptr(workspace),
+              _nbytes(workspace) if workspace is not None and not isinstance(workspace, int) else 0,
+              _stream(stream)))
+
+
+def q4_gemv(packed, N: int, K: int, x, M: int, y, workspace, stream=None) -> None:
+    """y[M][N] (fp32, device) = W x for packed q4 W and bf16 x [M][K] (device)."""
+    _gemv(_lib.q4_gemv, packed, N, K, x, M, y, workspace, stream)
+
+
+def q8_gemv(packed, N: int, K: int, x, M: int, y, workspace, stream=None) -> None:
+    """y[M][N] (fp32, device) = W x for packed q8 W and bf16 x [M][K] (device)."""
+    _gemv(_lib.q8_gemv, packed, N, K, x, M, y, workspace, stream)
+
+
+def q4_workspace_check(workspace, stream=None) -> None:
+    _check(_lib.q4_workspace_check(_dev_ptr(workspace), _nbytes(workspace), _stream(stream)))
+
+
+def q4_set_wait_timeout_ns(ns: int) -> None:
+    _check(_lib.q4_set_wait_timeout_ns(int(ns)))
+
+
+def q4_unpack_device(bits: int, packed, N: int, K: int, q_out, scales_out, stream=None) -> None:
+    _check(_lib.q4_unpack_device(bits, _dev_ptr(packed), N, K, _dev_ptr(q_out), _dev_ptr(scales_out),
+                                 _stream(stream)))
+
+
+def q4_selftest_wait_timeout(timeout_ns: int) -> int:
+    out = ctypes.c_int(-1)
+    _check(_lib.q4_selftest_wait_timeout(int(timeout_ns), ctypes.byref(out)))
+    return out.value
+
+
+# ----------------------------------------------------------------------------
+# layer stack
+# ----------------------------------------------------------------------------
+class LayerStack:
+    """Owner of a captured q4_stack; keeps the entry tensors alive."""
+
+    def __init__(self, handle: int, keepalive):
+        self.handle = handle
+        self._keepalive = keepalive
+
+    def launches(self) -> int:
+        return int(_lib.layer_stack_launches(self.handle))
+
+    def close(self) -> None:
+        if self.handle:
+            _lib.layer_stack_destroy(self.handle)
+            self.handle = 0
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+def layer_stack_create(entries, M: int, flags: int = 0) -> LayerStack:
+    """entries: sequence of (bits, N, K, packed, x, y) with device tensors."""
+    arr = (StackEntry * max(len(entries), 1))()
+    keep = []
+    for i, (bits, N, K, packed, x, y) in enumerate(entries):
+        arr[i] = StackEntry(bits, N, K, _dev_ptr(packed), _dev_ptr(x), _dev_ptr(y))
+        keep.append((packed, x, y))
+    h = ctypes.c_void_p(0)
+    _check(_lib.layer_stack_create(arr, len(entries), M, flags, ctypes.byref(h)))
+    return LayerStack(h.value, keep)
+
+
+def layer_stack_run(stack: LayerStack, stream=None) -> None:
+    _check(_lib.layer_stack_run(stack.handle, _stream(stream)))
+
+
+def layer_stack_check(stack: LayerStack, stream=None) -> None:
+    _check(_lib.layer_stack_check(stack.handle, _stream(stream)))
+
+
+def layer_stack_destroy(stack: LayerStack) -> None:
+    stack.close()
+
+
+__all__ = [
+    "Q4Error", "LayerStack", "StackEntry", "EXPORTED", "lib", "q4_last_error", "q4_packed_bytes",
+    "q4_pack_weights", "q4_pack_weights_device", "q4_unpack_weights", "q4_gemv_workspace_bytes", "q4_gemv", "q8_gemv",
+    "q4_workspace_check", "q4_set_wait_timeout_ns", "q4_unpack_device", "q4_selftest_wait_timeout",
+    "layer_stack_create", "layer_stack_run", "layer_stack_check", "layer_stack_destroy",
+]

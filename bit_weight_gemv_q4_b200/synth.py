@@ -1,4 +1,4 @@
-"""Python binding of the seeded synthetic-input generator (``csrc/synth.c``).
+"""Python binding of the seeded synthetic-input generator (``csrc/synth.cu``).
 
 Every array returned is in the canonical (interchange) layout:
 
@@ -10,7 +10,9 @@ Every array returned is in the canonical (interchange) layout:
 
 Streams identify tensors: one (seed, stream) pair per weight tensor, a separate
 stream for its scales and one per activation block, so any row of any tensor
-can be regenerated on its own.
+can be regenerated on its own.  The ``*_device`` functions write the same bits
+into device memory (torch CUDA tensors), for workloads too large to generate on
+the host.
 """
 from __future__ import annotations
 
@@ -40,11 +42,18 @@ def lib() -> ctypes.CDLL:
         L.synth_f64_to_f16_array.argtypes = [vp, i64, vp]
         L.synth_f64_to_bf16_array.argtypes = [vp, i64, vp]
         L.synth_words.argtypes = [u64, u64, i64, i64, vp]
-        for f in (L.synth_q4, L.synth_q8, L.synth_scales, L.synth_bf16_normals, L.synth_normals_f64):
+        L.synth_log_array.argtypes = [vp, i64, vp]
+        L.synth_cos2pi_array.argtypes = [vp, i64, vp]
+        L.synth_q4_device.argtypes = [u64, u64, i64, i64, i64, vp, vp]
+        L.synth_q8_device.argtypes = [u64, u64, i64, i64, i64, vp, vp]
+        L.synth_scales_device.argtypes = [u64, u64, i64, i64, i64, ctypes.c_double, vp, vp]
+        L.synth_bf16_normals_device.argtypes = [u64, u64, i64, i64, vp, vp]
+        for f in (L.synth_q4, L.synth_q8, L.synth_scales, L.synth_bf16_normals, L.synth_normals_f64,
+                  L.synth_q4_device, L.synth_q8_device, L.synth_scales_device, L.synth_bf16_normals_device):
             f.restype = ctypes.c_int
-        L.synth_f64_to_f16_array.restype = None
-        L.synth_f64_to_bf16_array.restype = None
-        L.synth_words.restype = None
+        for f in (L.synth_f64_to_f16_array, L.synth_f64_to_bf16_array, L.synth_words, L.synth_log_array,
+                  L.synth_cos2pi_array):
+            f.restype = None
         _lib = L
     return _lib
 
@@ -96,6 +105,20 @@ def words(seed: int, stream: int, i0: int, count: int) -> np.ndarray:
     return out
 
 
+def log_f64(a: np.ndarray) -> np.ndarray:
+    a = np.ascontiguousarray(a, dtype=np.float64)
+    out = np.empty_like(a)
+    lib().synth_log_array(_ptr(a), a.size, _ptr(out))
+    return out
+
+
+def cos2pi_f64(a: np.ndarray) -> np.ndarray:
+    a = np.ascontiguousarray(a, dtype=np.float64)
+    out = np.empty_like(a)
+    lib().synth_cos2pi_array(_ptr(a), a.size, _ptr(out))
+    return out
+
+
 def f64_to_f16_bits(a: np.ndarray) -> np.ndarray:
     a = np.ascontiguousarray(a, dtype=np.float64)
     out = np.empty(a.shape, dtype=np.uint16)
@@ -139,7 +162,53 @@ def tensor(bits: int, seed: int, tensor_id: int, N: int, K: int, row0: int = 0, 
     return q, s
 
 
+# ----------------------------------------------------------------------------
+# device-side generation (same bits, written into torch CUDA tensors)
+# ----------------------------------------------------------------------------
+def _dev(t) -> int:
+    if not getattr(t, "is_cuda", False) or not t.is_contiguous():
+        raise ValueError("expected a contiguous CUDA tensor")
+    return t.data_ptr()
+
+
+def _stream(stream) -> int:
+    if stream is None:
+        import torch
+
+        return torch.cuda.current_stream().cuda_stream
+    return stream if isinstance(stream, int) else stream.cuda_stream
+
+
+def _dev_check(rc: int, what: str) -> None:
+    if rc != 0:
+        raise RuntimeError(f"synth {what}: {'bad arguments' if rc == -1 else 'CUDA launch failed'}")
+
+
+def weights_device(bits: int, seed: int, stream_id: int, K: int, row0: int, nrows: int, out, stream=None) -> None:
+    """Canonical weights of rows [row0, row0+nrows) into `out` (uint8 [nrows][K/2] or int8 [nrows][K])."""
+    expect = nrows * (K // 2 if bits == 4 else K)
+    if out.numel() * out.element_size() < expect:
+        raise ValueError("output tensor too small")
+    fn = lib().synth_q4_device if bits == 4 else lib().synth_q8_device
+    _dev_check(fn(seed, stream_id, K, row0, nrows, _dev(out), _stream(stream)), "weights")
+
+
+def scales_device(seed: int, stream_id: int, K: int, row0: int, nrows: int, out, std: float = SCALE_STD,
+                  stream=None) -> None:
+    if out.numel() * out.element_size() < 2 * nrows * (K // 32):
+        raise ValueError("output tensor too small")
+    _dev_check(lib().synth_scales_device(seed, stream_id, K, row0, nrows, float(std), _dev(out), _stream(stream)),
+               "scales")
+
+
+def activations_device(seed: int, stream_id: int, M: int, K: int, out, stream=None) -> None:
+    if out.numel() * out.element_size() < 2 * M * K:
+        raise ValueError("output tensor too small")
+    _dev_check(lib().synth_bf16_normals_device(seed, stream_id, 0, M * K, _dev(out), _stream(stream)), "activations")
+
+
 __all__ = [
+    "weights_device", "scales_device", "activations_device", "log_f64", "cos2pi_f64",
     "weights", "scales", "activations", "normals_f64", "words", "f64_to_f16_bits", "f64_to_bf16_bits",
     "tensor", "weight_stream", "scale_stream", "act_stream", "SCALE_STD", "lib",
 ]

@@ -1,0 +1,224 @@
+/*
+ * q4gemv -- group-quantised weight x activation products for single-user LLM
+ * decode on NVIDIA B200 (sm_100a).
+ *
+ * The operation.  Single-user decode of a dense ~27B hybrid model streams every
+ * low-bit weight once per generated token, so its speed is set by how fast the
+ * weight bytes leave HBM ("Fit != Speed": wiselychen guide "Qwen3.8-27B
+ * measured: RTX 3090/4090/5090/PRO 6000/DGX Spark/Mac", section "Before
+ * deploying: weights, KV cache, memory bandwidth"; bs178.com llamAmpere post,
+ * "Why it is this fast", part two).  The weights are 4-bit integers ("INT4",
+ * four bits instead of sixteen: jdon.com "Two RTX 3090s, 105 tok/s", section
+ * "27 billion parameters into 24 GB"), with 8-bit integers for the sensitive
+ * attention projections and the output head (bs178.com post, part two), and
+ * 16-bit activations ("W4A16": jdon.com page, section "Schools of
+ * quantisation").  The pages give no bit layout; this library reads the formats
+ * as: groups of 32 consecutive k, one fp16 scale per group, symmetric (no zero
+ * point), q4 in [-8, 7], q8 in [-127, 127].
+ *
+ *   W[n][k] = s[n][k/32] * q[n][k]                  (N x K)
+ *   y[m][n] = sum_k W[n][k] * x[m][k]               m < M <= 4, x bf16, y fp32
+ *
+ * M = 1 is plain decode; M = 4 is one verification pass over three drafted
+ * tokens plus one (multi-token-prediction speculative decoding with depth 3:
+ * bs178.com post, part four).
+ *
+ * Conventions for every entry point:
+ *   - Return value: Q4_OK (0) or a negative Q4_ERR_* code; q4_last_error()
+ *     then returns a message for the calling thread.
+ *   - Argument errors are detected on the host, synchronously, before any
+ *     launch; nothing is launched when a call fails.
+ *   - "device" pointers are CUDA device (or managed) memory owned by the
+ *     caller; "host" pointers are ordinary host memory owned by the caller.
+ *   - Device work is asynchronous on the caller's stream (a cudaStream_t passed
+ *     as void*; NULL is the legacy default stream).  No entry point except
+ *     layer_stack_create / layer_stack_destroy / q4_workspace_check allocates,
+ *     frees or synchronises.
+ *   - There is no CPU fallback: without a usable sm_100a device the GPU entry
+ *     points fail with Q4_ERR_CUDA.
+ *
+ * ---------------------------------------------------------------------------
+ * Canonical (interchange) layout -- the input of q4_pack_weights:
+ *   q4:     uint8 [N][K/2]; element k of a row is in byte k/2, low nibble for
+ *           even k; 4-bit two's complement (-8..7).
+ *   q8:     int8  [N][K].
+ *   scales: uint16 [N][K/32], IEEE binary16 bits.
+ *   x:      uint16 [M][K], bfloat16 bits, row-major (leading dimension K).
+ *   y:      float  [M][N], row-major (leading dimension N); overwritten.
+ *
+ * Kernel-native packed layout -- the output of q4_pack_weights:
+ *   Rows are cut into T = ceil(N/32) tiles of 32 rows.  Each tile is cut along
+ *   K into C chunks: q4 chunks cover 64 k (two groups), C = ceil(K/64); q8
+ *   chunks cover 32 k (one group), C = K/32.  Chunk (t, c) is CB bytes at
+ *   offset (t*C + c)*CB, CB = 1152 (q4) or 1088 (q8), so each tile, and the
+ *   whole tensor, is one contiguous run in memory order t, c.
+ *   A chunk is two 512-byte code blocks, h = 0, 1 (rows 32t + 16h .. +15),
+ *   then the scales of its groups.  Code block h is 32 slots of 16 bytes,
+ *   slot L = 4*gi + ti (gi in 0..7, ti in 0..3), each four little-endian
+ *   32-bit words.  With R = 32t + 16h + gi and R' = R + 8:
+ *   q4: word j = 2G + e (G, e in {0,1}) holds eight nibbles; nibble i (bits
+ *       4i..4i+3) is u = q + 8 of row (i odd ? R' : R), column
+ *       64c + 32G + 8ti + 4e + 2*((i>>1)&1) + (i>>2).
+ *       Scales (at byte 1024): 8 entries of 16 bytes; entry gi holds the
+ *       fp16 scales s(r, 2c + g) at position 4h + 2up + g for the rows
+ *       r = 32t + 16h + gi + 8up (h, up, g in {0,1}).
+ *   q8: word j = 2e + f holds four bytes; byte b (bits 8b..8b+7) is
+ *       u = q + 128 of row (b odd ? R' : R), column 32c + 8ti + 4e + 2f + (b>>1).
+ *       Scales (at byte 1024): 8 entries of 8 bytes; entry gi holds s(r, c)
+ *       at position 2h + up for r = 32t + 16h + gi + 8up.
+ *   Padding rows (>= N) and padding groups (>= K/32) hold q = 0 and scale 0.
+ *   This places, for one warp, exactly the operands of bf16 m16n8k16 tensor-core
+ *   products: slot L of block h is lane L's A fragment for the 16-row half h,
+ *   and every word decodes to bf16 pairs with one mask-and-or per pair.  The
+ *   packed buffer must be 16-byte aligned.
+ * ---------------------------------------------------------------------------
+ */
+#ifndef Q4GEMV_H
+#define Q4GEMV_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define Q4_API __attribute__((visibility("default")))
+#else
+#define Q4_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define Q4_OK 0
+#define Q4_ERR_INVALID_ARG (-1)      /* null pointer, bits not 4/8, M outside 0..4 */
+#define Q4_ERR_SHAPE (-2)            /* K % 32 != 0, negative sizes, sizes too large */
+#define Q4_ERR_ALIGN (-3)            /* packed / x / workspace not 16-byte aligned, y not 4-byte */
+#define Q4_ERR_BUFFER_TOO_SMALL (-4) /* output or workspace smaller than required */
+#define Q4_ERR_CUDA (-5)             /* a CUDA call failed (message has the CUDA error) */
+#define Q4_ERR_TIMEOUT (-6)          /* a bounded device wait gave up (see q4_workspace_check) */
+#define Q4_ERR_UNSUPPORTED (-7)      /* no sm_100 device, or a request this build does not serve */
+
+/* Message of the last failing call on this thread ("" if none). */
+Q4_API const char* q4_last_error(void);
+
+/* Bytes of the packed layout for an N x K tensor of `bits` (4 or 8); 0 when
+ * bits is not 4 or 8, N or K is negative, or K % 32 != 0.
+ * Weight-stream bytes are the algorithmic N*K/2 + N*K/16 (q4) or
+ * N*K + N*K/16 (q8); the packed size adds only the row and group padding. */
+Q4_API size_t q4_packed_bytes(int bits, int64_t N, int64_t K);
+
+/* Offline repack (host -> host), once per tensor, not per token.  Reads the
+ * canonical q (uint8 [N][K/2] for bits=4, int8 [N][K] for bits=8) and fp16
+ * scales [N][K/32]; writes the packed layout into `out` (out_bytes >=
+ * q4_packed_bytes).  A pure byte and bit permutation plus the q -> q+8 / q+128
+ * offset; bit-exact inverse: q4_unpack_weights.  The same call packs q8
+ * (bits = 8).  Errors: INVALID_ARG, SHAPE, BUFFER_TOO_SMALL. */
+Q4_API int q4_pack_weights(int bits, const void* canon_q, const uint16_t* scales_fp16, int64_t N, int64_t K,
+                           void* out, size_t out_bytes);
+
+/* The same repack on the device: canonical q and scales in device memory,
+ * packed bytes written to `out` (device, 16-byte aligned, out_bytes >=
+ * q4_packed_bytes), asynchronously on `stream`.  Produces exactly the bytes
+ * q4_pack_weights produces.  Errors: INVALID_ARG, SHAPE, ALIGN,
+ * BUFFER_TOO_SMALL, CUDA. */
+Q4_API int q4_pack_weights_device(int bits, const void* canon_q, const uint16_t* scales_fp16, int64_t N, int64_t K,
+                                  void* out, size_t out_bytes, void* stream);
+
+/* Inverse of q4_pack_weights (host -> host): writes canonical q and scales.
+ * Padding is dropped.  packed_bytes must be >= q4_packed_bytes. */
+Q4_API int q4_unpack_weights(int bits, const void* packed, size_t packed_bytes, int64_t N, int64_t K,
+                             void* canon_q_out, uint16_t* scales_out);
+
+/* Bytes of device workspace q4_gemv / q8_gemv need for this shape on the
+ * current device.  The workspace holds a status word, the per-warp partial
+ * sums of tiles split between warps (a region of fixed size per device) and
+ * one arrival counter per 16-row tile.  It must be zero-filled before its
+ * first use; every completed call leaves the status word and the counters
+ * zero again, so one workspace serves any sequence of stream-ordered calls,
+ * of any shapes and M, whose requirements it meets.  Calls that may run
+ * concurrently need separate workspaces.  Returns 0 for invalid arguments. */
+Q4_API size_t q4_gemv_workspace_bytes(int bits, int64_t N, int64_t K, int M);
+
+/* y = W x for packed q4 weights (device), bf16 x [M][K] (device, 16-byte
+ * aligned), fp32 y [M][N] (device, overwritten).  M in 0..4; M = 0 or N = 0
+ * is a no-op; K = 0 writes y = 0.  Asynchronous on `stream`; launches one
+ * kernel; deterministic (bitwise-identical y for identical inputs and device).
+ * Errors: INVALID_ARG, SHAPE, ALIGN, BUFFER_TOO_SMALL (workspace), CUDA.
+ * A device-side wait that gives up is reported by q4_workspace_check. */
+Q4_API int q4_gemv(const void* packed, int64_t N, int64_t K, const uint16_t* x, int M, float* y, void* workspace,
+                   size_t workspace_bytes, void* stream);
+
+/* The same product for packed q8 weights. */
+Q4_API int q8_gemv(const void* packed, int64_t N, int64_t K, const uint16_t* x, int M, float* y, void* workspace,
+                   size_t workspace_bytes, void* stream);
+
+/* Synchronises `stream`, then reads and clears the workspace's status word.
+ * Returns Q4_OK, or Q4_ERR_TIMEOUT when a kernel that used this workspace gave
+ * up a bounded wait since the last check (that call's y is then undefined);
+ * in that case the whole workspace is zero-filled again before returning. */
+Q4_API int q4_workspace_check(void* workspace, size_t workspace_bytes, void* stream);
+
+/* Upper bound, in nanoseconds, of every device-side wait the library's kernels
+ * make (on the arrival of their own bulk copies).  Default 2e9.  Applies to
+ * launches and stack captures made after the call.  0 restores the default. */
+Q4_API int q4_set_wait_timeout_ns(uint64_t ns);
+
+/* Debug decode on the device: runs the kernels' in-register dequantisation on
+ * every packed word and writes the integers q (int8 [N][K], device) and the
+ * scales (uint16 [N][K/32], device).  Used to check that in-register unpack is
+ * bit-exact against the canonical weights. */
+Q4_API int q4_unpack_device(int bits, const void* packed, int64_t N, int64_t K, int8_t* q_out, uint16_t* scales_out,
+                            void* stream);
+
+/* Self-test of the bounded device wait: launches one kernel that waits, with
+ * the library's wait routine and a limit of timeout_ns, on a barrier that
+ * nothing completes, then reports.  *status_out (host) receives 1 when the
+ * wait gave up as designed, 0 if it (wrongly) succeeded.  Synchronous. */
+Q4_API int q4_selftest_wait_timeout(uint64_t timeout_ns, int* status_out);
+
+/* ---------------------------------------------------------------------------
+ * The 64-layer weight stream of one decode step.  A model with 64 layers (16
+ * gated-attention, 48 Gated DeltaNet: wiselychen guide, section "Before
+ * deploying") reads every projection once per token; engines capture the
+ * decode step in a CUDA graph (wiselychen guide, section "RTX 5090 32GB",
+ * "SGLang/vLLM + NVFP4").  layer_stack_create captures the listed products, in
+ * order, once; layer_stack_run replays them on a stream.
+ * -------------------------------------------------------------------------*/
+typedef struct q4_stack_entry {
+  int bits;            /* 4 or 8 */
+  int64_t N, K;        /* weight shape */
+  const void* packed;  /* device, packed layout */
+  const uint16_t* x;   /* device, bf16 [M][K] */
+  float* y;            /* device, fp32 [M][N] */
+} q4_stack_entry;
+
+typedef struct q4_stack q4_stack;
+
+#define Q4_STACK_NO_PDL 1 /* launch without programmatic dependent launch (for comparison) */
+
+/* Validates every entry, allocates the library-owned workspace, and captures
+ * the n_entries products as one CUDA graph on the current device.  Each
+ * product is launched in order; with PDL each kernel prefetches its first
+ * weight tiles while its predecessor finishes, and reads x only after the
+ * predecessor has completed.  The caller's buffers must outlive the stack.
+ * Errors: as q4_gemv, plus CUDA for allocation or capture failures. */
+Q4_API int layer_stack_create(const q4_stack_entry* entries, int n_entries, int M, int flags, q4_stack** out);
+
+/* Replays the captured products on `stream` (one cudaGraphLaunch). */
+Q4_API int layer_stack_run(q4_stack* stack, void* stream);
+
+/* Synchronises `stream` and reports a bounded wait that gave up during the
+ * stack's runs since the last check (Q4_ERR_TIMEOUT), as q4_workspace_check. */
+Q4_API int layer_stack_check(q4_stack* stack, void* stream);
+
+/* Number of kernel launches one layer_stack_run makes. */
+Q4_API int layer_stack_launches(const q4_stack* stack);
+
+/* Frees the graph and the workspace.  NULL is ignored. */
+Q4_API void layer_stack_destroy(q4_stack* stack);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* Q4GEMV_H */

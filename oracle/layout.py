@@ -12,14 +12,14 @@ from __future__ import annotations
 
 import numpy as np
 
-ROWS = 16
+TILE_ROWS = 32
 
 
 def _geometry(bits: int, N: int, K: int):
     kc = 64 if bits == 4 else 32
-    T = -(-N // ROWS)
+    T = -(-N // TILE_ROWS)
     C = -(-K // kc)
-    CB = 576 if bits == 4 else 544
+    CB = 1152 if bits == 4 else 1088
     return T, C, CB
 
 
@@ -30,21 +30,22 @@ def decode(bits: int, packed: np.ndarray, N: int, K: int) -> tuple[np.ndarray, n
     assert packed.size >= T * C * CB
     n = np.arange(N, dtype=np.int64)[:, None]
     k = np.arange(K, dtype=np.int64)[None, :]
-    t = n // ROWS
-    rr = n % ROWS
+    t = n // TILE_ROWS
+    rr = n % TILE_ROWS
+    h = rr // 16          # which 16-row half of the tile
     gi = rr % 8
-    upper = rr // 8  # 1 for the row R + 8 of the slot
+    upper = (rr % 16) // 8  # 1 for the row R + 8 of the slot
     if bits == 4:
         c = k // 64
         kk = k % 64
-        h = kk // 32
+        G = kk // 32
         within = kk % 32
         ti = within // 8
         e = (within % 8) // 4
         r4 = within % 4  # = 2*((i>>1)&1) + (i>>2)
         i = 4 * (r4 % 2) + 2 * (r4 // 2) + upper
-        j = 2 * h + e
-        off = (t * C + c) * CB + 16 * (4 * gi + ti) + 4 * j
+        j = 2 * G + e
+        off = (t * C + c) * CB + 512 * h + 16 * (4 * gi + ti) + 4 * j
         word = _word(packed, off)
         u = (word >> (4 * i).astype(np.uint32)) & 0xF
         q = u.astype(np.int64) - 8
@@ -57,18 +58,19 @@ def decode(bits: int, packed: np.ndarray, N: int, K: int) -> tuple[np.ndarray, n
         f = r4 // 2
         b = 2 * (r4 % 2) + upper
         j = 2 * e + f
-        off = (t * C + c) * CB + 16 * (4 * gi + ti) + 4 * j
+        off = (t * C + c) * CB + 512 * h + 16 * (4 * gi + ti) + 4 * j
         word = _word(packed, off)
         u = (word >> (8 * b).astype(np.uint32)) & 0xFF
         q = u.astype(np.int64) - 128
-    G = K // 32
-    g = np.arange(G, dtype=np.int64)[None, :]
+    Gn = K // 32
+    g = np.arange(Gn, dtype=np.int64)[None, :]
     if bits == 4:
         cs = g // 2
-        half = 2 * upper + (g % 2)
-        soff = (t * C + cs) * CB + 512 + 8 * gi + 2 * half
+        slot = 4 * h + 2 * upper + (g % 2)
+        soff = (t * C + cs) * CB + 1024 + 16 * gi + 2 * slot
     else:
-        soff = (t * C + g) * CB + 512 + 4 * gi + 2 * upper
+        slot = 2 * h + upper
+        soff = (t * C + g) * CB + 1024 + 8 * gi + 2 * slot
     s = packed[soff].astype(np.uint16) | (packed[soff + 1].astype(np.uint16) << 8)
     return q, s
 
@@ -81,7 +83,7 @@ def _word(packed: np.ndarray, off: np.ndarray) -> np.ndarray:
 def padding_is_zero(bits: int, packed: np.ndarray, N: int, K: int) -> bool:
     """Rows >= N and groups >= K/32 of the padded tiles decode to q = 0, scale 0."""
     T, C, CB = _geometry(bits, N, K)
-    Np = T * ROWS
+    Np = T * TILE_ROWS
     Kp = C * (64 if bits == 4 else 32)
     q, s = decode(bits, packed, Np, Kp)
     return bool(np.all(q[N:, :] == 0) and np.all(q[:, K:] == 0) and np.all(s[N:, :] == 0) and np.all(s[:, K // 32:] == 0))

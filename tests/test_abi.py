@@ -1,0 +1,96 @@
+"""The C-ABI library loads, exports every declared symbol, and rejects bad
+arguments on the host before touching a device (no GPU needed)."""
+import os
+import re
+import subprocess
+
+import numpy as np
+import pytest
+
+import bit_weight_gemv_q4_b200 as q4
+from bit_weight_gemv_q4_b200 import build
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "q4gemv.h")
+
+
+def declared_symbols():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"Q4_API\s+[\w\s\*]+?\b(\w+)\s*\(", text)))
+
+
+def test_header_declarations_match_binding():
+    assert declared_symbols() == sorted(q4.EXPORTED)
+
+
+def test_every_declared_symbol_is_exported():
+    out = subprocess.run(["nm", "-D", "--defined-only", build.GEMV_LIB], stdout=subprocess.PIPE, text=True, check=True)
+    exported = {line.split()[-1] for line in out.stdout.splitlines() if line.strip()}
+    for name in declared_symbols():
+        assert name in exported, name
+        assert hasattr(q4.lib(), name)
+
+
+def test_only_declared_symbols_are_exported():
+    out = subprocess.run(["nm", "-D", "--defined-only", build.GEMV_LIB], stdout=subprocess.PIPE, text=True, check=True)
+    ours = {line.split()[-1] for line in out.stdout.splitlines() if " T " in line}
+    assert {s for s in ours if s.startswith(("q4_", "q8_", "layer_stack_"))} == set(declared_symbols())
+
+
+# Host-side validation happens before any CUDA call, so these run without a GPU.
+ALIGNED = 1 << 20  # a fake, 16-byte-aligned device address (never dereferenced)
+
+
+@pytest.mark.parametrize("fn", ["q4_gemv", "q8_gemv"])
+def test_argument_errors_are_detected_on_the_host(fn):
+    f = getattr(q4.lib(), fn)
+    ws = 1 << 20
+    # M outside 0..4
+    assert f(ALIGNED, 16, 64, ALIGNED, 5, ALIGNED, ALIGNED, ws, None) == q4.Q4_ERR_INVALID_ARG
+    assert f(ALIGNED, 16, 64, ALIGNED, -1, ALIGNED, ALIGNED, ws, None) == q4.Q4_ERR_INVALID_ARG
+    # K not a multiple of 32, negative sizes
+    assert f(ALIGNED, 16, 48, ALIGNED, 1, ALIGNED, ALIGNED, ws, None) == q4.Q4_ERR_SHAPE
+    assert f(ALIGNED, -16, 64, ALIGNED, 1, ALIGNED, ALIGNED, ws, None) == q4.Q4_ERR_SHAPE
+    # null pointers
+    assert f(None, 16, 64, ALIGNED, 1, ALIGNED, ALIGNED, ws, None) == q4.Q4_ERR_INVALID_ARG
+    assert f(ALIGNED, 16, 64, None, 1, ALIGNED, ALIGNED, ws, None) == q4.Q4_ERR_INVALID_ARG
+    assert f(ALIGNED, 16, 64, ALIGNED, 1, None, ALIGNED, ws, None) == q4.Q4_ERR_INVALID_ARG
+    assert f(ALIGNED, 16, 64, ALIGNED, 1, ALIGNED, None, ws, None) == q4.Q4_ERR_INVALID_ARG
+    # misaligned operands
+    assert f(ALIGNED + 8, 16, 64, ALIGNED, 1, ALIGNED, ALIGNED, ws, None) == q4.Q4_ERR_ALIGN
+    assert f(ALIGNED, 16, 64, ALIGNED + 2, 1, ALIGNED, ALIGNED, ws, None) == q4.Q4_ERR_ALIGN
+    assert f(ALIGNED, 16, 64, ALIGNED, 1, ALIGNED + 2, ALIGNED, ws, None) == q4.Q4_ERR_ALIGN
+    assert f(ALIGNED, 16, 64, ALIGNED, 1, ALIGNED, ALIGNED + 4, ws, None) == q4.Q4_ERR_ALIGN
+    assert q4.q4_last_error()
+    # empty problems are no-ops and touch nothing
+    assert f(None, 0, 64, None, 1, None, None, 0, None) == q4.Q4_OK
+    assert f(None, 16, 64, None, 0, None, None, 0, None) == q4.Q4_OK
+
+
+def test_stack_argument_errors():
+    lib = q4.lib()
+    import ctypes
+
+    h = ctypes.c_void_p(0)
+    assert lib.layer_stack_create(None, 1, 1, 0, ctypes.byref(h)) == q4.Q4_ERR_INVALID_ARG
+    arr = (q4.StackEntry * 1)()
+    assert lib.layer_stack_create(arr, 1, 0, 0, ctypes.byref(h)) == q4.Q4_ERR_INVALID_ARG
+    assert lib.layer_stack_create(arr, 1, 5, 0, ctypes.byref(h)) == q4.Q4_ERR_INVALID_ARG
+    assert lib.layer_stack_run(None, None) == q4.Q4_ERR_INVALID_ARG
+    lib.layer_stack_destroy(None)
+
+
+def test_without_a_device_gpu_calls_fail_loudly():
+    """No silent CPU fallback: on a host without a usable device the product
+    entry points return an error (there is nothing else they could do)."""
+    try:
+        import torch
+
+        if torch.cuda.is_available():
+            pytest.skip("a device is present")
+    except ImportError:
+        pass
+    rc = q4.lib().q4_gemv(ALIGNED, 16, 64, ALIGNED, 1, ALIGNED, ALIGNED, 1 << 20, None)
+    assert rc in (q4.Q4_ERR_CUDA, q4.Q4_ERR_UNSUPPORTED)
+    with pytest.raises(q4.Q4Error):
+        q4.q4_gemv_workspace_bytes(4, 16, 64, 1)
+    _ = np  # numpy imported for parity with other test modules

@@ -422,6 +422,76 @@ extern "C" Q4_API int q4_selftest_wait_timeout(uint64_t timeout_ns, int* status_
 }
 
 // ----------------------------------------------------------------------------
+// q4 product without a caller-provided workspace.  Some callers cannot
+// allocate device memory at the point where they run the product: code inside
+// an open stream capture (cudaMalloc is not a stream operation and is not
+// allowed while a global or thread-local capture is open), plug-ins that run
+// under a host application's memory budget or allocator they do not own, and
+// latency-critical loops that must not take the driver's allocation path.
+// For them the split-tile scratch lives in this file-scope device array
+// instead.  Every GPU that loads the library holds it until the process exits.
+// ----------------------------------------------------------------------------
+constexpr size_t kNoAllocWorkspaceBytes = size_t(4) << 20;  // 4 MiB per device
+static __device__ __align__(256) unsigned char g_noalloc_workspace[kNoAllocWorkspaceBytes];
+
+namespace {
+std::mutex g_noalloc_mutex;
+std::vector<void*> g_noalloc_ptr;  // device address of the array, per device
+
+// The array's name in host code is only a stand-in: its device address comes
+// from cudaGetSymbolAddress, once per device, with that device current.
+int noalloc_workspace(void** out) {
+  int dev = 0;
+  cudaError_t err = cudaGetDevice(&dev);
+  if (err != cudaSuccess) return cuda_fail(err, "q4_gemv_noalloc: cudaGetDevice");
+  std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+  if (static_cast<int>(g_noalloc_ptr.size()) <= dev) g_noalloc_ptr.resize(dev + 1, nullptr);
+  if (!g_noalloc_ptr[dev]) {
+    void* ptr = nullptr;
+    err = cudaGetSymbolAddress(&ptr, g_noalloc_workspace);
+    if (err != cudaSuccess) return cuda_fail(err, "q4_gemv_noalloc: cudaGetSymbolAddress");
+    g_noalloc_ptr[dev] = ptr;
+  }
+  *out = g_noalloc_ptr[dev];
+  return Q4_OK;
+}
+}  // namespace
+
+extern "C" Q4_API int q4_gemv_noalloc(const void* packed, int64_t N, int64_t K, const uint16_t* x, int M, float* y,
+                                      void* stream) {
+  const char* who = "q4_gemv_noalloc";
+  Shape s;
+  int rc = make_shape(4, N, K, &s, who);
+  if (rc) return rc;
+  if (M < 0 || M > 4) return fail(Q4_ERR_INVALID_ARG, "%s: M must be in 0..4 (got %d)", who, M);
+  if (N == 0 || M == 0 || K == 0)  // nothing to stage: same as q4_gemv
+    return gemv_entry(4, packed, N, K, x, M, y, nullptr, 0, stream, who);
+  DeviceInfo dev;
+  if ((rc = device_info(&dev))) return rc;
+  const size_t need = workspace_bytes(s, M, dev);
+  if (need > kNoAllocWorkspaceBytes)
+    return fail(Q4_ERR_UNSUPPORTED,
+                "%s: this shape needs %zu bytes of scratch, more than the %zu-byte static array "
+                "(at most %lld rows on this device); use q4_gemv with a workspace",
+                who, need, kNoAllocWorkspaceBytes,
+                static_cast<long long>((kNoAllocWorkspaceBytes - kWsHeader - partials_bytes(dev)) / 4 * 32));
+  void* ws = nullptr;
+  if ((rc = noalloc_workspace(&ws))) return rc;
+  Launch L;
+  if ((rc = prepare(4, packed, N, K, x, M, y, ws, kNoAllocWorkspaceBytes, who, &L))) return rc;
+  L.params.y = y;
+  // The array keeps whatever the last call left: clear the status word and
+  // this shape's tile counters, which must start at zero.
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  unsigned char* base = static_cast<unsigned char*>(ws);
+  cudaError_t err = cudaMemsetAsync(base, 0, kWsHeader, st);
+  if (err == cudaSuccess)
+    err = cudaMemsetAsync(base + kWsHeader + partials_bytes(dev), 0, static_cast<size_t>(s.T) * 4, st);
+  if (err != cudaSuccess) return cuda_fail(err, "q4_gemv_noalloc: cudaMemsetAsync");
+  return launch(L, st, true);
+}
+
+// ----------------------------------------------------------------------------
 // Layer stack: the ordered products of one decode step, captured once.
 // ----------------------------------------------------------------------------
 struct q4_stack {

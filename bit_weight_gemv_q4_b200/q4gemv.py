@@ -42,7 +42,7 @@ ERROR_NAMES = {
 EXPORTED = [
     "q4_last_error", "q4_packed_bytes", "q4_pack_weights", "q4_pack_weights_device", "q4_unpack_weights",
     "q4_gemv_workspace_bytes",
-    "q4_gemv", "q8_gemv", "q4_workspace_check", "q4_set_wait_timeout_ns", "q4_unpack_device",
+    "q4_gemv", "q8_gemv", "q4_gemv_noalloc", "q4_workspace_check", "q4_set_wait_timeout_ns", "q4_unpack_device",
     "q4_selftest_wait_timeout", "layer_stack_create", "layer_stack_run", "layer_stack_check",
     "layer_stack_launches", "layer_stack_destroy",
 ]
@@ -83,6 +83,7 @@ def _load() -> ctypes.CDLL:
         "q4_gemv_workspace_bytes": ([i32, i64, i64, i32], sz),
         "q4_gemv": ([vp, i64, i64, vp, i32, vp, vp, sz, vp], i32),
         "q8_gemv": ([vp, i64, i64, vp, i32, vp, vp, sz, vp], i32),
+        "q4_gemv_noalloc": ([vp, i64, i64, vp, i32, vp, vp], i32),
         "q4_workspace_check": ([vp, sz, vp], i32),
         "q4_set_wait_timeout_ns": ([u64], i32),
         "q4_unpack_device": ([i32, vp, i64, i64, vp, vp, vp], i32),
@@ -200,6 +201,12 @@ def q8_gemv(packed, N: int, K: int, x, M: int, y, workspace, stream=None) -> Non
     _gemv(_lib.q8_gemv, packed, N, K, x, M, y, workspace, stream)
 
 
+def q4_gemv_noalloc(packed, N: int, K: int, x, M: int, y, stream=None) -> None:
+    """q4_gemv with the library's static scratch array instead of a workspace
+    (for callers that cannot allocate device memory where they run)."""
+    _check(_lib.q4_gemv_noalloc(_dev_ptr(packed), N, K, _dev_ptr(x), M, _dev_ptr(y), _stream(stream)))
+
+
 def q4_workspace_check(workspace, stream=None) -> None:
     _check(_lib.q4_workspace_check(_dev_ptr(workspace), _nbytes(workspace), _stream(stream)))
 
@@ -271,6 +278,7 @@ def layer_stack_destroy(stack: LayerStack) -> None:
 __all__ = [
     "Q4Error", "LayerStack", "StackEntry", "EXPORTED", "lib", "q4_last_error", "q4_packed_bytes",
     "q4_pack_weights", "q4_pack_weights_device", "q4_unpack_weights", "q4_gemv_workspace_bytes", "q4_gemv", "q8_gemv",
+    "q4_gemv_noalloc",
     "q4_workspace_check", "q4_set_wait_timeout_ns", "q4_unpack_device", "q4_selftest_wait_timeout",
     "layer_stack_create", "layer_stack_run", "layer_stack_check", "layer_stack_destroy",
 ]

@@ -152,6 +152,26 @@ Q4_API int q4_gemv(const void* packed, int64_t N, int64_t K, const uint16_t* x, 
 Q4_API int q8_gemv(const void* packed, int64_t N, int64_t K, const uint16_t* x, int M, float* y, void* workspace,
                    size_t workspace_bytes, void* stream);
 
+/* q4_gemv for callers that cannot allocate device memory where they run the
+ * product: code inside an open stream capture (cudaMalloc is not allowed
+ * there), plug-ins that run under a host application's memory budget or
+ * allocator, and loops that must not take the driver's allocation path.  The
+ * pages describe no such entry point; it has no counterpart there.
+ * Same product, arguments and errors as q4_gemv, without the workspace: the
+ * split-tile scratch is a file-scope device array of 4 MiB that every GPU
+ * loading the library holds until the process exits.  Shapes whose scratch
+ * does not fit (more than about 14 million rows on a 148-SM device) are
+ * rejected with Q4_ERR_UNSUPPORTED.  Allocates and frees nothing.  The first
+ * call on a device looks up the array's device address
+ * (cudaGetSymbolAddress); make that first call before any stream capture.
+ * Each call clears the array's status word and counters with two
+ * asynchronous memsets on `stream` before its kernel.  All calls share the
+ * one array: calls that may overlap on the GPU (different streams without
+ * ordering between them) race and give undefined results.  A device wait that
+ * gives up is not reported by this entry point. */
+Q4_API int q4_gemv_noalloc(const void* packed, int64_t N, int64_t K, const uint16_t* x, int M, float* y,
+                           void* stream);
+
 /* Synchronises `stream`, then reads and clears the workspace's status word.
  * Returns Q4_OK, or Q4_ERR_TIMEOUT when a kernel that used this workspace gave
  * up a bounded wait since the last check (that call's y is then undefined);

@@ -53,7 +53,8 @@ def measured_peaks():
 
 def kernel_source_sha() -> str:
     h = hashlib.sha256()
-    for rel in ("bit_weight_gemv_q4_b200/csrc/q4gemv_kernels.cuh", "bit_weight_gemv_q4_b200/csrc/q4gemv.cu"):
+    for rel in ("bit_weight_gemv_q4_b200/csrc/q4gemv_kernels.cuh", "bit_weight_gemv_q4_b200/csrc/q4stack_kernel.cuh",
+                "bit_weight_gemv_q4_b200/csrc/q4gemv.cu"):
         with open(os.path.join(ROOT, rel), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
@@ -177,9 +178,11 @@ def oracle_sample_rate(target_s: float = 12.0, seed: int = 0):
             oracle.gemv(t.bits, q, s, x[t.K])
         return nbytes, time.perf_counter() - t0
 
-    nb, dt = run(2)
-    rows = max(2, min(4096, int(2 * target_s / max(dt, 1e-3))))
+    rows = 2
     nb, dt = run(rows)
+    while dt < 0.25 * target_s and rows < 4096:  # grow the sample until it takes about target_s
+        rows = min(4096, rows * max(2, int(target_s / max(dt, 1e-3) / 2)))
+        nb, dt = run(rows)
     desc = (f"{rows} whole rows (evenly strided) of each of the 257 tensors of the M=1 decode stream, "
             f"{nb / 1e6:.1f} MB of weights, fp64 oracle, {dt:.1f} s")
     return nb / dt / 1e9, oracle.threads(), desc, dt
@@ -262,7 +265,9 @@ def run_ours(args, d: Dist):
     tensors = workloads.decode_stream(fused=True)
     peak, peak_kind = measured_peaks()
 
-    st = workloads.DeviceStream(tensors, 1, seed=args.seed)
+    # the step: the 257 products of one decode token, independent (each reads
+    # its own activation block), as one persistent stream-mode launch
+    st = workloads.DeviceStream(tensors, 1, seed=args.seed, flags=q4.Q4_STACK_INDEPENDENT)
     n_launch = st.stack.launches()
     wbytes = st.weight_bytes
 
@@ -280,21 +285,25 @@ def run_ours(args, d: Dist):
     st.check()
     ms_step = d.max(ms / args.steps)
     value = wbytes * d.world / (ms_step * 1e6)  # GB/s over all ranks
+    launch_us = ms / args.steps / n_launch * 1e3  # this rank's own launches
+    achieved = wbytes / n_launch / (launch_us * 1e-6) / 1e9
 
-    # dominant kernel: the q4 instantiation (82% of the bytes), timed as the
-    # sequence of its launches in the stream (same buffers, own captured stack)
-    q4_idx = [i for i, t in enumerate(tensors) if t.bits == 4]
-    q4_entries = [(4, tensors[i].N, tensors[i].K, st.packed[i], st.x[tensors[i].K], st.y[i]) for i in q4_idx]
-    q4_stack = q4.layer_stack_create(q4_entries, 1)
-    q4_bytes = sum(tensors[i].bytes for i in q4_idx)
-    for _ in range(max(3, args.warmup)):
-        q4.layer_stack_run(q4_stack)
-    q4_steps = max(3, args.steps // 2)
-    ms_q4 = time_region(torch, lambda: q4.layer_stack_run(q4_stack), q4_steps, stream) / q4_steps
-    q4.layer_stack_check(q4_stack)
-    launch_us = ms_q4 * 1e3 / len(q4_idx)
-    achieved = q4_bytes / len(q4_idx) / (launch_us * 1e-6) / 1e9
-    q4_stack.close()
+    # the same products with an ordering between consecutive products (each
+    # product's outputs complete before the next reads its activations), as
+    # one ordered persistent launch and as a graph of one launch per product
+    other = {}
+    for flags, name in ((0, "ordered"), (q4.Q4_STACK_GRAPH, "graph")):
+        alt = st.make_stack(flags)
+        run_alt = lambda: q4.layer_stack_run(alt)  # noqa: E731
+        for _ in range(max(3, args.warmup // 2)):
+            run_alt()
+        n_alt = max(3, args.steps // 4)
+        ms_alt = d.max(time_region(torch, run_alt, n_alt, stream) / n_alt)
+        q4.layer_stack_check(alt)
+        other[name] = {"value": round(wbytes * d.world / (ms_alt * 1e6), 1), "ms_per_step": round(ms_alt, 5),
+                       "pct_of_hbm_peak": round(100 * wbytes / (ms_alt * 1e6) / peak, 2),
+                       "launches": alt.launches()}
+        alt.close()
 
     # e2e through the public API: activations from pinned host memory in,
     # the stack, the logits (head output) back to pinned host memory
@@ -320,7 +329,7 @@ def run_ours(args, d: Dist):
     torch.cuda.empty_cache()
 
     # M = 4: one verification pass of three drafted tokens plus one
-    st4 = workloads.DeviceStream(tensors, 4, seed=args.seed)
+    st4 = workloads.DeviceStream(tensors, 4, seed=args.seed, flags=q4.Q4_STACK_INDEPENDENT)
     for _ in range(args.warmup):
         st4.run()
     d.barrier()
@@ -356,6 +365,7 @@ def run_ours(args, d: Dist):
             "tensors": len(tensors),
             "weight_bytes_per_step": wbytes,
             "M": 1,
+            "mode": "stream (independent products, one persistent launch)",
             "parallelism": "replicas" if d.world > 1 else "single GPU",
             "l2": "inputs larger than L2 (13.7 GB of weights per step vs 126 MB L2); no flush",
         },
@@ -363,6 +373,8 @@ def run_ours(args, d: Dist):
         "hbm_peak_gbs": peak,
         "hbm_peak_kind": peak_kind,
         "tok_per_s": round(1000.0 / ms_step, 1),
+        "ordered": other["ordered"],
+        "graph": other["graph"],
         "m4": {
             "value": round(wbytes * d.world / (ms4 * 1e6), 1),
             "unit": UNIT,
@@ -372,15 +384,15 @@ def run_ours(args, d: Dist):
         },
         "roofline": {
             "bound": "hbm",
-            "kernel": "q4gemv gemv_kernel<4,1> (q4 products of the stream)",
+            "kernel": "stream_kernel<M=1> (the whole decode stream, one launch per step)",
             "achieved": round(achieved, 1),
             "peak": peak,
             "unit": "GB/s",
             "frac": round(achieved / peak, 4),
             "traffic": traffic,
-            "bytes_per_launch": q4_bytes // len(q4_idx),
+            "bytes_per_launch": wbytes // n_launch,
             "launch_us": round(launch_us, 3),
-            "launches": len(q4_idx),
+            "launches_per_step": n_launch,
             "peak_kind": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs, copy burst)" if peak_kind == "measured" else peak_kind,
         },
         "cpu_baseline": cpu,
@@ -453,12 +465,27 @@ def run_reference(args, d: Dist):
 
 
 def run_profile_case(args):
-    """A small single-product case for ncu: a q4 65536 x 5120 tensor (189 MB,
-    larger than L2), `--profile-launches` launches at M = args.m."""
+    """Small cases for ncu.  Default: a q4 (or q8) 65536 x 5120 tensor (189 MB,
+    larger than L2), `--profile-launches` launches at M = args.m.  With
+    --profile-layers L: the first L layers of the decode stream (about 0.2 GB
+    per layer) as one stream-mode stack launch."""
     import torch
 
+    import bit_weight_gemv_q4_b200 as q4
     from bit_weight_gemv_q4_b200 import workloads
 
+    if args.profile_layers > 0:
+        tensors = workloads.decode_stream(fused=True)[: 4 * args.profile_layers]
+        st = workloads.DeviceStream(tensors, args.m, seed=args.seed, flags=q4.Q4_STACK_INDEPENDENT)
+        for _ in range(args.profile_launches):
+            st.run()
+        torch.cuda.synchronize()
+        st.check()
+        print(json.dumps({"profile_case": f"stream of {args.profile_layers} layers", "products": len(tensors),
+                          "M": args.m, "launches": args.profile_launches, "weight_bytes": st.weight_bytes,
+                          "kernel_source_sha": kernel_source_sha()}))
+        st.close()
+        return
     t = workloads.Tensor("profile.q4", 4 if args.profile_bits == 4 else 8, 65536, 5120, 900)
     st = workloads.DeviceStream([t], args.m, seed=args.seed)
     for _ in range(args.profile_launches):
@@ -484,6 +511,7 @@ def main():
     ap.add_argument("--profile-case", action="store_true", help="run the small ncu case and exit")
     ap.add_argument("--profile-bits", type=int, default=4)
     ap.add_argument("--profile-launches", type=int, default=3)
+    ap.add_argument("--profile-layers", type=int, default=0)
     ap.add_argument("--m", type=int, default=1)
     args = ap.parse_args()
     if args.warmup < 3 and not args.profile_case:

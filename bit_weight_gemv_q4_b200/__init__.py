@@ -13,9 +13,14 @@ from __future__ import annotations
 import importlib
 
 
+_SUBMODULES = ("build", "q4gemv", "synth", "workloads")
+
+
 def __getattr__(name):
     if name.startswith("_"):
         raise AttributeError(name)
+    if name in _SUBMODULES:  # `from package import build` must not load the library first
+        return importlib.import_module(f".{name}", __name__)
     mod = importlib.import_module(".q4gemv", __name__)
     try:
         return getattr(mod, name)

@@ -14,6 +14,7 @@
 
 #include "q4gemv.h"
 #include "q4gemv_kernels.cuh"
+#include "q4stack_kernel.cuh"
 
 namespace q4 {
 
@@ -49,6 +50,14 @@ constexpr int kCtasPerSm = Q4_TUNE_CTAS_PER_SM;
 constexpr int kRingChunks = Q4_TUNE_RING_CHUNKS;
 constexpr int kMaxU = Q4_TUNE_MAX_U;
 static_assert(kRingChunks % 2 == 0 && kRingChunks >= 4, "ring must hold two stages of two chunks");
+#ifndef Q4_TUNE_STACK_D
+#define Q4_TUNE_STACK_D 2
+#endif
+#ifndef Q4_TUNE_STACK_PF
+#define Q4_TUNE_STACK_PF 0
+#endif
+constexpr int kStackD = Q4_TUNE_STACK_D;    // stages of 2 chunks per warp in the persistent stack kernel
+constexpr int kStackPF = Q4_TUNE_STACK_PF;  // further stages prefetched into L2
 // shared memory a CTA may use (B200: 227 KB per CTA)
 constexpr int kSmemLimit = 227 * 1024 / kCtasPerSm;
 constexpr size_t kWsHeader = 256;
@@ -124,6 +133,8 @@ int make_shape(int bits, int64_t N, int64_t K, Shape* s, const char* who) {
   const int kc = bits == 4 ? 64 : 32;
   s->C = static_cast<int>((K + kc - 1) / kc);
   s->TC = static_cast<long long>(s->T) * s->C;
+  // the kernels' range arithmetic needs (chunks x warps) below 2^52
+  if (s->TC >= (int64_t(1) << 38)) return fail(Q4_ERR_SHAPE, "%s: tensor too large", who);
   return Q4_OK;
 }
 
@@ -492,74 +503,173 @@ extern "C" Q4_API int q4_gemv_noalloc(const void* packed, int64_t N, int64_t K, 
 }
 
 // ----------------------------------------------------------------------------
-// Layer stack: the ordered products of one decode step, captured once.
+// Layer stack: the ordered products of one decode step.
 // ----------------------------------------------------------------------------
 struct q4_stack {
+  // graph mode: one kernel per product, captured once
   cudaGraph_t graph = nullptr;
   cudaGraphExec_t exec = nullptr;
+  // persistent mode: one cooperative kernel over the whole list
+  bool persistent = false;
+  q4k::StackEntryDev* entries_dev = nullptr;
+  void* fn = nullptr;
+  int grid = 0, block = 0, smem = 0;
+  q4k::StackParams params{};
   void* workspace = nullptr;
   size_t workspace_bytes = 0;
   int launches = 0;
   int device = 0;
 };
 
-extern "C" Q4_API int layer_stack_create(const q4_stack_entry* entries, int n_entries, int M, int flags,
-                                         q4_stack** out) {
-  if (!out) return fail(Q4_ERR_INVALID_ARG, "layer_stack_create: out is null");
-  *out = nullptr;
-  if (n_entries < 0 || (n_entries > 0 && !entries))
-    return fail(Q4_ERR_INVALID_ARG, "layer_stack_create: bad entry list");
-  if (M < 1 || M > 4) return fail(Q4_ERR_INVALID_ARG, "layer_stack_create: M must be in 1..4");
-  DeviceInfo dev;
-  int rc = device_info(&dev);
-  if (rc) return rc;
-  // workspace sized for the largest entry; all entries run in stream order
-  size_t ws = kWsHeader;
-  for (int i = 0; i < n_entries; ++i) {
+namespace {
+
+template <int M>
+void* stack_kernel_ptr() {
+  return reinterpret_cast<void*>(&q4k::stack_kernel<M, kNW, kStackD, kStackPF>);
+}
+
+template <int M>
+void* stream_kernel_ptr() {
+  return reinterpret_cast<void*>(&q4k::stream_kernel<M, kNW, kStackD, kStackPF>);
+}
+
+void* select_stack_kernel(int M, bool independent) {
+  static void* const table[2][4] = {
+      {stack_kernel_ptr<1>(), stack_kernel_ptr<2>(), stack_kernel_ptr<3>(), stack_kernel_ptr<4>()},
+      {stream_kernel_ptr<1>(), stream_kernel_ptr<2>(), stream_kernel_ptr<3>(), stream_kernel_ptr<4>()}};
+  return table[independent ? 1 : 0][M - 1];
+}
+
+int stack_smem_bytes() { return kNW * kStackD * q4k::kStackSlotBytes + kNW * kStackD * 8; }
+
+void free_stack(q4_stack* st) {
+  if (st->exec) cudaGraphExecDestroy(st->exec);
+  if (st->graph) cudaGraphDestroy(st->graph);
+  if (st->entries_dev) cudaFree(st->entries_dev);
+  if (st->workspace) cudaFree(st->workspace);
+  delete st;
+}
+
+// Persistent mode: every product non-empty, with an even number of chunks per
+// tile (stages of two chunks).
+bool stack_eligible(const q4_stack_entry* entries, int n) {
+  if (n <= 0) return false;
+  for (int i = 0; i < n; ++i) {
     Shape s;
-    char who[64];
-    snprintf(who, sizeof(who), "layer_stack_create entry %d", i);
-    if ((rc = make_shape(entries[i].bits, entries[i].N, entries[i].K, &s, who))) return rc;
-    const size_t need = workspace_bytes(s, M, dev);
-    if (need > ws) ws = need;
+    if (make_shape(entries[i].bits, entries[i].N, entries[i].K, &s, "layer_stack_create")) return false;
+    if (s.N == 0 || s.K == 0 || s.C % 2 != 0) return false;
   }
-  q4_stack* st = new q4_stack();
-  cudaGetDevice(&st->device);
-  cudaError_t err = cudaMalloc(&st->workspace, ws);
-  if (err != cudaSuccess) {
-    delete st;
-    return cuda_fail(err, "layer_stack_create: cudaMalloc(workspace)");
-  }
-  st->workspace_bytes = ws;
-  err = cudaMemset(st->workspace, 0, ws);
-  std::vector<Launch> launches(static_cast<size_t>(n_entries));
-  for (int i = 0; i < n_entries && err == cudaSuccess; ++i) {
+  return true;
+}
+
+int create_persistent(const q4_stack_entry* entries, int n, int M, bool independent, const DeviceInfo& dev,
+                      q4_stack* st) {
+  long long max_t = 1, total_blocks = 0, total_tiles = 0;
+  std::vector<q4k::StackEntryDev> host(static_cast<size_t>(n));
+  const long long warps = static_cast<long long>(dev.sms) * kNW;
+  for (int i = 0; i < n; ++i) {
     const q4_stack_entry& en = entries[i];
     char who[64];
     snprintf(who, sizeof(who), "layer_stack_create entry %d", i);
-    rc = prepare(en.bits, en.packed, en.N, en.K, en.x, M, en.y, st->workspace, ws, who, &launches[i]);
-    if (rc) {
-      cudaFree(st->workspace);
-      delete st;
-      return rc;
-    }
-    launches[i].params.y = en.y;
+    Shape s;
+    int rc = make_shape(en.bits, en.N, en.K, &s, who);
+    if (rc) return rc;
+    if (!en.packed || !en.x || !en.y) return fail(Q4_ERR_INVALID_ARG, "%s: null device pointer", who);
+    if (reinterpret_cast<uintptr_t>(en.packed) % 16 || reinterpret_cast<uintptr_t>(en.x) % 16 ||
+        reinterpret_cast<uintptr_t>(en.y) % 4)
+      return fail(Q4_ERR_ALIGN, "%s: packed and x must be 16-byte aligned, y 4-byte aligned", who);
+    long long P = warps;
+    if (P > s.TC / q4k::kStackU) P = s.TC / q4k::kStackU;
+    q4k::StackEntryDev& d = host[static_cast<size_t>(i)];
+    d.packed = static_cast<const uint8_t*>(en.packed);
+    d.x = en.x;
+    d.y = en.y;
+    d.N = s.N;
+    d.K = s.K;
+    d.TC = s.TC;
+    d.T = s.T;
+    d.C = s.C;
+    d.bits = en.bits;
+    d.P = static_cast<int>(P);
+    d.khalf = (en.bits == 4 && s.K % 64 == 32) ? 1 : 0;
+    d.blk_off = total_blocks;
+    d.tile_off = static_cast<int>(total_tiles);
+    total_blocks += s.TC / q4k::kStackU;
+    total_tiles += s.T;
+    if (s.T > max_t) max_t = s.T;
   }
-  if (err != cudaSuccess) {
-    cudaFree(st->workspace);
-    delete st;
-    return cuda_fail(err, "layer_stack_create: cudaMemset(workspace)");
+  if (total_tiles >= (1LL << 31)) return fail(Q4_ERR_SHAPE, "layer_stack_create: too many tiles");
+  // ordered mode re-uses one counter per tile of the largest product; stream
+  // mode keeps one per tile of every product
+  const size_t counters = (static_cast<size_t>(independent ? total_tiles : max_t) * 4 + 255) / 256 * 256;
+  st->workspace_bytes = kWsHeader + partials_bytes(dev) + counters;
+  cudaError_t err = cudaMalloc(&st->workspace, st->workspace_bytes);
+  if (err == cudaSuccess) err = cudaMemset(st->workspace, 0, st->workspace_bytes);
+  if (err == cudaSuccess) err = cudaMalloc(&st->entries_dev, sizeof(q4k::StackEntryDev) * host.size());
+  if (err == cudaSuccess)
+    err = cudaMemcpy(st->entries_dev, host.data(), sizeof(q4k::StackEntryDev) * host.size(), cudaMemcpyHostToDevice);
+  if (err != cudaSuccess) return cuda_fail(err, "layer_stack_create: allocation");
+  st->fn = select_stack_kernel(M, independent);
+  st->smem = stack_smem_bytes();
+  st->block = kNW * 32;
+  st->grid = dev.sms;
+  err = cudaFuncSetAttribute(st->fn, cudaFuncAttributeMaxDynamicSharedMemorySize, st->smem);
+  if (err != cudaSuccess) return cuda_fail(err, "layer_stack_create: cudaFuncSetAttribute");
+  int per_sm = 0;
+  err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, st->fn, st->block, st->smem);
+  if (err != cudaSuccess) return cuda_fail(err, "layer_stack_create: occupancy query");
+  if (per_sm < 1) return fail(Q4_ERR_UNSUPPORTED, "layer_stack_create: the stack kernel does not fit on an SM");
+  unsigned char* ws = static_cast<unsigned char*>(st->workspace);
+  q4k::StackParams& p = st->params;
+  p.entries = st->entries_dev;
+  p.E = n;
+  p.status = reinterpret_cast<unsigned*>(ws);
+  p.grid_bar = reinterpret_cast<unsigned*>(ws + 16);
+  p.partials = reinterpret_cast<float*>(ws + kWsHeader);
+  p.counters = reinterpret_cast<unsigned*>(ws + kWsHeader + partials_bytes(dev));
+  p.G = st->grid;
+  p.timeout_ns = g_timeout_ns.load();
+  p.TBg = total_blocks;
+  p.Pg = static_cast<int>(total_blocks < warps ? total_blocks : warps);
+  st->persistent = true;
+  st->launches = 1;
+  return Q4_OK;
+}
+
+int create_graph(const q4_stack_entry* entries, int n, int M, int flags, const DeviceInfo& dev, q4_stack* st) {
+  size_t ws = kWsHeader;
+  for (int i = 0; i < n; ++i) {
+    Shape s;
+    char who[64];
+    snprintf(who, sizeof(who), "layer_stack_create entry %d", i);
+    int rc = make_shape(entries[i].bits, entries[i].N, entries[i].K, &s, who);
+    if (rc) return rc;
+    const size_t need = workspace_bytes(s, M, dev);
+    if (need > ws) ws = need;
+  }
+  cudaError_t err = cudaMalloc(&st->workspace, ws);
+  if (err != cudaSuccess) return cuda_fail(err, "layer_stack_create: cudaMalloc(workspace)");
+  st->workspace_bytes = ws;
+  err = cudaMemset(st->workspace, 0, ws);
+  if (err != cudaSuccess) return cuda_fail(err, "layer_stack_create: cudaMemset(workspace)");
+  std::vector<Launch> launches(static_cast<size_t>(n));
+  for (int i = 0; i < n; ++i) {
+    const q4_stack_entry& en = entries[i];
+    char who[64];
+    snprintf(who, sizeof(who), "layer_stack_create entry %d", i);
+    int rc = prepare(en.bits, en.packed, en.N, en.K, en.x, M, en.y, st->workspace, ws, who, &launches[i]);
+    if (rc) return rc;
+    launches[i].params.y = en.y;
   }
   cudaStream_t cs = nullptr;
   err = cudaStreamCreateWithFlags(&cs, cudaStreamNonBlocking);
   if (err == cudaSuccess) err = cudaStreamBeginCapture(cs, cudaStreamCaptureModeThreadLocal);
   if (err != cudaSuccess) {
     if (cs) cudaStreamDestroy(cs);
-    cudaFree(st->workspace);
-    delete st;
     return cuda_fail(err, "layer_stack_create: begin capture");
   }
   const bool pdl = (flags & Q4_STACK_NO_PDL) == 0;
+  int rc = Q4_OK;
   for (auto& L : launches) {
     if (L.noop) continue;
     rc = launch(L, cs, pdl);
@@ -571,25 +681,63 @@ extern "C" Q4_API int layer_stack_create(const q4_stack_entry* entries, int n_en
   cudaStreamDestroy(cs);
   if (rc || end_err != cudaSuccess) {
     if (graph) cudaGraphDestroy(graph);
-    cudaFree(st->workspace);
-    delete st;
     return rc ? rc : cuda_fail(end_err, "layer_stack_create: end capture");
   }
   st->graph = graph;
   err = cudaGraphInstantiate(&st->exec, graph, 0);
-  if (err != cudaSuccess) {
-    cudaGraphDestroy(graph);
-    cudaFree(st->workspace);
-    delete st;
-    return cuda_fail(err, "layer_stack_create: cudaGraphInstantiate");
+  if (err != cudaSuccess) return cuda_fail(err, "layer_stack_create: cudaGraphInstantiate");
+  return Q4_OK;
+}
+
+}  // namespace
+
+extern "C" Q4_API int layer_stack_create(const q4_stack_entry* entries, int n_entries, int M, int flags,
+                                         q4_stack** out) {
+  if (!out) return fail(Q4_ERR_INVALID_ARG, "layer_stack_create: out is null");
+  *out = nullptr;
+  if (n_entries < 0 || (n_entries > 0 && !entries))
+    return fail(Q4_ERR_INVALID_ARG, "layer_stack_create: bad entry list");
+  if (M < 1 || M > 4) return fail(Q4_ERR_INVALID_ARG, "layer_stack_create: M must be in 1..4");
+  DeviceInfo dev;
+  int rc = device_info(&dev);
+  if (rc) return rc;
+  q4_stack* st = new q4_stack();
+  cudaGetDevice(&st->device);
+  const bool graph = (flags & (Q4_STACK_GRAPH | Q4_STACK_NO_PDL)) != 0 || !stack_eligible(entries, n_entries);
+  // stream mode also needs whole q4 chunks (K a multiple of 64); else ordered
+  bool independent = (flags & Q4_STACK_INDEPENDENT) != 0;
+  for (int i = 0; independent && i < n_entries; ++i)
+    if (entries[i].bits == 4 && entries[i].K % 64 != 0) independent = false;
+  rc = graph ? create_graph(entries, n_entries, M, flags, dev, st)
+             : create_persistent(entries, n_entries, M, independent, dev, st);
+  if (rc) {
+    free_stack(st);
+    return rc;
   }
   *out = st;
   return Q4_OK;
 }
 
 extern "C" Q4_API int layer_stack_run(q4_stack* st, void* stream) {
-  if (!st || !st->exec) return fail(Q4_ERR_INVALID_ARG, "layer_stack_run: null stack");
-  cudaError_t err = cudaGraphLaunch(st->exec, static_cast<cudaStream_t>(stream));
+  if (!st) return fail(Q4_ERR_INVALID_ARG, "layer_stack_run: null stack");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (st->persistent) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(st->grid);
+    cfg.blockDim = dim3(st->block);
+    cfg.dynamicSmemBytes = static_cast<size_t>(st->smem);
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeCooperative;  // all CTAs resident, or the launch fails
+    attr[0].val.cooperative = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    void* args[] = {&st->params};
+    cudaError_t err = cudaLaunchKernelExC(&cfg, st->fn, args);
+    return err == cudaSuccess ? Q4_OK : cuda_fail(err, "layer_stack_run: cooperative launch");
+  }
+  if (!st->exec) return Q4_OK;  // nothing to run
+  cudaError_t err = cudaGraphLaunch(st->exec, s);
   return err == cudaSuccess ? Q4_OK : cuda_fail(err, "cudaGraphLaunch");
 }
 
@@ -602,8 +750,5 @@ extern "C" Q4_API int layer_stack_launches(const q4_stack* st) { return st ? st-
 
 extern "C" Q4_API void layer_stack_destroy(q4_stack* st) {
   if (!st) return;
-  if (st->exec) cudaGraphExecDestroy(st->exec);
-  if (st->graph) cudaGraphDestroy(st->graph);
-  if (st->workspace) cudaFree(st->workspace);
-  delete st;
+  free_stack(st);
 }

@@ -118,26 +118,23 @@ __device__ __forceinline__ unsigned long long global_timer_ns() {
   return t;
 }
 
-// Polls until the phase with the given parity completes or timeout_ns passes.
+// Polls, warp-uniformly, until the phase with the given parity completes or
+// timeout_ns passes (lane 0's clock decides, so every lane leaves together).
 __device__ __noinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity, unsigned long long timeout_ns) {
   const unsigned long long t0 = global_timer_ns();
-  bool ok;
-  while (!(ok = mbar_try_wait(bar, parity))) {
-    if (global_timer_ns() - t0 > timeout_ns) break;
+  while (true) {
+    if (__all_sync(0xFFFFFFFFu, mbar_try_wait(bar, parity))) return true;
+    const unsigned long long waited = __shfl_sync(0xFFFFFFFFu, global_timer_ns() - t0, 0);
+    if (waited > timeout_ns) return false;
   }
-  return ok;
 }
 
 // Waits for the phase with the given parity to complete, for at most
 // timeout_ns.  Returns false when the limit was reached.  Every lane of the
-// warp calls it; the result is uniform across the warp.
+// warp calls it; control flow and result are uniform across the warp.
 __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity, unsigned long long timeout_ns) {
-  bool ok = mbar_try_wait(bar, parity);
-  if (!__all_sync(0xFFFFFFFFu, ok)) {
-    if (!ok) ok = mbar_wait_slow(bar, parity, timeout_ns);
-    ok = __all_sync(0xFFFFFFFFu, ok);
-  }
-  return ok;
+  if (__all_sync(0xFFFFFFFFu, mbar_try_wait(bar, parity))) return true;
+  return mbar_wait_slow(bar, parity, timeout_ns);
 }
 
 __device__ __forceinline__ uint64_t l2_evict_first_policy() {
@@ -153,6 +150,19 @@ __device__ __forceinline__ void bulk_copy_g2s(uint32_t dst, const void* src, uin
       "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1], %2, [%3], %4;" ::
           "r"(dst),
       "l"(src), "r"(bytes), "r"(bar), "l"(policy)
+      : "memory");
+}
+
+// Lane 0 (pred) arms `bar` for `bytes` and starts the bulk copy; every lane
+// executes this one predicated block, so the warp does not branch.
+__device__ __forceinline__ void bulk_copy_g2s_if(bool pred, uint32_t dst, const void* src, uint32_t bytes,
+                                                 uint32_t bar, uint64_t policy) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %5, 0;\n\t"
+      "@p mbarrier.arrive.expect_tx.shared::cta.b64 _, [%3], %2;\n\t"
+      "@p cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1], %2, [%3], %4;"
+      "\n\t}" ::"r"(dst),
+      "l"(src), "r"(bytes), "r"(bar), "l"(policy), "r"(static_cast<int>(pred))
       : "memory");
 }
 
@@ -310,16 +320,51 @@ __device__ __forceinline__ void q8_chunk_mac(float (&acc)[2][4], const ChunkRegs
 
 // The flat sequence of TB blocks (U chunks each) is cut into P ranges,
 // range p = [floor(p*TB/P), floor((p+1)*TB/P)); P <= TB, so none is empty.
-// owner_of(i) is the range holding block i: the largest p with begin <= i.
+// owner_of(i) is the range holding block i: the largest p with begin <= i,
+// i.e. floor(((i+1)*P - 1) / TB).
+// Both floors are computed in double precision, which is exact here: the
+// numerators are integers below 2^52 (the host keeps TB*P below 2^52), and a
+// non-integer quotient lies at least 1/denominator from the next integer,
+// far more than the quotient's rounding error.  (64-bit integer division has
+// no hardware instruction and costs a long software sequence.)
+__device__ __forceinline__ long long floor_div(long long num, long long den) {
+  return static_cast<long long>(floor(static_cast<double>(num) / static_cast<double>(den)));
+}
 __device__ __forceinline__ int owner_of(long long i, long long TB, int P) {
-  return static_cast<int>(((i + 1) * P - 1) / TB);
+  return static_cast<int>(floor_div((i + 1) * P - 1, TB));
 }
 __device__ __forceinline__ long long range_begin(int p, long long TB, int P) {
-  return static_cast<long long>(p) * TB / P;
+  return floor_div(static_cast<long long>(p) * TB, P);
 }
 
+// ----------------------------------------------------------------------------
+// Finishing tiles.  A tile covered entirely by one warp's range is stored
+// directly.  A tile split between warps (at most two per warp: the one its
+// range starts in and the one it ends in) is finished after the warp's last
+// chunk: the warp writes its partial sums to its slot (0: the tile holding
+// its first chunk, 1: otherwise), then arrives on the tile's counter; the last
+// arrival adds every contributor's partial in warp order (one row per lane,
+// independent loads) and writes y.
+// ----------------------------------------------------------------------------
+// How a product's flat sequence of blocks (U chunks each) is cut among warps.
+struct Partition {
+  long long TB;        // blocks in the partitioned sequence
+  int P;               // warps with work
+  float* partials;     // [P][2][M][32]
+};
+
+// A tile split between warps: its output rows, its arrival counter, and its
+// blocks [blo, bhi) in the partitioned sequence.
+struct SplitTile {
+  float* y;
+  long long N;
+  int r;
+  unsigned* counter;
+  long long blo, bhi;
+};
+
 template <int M>
-__device__ __forceinline__ void store_tile(const GemvParams& p, int r, const float (&v)[2][4], int lane) {
+__device__ __forceinline__ void store_tile(float* y, long long N, int r, const float (&v)[2][4], int lane) {
   const int gi = lane >> 2, ti = lane & 3;
   const int m0 = 2 * ti, m1 = 2 * ti + 1;
 #pragma unroll
@@ -327,32 +372,21 @@ __device__ __forceinline__ void store_tile(const GemvParams& p, int r, const flo
     const long long row0 = static_cast<long long>(r) * kTileRows + 16 * h + gi;
     const long long row1 = row0 + 8;
     if (m0 < M) {
-      if (row0 < p.N) p.y[m0 * p.N + row0] = v[h][0];
-      if (row1 < p.N) p.y[m0 * p.N + row1] = v[h][2];
+      if (row0 < N) y[m0 * N + row0] = v[h][0];
+      if (row1 < N) y[m0 * N + row1] = v[h][2];
     }
     if (m1 < M) {
-      if (row0 < p.N) p.y[m1 * p.N + row0] = v[h][1];
-      if (row1 < p.N) p.y[m1 * p.N + row1] = v[h][3];
+      if (row0 < N) y[m1 * N + row0] = v[h][1];
+      if (row1 < N) y[m1 * N + row1] = v[h][3];
     }
   }
 }
 
-// Writes a finished tile's sums, or hands a split tile's partial sums to the
-// deterministic fix-up.
-template <int M, int U>
-__device__ __forceinline__ void finish_tile(const GemvParams& p, int pw, long long b, long long e, int r,
-                                         const float (&acc)[2][4], int lane) {
+template <int M>
+__device__ __forceinline__ void write_partial(float* partials, int pw, int slot, const float (&acc)[2][4], int lane) {
   const int gi = lane >> 2, ti = lane & 3;
   const int m0 = 2 * ti, m1 = 2 * ti + 1;
-  const long long tile_lo = static_cast<long long>(r) * p.C;
-  const long long tile_hi = tile_lo + p.C;
-  if (tile_lo >= b && tile_hi <= e) {
-    store_tile<M>(p, r, acc, lane);
-    return;
-  }
-  // split tile: this warp's partial goes to slot 0 (its first tile) or 1
-  const int slot = (tile_lo <= b) ? 0 : 1;
-  float* mine = p.partials + (static_cast<long long>(pw) * 2 + slot) * (M * kTileRows);
+  float* mine = partials + (static_cast<long long>(pw) * 2 + slot) * (M * kTileRows);
 #pragma unroll
   for (int h = 0; h < 2; ++h) {
     const int row0 = 16 * h + gi, row1 = row0 + 8;
@@ -365,36 +399,61 @@ __device__ __forceinline__ void finish_tile(const GemvParams& p, int pw, long lo
       mine[m1 * kTileRows + row1] = acc[h][3];
     }
   }
+}
+
+__device__ __forceinline__ unsigned tile_contributors(const Partition& pt, const SplitTile& st) {
+  return static_cast<unsigned>(owner_of(st.bhi - 1, pt.TB, pt.P) - owner_of(st.blo, pt.TB, pt.P) + 1);
+}
+
+// Last arrival on a split tile: sum the partials of its contributing warps in
+// warp order (one row per lane) and store the tile; then re-zero its counter.
+template <int M>
+__device__ __forceinline__ void reduce_tile(const Partition& pt, const SplitTile& st, int lane) {
+  const int p_lo = owner_of(st.blo, pt.TB, pt.P);
+  const int p_hi = owner_of(st.bhi - 1, pt.TB, pt.P);
+  const long long row = static_cast<long long>(st.r) * kTileRows + lane;
+  // Warp p_lo's range begins at or before the tile: the tile is its first
+  // (slot 0) only if it begins exactly at blo.  Every later contributor
+  // begins inside the tile, so the tile is its first: slot 0.
+  const int slot_lo = (range_begin(p_lo, pt.TB, pt.P) == st.blo) ? 0 : 1;
+  const float* base = pt.partials + lane;
+#pragma unroll
+  for (int m = 0; m < M; ++m) {
+    float sum = __ldcg(base + (static_cast<long long>(p_lo) * 2 + slot_lo) * (M * kTileRows) + m * kTileRows);
+#pragma unroll 4
+    for (int q = p_lo + 1; q <= p_hi; ++q)
+      sum += __ldcg(base + (static_cast<long long>(q) * 2) * (M * kTileRows) + m * kTileRows);
+    if (row < st.N) st.y[m * st.N + row] = sum;
+  }
+  if (lane == 0) *st.counter = 0u;
+}
+
+// Finishes the (at most two) split tiles of warp pw after its last chunk:
+// `first` (partial kept in acc_first, slot 0) is the tile holding the range's
+// first block when that tile began in an earlier warp's range; `last`
+// (acc_last, slot_last) is the tile holding the range's last block when the
+// range ends inside it.  Absent tiles have r < 0.
+template <int M>
+__device__ __forceinline__ void finish_split_tiles(const Partition& pt, int pw, const SplitTile& first,
+                                                   const float (&acc_first)[2][4], const SplitTile& last,
+                                                   int slot_last, const float (&acc_last)[2][4], int lane) {
+  if (first.r < 0 && last.r < 0) return;
+  if (first.r >= 0) write_partial<M>(pt.partials, pw, 0, acc_first, lane);
+  if (last.r >= 0) write_partial<M>(pt.partials, pw, slot_last, acc_last, lane);
   __threadfence();
   __syncwarp();
-  unsigned arrived = 0;
-  if (lane == 0) arrived = atomicAdd(p.counters + r, 1u);
-  arrived = __shfl_sync(0xFFFFFFFFu, arrived, 0);
-  const long long TB = p.TC / U;
-  const int p_lo = owner_of(tile_lo / U, TB, p.P);
-  const int p_hi = owner_of(tile_hi / U - 1, TB, p.P);
-  if (arrived != static_cast<unsigned>(p_hi - p_lo)) return;
-  // last arrival: add the partial sums in fixed warp order
-  __threadfence();
-  float s[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-  for (int q = p_lo; q <= p_hi; ++q) {
-    const int qslot = (tile_lo <= range_begin(q, TB, p.P) * U) ? 0 : 1;
-    const float* part = p.partials + (static_cast<long long>(q) * 2 + qslot) * (M * kTileRows);
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      const int row0 = 16 * h + gi, row1 = row0 + 8;
-      if (m0 < M) {
-        s[h][0] += __ldcg(part + m0 * kTileRows + row0);
-        s[h][2] += __ldcg(part + m0 * kTileRows + row1);
-      }
-      if (m1 < M) {
-        s[h][1] += __ldcg(part + m1 * kTileRows + row0);
-        s[h][3] += __ldcg(part + m1 * kTileRows + row1);
-      }
-    }
+  unsigned a_first = 0, a_last = 0;
+  if (lane == 0) {
+    if (first.r >= 0) a_first = atomicAdd(first.counter, 1u);
+    if (last.r >= 0) a_last = atomicAdd(last.counter, 1u);
   }
-  store_tile<M>(p, r, s, lane);
-  if (lane == 0) p.counters[r] = 0u;
+  a_first = __shfl_sync(0xFFFFFFFFu, a_first, 0);
+  a_last = __shfl_sync(0xFFFFFFFFu, a_last, 0);
+  const bool red_first = first.r >= 0 && a_first + 1 == tile_contributors(pt, first);
+  const bool red_last = last.r >= 0 && a_last + 1 == tile_contributors(pt, last);
+  if (red_first || red_last) __threadfence();
+  if (red_first) reduce_tile<M>(pt, first, lane);
+  if (red_last) reduce_tile<M>(pt, last, lane);
 }
 
 // ----------------------------------------------------------------------------
@@ -490,13 +549,15 @@ __global__ void __launch_bounds__(NW * 32, 1) gemv_kernel(const GemvParams p) {
     }
   }
 
-  int r = static_cast<int>(b / p.C);
+  int r = static_cast<int>(floor_div(b, p.C));
   int c = static_cast<int>(b - static_cast<long long>(r) * p.C);
   const bool x_lane = gi < M;
   // shared-memory activations: lanes whose column is not a token read row 0
   const uint32_t xs_lane = xsm + (x_lane ? gi : 0) * xstride + 16 * ti;
   const uint16_t* xrow = p.x + static_cast<long long>(x_lane ? gi : 0) * p.K + 8 * ti;
   float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+  float acc_first[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+  int r_first = -1;  // split first tile, finished after the last chunk
   uint4 xa = make_uint4(0, 0, 0, 0), xb = make_uint4(0, 0, 0, 0);
 
   bool ok = true;
@@ -526,11 +587,8 @@ __global__ void __launch_bounds__(NW * 32, 1) gemv_kernel(const GemvParams p) {
     // release would give a separate consumer); lane 0 refills the slot.
     __syncwarp();
     if (i + D < nst) {
-      if (lane == 0) {
-        mbar_arrive_expect_tx(bars + 8 * slot, Cfg::kStageBytes);
-        bulk_copy_g2s(stage, src + static_cast<long long>(i + D) * Cfg::kStageBytes, Cfg::kStageBytes,
-                      bars + 8 * slot, policy);
-      }
+      bulk_copy_g2s_if(lane == 0, stage, src + static_cast<long long>(i + D) * Cfg::kStageBytes, Cfg::kStageBytes,
+                       bars + 8 * slot, policy);
       issued = i + D + 1;
     }
 #pragma unroll
@@ -556,7 +614,16 @@ __global__ void __launch_bounds__(NW * 32, 1) gemv_kernel(const GemvParams p) {
     }
     c += U;
     if (c == p.C) {
-      finish_tile<M, U>(p, pw, b, e, r, acc, lane);
+      const long long tile_lo = static_cast<long long>(r) * p.C;
+      if (tile_lo < b) {  // the first tile began in an earlier warp's range
+        r_first = r;
+#pragma unroll
+        for (int h = 0; h < 2; ++h)
+#pragma unroll
+          for (int q = 0; q < 4; ++q) acc_first[h][q] = acc[h][q];
+      } else {
+        store_tile<M>(p.y, p.N, r, acc, lane);
+      }
       ++r;
       c = 0;
 #pragma unroll
@@ -576,7 +643,21 @@ __global__ void __launch_bounds__(NW * 32, 1) gemv_kernel(const GemvParams p) {
     if (XS) (void)mbar_wait_bounded(xbar, 0, p.timeout_ns);
     return;
   }
-  if (nst > 0 && c != 0) finish_tile<M, U>(p, pw, b, e, r, acc, lane);
+  if (nst == 0) return;
+  // the range may end inside a tile: that tile's partial goes to slot 0 when
+  // it is also the tile the range began in, else to slot 1
+  int r_last = -1, slot_last = 1;
+  if (c != 0) {
+    r_last = r;
+    slot_last = (static_cast<long long>(r) * p.C <= b) ? 0 : 1;
+  }
+  const Partition pt{TB, p.P, p.partials};
+  const int bpt = p.C / U;  // blocks per tile
+  const SplitTile first{p.y, p.N, r_first, p.counters + (r_first < 0 ? 0 : r_first),
+                        static_cast<long long>(r_first) * bpt, static_cast<long long>(r_first + 1) * bpt};
+  const SplitTile last{p.y, p.N, r_last, p.counters + (r_last < 0 ? 0 : r_last),
+                       static_cast<long long>(r_last) * bpt, static_cast<long long>(r_last + 1) * bpt};
+  finish_split_tiles<M>(pt, pw, first, acc_first, last, slot_last, acc, lane);
 }
 
 // ----------------------------------------------------------------------------

@@ -1,0 +1,541 @@
+// The layer stack as ONE persistent cooperative kernel.
+//
+// A decode step is an ordered list of products (the 64 layers' q|k|v, o,
+// gate|up, down, then the output head).  Launching one kernel per product
+// pays a launch, a prologue and a tail per product; here one CTA per SM runs
+// the whole list:
+//  * For each product every warp streams its stream-K range exactly as the
+//    single-product kernel does (same ranges, same arithmetic, same fix-up),
+//    so every output is bitwise equal to the corresponding q4_gemv / q8_gemv.
+//  * The warp's bulk-copy ring runs ahead ACROSS products: while a warp
+//    finishes product e (and waits at the barrier below), the first stages of
+//    its range in product e+1 are already in flight.  Weights never depend on
+//    activations, so prefetching them early is always valid.
+//  * Between products a grid-wide barrier (generation counter, bounded wait)
+//    guarantees that every output of product e, including the split-tile
+//    fix-ups, is written before any warp reads product e+1's activations:
+//    the same ordering as a stream of one launch per product.
+//  * Every wait is bounded.  A warp whose ring wait gives up marks the CTA
+//    aborted; the CTA stops at the next barrier, drains its in-flight copies
+//    (bounded) and exits; the other CTAs' barrier waits then give up too.
+#pragma once
+
+#include "q4gemv_kernels.cuh"
+
+namespace q4k {
+
+struct StackEntryDev {
+  const uint8_t* packed;
+  const uint16_t* x;
+  float* y;
+  long long N, K, TC;
+  long long blk_off;  // first block of this product in the concatenated sequence (stream mode)
+  int T, C, bits, P, khalf;
+  int tile_off;       // first counter of this product (stream mode)
+};
+
+struct StackParams {
+  const StackEntryDev* entries;
+  int E;
+  float* partials;      // [P][2][M][32]
+  unsigned* counters;   // one per tile of the largest product (re-zeroed as used)
+  unsigned* status;
+  unsigned* grid_bar;   // [0] arrivals, [1] generation
+  int G;                // CTAs in the grid (all resident: cooperative launch)
+  unsigned long long timeout_ns;
+  long long TBg;        // stream mode: blocks of all products, concatenated
+  int Pg;               // stream mode: warps with work
+};
+
+constexpr int kStackU = 2;                                   // chunks per stage
+constexpr int kStackSlotBytes = kStackU * Format<4>::kChunkBytes;  // the larger of the two formats
+
+__device__ __forceinline__ unsigned ld_acquire_gpu(const unsigned* p) {
+  unsigned v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+// L2 prefetch of a contiguous byte range (no shared memory involved).
+__device__ __forceinline__ void bulk_prefetch_l2(const void* src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
+
+// Walks one warp's stages of all products in order: (source, bytes) of the
+// next stage.  Warp-uniform state.
+struct StageCursor {
+  int pe = -1;
+  int left = 0;
+  const uint8_t* src = nullptr;
+  uint32_t bytes = 0;
+
+  __device__ __forceinline__ bool next(const StackParams& sp, int pw, const uint8_t** out_src, uint32_t* out_bytes);
+};
+
+// Grid-wide barrier of the G resident CTAs; all threads of the CTA call it.
+// Returns false when this CTA is aborting (its own abort flag, or a wait that
+// gave up).
+__device__ __forceinline__ bool grid_barrier(const StackParams& sp, int* s_abort) {
+  __syncthreads();
+  if (threadIdx.x == 0 && !*s_abort) {
+    unsigned* count = sp.grid_bar;
+    unsigned* gen = sp.grid_bar + 1;
+    const unsigned my_gen = ld_acquire_gpu(gen);
+    __threadfence();  // this CTA's outputs before its arrival
+    const unsigned arrived = atomicAdd(count, 1u);
+    if (arrived == static_cast<unsigned>(sp.G) - 1u) {
+      atomicExch(count, 0u);
+      __threadfence();
+      atomicAdd(gen, 1u);  // releases the waiting CTAs
+    } else {
+      const unsigned long long t0 = global_timer_ns();
+      while (ld_acquire_gpu(gen) == my_gen) {
+        if (global_timer_ns() - t0 > sp.timeout_ns) {
+          *s_abort = 1;
+          atomicOr(sp.status, kStatusTimeout);
+          break;
+        }
+      }
+    }
+    __threadfence();
+  }
+  __syncthreads();
+  return !*s_abort;
+}
+
+__device__ __forceinline__ bool StageCursor::next(const StackParams& sp, int pw, const uint8_t** out_src,
+                                                  uint32_t* out_bytes) {
+  while (left == 0) {
+    if (pe + 1 >= sp.E) return false;
+    ++pe;
+    const StackEntryDev& en = sp.entries[pe];
+    if (pw >= en.P) continue;
+    const long long TB = en.TC / kStackU;
+    const long long b = range_begin(pw, TB, en.P) * kStackU;
+    const long long e = range_begin(pw + 1, TB, en.P) * kStackU;
+    const int CB = en.bits == 4 ? Format<4>::kChunkBytes : Format<8>::kChunkBytes;
+    src = en.packed + b * CB;
+    left = static_cast<int>((e - b) / kStackU);
+    bytes = static_cast<uint32_t>(kStackU * CB);
+  }
+  *out_src = src;
+  *out_bytes = bytes;
+  src += bytes;
+  --left;
+  return true;
+}
+
+// PF: how many stages ahead of the shared-memory ring the weights are
+// prefetched into L2, so HBM keeps streaming while warps wait at a barrier.
+template <int M, int NW, int D, int PF>
+__global__ void __launch_bounds__(NW * 32, 1) stack_kernel(const StackParams sp) {
+  constexpr int U = kStackU;
+  constexpr int SLOT = kStackSlotBytes;
+  extern __shared__ __align__(128) unsigned char smem[];
+  __shared__ int s_abort;
+
+  const int lane = threadIdx.x & 31;
+  const int warp = threadIdx.x >> 5;
+  const int gi = lane >> 2, ti = lane & 3;
+  const int pw = blockIdx.x * NW + warp;
+  const uint32_t ring = smem_addr(smem + warp * D * SLOT);
+  const uint32_t bars = smem_addr(smem + NW * D * SLOT) + warp * D * 8;
+
+  if (threadIdx.x == 0) s_abort = 0;
+  if (lane == 0) {
+    for (int s = 0; s < D; ++s) mbar_init(bars + 8 * s, 1);
+    fence_barrier_init();
+  }
+  __syncthreads();
+  const uint64_t policy = l2_evict_first_policy();
+
+  // ---- producer: the warp's stages of all products, in order; `ahead` runs
+  // PF stages in front and only prefetches into L2
+  StageCursor ring_cur, ahead;
+  int g_issued = 0, g_consumed = 0;  // stages of this warp, all products
+  for (int s = 0; s < D + PF; ++s) {
+    const uint8_t* a;
+    uint32_t nb;
+    if (!ahead.next(sp, pw, &a, &nb)) break;
+    if (s >= D && lane == 0) bulk_prefetch_l2(a, nb);
+  }
+  auto produce = [&]() {
+    const uint8_t* src;
+    uint32_t nbytes;
+    if (!ring_cur.next(sp, pw, &src, &nbytes)) return;
+    const int slot = g_issued % D;
+    bulk_copy_g2s_if(lane == 0, ring + slot * SLOT, src, nbytes, bars + 8 * slot, policy);
+    ++g_issued;
+    if (PF > 0) {
+      const uint8_t* a;
+      uint32_t nb;
+      if (ahead.next(sp, pw, &a, &nb) && lane == 0) bulk_prefetch_l2(a, nb);
+    }
+  };
+  for (int s = 0; s < D; ++s) produce();
+
+  grid_dependency_wait();
+  grid_dependents_launch();
+
+  for (int ei = 0; ei < sp.E; ++ei) {
+    const StackEntryDev en = sp.entries[ei];
+    const long long TB = en.TC / U;
+    long long b = 0, e = 0;
+    if (pw < en.P) {
+      b = range_begin(pw, TB, en.P) * U;
+      e = range_begin(pw + 1, TB, en.P) * U;
+    }
+    const int nst = static_cast<int>((e - b) / U);
+    int r = static_cast<int>(floor_div(b, en.C));
+    int c = static_cast<int>(b - static_cast<long long>(r) * en.C);
+    const bool x_lane = gi < M;
+    const uint16_t* xrow = en.x + static_cast<long long>(x_lane ? gi : 0) * en.K + 8 * ti;
+    float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+    float acc_first[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+    int r_first = -1;
+    uint4 xa = make_uint4(0, 0, 0, 0), xb = make_uint4(0, 0, 0, 0);
+    const int KC = en.bits == 4 ? Format<4>::kKPerChunk : Format<8>::kKPerChunk;
+    const int CB = en.bits == 4 ? Format<4>::kChunkBytes : Format<8>::kChunkBytes;
+
+    bool ok = true;
+    for (int i = 0; i < nst; ++i) {
+      const int slot = g_consumed % D;
+      const uint32_t phase = static_cast<uint32_t>((g_consumed / D) & 1);
+      if (!mbar_wait_bounded(bars + 8 * slot, phase, sp.timeout_ns)) {
+        ok = false;
+        break;
+      }
+      const uint32_t stage = ring + slot * SLOT;
+      ChunkRegs regs[U];
+      if (en.bits == 4) {
+#pragma unroll
+        for (int j = 0; j < U; ++j) {
+          regs[j].codes[0] = lds128(stage + j * Format<4>::kChunkBytes + 16 * lane);
+          regs[j].codes[1] = lds128(stage + j * Format<4>::kChunkBytes + kHalfBytes + 16 * lane);
+          regs[j].scales = lds128(stage + j * Format<4>::kChunkBytes + kCodeBytes + 16 * gi);
+        }
+      } else {
+#pragma unroll
+        for (int j = 0; j < U; ++j) {
+          regs[j].codes[0] = lds128(stage + j * Format<8>::kChunkBytes + 16 * lane);
+          regs[j].codes[1] = lds128(stage + j * Format<8>::kChunkBytes + kHalfBytes + 16 * lane);
+          const uint2 s2 = lds64(stage + j * Format<8>::kChunkBytes + kCodeBytes + 8 * gi);
+          regs[j].scales = make_uint4(s2.x, s2.y, 0u, 0u);
+        }
+      }
+      // every lane has read the slot; lane 0 refills it with the next stage
+      __syncwarp();
+      produce();
+      ++g_consumed;
+      (void)CB;
+#pragma unroll
+      for (int j = 0; j < U; ++j) {
+        const uint16_t* xs = xrow + static_cast<long long>(c + j) * KC;
+        ldg128_pred(xa, xs, x_lane);
+        if (en.bits == 4) {
+          const bool half_empty = en.khalf && c + j == en.C - 1;
+          ldg128_pred(xb, xs + 32, x_lane && !half_empty);
+          if (half_empty) xb = make_uint4(0, 0, 0, 0);
+          q4_chunk_mac(acc, regs[j], xa, xb);
+        } else {
+          q8_chunk_mac(acc, regs[j], xa);
+        }
+      }
+      c += U;
+      if (c == en.C) {
+        if (static_cast<long long>(r) * en.C < b) {
+          r_first = r;
+#pragma unroll
+          for (int h = 0; h < 2; ++h)
+#pragma unroll
+            for (int q = 0; q < 4; ++q) acc_first[h][q] = acc[h][q];
+        } else {
+          store_tile<M>(en.y, en.N, r, acc, lane);
+        }
+        ++r;
+        c = 0;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) acc[h][0] = acc[h][1] = acc[h][2] = acc[h][3] = 0.f;
+      }
+    }
+    if (!ok) {
+      if (lane == 0) {
+        atomicOr(sp.status, kStatusTimeout);
+        atomicOr(&s_abort, 1);
+      }
+    } else if (nst > 0) {
+      int r_last = -1, slot_last = 1;
+      if (c != 0) {
+        r_last = r;
+        slot_last = (static_cast<long long>(r) * en.C <= b) ? 0 : 1;
+      }
+      const Partition pt{TB, en.P, sp.partials};
+      const int bpt = en.C / U;
+      const SplitTile first{en.y, en.N, r_first, sp.counters + (r_first < 0 ? 0 : r_first),
+                            static_cast<long long>(r_first) * bpt, static_cast<long long>(r_first + 1) * bpt};
+      const SplitTile last{en.y, en.N, r_last, sp.counters + (r_last < 0 ? 0 : r_last),
+                           static_cast<long long>(r_last) * bpt, static_cast<long long>(r_last + 1) * bpt};
+      finish_split_tiles<M>(pt, pw, first, acc_first, last, slot_last, acc, lane);
+    }
+    // every output of this product is written before the next reads its input
+    if (ei + 1 < sp.E) {
+      if (!grid_barrier(sp, &s_abort)) break;
+    }
+  }
+  if (s_abort) {
+    // wait (bounded) for this warp's copies still in flight, then leave
+    for (int g = g_consumed; g < g_issued; ++g) {
+      if (!mbar_wait_bounded(bars + 8 * (g % D), static_cast<uint32_t>((g / D) & 1), sp.timeout_ns)) break;
+    }
+  }
+}
+
+// ----------------------------------------------------------------------------
+// Stream mode: the products do not read each other's outputs, so the whole
+// list is ONE stream-K problem.  Its blocks (two chunks each) are concatenated
+// product after product, and every warp streams one contiguous range of the
+// concatenation, crossing product boundaries (which are tile boundaries)
+// without any synchronisation.  Only the tiles holding a range's two ends are
+// split between warps, so each warp finishes at most two split tiles, at the
+// very end.  No grid barrier; every wait is a bounded ring wait.
+// ----------------------------------------------------------------------------
+
+// Product holding concatenated block gb (products are in block order).
+__device__ __forceinline__ int entry_of_block(const StackParams& sp, long long gb) {
+  int lo = 0, hi = sp.E - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (sp.entries[mid].blk_off <= gb)
+      lo = mid;
+    else
+      hi = mid - 1;
+  }
+  return lo;
+}
+
+// The producer side of a warp's ring in stream mode: the next stage to copy
+// in the warp's range, crossing products.  Warp-uniform state.
+struct StreamProducer {
+  int e = 0;                 // product of the next stage
+  int left_entry = 0;        // stages left in that product
+  long long left_total = 0;  // stages left in the range
+  const uint8_t* src = nullptr;
+  uint32_t bytes = 0;
+
+  __device__ __forceinline__ void enter(const StackParams& sp, int entry, long long lb) {
+    const StackEntryDev& en = sp.entries[entry];
+    const int CB = en.bits == 4 ? Format<4>::kChunkBytes : Format<8>::kChunkBytes;
+    e = entry;
+    bytes = static_cast<uint32_t>(kStackU * CB);
+    src = en.packed + lb * kStackU * CB;
+    const long long in_entry = en.TC / kStackU - lb;
+    left_entry = static_cast<int>(in_entry < left_total ? in_entry : left_total);
+  }
+  // Copies the next stage into `dst` (lane 0), completing on `bar`.
+  __device__ __forceinline__ bool issue(const StackParams& sp, uint32_t dst, uint32_t bar, uint64_t policy,
+                                        int lane) {
+    if (left_total == 0) return false;
+    if (left_entry == 0) enter(sp, e + 1, 0);
+    bulk_copy_g2s_if(lane == 0, dst, src, bytes, bar, policy);
+    src += bytes;
+    --left_entry;
+    --left_total;
+    return true;
+  }
+};
+
+// The warp's ring: D slots of one stage each, and the stage counters.
+struct StreamRing {
+  uint32_t ring, bars;
+  int slot = 0;          // slot of the next stage to consume
+  uint32_t phase = 0;
+  int in_flight = 0;     // stages issued and not yet consumed
+};
+
+// Consumes `nblk` stages of one product (format BITS), from local block lb0.
+// Keeps the split-tile bookkeeping of the warp's range [gb, ...): a tile that
+// began before gb is kept in acc_first / first; a tile still open at the end
+// stays in acc with (r, c).  Returns false if a ring wait gave up.
+template <int BITS, int M, bool KHALF, int D>
+__device__ __forceinline__ bool stream_segment(const StackParams& sp, const StackEntryDev& en, int e, long long lb0,
+                                               long long nblk, long long gb, StreamRing& rg, StreamProducer& pr,
+                                               uint64_t policy, float (&acc)[2][4], int pw, int& e_first,
+                                               int& r_first, int& r, int& c, int lane) {
+  constexpr int U = kStackU;
+  constexpr int CB = Format<BITS>::kChunkBytes;
+  constexpr int KC = Format<BITS>::kKPerChunk;
+  const int gi = lane >> 2, ti = lane & 3;
+  const int bpt = en.C / U;
+  const bool x_lane = gi < M;
+  const uint16_t* xrow = en.x + static_cast<long long>(x_lane ? gi : 0) * en.K + 8 * ti;
+  r = static_cast<int>(floor_div(lb0, bpt));
+  c = static_cast<int>(lb0 - static_cast<long long>(r) * bpt) * U;
+  const uint16_t* xs = xrow + c * KC;
+  uint4 xa = make_uint4(0, 0, 0, 0), xb = make_uint4(0, 0, 0, 0);
+  for (long long i = 0; i < nblk; ++i) {
+    const uint32_t bar = rg.bars + 8 * rg.slot;
+    if (!mbar_wait_bounded(bar, rg.phase, sp.timeout_ns)) return false;
+    const uint32_t stage = rg.ring + rg.slot * kStackSlotBytes;
+    ChunkRegs regs[U];
+#pragma unroll
+    for (int j = 0; j < U; ++j) {
+      regs[j].codes[0] = lds128(stage + j * CB + 16 * lane);
+      regs[j].codes[1] = lds128(stage + j * CB + kHalfBytes + 16 * lane);
+      if (BITS == 4) {
+        regs[j].scales = lds128(stage + j * CB + kCodeBytes + 16 * gi);
+      } else {
+        const uint2 s2 = lds64(stage + j * CB + kCodeBytes + 8 * gi);
+        regs[j].scales = make_uint4(s2.x, s2.y, 0u, 0u);
+      }
+    }
+    // every lane has read the slot; lane 0 refills it with the next stage
+    __syncwarp();
+    if (!pr.issue(sp, stage, bar, policy, lane)) --rg.in_flight;
+    if (++rg.slot == D) {
+      rg.slot = 0;
+      rg.phase ^= 1u;
+    }
+#pragma unroll
+    for (int j = 0; j < U; ++j) {
+      ldg128_pred(xa, xs + j * KC, x_lane);
+      if (BITS == 4) {
+        if (KHALF && c + j == en.C - 1) {
+          xb = make_uint4(0, 0, 0, 0);  // a K that is an odd multiple of 32: the half-empty last chunk
+        } else {
+          ldg128_pred(xb, xs + j * KC + 32, x_lane);
+        }
+        q4_chunk_mac(acc, regs[j], xa, xb);
+      } else {
+        q8_chunk_mac(acc, regs[j], xa);
+      }
+    }
+    xs += U * KC;
+    c += U;
+    if (c == en.C) {
+      const long long tile_g = en.blk_off + static_cast<long long>(r) * bpt;  // the tile's first block
+      if (tile_g < gb) {  // began in an earlier warp's range: its partial goes to slot 0 now
+        write_partial<M>(sp.partials, pw, 0, acc, lane);
+        e_first = e;
+        r_first = r;
+      } else {
+        store_tile<M>(en.y, en.N, r, acc, lane);
+      }
+      ++r;
+      c = 0;
+      xs = xrow;
+#pragma unroll
+      for (int h = 0; h < 2; ++h) acc[h][0] = acc[h][1] = acc[h][2] = acc[h][3] = 0.f;
+    }
+  }
+  return true;
+}
+
+template <int M, int NW, int D, int PF>
+__global__ void __launch_bounds__(NW * 32, 1) stream_kernel(const StackParams sp) {
+  static_assert(PF == 0, "stream mode prefetches through its ring only");
+  extern __shared__ __align__(128) unsigned char smem[];
+
+  const int lane = threadIdx.x & 31;
+  const int warp = threadIdx.x >> 5;
+  const int pw = blockIdx.x * NW + warp;
+  StreamRing rg;
+  rg.ring = smem_addr(smem + warp * D * kStackSlotBytes);
+  rg.bars = smem_addr(smem + NW * D * kStackSlotBytes) + warp * D * 8;
+
+  if (lane == 0) {
+    for (int s = 0; s < D; ++s) mbar_init(rg.bars + 8 * s, 1);
+    fence_barrier_init();
+  }
+  __syncwarp();
+  const uint64_t policy = l2_evict_first_policy();
+
+  long long gb = 0, ge = 0;
+  if (pw < sp.Pg) {
+    gb = range_begin(pw, sp.TBg, sp.Pg);
+    ge = range_begin(pw + 1, sp.TBg, sp.Pg);
+  }
+  if (ge <= gb) {
+    grid_dependency_wait();
+    grid_dependents_launch();
+    return;
+  }
+  const int e0 = entry_of_block(sp, gb);
+  StreamProducer pr;
+  pr.left_total = ge - gb;
+  pr.enter(sp, e0, gb - sp.entries[e0].blk_off);
+  for (int s = 0; s < D; ++s) {
+    if (!pr.issue(sp, rg.ring + s * kStackSlotBytes, rg.bars + 8 * s, policy, lane)) break;
+    ++rg.in_flight;
+  }
+
+  grid_dependency_wait();
+  grid_dependents_launch();
+
+  float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+  int e_first = -1, r_first = -1;  // split first tile (its partial is written when it completes)
+  int r = 0, c = 0;
+  int e = e0;
+  long long lb = gb - sp.entries[e0].blk_off;
+  long long left = ge - gb;
+  StackEntryDev en = sp.entries[e];
+  bool ok = true;
+  while (left > 0) {
+    const long long in_entry = en.TC / kStackU - lb;
+    const long long n = in_entry < left ? in_entry : left;
+    if (en.bits == 4) {  // stream mode has no product with a half-empty last chunk (checked on the host)
+      ok = stream_segment<4, M, false, D>(sp, en, e, lb, n, gb, rg, pr, policy, acc, pw, e_first, r_first, r, c, lane);
+    } else {
+      ok = stream_segment<8, M, false, D>(sp, en, e, lb, n, gb, rg, pr, policy, acc, pw, e_first, r_first, r, c, lane);
+    }
+    if (!ok) break;
+    left -= n;
+    if (left > 0) {
+      en = sp.entries[++e];
+      lb = 0;
+    }
+  }
+  if (!ok) {
+    if (lane == 0) atomicOr(sp.status, kStatusTimeout);
+    // wait (bounded) for this warp's copies still in flight, then leave
+    for (int k = 0; k < rg.in_flight; ++k) {
+      if (!mbar_wait_bounded(rg.bars + 8 * rg.slot, rg.phase, sp.timeout_ns)) break;
+      if (++rg.slot == D) {
+        rg.slot = 0;
+        rg.phase ^= 1u;
+      }
+    }
+    return;
+  }
+  // finish the split tiles: the first one's partial is already in slot 0
+  SplitTile first{nullptr, 0, -1, sp.counters, 0, 0}, last{nullptr, 0, -1, sp.counters, 0, 0};
+  if (r_first >= 0) {
+    const StackEntryDev& ef = sp.entries[e_first];
+    const int bpt = ef.C / kStackU;
+    const long long tile_g = ef.blk_off + static_cast<long long>(r_first) * bpt;
+    first = SplitTile{ef.y, ef.N, r_first, sp.counters + ef.tile_off + r_first, tile_g, tile_g + bpt};
+  }
+  if (c != 0) {
+    const int bpt = en.C / kStackU;
+    const long long tile_g = en.blk_off + static_cast<long long>(r) * bpt;
+    last = SplitTile{en.y, en.N, r, sp.counters + en.tile_off + r, tile_g, tile_g + bpt};
+    write_partial<M>(sp.partials, pw, tile_g <= gb ? 0 : 1, acc, lane);
+  }
+  if (first.r < 0 && last.r < 0) return;
+  __threadfence();
+  __syncwarp();
+  unsigned a_first = 0, a_last = 0;
+  if (lane == 0) {
+    if (first.r >= 0) a_first = atomicAdd(first.counter, 1u);
+    if (last.r >= 0) a_last = atomicAdd(last.counter, 1u);
+  }
+  a_first = __shfl_sync(0xFFFFFFFFu, a_first, 0);
+  a_last = __shfl_sync(0xFFFFFFFFu, a_last, 0);
+  const Partition pt{sp.TBg, sp.Pg, sp.partials};
+  const bool red_first = first.r >= 0 && a_first + 1 == tile_contributors(pt, first);
+  const bool red_last = last.r >= 0 && a_last + 1 == tile_contributors(pt, last);
+  if (red_first || red_last) __threadfence();
+  if (red_first) reduce_tile<M>(pt, first, lane);
+  if (red_last) reduce_tile<M>(pt, last, lane);
+}
+
+}  // namespace q4k

@@ -27,6 +27,8 @@ Q4_ERR_CUDA = -5
 Q4_ERR_TIMEOUT = -6
 Q4_ERR_UNSUPPORTED = -7
 Q4_STACK_NO_PDL = 1
+Q4_STACK_GRAPH = 2
+Q4_STACK_INDEPENDENT = 4
 
 ERROR_NAMES = {
     Q4_ERR_INVALID_ARG: "INVALID_ARG",

@@ -148,8 +148,14 @@ class DeviceStream:
             self.x[K] = xb
         self.y = [torch.empty(M * t.N, dtype=torch.float32, device=dev) for t in self.tensors]
         torch.cuda.synchronize()
+        self.stack = self.make_stack(flags)
+
+    def make_stack(self, flags: int = 0):
+        """Another layer stack over the same device buffers (e.g. another mode)."""
+        import bit_weight_gemv_q4_b200 as q4
+
         entries = [(t.bits, t.N, t.K, p, self.x[t.K], y) for t, p, y in zip(self.tensors, self.packed, self.y)]
-        self.stack = q4.layer_stack_create(entries, M, flags)
+        return q4.layer_stack_create(entries, self.M, flags)
 
     @property
     def weight_bytes(self) -> int:

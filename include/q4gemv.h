@@ -214,17 +214,40 @@ typedef struct q4_stack_entry {
 
 typedef struct q4_stack q4_stack;
 
-#define Q4_STACK_NO_PDL 1 /* launch without programmatic dependent launch (for comparison) */
+#define Q4_STACK_NO_PDL 1 /* graph mode, launched without programmatic dependent launch */
+#define Q4_STACK_GRAPH 2  /* graph mode: one kernel per product, captured as a CUDA graph */
+#define Q4_STACK_INDEPENDENT 4 /* stream mode: the caller asserts no product reads another's output */
 
-/* Validates every entry, allocates the library-owned workspace, and captures
- * the n_entries products as one CUDA graph on the current device.  Each
- * product is launched in order; with PDL each kernel prefetches its first
- * weight tiles while its predecessor finishes, and reads x only after the
- * predecessor has completed.  The caller's buffers must outlive the stack.
- * Errors: as q4_gemv, plus CUDA for allocation or capture failures. */
+/* Validates every entry and prepares the stack on the current device.
+ * Default (ordered persistent) mode: one cooperative kernel, one CTA per SM,
+ * runs the whole list; each product's weights are streamed exactly as by
+ * q4_gemv / q8_gemv (bitwise-equal outputs), the bulk-copy rings prefetch the
+ * next product's weights while the current one finishes, and a grid-wide
+ * barrier between products guarantees that every output of a product is
+ * written before any of the next product's activations are read -- the
+ * ordering of a stream of one launch per product.
+ * Stream mode (Q4_STACK_INDEPENDENT): for products that do not read each
+ * other's outputs (the activations are inputs of the step, not outputs of an
+ * earlier product).  One cooperative kernel treats the concatenated products
+ * as a single work-split problem: every warp streams one contiguous range
+ * across product boundaries with no synchronisation, so the HBM stream never
+ * pauses between products.  Outputs agree with q4_gemv / q8_gemv within the
+ * product tolerance (tiles may be split at other places).
+ * Both persistent modes need every product non-empty with an even number of
+ * chunks per tile; other lists use graph mode.  Stream mode also needs every
+ * q4 K to be a multiple of 64; otherwise the ordered mode is used.
+ * Graph mode (Q4_STACK_GRAPH, or Q4_STACK_NO_PDL): the products are launched in
+ * order, each as its own kernel, and captured once as a CUDA graph; with PDL
+ * each kernel prefetches its first weight tiles while its predecessor
+ * finishes and reads x only after the predecessor has completed.
+ * Either mode allocates a library-owned workspace (and, persistent, the entry
+ * table); the caller's buffers must outlive the stack.
+ * Errors: as q4_gemv, plus CUDA for allocation or capture failures and
+ * UNSUPPORTED if the persistent kernel cannot be resident on every SM. */
 Q4_API int layer_stack_create(const q4_stack_entry* entries, int n_entries, int M, int flags, q4_stack** out);
 
-/* Replays the captured products on `stream` (one cudaGraphLaunch). */
+/* Runs the products on `stream`: one cooperative kernel launch (persistent
+ * mode) or one cudaGraphLaunch (graph mode).  Asynchronous. */
 Q4_API int layer_stack_run(q4_stack* stack, void* stream);
 
 /* Synchronises `stream` and reports a bounded wait that gave up during the

@@ -9,10 +9,17 @@ import gpu_helpers as H
 
 pytestmark = pytest.mark.gpu
 
+# every product has an even number of chunks per tile and whole q4 chunks:
+# eligible for both persistent modes
 MIXED = [
-    Tensor("a", 4, 1000, 5120, 201), Tensor("b", 8, 37, 96, 202), Tensor("c", 4, 17, 17408, 203),
-    Tensor("d", 8, 4099, 5120, 204), Tensor("e", 4, 64, 4096 + 32, 205), Tensor("f", 4, 7168, 5120, 206),
+    Tensor("a", 4, 1000, 5120, 201), Tensor("b", 8, 37, 128, 202), Tensor("c", 4, 17, 17408, 203),
+    Tensor("d", 8, 4099, 5120, 204), Tensor("e", 4, 64, 128, 205), Tensor("f", 4, 7168, 5120, 206),
 ]
+# a q4 K that is an odd multiple of 32 (even chunk count): ordered persistent
+# mode, also when stream mode is asked for
+HALF = [Tensor("j", 4, 64, 96, 210), Tensor("k", 8, 100, 5120, 211)]
+# odd chunk counts per tile: graph mode only
+ODD = [Tensor("g", 8, 37, 96, 207), Tensor("h", 4, 64, 4096 + 32, 208), Tensor("i", 4, 300, 5120, 209)]
 
 
 @pytest.fixture(scope="module")
@@ -34,50 +41,93 @@ def _host_rows(stream, i, r0, n):
     return q, s, x
 
 
-@pytest.mark.parametrize("M", [1, 4])
-def test_stack_equals_single_calls_and_oracle(q4, M):
+def _check_stack(q4, tensors, M, flags, expect_launches):
     torch = H.torch()
-    st = workloads.DeviceStream(MIXED, M)
-    assert st.stack.launches() == len(MIXED)
+    st = workloads.DeviceStream(tensors, M, flags=flags)
+    assert st.stack.launches() == expect_launches
     st.run()
     st.check()
-    first = [_y(st, i).copy() for i in range(len(MIXED))]
-    # a second replay is bitwise identical
+    first = [_y(st, i).copy() for i in range(len(tensors))]
+    # a second run is bitwise identical
     for y in st.y:
         y.fill_(float("nan"))
     st.run()
     st.check()
-    for i in range(len(MIXED)):
+    for i in range(len(tensors)):
         assert np.array_equal(_y(st, i), first[i])
     # each product equals a direct call on the same device buffers
-    for i, t in enumerate(MIXED):
+    for i, t in enumerate(tensors):
         ws = H.workspace(t.bits, t.N, t.K, M)
         y = torch.empty(M * t.N, device="cuda")
         (q4.q4_gemv if t.bits == 4 else q4.q8_gemv)(st.packed[i], t.N, t.K, st.x[t.K], M, y, ws)
         q4.q4_workspace_check(ws)
         assert np.array_equal(y.cpu().numpy().reshape(M, t.N), first[i]), t.name
     # and the oracle, on every row
-    for i, t in enumerate(MIXED):
+    for i, t in enumerate(tensors):
         q, s, x = _host_rows(st, i, 0, t.N)
         H.assert_parity(first[i], q, s, x, t.bits)
-    # without programmatic dependent launch the results are the same bits
-    st2 = workloads.DeviceStream(MIXED, M, flags=q4.Q4_STACK_NO_PDL)
-    st2.run()
-    st2.check()
-    for i in range(len(MIXED)):
-        assert np.array_equal(_y(st2, i), first[i])
     st.close()
-    st2.close()
+    return first
 
 
 @pytest.mark.parametrize("M", [1, 4])
-def test_full_decode_stream_sampled(q4, M):
-    """All 257 products of one decode step (64 layers + q8 head, 13.7 GB) in the
-    captured stack; sampled rows of several tensors against the oracle."""
+def test_stack_modes_equal_single_calls_and_oracle(q4, M):
+    persistent = _check_stack(q4, MIXED, M, 0, 1)
+    graph = _check_stack(q4, MIXED, M, q4.Q4_STACK_GRAPH, len(MIXED))
+    nopdl = _check_stack(q4, MIXED, M, q4.Q4_STACK_NO_PDL, len(MIXED))
+    for a, b, c in zip(persistent, graph, nopdl):
+        assert np.array_equal(a, b) and np.array_equal(a, c)
+
+
+@pytest.mark.parametrize("M", [1, 4])
+def test_stream_mode_of_independent_products(q4, M):
+    """Stream mode splits the concatenated products between warps differently
+    from one call per product: the outputs are compared with the oracle (every
+    row) and with single calls within the product tolerance, and two runs are
+    bitwise identical."""
+    torch = H.torch()
+    st = workloads.DeviceStream(MIXED, M, flags=q4.Q4_STACK_INDEPENDENT)
+    assert st.stack.launches() == 1
+    st.run()
+    st.check()
+    first = [_y(st, i).copy() for i in range(len(MIXED))]
+    for y in st.y:
+        y.fill_(float("nan"))
+    st.run()
+    st.check()
+    for i, t in enumerate(MIXED):
+        assert np.array_equal(_y(st, i), first[i]), t.name
+        q, s, x = _host_rows(st, i, 0, t.N)
+        H.assert_parity(first[i], q, s, x, t.bits)
+        ws = H.workspace(t.bits, t.N, t.K, M)
+        y = torch.empty(M * t.N, device="cuda")
+        (q4.q4_gemv if t.bits == 4 else q4.q8_gemv)(st.packed[i], t.N, t.K, st.x[t.K], M, y, ws)
+        q4.q4_workspace_check(ws)
+        import oracle
+        _, B = oracle.gemv(t.bits, q, s, x)
+        ok, _, _ = oracle.within_tolerance(first[i], y.cpu().numpy().reshape(M, t.N).astype(np.float64), B)
+        assert ok.all(), t.name
+    st.close()
+
+
+@pytest.mark.parametrize("M", [1, 2])
+def test_half_empty_chunks_fall_back_to_ordered_mode(q4, M):
+    _check_stack(q4, HALF, M, q4.Q4_STACK_INDEPENDENT, 1)
+
+
+@pytest.mark.parametrize("M", [1, 3])
+def test_stack_with_odd_chunk_counts_uses_graph_mode(q4, M):
+    _check_stack(q4, ODD, M, 0, len(ODD))
+
+
+@pytest.mark.parametrize("M,mode", [(1, "ordered"), (4, "ordered"), (1, "stream"), (4, "stream")])
+def test_full_decode_stream_sampled(q4, M, mode):
+    """All 257 products of one decode step (64 layers + q8 head, 13.7 GB) in one
+    persistent kernel; sampled rows of several tensors against the oracle."""
     torch = H.torch()
     tensors = workloads.decode_stream(fused=True)
-    st = workloads.DeviceStream(tensors, M)
-    assert st.stack.launches() == 257
+    st = workloads.DeviceStream(tensors, M, flags=0 if mode == "ordered" else q4.Q4_STACK_INDEPENDENT)
+    assert st.stack.launches() == 1  # one persistent kernel for the 257 products
     st.run()
     st.run()
     st.check()

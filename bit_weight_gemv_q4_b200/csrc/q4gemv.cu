@@ -56,8 +56,12 @@ static_assert(kRingChunks % 2 == 0 && kRingChunks >= 4, "ring must hold two stag
 #ifndef Q4_TUNE_STACK_PF
 #define Q4_TUNE_STACK_PF 0
 #endif
-constexpr int kStackD = Q4_TUNE_STACK_D;    // stages of 2 chunks per warp in the persistent stack kernel
-constexpr int kStackPF = Q4_TUNE_STACK_PF;  // further stages prefetched into L2
+#ifndef Q4_TUNE_STREAM_U
+#define Q4_TUNE_STREAM_U 4
+#endif
+constexpr int kStackD = Q4_TUNE_STACK_D;    // stages per warp in the persistent stack kernels
+constexpr int kStackPF = Q4_TUNE_STACK_PF;  // further stages prefetched into L2 (ordered mode)
+constexpr int kStreamU = Q4_TUNE_STREAM_U;  // chunks per stage in stream mode, when the shapes allow
 // shared memory a CTA may use (B200: 227 KB per CTA)
 constexpr int kSmemLimit = 227 * 1024 / kCtasPerSm;
 constexpr size_t kWsHeader = 256;
@@ -528,19 +532,25 @@ void* stack_kernel_ptr() {
   return reinterpret_cast<void*>(&q4k::stack_kernel<M, kNW, kStackD, kStackPF>);
 }
 
-template <int M>
+template <int M, int SU>
 void* stream_kernel_ptr() {
-  return reinterpret_cast<void*>(&q4k::stream_kernel<M, kNW, kStackD, kStackPF>);
+  return reinterpret_cast<void*>(&q4k::stream_kernel<M, kNW, kStackD, SU>);
 }
 
-void* select_stack_kernel(int M, bool independent) {
-  static void* const table[2][4] = {
+// su: chunks per stage of the stream-mode kernel (0 = ordered mode)
+void* select_stack_kernel(int M, int su) {
+  static void* const table[3][4] = {
       {stack_kernel_ptr<1>(), stack_kernel_ptr<2>(), stack_kernel_ptr<3>(), stack_kernel_ptr<4>()},
-      {stream_kernel_ptr<1>(), stream_kernel_ptr<2>(), stream_kernel_ptr<3>(), stream_kernel_ptr<4>()}};
-  return table[independent ? 1 : 0][M - 1];
+      {stream_kernel_ptr<1, 2>(), stream_kernel_ptr<2, 2>(), stream_kernel_ptr<3, 2>(), stream_kernel_ptr<4, 2>()},
+      {stream_kernel_ptr<1, kStreamU>(), stream_kernel_ptr<2, kStreamU>(), stream_kernel_ptr<3, kStreamU>(),
+       stream_kernel_ptr<4, kStreamU>()}};
+  return table[su == 0 ? 0 : (su == 2 ? 1 : 2)][M - 1];
 }
 
-int stack_smem_bytes() { return kNW * kStackD * q4k::kStackSlotBytes + kNW * kStackD * 8; }
+int stack_smem_bytes(int su) {
+  const int slot = (su == 0 ? q4k::kStackU : su) * q4k::Format<4>::kChunkBytes;
+  return kNW * kStackD * slot + kNW * kStackD * 8;
+}
 
 void free_stack(q4_stack* st) {
   if (st->exec) cudaGraphExecDestroy(st->exec);
@@ -562,8 +572,11 @@ bool stack_eligible(const q4_stack_entry* entries, int n) {
   return true;
 }
 
-int create_persistent(const q4_stack_entry* entries, int n, int M, bool independent, const DeviceInfo& dev,
-                      q4_stack* st) {
+// su: stream mode with stages of su chunks (every product's C a multiple of
+// su), or 0 for ordered mode.
+int create_persistent(const q4_stack_entry* entries, int n, int M, int su, const DeviceInfo& dev, q4_stack* st) {
+  const bool independent = su != 0;
+  const long long blk = independent ? su : q4k::kStackU;  // chunks per stream-K block
   long long max_t = 1, total_blocks = 0, total_tiles = 0;
   std::vector<q4k::StackEntryDev> host(static_cast<size_t>(n));
   const long long warps = static_cast<long long>(dev.sms) * kNW;
@@ -594,7 +607,7 @@ int create_persistent(const q4_stack_entry* entries, int n, int M, bool independ
     d.khalf = (en.bits == 4 && s.K % 64 == 32) ? 1 : 0;
     d.blk_off = total_blocks;
     d.tile_off = static_cast<int>(total_tiles);
-    total_blocks += s.TC / q4k::kStackU;
+    total_blocks += s.TC / blk;
     total_tiles += s.T;
     if (s.T > max_t) max_t = s.T;
   }
@@ -609,8 +622,8 @@ int create_persistent(const q4_stack_entry* entries, int n, int M, bool independ
   if (err == cudaSuccess)
     err = cudaMemcpy(st->entries_dev, host.data(), sizeof(q4k::StackEntryDev) * host.size(), cudaMemcpyHostToDevice);
   if (err != cudaSuccess) return cuda_fail(err, "layer_stack_create: allocation");
-  st->fn = select_stack_kernel(M, independent);
-  st->smem = stack_smem_bytes();
+  st->fn = select_stack_kernel(M, su);
+  st->smem = stack_smem_bytes(su);
   st->block = kNW * 32;
   st->grid = dev.sms;
   err = cudaFuncSetAttribute(st->fn, cudaFuncAttributeMaxDynamicSharedMemorySize, st->smem);
@@ -704,12 +717,21 @@ extern "C" Q4_API int layer_stack_create(const q4_stack_entry* entries, int n_en
   q4_stack* st = new q4_stack();
   cudaGetDevice(&st->device);
   const bool graph = (flags & (Q4_STACK_GRAPH | Q4_STACK_NO_PDL)) != 0 || !stack_eligible(entries, n_entries);
-  // stream mode also needs whole q4 chunks (K a multiple of 64); else ordered
-  bool independent = (flags & Q4_STACK_INDEPENDENT) != 0;
-  for (int i = 0; independent && i < n_entries; ++i)
-    if (entries[i].bits == 4 && entries[i].K % 64 != 0) independent = false;
+  // stream mode also needs whole q4 chunks (K a multiple of 64); else ordered.
+  // Its stages hold kStreamU chunks when every product's chunks per tile is a
+  // multiple of kStreamU, else 2.
+  int su = (flags & Q4_STACK_INDEPENDENT) != 0 ? kStreamU : 0;
+  for (int i = 0; su != 0 && i < n_entries; ++i) {
+    if (entries[i].bits == 4 && entries[i].K % 64 != 0) {
+      su = 0;
+    } else {
+      const long long kc = entries[i].bits == 4 ? 64 : 32;
+      const long long C = (entries[i].K + kc - 1) / kc;
+      if (C % su != 0) su = 2;
+    }
+  }
   rc = graph ? create_graph(entries, n_entries, M, flags, dev, st)
-             : create_persistent(entries, n_entries, M, independent, dev, st);
+             : create_persistent(entries, n_entries, M, su, dev, st);
   if (rc) {
     free_stack(st);
     return rc;

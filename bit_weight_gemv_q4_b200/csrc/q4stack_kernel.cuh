@@ -292,7 +292,7 @@ __global__ void __launch_bounds__(NW * 32, 1) stack_kernel(const StackParams sp)
 
 // ----------------------------------------------------------------------------
 // Stream mode: the products do not read each other's outputs, so the whole
-// list is ONE stream-K problem.  Its blocks (two chunks each) are concatenated
+// list is ONE stream-K problem.  Its blocks (SU chunks each) are concatenated
 // product after product, and every warp streams one contiguous range of the
 // concatenation, crossing product boundaries (which are tile boundaries)
 // without any synchronisation.  Only the tiles holding a range's two ends are
@@ -313,8 +313,9 @@ __device__ __forceinline__ int entry_of_block(const StackParams& sp, long long g
   return lo;
 }
 
-// The producer side of a warp's ring in stream mode: the next stage to copy
-// in the warp's range, crossing products.  Warp-uniform state.
+// The producer side of a warp's ring in stream mode: the next stage (SU
+// chunks) to copy in the warp's range, crossing products.  Warp-uniform state.
+template <int SU>
 struct StreamProducer {
   int e = 0;                 // product of the next stage
   int left_entry = 0;        // stages left in that product
@@ -326,9 +327,9 @@ struct StreamProducer {
     const StackEntryDev& en = sp.entries[entry];
     const int CB = en.bits == 4 ? Format<4>::kChunkBytes : Format<8>::kChunkBytes;
     e = entry;
-    bytes = static_cast<uint32_t>(kStackU * CB);
-    src = en.packed + lb * kStackU * CB;
-    const long long in_entry = en.TC / kStackU - lb;
+    bytes = static_cast<uint32_t>(SU * CB);
+    src = en.packed + lb * SU * CB;
+    const long long in_entry = en.TC / SU - lb;
     left_entry = static_cast<int>(in_entry < left_total ? in_entry : left_total);
   }
   // Copies the next stage into `dst` (lane 0), completing on `bar`.
@@ -352,16 +353,18 @@ struct StreamRing {
   int in_flight = 0;     // stages issued and not yet consumed
 };
 
-// Consumes `nblk` stages of one product (format BITS), from local block lb0.
-// Keeps the split-tile bookkeeping of the warp's range [gb, ...): a tile that
-// began before gb is kept in acc_first / first; a tile still open at the end
-// stays in acc with (r, c).  Returns false if a ring wait gave up.
-template <int BITS, int M, bool KHALF, int D>
+// Consumes `nblk` stages (SU chunks each) of one product (format BITS), from
+// local block lb0.  Keeps the split-tile bookkeeping of the warp's range
+// [gb, ...): the partial of a tile that began before gb goes to partial slot
+// 0 when the tile ends (e_first, r_first); a tile still open at the end stays
+// in acc with (r, c).  Returns false if a ring wait gave up.
+template <int BITS, int M, int D, int SU>
 __device__ __forceinline__ bool stream_segment(const StackParams& sp, const StackEntryDev& en, int e, long long lb0,
-                                               long long nblk, long long gb, StreamRing& rg, StreamProducer& pr,
+                                               long long nblk, long long gb, StreamRing& rg, StreamProducer<SU>& pr,
                                                uint64_t policy, float (&acc)[2][4], int pw, int& e_first,
                                                int& r_first, int& r, int& c, int lane) {
-  constexpr int U = kStackU;
+  constexpr int U = SU;
+  constexpr int SLOT = SU * Format<4>::kChunkBytes;
   constexpr int CB = Format<BITS>::kChunkBytes;
   constexpr int KC = Format<BITS>::kKPerChunk;
   const int gi = lane >> 2, ti = lane & 3;
@@ -375,38 +378,33 @@ __device__ __forceinline__ bool stream_segment(const StackParams& sp, const Stac
   for (long long i = 0; i < nblk; ++i) {
     const uint32_t bar = rg.bars + 8 * rg.slot;
     if (!mbar_wait_bounded(bar, rg.phase, sp.timeout_ns)) return false;
-    const uint32_t stage = rg.ring + rg.slot * kStackSlotBytes;
-    ChunkRegs regs[U];
+    const uint32_t stage = rg.ring + rg.slot * SLOT;
 #pragma unroll
     for (int j = 0; j < U; ++j) {
-      regs[j].codes[0] = lds128(stage + j * CB + 16 * lane);
-      regs[j].codes[1] = lds128(stage + j * CB + kHalfBytes + 16 * lane);
+      ChunkRegs cr;
+      cr.codes[0] = lds128(stage + j * CB + 16 * lane);
+      cr.codes[1] = lds128(stage + j * CB + kHalfBytes + 16 * lane);
       if (BITS == 4) {
-        regs[j].scales = lds128(stage + j * CB + kCodeBytes + 16 * gi);
+        cr.scales = lds128(stage + j * CB + kCodeBytes + 16 * gi);
       } else {
         const uint2 s2 = lds64(stage + j * CB + kCodeBytes + 8 * gi);
-        regs[j].scales = make_uint4(s2.x, s2.y, 0u, 0u);
+        cr.scales = make_uint4(s2.x, s2.y, 0u, 0u);
       }
-    }
-    // every lane has read the slot; lane 0 refills it with the next stage
-    __syncwarp();
-    if (!pr.issue(sp, stage, bar, policy, lane)) --rg.in_flight;
-    if (++rg.slot == D) {
-      rg.slot = 0;
-      rg.phase ^= 1u;
-    }
-#pragma unroll
-    for (int j = 0; j < U; ++j) {
-      ldg128_pred(xa, xs + j * KC, x_lane);
-      if (BITS == 4) {
-        if (KHALF && c + j == en.C - 1) {
-          xb = make_uint4(0, 0, 0, 0);  // a K that is an odd multiple of 32: the half-empty last chunk
-        } else {
-          ldg128_pred(xb, xs + j * KC + 32, x_lane);
+      if (j == U - 1) {
+        // every lane has read the slot; lane 0 refills it with the next stage
+        __syncwarp();
+        if (!pr.issue(sp, stage, bar, policy, lane)) --rg.in_flight;
+        if (++rg.slot == D) {
+          rg.slot = 0;
+          rg.phase ^= 1u;
         }
-        q4_chunk_mac(acc, regs[j], xa, xb);
+      }
+      ldg128_pred(xa, xs + j * KC, x_lane);
+      if (BITS == 4) {  // stream mode has whole q4 chunks only (K % 64 == 0, checked on the host)
+        ldg128_pred(xb, xs + j * KC + 32, x_lane);
+        q4_chunk_mac(acc, cr, xa, xb);
       } else {
-        q8_chunk_mac(acc, regs[j], xa);
+        q8_chunk_mac(acc, cr, xa);
       }
     }
     xs += U * KC;
@@ -430,17 +428,19 @@ __device__ __forceinline__ bool stream_segment(const StackParams& sp, const Stac
   return true;
 }
 
-template <int M, int NW, int D, int PF>
+// SU: chunks per stage and per stream-K block (2 or 4; every product's
+// chunks per tile is a multiple of SU, checked on the host).
+template <int M, int NW, int D, int SU>
 __global__ void __launch_bounds__(NW * 32, 1) stream_kernel(const StackParams sp) {
-  static_assert(PF == 0, "stream mode prefetches through its ring only");
+  constexpr int SLOT = SU * Format<4>::kChunkBytes;  // the larger of the two formats
   extern __shared__ __align__(128) unsigned char smem[];
 
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
   const int pw = blockIdx.x * NW + warp;
   StreamRing rg;
-  rg.ring = smem_addr(smem + warp * D * kStackSlotBytes);
-  rg.bars = smem_addr(smem + NW * D * kStackSlotBytes) + warp * D * 8;
+  rg.ring = smem_addr(smem + warp * D * SLOT);
+  rg.bars = smem_addr(smem + NW * D * SLOT) + warp * D * 8;
 
   if (lane == 0) {
     for (int s = 0; s < D; ++s) mbar_init(rg.bars + 8 * s, 1);
@@ -460,11 +460,11 @@ __global__ void __launch_bounds__(NW * 32, 1) stream_kernel(const StackParams sp
     return;
   }
   const int e0 = entry_of_block(sp, gb);
-  StreamProducer pr;
+  StreamProducer<SU> pr;
   pr.left_total = ge - gb;
   pr.enter(sp, e0, gb - sp.entries[e0].blk_off);
   for (int s = 0; s < D; ++s) {
-    if (!pr.issue(sp, rg.ring + s * kStackSlotBytes, rg.bars + 8 * s, policy, lane)) break;
+    if (!pr.issue(sp, rg.ring + s * SLOT, rg.bars + 8 * s, policy, lane)) break;
     ++rg.in_flight;
   }
 
@@ -480,12 +480,12 @@ __global__ void __launch_bounds__(NW * 32, 1) stream_kernel(const StackParams sp
   StackEntryDev en = sp.entries[e];
   bool ok = true;
   while (left > 0) {
-    const long long in_entry = en.TC / kStackU - lb;
+    const long long in_entry = en.TC / SU - lb;
     const long long n = in_entry < left ? in_entry : left;
-    if (en.bits == 4) {  // stream mode has no product with a half-empty last chunk (checked on the host)
-      ok = stream_segment<4, M, false, D>(sp, en, e, lb, n, gb, rg, pr, policy, acc, pw, e_first, r_first, r, c, lane);
+    if (en.bits == 4) {
+      ok = stream_segment<4, M, D, SU>(sp, en, e, lb, n, gb, rg, pr, policy, acc, pw, e_first, r_first, r, c, lane);
     } else {
-      ok = stream_segment<8, M, false, D>(sp, en, e, lb, n, gb, rg, pr, policy, acc, pw, e_first, r_first, r, c, lane);
+      ok = stream_segment<8, M, D, SU>(sp, en, e, lb, n, gb, rg, pr, policy, acc, pw, e_first, r_first, r, c, lane);
     }
     if (!ok) break;
     left -= n;
@@ -510,12 +510,12 @@ __global__ void __launch_bounds__(NW * 32, 1) stream_kernel(const StackParams sp
   SplitTile first{nullptr, 0, -1, sp.counters, 0, 0}, last{nullptr, 0, -1, sp.counters, 0, 0};
   if (r_first >= 0) {
     const StackEntryDev& ef = sp.entries[e_first];
-    const int bpt = ef.C / kStackU;
+    const int bpt = ef.C / SU;
     const long long tile_g = ef.blk_off + static_cast<long long>(r_first) * bpt;
     first = SplitTile{ef.y, ef.N, r_first, sp.counters + ef.tile_off + r_first, tile_g, tile_g + bpt};
   }
   if (c != 0) {
-    const int bpt = en.C / kStackU;
+    const int bpt = en.C / SU;
     const long long tile_g = en.blk_off + static_cast<long long>(r) * bpt;
     last = SplitTile{en.y, en.N, r, sp.counters + en.tile_off + r, tile_g, tile_g + bpt};
     write_partial<M>(sp.partials, pw, tile_g <= gb ? 0 : 1, acc, lane);

@@ -15,6 +15,13 @@ MIXED = [
     Tensor("a", 4, 1000, 5120, 201), Tensor("b", 8, 37, 128, 202), Tensor("c", 4, 17, 17408, 203),
     Tensor("d", 8, 4099, 5120, 204), Tensor("e", 4, 64, 128, 205), Tensor("f", 4, 7168, 5120, 206),
 ]
+# every product's chunks per tile a multiple of 4: stream mode with stages of
+# four chunks (MIXED, with a q4 K of 128 = 2 chunks, uses stages of two)
+MIXED4 = [
+    Tensor("a4", 4, 1000, 5120, 221), Tensor("b4", 8, 37, 128, 222), Tensor("c4", 4, 17, 17408, 223),
+    Tensor("d4", 8, 4099, 5120, 224), Tensor("e4", 4, 64, 256, 225), Tensor("f4", 4, 7168, 5120, 226),
+    Tensor("g4", 8, 3, 256, 227),
+]
 # a q4 K that is an odd multiple of 32 (even chunk count): ordered persistent
 # mode, also when stream mode is asked for
 HALF = [Tensor("j", 4, 64, 96, 210), Tensor("k", 8, 100, 5120, 211)]
@@ -79,23 +86,24 @@ def test_stack_modes_equal_single_calls_and_oracle(q4, M):
         assert np.array_equal(a, b) and np.array_equal(a, c)
 
 
-@pytest.mark.parametrize("M", [1, 4])
-def test_stream_mode_of_independent_products(q4, M):
+@pytest.mark.parametrize("M", [1, 2, 4])
+@pytest.mark.parametrize("tensors", [MIXED, MIXED4], ids=["stages2", "stages4"])
+def test_stream_mode_of_independent_products(q4, M, tensors):
     """Stream mode splits the concatenated products between warps differently
     from one call per product: the outputs are compared with the oracle (every
     row) and with single calls within the product tolerance, and two runs are
     bitwise identical."""
     torch = H.torch()
-    st = workloads.DeviceStream(MIXED, M, flags=q4.Q4_STACK_INDEPENDENT)
+    st = workloads.DeviceStream(tensors, M, flags=q4.Q4_STACK_INDEPENDENT)
     assert st.stack.launches() == 1
     st.run()
     st.check()
-    first = [_y(st, i).copy() for i in range(len(MIXED))]
+    first = [_y(st, i).copy() for i in range(len(tensors))]
     for y in st.y:
         y.fill_(float("nan"))
     st.run()
     st.check()
-    for i, t in enumerate(MIXED):
+    for i, t in enumerate(tensors):
         assert np.array_equal(_y(st, i), first[i]), t.name
         q, s, x = _host_rows(st, i, 0, t.N)
         H.assert_parity(first[i], q, s, x, t.bits)

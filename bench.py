@@ -285,8 +285,9 @@ def run_ours(args, d: Dist):
     st.check()
     ms_step = d.max(ms / args.steps)
     value = wbytes * d.world / (ms_step * 1e6)  # GB/s over all ranks
-    launch_us = ms / args.steps / n_launch * 1e3  # this rank's own launches
-    achieved = wbytes / n_launch / (launch_us * 1e-6) / 1e9
+    # the step is one launch of stream_kernel, the dominant (only) kernel
+    step_us = ms / args.steps * 1e3  # this rank's own step
+    achieved = wbytes / (step_us * 1e-6) / 1e9
 
     # the same products with an ordering between consecutive products (each
     # product's outputs complete before the next reads its activations), as
@@ -390,8 +391,8 @@ def run_ours(args, d: Dist):
             "unit": "GB/s",
             "frac": round(achieved / peak, 4),
             "traffic": traffic,
-            "bytes_per_launch": wbytes // n_launch,
-            "launch_us": round(launch_us, 3),
+            "bytes_per_launch": wbytes,
+            "launch_us": round(step_us, 3),
             "launches_per_step": n_launch,
             "peak_kind": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs, copy burst)" if peak_kind == "measured" else peak_kind,
         },

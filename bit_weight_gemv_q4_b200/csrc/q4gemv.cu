@@ -519,6 +519,7 @@ struct q4_stack {
   void* fn = nullptr;
   int grid = 0, block = 0, smem = 0;
   q4k::StackParams params{};
+  bool cooperative = false;  // ordered mode: its grid barrier needs every CTA resident
   void* workspace = nullptr;
   size_t workspace_bytes = 0;
   int launches = 0;
@@ -618,6 +619,7 @@ int create_persistent(const q4_stack_entry* entries, int n, int M, int su, const
   st->workspace_bytes = kWsHeader + partials_bytes(dev) + counters;
   cudaError_t err = cudaMalloc(&st->workspace, st->workspace_bytes);
   if (err == cudaSuccess) err = cudaMemset(st->workspace, 0, st->workspace_bytes);
+  st->cooperative = !independent;
   if (err == cudaSuccess) err = cudaMalloc(&st->entries_dev, sizeof(q4k::StackEntryDev) * host.size());
   if (err == cudaSuccess)
     err = cudaMemcpy(st->entries_dev, host.data(), sizeof(q4k::StackEntryDev) * host.size(), cudaMemcpyHostToDevice);
@@ -750,13 +752,20 @@ extern "C" Q4_API int layer_stack_run(q4_stack* st, void* stream) {
     cfg.dynamicSmemBytes = static_cast<size_t>(st->smem);
     cfg.stream = s;
     cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeCooperative;  // all CTAs resident, or the launch fails
-    attr[0].val.cooperative = 1;
+    if (st->cooperative) {
+      attr[0].id = cudaLaunchAttributeCooperative;  // all CTAs resident, or the launch fails
+      attr[0].val.cooperative = 1;
+    } else {
+      // stream mode has no grid barrier: a plain launch that may start its
+      // weight copies while the previous kernel in the stream finishes
+      attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+      attr[0].val.programmaticStreamSerializationAllowed = 1;
+    }
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     void* args[] = {&st->params};
     cudaError_t err = cudaLaunchKernelExC(&cfg, st->fn, args);
-    return err == cudaSuccess ? Q4_OK : cuda_fail(err, "layer_stack_run: cooperative launch");
+    return err == cudaSuccess ? Q4_OK : cuda_fail(err, "layer_stack_run: persistent launch");
   }
   if (!st->exec) return Q4_OK;  // nothing to run
   cudaError_t err = cudaGraphLaunch(st->exec, s);

@@ -13,17 +13,15 @@
 //    stages completed on mbarriers, with an L2 evict-first hint (the weights
 //    are read once).  Lane 0 of each warp is that warp's producer.
 //  * Dequantisation happens in registers.  A 32-bit word of codes decodes to
-//    four bf16 pairs with one mask-and-or each: the code u becomes the
-//    mantissa of 128 + u, an exact integer q + c (c = 136 for q4; for q8 the
-//    byte is split into a (2048 + 16 u_hi) and a (128 + u_lo) part, summing
-//    to q + 2304).  The pairs are already the A fragments of mma.sync
-//    m16n8k16 (bf16 in, fp32 accumulate) and the activations are its B
-//    fragments (columns >= M are never stored).  The offset c is removed
-//    inside the tensor core: each group's accumulator starts from (-c) * x,
-//    one product of a constant matrix with the same B fragment, shared by the
-//    two 16-row halves of the chunk.  Every product of a <= 12-bit integer
-//    and a bf16 is exact; each group's fp32 sum is scaled by its fp16 scale
-//    with one fp32 FMA per output.
+//    four bf16 pairs with one mask-and-or and one bf16x2 subtraction each:
+//    the code u becomes the mantissa of 128 + u, and subtracting 128 + the
+//    code offset leaves the integer q exactly (for q8 the byte is split into
+//    a 16 u_hi - 128 and a u_lo part that sum to q).  The pairs are already
+//    the A fragments of mma.sync m16n8k16 (bf16 in, fp32 accumulate) and the
+//    activations are its B fragments (columns >= M are never stored).  Every
+//    product of a <= 8-bit integer and a bf16 is exact, so a group's fp32
+//    sum errs only relative to sum |q x|; it is scaled by its fp16 scale with
+//    one fp32 FMA per output.
 //  * Tiles split between warps are finished deterministically: each warp
 //    writes its partial sums to the workspace, and the last of the tile's
 //    warps to arrive (an integer counter) adds them in fixed warp order,
@@ -225,33 +223,45 @@ __device__ __forceinline__ float2 half2_bits_to_float2(uint32_t h2) {
 // In-register dequantisation (shared by the product and the debug decoder)
 // ----------------------------------------------------------------------------
 constexpr uint32_t kNibbleMask = 0x000F000Fu;
-constexpr uint32_t kBf16_128 = 0x43004300u;    // bf16 pair (128, 128): mantissa LSB = 1
-constexpr uint32_t kBf16_2048 = 0x45004500u;   // (2048, 2048): mantissa LSB = 16
-constexpr uint32_t kBf16_m136 = 0xC308C308u;   // (-136, -136): removes the q4 offset 128 + 8
-constexpr uint32_t kBf16_m2304 = 0xC510C510u;  // (-2304, -2304): removes the q8 offset 2048 + 128 + 128
-constexpr int kQ4Offset = 136;
-constexpr int kQ8Offset = 2304;
+constexpr uint32_t kBf16_128 = 0x43004300u;   // bf16 pair (128, 128): mantissa LSB = 1
+constexpr uint32_t kBf16_2048 = 0x45004500u;  // (2048, 2048): mantissa LSB = 16
+constexpr uint32_t kBf16_136 = 0x43084308u;   // (136, 136) = 128 + the q4 code offset 8
+constexpr uint32_t kBf16_2176 = 0x45084508u;  // (2176, 2176) = 2048 + the q8 code offset 128
 
-// One q4 word -> A fragment registers a[0..3] holding exact integers q + 136.
-// a[i] takes nibbles i and i + 4 (bits 4i and 16 + 4i).
-__device__ __forceinline__ void dequant_q4_word(uint32_t w, uint32_t (&a)[4]) {
-  a[0] = lop3_and_or(w, kNibbleMask, kBf16_128);
-  a[1] = lop3_and_or(w >> 4, kNibbleMask, kBf16_128);
-  a[2] = lop3_and_or(w >> 8, kNibbleMask, kBf16_128);
-  a[3] = lop3_and_or(w >> 12, kNibbleMask, kBf16_128);
+// a - b on bf16 pairs.  Used only where the result is an exactly
+// representable small integer, so the rounding mode never matters.
+__device__ __forceinline__ uint32_t bf16x2_sub(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("sub.rn.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
 }
 
-// Two q8 words (one m16n8k16 block) -> A fragments hi, lo with
-// hi + lo = q + 2304 exactly: hi = 2048 + 16 u_hi, lo = 128 + u_lo, u = q + 128.
+// One q4 word -> A fragment registers a[0..3] holding the codes q exactly as
+// bf16.  a[i] takes nibbles i and i + 4 (bits 4i and 16 + 4i).  The mask-and-
+// or makes the nibble u = q + 8 the mantissa of 128 + u; subtracting 136
+// leaves q, exact in bf16.  (Removing the offset here, not after the
+// accumulation, keeps every product q * x and every partial sum free of the
+// offset, so the fp32 sums err only relative to sum |q x|: an all-zero row
+// gives exactly 0.)
+__device__ __forceinline__ void dequant_q4_word(uint32_t w, uint32_t (&a)[4]) {
+  a[0] = bf16x2_sub(lop3_and_or(w, kNibbleMask, kBf16_128), kBf16_136);
+  a[1] = bf16x2_sub(lop3_and_or(w >> 4, kNibbleMask, kBf16_128), kBf16_136);
+  a[2] = bf16x2_sub(lop3_and_or(w >> 8, kNibbleMask, kBf16_128), kBf16_136);
+  a[3] = bf16x2_sub(lop3_and_or(w >> 12, kNibbleMask, kBf16_128), kBf16_136);
+}
+
+// Two q8 words (one m16n8k16 block) -> A fragments hi, lo with hi + lo = q
+// exactly: the byte u = q + 128 = 16 u_hi + u_lo gives hi = 16 u_hi - 128
+// (from 2048 + 16 u_hi) and lo = u_lo (from 128 + u_lo), both exact in bf16.
 __device__ __forceinline__ void dequant_q8_block(uint32_t w0, uint32_t w1, uint32_t (&hi)[4], uint32_t (&lo)[4]) {
-  lo[0] = lop3_and_or(w0, kNibbleMask, kBf16_128);
-  lo[1] = lop3_and_or(w0 >> 8, kNibbleMask, kBf16_128);
-  lo[2] = lop3_and_or(w1, kNibbleMask, kBf16_128);
-  lo[3] = lop3_and_or(w1 >> 8, kNibbleMask, kBf16_128);
-  hi[0] = lop3_and_or(w0 >> 4, kNibbleMask, kBf16_2048);
-  hi[1] = lop3_and_or(w0 >> 12, kNibbleMask, kBf16_2048);
-  hi[2] = lop3_and_or(w1 >> 4, kNibbleMask, kBf16_2048);
-  hi[3] = lop3_and_or(w1 >> 12, kNibbleMask, kBf16_2048);
+  lo[0] = bf16x2_sub(lop3_and_or(w0, kNibbleMask, kBf16_128), kBf16_128);
+  lo[1] = bf16x2_sub(lop3_and_or(w0 >> 8, kNibbleMask, kBf16_128), kBf16_128);
+  lo[2] = bf16x2_sub(lop3_and_or(w1, kNibbleMask, kBf16_128), kBf16_128);
+  lo[3] = bf16x2_sub(lop3_and_or(w1 >> 8, kNibbleMask, kBf16_128), kBf16_128);
+  hi[0] = bf16x2_sub(lop3_and_or(w0 >> 4, kNibbleMask, kBf16_2048), kBf16_2176);
+  hi[1] = bf16x2_sub(lop3_and_or(w0 >> 12, kNibbleMask, kBf16_2048), kBf16_2176);
+  hi[2] = bf16x2_sub(lop3_and_or(w1 >> 4, kNibbleMask, kBf16_2048), kBf16_2176);
+  hi[3] = bf16x2_sub(lop3_and_or(w1 >> 12, kNibbleMask, kBf16_2048), kBf16_2176);
 }
 
 // ----------------------------------------------------------------------------
@@ -265,21 +275,18 @@ struct ChunkRegs {
 
 __device__ __forceinline__ void q4_chunk_mac(float (&acc)[2][4], const ChunkRegs& r, const uint4& xa,
                                              const uint4& xb) {
-  const uint32_t cst[4] = {kBf16_m136, kBf16_m136, kBf16_m136, kBf16_m136};
   const uint32_t sc[4] = {r.scales.x, r.scales.y, r.scales.z, r.scales.w};
+  const float zero[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-  for (int G = 0; G < 2; ++G) {
+  for (int G = 0; G < 2; ++G) {  // the chunk's two groups
     const uint4& xg = G ? xb : xa;
-    float corr[4] = {0.f, 0.f, 0.f, 0.f};  // -136 * (sum of x over the group), every row
-    mma_bf16_m16n8k16(corr, cst, xg.x, xg.y);
-    mma_bf16_m16n8k16(corr, cst, xg.z, xg.w);
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
       const uint4& w = r.codes[h];
       float d[4];
       uint32_t a[4];
       dequant_q4_word(G ? w.z : w.x, a);
-      mma_bf16_m16n8k16_c(d, a, xg.x, xg.y, corr);
+      mma_bf16_m16n8k16_c(d, a, xg.x, xg.y, zero);
       dequant_q4_word(G ? w.w : w.y, a);
       mma_bf16_m16n8k16(d, a, xg.z, xg.w);
       const float2 s_r = half2_bits_to_float2(sc[2 * h]);       // row 16h + gi: groups 2c, 2c+1
@@ -295,17 +302,14 @@ __device__ __forceinline__ void q4_chunk_mac(float (&acc)[2][4], const ChunkRegs
 }
 
 __device__ __forceinline__ void q8_chunk_mac(float (&acc)[2][4], const ChunkRegs& r, const uint4& xa) {
-  const uint32_t cst[4] = {kBf16_m2304, kBf16_m2304, kBf16_m2304, kBf16_m2304};
-  float corr[4] = {0.f, 0.f, 0.f, 0.f};  // -2304 * (sum of x over the group), every row
-  mma_bf16_m16n8k16(corr, cst, xa.x, xa.y);
-  mma_bf16_m16n8k16(corr, cst, xa.z, xa.w);
+  const float zero[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
   for (int h = 0; h < 2; ++h) {
     const uint4& w = r.codes[h];
     float d[4];
     uint32_t hi[4], lo[4];
     dequant_q8_block(w.x, w.y, hi, lo);
-    mma_bf16_m16n8k16_c(d, hi, xa.x, xa.y, corr);
+    mma_bf16_m16n8k16_c(d, hi, xa.x, xa.y, zero);
     mma_bf16_m16n8k16(d, lo, xa.x, xa.y);
     dequant_q8_block(w.z, w.w, hi, lo);
     mma_bf16_m16n8k16(d, hi, xa.z, xa.w);
@@ -696,8 +700,8 @@ __global__ void unpack_kernel(const uint8_t* packed, long long N, long long K, i
         for (int reg = 0; reg < 4; ++reg) {
           const long long row = R + 8 * (reg & 1);
           const long long col = kb + 2 * (reg >> 1);
-          put(row, col, bf16_bits_to_int(a[reg]) - kQ4Offset);
-          put(row, col + 1, bf16_bits_to_int(a[reg] >> 16) - kQ4Offset);
+          put(row, col, bf16_bits_to_int(a[reg]));
+          put(row, col + 1, bf16_bits_to_int(a[reg] >> 16));
         }
       }
     } else {
@@ -708,8 +712,8 @@ __global__ void unpack_kernel(const uint8_t* packed, long long N, long long K, i
         for (int reg = 0; reg < 4; ++reg) {
           const long long row = R + 8 * (reg & 1);
           const long long col = kb + 2 * (reg >> 1);
-          put(row, col, bf16_bits_to_int(hi[reg]) + bf16_bits_to_int(lo[reg]) - kQ8Offset);
-          put(row, col + 1, bf16_bits_to_int(hi[reg] >> 16) + bf16_bits_to_int(lo[reg] >> 16) - kQ8Offset);
+          put(row, col, bf16_bits_to_int(hi[reg]) + bf16_bits_to_int(lo[reg]));
+          put(row, col + 1, bf16_bits_to_int(hi[reg] >> 16) + bf16_bits_to_int(lo[reg] >> 16));
         }
       }
     }

@@ -73,3 +73,33 @@ def assert_parity(y, q, s, x, bits, rel=1e-3, abs_=1e-6):
         details = [(tuple(i), float(y[tuple(i)]), float(y_ref[tuple(i)]), float(bound[tuple(i)])) for i in idx]
         raise AssertionError(f"{(~ok).sum()} of {ok.size} outside tolerance; first (idx, y, y_ref, bound): {details}")
     return float((err / np.maximum(B, 1e-30)).max()) if B.size else 0.0
+
+
+def degenerate_rows(bits, N, K, seed=3):
+    """Canonical q/s with degenerate rows: every fourth row all zero (nonzero
+    scales), the next holds a single nonzero code, the next is zero except for
+    one group, the rest random.  The tolerance allows only 1e-6 on a zero row."""
+    q, s = synth.tensor(bits, seed, 40, N, K)
+    q = q.copy()
+    rng = np.random.default_rng(seed)
+    for r in range(N):
+        kind = r % 4
+        if kind == 3:
+            continue
+        q[r] = 0
+        if kind == 1:
+            k = int(rng.integers(0, K))
+            v = 7 if bits == 4 else 127
+            if bits == 4:
+                q[r, k // 2] = (v & 0xF) << (4 * (k % 2))
+            else:
+                q[r, k] = v
+        elif kind == 2:
+            g = int(rng.integers(0, K // 32))
+            vals = rng.integers(-8, 8, 32) if bits == 4 else rng.integers(-127, 128, 32)
+            if bits == 4:
+                nib = (vals & 0xF).astype(np.uint8)
+                q[r, 16 * g: 16 * g + 16] = nib[0::2] | (nib[1::2] << 4)
+            else:
+                q[r, 32 * g: 32 * g + 32] = vals.astype(np.int8)
+    return q, s

@@ -261,3 +261,14 @@ def test_bad_workspace_is_rejected(q4):
     with pytest.raises(q4.Q4Error) as e:
         q4.q4_gemv(packed, N, K, H.to_device_x(x), 1, y, small)
     assert e.value.code == q4.Q4_ERR_BUFFER_TOO_SMALL
+
+
+@pytest.mark.parametrize("bits", [4, 8])
+@pytest.mark.parametrize("M", [1, 4])
+def test_degenerate_rows(q4, bits, M):
+    N, K = 96, 5120
+    q, s = H.degenerate_rows(bits, N, K)
+    x = synth.activations(3, synth.act_stream(41), M, K)
+    y, ok = H.run_gemv(bits, H.to_device_packed(bits, q, s, N, K), N, K, H.to_device_x(x), M)
+    assert ok
+    H.assert_parity(y, q, s, x, bits)

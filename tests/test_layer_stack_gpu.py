@@ -152,3 +152,30 @@ def test_full_decode_stream_sampled(q4, M, mode):
         assert np.all(np.isfinite(y)), t.name
     st.close()
     torch.cuda.empty_cache()
+
+
+@pytest.mark.parametrize("mode", ["ordered", "stream", "graph"])
+@pytest.mark.parametrize("M", [1, 3])
+def test_degenerate_rows_in_stacks(q4, mode, M):
+    """All-zero rows (nonzero scales), single-code rows and one-group rows in
+    every stack mode: within the tolerance, which is 1e-6 on a zero row."""
+    torch = H.torch()
+    K = 5120
+    specs = [(4, 96), (8, 64)]
+    x = synth.activations(5, synth.act_stream(42), M, K)
+    x_dev = H.to_device_x(x)
+    entries, hosts, ys = [], [], []
+    for bits, N in specs:
+        q, s = H.degenerate_rows(bits, N, K, seed=bits)
+        y = torch.full((M * N,), float("nan"), dtype=torch.float32, device="cuda")
+        entries.append((bits, N, K, H.to_device_packed(bits, q, s, N, K), x_dev, y))
+        hosts.append((q, s))
+        ys.append(y)
+    flags = {"ordered": 0, "stream": q4.Q4_STACK_INDEPENDENT, "graph": q4.Q4_STACK_GRAPH}[mode]
+    st = q4.layer_stack_create(entries, M, flags)
+    q4.layer_stack_run(st)
+    q4.layer_stack_check(st)
+    torch.cuda.synchronize()
+    for (bits, N), (q, s), y in zip(specs, hosts, ys):
+        H.assert_parity(y.cpu().numpy().reshape(M, N), q, s, x, bits)
+    st.close()

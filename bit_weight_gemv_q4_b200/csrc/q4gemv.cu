@@ -520,6 +520,11 @@ struct q4_stack {
   int grid = 0, block = 0, smem = 0;
   q4k::StackParams params{};
   bool cooperative = false;  // ordered mode: its grid barrier needs every CTA resident
+  // stream mode: one activation preparation per distinct (x, K), run before
+  // the stream kernel on every layer_stack_run
+  q4k::XPrepJob* xprep_dev = nullptr;
+  int xprep_jobs = 0;
+  int M = 1;
   void* workspace = nullptr;
   size_t workspace_bytes = 0;
   int launches = 0;
@@ -557,6 +562,7 @@ void free_stack(q4_stack* st) {
   if (st->exec) cudaGraphExecDestroy(st->exec);
   if (st->graph) cudaGraphDestroy(st->graph);
   if (st->entries_dev) cudaFree(st->entries_dev);
+  if (st->xprep_dev) cudaFree(st->xprep_dev);
   if (st->workspace) cudaFree(st->workspace);
   delete st;
 }
@@ -616,10 +622,50 @@ int create_persistent(const q4_stack_entry* entries, int n, int M, int su, const
   // ordered mode re-uses one counter per tile of the largest product; stream
   // mode keeps one per tile of every product
   const size_t counters = (static_cast<size_t>(independent ? total_tiles : max_t) * 4 + 255) / 256 * 256;
-  st->workspace_bytes = kWsHeader + partials_bytes(dev) + counters;
+  // stream mode: per distinct (x, K) an fp16 copy [M][K] and its XInfo
+  std::vector<q4k::XPrepJob> jobs;
+  std::vector<size_t> job_of(static_cast<size_t>(n), 0), x16_off, info_off;
+  size_t prep_bytes = 0;
+  if (independent) {
+    for (int i = 0; i < n; ++i) {
+      size_t jdx = jobs.size();
+      for (size_t k = 0; k < jobs.size(); ++k)
+        if (jobs[k].x == entries[i].x && jobs[k].K == entries[i].K) jdx = k;
+      if (jdx == jobs.size()) {
+        q4k::XPrepJob j{};
+        j.x = entries[i].x;
+        j.K = entries[i].K;
+        jobs.push_back(j);
+        x16_off.push_back(prep_bytes);
+        prep_bytes += (static_cast<size_t>(M) * entries[i].K * 2 + 255) / 256 * 256;
+        info_off.push_back(prep_bytes);
+        prep_bytes += 256;
+      }
+      job_of[static_cast<size_t>(i)] = jdx;
+    }
+  }
+  const size_t prep_base = kWsHeader + partials_bytes(dev) + counters;
+  st->workspace_bytes = prep_base + prep_bytes;
   cudaError_t err = cudaMalloc(&st->workspace, st->workspace_bytes);
   if (err == cudaSuccess) err = cudaMemset(st->workspace, 0, st->workspace_bytes);
   st->cooperative = !independent;
+  st->M = M;
+  if (independent && err == cudaSuccess) {
+    unsigned char* base = static_cast<unsigned char*>(st->workspace) + prep_base;
+    for (size_t k = 0; k < jobs.size(); ++k) {
+      jobs[k].x16 = reinterpret_cast<uint16_t*>(base + x16_off[k]);
+      jobs[k].info = reinterpret_cast<q4k::XInfo*>(base + info_off[k]);
+    }
+    for (int i = 0; i < n; ++i) {
+      const q4k::XPrepJob& j = jobs[job_of[static_cast<size_t>(i)]];
+      host[static_cast<size_t>(i)].x16 = j.x16;
+      host[static_cast<size_t>(i)].xinfo = j.info;
+    }
+    err = cudaMalloc(&st->xprep_dev, sizeof(q4k::XPrepJob) * jobs.size());
+    if (err == cudaSuccess)
+      err = cudaMemcpy(st->xprep_dev, jobs.data(), sizeof(q4k::XPrepJob) * jobs.size(), cudaMemcpyHostToDevice);
+    st->xprep_jobs = static_cast<int>(jobs.size());
+  }
   if (err == cudaSuccess) err = cudaMalloc(&st->entries_dev, sizeof(q4k::StackEntryDev) * host.size());
   if (err == cudaSuccess)
     err = cudaMemcpy(st->entries_dev, host.data(), sizeof(q4k::StackEntryDev) * host.size(), cudaMemcpyHostToDevice);
@@ -647,7 +693,7 @@ int create_persistent(const q4_stack_entry* entries, int n, int M, int su, const
   p.TBg = total_blocks;
   p.Pg = static_cast<int>(total_blocks < warps ? total_blocks : warps);
   st->persistent = true;
-  st->launches = 1;
+  st->launches = independent ? 2 : 1;  // stream mode: xprep_kernel + stream_kernel
   return Q4_OK;
 }
 
@@ -756,8 +802,13 @@ extern "C" Q4_API int layer_stack_run(q4_stack* st, void* stream) {
       attr[0].id = cudaLaunchAttributeCooperative;  // all CTAs resident, or the launch fails
       attr[0].val.cooperative = 1;
     } else {
-      // stream mode has no grid barrier: a plain launch that may start its
-      // weight copies while the previous kernel in the stream finishes
+      // stream mode: the activation preparation, then the stream kernel,
+      // which has no grid barrier: a plain launch that starts its weight
+      // copies while xprep_kernel runs and waits for it (griddepcontrol.wait)
+      // before it reads an activation
+      q4k::xprep_kernel<<<st->xprep_jobs, q4k::kXPrepThreads, 0, s>>>(st->xprep_dev, st->M);
+      cudaError_t perr = cudaGetLastError();
+      if (perr != cudaSuccess) return cuda_fail(perr, "layer_stack_run: xprep_kernel launch");
       attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
       attr[0].val.programmaticStreamSerializationAllowed = 1;
     }

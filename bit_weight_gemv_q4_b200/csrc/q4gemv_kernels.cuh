@@ -196,23 +196,42 @@ __device__ __forceinline__ uint32_t lop3_and_or(uint32_t a, uint32_t mask, uint3
   return d;
 }
 
-// D += A (16x16, bf16, row) * B (16x8, bf16, col), fp32 accumulators.
-__device__ __forceinline__ void mma_bf16_m16n8k16(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 "
-      "{%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
-      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+// D += A (16x16, row) * B (16x8, col), fp32 accumulators; A and B both bf16
+// (F16 = false) or both fp16 (F16 = true).
+template <bool F16 = false>
+__device__ __forceinline__ void mma_m16n8k16(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  if constexpr (F16) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 "
+        "{%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+  } else {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 "
+        "{%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+  }
 }
 
-// D = A * B + C with separate C registers (no copies of C into D).
-__device__ __forceinline__ void mma_bf16_m16n8k16_c(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1,
-                                                    const float (&c)[4]) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 "
-      "{%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, {%10, %11, %12, %13};"
-      : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
-      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1), "f"(c[0]), "f"(c[1]), "f"(c[2]), "f"(c[3]));
+// D = A * B (no accumulator input).
+template <bool F16 = false>
+__device__ __forceinline__ void mma_m16n8k16_first(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  const float z = 0.f;
+  if constexpr (F16) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 "
+        "{%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, {%10, %10, %10, %10};"
+        : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1), "f"(z));
+  } else {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 "
+        "{%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, {%10, %10, %10, %10};"
+        : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1), "f"(z));
+  }
 }
 
 __device__ __forceinline__ float2 half2_bits_to_float2(uint32_t h2) {
@@ -264,6 +283,50 @@ __device__ __forceinline__ void dequant_q8_block(uint32_t w0, uint32_t w1, uint3
   hi[3] = bf16x2_sub(lop3_and_or(w1 >> 12, kNibbleMask, kBf16_2048), kBf16_2176);
 }
 
+// fp16 decode (activations in fp16, see xprep_kernel).  fp16 has 10
+// mantissa bits, so a nibble sits in the mantissa of 1024 + v at bits 0-3 or
+// 4-7 without a shift, and a q8 byte at bits 0-7.
+constexpr uint32_t kNibbleMaskHi = 0x00F000F0u;
+constexpr uint32_t kByteMask = 0x00FF00FFu;
+constexpr uint32_t kF16_1024 = 0x64006400u;   // fp16 pair (1024, 1024): mantissa LSB = 1
+constexpr uint32_t kF16_1032 = 0x64086408u;   // (1032, 1032) = 1024 + the q4 code offset 8
+constexpr uint32_t kF16_1152 = 0x64806480u;   // (1152, 1152) = 1024 + the q8 code offset 128
+constexpr uint32_t kF16_1_16 = 0x2C002C00u;   // (1/16, 1/16)
+constexpr uint32_t kF16_m72 = 0xD480D480u;    // (-72, -72) = -(1024 / 16 + 8)
+
+// a - b and a * b + c on fp16 pairs, used only where the result is an exactly
+// representable small integer.
+__device__ __forceinline__ uint32_t f16x2_sub(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+__device__ __forceinline__ uint32_t f16x2_fma(uint32_t a, uint32_t b, uint32_t c) {
+  uint32_t d;
+  asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+  return d;
+}
+
+// One q4 word -> the same four A fragments as dequant_q4_word, in fp16: the
+// nibbles at bits 4-7 of each half become 1024 + 16 u, brought to q by
+// (v / 16) - 72; one shift instead of three.
+__device__ __forceinline__ void dequant_q4_word_f16(uint32_t w, uint32_t (&a)[4]) {
+  const uint32_t t = w >> 8;
+  a[0] = f16x2_sub(lop3_and_or(w, kNibbleMask, kF16_1024), kF16_1032);
+  a[1] = f16x2_fma(lop3_and_or(w, kNibbleMaskHi, kF16_1024), kF16_1_16, kF16_m72);
+  a[2] = f16x2_sub(lop3_and_or(t, kNibbleMask, kF16_1024), kF16_1032);
+  a[3] = f16x2_fma(lop3_and_or(t, kNibbleMaskHi, kF16_1024), kF16_1_16, kF16_m72);
+}
+
+// Two q8 words -> the four A fragments of one m16n8k16 block holding q
+// exactly (a[0], a[1] from w0's bytes (0, 2) and (1, 3); a[2], a[3] from w1).
+__device__ __forceinline__ void dequant_q8_block_f16(uint32_t w0, uint32_t w1, uint32_t (&a)[4]) {
+  a[0] = f16x2_sub(lop3_and_or(w0, kByteMask, kF16_1024), kF16_1152);
+  a[1] = f16x2_sub(lop3_and_or(w0 >> 8, kByteMask, kF16_1024), kF16_1152);
+  a[2] = f16x2_sub(lop3_and_or(w1, kByteMask, kF16_1024), kF16_1152);
+  a[3] = f16x2_sub(lop3_and_or(w1 >> 8, kByteMask, kF16_1024), kF16_1152);
+}
+
 // ----------------------------------------------------------------------------
 // One chunk's contribution to this lane's accumulators acc[h][0..3]
 // (half h: rows 16h + gi and 16h + gi + 8 of the tile; columns 2ti, 2ti + 1).
@@ -273,10 +336,12 @@ struct ChunkRegs {
   uint4 scales;    // q4: (R0: 2c, 2c+1) (R0+8) (R1) (R1+8);  q8: .x = (R0, R0+8), .y = (R1, R1+8)
 };
 
+// F16: activations and codes in fp16 (xprep_kernel made x fp16-exact),
+// else bf16.
+template <bool F16 = false>
 __device__ __forceinline__ void q4_chunk_mac(float (&acc)[2][4], const ChunkRegs& r, const uint4& xa,
                                              const uint4& xb) {
   const uint32_t sc[4] = {r.scales.x, r.scales.y, r.scales.z, r.scales.w};
-  const float zero[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
   for (int G = 0; G < 2; ++G) {  // the chunk's two groups
     const uint4& xg = G ? xb : xa;
@@ -285,10 +350,10 @@ __device__ __forceinline__ void q4_chunk_mac(float (&acc)[2][4], const ChunkRegs
       const uint4& w = r.codes[h];
       float d[4];
       uint32_t a[4];
-      dequant_q4_word(G ? w.z : w.x, a);
-      mma_bf16_m16n8k16_c(d, a, xg.x, xg.y, zero);
-      dequant_q4_word(G ? w.w : w.y, a);
-      mma_bf16_m16n8k16(d, a, xg.z, xg.w);
+      if constexpr (F16) dequant_q4_word_f16(G ? w.z : w.x, a); else dequant_q4_word(G ? w.z : w.x, a);
+      mma_m16n8k16_first<F16>(d, a, xg.x, xg.y);
+      if constexpr (F16) dequant_q4_word_f16(G ? w.w : w.y, a); else dequant_q4_word(G ? w.w : w.y, a);
+      mma_m16n8k16<F16>(d, a, xg.z, xg.w);
       const float2 s_r = half2_bits_to_float2(sc[2 * h]);       // row 16h + gi: groups 2c, 2c+1
       const float2 s_r8 = half2_bits_to_float2(sc[2 * h + 1]);  // row 16h + gi + 8
       const float sr = G ? s_r.y : s_r.x;
@@ -301,19 +366,27 @@ __device__ __forceinline__ void q4_chunk_mac(float (&acc)[2][4], const ChunkRegs
   }
 }
 
+template <bool F16 = false>
 __device__ __forceinline__ void q8_chunk_mac(float (&acc)[2][4], const ChunkRegs& r, const uint4& xa) {
-  const float zero[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
   for (int h = 0; h < 2; ++h) {
     const uint4& w = r.codes[h];
     float d[4];
-    uint32_t hi[4], lo[4];
-    dequant_q8_block(w.x, w.y, hi, lo);
-    mma_bf16_m16n8k16_c(d, hi, xa.x, xa.y, zero);
-    mma_bf16_m16n8k16(d, lo, xa.x, xa.y);
-    dequant_q8_block(w.z, w.w, hi, lo);
-    mma_bf16_m16n8k16(d, hi, xa.z, xa.w);
-    mma_bf16_m16n8k16(d, lo, xa.z, xa.w);
+    if constexpr (F16) {
+      uint32_t a[4];
+      dequant_q8_block_f16(w.x, w.y, a);
+      mma_m16n8k16_first<true>(d, a, xa.x, xa.y);
+      dequant_q8_block_f16(w.z, w.w, a);
+      mma_m16n8k16<true>(d, a, xa.z, xa.w);
+    } else {
+      uint32_t hi[4], lo[4];
+      dequant_q8_block(w.x, w.y, hi, lo);
+      mma_m16n8k16_first<false>(d, hi, xa.x, xa.y);
+      mma_m16n8k16<false>(d, lo, xa.x, xa.y);
+      dequant_q8_block(w.z, w.w, hi, lo);
+      mma_m16n8k16<false>(d, hi, xa.z, xa.w);
+      mma_m16n8k16<false>(d, lo, xa.z, xa.w);
+    }
     const float2 s = half2_bits_to_float2(h ? r.scales.y : r.scales.x);  // rows 16h + gi, 16h + gi + 8
     acc[h][0] = fmaf(s.x, d[0], acc[h][0]);
     acc[h][1] = fmaf(s.x, d[1], acc[h][1]);
@@ -668,6 +741,10 @@ __global__ void __launch_bounds__(NW * 32, 1) gemv_kernel(const GemvParams p) {
 // Debug decoder: one warp per chunk, using the same in-register dequantisation
 // as the product kernel; writes int8 q [N][K] and fp16 scales [N][K/32].
 // ----------------------------------------------------------------------------
+__device__ __forceinline__ int f16_bits_to_int(uint32_t h) {
+  return static_cast<int>(__half2float(__ushort_as_half(static_cast<unsigned short>(h & 0xFFFF))));
+}
+
 __device__ __forceinline__ int bf16_bits_to_int(uint32_t h) {
   const uint16_t b = static_cast<uint16_t>(h & 0xFFFF);
   return static_cast<int>(__bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(&b)));
@@ -691,29 +768,35 @@ __global__ void unpack_kernel(const uint8_t* packed, long long N, long long K, i
     const uint4 codes = *reinterpret_cast<const uint4*>(base + kHalfBytes * h + 16 * lane);
     const uint32_t w[4] = {codes.x, codes.y, codes.z, codes.w};
     const long long R = static_cast<long long>(t) * kTileRows + 16 * h + gi;
+    // the bf16 and the fp16 decode must agree; a disagreement writes -128,
+    // a value neither format holds
+    auto both = [](int qb, int qh) { return qb == qh ? qb : -128; };
     if (BITS == 4) {
       for (int j = 0; j < 4; ++j) {
-        uint32_t a[4];
+        uint32_t a[4], af[4];
         dequant_q4_word(w[j], a);
+        dequant_q4_word_f16(w[j], af);
         const long long kb = 64LL * c + 32 * (j >> 1) + 8 * ti + 4 * (j & 1);
         // a[0]: row R, k kb, kb+1; a[1]: row R+8; a[2]: row R, kb+2, kb+3; a[3]: row R+8
         for (int reg = 0; reg < 4; ++reg) {
           const long long row = R + 8 * (reg & 1);
           const long long col = kb + 2 * (reg >> 1);
-          put(row, col, bf16_bits_to_int(a[reg]));
-          put(row, col + 1, bf16_bits_to_int(a[reg] >> 16));
+          put(row, col, both(bf16_bits_to_int(a[reg]), f16_bits_to_int(af[reg])));
+          put(row, col + 1, both(bf16_bits_to_int(a[reg] >> 16), f16_bits_to_int(af[reg] >> 16)));
         }
       }
     } else {
       for (int blk = 0; blk < 2; ++blk) {
-        uint32_t hi[4], lo[4];
+        uint32_t hi[4], lo[4], af[4];
         dequant_q8_block(w[2 * blk], w[2 * blk + 1], hi, lo);
+        dequant_q8_block_f16(w[2 * blk], w[2 * blk + 1], af);
         const long long kb = 32LL * c + 8 * ti + 4 * blk;
         for (int reg = 0; reg < 4; ++reg) {
           const long long row = R + 8 * (reg & 1);
           const long long col = kb + 2 * (reg >> 1);
-          put(row, col, bf16_bits_to_int(hi[reg]) + bf16_bits_to_int(lo[reg]));
-          put(row, col + 1, bf16_bits_to_int(hi[reg] >> 16) + bf16_bits_to_int(lo[reg] >> 16));
+          put(row, col, both(bf16_bits_to_int(hi[reg]) + bf16_bits_to_int(lo[reg]), f16_bits_to_int(af[reg])));
+          put(row, col + 1,
+              both(bf16_bits_to_int(hi[reg] >> 16) + bf16_bits_to_int(lo[reg] >> 16), f16_bits_to_int(af[reg] >> 16)));
         }
       }
     }

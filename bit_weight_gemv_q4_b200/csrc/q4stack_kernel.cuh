@@ -20,14 +20,38 @@
 //    (bounded) and exits; the other CTAs' barrier waits then give up too.
 #pragma once
 
+#include <climits>
+
 #include "q4gemv_kernels.cuh"
 
 namespace q4k {
+
+// Activation preparation for stream mode (xprep_kernel).  An activation
+// tensor is used in fp16 when a power of two 2^sigma exists with every
+// x * 2^-sigma exactly representable in fp16: then x16 = x * 2^-sigma, and
+// outputs computed from x16 are multiplied back by scale = 2^sigma (exact).
+// Otherwise (a dynamic range beyond fp16's, inf or NaN) ok = 0 and the
+// products of that tensor use the bf16 path on x itself.
+struct XInfo {
+  int ok;
+  int sigma;
+  float scale;
+  int pad;
+};
+
+struct XPrepJob {
+  const uint16_t* x;  // bf16 [M][K]
+  uint16_t* x16;      // fp16 [M][K]
+  XInfo* info;
+  long long K;
+};
 
 struct StackEntryDev {
   const uint8_t* packed;
   const uint16_t* x;
   float* y;
+  const uint16_t* x16;   // stream mode: fp16 copy of x (valid when xinfo->ok)
+  const XInfo* xinfo;    // stream mode
   long long N, K, TC;
   long long blk_off;  // first block of this product in the concatenated sequence (stream mode)
   int T, C, bits, P, khalf;
@@ -291,6 +315,80 @@ __global__ void __launch_bounds__(NW * 32, 1) stack_kernel(const StackParams sp)
 }
 
 // ----------------------------------------------------------------------------
+// xprep_kernel: one CTA per activation tensor.  Finds the largest binary
+// exponent emax and the lowest set significand bit lsb over the nonzero
+// elements; with sigma = emax - 15 every element scaled by 2^-sigma is below
+// 2^16 in magnitude (fp16 max 65504 > 1.9921875 * 2^15), and it is exact in
+// fp16 when its lowest set bit is at least 2^-24 (the fp16 subnormal step):
+// lsb - sigma >= -24 for every element.
+// ----------------------------------------------------------------------------
+constexpr int kXPrepThreads = 1024;
+
+__device__ __forceinline__ float pow2_float(int e) {  // 2^e for e in [-149, 127], built from its bits
+  return e >= -126 ? __int_as_float((e + 127) << 23) : __int_as_float(1 << (e + 149));
+}
+
+__global__ void __launch_bounds__(kXPrepThreads) xprep_kernel(const XPrepJob* jobs, int M) {
+  asm volatile("griddepcontrol.launch_dependents;");
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  __shared__ int s_emax[32], s_lsb[32], s_bad[32];
+  __shared__ int s_ok, s_sigma;
+  const XPrepJob j = jobs[blockIdx.x];
+  const long long n = static_cast<long long>(M) * j.K;
+  int emax = INT_MIN, lsb = INT_MAX, bad = 0;
+  for (long long i = threadIdx.x; i < n; i += blockDim.x) {
+    const uint32_t b = j.x[i];
+    const int e = static_cast<int>((b >> 7) & 0xFF);
+    const uint32_t f = b & 0x7F;
+    if (e == 0xFF) {  // inf or NaN
+      bad = 1;
+    } else if (e != 0) {  // normal: (0x80 | f) * 2^(e - 134)
+      emax = max(emax, e - 127);
+      lsb = min(lsb, e - 134 + __ffs(static_cast<int>(0x80 | f)) - 1);
+    } else if (f != 0) {  // subnormal: f * 2^-133
+      emax = max(emax, -133 + 31 - __clz(static_cast<int>(f)));
+      lsb = min(lsb, -133 + __ffs(static_cast<int>(f)) - 1);
+    }
+  }
+  for (int o = 16; o > 0; o >>= 1) {
+    emax = max(emax, __shfl_xor_sync(0xFFFFFFFFu, emax, o));
+    lsb = min(lsb, __shfl_xor_sync(0xFFFFFFFFu, lsb, o));
+    bad |= __shfl_xor_sync(0xFFFFFFFFu, bad, o);
+  }
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
+  if (lane == 0) {
+    s_emax[warp] = emax;
+    s_lsb[warp] = lsb;
+    s_bad[warp] = bad;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    for (int w = 1; w < nw; ++w) {
+      emax = max(emax, s_emax[w]);
+      lsb = min(lsb, s_lsb[w]);
+      bad |= s_bad[w];
+    }
+    int sigma = 0, ok = !bad;
+    if (emax != INT_MIN) {
+      sigma = emax - 15;
+      ok = ok && (lsb - sigma >= -24);
+    }
+    s_ok = ok;
+    s_sigma = sigma;
+    j.info->ok = ok;
+    j.info->sigma = sigma;
+    j.info->scale = pow2_float(sigma);
+  }
+  __syncthreads();
+  if (!s_ok) return;
+  const double down = ldexp(1.0, -s_sigma);
+  for (long long i = threadIdx.x; i < n; i += blockDim.x) {
+    const float v = __uint_as_float(static_cast<uint32_t>(j.x[i]) << 16);
+    j.x16[i] = __half_as_ushort(__double2half(static_cast<double>(v) * down));  // exact by the test above
+  }
+}
+
+// ----------------------------------------------------------------------------
 // Stream mode: the products do not read each other's outputs, so the whole
 // list is ONE stream-K problem.  Its blocks (SU chunks each) are concatenated
 // product after product, and every warp streams one contiguous range of the
@@ -345,6 +443,14 @@ struct StreamProducer {
   }
 };
 
+// Multiplies a tile's accumulators by a power of two (exact).
+__device__ __forceinline__ void scale_acc(float (&acc)[2][4], float scale) {
+#pragma unroll
+  for (int h = 0; h < 2; ++h)
+#pragma unroll
+    for (int q = 0; q < 4; ++q) acc[h][q] *= scale;
+}
+
 // The warp's ring: D slots of one stage each, and the stage counters.
 struct StreamRing {
   uint32_t ring, bars;
@@ -358,11 +464,12 @@ struct StreamRing {
 // [gb, ...): the partial of a tile that began before gb goes to partial slot
 // 0 when the tile ends (e_first, r_first); a tile still open at the end stays
 // in acc with (r, c).  Returns false if a ring wait gave up.
-template <int BITS, int M, int D, int SU>
+// F16: the activations are used in fp16 (en.x16, outputs times `scale`).
+template <int BITS, int M, int D, int SU, bool F16>
 __device__ __forceinline__ bool stream_segment(const StackParams& sp, const StackEntryDev& en, int e, long long lb0,
                                                long long nblk, long long gb, StreamRing& rg, StreamProducer<SU>& pr,
-                                               uint64_t policy, float (&acc)[2][4], int pw, int& e_first,
-                                               int& r_first, int& r, int& c, int lane) {
+                                               uint64_t policy, float scale, float (&acc)[2][4], int pw,
+                                               int& e_first, int& r_first, int& r, int& c, int lane) {
   constexpr int U = SU;
   constexpr int SLOT = SU * Format<4>::kChunkBytes;
   constexpr int CB = Format<BITS>::kChunkBytes;
@@ -370,7 +477,7 @@ __device__ __forceinline__ bool stream_segment(const StackParams& sp, const Stac
   const int gi = lane >> 2, ti = lane & 3;
   const int bpt = en.C / U;
   const bool x_lane = gi < M;
-  const uint16_t* xrow = en.x + static_cast<long long>(x_lane ? gi : 0) * en.K + 8 * ti;
+  const uint16_t* xrow = (F16 ? en.x16 : en.x) + static_cast<long long>(x_lane ? gi : 0) * en.K + 8 * ti;
   r = static_cast<int>(floor_div(lb0, bpt));
   c = static_cast<int>(lb0 - static_cast<long long>(r) * bpt) * U;
   const uint16_t* xs = xrow + c * KC;
@@ -402,14 +509,15 @@ __device__ __forceinline__ bool stream_segment(const StackParams& sp, const Stac
       ldg128_pred(xa, xs + j * KC, x_lane);
       if (BITS == 4) {  // stream mode has whole q4 chunks only (K % 64 == 0, checked on the host)
         ldg128_pred(xb, xs + j * KC + 32, x_lane);
-        q4_chunk_mac(acc, cr, xa, xb);
+        q4_chunk_mac<F16>(acc, cr, xa, xb);
       } else {
-        q8_chunk_mac(acc, cr, xa);
+        q8_chunk_mac<F16>(acc, cr, xa);
       }
     }
     xs += U * KC;
     c += U;
     if (c == en.C) {
+      if (F16) scale_acc(acc, scale);
       const long long tile_g = en.blk_off + static_cast<long long>(r) * bpt;  // the tile's first block
       if (tile_g < gb) {  // began in an earlier warp's range: its partial goes to slot 0 now
         write_partial<M>(sp.partials, pw, 0, acc, lane);
@@ -479,13 +587,22 @@ __global__ void __launch_bounds__(NW * 32, 1) stream_kernel(const StackParams sp
   long long left = ge - gb;
   StackEntryDev en = sp.entries[e];
   bool ok = true;
+  float scale = 1.f;
   while (left > 0) {
     const long long in_entry = en.TC / SU - lb;
     const long long n = in_entry < left ? in_entry : left;
+    const XInfo xi = *en.xinfo;  // written by xprep_kernel, complete once griddepcontrol.wait returned
+    scale = xi.ok ? xi.scale : 1.f;
     if (en.bits == 4) {
-      ok = stream_segment<4, M, D, SU>(sp, en, e, lb, n, gb, rg, pr, policy, acc, pw, e_first, r_first, r, c, lane);
+      ok = xi.ok ? stream_segment<4, M, D, SU, true>(sp, en, e, lb, n, gb, rg, pr, policy, scale, acc, pw, e_first,
+                                                     r_first, r, c, lane)
+                 : stream_segment<4, M, D, SU, false>(sp, en, e, lb, n, gb, rg, pr, policy, scale, acc, pw,
+                                                      e_first, r_first, r, c, lane);
     } else {
-      ok = stream_segment<8, M, D, SU>(sp, en, e, lb, n, gb, rg, pr, policy, acc, pw, e_first, r_first, r, c, lane);
+      ok = xi.ok ? stream_segment<8, M, D, SU, true>(sp, en, e, lb, n, gb, rg, pr, policy, scale, acc, pw, e_first,
+                                                     r_first, r, c, lane)
+                 : stream_segment<8, M, D, SU, false>(sp, en, e, lb, n, gb, rg, pr, policy, scale, acc, pw,
+                                                      e_first, r_first, r, c, lane);
     }
     if (!ok) break;
     left -= n;
@@ -518,6 +635,7 @@ __global__ void __launch_bounds__(NW * 32, 1) stream_kernel(const StackParams sp
     const int bpt = en.C / SU;
     const long long tile_g = en.blk_off + static_cast<long long>(r) * bpt;
     last = SplitTile{en.y, en.N, r, sp.counters + en.tile_off + r, tile_g, tile_g + bpt};
+    scale_acc(acc, scale);
     write_partial<M>(sp.partials, pw, tile_g <= gb ? 0 : 1, acc, lane);
   }
   if (first.r < 0 && last.r < 0) return;

@@ -185,7 +185,9 @@ Q4_API int q4_set_wait_timeout_ns(uint64_t ns);
 
 /* Debug decode on the device: runs the kernels' in-register dequantisation on
  * every packed word and writes the integers q (int8 [N][K], device) and the
- * scales (uint16 [N][K/32], device).  Used to check that in-register unpack is
+ * scales (uint16 [N][K/32], device).  Both decodes the kernels use (to bf16
+ * and to fp16) run; an element where they disagree is written as -128, a
+ * value neither format holds.  Used to check that in-register unpack is
  * bit-exact against the canonical weights. */
 Q4_API int q4_unpack_device(int bits, const void* packed, int64_t N, int64_t K, int8_t* q_out, uint16_t* scales_out,
                             void* stream);
@@ -228,11 +230,15 @@ typedef struct q4_stack q4_stack;
  * ordering of a stream of one launch per product.
  * Stream mode (Q4_STACK_INDEPENDENT): for products that do not read each
  * other's outputs (the activations are inputs of the step, not outputs of an
- * earlier product).  One cooperative kernel treats the concatenated products
+ * earlier product).  One kernel treats the concatenated products
  * as a single work-split problem: every warp streams one contiguous range
  * across product boundaries with no synchronisation, so the HBM stream never
- * pauses between products.  Outputs agree with q4_gemv / q8_gemv within the
- * product tolerance (tiles may be split at other places).
+ * pauses between products.  Before it, a small kernel prepares each distinct
+ * activation tensor: when a power of two 2^s makes every x * 2^-s exactly
+ * representable in fp16, the products of that tensor run on that fp16 copy
+ * (a shorter decode; outputs scaled back by 2^s, exactly), otherwise on x in
+ * bf16.  Outputs agree with q4_gemv / q8_gemv within the product tolerance
+ * (tiles may be split at other places, and fp16 sums round differently).
  * Both persistent modes need every product non-empty with an even number of
  * chunks per tile; other lists use graph mode.  Stream mode also needs every
  * q4 K to be a multiple of 64; otherwise the ordered mode is used.
@@ -246,8 +252,9 @@ typedef struct q4_stack q4_stack;
  * UNSUPPORTED if the persistent kernel cannot be resident on every SM. */
 Q4_API int layer_stack_create(const q4_stack_entry* entries, int n_entries, int M, int flags, q4_stack** out);
 
-/* Runs the products on `stream`: one cooperative kernel launch (persistent
- * mode) or one cudaGraphLaunch (graph mode).  Asynchronous. */
+/* Runs the products on `stream`: one cooperative kernel launch (ordered
+ * mode), the activation preparation and one kernel launch (stream mode), or
+ * one cudaGraphLaunch (graph mode).  Asynchronous. */
 Q4_API int layer_stack_run(q4_stack* stack, void* stream);
 
 /* Synchronises `stream` and reports a bounded wait that gave up during the

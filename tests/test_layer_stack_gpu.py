@@ -95,7 +95,7 @@ def test_stream_mode_of_independent_products(q4, M, tensors):
     bitwise identical."""
     torch = H.torch()
     st = workloads.DeviceStream(tensors, M, flags=q4.Q4_STACK_INDEPENDENT)
-    assert st.stack.launches() == 1
+    assert st.stack.launches() == 2  # activation preparation + stream kernel
     st.run()
     st.check()
     first = [_y(st, i).copy() for i in range(len(tensors))]
@@ -135,7 +135,8 @@ def test_full_decode_stream_sampled(q4, M, mode):
     torch = H.torch()
     tensors = workloads.decode_stream(fused=True)
     st = workloads.DeviceStream(tensors, M, flags=0 if mode == "ordered" else q4.Q4_STACK_INDEPENDENT)
-    assert st.stack.launches() == 1  # one persistent kernel for the 257 products
+    # one persistent kernel for the 257 products (stream mode: after xprep_kernel)
+    assert st.stack.launches() == (1 if mode == "ordered" else 2)
     st.run()
     st.run()
     st.check()
@@ -178,4 +179,47 @@ def test_degenerate_rows_in_stacks(q4, mode, M):
     torch.cuda.synchronize()
     for (bits, N), (q, s), y in zip(specs, hosts, ys):
         H.assert_parity(y.cpu().numpy().reshape(M, N), q, s, x, bits)
+    st.close()
+
+
+@pytest.mark.parametrize("case", ["wide_range", "tiny", "huge", "zeros", "subnormal"])
+@pytest.mark.parametrize("M", [1, 4])
+def test_stream_mode_activation_ranges(q4, case, M):
+    """Activations that fp16 cannot hold after any power-of-two scaling (a
+    dynamic range beyond 2^40: the bf16 fallback), activations far below or
+    above fp16's range (scaled into it exactly), all-zero activations and
+    bf16 subnormals: every product within the tolerance."""
+    torch = H.torch()
+    K = 5120
+    x = synth.activations(6, synth.act_stream(43), M, K)
+    xf = (x.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    if case == "wide_range":
+        xf[:, ::7] *= 2.0 ** 60
+        xf[:, 3::11] *= 2.0 ** -60
+    elif case == "tiny":
+        xf *= 2.0 ** -100
+    elif case == "huge":
+        xf *= 2.0 ** 100
+    elif case == "zeros":
+        xf[:] = 0.0
+    else:
+        xf *= 2.0 ** -128  # many elements become bf16 subnormals
+    x = synth.f64_to_bf16_bits(xf.ravel()).reshape(M, K)
+    x_dev = H.to_device_x(x)
+    entries, hosts, ys = [], [], []
+    for bits, N, tid in ((4, 160, 51), (8, 96, 52)):
+        q, s = synth.tensor(bits, 6, tid, N, K)
+        y = torch.full((M * N,), float("nan"), dtype=torch.float32, device="cuda")
+        entries.append((bits, N, K, H.to_device_packed(bits, q, s, N, K), x_dev, y))
+        hosts.append((bits, N, q, s))
+        ys.append(y)
+    st = q4.layer_stack_create(entries, M, q4.Q4_STACK_INDEPENDENT)
+    q4.layer_stack_run(st)
+    q4.layer_stack_check(st)
+    torch.cuda.synchronize()
+    for (bits, N, q, s), y in zip(hosts, ys):
+        yy = y.cpu().numpy().reshape(M, N)
+        if case == "zeros":
+            assert np.all(yy == 0.0)
+        H.assert_parity(yy, q, s, x, bits)
     st.close()

@@ -192,21 +192,31 @@ def oracle_sample_rate(target_s: float = 12.0, seed: int = 0):
 # distributed plumbing
 # ----------------------------------------------------------------------------
 class Dist:
-    def __init__(self, gpus: int):
+    """One process per GPU (torch.distributed.run sets RANK, LOCAL_RANK,
+    WORLD_SIZE, MASTER_*).  The step has no data exchange (replicas): the
+    process group only brackets the timed region with barriers and takes the
+    max of the ranks' device times.  backend "gloo" (CPU tensors) serves the
+    host-side tests."""
+
+    def __init__(self, gpus: int, backend: str = "nccl"):
         self.world = int(os.environ.get("WORLD_SIZE", "1"))
         self.rank = int(os.environ.get("RANK", "0"))
         self.local = int(os.environ.get("LOCAL_RANK", "0"))
         self.pg = False
-        if self.world != gpus and not (self.world == 1 and gpus == 1):
-            if self.world == 1:
-                raise SystemExit(f"--gpus {gpus} needs torch.distributed.run with {gpus} processes")
+        self.backend = backend
+        if self.world != gpus:
+            raise SystemExit(f"--gpus {gpus} needs torch.distributed.run with {gpus} processes "
+                             f"(WORLD_SIZE is {self.world})")
         if self.world > 1:
             import torch
             import torch.distributed as dist
 
-            torch.cuda.set_device(self.local)
-            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                    device_id=torch.device("cuda", self.local))
+            timeout = datetime.timedelta(seconds=120)
+            if backend == "nccl":
+                torch.cuda.set_device(self.local)
+                dist.init_process_group("nccl", timeout=timeout, device_id=torch.device("cuda", self.local))
+            else:
+                dist.init_process_group(backend, timeout=timeout)
             self.pg = True
 
     @classmethod
@@ -228,7 +238,7 @@ class Dist:
         import torch
         import torch.distributed as dist
 
-        t = torch.tensor([v], dtype=torch.float64, device="cuda")
+        t = torch.tensor([v], dtype=torch.float64, device="cuda" if self.backend == "nccl" else "cpu")
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         return float(t.item())
 
@@ -449,7 +459,7 @@ def run_reference(args, d: Dist):
         "metric": METRIC,
         "value": round(value, 4),
         "unit": UNIT,
-        "n_gpus": d.world,
+        "n_gpus": args.gpus,
         "steps": args.steps,
         "warmup": args.warmup,
         "ms_per_step": round(dt * 1e3, 3),

@@ -8,7 +8,12 @@ layer stack.  13.7 GB of packed weights are resident in HBM; x and y are small.
 
 Metric: weight-stream GB/s (algorithmic weight bytes / device time per step)
 at M = 1, with % of the measured HBM peak and the implied decode tok/s; the
-same at M = 4 (one verification pass of 3 drafted tokens + 1) in "m4".
+same at M = 4 (one verification pass of 3 drafted tokens + 1) in "m4".  The
+line also reports the ordered and graph stack modes, the end-to-end step
+through the public API ("e2e"), the roofline of the dominant kernel, the CPU
+oracle's rate ("cpu_baseline"), the SM clock under load, and "per_config":
+microseconds per product of the single-tensor configurations (q4 4096 x 4096,
+each projection of one layer at M = 1 and 4, the q8 vocabulary heads).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
@@ -264,6 +269,56 @@ def time_region(torch, fn, steps, stream):
     return e0.elapsed_time(e1)  # ms
 
 
+def per_config(args, d: Dist, torch, q4, workloads, peak):
+    """Microseconds per product for the single-tensor configurations: a
+    q4 4096 x 4096 product (M = 1), each projection of one 27B-shaped layer
+    (M = 1 and M = 4) and the q8 vocabulary heads (M = 1).  Each shape is
+    replicated until the copies exceed twice the L2, and the copies run in
+    turn, so no launch finds its weights in L2.  `graph`: one q4_gemv /
+    q8_gemv launch per product (captured as a graph with programmatic
+    dependent launch, the single-call kernels back to back); `stream`: the
+    same copies as one stream-mode stack.  Device time per product."""
+    l2 = torch.cuda.get_device_properties(d.local).L2_cache_size
+    stream = torch.cuda.current_stream()
+    iters = max(3, min(20, args.steps // 10))
+
+    def time_stack(stack):
+        run = lambda: q4.layer_stack_run(stack)  # noqa: E731
+        for _ in range(3):
+            run()
+        ms = d.max(time_region(torch, run, iters, stream) / iters)
+        q4.layer_stack_check(stack)
+        return ms
+
+    def shape(name, bits, N, K, M, tid):
+        one = workloads.weight_bytes(bits, N, K)
+        copies = max(2, -(-2 * l2 // one))
+        tensors = [workloads.Tensor(f"{name}.{i}", bits, N, K, tid + i) for i in range(copies)]
+        out = {"N": N, "K": K, "bits": bits, "M": M, "bytes": one, "copies": copies}
+        st = workloads.DeviceStream(tensors, M, seed=args.seed, flags=q4.Q4_STACK_GRAPH)
+        for stack, key in ((st.stack, "graph"), (st.make_stack(q4.Q4_STACK_INDEPENDENT), "stream")):
+            us = time_stack(stack) * 1e3 / copies
+            out[key] = {"us": round(us, 2), "GBps": round(one / (us * 1e3), 1),
+                        "pct_of_hbm_peak": round(100 * one / (us * 1e3) / peak, 1)}
+            stack.close()
+        st.close()
+        del st
+        torch.cuda.empty_cache()
+        return out
+
+    res = {"note": "device us per product, L2 defeated by rotating copies (> 2x L2)",
+           "q4_4096x4096_M1": shape("w4096", 4, 4096, 4096, 1, 3000)}
+    for M in (1, 4):
+        layer = {}
+        for t in workloads.layer_q4():
+            layer[t.name] = shape(t.name, t.bits, t.N, t.K, M, 3100 + 100 * len(layer))
+        layer["sum_us"] = {k: round(sum(v[k]["us"] for v in layer.values()), 2) for k in ("graph", "stream")}
+        res[f"layer_q4_M{M}"] = layer
+    for h in workloads.draft_heads():
+        res[f"{h.name}_q8_{h.N}x{h.K}_M1"] = shape(h.name, h.bits, h.N, h.K, 1, 3900 + h.tensor_id)
+    return res
+
+
 def run_ours(args, d: Dist):
     import torch
 
@@ -350,6 +405,8 @@ def run_ours(args, d: Dist):
     del st4
     torch.cuda.empty_cache()
 
+    configs = None if args.no_configs else per_config(args, d, torch, q4, workloads, peak)
+
     cpu = None
     if d.rank == 0 and not args.no_cpu_baseline:
         rate, threads, desc, _ = oracle_sample_rate(args.cpu_seconds, args.seed)
@@ -414,6 +471,7 @@ def run_ours(args, d: Dist):
             "h2d_bytes_per_step": h2d,
             "d2h_bytes_per_step": d2h,
         },
+        "per_config": configs,
         "gpu_launches": n_launch * args.steps,
         "clocks": clocks,
     }
@@ -518,6 +576,7 @@ def main():
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU time of the oracle sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-configs", action="store_true", help="skip the per-configuration product timings")
     ap.add_argument("--reference-rows", type=int, default=8, help="rows per tensor per reference step")
     ap.add_argument("--profile-case", action="store_true", help="run the small ncu case and exit")
     ap.add_argument("--profile-bits", type=int, default=4)

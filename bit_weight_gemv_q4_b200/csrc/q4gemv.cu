@@ -553,8 +553,11 @@ void* select_stack_kernel(int M, int su) {
   return table[su == 0 ? 0 : (su == 2 ? 1 : 2)][M - 1];
 }
 
-int stack_smem_bytes(int su) {
-  const int slot = (su == 0 ? q4k::kStackU : su) * q4k::Format<4>::kChunkBytes;
+// su: stream mode with stages of su chunks (weights + activation slice of M
+// rows), or 0 for ordered mode (weights only, stages of kStackU chunks).
+int stack_smem_bytes(int su, int M) {
+  const int slot = su == 0 ? q4k::kStackU * q4k::Format<4>::kChunkBytes
+                           : su * (q4k::Format<4>::kChunkBytes + M * q4k::Format<4>::kKPerChunk * 2);
   return kNW * kStackD * slot + kNW * kStackD * 8;
 }
 
@@ -622,19 +625,21 @@ int create_persistent(const q4_stack_entry* entries, int n, int M, int su, const
   // ordered mode re-uses one counter per tile of the largest product; stream
   // mode keeps one per tile of every product
   const size_t counters = (static_cast<size_t>(independent ? total_tiles : max_t) * 4 + 255) / 256 * 256;
-  // stream mode: per distinct (x, K) an fp16 copy [M][K] and its XInfo
+  // stream mode: per distinct (x, K, format) a chunk-major copy of x and its XInfo
   std::vector<q4k::XPrepJob> jobs;
   std::vector<size_t> job_of(static_cast<size_t>(n), 0), x16_off, info_off;
   size_t prep_bytes = 0;
   if (independent) {
     for (int i = 0; i < n; ++i) {
+      const int KC = entries[i].bits == 4 ? q4k::Format<4>::kKPerChunk : q4k::Format<8>::kKPerChunk;
       size_t jdx = jobs.size();
       for (size_t k = 0; k < jobs.size(); ++k)
-        if (jobs[k].x == entries[i].x && jobs[k].K == entries[i].K) jdx = k;
+        if (jobs[k].x == entries[i].x && jobs[k].K == entries[i].K && jobs[k].KC == KC) jdx = k;
       if (jdx == jobs.size()) {
         q4k::XPrepJob j{};
         j.x = entries[i].x;
         j.K = entries[i].K;
+        j.KC = KC;
         jobs.push_back(j);
         x16_off.push_back(prep_bytes);
         prep_bytes += (static_cast<size_t>(M) * entries[i].K * 2 + 255) / 256 * 256;
@@ -653,12 +658,12 @@ int create_persistent(const q4_stack_entry* entries, int n, int M, int su, const
   if (independent && err == cudaSuccess) {
     unsigned char* base = static_cast<unsigned char*>(st->workspace) + prep_base;
     for (size_t k = 0; k < jobs.size(); ++k) {
-      jobs[k].x16 = reinterpret_cast<uint16_t*>(base + x16_off[k]);
+      jobs[k].xc = reinterpret_cast<uint16_t*>(base + x16_off[k]);
       jobs[k].info = reinterpret_cast<q4k::XInfo*>(base + info_off[k]);
     }
     for (int i = 0; i < n; ++i) {
       const q4k::XPrepJob& j = jobs[job_of[static_cast<size_t>(i)]];
-      host[static_cast<size_t>(i)].x16 = j.x16;
+      host[static_cast<size_t>(i)].xc = j.xc;
       host[static_cast<size_t>(i)].xinfo = j.info;
     }
     err = cudaMalloc(&st->xprep_dev, sizeof(q4k::XPrepJob) * jobs.size());
@@ -671,7 +676,7 @@ int create_persistent(const q4_stack_entry* entries, int n, int M, int su, const
     err = cudaMemcpy(st->entries_dev, host.data(), sizeof(q4k::StackEntryDev) * host.size(), cudaMemcpyHostToDevice);
   if (err != cudaSuccess) return cuda_fail(err, "layer_stack_create: allocation");
   st->fn = select_stack_kernel(M, su);
-  st->smem = stack_smem_bytes(su);
+  st->smem = stack_smem_bytes(su, M);
   st->block = kNW * 32;
   st->grid = dev.sms;
   err = cudaFuncSetAttribute(st->fn, cudaFuncAttributeMaxDynamicSharedMemorySize, st->smem);

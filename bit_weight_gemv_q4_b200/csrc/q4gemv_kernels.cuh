@@ -164,6 +164,39 @@ __device__ __forceinline__ void bulk_copy_g2s_if(bool pred, uint32_t dst, const 
       : "memory");
 }
 
+// Lane 0 (pred) arms `bar` for a stage of weights and its activation slice
+// (bytes_w + bytes_x), copies the weights (L2 evict-first: read once) and,
+// when with_x, the activations (default policy: many warps read them); a
+// stage armed without them gets them from bulk_copy_x_if later.  One
+// predicated block, so the warp does not branch.
+__device__ __forceinline__ void bulk_copy_g2s_x_if(bool pred, uint32_t dst_w, const void* src_w, uint32_t bytes_w,
+                                                   uint32_t dst_x, const void* src_x, uint32_t bytes_x, bool with_x,
+                                                   uint32_t bar, uint64_t policy) {
+  asm volatile(
+      "{\n\t.reg .pred p, px;\n\tsetp.ne.b32 p, %8, 0;\n\t"
+      "setp.ne.and.b32 px, %9, 0, p;\n\t"
+      "@p mbarrier.arrive.expect_tx.shared::cta.b64 _, [%6], %7;\n\t"
+      "@p cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1], %2, [%6], %10;"
+      "\n\t"
+      "@px cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%3], [%4], %5, [%6];"
+      "\n\t}" ::"r"(dst_w),
+      "l"(src_w), "r"(bytes_w), "r"(dst_x), "l"(src_x), "r"(bytes_x), "r"(bar), "r"(bytes_w + bytes_x),
+      "r"(static_cast<int>(pred)), "r"(static_cast<int>(with_x)), "l"(policy)
+      : "memory");
+}
+
+// Lane 0 (pred) copies an activation slice into a stage that is already
+// armed for its bytes.
+__device__ __forceinline__ void bulk_copy_x_if(bool pred, uint32_t dst, const void* src, uint32_t bytes,
+                                               uint32_t bar) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "@p cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+      "\n\t}" ::"r"(dst),
+      "l"(src), "r"(bytes), "r"(bar), "r"(static_cast<int>(pred))
+      : "memory");
+}
+
 __device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void grid_dependents_launch() { asm volatile("griddepcontrol.launch_dependents;"); }
 

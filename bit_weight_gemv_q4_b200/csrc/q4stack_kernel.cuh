@@ -39,18 +39,22 @@ struct XInfo {
   int pad;
 };
 
+// xc: the activations chunk-major, [K/KC][M][KC] (KC = k per chunk of the
+// product's format), so the slice of a stage of chunks is one contiguous
+// copy: fp16 x * 2^-sigma when info->ok, else the bf16 x itself.
 struct XPrepJob {
   const uint16_t* x;  // bf16 [M][K]
-  uint16_t* x16;      // fp16 [M][K]
+  uint16_t* xc;       // [K/KC][M][KC]
   XInfo* info;
   long long K;
+  int KC;
 };
 
 struct StackEntryDev {
   const uint8_t* packed;
   const uint16_t* x;
   float* y;
-  const uint16_t* x16;   // stream mode: fp16 copy of x (valid when xinfo->ok)
+  const uint16_t* xc;    // stream mode: chunk-major activations (XPrepJob)
   const XInfo* xinfo;    // stream mode
   long long N, K, TC;
   long long blk_off;  // first block of this product in the concatenated sequence (stream mode)
@@ -380,11 +384,18 @@ __global__ void __launch_bounds__(kXPrepThreads) xprep_kernel(const XPrepJob* jo
     j.info->scale = pow2_float(sigma);
   }
   __syncthreads();
-  if (!s_ok) return;
+  const bool f16 = s_ok != 0;
   const double down = ldexp(1.0, -s_sigma);
   for (long long i = threadIdx.x; i < n; i += blockDim.x) {
-    const float v = __uint_as_float(static_cast<uint32_t>(j.x[i]) << 16);
-    j.x16[i] = __half_as_ushort(__double2half(static_cast<double>(v) * down));  // exact by the test above
+    const long long m = i / j.K, k = i - m * j.K;
+    const long long chunk = k / j.KC, kk = k - chunk * j.KC;
+    const uint16_t b = j.x[i];
+    uint16_t out = b;
+    if (f16) {
+      const float v = __uint_as_float(static_cast<uint32_t>(b) << 16);
+      out = __half_as_ushort(__double2half(static_cast<double>(v) * down));  // exact by the test above
+    }
+    j.xc[(chunk * M + m) * j.KC + kk] = out;
   }
 }
 
@@ -413,13 +424,28 @@ __device__ __forceinline__ int entry_of_block(const StackParams& sp, long long g
 
 // The producer side of a warp's ring in stream mode: the next stage (SU
 // chunks) to copy in the warp's range, crossing products.  Warp-uniform state.
-template <int SU>
+// A stage is SU chunks of weights followed, in the same slot and on the same
+// mbarrier, by the matching activation slice (SU chunks x M rows x KC
+// values, one contiguous copy from the chunk-major xc).
+template <int SU, int M>
+struct StreamSlot {
+  static constexpr int kWeightBytes = SU * Format<4>::kChunkBytes;  // the larger of the two formats
+  static constexpr int kXBytes = SU * M * Format<4>::kKPerChunk * 2;
+  static constexpr int kBytes = kWeightBytes + kXBytes;
+};
+
+// The producer side of a warp's ring in stream mode: the next stage (SU
+// chunks) to copy in the warp's range, crossing products.  Warp-uniform state.
+template <int SU, int M>
 struct StreamProducer {
   int e = 0;                 // product of the next stage
   int left_entry = 0;        // stages left in that product
   long long left_total = 0;  // stages left in the range
   const uint8_t* src = nullptr;
   uint32_t bytes = 0;
+  const uint16_t* xc = nullptr;  // the product's chunk-major activations
+  int cpos = 0;                  // chunk of the tile where the next stage starts
+  int C = 0, KC = 0;
 
   __device__ __forceinline__ void enter(const StackParams& sp, int entry, long long lb) {
     const StackEntryDev& en = sp.entries[entry];
@@ -429,14 +455,32 @@ struct StreamProducer {
     src = en.packed + lb * SU * CB;
     const long long in_entry = en.TC / SU - lb;
     left_entry = static_cast<int>(in_entry < left_total ? in_entry : left_total);
+    xc = en.xc;
+    C = en.C;
+    KC = en.bits == 4 ? Format<4>::kKPerChunk : Format<8>::kKPerChunk;
+    const int bpt = en.C / SU;
+    cpos = static_cast<int>(lb - static_cast<long long>(floor_div(lb, bpt)) * bpt) * SU;
   }
-  // Copies the next stage into `dst` (lane 0), completing on `bar`.
+  __device__ __forceinline__ const uint16_t* x_src() const { return xc + static_cast<long long>(cpos) * M * KC; }
+  __device__ __forceinline__ uint32_t x_bytes() const { return static_cast<uint32_t>(SU * M * KC * 2); }
+  // Copies the next stage into the slot at `dst` (lane 0), completing on
+  // `bar`; with_x = false leaves the activation slice for issue_x (before
+  // griddepcontrol.wait, when the activations may not be ready yet), but the
+  // barrier already expects its bytes.
   __device__ __forceinline__ bool issue(const StackParams& sp, uint32_t dst, uint32_t bar, uint64_t policy,
-                                        int lane) {
+                                        int lane, bool with_x, const uint16_t** x_later, uint32_t* x_later_bytes) {
     if (left_total == 0) return false;
     if (left_entry == 0) enter(sp, e + 1, 0);
-    bulk_copy_g2s_if(lane == 0, dst, src, bytes, bar, policy);
+    const uint32_t xb = x_bytes();
+    bulk_copy_g2s_x_if(lane == 0, dst, src, bytes, dst + StreamSlot<SU, M>::kWeightBytes, x_src(), xb, with_x,
+                       bar, policy);
+    if (!with_x) {
+      *x_later = x_src();
+      *x_later_bytes = xb;
+    }
     src += bytes;
+    cpos += SU;
+    if (cpos == C) cpos = 0;
     --left_entry;
     --left_total;
     return true;
@@ -467,21 +511,21 @@ struct StreamRing {
 // F16: the activations are used in fp16 (en.x16, outputs times `scale`).
 template <int BITS, int M, int D, int SU, bool F16>
 __device__ __forceinline__ bool stream_segment(const StackParams& sp, const StackEntryDev& en, int e, long long lb0,
-                                               long long nblk, long long gb, StreamRing& rg, StreamProducer<SU>& pr,
-                                               uint64_t policy, float scale, float (&acc)[2][4], int pw,
-                                               int& e_first, int& r_first, int& r, int& c, int lane) {
+                                               long long nblk, long long gb, StreamRing& rg,
+                                               StreamProducer<SU, M>& pr, uint64_t policy, float scale,
+                                               float (&acc)[2][4], int pw, int& e_first, int& r_first, int& r,
+                                               int& c, int lane) {
   constexpr int U = SU;
-  constexpr int SLOT = SU * Format<4>::kChunkBytes;
+  constexpr int SLOT = StreamSlot<SU, M>::kBytes;
   constexpr int CB = Format<BITS>::kChunkBytes;
   constexpr int KC = Format<BITS>::kKPerChunk;
   const int gi = lane >> 2, ti = lane & 3;
   const int bpt = en.C / U;
-  const bool x_lane = gi < M;
-  const uint16_t* xrow = (F16 ? en.x16 : en.x) + static_cast<long long>(x_lane ? gi : 0) * en.K + 8 * ti;
+  // this lane's B fragment in the slot's activation slice: row min(gi, M-1)
+  // (columns >= M only feed outputs that are never stored), 8 values at 8 ti
+  const uint32_t xlane = StreamSlot<SU, M>::kWeightBytes + ((gi < M ? gi : M - 1) * KC + 8 * ti) * 2;
   r = static_cast<int>(floor_div(lb0, bpt));
   c = static_cast<int>(lb0 - static_cast<long long>(r) * bpt) * U;
-  const uint16_t* xs = xrow + c * KC;
-  uint4 xa = make_uint4(0, 0, 0, 0), xb = make_uint4(0, 0, 0, 0);
   for (long long i = 0; i < nblk; ++i) {
     const uint32_t bar = rg.bars + 8 * rg.slot;
     if (!mbar_wait_bounded(bar, rg.phase, sp.timeout_ns)) return false;
@@ -489,6 +533,8 @@ __device__ __forceinline__ bool stream_segment(const StackParams& sp, const Stac
 #pragma unroll
     for (int j = 0; j < U; ++j) {
       ChunkRegs cr;
+      const uint4 xa = lds128(stage + xlane + j * M * KC * 2);
+      const uint4 xb = BITS == 4 ? lds128(stage + xlane + j * M * KC * 2 + 64) : make_uint4(0, 0, 0, 0);
       cr.codes[0] = lds128(stage + j * CB + 16 * lane);
       cr.codes[1] = lds128(stage + j * CB + kHalfBytes + 16 * lane);
       if (BITS == 4) {
@@ -500,21 +546,18 @@ __device__ __forceinline__ bool stream_segment(const StackParams& sp, const Stac
       if (j == U - 1) {
         // every lane has read the slot; lane 0 refills it with the next stage
         __syncwarp();
-        if (!pr.issue(sp, stage, bar, policy, lane)) --rg.in_flight;
+        if (!pr.issue(sp, stage, bar, policy, lane, true, nullptr, nullptr)) --rg.in_flight;
         if (++rg.slot == D) {
           rg.slot = 0;
           rg.phase ^= 1u;
         }
       }
-      ldg128_pred(xa, xs + j * KC, x_lane);
       if (BITS == 4) {  // stream mode has whole q4 chunks only (K % 64 == 0, checked on the host)
-        ldg128_pred(xb, xs + j * KC + 32, x_lane);
         q4_chunk_mac<F16>(acc, cr, xa, xb);
       } else {
         q8_chunk_mac<F16>(acc, cr, xa);
       }
     }
-    xs += U * KC;
     c += U;
     if (c == en.C) {
       if (F16) scale_acc(acc, scale);
@@ -528,7 +571,6 @@ __device__ __forceinline__ bool stream_segment(const StackParams& sp, const Stac
       }
       ++r;
       c = 0;
-      xs = xrow;
 #pragma unroll
       for (int h = 0; h < 2; ++h) acc[h][0] = acc[h][1] = acc[h][2] = acc[h][3] = 0.f;
     }
@@ -540,7 +582,7 @@ __device__ __forceinline__ bool stream_segment(const StackParams& sp, const Stac
 // chunks per tile is a multiple of SU, checked on the host).
 template <int M, int NW, int D, int SU>
 __global__ void __launch_bounds__(NW * 32, 1) stream_kernel(const StackParams sp) {
-  constexpr int SLOT = SU * Format<4>::kChunkBytes;  // the larger of the two formats
+  constexpr int SLOT = StreamSlot<SU, M>::kBytes;
   extern __shared__ __align__(128) unsigned char smem[];
 
   const int lane = threadIdx.x & 31;
@@ -568,16 +610,27 @@ __global__ void __launch_bounds__(NW * 32, 1) stream_kernel(const StackParams sp
     return;
   }
   const int e0 = entry_of_block(sp, gb);
-  StreamProducer<SU> pr;
+  StreamProducer<SU, M> pr;
   pr.left_total = ge - gb;
   pr.enter(sp, e0, gb - sp.entries[e0].blk_off);
+  // the first stages' weights now; their activation slices once the
+  // activation preparation (the preceding kernel) has completed
+  const uint16_t* x_later[D];
+  uint32_t x_later_bytes[D];
   for (int s = 0; s < D; ++s) {
-    if (!pr.issue(sp, rg.ring + s * SLOT, rg.bars + 8 * s, policy, lane)) break;
+    if (!pr.issue(sp, rg.ring + s * SLOT, rg.bars + 8 * s, policy, lane, false, &x_later[s], &x_later_bytes[s]))
+      break;
     ++rg.in_flight;
   }
 
   grid_dependency_wait();
   grid_dependents_launch();
+#pragma unroll
+  for (int s = 0; s < D; ++s) {
+    if (s < rg.in_flight)
+      bulk_copy_x_if(lane == 0, rg.ring + s * SLOT + StreamSlot<SU, M>::kWeightBytes, x_later[s], x_later_bytes[s],
+                     rg.bars + 8 * s);
+  }
 
   float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
   int e_first = -1, r_first = -1;  // split first tile (its partial is written when it completes)

@@ -510,7 +510,8 @@ struct StreamRing {
 // in acc with (r, c).  Returns false if a ring wait gave up.
 // F16: the activations are used in fp16 (en.x16, outputs times `scale`).
 template <int BITS, int M, int D, int SU, bool F16>
-__device__ __forceinline__ bool stream_segment(const StackParams& sp, const StackEntryDev& en, int e, long long lb0,
+__device__ __forceinline__ bool stream_segment(const StackParams& sp, const StackEntryDev* __restrict__ ep, int e,
+                                               long long lb0,
                                                long long nblk, long long gb, StreamRing& rg,
                                                StreamProducer<SU, M>& pr, uint64_t policy, float scale,
                                                float (&acc)[2][4], int pw, int& e_first, int& r_first, int& r,
@@ -520,7 +521,8 @@ __device__ __forceinline__ bool stream_segment(const StackParams& sp, const Stac
   constexpr int CB = Format<BITS>::kChunkBytes;
   constexpr int KC = Format<BITS>::kKPerChunk;
   const int gi = lane >> 2, ti = lane & 3;
-  const int bpt = en.C / U;
+  const int C = ep->C;  // the entry's other fields are read where they are used, not held in registers
+  const int bpt = C / U;
   // this lane's B fragment in the slot's activation slice: row min(gi, M-1)
   // (columns >= M only feed outputs that are never stored), 8 values at 8 ti
   const uint32_t xlane = StreamSlot<SU, M>::kWeightBytes + ((gi < M ? gi : M - 1) * KC + 8 * ti) * 2;
@@ -559,15 +561,15 @@ __device__ __forceinline__ bool stream_segment(const StackParams& sp, const Stac
       }
     }
     c += U;
-    if (c == en.C) {
+    if (c == C) {
       if (F16) scale_acc(acc, scale);
-      const long long tile_g = en.blk_off + static_cast<long long>(r) * bpt;  // the tile's first block
+      const long long tile_g = ep->blk_off + static_cast<long long>(r) * bpt;  // the tile's first block
       if (tile_g < gb) {  // began in an earlier warp's range: its partial goes to slot 0 now
         write_partial<M>(sp.partials, pw, 0, acc, lane);
         e_first = e;
         r_first = r;
       } else {
-        store_tile<M>(en.y, en.N, r, acc, lane);
+        store_tile<M>(ep->y, ep->N, r, acc, lane);
       }
       ++r;
       c = 0;
@@ -638,29 +640,29 @@ __global__ void __launch_bounds__(NW * 32, 1) stream_kernel(const StackParams sp
   int e = e0;
   long long lb = gb - sp.entries[e0].blk_off;
   long long left = ge - gb;
-  StackEntryDev en = sp.entries[e];
+  const StackEntryDev* __restrict__ ep = sp.entries + e;
   bool ok = true;
   float scale = 1.f;
   while (left > 0) {
-    const long long in_entry = en.TC / SU - lb;
+    const long long in_entry = ep->TC / SU - lb;
     const long long n = in_entry < left ? in_entry : left;
-    const XInfo xi = *en.xinfo;  // written by xprep_kernel, complete once griddepcontrol.wait returned
+    const XInfo xi = *ep->xinfo;  // written by xprep_kernel, complete once griddepcontrol.wait returned
     scale = xi.ok ? xi.scale : 1.f;
-    if (en.bits == 4) {
-      ok = xi.ok ? stream_segment<4, M, D, SU, true>(sp, en, e, lb, n, gb, rg, pr, policy, scale, acc, pw, e_first,
+    if (ep->bits == 4) {
+      ok = xi.ok ? stream_segment<4, M, D, SU, true>(sp, ep, e, lb, n, gb, rg, pr, policy, scale, acc, pw, e_first,
                                                      r_first, r, c, lane)
-                 : stream_segment<4, M, D, SU, false>(sp, en, e, lb, n, gb, rg, pr, policy, scale, acc, pw,
+                 : stream_segment<4, M, D, SU, false>(sp, ep, e, lb, n, gb, rg, pr, policy, scale, acc, pw,
                                                       e_first, r_first, r, c, lane);
     } else {
-      ok = xi.ok ? stream_segment<8, M, D, SU, true>(sp, en, e, lb, n, gb, rg, pr, policy, scale, acc, pw, e_first,
+      ok = xi.ok ? stream_segment<8, M, D, SU, true>(sp, ep, e, lb, n, gb, rg, pr, policy, scale, acc, pw, e_first,
                                                      r_first, r, c, lane)
-                 : stream_segment<8, M, D, SU, false>(sp, en, e, lb, n, gb, rg, pr, policy, scale, acc, pw,
+                 : stream_segment<8, M, D, SU, false>(sp, ep, e, lb, n, gb, rg, pr, policy, scale, acc, pw,
                                                       e_first, r_first, r, c, lane);
     }
     if (!ok) break;
     left -= n;
     if (left > 0) {
-      en = sp.entries[++e];
+      ep = sp.entries + (++e);
       lb = 0;
     }
   }
@@ -685,9 +687,9 @@ __global__ void __launch_bounds__(NW * 32, 1) stream_kernel(const StackParams sp
     first = SplitTile{ef.y, ef.N, r_first, sp.counters + ef.tile_off + r_first, tile_g, tile_g + bpt};
   }
   if (c != 0) {
-    const int bpt = en.C / SU;
-    const long long tile_g = en.blk_off + static_cast<long long>(r) * bpt;
-    last = SplitTile{en.y, en.N, r, sp.counters + en.tile_off + r, tile_g, tile_g + bpt};
+    const int bpt = ep->C / SU;
+    const long long tile_g = ep->blk_off + static_cast<long long>(r) * bpt;
+    last = SplitTile{ep->y, ep->N, r, sp.counters + ep->tile_off + r, tile_g, tile_g + bpt};
     scale_acc(acc, scale);
     write_partial<M>(sp.partials, pw, tile_g <= gb ? 0 : 1, acc, lane);
   }

@@ -4,6 +4,7 @@
 // q4gemv_kernels.cuh.
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <atomic>
 #include <cstdarg>
 #include <cstdio>
@@ -524,6 +525,7 @@ struct q4_stack {
   // the stream kernel on every layer_stack_run
   q4k::XPrepJob* xprep_dev = nullptr;
   int xprep_jobs = 0;
+  int xprep_ctas = 1;  // CTAs per job
   int M = 1;
   void* workspace = nullptr;
   size_t workspace_bytes = 0;
@@ -670,6 +672,9 @@ int create_persistent(const q4_stack_entry* entries, int n, int M, int su, const
     if (err == cudaSuccess)
       err = cudaMemcpy(st->xprep_dev, jobs.data(), sizeof(q4k::XPrepJob) * jobs.size(), cudaMemcpyHostToDevice);
     st->xprep_jobs = static_cast<int>(jobs.size());
+    long long most = 0;
+    for (const auto& j : jobs) most = std::max(most, static_cast<long long>(M) * j.K / 8);
+    st->xprep_ctas = static_cast<int>(std::max(1LL, (most + q4k::kXPrepThreads - 1) / q4k::kXPrepThreads));
   }
   if (err == cudaSuccess) err = cudaMalloc(&st->entries_dev, sizeof(q4k::StackEntryDev) * host.size());
   if (err == cudaSuccess)
@@ -811,7 +816,7 @@ extern "C" Q4_API int layer_stack_run(q4_stack* st, void* stream) {
       // which has no grid barrier: a plain launch that starts its weight
       // copies while xprep_kernel runs and waits for it (griddepcontrol.wait)
       // before it reads an activation
-      q4k::xprep_kernel<<<st->xprep_jobs, q4k::kXPrepThreads, 0, s>>>(st->xprep_dev, st->M);
+      q4k::xprep_kernel<<<dim3(st->xprep_ctas, st->xprep_jobs), q4k::kXPrepThreads, 0, s>>>(st->xprep_dev, st->M);
       cudaError_t perr = cudaGetLastError();
       if (perr != cudaSuccess) return cuda_fail(perr, "layer_stack_run: xprep_kernel launch");
       attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;

@@ -319,11 +319,14 @@ __global__ void __launch_bounds__(NW * 32, 1) stack_kernel(const StackParams sp)
 }
 
 // ----------------------------------------------------------------------------
-// xprep_kernel: one CTA per activation tensor.  Finds the largest binary
+// xprep_kernel: grid (G, jobs).  Every CTA of a job scans the whole tensor
+// (16-byte loads; the tensor is small and L2-resident) for the largest binary
 // exponent emax and the lowest set significand bit lsb over the nonzero
-// elements; with sigma = emax - 15 every element scaled by 2^-sigma is below
-// 2^16 in magnitude (fp16 max 65504 > 1.9921875 * 2^15), and it is exact in
-// fp16 when its lowest set bit is at least 2^-24 (the fp16 subnormal step):
+// elements, so all G CTAs reach the same decision without a grid-wide sync;
+// then CTA g writes its share of the chunk-major copy.  With
+// sigma = emax - 15 every element scaled by 2^-sigma is below 2^16 in
+// magnitude (fp16 max 65504 > 1.9921875 * 2^15), and it is exact in fp16 when
+// its lowest set bit is at least 2^-24 (the fp16 subnormal step):
 // lsb - sigma >= -24 for every element.
 // ----------------------------------------------------------------------------
 constexpr int kXPrepThreads = 1024;
@@ -332,26 +335,37 @@ __device__ __forceinline__ float pow2_float(int e) {  // 2^e for e in [-149, 127
   return e >= -126 ? __int_as_float((e + 127) << 23) : __int_as_float(1 << (e + 149));
 }
 
+__device__ __forceinline__ void xprep_scan(uint32_t b, int& emax, int& lsb, int& bad) {
+  const int e = static_cast<int>((b >> 7) & 0xFF);
+  const uint32_t f = b & 0x7F;
+  if (e == 0xFF) {  // inf or NaN
+    bad = 1;
+  } else if (e != 0) {  // normal: (0x80 | f) * 2^(e - 134)
+    emax = max(emax, e - 127);
+    lsb = min(lsb, e - 134 + __ffs(static_cast<int>(0x80 | f)) - 1);
+  } else if (f != 0) {  // subnormal: f * 2^-133
+    emax = max(emax, -133 + 31 - __clz(static_cast<int>(f)));
+    lsb = min(lsb, -133 + __ffs(static_cast<int>(f)) - 1);
+  }
+}
+
+// M * K is a multiple of 8 and x is 16-byte aligned (K % 32 == 0 for every product).
 __global__ void __launch_bounds__(kXPrepThreads) xprep_kernel(const XPrepJob* jobs, int M) {
   asm volatile("griddepcontrol.launch_dependents;");
   asm volatile("griddepcontrol.wait;" ::: "memory");
   __shared__ int s_emax[32], s_lsb[32], s_bad[32];
   __shared__ int s_ok, s_sigma;
-  const XPrepJob j = jobs[blockIdx.x];
-  const long long n = static_cast<long long>(M) * j.K;
+  const XPrepJob j = jobs[blockIdx.y];
+  const long long n8 = static_cast<long long>(M) * j.K / 8;  // 16-byte groups of 8 values
+  const uint4* x8 = reinterpret_cast<const uint4*>(j.x);
   int emax = INT_MIN, lsb = INT_MAX, bad = 0;
-  for (long long i = threadIdx.x; i < n; i += blockDim.x) {
-    const uint32_t b = j.x[i];
-    const int e = static_cast<int>((b >> 7) & 0xFF);
-    const uint32_t f = b & 0x7F;
-    if (e == 0xFF) {  // inf or NaN
-      bad = 1;
-    } else if (e != 0) {  // normal: (0x80 | f) * 2^(e - 134)
-      emax = max(emax, e - 127);
-      lsb = min(lsb, e - 134 + __ffs(static_cast<int>(0x80 | f)) - 1);
-    } else if (f != 0) {  // subnormal: f * 2^-133
-      emax = max(emax, -133 + 31 - __clz(static_cast<int>(f)));
-      lsb = min(lsb, -133 + __ffs(static_cast<int>(f)) - 1);
+  for (long long i = threadIdx.x; i < n8; i += blockDim.x) {
+    const uint4 v = x8[i];
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      xprep_scan(w[q] & 0xFFFF, emax, lsb, bad);
+      xprep_scan(w[q] >> 16, emax, lsb, bad);
     }
   }
   for (int o = 16; o > 0; o >>= 1) {
@@ -379,23 +393,39 @@ __global__ void __launch_bounds__(kXPrepThreads) xprep_kernel(const XPrepJob* jo
     }
     s_ok = ok;
     s_sigma = sigma;
-    j.info->ok = ok;
-    j.info->sigma = sigma;
-    j.info->scale = pow2_float(sigma);
+    if (blockIdx.x == 0) {
+      j.info->ok = ok;
+      j.info->sigma = sigma;
+      j.info->scale = pow2_float(sigma);
+    }
   }
   __syncthreads();
   const bool f16 = s_ok != 0;
   const double down = ldexp(1.0, -s_sigma);
-  for (long long i = threadIdx.x; i < n; i += blockDim.x) {
-    const long long m = i / j.K, k = i - m * j.K;
-    const long long chunk = k / j.KC, kk = k - chunk * j.KC;
-    const uint16_t b = j.x[i];
-    uint16_t out = b;
+  // this CTA's share: 16-byte groups [g0, g1); a group is 8 consecutive k of
+  // one row, inside one chunk (KC is a multiple of 8), so it stays 16 contiguous
+  // bytes in the chunk-major copy
+  const long long per = (n8 + gridDim.x - 1) / gridDim.x;
+  const long long g0 = per * blockIdx.x, g1 = min(n8, g0 + per);
+  uint4* xc8 = reinterpret_cast<uint4*>(j.xc);
+  const long long k8 = j.K / 8, kc8 = j.KC / 8;
+  for (long long i = g0 + threadIdx.x; i < g1; i += blockDim.x) {
+    uint4 v = x8[i];
     if (f16) {
-      const float v = __uint_as_float(static_cast<uint32_t>(b) << 16);
-      out = __half_as_ushort(__double2half(static_cast<double>(v) * down));  // exact by the test above
+      uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const double lo = static_cast<double>(__uint_as_float(w[q] << 16)) * down;
+        const double hi = static_cast<double>(__uint_as_float(w[q] & 0xFFFF0000u)) * down;
+        // exact by the test above
+        w[q] = static_cast<uint32_t>(__half_as_ushort(__double2half(lo))) |
+               (static_cast<uint32_t>(__half_as_ushort(__double2half(hi))) << 16);
+      }
+      v = make_uint4(w[0], w[1], w[2], w[3]);
     }
-    j.xc[(chunk * M + m) * j.KC + kk] = out;
+    const long long m = i / k8, k = i - m * k8;  // row, group of 8 within the row
+    const long long chunk = k / kc8, kk = k - chunk * kc8;
+    xc8[(chunk * M + m) * kc8 + kk] = v;
   }
 }
 

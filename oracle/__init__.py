@@ -18,7 +18,8 @@ the sensitive projections and the output head (bs178.com llamAmpere post,
 "Why it is this fast", part two).  Group size 32, one fp16 scale per group and
 the symmetric [-8, 7] / [-127, 127] ranges are the plain reading the pages leave
 open; ``layout.py`` decodes the kernel-native packed layout from its written
-specification.
+specification, and ``quantize.py`` is the offline quantiser (bf16 weights to
+codes and fp16 scales) with every rounding step fixed.
 """
 from __future__ import annotations
 

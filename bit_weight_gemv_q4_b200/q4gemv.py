@@ -29,6 +29,8 @@ Q4_ERR_UNSUPPORTED = -7
 Q4_STACK_NO_PDL = 1
 Q4_STACK_GRAPH = 2
 Q4_STACK_INDEPENDENT = 4
+Q4_QUANT_ABSMAX = 0
+Q4_QUANT_SIGNED_MAX = 1
 
 ERROR_NAMES = {
     Q4_ERR_INVALID_ARG: "INVALID_ARG",
@@ -46,7 +48,7 @@ EXPORTED = [
     "q4_gemv_workspace_bytes",
     "q4_gemv", "q8_gemv", "q4_gemv_noalloc", "q4_workspace_check", "q4_set_wait_timeout_ns", "q4_unpack_device",
     "q4_selftest_wait_timeout", "layer_stack_create", "layer_stack_run", "layer_stack_check",
-    "layer_stack_launches", "layer_stack_destroy",
+    "layer_stack_launches", "layer_stack_destroy", "q4_quantize", "q4_quantize_device",
 ]
 
 
@@ -95,6 +97,8 @@ def _load() -> ctypes.CDLL:
         "layer_stack_check": ([vp, vp], i32),
         "layer_stack_launches": ([vp], i32),
         "layer_stack_destroy": ([vp], None),
+        "q4_quantize": ([i32, i32, vp, i64, i64, vp, vp], i32),
+        "q4_quantize_device": ([i32, i32, vp, i64, i64, vp, vp, vp], i32),
     }
     for name, (args, res) in sig.items():
         f = getattr(L, name)
@@ -175,6 +179,22 @@ def q4_unpack_weights(bits: int, packed: np.ndarray, N: int, K: int) -> tuple[np
     s = np.zeros((N, K // 32), dtype=np.uint16)
     _check(_lib.q4_unpack_weights(bits, packed.ctypes.data, packed.size, N, K, q.ctypes.data, s.ctypes.data))
     return q, s
+
+
+def q4_quantize(bits: int, mode: int, w_bf16: np.ndarray) -> tuple[np.ndarray, np.ndarray]:
+    """bf16 weight bits [N][K] (numpy, host) -> (canonical codes, fp16 scale bits [N][K/32])."""
+    w = np.ascontiguousarray(w_bf16, dtype=np.uint16)
+    N, K = w.shape
+    q = np.zeros((N, K // 2) if bits == 4 else (N, K), dtype=np.uint8 if bits == 4 else np.int8)
+    s = np.zeros((N, max(K // 32, 0)), dtype=np.uint16)
+    _check(_lib.q4_quantize(bits, mode, w.ctypes.data, N, K, q.ctypes.data, s.ctypes.data))
+    return q, s
+
+
+def q4_quantize_device(bits: int, mode: int, w_bf16, N: int, K: int, canon_q_out, scales_out, stream=None) -> None:
+    """The same on device tensors (bf16 bits [N][K] in, canonical codes and scales out)."""
+    _check(_lib.q4_quantize_device(bits, mode, _dev_ptr(w_bf16), N, K, _dev_ptr(canon_q_out), _dev_ptr(scales_out),
+                                   _stream(stream)))
 
 
 # ----------------------------------------------------------------------------
@@ -283,4 +303,5 @@ __all__ = [
     "q4_gemv_noalloc",
     "q4_workspace_check", "q4_set_wait_timeout_ns", "q4_unpack_device", "q4_selftest_wait_timeout",
     "layer_stack_create", "layer_stack_run", "layer_stack_check", "layer_stack_destroy",
+    "q4_quantize", "q4_quantize_device", "Q4_QUANT_ABSMAX", "Q4_QUANT_SIGNED_MAX",
 ]

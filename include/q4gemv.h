@@ -124,6 +124,38 @@ Q4_API int q4_pack_weights(int bits, const void* canon_q, const uint16_t* scales
 Q4_API int q4_pack_weights_device(int bits, const void* canon_q, const uint16_t* scales_fp16, int64_t N, int64_t K,
                                   void* out, size_t out_bytes, void* stream);
 
+/* ---------------------------------------------------------------------------
+ * Offline quantiser: bf16 weights -> canonical codes and fp16 scales (the
+ * input of q4_pack_weights).  Round to nearest, group 32 along K, symmetric
+ * (no zero point).  The pages name 4-bit and 8-bit formats and say that a
+ * quantiser's grouping and scale computation matter (jdon.com "Two RTX 3090s,
+ * 105 tok/s", section "Schools of quantisation"; bs178.com llamAmpere post,
+ * "Why it is this fast", part two) but give no recipe; this one fixes every
+ * rounding step, so host and device produce the same bits.  Per group of 32
+ * values w (fp32, exact from bf16):
+ *   ABSMAX:      s32 = max|w| / qmax   (qmax 7 for q4, 127 for q8), IEEE fp32 division
+ *   SIGNED_MAX:  s32 = w_m / -8        (q4 only; w_m the first value of largest
+ *                                       magnitude, which then gets the code -8)
+ *   s16 = fp16 of s32, round to nearest even, saturated to +-65504; s = s16 as fp32
+ *   q   = 0 if s == 0, else clamp(rint(w / s), lo, hi): IEEE division, ties to
+ *         even; [lo, hi] = [-7, 7] (ABSMAX q4), [-8, 7] (SIGNED_MAX), [-127, 127] (q8)
+ * ABSMAX never uses the q4 code -8; SIGNED_MAX uses all sixteen.  Weights must
+ * be finite.  Outputs: canonical q (q4: uint8 [N][K/2], low nibble = even k;
+ * q8: int8 [N][K]) and scales (fp16 bits [N][K/32]).
+ * -------------------------------------------------------------------------*/
+#define Q4_QUANT_ABSMAX 0
+#define Q4_QUANT_SIGNED_MAX 1
+
+/* Host: w_bf16 [N][K] in host memory, outputs in host memory.  Errors:
+ * INVALID_ARG (bits, mode, null), SHAPE (K % 32), ALIGN (2-byte w, scales). */
+Q4_API int q4_quantize(int bits, int mode, const uint16_t* w_bf16, int64_t N, int64_t K, void* canon_q_out,
+                       uint16_t* scales_out);
+
+/* Device: the same computation, every pointer device memory, asynchronous on
+ * `stream`; bit-identical to q4_quantize.  Errors: as q4_quantize, plus CUDA. */
+Q4_API int q4_quantize_device(int bits, int mode, const uint16_t* w_bf16, int64_t N, int64_t K, void* canon_q_out,
+                              uint16_t* scales_out, void* stream);
+
 /* Inverse of q4_pack_weights (host -> host): writes canonical q and scales.
  * Padding is dropped.  packed_bytes must be >= q4_packed_bytes. */
 Q4_API int q4_unpack_weights(int bits, const void* packed, size_t packed_bytes, int64_t N, int64_t K,

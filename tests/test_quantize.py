@@ -171,3 +171,96 @@ def test_canonical_layout_matches_the_nibble_convention():
             assert oracle.q4_value(c[n], k) == q[n, k]
     c8 = OQ.to_canonical(8, np.clip(q * 18, -127, 127))
     assert c8.dtype == np.int8 and np.array_equal(c8.astype(np.int32), np.clip(q * 18, -127, 127))
+
+
+# ---------------------------------------------------------------- library vs oracle
+def _finite_bf16_patterns(N, K, seed):
+    """Every kind of finite bf16: random bit patterns (subnormals, huge values,
+    signed zeros) with the inf/NaN exponent replaced."""
+    rng = np.random.default_rng(seed)
+    b = rng.integers(0, 1 << 16, (N, K), dtype=np.uint32).astype(np.uint16)
+    bad = (b & 0x7F80) == 0x7F80
+    b[bad] &= 0xBFFF  # exponent 0x7F -> 0x3F
+    b[0, :32] = 0x8000  # a group of negative zeros
+    b[0, 32:64] = 0x0001  # smallest subnormals
+    return b
+
+
+def _weight_cases():
+    yield "normal", _bf16_bits(RNG.normal(0, 0.02, (37, 256)))
+    yield "patterns", _finite_bf16_patterns(23, 128, 7)
+    yield "ties", _bf16_bits(np.round(RNG.normal(0, 1, (9, 64)) * 4) / 8)
+
+
+@pytest.mark.parametrize("bits,mode", [(4, OQ.ABSMAX), (4, OQ.SIGNED_MAX), (8, OQ.ABSMAX)])
+def test_host_quantiser_is_bit_exact(bits, mode):
+    import bit_weight_gemv_q4_b200 as q4
+
+    for name, wb in _weight_cases():
+        q, s = q4.q4_quantize(bits, mode, wb)
+        qo, so = OQ.quantize(bits, mode, wb)
+        assert np.array_equal(s, so), name
+        assert np.array_equal(q.view(np.uint8), qo.view(np.uint8)), name
+
+
+def test_quantiser_argument_errors():
+    import bit_weight_gemv_q4_b200 as q4
+
+    w = np.zeros((2, 64), dtype=np.uint16)
+    with pytest.raises(q4.Q4Error):
+        q4.q4_quantize(8, q4.Q4_QUANT_SIGNED_MAX, w)  # signed mode is q4 only
+    with pytest.raises(q4.Q4Error):
+        q4.q4_quantize(5, q4.Q4_QUANT_ABSMAX, w)
+    with pytest.raises(q4.Q4Error):
+        q4.q4_quantize(4, q4.Q4_QUANT_ABSMAX, np.zeros((2, 48), dtype=np.uint16))  # K % 32
+    q, s = q4.q4_quantize(4, q4.Q4_QUANT_ABSMAX, np.zeros((0, 64), dtype=np.uint16))
+    assert q.size == 0 and s.size == 0
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("bits,mode", [(4, OQ.ABSMAX), (4, OQ.SIGNED_MAX), (8, OQ.ABSMAX)])
+def test_device_quantiser_is_bit_exact(cuda_device, bits, mode):
+    import torch
+
+    import bit_weight_gemv_q4_b200 as q4
+
+    for name, wb in _weight_cases():
+        N, K = wb.shape
+        w = torch.from_numpy(wb.view(np.int16)).cuda()
+        q = torch.zeros(N * (K // 2 if bits == 4 else K), dtype=torch.uint8, device="cuda")
+        s = torch.zeros(N * (K // 32), dtype=torch.int16, device="cuda")
+        q4.q4_quantize_device(bits, mode, w, N, K, q, s)
+        torch.cuda.synchronize()
+        qo, so = OQ.quantize(bits, mode, wb)
+        assert np.array_equal(s.cpu().numpy().view(np.uint16).reshape(N, K // 32), so), name
+        assert np.array_equal(q.cpu().numpy().reshape(qo.shape), qo.view(np.uint8)), name
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("bits,mode", [(4, OQ.SIGNED_MAX), (8, OQ.ABSMAX)])
+def test_quantise_pack_and_multiply_on_the_device(cuda_device, bits, mode):
+    """bf16 weights -> device quantiser -> device packer -> product, against
+    the oracle product of the oracle's quantisation of the same weights."""
+    import torch
+
+    import bit_weight_gemv_q4_b200 as q4
+    from bit_weight_gemv_q4_b200 import synth
+
+    N, K, M = 300, 1024, 2
+    wb = _bf16_bits(RNG.normal(0, 0.02, (N, K)))
+    w = torch.from_numpy(wb.view(np.int16)).cuda()
+    q = torch.zeros(N * (K // 2 if bits == 4 else K), dtype=torch.uint8, device="cuda")
+    s = torch.zeros(N * (K // 32), dtype=torch.int16, device="cuda")
+    q4.q4_quantize_device(bits, mode, w, N, K, q, s)
+    packed = torch.zeros(q4.q4_packed_bytes(bits, N, K), dtype=torch.uint8, device="cuda")
+    q4.q4_pack_weights_device(bits, q, s, N, K, packed)
+    x = synth.activations(9, synth.act_stream(77), M, K)
+    xd = torch.from_numpy(np.ascontiguousarray(x).view(np.int16)).cuda()
+    y = torch.empty(M * N, dtype=torch.float32, device="cuda")
+    ws = torch.zeros(q4.q4_gemv_workspace_bytes(bits, N, K, M), dtype=torch.uint8, device="cuda")
+    (q4.q4_gemv if bits == 4 else q4.q8_gemv)(packed, N, K, xd, M, y, ws)
+    q4.q4_workspace_check(ws)
+    qo, so = OQ.quantize(bits, mode, wb)
+    y_ref, B = oracle.gemv(bits, qo, so, x)
+    ok, _, _ = oracle.within_tolerance(y.cpu().numpy().reshape(M, N).astype(np.float64), y_ref, B)
+    assert ok.all()

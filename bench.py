@@ -316,7 +316,34 @@ def per_config(args, d: Dist, torch, q4, workloads, peak):
         res[f"layer_q4_M{M}"] = layer
     for h in workloads.draft_heads():
         res[f"{h.name}_q8_{h.N}x{h.K}_M1"] = shape(h.name, h.bits, h.N, h.K, 1, 3900 + h.tensor_id)
+    res["quantize"] = quantize_rates(args, d, torch, q4, peak)
     return res
+
+
+def quantize_rates(args, d: Dist, torch, q4, peak):
+    """The offline quantiser on the device: bf16 weights of a gate|up-sized
+    tensor (q4) and of the full vocabulary head (q8) to codes and scales; GB/s
+    of bytes moved (2 B read per weight, codes and scales written)."""
+    out = {}
+    stream = torch.cuda.current_stream()
+    for name, bits, mode, N, K in (("q4_signed_34816x5120", 4, q4.Q4_QUANT_SIGNED_MAX, 34816, 5120),
+                                   ("q8_absmax_248320x5120", 8, q4.Q4_QUANT_ABSMAX, 248320, 5120)):
+        g = torch.Generator(device="cuda")
+        g.manual_seed(args.seed)
+        w = (torch.randn(N, K, device="cuda", generator=g) * 0.02).to(torch.bfloat16).view(torch.int16)
+        q = torch.empty(N * (K // 2 if bits == 4 else K), dtype=torch.uint8, device="cuda")
+        s = torch.empty(N * (K // 32), dtype=torch.int16, device="cuda")
+        run = lambda: q4.q4_quantize_device(bits, mode, w, N, K, q, s)  # noqa: E731
+        for _ in range(3):
+            run()
+        n = 10
+        ms = d.max(time_region(torch, run, n, stream) / n)
+        moved = N * K * 2 + q.numel() + s.numel() * 2
+        out[name] = {"us": round(ms * 1e3, 1), "GBps": round(moved / (ms * 1e6), 1),
+                     "pct_of_hbm_peak": round(100 * moved / (ms * 1e6) / peak, 1), "bytes_moved": moved}
+        del w, q, s
+        torch.cuda.empty_cache()
+    return out
 
 
 def run_ours(args, d: Dist):

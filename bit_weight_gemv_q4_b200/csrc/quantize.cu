@@ -10,7 +10,14 @@
 //   s32 = w_m / -8                      (signed, q4 only; w_m the first value of
 //                                        largest magnitude)
 //   s16 = fp16(s32), nearest even, saturated to +-65504;  s = s16 as fp32
-//   q   = 0 if s == 0, else clamp(rint(w / s), lo, hi)   (IEEE division, ties to even)
+//   q   = 0 if s == 0, else clamp(nearest(w / s), lo, hi): the integer nearest
+//         to the exact quotient, ties to even
+// The host forms the quotient in fp64 (w has an 8-bit, s an 11-bit
+// significand: a quotient above 1/2 that is not half-way lies >= 2^-21 from
+// the half-way point, beyond fp64's rounding, so rint decides exactly).  The
+// device takes a candidate from a reciprocal multiply (within one of the
+// nearest integer) and settles it with the exact remainder w - q s (one FMA;
+// exact by Sterbenz's lemma, as q s is within a factor 2 of w).
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
@@ -131,8 +138,8 @@ void quantize_group_host(int bits, int mode, const QRange& r, const uint16_t* w,
   for (int i = 0; i < 32; ++i) {
     int q = 0;
     if (s != 0.f) {
-      float v = std::rint(wf[i] / s);
-      v = std::fmin(std::fmax(v, static_cast<float>(r.lo)), static_cast<float>(r.hi));
+      double v = std::rint(static_cast<double>(wf[i]) / static_cast<double>(s));
+      v = std::fmin(std::fmax(v, static_cast<double>(r.lo)), static_cast<double>(r.hi));
       q = static_cast<int>(v);
     }
     if (bits == 8) {
@@ -146,40 +153,113 @@ void quantize_group_host(int bits, int mode, const QRange& r, const uint16_t* w,
 }
 
 // ---------------------------------------------------------------- device
-// One warp per group: lane i holds w[i]; the warp finds the largest magnitude
-// (and, for the signed mode, the first lane holding it), lane 0 writes the
-// scale, every lane its code (q4: even lanes write the byte of a pair).
-__global__ void quantize_kernel(int bits, int mode, int lo, int hi, float qmax, const uint16_t* __restrict__ w,
-                                long long N, long long K, uint8_t* __restrict__ q_out, uint16_t* __restrict__ s_out) {
-  const long long G = K / 32;
-  const long long grp = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
-  const int lane = threadIdx.x & 31;
-  if (grp >= N * G) return;  // whole warps leave together (32 threads per group)
-  const long long n = grp / G, g = grp - n * G;
-  const float wf = __uint_as_float(static_cast<uint32_t>(w[n * K + 32 * g + lane]) << 16);
-  float amax = fabsf(wf);
-  int first = lane;
-  for (int o = 16; o > 0; o >>= 1) {
-    const float oa = __shfl_xor_sync(0xFFFFFFFFu, amax, o);
-    const int of = __shfl_xor_sync(0xFFFFFFFFu, first, o);
-    if (oa > amax || (oa == amax && of < first)) {
-      amax = oa;
-      first = of;
+constexpr int kQuantGroupsPerLane = 2;  // loads in flight per thread
+
+// One group-part: a lane holds eight values of a group (four lanes per group).
+// The lane finds the largest magnitude among its values (the first on ties),
+// the four lanes combine theirs in lane order, the group's first lane writes
+// the scale, and every lane its eight codes (q4: one 32-bit store, q8: one
+// 64-bit store).  All 32 lanes run it (the shuffles need them); `live` lanes
+// store.
+__device__ __forceinline__ void quantize_part(int bits, int mode, int lo, int hi, float qmax, const uint4 v, bool live,
+                                              int part, long long n, long long g, long long G, long long K,
+                                              uint8_t* __restrict__ q_out, uint16_t* __restrict__ s_out) {
+  const uint32_t words[4] = {v.x, v.y, v.z, v.w};
+  float wf[8];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    wf[2 * i] = __uint_as_float(words[i] << 16);
+    wf[2 * i + 1] = __uint_as_float(words[i] & 0xFFFF0000u);
+  }
+  float amax = fabsf(wf[0]), wm = wf[0];
+#pragma unroll
+  for (int i = 1; i < 8; ++i) {
+    if (fabsf(wf[i]) > amax) {
+      amax = fabsf(wf[i]);
+      wm = wf[i];
     }
   }
-  const float wm = __shfl_sync(0xFFFFFFFFu, wf, first);
+  // combine the four lanes of the group: a later lane wins only if strictly larger
+#pragma unroll
+  for (int o = 1; o < 4; o <<= 1) {
+    const float oa = __shfl_xor_sync(0xFFFFFFFFu, amax, o);
+    const float ow = __shfl_xor_sync(0xFFFFFFFFu, wm, o);
+    const int opart = part ^ o;
+    if (oa > amax || (oa == amax && opart < part)) {
+      amax = oa;
+      wm = ow;
+    }
+  }
+  if (!live) return;
   const float s32 = mode == Q4_QUANT_ABSMAX ? __fdiv_rn(amax, qmax) : __fdiv_rn(wm, -8.f);
   __half h = __float2half_rn(s32);
   if (__hisinf(h)) h = __float2half_rn(s32 > 0.f ? 65504.f : -65504.f);
   const float s = __half2float(h);
-  if (lane == 0) s_out[n * G + g] = __half_as_ushort(h);
-  int q = 0;
-  if (s != 0.f) q = static_cast<int>(fminf(fmaxf(rintf(__fdiv_rn(wf, s)), static_cast<float>(lo)), static_cast<float>(hi)));
+  if (part == 0) s_out[n * G + g] = __half_as_ushort(h);
+  int q[8];
+  // any reciprocal within a few ulp will do: the candidate it gives is within
+  // one of the nearest integer, and the exact remainder settles the rest
+  const float rcp = s != 0.f ? __fdividef(1.f, s) : 0.f;
+  const float half = 0.5f * fabsf(s);
+  const bool s_pos = s > 0.f;  // the quotient grows with w - q s when s > 0
+  // adding 1.5 * 2^23 to a float below 2^22 in magnitude rounds it to an
+  // integer (nearest, ties to even) held in the low mantissa bits, exactly
+  constexpr float kMagic = 12582912.f;
+  constexpr int kMagicBits = 0x4B400000;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    // candidate within one of the nearest integer, kept small
+    const float x = fminf(fmaxf(wf[i] * rcp, static_cast<float>(lo - 1)), static_cast<float>(hi + 1));
+    const float cm = x + kMagic;
+    const float c = cm - kMagic;
+    int ci = __float_as_int(cm) - kMagicBits;
+    const float rem = fmaf(-c, s, wf[i]);  // exact: w - c s
+    const float ar = fabsf(rem);
+    const int step = ((rem > 0.f) == s_pos) ? 1 : -1;
+    if (ar > half || (ar == half && (ci & 1))) ci += step;  // past half-way, or a tie to the even one
+    q[i] = s != 0.f ? min(max(ci, lo), hi) : 0;
+  }
+  const long long base = n * K + 32 * g + 8 * part;
   if (bits == 8) {
-    reinterpret_cast<int8_t*>(q_out)[n * K + 32 * g + lane] = static_cast<int8_t>(q);
+    uint32_t lo4 = 0, hi4 = 0;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      lo4 |= static_cast<uint32_t>(q[i] & 0xFF) << (8 * i);
+      hi4 |= static_cast<uint32_t>(q[4 + i] & 0xFF) << (8 * i);
+    }
+    *reinterpret_cast<uint2*>(q_out + base) = make_uint2(lo4, hi4);
   } else {
-    const int odd = __shfl_down_sync(0xFFFFFFFFu, q, 1);
-    if ((lane & 1) == 0) q_out[n * (K / 2) + 16 * g + lane / 2] = static_cast<uint8_t>((q & 0xF) | ((odd & 0xF) << 4));
+    uint32_t nib = 0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) nib |= static_cast<uint32_t>(q[i] & 0xF) << (4 * i);
+    *reinterpret_cast<uint32_t*>(q_out + base / 2) = nib;
+  }
+}
+
+// Grid (ceil(4 G / 256), rows): thread t of the x dimension handles part
+// t % 4 of group t / 4 of rows blockIdx.y, blockIdx.y + gridDim.y, ...; the
+// loads of kQuantGroupsPerLane rows are issued together.  (32-bit index math:
+// a 64-bit division per group would cost more than the quantisation.)
+__global__ void quantize_kernel(int bits, int mode, int lo, int hi, float qmax, const uint16_t* __restrict__ w,
+                                long long N, long long K, uint8_t* __restrict__ q_out, uint16_t* __restrict__ s_out) {
+  const int G = static_cast<int>(K / 32);
+  const int t = blockIdx.x * blockDim.x + threadIdx.x;
+  const int g = t >> 2, part = t & 3;
+  const bool in_row = g < G;
+  for (long long n0 = blockIdx.y; n0 < N; n0 += static_cast<long long>(gridDim.y) * kQuantGroupsPerLane) {
+    uint4 v[kQuantGroupsPerLane];
+#pragma unroll
+    for (int j = 0; j < kQuantGroupsPerLane; ++j) {
+      const long long n = n0 + static_cast<long long>(j) * gridDim.y;
+      v[j] = make_uint4(0, 0, 0, 0);
+      if (in_row && n < N) v[j] = __ldcs(reinterpret_cast<const uint4*>(w + n * K + 32 * g + 8 * part));
+    }
+#pragma unroll
+    for (int j = 0; j < kQuantGroupsPerLane; ++j) {
+      const long long n = n0 + static_cast<long long>(j) * gridDim.y;
+      if (n >= N) break;  // the same for the whole block
+      quantize_part(bits, mode, lo, hi, qmax, v[j], in_row, part, n, g, G, K, q_out, s_out);
+    }
   }
 }
 
@@ -208,10 +288,14 @@ extern "C" Q4_API int q4_quantize_device(int bits, int mode, const uint16_t* w_b
   if (rc) return rc;
   const long long groups = N * (K / 32);
   if (groups == 0) return Q4_OK;
-  const int threads = 256;
-  const long long blocks = (groups * 32 + threads - 1) / threads;
-  if (blocks > 0x7FFFFFFFLL) return qfail(Q4_ERR_SHAPE, "q4_quantize_device: too many groups");
-  quantize_kernel<<<static_cast<unsigned>(blocks), threads, 0, static_cast<cudaStream_t>(stream)>>>(
+  if (reinterpret_cast<uintptr_t>(w_bf16) % 16 || reinterpret_cast<uintptr_t>(canon_q_out) % 8)
+    return qfail(Q4_ERR_ALIGN, "q4_quantize_device: weights must be 16-byte and codes 8-byte aligned");
+  const int threads = 128;
+  const long long G = K / 32;
+  const long long passes = (N + kQuantGroupsPerLane - 1) / kQuantGroupsPerLane;  // rows handled together
+  const dim3 grid(static_cast<unsigned>((4 * G + threads - 1) / threads),
+                  static_cast<unsigned>(passes < 65535 ? passes : 65535));
+  quantize_kernel<<<grid, threads, 0, static_cast<cudaStream_t>(stream)>>>(
       bits, mode, r.lo, r.hi, r.qmax, w_bf16, N, K, static_cast<uint8_t*>(canon_q_out), scales_out);
   const cudaError_t err = cudaGetLastError();
   if (err != cudaSuccess)

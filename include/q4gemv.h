@@ -151,8 +151,9 @@ Q4_API int q4_pack_weights_device(int bits, const void* canon_q, const uint16_t*
 Q4_API int q4_quantize(int bits, int mode, const uint16_t* w_bf16, int64_t N, int64_t K, void* canon_q_out,
                        uint16_t* scales_out);
 
-/* Device: the same computation, every pointer device memory, asynchronous on
- * `stream`; bit-identical to q4_quantize.  Errors: as q4_quantize, plus CUDA. */
+/* Device: the same computation, every pointer device memory (w 16-byte and
+ * codes 8-byte aligned), asynchronous on `stream`; bit-identical to
+ * q4_quantize.  Errors: as q4_quantize, plus CUDA. */
 Q4_API int q4_quantize_device(int bits, int mode, const uint16_t* w_bf16, int64_t N, int64_t K, void* canon_q_out,
                               uint16_t* scales_out, void* stream);
 

@@ -1,13 +1,13 @@
 """CPU oracle of the offline quantiser -- TEST INFRASTRUCTURE (see __init__.py).
 
 Round-to-nearest, group-32, symmetric (no zero point) quantisation of bf16
-weights into the canonical code and scale layout, written as plain numpy in
-fp32 arithmetic, step by step.  The pages say only that a quantiser's grouping,
+weights into the canonical code and scale layout, written as plain numpy,
+step by step.  The pages say only that a quantiser's grouping,
 scale computation and outlier handling matter (jdon.com "Two RTX 3090s, 105
 tok/s", section "Schools of quantisation") and name 4-bit and 8-bit formats
 (bs178.com llamAmpere post, "Why it is this fast", part two); the recipe below
 is the plain reading, with every rounding step fixed so that any faithful
-implementation in fp32 produces the same bits:
+implementation produces the same bits:
 
 For each row n and group g (32 consecutive k), with w the group's values as
 fp32 (exact from bf16):
@@ -17,9 +17,17 @@ fp32 (exact from bf16):
                                                            magnitude, first in k order
   s16 = fp16 round-to-nearest-even of s32, saturated to +-65504
   s   = s16 as fp32
-  q   = 0 if s == 0, else clamp(rint(w / s), lo, hi)       fp32 division, ties to even;
+  q   = 0 if s == 0, else clamp(nearest(w / s), lo, hi)    the integer nearest to the
+                                                           exact quotient, ties to even;
                                                            [lo, hi] = [-7, 7] absmax q4,
                                                            [-8, 7] signed q4, [-127, 127] q8
+
+The quotient is formed in fp64 here: w has an 8-bit and s an 11-bit
+significand, so a quotient that is not exactly half-way between two integers
+lies at least 2^-21 from that half-way point whenever it is above 1/2 in
+magnitude, far beyond the fp64 rounding error (2^-45 at most), and an exact
+half-way quotient is exactly representable: rint of the fp64 quotient is the
+nearest integer of the exact one, ties to even.
 
 Absmax mode never uses the code -8; signed mode maps the largest-magnitude
 value to -8 exactly and so uses all sixteen codes.  The outputs are the
@@ -74,7 +82,7 @@ def quantize_ints(bits: int, mode: int, w_bits: np.ndarray) -> tuple[np.ndarray,
     s = s16.astype(np.float32)[..., None]
     lo, hi = code_range(bits, mode)
     with np.errstate(divide="ignore", invalid="ignore"):
-        ratio = (wf / np.where(s == 0, np.float32(1.0), s)).astype(np.float32)
+        ratio = wf.astype(np.float64) / np.where(s == 0, np.float32(1.0), s).astype(np.float64)
     q = np.clip(np.rint(ratio), lo, hi)
     q = np.where(s == 0, 0, q).astype(np.int32)
     return q.reshape(N, K), s16.view(np.uint16)

@@ -81,8 +81,7 @@ def test_scales_follow_the_stated_rounding_exactly(bits, mode):
 @pytest.mark.parametrize("bits,mode", [(4, OQ.ABSMAX), (4, OQ.SIGNED_MAX), (8, OQ.ABSMAX)])
 def test_codes_are_the_nearest_in_range(bits, mode):
     """Brute force in exact arithmetic: each code is the integer in range
-    nearest to w / s (ties to even), except where the fp32 quotient differs
-    from the exact one across a tie (|w/s - (j + 1/2)| below 2^-20)."""
+    nearest to the exact quotient w / s, ties to even."""
     wb = _groups()
     q, s = OQ.quantize_ints(bits, mode, wb)
     lo, hi = OQ.code_range(bits, mode)
@@ -96,9 +95,7 @@ def test_codes_are_the_nearest_in_range(bits, mode):
                 continue
             r = Fraction(float(wf[n, k])) / sv
             best = min(range(lo, hi + 1), key=lambda j: (abs(r - j), j % 2))
-            if q[n, k] != best:
-                frac = r - math.floor(r)
-                assert abs(frac - Fraction(1, 2)) < Fraction(1, 2 ** 20), (n, k, float(r), q[n, k], best)
+            assert q[n, k] == best, (n, k, float(r), q[n, k], best)
 
 
 def test_hand_worked_group():

@@ -15,6 +15,7 @@
 
 #include "q4gemv.h"
 #include "q4gemv_kernels.cuh"
+#include "q4chain_kernel.cuh"
 #include "q4stack_kernel.cuh"
 
 namespace q4 {
@@ -793,6 +794,180 @@ extern "C" Q4_API int layer_stack_create(const q4_stack_entry* entries, int n_en
   if (rc) {
     free_stack(st);
     return rc;
+  }
+  *out = st;
+  return Q4_OK;
+}
+
+namespace {
+
+int launch_pdl(const void* fn, dim3 grid, dim3 block, void** args, cudaStream_t stream, bool pdl, const char* who) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  const cudaError_t err = cudaLaunchKernelExC(&cfg, fn, args);
+  return err == cudaSuccess ? Q4_OK : cuda_fail(err, who);
+}
+
+bool misaligned(const void* p, uintptr_t a) { return reinterpret_cast<uintptr_t>(p) % a != 0; }
+
+int check_chain_op(const q4_chain_op& op, int i) {
+  char who[64];
+  snprintf(who, sizeof(who), "layer_chain_create op %d", i);
+  if (op.kind == Q4_OP_PRODUCT) {
+    Shape s;
+    return make_shape(op.bits, op.N, op.K, &s, who);
+  }
+  if (op.kind != Q4_OP_RESIDUAL_RMSNORM && op.kind != Q4_OP_SWIGLU)
+    return fail(Q4_ERR_INVALID_ARG, "%s: unknown kind %d", who, op.kind);
+  if (op.N <= 0 || op.N > (int64_t(1) << 30)) return fail(Q4_ERR_SHAPE, "%s: N must be in 1..2^30", who);
+  if (!op.out) return fail(Q4_ERR_INVALID_ARG, "%s: out is null", who);
+  if (misaligned(op.out, 2)) return fail(Q4_ERR_ALIGN, "%s: out must be 2-byte aligned", who);
+  if (op.kind == Q4_OP_RESIDUAL_RMSNORM) {
+    if (!op.resid) return fail(Q4_ERR_INVALID_ARG, "%s: resid is null", who);
+    if (op.bits == 1 && !op.in) return fail(Q4_ERR_INVALID_ARG, "%s: a setting norm needs in", who);
+    if (misaligned(op.resid, 4) || misaligned(op.in, 4) || misaligned(op.packed, 2))
+      return fail(Q4_ERR_ALIGN, "%s: resid and in must be 4-byte, gamma 2-byte aligned", who);
+  } else {
+    if (!op.in) return fail(Q4_ERR_INVALID_ARG, "%s: in is null", who);
+    if (misaligned(op.in, 4)) return fail(Q4_ERR_ALIGN, "%s: in must be 4-byte aligned", who);
+  }
+  return Q4_OK;
+}
+
+}  // namespace
+
+extern "C" Q4_API int q4_residual_rmsnorm(float* h, const float* y, const uint16_t* gamma, uint16_t* x, int64_t N,
+                                          int M, int set, void* stream) {
+  q4_chain_op op{};
+  op.kind = Q4_OP_RESIDUAL_RMSNORM;
+  op.bits = set ? 1 : 0;
+  op.N = N;
+  op.packed = gamma;
+  op.in = y;
+  op.out = x;
+  op.resid = h;
+  int rc = check_chain_op(op, 0);
+  if (rc) return rc;
+  if (M < 1 || M > 4) return fail(Q4_ERR_INVALID_ARG, "q4_residual_rmsnorm: M must be in 1..4");
+  int Ni = static_cast<int>(N), seti = set ? 1 : 0;
+  float eps = 1e-6f;
+  void* args[] = {&h, &y, &gamma, &x, &Ni, &eps, &seti};
+  return launch_pdl(reinterpret_cast<const void*>(&q4k::residual_rmsnorm_kernel), dim3(M), dim3(q4k::kNormThreads),
+                    args, static_cast<cudaStream_t>(stream), true, "q4_residual_rmsnorm: launch");
+}
+
+extern "C" Q4_API int q4_swiglu(const float* y_gu, uint16_t* x, int64_t N, int M, void* stream) {
+  q4_chain_op op{};
+  op.kind = Q4_OP_SWIGLU;
+  op.N = N;
+  op.in = y_gu;
+  op.out = x;
+  int rc = check_chain_op(op, 0);
+  if (rc) return rc;
+  if (M < 1 || M > 4) return fail(Q4_ERR_INVALID_ARG, "q4_swiglu: M must be in 1..4");
+  int Ni = static_cast<int>(N), Mi = M;
+  void* args[] = {&y_gu, &x, &Ni, &Mi};
+  const long long total = static_cast<long long>(M) * N;
+  return launch_pdl(reinterpret_cast<const void*>(&q4k::swiglu_kernel), dim3(static_cast<unsigned>((total + 255) / 256)),
+                    dim3(256), args, static_cast<cudaStream_t>(stream), true, "q4_swiglu: launch");
+}
+
+extern "C" Q4_API int layer_chain_create(const q4_chain_op* ops, int n_ops, int M, int flags, q4_stack** out) {
+  if (!out) return fail(Q4_ERR_INVALID_ARG, "layer_chain_create: out is null");
+  *out = nullptr;
+  if (n_ops < 0 || (n_ops > 0 && !ops)) return fail(Q4_ERR_INVALID_ARG, "layer_chain_create: bad op list");
+  if (M < 1 || M > 4) return fail(Q4_ERR_INVALID_ARG, "layer_chain_create: M must be in 1..4");
+  DeviceInfo dev;
+  int rc = device_info(&dev);
+  if (rc) return rc;
+  size_t ws = kWsHeader;
+  for (int i = 0; i < n_ops; ++i) {
+    if ((rc = check_chain_op(ops[i], i))) return rc;
+    if (ops[i].kind == Q4_OP_PRODUCT) {
+      Shape s;
+      make_shape(ops[i].bits, ops[i].N, ops[i].K, &s, "layer_chain_create");
+      ws = std::max(ws, workspace_bytes(s, M, dev));
+    }
+  }
+  q4_stack* st = new q4_stack();
+  cudaGetDevice(&st->device);
+  cudaError_t err = cudaMalloc(&st->workspace, ws);
+  if (err == cudaSuccess) err = cudaMemset(st->workspace, 0, ws);
+  if (err != cudaSuccess) {
+    free_stack(st);
+    return cuda_fail(err, "layer_chain_create: workspace");
+  }
+  st->workspace_bytes = ws;
+  std::vector<Launch> products(static_cast<size_t>(n_ops));
+  for (int i = 0; i < n_ops; ++i) {
+    if (ops[i].kind != Q4_OP_PRODUCT) continue;
+    char who[64];
+    snprintf(who, sizeof(who), "layer_chain_create op %d", i);
+    rc = prepare(ops[i].bits, ops[i].packed, ops[i].N, ops[i].K, static_cast<const uint16_t*>(ops[i].in), M,
+                 static_cast<float*>(ops[i].out), st->workspace, ws, who, &products[static_cast<size_t>(i)]);
+    if (rc) {
+      free_stack(st);
+      return rc;
+    }
+  }
+  cudaStream_t cs = nullptr;
+  err = cudaStreamCreateWithFlags(&cs, cudaStreamNonBlocking);
+  if (err == cudaSuccess) err = cudaStreamBeginCapture(cs, cudaStreamCaptureModeThreadLocal);
+  if (err != cudaSuccess) {
+    if (cs) cudaStreamDestroy(cs);
+    free_stack(st);
+    return cuda_fail(err, "layer_chain_create: begin capture");
+  }
+  const bool pdl = (flags & Q4_STACK_NO_PDL) == 0;
+  for (int i = 0; i < n_ops && rc == Q4_OK; ++i) {
+    const q4_chain_op& op = ops[i];
+    if (op.kind == Q4_OP_PRODUCT) {
+      Launch& L = products[static_cast<size_t>(i)];
+      if (L.noop) continue;
+      rc = launch(L, cs, pdl);
+    } else if (op.kind == Q4_OP_RESIDUAL_RMSNORM) {
+      float* h = op.resid;
+      const float* y = static_cast<const float*>(op.in);
+      const uint16_t* gamma = static_cast<const uint16_t*>(op.packed);
+      uint16_t* x = static_cast<uint16_t*>(op.out);
+      int N = static_cast<int>(op.N);
+      float eps = 1e-6f;
+      int set = op.bits == 1 ? 1 : 0;
+      void* args[] = {&h, &y, &gamma, &x, &N, &eps, &set};
+      rc = launch_pdl(reinterpret_cast<const void*>(&q4k::residual_rmsnorm_kernel), dim3(M), dim3(q4k::kNormThreads),
+                      args, cs, pdl, "layer_chain_create: rmsnorm launch");
+    } else {
+      const float* y = static_cast<const float*>(op.in);
+      uint16_t* x = static_cast<uint16_t*>(op.out);
+      int N = static_cast<int>(op.N), Mi = M;
+      void* args[] = {&y, &x, &N, &Mi};
+      const long long total = static_cast<long long>(M) * op.N;
+      rc = launch_pdl(reinterpret_cast<const void*>(&q4k::swiglu_kernel),
+                      dim3(static_cast<unsigned>((total + 255) / 256)), dim3(256), args, cs, pdl,
+                      "layer_chain_create: swiglu launch");
+    }
+    if (rc == Q4_OK) ++st->launches;
+  }
+  cudaGraph_t graph = nullptr;
+  const cudaError_t end_err = cudaStreamEndCapture(cs, &graph);
+  cudaStreamDestroy(cs);
+  if (rc || end_err != cudaSuccess) {
+    if (graph) cudaGraphDestroy(graph);
+    free_stack(st);
+    return rc ? rc : cuda_fail(end_err, "layer_chain_create: end capture");
+  }
+  st->graph = graph;
+  err = cudaGraphInstantiate(&st->exec, graph, 0);
+  if (err != cudaSuccess) {
+    free_stack(st);
+    return cuda_fail(err, "layer_chain_create: cudaGraphInstantiate");
   }
   *out = st;
   return Q4_OK;

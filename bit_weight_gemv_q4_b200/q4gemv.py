@@ -31,6 +31,9 @@ Q4_STACK_GRAPH = 2
 Q4_STACK_INDEPENDENT = 4
 Q4_QUANT_ABSMAX = 0
 Q4_QUANT_SIGNED_MAX = 1
+Q4_OP_PRODUCT = 0
+Q4_OP_RESIDUAL_RMSNORM = 1
+Q4_OP_SWIGLU = 2
 
 ERROR_NAMES = {
     Q4_ERR_INVALID_ARG: "INVALID_ARG",
@@ -48,7 +51,8 @@ EXPORTED = [
     "q4_gemv_workspace_bytes",
     "q4_gemv", "q8_gemv", "q4_gemv_noalloc", "q4_workspace_check", "q4_set_wait_timeout_ns", "q4_unpack_device",
     "q4_selftest_wait_timeout", "layer_stack_create", "layer_stack_run", "layer_stack_check",
-    "layer_stack_launches", "layer_stack_destroy", "q4_quantize", "q4_quantize_device",
+    "layer_stack_launches", "layer_stack_destroy", "q4_quantize", "q4_quantize_device", "layer_chain_create",
+    "q4_residual_rmsnorm", "q4_swiglu",
 ]
 
 
@@ -66,6 +70,19 @@ class StackEntry(ctypes.Structure):
         ("packed", ctypes.c_void_p),
         ("x", ctypes.c_void_p),
         ("y", ctypes.c_void_p),
+    ]
+
+
+class ChainOp(ctypes.Structure):
+    _fields_ = [
+        ("kind", ctypes.c_int),
+        ("bits", ctypes.c_int),
+        ("N", ctypes.c_int64),
+        ("K", ctypes.c_int64),
+        ("packed", ctypes.c_void_p),
+        ("inp", ctypes.c_void_p),
+        ("out", ctypes.c_void_p),
+        ("resid", ctypes.c_void_p),
     ]
 
 
@@ -98,6 +115,9 @@ def _load() -> ctypes.CDLL:
         "layer_stack_launches": ([vp], i32),
         "layer_stack_destroy": ([vp], None),
         "q4_quantize": ([i32, i32, vp, i64, i64, vp, vp], i32),
+        "layer_chain_create": ([ctypes.POINTER(ChainOp), i32, i32, i32, ctypes.POINTER(vp)], i32),
+        "q4_residual_rmsnorm": ([vp, vp, vp, vp, i64, i32, i32, vp], i32),
+        "q4_swiglu": ([vp, vp, i64, i32, vp], i32),
         "q4_quantize_device": ([i32, i32, vp, i64, i64, vp, vp, vp], i32),
     }
     for name, (args, res) in sig.items():
@@ -285,6 +305,31 @@ def layer_stack_create(entries, M: int, flags: int = 0) -> LayerStack:
     return LayerStack(h.value, keep)
 
 
+def layer_chain_create(ops, M: int, flags: int = 0) -> LayerStack:
+    """ops: sequence of (kind, bits, N, K, packed, inp, out, resid); device
+    tensors, raw addresses or None (NULL)."""
+    arr = (ChainOp * max(len(ops), 1))()
+    keep = []
+    for i, (kind, bits, N, K, packed, inp, out, resid) in enumerate(ops):
+        ptr = lambda t: 0 if t is None else _dev_ptr(t)  # noqa: E731
+        arr[i] = ChainOp(kind, bits, N, K, ptr(packed), ptr(inp), ptr(out), ptr(resid))
+        keep.append((packed, inp, out, resid))
+    h = ctypes.c_void_p(0)
+    _check(_lib.layer_chain_create(arr, len(ops), M, flags, ctypes.byref(h)))
+    return LayerStack(h.value, keep)
+
+
+def q4_residual_rmsnorm(h, y, gamma, x, N: int, M: int, set_: bool = False, stream=None) -> None:
+    """h (fp32 [M][N]) <- h + y (or y when set_); x (bf16 bits [M][N]) = RMSNorm(h) * gamma."""
+    _check(_lib.q4_residual_rmsnorm(_dev_ptr(h), _dev_ptr(y), _dev_ptr(gamma), _dev_ptr(x), N, M, int(set_),
+                                    _stream(stream)))
+
+
+def q4_swiglu(y_gu, x, N: int, M: int, stream=None) -> None:
+    """x (bf16 bits [M][N]) = silu(gate) * up from y_gu (fp32 [M][2N])."""
+    _check(_lib.q4_swiglu(_dev_ptr(y_gu), _dev_ptr(x), N, M, _stream(stream)))
+
+
 def layer_stack_run(stack: LayerStack, stream=None) -> None:
     _check(_lib.layer_stack_run(stack.handle, _stream(stream)))
 
@@ -304,4 +349,6 @@ __all__ = [
     "q4_workspace_check", "q4_set_wait_timeout_ns", "q4_unpack_device", "q4_selftest_wait_timeout",
     "layer_stack_create", "layer_stack_run", "layer_stack_check", "layer_stack_destroy",
     "q4_quantize", "q4_quantize_device", "Q4_QUANT_ABSMAX", "Q4_QUANT_SIGNED_MAX",
+    "layer_chain_create", "ChainOp", "Q4_OP_PRODUCT", "Q4_OP_RESIDUAL_RMSNORM", "Q4_OP_SWIGLU",
+    "q4_residual_rmsnorm", "q4_swiglu",
 ]

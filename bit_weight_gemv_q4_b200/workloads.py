@@ -176,3 +176,152 @@ class DeviceStream:
         self.packed.clear()
         self.y.clear()
         self.x.clear()
+
+
+# ----------------------------------------------------------------------------
+# The dependent decode chain: the same products, with the steps between them
+# (residual + RMSNorm before q|k|v and gate|up, SwiGLU before down, a final
+# norm before the head).  The attention / DeltaNet mixer is not computed: its
+# output (the o projection's input) is an input of the step.
+# ----------------------------------------------------------------------------
+@dataclass(frozen=True)
+class ChainShape:
+    layers: int = N_LAYERS
+    hidden: int = HIDDEN
+    ffn: int = FFN
+    kv: int = KV
+    vocab: int = VOCAB
+
+
+CHAIN_INPUT_BASE = 1 << 24  # generator streams of the chain's own inputs (beyond every K used as a stream id)
+
+
+def chain_tensors(shape: ChainShape) -> list[Tensor]:
+    """The chain's products in execution order (the default shape gives
+    exactly decode_stream(fused=True))."""
+    out: list[Tensor] = []
+    H, F, KVW = shape.hidden, shape.ffn, shape.kv
+    for layer in range(shape.layers):
+        mb = 8 if is_attention_layer(layer) else 4
+        base = 16 + 16 * layer
+        out += [
+            Tensor(f"L{layer}.qkv", mb, H + 2 * KVW, H, base + 7),
+            Tensor(f"L{layer}.o", mb, H, H, base + 3),
+            Tensor(f"L{layer}.gate_up", 4, 2 * F, H, base + 8),
+            Tensor(f"L{layer}.down", 4, H, F, base + 6),
+        ]
+    out.append(Tensor("head", 8, shape.vocab, H, 1023))
+    return out
+
+
+def chain_input_stream(j: int) -> int:
+    """j = 0: the embedding row(s); 1 + layer: that layer's mixer output."""
+    from . import synth
+
+    return synth.act_stream(CHAIN_INPUT_BASE + j)
+
+
+def chain_gammas(shape: ChainShape, seed: int):
+    """bf16 bits [2 * layers + 1][hidden]: the norm weights, 1 + z / 16."""
+    import numpy as np
+
+    from . import synth
+
+    n = 2 * shape.layers + 1
+    z = synth.normals_f64(seed, chain_input_stream(1 << 20), 0, n * shape.hidden)
+    return synth.f64_to_bf16_bits(1.0 + z / 16.0).reshape(n, shape.hidden)
+
+
+class DeviceChain:
+    """The dependent chain on the current CUDA device: the weights (as in
+    DeviceStream), the residual stream h (fp32), the embedding and mixer
+    inputs (seeded), the norm weights, every intermediate activation and
+    output, and the captured chain (layer_chain_create)."""
+
+    def __init__(self, shape: ChainShape, M: int, seed: int = 0, flags: int = 0):
+        import torch
+
+        import bit_weight_gemv_q4_b200 as q4
+
+        from . import synth
+
+        self.shape, self.M, self.seed = shape, M, seed
+        H, F, L = shape.hidden, shape.ffn, shape.layers
+        self.w = DeviceStream(chain_tensors(shape), M, seed=seed, flags=q4.Q4_STACK_GRAPH)
+        self.w.stack.close()
+        dev = torch.device("cuda")
+
+        def bf16(n):
+            return torch.empty(M * n, dtype=torch.int16, device=dev)
+
+        emb = bf16(H)
+        synth.activations_device(seed, chain_input_stream(0), M, H, emb)
+        self.emb = emb.view(torch.bfloat16).float()  # the residual stream starts from it (fp32)
+        self.h = torch.empty(M * H, dtype=torch.float32, device=dev)
+        self.gamma = torch.from_numpy(chain_gammas(shape, seed).view("int16")).to(dev)
+        self.x_mix = []
+        for layer in range(L):
+            xm = bf16(H)
+            synth.activations_device(seed, chain_input_stream(1 + layer), M, H, xm)
+            self.x_mix.append(xm)
+        self.x_qkv = [bf16(H) for _ in range(L)]
+        self.x_gu = [bf16(H) for _ in range(L)]
+        self.x_down = [bf16(F) for _ in range(L)]
+        self.x_head = bf16(H)
+        self.ops = self.make_ops()
+        torch.cuda.synchronize()
+        self.stack = q4.layer_chain_create(self.ops, M, flags)
+
+    def product_index(self, layer: int, which: str) -> int:
+        return 4 * layer + {"qkv": 0, "o": 1, "gate_up": 2, "down": 3}[which]
+
+    def make_ops(self):
+        import bit_weight_gemv_q4_b200 as q4
+
+        H, F, L = self.shape.hidden, self.shape.ffn, self.shape.layers
+        w = self.w
+        ops = []
+
+        def product(i, x):
+            t = w.tensors[i]
+            ops.append((q4.Q4_OP_PRODUCT, t.bits, t.N, t.K, w.packed[i], x, w.y[i], None))
+
+        def norm(y, g, x, first=False):
+            ops.append((q4.Q4_OP_RESIDUAL_RMSNORM, 1 if first else 0, H, 0, self.gamma[g], y, x, self.h))
+
+        for layer in range(L):
+            prev = self.emb if layer == 0 else w.y[self.product_index(layer - 1, "down")]
+            norm(prev, 2 * layer, self.x_qkv[layer], first=layer == 0)
+            product(self.product_index(layer, "qkv"), self.x_qkv[layer])
+            product(self.product_index(layer, "o"), self.x_mix[layer])
+            norm(w.y[self.product_index(layer, "o")], 2 * layer + 1, self.x_gu[layer])
+            product(self.product_index(layer, "gate_up"), self.x_gu[layer])
+            ops.append((q4.Q4_OP_SWIGLU, 0, F, 0, None, w.y[self.product_index(layer, "gate_up")],
+                        self.x_down[layer], None))
+            product(self.product_index(layer, "down"), self.x_down[layer])
+        last = self.emb if L == 0 else w.y[self.product_index(L - 1, "down")]
+        norm(last, 2 * L, self.x_head, first=L == 0)
+        product(4 * L, self.x_head)
+        return ops
+
+    @property
+    def weight_bytes(self) -> int:
+        return total_bytes(self.w.tensors)
+
+    @property
+    def logits(self):
+        return self.w.y[-1]
+
+    def run(self, stream=None) -> None:
+        import bit_weight_gemv_q4_b200 as q4
+
+        q4.layer_stack_run(self.stack, stream)
+
+    def check(self, stream=None) -> None:
+        import bit_weight_gemv_q4_b200 as q4
+
+        q4.layer_stack_check(self.stack, stream)
+
+    def close(self) -> None:
+        self.stack.close()
+        self.w.close()

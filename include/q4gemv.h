@@ -297,6 +297,57 @@ Q4_API int layer_stack_check(q4_stack* stack, void* stream);
 /* Number of kernel launches one layer_stack_run makes. */
 Q4_API int layer_stack_launches(const q4_stack* stack);
 
+/* ---------------------------------------------------------------------------
+ * A dependent decode chain: products whose activations come from the outputs
+ * of earlier products through the steps that sit between them in a decoder
+ * layer, all captured once as a CUDA graph with programmatic dependent launch
+ * (each kernel starts its prologue -- a product its first weight copies --
+ * while the one before it finishes, and reads its input only after that one
+ * has completed).  The pages name the layer structure (64 layers: 16 gated
+ * attention, 48 Gated DeltaNet: wiselychen guide, section "Before deploying")
+ * but not the steps; the plain textbook forms are used:
+ *   Q4_OP_RESIDUAL_RMSNORM: h <- h + in (in may be NULL: h unchanged), or,
+ *       with bits = 1, h <- in (the residual stream starts from `in`);
+ *       out = bf16( h / sqrt(mean_k h_k^2 + 1e-6) * gamma )  per row, gamma
+ *       bf16 [N] or NULL for 1; h fp32 [M][N] in `resid`, updated in place
+ *   Q4_OP_SWIGLU: out = bf16( silu(g) * u ), silu(z) = z / (1 + e^-z), with
+ *       in = fp32 [M][2N] holding g = in[:, :N] and u = in[:, N:]
+ *   Q4_OP_PRODUCT: out (fp32 [M][N]) = W in, W packed (bits 4 or 8, N x K),
+ *       in bf16 [M][K] -- q4_gemv / q8_gemv
+ * bf16 rounding is to nearest, ties to even.  The attention / DeltaNet mixer
+ * is not part of the chain: its output enters as an input buffer.
+ * -------------------------------------------------------------------------*/
+#define Q4_OP_PRODUCT 0
+#define Q4_OP_RESIDUAL_RMSNORM 1
+#define Q4_OP_SWIGLU 2
+
+typedef struct q4_chain_op {
+  int kind;            /* Q4_OP_* */
+  int bits;            /* product: 4 or 8; else ignored */
+  int64_t N, K;        /* product: weight shape; RMSNORM: row length; SWIGLU: output row length */
+  const void* packed;  /* product: packed weights (16-byte aligned); RMSNORM: gamma (bf16 [N]) or NULL */
+  const void* in;      /* see above (device) */
+  void* out;           /* see above (device) */
+  float* resid;        /* RMSNORM: residual stream h (fp32 [M][N], device); else NULL */
+} q4_chain_op;
+
+/* Validates the ops and captures them, in order, on the current device.
+ * flags: Q4_STACK_NO_PDL launches without programmatic dependent launch.
+ * The returned stack runs with layer_stack_run, is checked with
+ * layer_stack_check and freed with layer_stack_destroy.  Errors: as
+ * layer_stack_create (INVALID_ARG for an unknown kind, a null or misaligned
+ * buffer: fp32 4-byte, bf16 2-byte). */
+Q4_API int layer_chain_create(const q4_chain_op* ops, int n_ops, int M, int flags, q4_stack** out);
+
+/* The chain's two steps as single asynchronous calls on `stream` (the same
+ * kernels the chain captures).  q4_residual_rmsnorm: h (fp32 [M][N]) <- h + y
+ * (y may be NULL) or, when set != 0, h <- y; x (bf16 [M][N]) = the
+ * normalised h times gamma (bf16 [N], or NULL for 1).  q4_swiglu: x (bf16
+ * [M][N]) from y_gu (fp32 [M][2N]).  M in 1..4; errors as layer_chain_create. */
+Q4_API int q4_residual_rmsnorm(float* h, const float* y, const uint16_t* gamma, uint16_t* x, int64_t N, int M,
+                               int set, void* stream);
+Q4_API int q4_swiglu(const float* y_gu, uint16_t* x, int64_t N, int M, void* stream);
+
 /* Frees the graph and the workspace.  NULL is ignored. */
 Q4_API void layer_stack_destroy(q4_stack* stack);
 

@@ -33,7 +33,7 @@ def test_every_declared_symbol_is_exported():
 def test_only_declared_symbols_are_exported():
     out = subprocess.run(["nm", "-D", "--defined-only", build.GEMV_LIB], stdout=subprocess.PIPE, text=True, check=True)
     ours = {line.split()[-1] for line in out.stdout.splitlines() if " T " in line}
-    assert {s for s in ours if s.startswith(("q4_", "q8_", "layer_stack_"))} == set(declared_symbols())
+    assert {s for s in ours if s.startswith(("q4_", "q8_", "layer_stack_", "layer_chain_"))} == set(declared_symbols())
 
 
 # Host-side validation happens before any CUDA call, so these run without a GPU.

@@ -1,0 +1,267 @@
+"""The dependent decode chain: the oracle's steps pinned by closed forms and
+identities (CPU); each step kernel against the oracle, the captured chain
+against the same steps called one by one, and a short chain against the
+oracle's own chain (GPU)."""
+import numpy as np
+import pytest
+
+from oracle import chain as OC
+import oracle
+from bit_weight_gemv_q4_b200 import synth, workloads
+
+SMALL = workloads.ChainShape(layers=2, hidden=1024, ffn=2048, kv=256, vocab=4096)
+
+
+# ---------------------------------------------------------------- oracle pins
+def test_bf16_rounding_hand_values():
+    vals = np.array([1.0, 1 + 2.0 ** -8, 1 + 3 * 2.0 ** -8, -2.5, 2.0 ** -130, 0.0, 1 + 2.0 ** -8 + 2.0 ** -30])
+    # ties go to the even mantissa: 1 + 2^-8 -> 1.0, 1 + 3*2^-8 -> 1 + 2^-6; the subnormal 2^-130 is 8 * 2^-133;
+    # just above the tie rounds up
+    assert OC.bf16_exact(vals).tolist() == [0x3F80, 0x3F80, 0x3F82, 0xC020, 0x0008, 0x0000, 0x3F81]
+    # the two-step conversion (fp64 -> fp32 -> bf16) differs from the one-step
+    # rounding only where the fp32 value lands exactly on a bf16 tie
+    z = np.random.default_rng(1).normal(0, 3, 20000)
+    d = OC.bf16_exact(z) != OC.bf16_bits(z)
+    f32 = z.astype(np.float32).view(np.uint32)
+    assert np.all((f32[d] & 0xFFFF) == 0x8000)
+
+
+def test_silu_identities():
+    z = np.linspace(-30, 30, 601)
+    assert np.allclose(OC.silu(z) - OC.silu(-z), z, rtol=0, atol=1e-12)  # silu(z) - silu(-z) = z
+    assert OC.silu(np.array([0.0]))[0] == 0.0
+    assert abs(OC.silu(np.array([40.0]))[0] - 40.0) < 1e-12
+    assert abs(OC.silu(np.array([1.0]))[0] - 1.0 / (1.0 + np.exp(-1.0))) < 1e-16
+
+
+def test_rmsnorm_closed_forms():
+    c = np.full((1, 512), 3.0)
+    h, z = OC.residual_rmsnorm(None, c, None)
+    assert np.array_equal(h, c)
+    assert np.allclose(z, 3.0 / np.sqrt(9.0 + OC.EPS), rtol=0, atol=1e-15)
+    rng = np.random.default_rng(2)
+    h0, y = rng.normal(0, 2, (3, 256)), rng.normal(0, 2, (3, 256))
+    g = 1 + rng.normal(0, 0.1, 256)
+    h1, z = OC.residual_rmsnorm(h0, y, g)
+    assert np.allclose(h1, h0 + y, rtol=0, atol=1e-15)
+    zn = z / g  # mean square of the normalised rows is ms / (ms + eps)
+    ms = np.mean(h1 * h1, axis=1)
+    assert np.allclose(np.mean(zn * zn, axis=1), ms / (ms + OC.EPS), rtol=1e-12)
+    # invariant under scaling when eps is negligible against the mean square
+    _, z2 = OC.residual_rmsnorm(None, (h0 + y) * 1e3, g)
+    assert np.allclose(z, z2, rtol=1e-6)
+
+
+def test_swiglu_closed_forms():
+    y = np.zeros((2, 8))
+    y[0, :4] = [0.0, 1.0, -1.0, 40.0]
+    y[0, 4:] = [5.0, 0.0, 2.0, 0.5]
+    z = OC.swiglu(y, 4)
+    assert z[0, 0] == 0.0 and z[0, 1] == 0.0
+    assert np.isclose(z[0, 2], -1.0 / (1.0 + np.e) * 2.0)
+    assert np.isclose(z[0, 3], 40.0 * 0.5)
+    assert not z[1].any()
+
+
+def test_near_tie_window():
+    t = np.array([1 + 2.0 ** -8, 1.0, 1 + 2.0 ** -8 + 2.0 ** -20])
+    assert OC.near_bf16_tie(t, 0.0).tolist() == [True, False, False]
+    assert OC.near_bf16_tie(t, 2.0 ** -18).tolist() == [True, False, True]
+
+
+def test_chain_shape_of_the_decode_stream():
+    assert workloads.chain_tensors(workloads.ChainShape()) == workloads.decode_stream(fused=True)
+
+
+# ---------------------------------------------------------------- oracle chain
+def oracle_chain(shape, M, seed):
+    """Every intermediate of the chain from the oracle alone (inputs from the
+    seeded generator): dict with x (bf16 bits), z (pre-rounding), y, B."""
+    H, F, L = shape.hidden, shape.ffn, shape.layers
+    tensors = workloads.chain_tensors(shape)
+    gam = OC.bf16_value(workloads.chain_gammas(shape, seed))
+    emb = OC.bf16_value(synth.activations(seed, workloads.chain_input_stream(0), M, H))
+    out = {"x": {}, "z": {}, "y": {}, "B": {}}
+
+    def prod(i, xbits):
+        t = tensors[i]
+        q, s = synth.tensor(t.bits, seed, t.tensor_id, t.N, t.K)
+        y, B = OC.product(t.bits, q, s, xbits)
+        out["y"][i], out["B"][i] = y, B
+        return y
+
+    h = None
+    y_prev = emb
+    for layer in range(L):
+        h, z = OC.residual_rmsnorm(h, y_prev, gam[2 * layer])
+        x = OC.bf16_exact(z)
+        out["z"][("qkv", layer)], out["x"][("qkv", layer)] = z, x
+        prod(4 * layer, x)
+        xm = synth.activations(seed, workloads.chain_input_stream(1 + layer), M, H)
+        y_o = prod(4 * layer + 1, xm)
+        h, z = OC.residual_rmsnorm(h, y_o, gam[2 * layer + 1])
+        x = OC.bf16_exact(z)
+        out["z"][("gu", layer)], out["x"][("gu", layer)] = z, x
+        y_gu = prod(4 * layer + 2, x)
+        z = OC.swiglu(y_gu, F)
+        x = OC.bf16_exact(z)
+        out["z"][("down", layer)], out["x"][("down", layer)] = z, x
+        y_prev = prod(4 * layer + 3, x)
+    h, z = OC.residual_rmsnorm(h, y_prev, gam[2 * L])
+    x = OC.bf16_exact(z)
+    out["z"][("head", L)], out["x"][("head", L)] = z, x
+    prod(4 * L, x)
+    out["h"] = h
+    return out
+
+
+# ---------------------------------------------------------------- GPU
+def _torch():
+    import torch
+
+    return torch
+
+
+def _f32(host):
+    return _torch().from_numpy(np.ascontiguousarray(host, dtype=np.float32)).cuda()
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("M", [1, 4])
+@pytest.mark.parametrize("set_", [False, True])
+def test_rmsnorm_kernel_matches_the_oracle(cuda_device, M, set_):
+    """bf16 outputs equal the oracle's except within 2^-17 (relative) of a
+    rounding tie, where the fp32 computation may round either way; h is the
+    fp32 sum."""
+    import bit_weight_gemv_q4_b200 as q4
+
+    torch = _torch()
+    N = 5120
+    h0 = synth.normals_f64(3, 900, 0, M * N).astype(np.float32).reshape(M, N) * 4
+    y = synth.normals_f64(3, 901, 0, M * N).astype(np.float32).reshape(M, N) * 7
+    g = synth.f64_to_bf16_bits(1 + synth.normals_f64(3, 902, 0, N) / 16)
+    hd, yd = _f32(h0), _f32(y)
+    gd = torch.from_numpy(g.view(np.int16)).cuda()
+    xd = torch.empty(M * N, dtype=torch.int16, device="cuda")
+    q4.q4_residual_rmsnorm(hd, yd, gd, xd, N, M, set_)
+    torch.cuda.synchronize()
+    h_ref, z = OC.residual_rmsnorm(None if set_ else h0.astype(np.float64), y.astype(np.float64), OC.bf16_value(g))
+    assert np.array_equal(hd.cpu().numpy().reshape(M, N), (y if set_ else h0 + y).astype(np.float32))
+    x = xd.cpu().numpy().view(np.uint16).reshape(M, N)
+    diff = x != OC.bf16_exact(z)
+    assert not (diff & ~OC.near_bf16_tie(z, 2.0 ** -17)).any()
+    assert diff.mean() < 1e-3
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("M", [1, 3])
+def test_swiglu_kernel_matches_the_oracle(cuda_device, M):
+    import bit_weight_gemv_q4_b200 as q4
+
+    torch = _torch()
+    N = 17408
+    y = (synth.normals_f64(4, 903, 0, M * 2 * N) * 6).astype(np.float32).reshape(M, 2 * N)
+    xd = torch.empty(M * N, dtype=torch.int16, device="cuda")
+    q4.q4_swiglu(_f32(y), xd, N, M)
+    torch.cuda.synchronize()
+    z = OC.swiglu(y.astype(np.float64), N)
+    x = xd.cpu().numpy().view(np.uint16).reshape(M, N)
+    diff = x != OC.bf16_exact(z)
+    assert not (diff & ~OC.near_bf16_tie(z, 2.0 ** -19)).any()
+    assert diff.mean() < 1e-3
+
+
+def _outputs(ch):
+    torch = _torch()
+    torch.cuda.synchronize()
+    got = {"y": [y.cpu().numpy().copy() for y in ch.w.y]}
+    got["x"] = [t.cpu().numpy().copy() for t in ch.x_qkv + ch.x_gu + ch.x_down + [ch.x_head]]
+    got["h"] = ch.h.cpu().numpy().copy()
+    return got
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("M", [1, 4])
+def test_chain_equals_its_steps_called_one_by_one(cuda_device, M):
+    """The captured chain (with and without programmatic dependent launch) is
+    bitwise the sequence of single calls on the same buffers."""
+    import bit_weight_gemv_q4_b200 as q4
+
+    torch = _torch()
+    ch = workloads.DeviceChain(SMALL, M, seed=5)
+    ch.run()
+    ch.check()
+    graph = _outputs(ch)
+    ch.run()
+    again = _outputs(ch)
+    assert all(np.array_equal(a, b) for a, b in zip(graph["y"] + graph["x"], again["y"] + again["x"]))
+    nopdl = q4.layer_chain_create(ch.ops, M, q4.Q4_STACK_NO_PDL)
+    q4.layer_stack_run(nopdl)
+    q4.layer_stack_check(nopdl)
+    third = _outputs(ch)
+    assert all(np.array_equal(a, b) for a, b in zip(graph["y"] + graph["x"], third["y"] + third["x"]))
+    nopdl.close()
+    # the same ops, one call each
+    for y in ch.w.y:
+        y.fill_(float("nan"))
+    ws = torch.zeros(max(q4.q4_gemv_workspace_bytes(t.bits, t.N, t.K, M) for t in ch.w.tensors), dtype=torch.uint8,
+                     device="cuda")
+    for kind, bits, N, K, packed, inp, out, resid in ch.ops:
+        if kind == q4.Q4_OP_PRODUCT:
+            (q4.q4_gemv if bits == 4 else q4.q8_gemv)(packed, N, K, inp, M, out, ws)
+        elif kind == q4.Q4_OP_RESIDUAL_RMSNORM:
+            q4.q4_residual_rmsnorm(resid, inp, packed, out, N, M, bits == 1)
+        else:
+            q4.q4_swiglu(inp, out, N, M)
+    q4.q4_workspace_check(ws)
+    single = _outputs(ch)
+    assert all(np.array_equal(a, b) for a, b in zip(graph["y"] + graph["x"], single["y"] + single["x"]))
+    assert np.array_equal(graph["h"], single["h"])
+    ch.close()
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("M", [1, 2])
+def test_chain_against_the_oracle_chain(cuda_device, M):
+    """A two-layer chain against the oracle's chain computed alone: the first
+    activations equal the oracle's away from rounding ties, the first product
+    is within the product tolerance, and the end (after nine dependent steps)
+    stays within 1e-3 in relative norm."""
+    ch = workloads.DeviceChain(SMALL, M, seed=6)
+    ch.run()
+    ch.check()
+    got = _outputs(ch)
+    ref = oracle_chain(SMALL, M, 6)
+    x0 = got["x"][0].view(np.uint16).reshape(M, SMALL.hidden)
+    z0 = ref["z"][("qkv", 0)]
+    diff = x0 != ref["x"][("qkv", 0)]
+    assert not (diff & ~OC.near_bf16_tie(z0, 2.0 ** -17)).any()
+    t0 = workloads.chain_tensors(SMALL)[0]
+    y0 = got["y"][0].reshape(M, t0.N).astype(np.float64)
+    if not diff.any():
+        ok, _, _ = oracle.within_tolerance(y0, ref["y"][0], ref["B"][0])
+        assert ok.all()
+    for i in range(len(got["y"])):
+        t = workloads.chain_tensors(SMALL)[i]
+        y = got["y"][i].reshape(M, t.N).astype(np.float64)
+        r = ref["y"][i]
+        assert np.all(np.isfinite(y))
+        assert np.linalg.norm(y - r) <= 1e-3 * np.linalg.norm(r) + 1e-6, t.name
+    ch.close()
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("M", [1, 4])
+def test_full_chain_runs_and_is_reproducible(cuda_device, M):
+    torch = _torch()
+    ch = workloads.DeviceChain(workloads.ChainShape(), M)
+    assert ch.stack.launches() == 64 * 7 + 2
+    ch.run()
+    ch.check()
+    a = ch.logits.cpu().numpy().copy()
+    ch.run()
+    ch.check()
+    b = ch.logits.cpu().numpy().copy()
+    assert np.all(np.isfinite(a)) and np.array_equal(a, b)
+    ch.close()
+    torch.cuda.empty_cache()

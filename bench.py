@@ -11,7 +11,9 @@ at M = 1, with % of the measured HBM peak and the implied decode tok/s; the
 same at M = 4 (one verification pass of 3 drafted tokens + 1) in "m4".  The
 line also reports the ordered and graph stack modes, the end-to-end step
 through the public API ("e2e"), the roofline of the dominant kernel, the CPU
-oracle's rate ("cpu_baseline"), the SM clock under load, and "per_config":
+oracle's rate ("cpu_baseline"), the SM clock under load, "chain" (the same
+products as a dependent chain with the residual + RMSNorm and SwiGLU steps
+between them, M = 1 and 4), and "per_config":
 microseconds per product of the single-tensor configurations (q4 4096 x 4096,
 each projection of one layer at M = 1 and 4, the q8 vocabulary heads).
 
@@ -432,6 +434,23 @@ def run_ours(args, d: Dist):
     del st4
     torch.cuda.empty_cache()
 
+    # the dependent chain: the same products with the steps between them
+    # (residual + RMSNorm, SwiGLU), one CUDA graph with programmatic dependent launch
+    chain = {}
+    for M in (1, 4):
+        ch = workloads.DeviceChain(workloads.ChainShape(), M, seed=args.seed)
+        for _ in range(3):
+            ch.run()
+        n_ch = max(3, args.steps // 4)
+        ms_ch = d.max(time_region(torch, ch.run, n_ch, stream) / n_ch)
+        ch.check()
+        chain[f"M{M}"] = {"value": round(wbytes * d.world / (ms_ch * 1e6), 1), "unit": UNIT,
+                          "ms_per_step": round(ms_ch, 5), "pct_of_hbm_peak": round(100 * wbytes / (ms_ch * 1e6) / peak, 2),
+                          "tok_per_s": round(1000.0 / ms_ch, 1), "launches": ch.stack.launches()}
+        ch.close()
+        del ch
+        torch.cuda.empty_cache()
+
     configs = None if args.no_configs else per_config(args, d, torch, q4, workloads, peak)
 
     cpu = None
@@ -498,6 +517,7 @@ def run_ours(args, d: Dist):
             "h2d_bytes_per_step": h2d,
             "d2h_bytes_per_step": d2h,
         },
+        "chain": chain,
         "per_config": configs,
         "gpu_launches": n_launch * args.steps,
         "clocks": clocks,

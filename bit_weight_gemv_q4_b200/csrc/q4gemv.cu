@@ -652,7 +652,10 @@ int create_persistent(const q4_stack_entry* entries, int n, int M, int su, const
       job_of[static_cast<size_t>(i)] = jdx;
     }
   }
-  const size_t prep_base = kWsHeader + partials_bytes(dev) + counters;
+  // ordered mode: one barrier flag per CTA
+  const size_t flags_bytes = independent ? 0 : (static_cast<size_t>(dev.sms) * 4 + 255) / 256 * 256;
+  const size_t flags_base = kWsHeader + partials_bytes(dev) + counters;
+  const size_t prep_base = flags_base + flags_bytes;
   st->workspace_bytes = prep_base + prep_bytes;
   cudaError_t err = cudaMalloc(&st->workspace, st->workspace_bytes);
   if (err == cudaSuccess) err = cudaMemset(st->workspace, 0, st->workspace_bytes);
@@ -696,7 +699,7 @@ int create_persistent(const q4_stack_entry* entries, int n, int M, int su, const
   p.entries = st->entries_dev;
   p.E = n;
   p.status = reinterpret_cast<unsigned*>(ws);
-  p.grid_bar = reinterpret_cast<unsigned*>(ws + 16);
+  p.bar_flags = reinterpret_cast<unsigned*>(ws + flags_base);
   p.partials = reinterpret_cast<float*>(ws + kWsHeader);
   p.counters = reinterpret_cast<unsigned*>(ws + kWsHeader + partials_bytes(dev));
   p.G = st->grid;

@@ -68,7 +68,7 @@ struct StackParams {
   float* partials;      // [P][2][M][32]
   unsigned* counters;   // one per tile of the largest product (re-zeroed as used)
   unsigned* status;
-  unsigned* grid_bar;   // [0] arrivals, [1] generation
+  unsigned* bar_flags;  // ordered mode: [G] per-CTA barrier epochs
   int G;                // CTAs in the grid (all resident: cooperative launch)
   unsigned long long timeout_ns;
   long long TBg;        // stream mode: blocks of all products, concatenated
@@ -100,32 +100,40 @@ struct StageCursor {
   __device__ __forceinline__ bool next(const StackParams& sp, int pw, const uint8_t** out_src, uint32_t* out_bytes);
 };
 
+__device__ __forceinline__ void st_release_gpu(unsigned* p, unsigned v) {
+  asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
 // Grid-wide barrier of the G resident CTAs; all threads of the CTA call it.
-// Returns false when this CTA is aborting (its own abort flag, or a wait that
-// gave up).
-__device__ __forceinline__ bool grid_barrier(const StackParams& sp, int* s_abort) {
+// CTA b announces its arrival at barrier `epoch` by storing the epoch
+// (release) in its own flag, and passes once every CTA's flag has reached it
+// (acquire loads, one warp polling all G flags): no atomic, no contention on
+// one address.  Epochs only grow: each run continues from the last epoch its
+// CTA stored.  Returns false when this CTA is aborting (its own abort flag,
+// or a wait that gave up).
+__device__ __forceinline__ bool grid_barrier(const StackParams& sp, unsigned epoch, int* s_abort) {
   __syncthreads();
-  if (threadIdx.x == 0 && !*s_abort) {
-    unsigned* count = sp.grid_bar;
-    unsigned* gen = sp.grid_bar + 1;
-    const unsigned my_gen = ld_acquire_gpu(gen);
-    __threadfence();  // this CTA's outputs before its arrival
-    const unsigned arrived = atomicAdd(count, 1u);
-    if (arrived == static_cast<unsigned>(sp.G) - 1u) {
-      atomicExch(count, 0u);
-      __threadfence();
-      atomicAdd(gen, 1u);  // releases the waiting CTAs
-    } else {
-      const unsigned long long t0 = global_timer_ns();
-      while (ld_acquire_gpu(gen) == my_gen) {
-        if (global_timer_ns() - t0 > sp.timeout_ns) {
+  if (threadIdx.x < 32 && !*s_abort) {
+    const int lane = threadIdx.x;
+    if (lane == 0) {
+      __threadfence();  // this CTA's outputs before its arrival
+      st_release_gpu(sp.bar_flags + blockIdx.x, epoch);
+    }
+    __syncwarp();
+    const unsigned long long t0 = global_timer_ns();
+    while (true) {
+      bool here = true;
+      for (int i = lane; i < sp.G; i += 32) here &= static_cast<int>(ld_acquire_gpu(sp.bar_flags + i) - epoch) >= 0;
+      if (__all_sync(0xFFFFFFFFu, here)) break;
+      const unsigned long long waited = __shfl_sync(0xFFFFFFFFu, global_timer_ns() - t0, 0);
+      if (waited > sp.timeout_ns) {
+        if (lane == 0) {
           *s_abort = 1;
           atomicOr(sp.status, kStatusTimeout);
-          break;
         }
+        break;
       }
     }
-    __threadfence();
   }
   __syncthreads();
   return !*s_abort;
@@ -161,6 +169,7 @@ __global__ void __launch_bounds__(NW * 32, 1) stack_kernel(const StackParams sp)
   constexpr int SLOT = kStackSlotBytes;
   extern __shared__ __align__(128) unsigned char smem[];
   __shared__ int s_abort;
+  __shared__ unsigned s_epoch0;
 
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
@@ -169,12 +178,16 @@ __global__ void __launch_bounds__(NW * 32, 1) stack_kernel(const StackParams sp)
   const uint32_t ring = smem_addr(smem + warp * D * SLOT);
   const uint32_t bars = smem_addr(smem + NW * D * SLOT) + warp * D * 8;
 
-  if (threadIdx.x == 0) s_abort = 0;
+  if (threadIdx.x == 0) {
+    s_abort = 0;
+    s_epoch0 = ld_acquire_gpu(sp.bar_flags + blockIdx.x);  // the last barrier of the previous run
+  }
   if (lane == 0) {
     for (int s = 0; s < D; ++s) mbar_init(bars + 8 * s, 1);
     fence_barrier_init();
   }
   __syncthreads();
+  const unsigned epoch0 = s_epoch0;
   const uint64_t policy = l2_evict_first_policy();
 
   // ---- producer: the warp's stages of all products, in order; `ahead` runs
@@ -307,7 +320,7 @@ __global__ void __launch_bounds__(NW * 32, 1) stack_kernel(const StackParams sp)
     }
     // every output of this product is written before the next reads its input
     if (ei + 1 < sp.E) {
-      if (!grid_barrier(sp, &s_abort)) break;
+      if (!grid_barrier(sp, epoch0 + static_cast<unsigned>(ei) + 1u, &s_abort)) break;
     }
   }
   if (s_abort) {

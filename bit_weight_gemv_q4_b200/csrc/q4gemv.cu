@@ -47,7 +47,7 @@ std::atomic<unsigned long long> g_timeout_ns{kDefaultTimeoutNs};
 #ifndef Q4_TUNE_MAX_U
 #define Q4_TUNE_MAX_U 2
 #endif
-constexpr int kNW = Q4_TUNE_NW;
+constexpr int kNW = Q4_TUNE_NW;  // warps per CTA of the single-product kernel
 constexpr int kCtasPerSm = Q4_TUNE_CTAS_PER_SM;
 constexpr int kRingChunks = Q4_TUNE_RING_CHUNKS;
 constexpr int kMaxU = Q4_TUNE_MAX_U;
@@ -58,12 +58,16 @@ static_assert(kRingChunks % 2 == 0 && kRingChunks >= 4, "ring must hold two stag
 #ifndef Q4_TUNE_STACK_PF
 #define Q4_TUNE_STACK_PF 0
 #endif
+#ifndef Q4_TUNE_STACK_NW
+#define Q4_TUNE_STACK_NW 16
+#endif
 #ifndef Q4_TUNE_STREAM_U
 #define Q4_TUNE_STREAM_U 4
 #endif
 constexpr int kStackD = Q4_TUNE_STACK_D;    // stages per warp in the persistent stack kernels
 constexpr int kStackPF = Q4_TUNE_STACK_PF;  // further stages prefetched into L2 (ordered mode)
 constexpr int kStreamU = Q4_TUNE_STREAM_U;  // chunks per stage in stream mode, when the shapes allow
+constexpr int kStackNW = Q4_TUNE_STACK_NW;  // warps per CTA of the persistent kernels (one CTA per SM)
 // shared memory a CTA may use (B200: 227 KB per CTA)
 constexpr int kSmemLimit = 227 * 1024 / kCtasPerSm;
 constexpr size_t kWsHeader = 256;
@@ -150,8 +154,11 @@ long long max_warps(const DeviceInfo& dev) { return static_cast<long long>(dev.s
 // partial-sum region has one fixed size per device (M = 4 worst case), so the
 // counters sit at the same offset for every shape and M: one zero-filled
 // workspace serves any sequence of products, each leaving its counters zero.
+// partial sums of split tiles: two slots of up to 4 x 32 floats per warp, for
+// the most warps any kernel runs (single-product or persistent)
 size_t partials_bytes(const DeviceInfo& dev) {
-  return static_cast<size_t>(max_warps(dev)) * 2 * 4 * q4k::kTileRows * sizeof(float);
+  const long long warps = std::max(max_warps(dev), static_cast<long long>(dev.sms) * kStackNW);
+  return static_cast<size_t>(warps) * 2 * 4 * q4k::kTileRows * sizeof(float);
 }
 
 size_t workspace_bytes(const Shape& s, int M, const DeviceInfo& dev) {
@@ -538,12 +545,12 @@ namespace {
 
 template <int M>
 void* stack_kernel_ptr() {
-  return reinterpret_cast<void*>(&q4k::stack_kernel<M, kNW, kStackD, kStackPF>);
+  return reinterpret_cast<void*>(&q4k::stack_kernel<M, kStackNW, kStackD, kStackPF>);
 }
 
 template <int M, int SU>
 void* stream_kernel_ptr() {
-  return reinterpret_cast<void*>(&q4k::stream_kernel<M, kNW, kStackD, SU>);
+  return reinterpret_cast<void*>(&q4k::stream_kernel<M, kStackNW, kStackD, SU>);
 }
 
 // su: chunks per stage of the stream-mode kernel (0 = ordered mode)
@@ -561,7 +568,7 @@ void* select_stack_kernel(int M, int su) {
 int stack_smem_bytes(int su, int M) {
   const int slot = su == 0 ? q4k::kStackU * q4k::Format<4>::kChunkBytes
                            : su * (q4k::Format<4>::kChunkBytes + M * q4k::Format<4>::kKPerChunk * 2);
-  return kNW * kStackD * slot + kNW * kStackD * 8;
+  return kStackNW * kStackD * slot + kStackNW * kStackD * 8;
 }
 
 void free_stack(q4_stack* st) {
@@ -592,7 +599,7 @@ int create_persistent(const q4_stack_entry* entries, int n, int M, int su, const
   const long long blk = independent ? su : q4k::kStackU;  // chunks per stream-K block
   long long max_t = 1, total_blocks = 0, total_tiles = 0;
   std::vector<q4k::StackEntryDev> host(static_cast<size_t>(n));
-  const long long warps = static_cast<long long>(dev.sms) * kNW;
+  const long long warps = static_cast<long long>(dev.sms) * kStackNW;
   for (int i = 0; i < n; ++i) {
     const q4_stack_entry& en = entries[i];
     char who[64];
@@ -686,7 +693,7 @@ int create_persistent(const q4_stack_entry* entries, int n, int M, int su, const
   if (err != cudaSuccess) return cuda_fail(err, "layer_stack_create: allocation");
   st->fn = select_stack_kernel(M, su);
   st->smem = stack_smem_bytes(su, M);
-  st->block = kNW * 32;
+  st->block = kStackNW * 32;
   st->grid = dev.sms;
   err = cudaFuncSetAttribute(st->fn, cudaFuncAttributeMaxDynamicSharedMemorySize, st->smem);
   if (err != cudaSuccess) return cuda_fail(err, "layer_stack_create: cudaFuncSetAttribute");

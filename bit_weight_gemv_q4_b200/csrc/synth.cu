@@ -33,6 +33,12 @@ __global__ void scales_kernel(uint64_t key, int64_t G, int64_t row0, int64_t nro
     out[i] = synth_scale_value(key, G, row0 + i / G, i % G, std);
 }
 
+__global__ void e4m3_scales_kernel(uint64_t key, int64_t B, int64_t row0, int64_t nrows, uint8_t* out) {
+  const int64_t total = nrows * B;
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < total; i += (int64_t)gridDim.x * blockDim.x)
+    out[i] = synth_e4m3_scale(key, B, row0 + i / B, i % B);
+}
+
 __global__ void bf16_normals_kernel(uint64_t key, int64_t i0, int64_t count, uint16_t* out) {
   for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < count; i += (int64_t)gridDim.x * blockDim.x)
     out[i] = synth_f64_to_bf16(synth_normal(key, (uint64_t)(i0 + i)));
@@ -77,6 +83,17 @@ SYNTH_API int synth_scales(uint64_t seed, uint64_t stream, int64_t K, int64_t ro
 #pragma omp parallel for schedule(static)
   for (int64_t r = 0; r < nrows; ++r)
     for (int64_t g = 0; g < G; ++g) out[r * G + g] = synth_scale_value(key, G, row0 + r, g, std);
+  return 0;
+}
+
+// NVFP4 block scales (E4M3 bytes) [nrows][K/16]; K a multiple of 16.
+SYNTH_API int synth_e4m3_scales(uint64_t seed, uint64_t stream, int64_t K, int64_t row0, int64_t nrows, uint8_t* out) {
+  if (K < 0 || K % 16 || row0 < 0 || nrows < 0 || (!out && nrows > 0)) return -1;
+  const uint64_t key = synth_key(seed, stream);
+  const int64_t B = K / 16;
+#pragma omp parallel for schedule(static)
+  for (int64_t r = 0; r < nrows; ++r)
+    for (int64_t b = 0; b < B; ++b) out[r * B + b] = synth_e4m3_scale(key, B, row0 + r, b);
   return 0;
 }
 
@@ -143,6 +160,15 @@ SYNTH_API int synth_scales_device(uint64_t seed, uint64_t stream_id, int64_t K, 
   if (nrows == 0) return 0;
   scales_kernel<<<grid_for(nrows * (K / 32)), 256, 0, (cudaStream_t)stream>>>(synth_key(seed, stream_id), K / 32,
                                                                                  row0, nrows, std, out);
+  return launched();
+}
+
+SYNTH_API int synth_e4m3_scales_device(uint64_t seed, uint64_t stream_id, int64_t K, int64_t row0, int64_t nrows,
+                                       uint8_t* out, void* stream) {
+  if (K < 0 || K % 16 || row0 < 0 || nrows < 0 || (!out && nrows > 0)) return -1;
+  if (nrows == 0 || K == 0) return 0;
+  e4m3_scales_kernel<<<grid_for(nrows * (K / 16)), 256, 0, (cudaStream_t)stream>>>(synth_key(seed, stream_id), K / 16,
+                                                                                     row0, nrows, out);
   return launched();
 }
 

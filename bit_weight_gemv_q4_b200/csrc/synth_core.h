@@ -242,4 +242,11 @@ SYNTH_HD uint16_t synth_scale_value(uint64_t key, int64_t G, int64_t row, int64_
   return synth_f64_to_f16(v < 0 ? -v : v);
 }
 
+/* NVFP4 block scale (E4M3 bits) of block b of a row: finite, positive, from
+   0x28 (0.25) to 0x47 (3.75), uniform over the 32 byte values. */
+SYNTH_HD uint8_t synth_e4m3_scale(uint64_t key, int64_t B, int64_t row, int64_t b) {
+  const uint64_t w = synth_word(key, (uint64_t)row * (uint64_t)B + (uint64_t)b);
+  return (uint8_t)(0x28 + (w >> 59));
+}
+
 #endif /* Q4_SYNTH_CORE_H */

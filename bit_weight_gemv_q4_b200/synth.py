@@ -48,6 +48,8 @@ def lib() -> ctypes.CDLL:
         L.synth_q8_device.argtypes = [u64, u64, i64, i64, i64, vp, vp]
         L.synth_scales_device.argtypes = [u64, u64, i64, i64, i64, ctypes.c_double, vp, vp]
         L.synth_bf16_normals_device.argtypes = [u64, u64, i64, i64, vp, vp]
+        L.synth_e4m3_scales.argtypes = [u64, u64, i64, i64, i64, vp]
+        L.synth_e4m3_scales_device.argtypes = [u64, u64, i64, i64, i64, vp, vp]
         for f in (L.synth_q4, L.synth_q8, L.synth_scales, L.synth_bf16_normals, L.synth_normals_f64,
                   L.synth_q4_device, L.synth_q8_device, L.synth_scales_device, L.synth_bf16_normals_device):
             f.restype = ctypes.c_int
@@ -153,6 +155,29 @@ def act_stream(k_id: int) -> int:
     return ACT_STREAM_BASE + k_id
 
 
+def e4m3_scales(seed: int, stream: int, K: int, row0: int, nrows: int) -> np.ndarray:
+    """E4M3 bytes of NVFP4 block scales (0.25 .. 3.75), shape [nrows][K/16]."""
+    out = np.empty((nrows, K // 16), dtype=np.uint8)
+    if lib().synth_e4m3_scales(seed, stream, K, row0, nrows, _ptr(out)) != 0:
+        raise ValueError(f"synth: bad shape K={K}")
+    return out
+
+
+# the per-tensor scale of every synthetic NVFP4 tensor (fp32): with codes of
+# magnitude up to 6 and block scales up to 3.75, weights stay below 0.23
+NVFP4_TENSOR_SCALE = 0.01
+
+
+def nvfp4_tensor(seed: int, tensor_id: int, N: int, K: int, row0: int = 0, nrows: int | None = None):
+    """(canonical codes [nrows][K/2], E4M3 block scales [nrows][K/16], tensor scale) of a synthetic NVFP4 tensor:
+    uniform codes (every 4-bit pattern) from the q4 code stream of the tensor id, scales from its scale stream."""
+    if nrows is None:
+        nrows = N - row0
+    c = weights(4, seed, weight_stream(tensor_id), K, row0, nrows)
+    s = e4m3_scales(seed, scale_stream(tensor_id), K, row0, nrows)
+    return c, s, NVFP4_TENSOR_SCALE
+
+
 def tensor(bits: int, seed: int, tensor_id: int, N: int, K: int, row0: int = 0, nrows: int | None = None):
     """(canonical q, fp16 scale bits) of one synthetic weight tensor (or a row slice of it)."""
     if nrows is None:
@@ -201,6 +226,12 @@ def scales_device(seed: int, stream_id: int, K: int, row0: int, nrows: int, out,
                "scales")
 
 
+def e4m3_scales_device(seed: int, stream_id: int, K: int, row0: int, nrows: int, out, stream=None) -> None:
+    if out.numel() * out.element_size() < nrows * (K // 16):
+        raise ValueError("output tensor too small")
+    _dev_check(lib().synth_e4m3_scales_device(seed, stream_id, K, row0, nrows, _dev(out), _stream(stream)), "e4m3 scales")
+
+
 def activations_device(seed: int, stream_id: int, M: int, K: int, out, stream=None) -> None:
     if out.numel() * out.element_size() < 2 * M * K:
         raise ValueError("output tensor too small")
@@ -211,4 +242,5 @@ __all__ = [
     "weights_device", "scales_device", "activations_device", "log_f64", "cos2pi_f64",
     "weights", "scales", "activations", "normals_f64", "words", "f64_to_f16_bits", "f64_to_bf16_bits",
     "tensor", "weight_stream", "scale_stream", "act_stream", "SCALE_STD", "lib",
+    "e4m3_scales", "e4m3_scales_device", "nvfp4_tensor", "NVFP4_TENSOR_SCALE",
 ]

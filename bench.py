@@ -13,7 +13,8 @@ line also reports the ordered and graph stack modes, the end-to-end step
 through the public API ("e2e"), the roofline of the dominant kernel, the CPU
 oracle's rate ("cpu_baseline"), the SM clock under load, "chain" (the same
 products as a dependent chain with the residual + RMSNorm and SwiGLU steps
-between them, M = 1 and 4), and "per_config":
+between them, M = 1 and 4), "nvfp4" (the same stream with its 4-bit tensors
+in NVFP4, the same bytes, M = 1 and 4), and "per_config":
 microseconds per product of the single-tensor configurations (q4 4096 x 4096,
 each projection of one layer at M = 1 and 4, the q8 vocabulary heads).
 
@@ -434,6 +435,26 @@ def run_ours(args, d: Dist):
     del st4
     torch.cuda.empty_cache()
 
+    # the same stream with its 4-bit tensors in NVFP4 (E2M1 codes, E4M3 block
+    # scales of 16, fp32 tensor scale): the same shapes and weight bytes
+    nvfp4 = {}
+    nv_tensors = workloads.as_nvfp4(tensors)
+    assert workloads.total_bytes(nv_tensors) == wbytes
+    for M in (1, 4):
+        sn = workloads.DeviceStream(nv_tensors, M, seed=args.seed, flags=q4.Q4_STACK_INDEPENDENT)
+        for _ in range(args.warmup):
+            sn.run()
+        d.barrier()
+        n_nv = max(3, args.steps // 2)
+        ms_nv = d.max(time_region(torch, sn.run, n_nv, stream) / n_nv)
+        sn.check()
+        nvfp4[f"M{M}"] = {"value": round(wbytes * d.world / (ms_nv * 1e6), 1), "unit": UNIT,
+                          "ms_per_step": round(ms_nv, 5), "pct_of_hbm_peak": round(100 * wbytes / (ms_nv * 1e6) / peak, 2),
+                          "tok_per_s": round(1000.0 / ms_nv, 1), "launches": sn.stack.launches()}
+        sn.close()
+        del sn
+        torch.cuda.empty_cache()
+
     # the dependent chain: the same products with the steps between them
     # (residual + RMSNorm, SwiGLU), one CUDA graph with programmatic dependent launch
     chain = {}
@@ -518,6 +539,7 @@ def run_ours(args, d: Dist):
             "d2h_bytes_per_step": d2h,
         },
         "chain": chain,
+        "nvfp4": nvfp4,
         "per_config": configs,
         "gpu_launches": n_launch * args.steps,
         "clocks": clocks,

@@ -238,3 +238,139 @@ extern "C" Q4_API int q4_unpack_weights(int bits, const void* packed, size_t pac
   }
   return Q4_OK;
 }
+
+// ----------------------------------------------------------------------------
+// NVFP4 (FP4 E2M1 codes, one FP8 E4M3 scale per 16 values along K, one fp32
+// scale per tensor).  The chunk is that of q4 -- 32 rows x 64 columns, 1024
+// code bytes then 128 scale bytes -- with the codes of one tensor-core A
+// register in one byte (the hardware converts a byte of two E2M1 codes to an
+// fp16 pair, low nibble to the low half).  Byte r of word j in slot (gi, ti)
+// of half h holds row 16h + gi + 8 (r & 1), columns 32 (j >> 1) + 8 ti +
+// 4 (j & 1) + 2 (r >> 1) + {0, 1} of the chunk: the same positions as the q4
+// nibbles of register r, so both formats share the activation fragments.  A
+// lane then needs the block 4c + 2G + ti / 2 of group G: the 8 scale bytes at
+// 1024 + 8 (2 gi + ti / 2) are, at 4h + 2G + up, row 16h + gi + 8up.  The
+// tensor scale sits in the 16 bytes after the last chunk.
+// ----------------------------------------------------------------------------
+namespace {
+
+constexpr int64_t kNvfp4Trailer = 16;
+
+bool nvfp4_geometry(int64_t N, int64_t K, Geometry* g) {
+  if (!geometry(4, N, K, g)) return false;
+  return K % 64 == 0;
+}
+
+inline void nvfp4_coord(int64_t t, int64_t c, int h, int gi, int ti, int j, int r, int64_t* row, int64_t* col) {
+  *row = kTileRows * t + 16 * h + gi + 8 * (r & 1);
+  *col = 64 * c + 32 * (j >> 1) + 8 * ti + 4 * (j & 1) + 2 * (r >> 1);
+}
+
+inline int64_t nvfp4_scale_row(int64_t t, int h, int gi, int up) { return kTileRows * t + 16 * h + gi + 8 * up; }
+
+}  // namespace
+
+extern "C" Q4_API size_t q4_nvfp4_packed_bytes(int64_t N, int64_t K) {
+  Geometry g;
+  if (!nvfp4_geometry(N, K, &g)) return 0;
+  return static_cast<size_t>(g.T * g.C * g.chunk_bytes + kNvfp4Trailer);
+}
+
+extern "C" Q4_API int q4_pack_nvfp4(const uint8_t* codes, const uint8_t* scales, float tensor_scale, int64_t N,
+                                    int64_t K, void* out, size_t out_bytes) {
+  Geometry g;
+  if (!nvfp4_geometry(N, K, &g)) {
+    q4::set_error("q4_pack_nvfp4: need N >= 0, K >= 0, K % 64 == 0");
+    return Q4_ERR_SHAPE;
+  }
+  const size_t need = static_cast<size_t>(g.T * g.C * g.chunk_bytes + kNvfp4Trailer);
+  if (!out || (N * K > 0 && (!codes || !scales))) {
+    q4::set_error("q4_pack_nvfp4: null pointer");
+    return Q4_ERR_INVALID_ARG;
+  }
+  if (out_bytes < need) {
+    q4::set_error("q4_pack_nvfp4: out_bytes " + std::to_string(out_bytes) + " < " + std::to_string(need));
+    return Q4_ERR_BUFFER_TOO_SMALL;
+  }
+  const int64_t B = K / 16;
+  uint8_t* dst = static_cast<uint8_t*>(out);
+#pragma omp parallel for schedule(static)
+  for (int64_t t = 0; t < g.T; ++t) {
+    for (int64_t c = 0; c < g.C; ++c) {
+      uint8_t* chunk = dst + (t * g.C + c) * g.chunk_bytes;
+      for (int h = 0; h < 2; ++h)
+        for (int gi = 0; gi < 8; ++gi)
+          for (int ti = 0; ti < 4; ++ti) {
+            uint8_t slot[16];
+            for (int j = 0; j < 4; ++j)
+              for (int r = 0; r < 4; ++r) {
+                int64_t row, col;
+                nvfp4_coord(t, c, h, gi, ti, j, r, &row, &col);
+                // col is even: the two codes are the two nibbles of one canonical byte
+                slot[4 * j + r] = row < N ? codes[row * (K / 2) + col / 2] : 0;
+              }
+            std::memcpy(chunk + 512 * h + 16 * (4 * gi + ti), slot, 16);
+          }
+      for (int gi = 0; gi < 8; ++gi)
+        for (int tb = 0; tb < 2; ++tb) {
+          uint8_t s8[8];
+          for (int h = 0; h < 2; ++h)
+            for (int G = 0; G < 2; ++G)
+              for (int up = 0; up < 2; ++up) {
+                const int64_t row = nvfp4_scale_row(t, h, gi, up), blk = 4 * c + 2 * G + tb;
+                s8[4 * h + 2 * G + up] = row < N ? scales[row * B + blk] : 0;
+              }
+          std::memcpy(chunk + 1024 + 8 * (2 * gi + tb), s8, 8);
+        }
+    }
+  }
+  uint8_t trailer[kNvfp4Trailer] = {};
+  std::memcpy(trailer, &tensor_scale, 4);
+  std::memcpy(dst + g.T * g.C * g.chunk_bytes, trailer, kNvfp4Trailer);
+  return Q4_OK;
+}
+
+extern "C" Q4_API int q4_unpack_nvfp4(const void* packed, size_t packed_bytes, int64_t N, int64_t K,
+                                      uint8_t* codes_out, uint8_t* scales_out, float* tensor_scale_out) {
+  Geometry g;
+  if (!nvfp4_geometry(N, K, &g)) {
+    q4::set_error("q4_unpack_nvfp4: need N >= 0, K >= 0, K % 64 == 0");
+    return Q4_ERR_SHAPE;
+  }
+  const size_t need = static_cast<size_t>(g.T * g.C * g.chunk_bytes + kNvfp4Trailer);
+  if (!packed || !tensor_scale_out || (N * K > 0 && (!codes_out || !scales_out))) {
+    q4::set_error("q4_unpack_nvfp4: null pointer");
+    return Q4_ERR_INVALID_ARG;
+  }
+  if (packed_bytes < need) {
+    q4::set_error("q4_unpack_nvfp4: packed_bytes too small");
+    return Q4_ERR_BUFFER_TOO_SMALL;
+  }
+  const int64_t B = K / 16;
+  const uint8_t* src = static_cast<const uint8_t*>(packed);
+#pragma omp parallel for schedule(static)
+  for (int64_t t = 0; t < g.T; ++t) {
+    for (int64_t c = 0; c < g.C; ++c) {
+      const uint8_t* chunk = src + (t * g.C + c) * g.chunk_bytes;
+      for (int h = 0; h < 2; ++h)
+        for (int gi = 0; gi < 8; ++gi)
+          for (int ti = 0; ti < 4; ++ti)
+            for (int j = 0; j < 4; ++j)
+              for (int r = 0; r < 4; ++r) {
+                int64_t row, col;
+                nvfp4_coord(t, c, h, gi, ti, j, r, &row, &col);
+                if (row < N) codes_out[row * (K / 2) + col / 2] = chunk[512 * h + 16 * (4 * gi + ti) + 4 * j + r];
+              }
+      for (int gi = 0; gi < 8; ++gi)
+        for (int tb = 0; tb < 2; ++tb)
+          for (int h = 0; h < 2; ++h)
+            for (int G = 0; G < 2; ++G)
+              for (int up = 0; up < 2; ++up) {
+                const int64_t row = nvfp4_scale_row(t, h, gi, up), blk = 4 * c + 2 * G + tb;
+                if (row < N) scales_out[row * B + blk] = chunk[1024 + 8 * (2 * gi + tb) + 4 * h + 2 * G + up];
+              }
+    }
+  }
+  std::memcpy(tensor_scale_out, src + g.T * g.C * g.chunk_bytes, 4);
+  return Q4_OK;
+}

@@ -148,6 +148,17 @@ int make_shape(int bits, int64_t N, int64_t K, Shape* s, const char* who) {
   return Q4_OK;
 }
 
+// A stack entry's shape: bits 4 or 8, or Q4_FMT_NVFP4 (the q4 chunk geometry,
+// K a multiple of 64).
+int entry_shape(int bits, int64_t N, int64_t K, Shape* s, const char* who) {
+  if (bits != Q4_FMT_NVFP4) return make_shape(bits, N, K, s, who);
+  const int rc = make_shape(4, N, K, s, who);
+  if (rc) return rc;
+  if (K % 64 != 0) return fail(Q4_ERR_SHAPE, "%s: NVFP4 needs K %% 64 == 0 (K=%lld)", who, (long long)K);
+  s->bits = Q4_FMT_NVFP4;
+  return Q4_OK;
+}
+
 long long max_warps(const DeviceInfo& dev) { return static_cast<long long>(dev.sms) * kCtasPerSm * kNW; }
 
 // Workspace layout: [status word | partial sums | tile counters].  The
@@ -423,6 +434,46 @@ extern "C" Q4_API int q4_pack_weights_device(int bits, const void* canon_q, cons
   return err == cudaSuccess ? Q4_OK : cuda_fail(err, "pack kernel launch");
 }
 
+extern "C" Q4_API int q4_pack_nvfp4_device(const uint8_t* codes, const uint8_t* scales, float tensor_scale,
+                                           int64_t N, int64_t K, void* out, size_t out_bytes, void* stream) {
+  Shape s;
+  int rc = entry_shape(Q4_FMT_NVFP4, N, K, &s, "q4_pack_nvfp4_device");
+  if (rc) return rc;
+  const size_t need = static_cast<size_t>(s.TC) * q4k::Format<4>::kChunkBytes + q4k::kNvfp4TrailerBytes;
+  if (!out || (s.TC > 0 && (!codes || !scales))) return fail(Q4_ERR_INVALID_ARG, "q4_pack_nvfp4_device: null pointer");
+  if (reinterpret_cast<uintptr_t>(out) % 16)
+    return fail(Q4_ERR_ALIGN, "q4_pack_nvfp4_device: out must be 16-byte aligned");
+  if (out_bytes < need)
+    return fail(Q4_ERR_BUFFER_TOO_SMALL, "q4_pack_nvfp4_device: out_bytes %zu < %zu", out_bytes, need);
+  DeviceInfo dev;
+  if ((rc = device_info(&dev))) return rc;
+  const long long threads = std::max(1LL, s.TC * 64);
+  const long long blocks = (threads + 255) / 256;
+  if (blocks > 0x7FFFFFFFLL) return fail(Q4_ERR_SHAPE, "q4_pack_nvfp4_device: tensor too large");
+  q4k::pack_nvfp4_kernel<<<static_cast<unsigned>(blocks), 256, 0, static_cast<cudaStream_t>(stream)>>>(
+      codes, scales, tensor_scale, s.N, s.K, s.T, s.C, static_cast<uint8_t*>(out));
+  cudaError_t err = cudaGetLastError();
+  return err == cudaSuccess ? Q4_OK : cuda_fail(err, "NVFP4 pack kernel launch");
+}
+
+extern "C" Q4_API int q4_nvfp4_dequant_device(const void* packed, int64_t N, int64_t K, float* w_out, void* stream) {
+  Shape s;
+  int rc = entry_shape(Q4_FMT_NVFP4, N, K, &s, "q4_nvfp4_dequant_device");
+  if (rc) return rc;
+  if (s.TC == 0) return Q4_OK;
+  if (!packed || !w_out) return fail(Q4_ERR_INVALID_ARG, "q4_nvfp4_dequant_device: null pointer");
+  if (reinterpret_cast<uintptr_t>(packed) % 16 || reinterpret_cast<uintptr_t>(w_out) % 4)
+    return fail(Q4_ERR_ALIGN, "q4_nvfp4_dequant_device: packed must be 16-byte, w_out 4-byte aligned");
+  DeviceInfo dev;
+  if ((rc = device_info(&dev))) return rc;
+  const long long blocks = (s.TC * 64 + 255) / 256;
+  if (blocks > 0x7FFFFFFFLL) return fail(Q4_ERR_SHAPE, "q4_nvfp4_dequant_device: tensor too large");
+  q4k::dequant_nvfp4_kernel<<<static_cast<unsigned>(blocks), 256, 0, static_cast<cudaStream_t>(stream)>>>(
+      static_cast<const uint8_t*>(packed), s.N, s.K, s.T, s.C, w_out);
+  cudaError_t err = cudaGetLastError();
+  return err == cudaSuccess ? Q4_OK : cuda_fail(err, "NVFP4 dequant kernel launch");
+}
+
 extern "C" Q4_API int q4_selftest_wait_timeout(uint64_t timeout_ns, int* status_out) {
   if (!status_out) return fail(Q4_ERR_INVALID_ARG, "q4_selftest_wait_timeout: status_out is null");
   DeviceInfo dev;
@@ -586,7 +637,7 @@ bool stack_eligible(const q4_stack_entry* entries, int n) {
   if (n <= 0) return false;
   for (int i = 0; i < n; ++i) {
     Shape s;
-    if (make_shape(entries[i].bits, entries[i].N, entries[i].K, &s, "layer_stack_create")) return false;
+    if (entry_shape(entries[i].bits, entries[i].N, entries[i].K, &s, "layer_stack_create")) return false;
     if (s.N == 0 || s.K == 0 || s.C % 2 != 0) return false;
   }
   return true;
@@ -605,7 +656,7 @@ int create_persistent(const q4_stack_entry* entries, int n, int M, int su, const
     char who[64];
     snprintf(who, sizeof(who), "layer_stack_create entry %d", i);
     Shape s;
-    int rc = make_shape(en.bits, en.N, en.K, &s, who);
+    int rc = entry_shape(en.bits, en.N, en.K, &s, who);
     if (rc) return rc;
     if (!en.packed || !en.x || !en.y) return fail(Q4_ERR_INVALID_ARG, "%s: null device pointer", who);
     if (reinterpret_cast<uintptr_t>(en.packed) % 16 || reinterpret_cast<uintptr_t>(en.x) % 16 ||
@@ -641,7 +692,7 @@ int create_persistent(const q4_stack_entry* entries, int n, int M, int su, const
   size_t prep_bytes = 0;
   if (independent) {
     for (int i = 0; i < n; ++i) {
-      const int KC = entries[i].bits == 4 ? q4k::Format<4>::kKPerChunk : q4k::Format<8>::kKPerChunk;
+      const int KC = entries[i].bits == 8 ? q4k::Format<8>::kKPerChunk : q4k::Format<4>::kKPerChunk;
       size_t jdx = jobs.size();
       for (size_t k = 0; k < jobs.size(); ++k)
         if (jobs[k].x == entries[i].x && jobs[k].K == entries[i].K && jobs[k].KC == KC) jdx = k;
@@ -783,6 +834,18 @@ extern "C" Q4_API int layer_stack_create(const q4_stack_entry* entries, int n_en
   DeviceInfo dev;
   int rc = device_info(&dev);
   if (rc) return rc;
+  // NVFP4 products run in stream mode only
+  for (int i = 0; i < n_entries; ++i) {
+    if (entries[i].bits != Q4_FMT_NVFP4) continue;
+    char who[64];
+    snprintf(who, sizeof(who), "layer_stack_create entry %d", i);
+    Shape s;
+    if ((rc = entry_shape(entries[i].bits, entries[i].N, entries[i].K, &s, who))) return rc;
+    if ((flags & Q4_STACK_INDEPENDENT) == 0 || (flags & (Q4_STACK_GRAPH | Q4_STACK_NO_PDL)) != 0)
+      return fail(Q4_ERR_UNSUPPORTED, "%s: NVFP4 products need stream mode (Q4_STACK_INDEPENDENT alone)", who);
+    if (!stack_eligible(entries, n_entries))
+      return fail(Q4_ERR_UNSUPPORTED, "%s: NVFP4 needs every product non-empty with an even chunk count", who);
+  }
   q4_stack* st = new q4_stack();
   cudaGetDevice(&st->device);
   const bool graph = (flags & (Q4_STACK_GRAPH | Q4_STACK_NO_PDL)) != 0 || !stack_eligible(entries, n_entries);
@@ -794,11 +857,17 @@ extern "C" Q4_API int layer_stack_create(const q4_stack_entry* entries, int n_en
     if (entries[i].bits == 4 && entries[i].K % 64 != 0) {
       su = 0;
     } else {
-      const long long kc = entries[i].bits == 4 ? 64 : 32;
+      const long long kc = entries[i].bits == 8 ? 32 : 64;
       const long long C = (entries[i].K + kc - 1) / kc;
       if (C % su != 0) su = 2;
     }
   }
+  for (int i = 0; i < n_entries; ++i)
+    if (entries[i].bits == Q4_FMT_NVFP4 && su == 0) {
+      free_stack(st);
+      return fail(Q4_ERR_UNSUPPORTED, "layer_stack_create: NVFP4 products need stream mode, and a q4 product "
+                                      "with K %% 64 != 0 rules it out");
+    }
   rc = graph ? create_graph(entries, n_entries, M, flags, dev, st)
              : create_persistent(entries, n_entries, M, su, dev, st);
   if (rc) {

@@ -23,6 +23,7 @@
 #include <climits>
 
 #include "q4gemv_kernels.cuh"
+#include "q4nvfp4_kernel.cuh"
 
 namespace q4k {
 
@@ -492,7 +493,7 @@ struct StreamProducer {
 
   __device__ __forceinline__ void enter(const StackParams& sp, int entry, long long lb) {
     const StackEntryDev& en = sp.entries[entry];
-    const int CB = en.bits == 4 ? Format<4>::kChunkBytes : Format<8>::kChunkBytes;
+    const int CB = en.bits == 8 ? Format<8>::kChunkBytes : Format<4>::kChunkBytes;  // NVFP4: the q4 geometry
     e = entry;
     bytes = static_cast<uint32_t>(SU * CB);
     src = en.packed + lb * SU * CB;
@@ -500,7 +501,7 @@ struct StreamProducer {
     left_entry = static_cast<int>(in_entry < left_total ? in_entry : left_total);
     xc = en.xc;
     C = en.C;
-    KC = en.bits == 4 ? Format<4>::kKPerChunk : Format<8>::kKPerChunk;
+    KC = en.bits == 8 ? Format<8>::kKPerChunk : Format<4>::kKPerChunk;
     const int bpt = en.C / SU;
     cpos = static_cast<int>(lb - static_cast<long long>(floor_div(lb, bpt)) * bpt) * SU;
   }
@@ -546,12 +547,14 @@ struct StreamRing {
   int in_flight = 0;     // stages issued and not yet consumed
 };
 
-// Consumes `nblk` stages (SU chunks each) of one product (format BITS), from
+// Consumes `nblk` stages (SU chunks each) of one product (format BITS: 4, 8
+// or kFmtNvfp4), from
 // local block lb0.  Keeps the split-tile bookkeeping of the warp's range
 // [gb, ...): the partial of a tile that began before gb goes to partial slot
 // 0 when the tile ends (e_first, r_first); a tile still open at the end stays
 // in acc with (r, c).  Returns false if a ring wait gave up.
-// F16: the activations are used in fp16 (en.x16, outputs times `scale`).
+// F16: the activations are used in fp16 (en.x16).  Finished tile sums are
+// multiplied by `scale` (2^sigma when F16, times t for NVFP4).
 template <int BITS, int M, int D, int SU, bool F16>
 __device__ __forceinline__ bool stream_segment(const StackParams& sp, const StackEntryDev* __restrict__ ep, int e,
                                                long long lb0,
@@ -561,8 +564,10 @@ __device__ __forceinline__ bool stream_segment(const StackParams& sp, const Stac
                                                int& c, int lane) {
   constexpr int U = SU;
   constexpr int SLOT = StreamSlot<SU, M>::kBytes;
-  constexpr int CB = Format<BITS>::kChunkBytes;
-  constexpr int KC = Format<BITS>::kKPerChunk;
+  constexpr bool NV = BITS == kFmtNvfp4;
+  constexpr int FB = BITS == 8 ? 8 : 4;  // NVFP4 chunks have the q4 geometry
+  constexpr int CB = Format<FB>::kChunkBytes;
+  constexpr int KC = Format<FB>::kKPerChunk;
   const int gi = lane >> 2, ti = lane & 3;
   const int C = ep->C;  // the entry's other fields are read where they are used, not held in registers
   const int bpt = C / U;
@@ -579,10 +584,13 @@ __device__ __forceinline__ bool stream_segment(const StackParams& sp, const Stac
     for (int j = 0; j < U; ++j) {
       ChunkRegs cr;
       const uint4 xa = lds128(stage + xlane + j * M * KC * 2);
-      const uint4 xb = BITS == 4 ? lds128(stage + xlane + j * M * KC * 2 + 64) : make_uint4(0, 0, 0, 0);
+      const uint4 xb = FB == 4 ? lds128(stage + xlane + j * M * KC * 2 + 64) : make_uint4(0, 0, 0, 0);
       cr.codes[0] = lds128(stage + j * CB + 16 * lane);
       cr.codes[1] = lds128(stage + j * CB + kHalfBytes + 16 * lane);
-      if (BITS == 4) {
+      if (NV) {
+        const uint2 s2 = lds64(stage + j * CB + kCodeBytes + 8 * (2 * gi + (ti >> 1)));
+        cr.scales = make_uint4(s2.x, s2.y, 0u, 0u);
+      } else if (BITS == 4) {
         cr.scales = lds128(stage + j * CB + kCodeBytes + 16 * gi);
       } else {
         const uint2 s2 = lds64(stage + j * CB + kCodeBytes + 8 * gi);
@@ -597,7 +605,9 @@ __device__ __forceinline__ bool stream_segment(const StackParams& sp, const Stac
           rg.phase ^= 1u;
         }
       }
-      if (BITS == 4) {  // stream mode has whole q4 chunks only (K % 64 == 0, checked on the host)
+      if (NV) {
+        nvfp4_chunk_mac<F16>(acc, cr.codes, make_uint2(cr.scales.x, cr.scales.y), xa, xb);
+      } else if (BITS == 4) {  // stream mode has whole q4 chunks only (K % 64 == 0, checked on the host)
         q4_chunk_mac<F16>(acc, cr, xa, xb);
       } else {
         q8_chunk_mac<F16>(acc, cr, xa);
@@ -605,7 +615,7 @@ __device__ __forceinline__ bool stream_segment(const StackParams& sp, const Stac
     }
     c += U;
     if (c == C) {
-      if (F16) scale_acc(acc, scale);
+      if (F16 || NV) scale_acc(acc, scale);
       const long long tile_g = ep->blk_off + static_cast<long long>(r) * bpt;  // the tile's first block
       if (tile_g < gb) {  // began in an earlier warp's range: its partial goes to slot 0 now
         write_partial<M>(sp.partials, pw, 0, acc, lane);
@@ -691,7 +701,13 @@ __global__ void __launch_bounds__(NW * 32, 1) stream_kernel(const StackParams sp
     const long long n = in_entry < left ? in_entry : left;
     const XInfo xi = *ep->xinfo;  // written by xprep_kernel, complete once griddepcontrol.wait returned
     scale = xi.ok ? xi.scale : 1.f;
-    if (ep->bits == 4) {
+    if (ep->bits == kFmtNvfp4) {
+      scale *= *reinterpret_cast<const float*>(ep->packed + ep->TC * Format<4>::kChunkBytes);  // t
+      ok = xi.ok ? stream_segment<kFmtNvfp4, M, D, SU, true>(sp, ep, e, lb, n, gb, rg, pr, policy, scale, acc, pw,
+                                                             e_first, r_first, r, c, lane)
+                 : stream_segment<kFmtNvfp4, M, D, SU, false>(sp, ep, e, lb, n, gb, rg, pr, policy, scale, acc, pw,
+                                                              e_first, r_first, r, c, lane);
+    } else if (ep->bits == 4) {
       ok = xi.ok ? stream_segment<4, M, D, SU, true>(sp, ep, e, lb, n, gb, rg, pr, policy, scale, acc, pw, e_first,
                                                      r_first, r, c, lane)
                  : stream_segment<4, M, D, SU, false>(sp, ep, e, lb, n, gb, rg, pr, policy, scale, acc, pw,

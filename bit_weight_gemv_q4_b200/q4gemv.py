@@ -34,6 +34,7 @@ Q4_QUANT_SIGNED_MAX = 1
 Q4_OP_PRODUCT = 0
 Q4_OP_RESIDUAL_RMSNORM = 1
 Q4_OP_SWIGLU = 2
+Q4_FMT_NVFP4 = 16
 
 ERROR_NAMES = {
     Q4_ERR_INVALID_ARG: "INVALID_ARG",
@@ -52,7 +53,8 @@ EXPORTED = [
     "q4_gemv", "q8_gemv", "q4_gemv_noalloc", "q4_workspace_check", "q4_set_wait_timeout_ns", "q4_unpack_device",
     "q4_selftest_wait_timeout", "layer_stack_create", "layer_stack_run", "layer_stack_check",
     "layer_stack_launches", "layer_stack_destroy", "q4_quantize", "q4_quantize_device", "layer_chain_create",
-    "q4_residual_rmsnorm", "q4_swiglu",
+    "q4_residual_rmsnorm", "q4_swiglu", "q4_nvfp4_packed_bytes", "q4_pack_nvfp4", "q4_unpack_nvfp4",
+    "q4_pack_nvfp4_device", "q4_nvfp4_dequant_device",
 ]
 
 
@@ -119,6 +121,11 @@ def _load() -> ctypes.CDLL:
         "q4_residual_rmsnorm": ([vp, vp, vp, vp, i64, i32, i32, vp], i32),
         "q4_swiglu": ([vp, vp, i64, i32, vp], i32),
         "q4_quantize_device": ([i32, i32, vp, i64, i64, vp, vp, vp], i32),
+        "q4_nvfp4_packed_bytes": ([i64, i64], sz),
+        "q4_pack_nvfp4": ([vp, vp, ctypes.c_float, i64, i64, vp, sz], i32),
+        "q4_unpack_nvfp4": ([vp, sz, i64, i64, vp, vp, ctypes.POINTER(ctypes.c_float)], i32),
+        "q4_pack_nvfp4_device": ([vp, vp, ctypes.c_float, i64, i64, vp, sz, vp], i32),
+        "q4_nvfp4_dequant_device": ([vp, i64, i64, vp, vp], i32),
     }
     for name, (args, res) in sig.items():
         f = getattr(L, name)
@@ -199,6 +206,44 @@ def q4_unpack_weights(bits: int, packed: np.ndarray, N: int, K: int) -> tuple[np
     s = np.zeros((N, K // 32), dtype=np.uint16)
     _check(_lib.q4_unpack_weights(bits, packed.ctypes.data, packed.size, N, K, q.ctypes.data, s.ctypes.data))
     return q, s
+
+
+def q4_nvfp4_packed_bytes(N: int, K: int) -> int:
+    return int(_lib.q4_nvfp4_packed_bytes(N, K))
+
+
+def q4_pack_nvfp4(codes: np.ndarray, scales: np.ndarray, tensor_scale: float, N: int, K: int) -> np.ndarray:
+    """NVFP4 canonical codes [N][K/2], E4M3 scale bytes [N][K/16] and the fp32
+    tensor scale (host) -> packed bytes (numpy uint8)."""
+    c = np.ascontiguousarray(codes, dtype=np.uint8)
+    sc = np.ascontiguousarray(scales, dtype=np.uint8)
+    if c.size != N * (K // 2) or sc.size != N * (K // 16):
+        raise Q4Error(Q4_ERR_SHAPE, f"canonical NVFP4 arrays do not match N={N} K={K}")
+    n = q4_nvfp4_packed_bytes(N, K)
+    out = np.zeros(max(n, 1), dtype=np.uint8)
+    _check(_lib.q4_pack_nvfp4(c.ctypes.data, sc.ctypes.data, float(tensor_scale), N, K, out.ctypes.data, out.size))
+    return out[:n]
+
+
+def q4_unpack_nvfp4(packed: np.ndarray, N: int, K: int) -> tuple[np.ndarray, np.ndarray, float]:
+    packed = np.ascontiguousarray(packed, dtype=np.uint8)
+    c = np.zeros((N, K // 2), dtype=np.uint8)
+    sc = np.zeros((N, K // 16), dtype=np.uint8)
+    t = ctypes.c_float(0.0)
+    _check(_lib.q4_unpack_nvfp4(packed.ctypes.data, packed.size, N, K, c.ctypes.data, sc.ctypes.data,
+                                ctypes.byref(t)))
+    return c, sc, t.value
+
+
+def q4_pack_nvfp4_device(codes, scales, tensor_scale: float, N: int, K: int, out, stream=None) -> None:
+    """The NVFP4 repack on device tensors."""
+    _check(_lib.q4_pack_nvfp4_device(_dev_ptr(codes), _dev_ptr(scales), float(tensor_scale), N, K, _dev_ptr(out),
+                                     _nbytes(out), _stream(stream)))
+
+
+def q4_nvfp4_dequant_device(packed, N: int, K: int, w_out, stream=None) -> None:
+    """Debug decoder: the fp32 weights [N][K] the product kernels multiply."""
+    _check(_lib.q4_nvfp4_dequant_device(_dev_ptr(packed), N, K, _dev_ptr(w_out), _stream(stream)))
 
 
 def q4_quantize(bits: int, mode: int, w_bf16: np.ndarray) -> tuple[np.ndarray, np.ndarray]:
@@ -350,5 +395,6 @@ __all__ = [
     "layer_stack_create", "layer_stack_run", "layer_stack_check", "layer_stack_destroy",
     "q4_quantize", "q4_quantize_device", "Q4_QUANT_ABSMAX", "Q4_QUANT_SIGNED_MAX",
     "layer_chain_create", "ChainOp", "Q4_OP_PRODUCT", "Q4_OP_RESIDUAL_RMSNORM", "Q4_OP_SWIGLU",
-    "q4_residual_rmsnorm", "q4_swiglu",
+    "q4_residual_rmsnorm", "q4_swiglu", "Q4_FMT_NVFP4", "q4_nvfp4_packed_bytes", "q4_pack_nvfp4", "q4_unpack_nvfp4",
+    "q4_pack_nvfp4_device", "q4_nvfp4_dequant_device",
 ]

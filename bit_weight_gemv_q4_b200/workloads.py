@@ -13,6 +13,8 @@ post, part four).
 
 Algorithmic weight bytes per tensor: N*K/2 + 2*N*K/32 (q4) and
 N*K + 2*N*K/32 (q8): the integer codes plus one fp16 scale per group of 32.
+NVFP4 tensors (bits = NVFP4) hold N*K/2 code bytes plus one E4M3 byte per 16
+values, N*K/16: the same 4.5 bits per weight as q4.
 """
 from __future__ import annotations
 
@@ -24,10 +26,13 @@ KV = 1024
 VOCAB = 248320
 DRAFT_VOCAB = 65536
 N_LAYERS = 64
+NVFP4 = 16  # the format id of NVFP4 tensors (the library's Q4_FMT_NVFP4)
 
 
 def weight_bytes(bits: int, N: int, K: int) -> int:
-    """Algorithmic bytes of one N x K group-32 tensor (codes + fp16 scales)."""
+    """Algorithmic bytes of one N x K tensor (codes + scales)."""
+    if bits == NVFP4:
+        return N * K // 2 + N * (K // 16)
     codes = N * K // 2 if bits == 4 else N * K
     return codes + 2 * N * (K // 32)
 
@@ -95,6 +100,12 @@ def decode_stream(fused: bool = True) -> list[Tensor]:
     return out
 
 
+def as_nvfp4(tensors: list[Tensor]) -> list[Tensor]:
+    """The same list with every q4 tensor in NVFP4 instead (q8 tensors kept):
+    the same shapes and the same weight bytes."""
+    return [Tensor(t.name, NVFP4, t.N, t.K, t.tensor_id) if t.bits == 4 else t for t in tensors]
+
+
 def total_bytes(tensors: list[Tensor]) -> int:
     return sum(t.bytes for t in tensors)
 
@@ -127,18 +138,26 @@ class DeviceStream:
         self.M = M
         self.seed = seed
         dev = torch.device("cuda")
-        max_canon = max((t.N * (t.K // 2 if t.bits == 4 else t.K) for t in self.tensors), default=0)
-        max_scales = max((t.N * (t.K // 32) for t in self.tensors), default=0)
+        max_canon = max((t.N * (t.K if t.bits == 8 else t.K // 2) for t in self.tensors), default=0)
+        max_scales = max((t.N * (t.K // 16 if t.bits == NVFP4 else t.K // 32 * 2) for t in self.tensors), default=0)
         canon = torch.empty(max(max_canon, 16), dtype=torch.uint8, device=dev)
-        scales = torch.empty(max(max_scales, 8), dtype=torch.int16, device=dev)
+        scales = torch.empty(max(max_scales, 16), dtype=torch.uint8, device=dev)
         self.packed = []
         for t in self.tensors:
-            nq = t.N * (t.K // 2 if t.bits == 4 else t.K)
-            ns = t.N * (t.K // 32)
-            synth.weights_device(t.bits, seed, synth.weight_stream(t.tensor_id), t.K, 0, t.N, canon[:nq])
-            synth.scales_device(seed, synth.scale_stream(t.tensor_id), t.K, 0, t.N, scales[:ns])
-            p = torch.empty(q4.q4_packed_bytes(t.bits, t.N, t.K), dtype=torch.uint8, device=dev)
-            q4.q4_pack_weights_device(t.bits, canon[:nq], scales[:ns], t.N, t.K, p)
+            nq = t.N * (t.K if t.bits == 8 else t.K // 2)
+            if t.bits == NVFP4:  # codes from the q4 code stream, E4M3 scales from the scale stream
+                ns = t.N * (t.K // 16)
+                synth.weights_device(4, seed, synth.weight_stream(t.tensor_id), t.K, 0, t.N, canon[:nq])
+                synth.e4m3_scales_device(seed, synth.scale_stream(t.tensor_id), t.K, 0, t.N, scales[:ns])
+                p = torch.empty(q4.q4_nvfp4_packed_bytes(t.N, t.K), dtype=torch.uint8, device=dev)
+                q4.q4_pack_nvfp4_device(canon[:nq], scales[:ns], synth.NVFP4_TENSOR_SCALE, t.N, t.K, p)
+            else:
+                ns = t.N * (t.K // 32)
+                s16 = scales[: 2 * ns].view(torch.int16)
+                synth.weights_device(t.bits, seed, synth.weight_stream(t.tensor_id), t.K, 0, t.N, canon[:nq])
+                synth.scales_device(seed, synth.scale_stream(t.tensor_id), t.K, 0, t.N, s16)
+                p = torch.empty(q4.q4_packed_bytes(t.bits, t.N, t.K), dtype=torch.uint8, device=dev)
+                q4.q4_pack_weights_device(t.bits, canon[:nq], s16, t.N, t.K, p)
             self.packed.append(p)
         del canon, scales
         self.x = {}

@@ -162,6 +162,54 @@ Q4_API int q4_quantize_device(int bits, int mode, const uint16_t* w_bf16, int64_
 Q4_API int q4_unpack_weights(int bits, const void* packed, size_t packed_bytes, int64_t N, int64_t K,
                              void* canon_q_out, uint16_t* scales_out);
 
+/* ---------------------------------------------------------------------------
+ * NVFP4 weights (the 4-bit format the pages name for Blackwell engines:
+ * wiselychen.com guide, section "RTX 5090 32GB", SGLang / vLLM + NVFP4; the
+ * format's published definition).  Blocks of 16 values along K; each value an
+ * FP4 E2M1 code (sign, 2 exponent bits with bias 1, 1 mantissa bit: 0, 0.5,
+ * 1, 1.5, 2, 3, 4, 6 and negatives), each block one FP8 E4M3 scale (sign, 4
+ * exponent bits with bias 7, 3 mantissa bits, subnormals, S.1111.111 = NaN),
+ * the tensor one fp32 scale t:  w[n][k] = t * e4m3(s[n][k/16]) * e2m1(c[n][k]).
+ * Canonical layout: codes uint8 [N][K/2] (element k in byte k/2, low nibble
+ * for even k), scales uint8 [N][K/16] (E4M3 bits).  K % 64 == 0.
+ * Packed layout: T = ceil(N/32) tiles x C = K/64 chunks of 1152 bytes, in
+ * memory order t, c, then 16 bytes holding t (float, then zeros).  Chunk (t,c)
+ * covers rows 32t .. 32t+31, columns 64c .. 64c+63:
+ *   byte 512h + 16L + 4j + r (L = 4gi + ti; j = 2G + e; h, G, e in {0,1};
+ *   r in 0..3; gi in 0..7; ti in 0..3) holds the codes of row
+ *   32t + 16h + gi + 8(r & 1), columns 64c + 32G + 8ti + 4e + 2(r >> 1) + {0,1}
+ *   (low nibble the lower column);
+ *   byte 1024 + 8(2gi + b) + 4h + 2G + up (b, up in {0,1}) holds the scale of
+ *   row 32t + 16h + gi + 8up, block 4c + 2G + b.
+ * Padding rows hold code 0 and scale 0.  The code bytes are those of the q4
+ * layout's nibbles for the same tensor-core register, two per byte.
+ * -------------------------------------------------------------------------*/
+#define Q4_FMT_NVFP4 16 /* q4_stack_entry.bits value of an NVFP4 product (stream mode only) */
+
+/* Packed bytes of an N x K NVFP4 tensor (chunks plus the 16-byte trailer);
+ * 0 when N or K is negative or K % 64 != 0. */
+Q4_API size_t q4_nvfp4_packed_bytes(int64_t N, int64_t K);
+
+/* Host -> host repack.  Errors: INVALID_ARG (null), SHAPE, BUFFER_TOO_SMALL. */
+Q4_API int q4_pack_nvfp4(const uint8_t* codes, const uint8_t* scales, float tensor_scale, int64_t N, int64_t K,
+                         void* out, size_t out_bytes);
+
+/* Inverse of q4_pack_nvfp4 (host -> host); padding is dropped. */
+Q4_API int q4_unpack_nvfp4(const void* packed, size_t packed_bytes, int64_t N, int64_t K, uint8_t* codes_out,
+                           uint8_t* scales_out, float* tensor_scale_out);
+
+/* The same repack on the device (all pointers device memory, out 16-byte
+ * aligned), asynchronous on `stream`; the same bytes as q4_pack_nvfp4.
+ * Errors: as q4_pack_nvfp4, plus ALIGN and CUDA. */
+Q4_API int q4_pack_nvfp4_device(const uint8_t* codes, const uint8_t* scales, float tensor_scale, int64_t N,
+                                int64_t K, void* out, size_t out_bytes, void* stream);
+
+/* Debug decoder: the weights the product kernels multiply, through the same
+ * in-register conversion, as fp32 w_out [N][K] (device): the exact fp16
+ * product e4m3 * e2m1, times t in fp32.  Errors: INVALID_ARG, SHAPE, ALIGN,
+ * CUDA. */
+Q4_API int q4_nvfp4_dequant_device(const void* packed, int64_t N, int64_t K, float* w_out, void* stream);
+
 /* Bytes of device workspace q4_gemv / q8_gemv need for this shape on the
  * current device.  The workspace holds a status word, the per-warp partial
  * sums of tiles split between warps (a region of fixed size per device) and
@@ -240,7 +288,7 @@ Q4_API int q4_selftest_wait_timeout(uint64_t timeout_ns, int* status_out);
  * order, once; layer_stack_run replays them on a stream.
  * -------------------------------------------------------------------------*/
 typedef struct q4_stack_entry {
-  int bits;            /* 4 or 8 */
+  int bits;            /* 4 or 8, or Q4_FMT_NVFP4 (packed by q4_pack_nvfp4) */
   int64_t N, K;        /* weight shape */
   const void* packed;  /* device, packed layout */
   const uint16_t* x;   /* device, bf16 [M][K] */
@@ -275,6 +323,11 @@ typedef struct q4_stack q4_stack;
  * Both persistent modes need every product non-empty with an even number of
  * chunks per tile; other lists use graph mode.  Stream mode also needs every
  * q4 K to be a multiple of 64; otherwise the ordered mode is used.
+ * NVFP4 products (bits = Q4_FMT_NVFP4) run in stream mode only: a list holding
+ * one needs flags == Q4_STACK_INDEPENDENT and every product eligible for it,
+ * else UNSUPPORTED.  They decode each code byte and scale pair in one
+ * conversion and accumulate a whole tile on the tensor cores (the decoded
+ * weights are exact in fp16 and bf16); t multiplies the tile sums.
  * Graph mode (Q4_STACK_GRAPH, or Q4_STACK_NO_PDL): the products are launched in
  * order, each as its own kernel, and captured once as a CUDA graph; with PDL
  * each kernel prefetches its first weight tiles while its predecessor

@@ -62,7 +62,7 @@ def measured_peaks():
 def kernel_source_sha() -> str:
     h = hashlib.sha256()
     for rel in ("bit_weight_gemv_q4_b200/csrc/q4gemv_kernels.cuh", "bit_weight_gemv_q4_b200/csrc/q4stack_kernel.cuh",
-                "bit_weight_gemv_q4_b200/csrc/q4gemv.cu"):
+                "bit_weight_gemv_q4_b200/csrc/q4gemv.cu", "bit_weight_gemv_q4_b200/csrc/q4nvfp4_kernel.cuh"):
         with open(os.path.join(ROOT, rel), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
@@ -606,7 +606,8 @@ def run_profile_case(args):
     """Small cases for ncu.  Default: a q4 (or q8) 65536 x 5120 tensor (189 MB,
     larger than L2), `--profile-launches` launches at M = args.m.  With
     --profile-layers L: the first L layers of the decode stream (about 0.2 GB
-    per layer) as one stream-mode stack launch."""
+    per layer) as one stream-mode stack launch; --profile-nvfp4 puts their
+    4-bit tensors in NVFP4."""
     import torch
 
     import bit_weight_gemv_q4_b200 as q4
@@ -614,12 +615,15 @@ def run_profile_case(args):
 
     if args.profile_layers > 0:
         tensors = workloads.decode_stream(fused=True)[: 4 * args.profile_layers]
+        if args.profile_nvfp4:
+            tensors = workloads.as_nvfp4(tensors)
         st = workloads.DeviceStream(tensors, args.m, seed=args.seed, flags=q4.Q4_STACK_INDEPENDENT)
         for _ in range(args.profile_launches):
             st.run()
         torch.cuda.synchronize()
         st.check()
-        print(json.dumps({"profile_case": f"stream of {args.profile_layers} layers", "products": len(tensors),
+        print(json.dumps({"profile_case": f"stream of {args.profile_layers} layers"
+                          + (" (NVFP4)" if args.profile_nvfp4 else ""), "products": len(tensors),
                           "M": args.m, "launches": args.profile_launches, "weight_bytes": st.weight_bytes,
                           "kernel_source_sha": kernel_source_sha()}))
         st.close()
@@ -651,6 +655,7 @@ def main():
     ap.add_argument("--profile-bits", type=int, default=4)
     ap.add_argument("--profile-launches", type=int, default=3)
     ap.add_argument("--profile-layers", type=int, default=0)
+    ap.add_argument("--profile-nvfp4", action="store_true")
     ap.add_argument("--m", type=int, default=1)
     args = ap.parse_args()
     if args.warmup < 3 and not args.profile_case:

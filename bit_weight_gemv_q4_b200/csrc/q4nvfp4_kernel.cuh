@@ -29,18 +29,29 @@ namespace q4k {
 constexpr int kFmtNvfp4 = 16;           // format id of NVFP4 entries (the entry's `bits` field)
 constexpr int kNvfp4TrailerBytes = 16;  // the tensor scale, after the chunks
 
-// The E2M1 pair in the low byte of v -> fp16 pair (low nibble -> low half).
-__device__ __forceinline__ uint32_t e2m1x2_to_f16x2(uint32_t v) {
-  uint32_t d;
-  asm("{\n\t.reg .b8 t;\n\tcvt.u8.u32 t, %1;\n\tcvt.rn.f16x2.e2m1x2 %0, t;\n\t}" : "=r"(d) : "r"(v));
-  return d;
+// The four E2M1 pairs of a word -> four fp16 pairs: d[i] from byte i (low
+// nibble -> low half).  The word is split into byte registers by one vector
+// move, so the conversions read the bytes in place (no shifts).
+__device__ __forceinline__ void e2m1x8_to_f16x2(uint32_t w, uint32_t (&d)[4]) {
+  asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+      "mov.b32 {b0, b1, b2, b3}, %4;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %0, b0;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %1, b1;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %2, b2;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %3, b3;\n\t}"
+      : "=r"(d[0]), "=r"(d[1]), "=r"(d[2]), "=r"(d[3])
+      : "r"(w));
 }
 
-// The E4M3 pair in the low 16 bits of v -> fp16 pair (low byte -> low half).
-__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t v) {
-  uint32_t d;
-  asm("{\n\t.reg .b16 t;\n\tcvt.u16.u32 t, %1;\n\tcvt.rn.f16x2.e4m3x2 %0, t;\n\t}" : "=r"(d) : "r"(v));
-  return d;
+// The two E4M3 pairs of a word -> two fp16 pairs: lo from bytes 0, 1, hi
+// from bytes 2, 3 (the lower byte -> the low half).
+__device__ __forceinline__ void e4m3x4_to_f16x2(uint32_t w, uint32_t& lo, uint32_t& hi) {
+  asm("{\n\t.reg .b16 h0, h1;\n\t"
+      "mov.b32 {h0, h1}, %2;\n\t"
+      "cvt.rn.f16x2.e4m3x2 %0, h0;\n\t"
+      "cvt.rn.f16x2.e4m3x2 %1, h1;\n\t}"
+      : "=r"(lo), "=r"(hi)
+      : "r"(w));
 }
 
 __device__ __forceinline__ uint32_t f16x2_mul(uint32_t a, uint32_t b) {
@@ -74,19 +85,20 @@ __device__ __forceinline__ void nvfp4_chunk_mac(float (&acc)[2][4], const uint4 
 #pragma unroll
   for (int h = 0; h < 2; ++h) {
     const uint4& w = codes[h];
-    const uint32_t sw = h ? sc.y : sc.x;
+    uint32_t s2[2];  // per group G: (row 16h + gi, row 16h + gi + 8)
+    e4m3x4_to_f16x2(h ? sc.y : sc.x, s2[0], s2[1]);
 #pragma unroll
     for (int G = 0; G < 2; ++G) {
-      const uint32_t s2 = e4m3x2_to_f16x2(sw >> (16 * G));  // (row 16h + gi, row 16h + gi + 8)
-      const uint32_t s_r = byte_perm(s2, 0x1010u), s_r8 = byte_perm(s2, 0x3232u);
+      const uint32_t s_r = byte_perm(s2[G], 0x1010u), s_r8 = byte_perm(s2[G], 0x3232u);
       const uint4& xg = G ? xb : xa;
 #pragma unroll
       for (int e = 0; e < 2; ++e) {
         const uint32_t word = G ? (e ? w.w : w.z) : (e ? w.y : w.x);
         uint32_t a[4];
+        e2m1x8_to_f16x2(word, a);
 #pragma unroll
         for (int r = 0; r < 4; ++r) {
-          a[r] = f16x2_mul(e2m1x2_to_f16x2(word >> (8 * r)), (r & 1) ? s_r8 : s_r);
+          a[r] = f16x2_mul(a[r], (r & 1) ? s_r8 : s_r);
           if constexpr (!F16) a[r] = f16x2_to_bf16x2(a[r]);
         }
         mma_m16n8k16<F16>(acc[h], a, e ? xg.z : xg.x, e ? xg.w : xg.y);
@@ -161,14 +173,16 @@ __global__ void dequant_nvfp4_kernel(const uint8_t* packed, long long N, long lo
   const uint8_t* src = packed + chunk * Format<4>::kChunkBytes;
   const uint4 w = *reinterpret_cast<const uint4*>(src + kHalfBytes * h + 16 * slot);
   const uint2 sc = *reinterpret_cast<const uint2*>(src + kCodeBytes + 8 * (2 * gi + (ti >> 1)));
-  const uint32_t sw = h ? sc.y : sc.x;
+  uint32_t s2[2];
+  e4m3x4_to_f16x2(h ? sc.y : sc.x, s2[0], s2[1]);
   for (int j = 0; j < 4; ++j) {
     const int G = j >> 1, e = j & 1;
     const uint32_t word = j == 0 ? w.x : j == 1 ? w.y : j == 2 ? w.z : w.w;
-    const uint32_t s2 = e4m3x2_to_f16x2(sw >> (16 * G));
+    uint32_t c2[4];
+    e2m1x8_to_f16x2(word, c2);
     for (int r = 0; r < 4; ++r) {
-      const uint32_t sel = (r & 1) ? byte_perm(s2, 0x3232u) : byte_perm(s2, 0x1010u);
-      const float2 v = half2_bits_to_float2(f16x2_mul(e2m1x2_to_f16x2(word >> (8 * r)), sel));
+      const uint32_t sel = (r & 1) ? byte_perm(s2[G], 0x3232u) : byte_perm(s2[G], 0x1010u);
+      const float2 v = half2_bits_to_float2(f16x2_mul(c2[r], sel));
       const long long row = tt * kTileRows + 16 * h + gi + 8 * (r & 1);
       const long long col = 64 * c + 32 * G + 8 * ti + 4 * e + 2 * (r >> 1);
       if (row < N) {

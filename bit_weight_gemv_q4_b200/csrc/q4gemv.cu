@@ -599,19 +599,26 @@ void* stack_kernel_ptr() {
   return reinterpret_cast<void*>(&q4k::stack_kernel<M, kStackNW, kStackD, kStackPF>);
 }
 
-template <int M, int SU>
+template <int M, int SU, bool NV>
 void* stream_kernel_ptr() {
-  return reinterpret_cast<void*>(&q4k::stream_kernel<M, kStackNW, kStackD, SU>);
+  return reinterpret_cast<void*>(&q4k::stream_kernel<M, kStackNW, kStackD, SU, NV>);
 }
 
-// su: chunks per stage of the stream-mode kernel (0 = ordered mode)
-void* select_stack_kernel(int M, int su) {
-  static void* const table[3][4] = {
+// su: chunks per stage of the stream-mode kernel (0 = ordered mode); nv: the
+// list holds NVFP4 products
+void* select_stack_kernel(int M, int su, bool nv) {
+  static void* const table[5][4] = {
       {stack_kernel_ptr<1>(), stack_kernel_ptr<2>(), stack_kernel_ptr<3>(), stack_kernel_ptr<4>()},
-      {stream_kernel_ptr<1, 2>(), stream_kernel_ptr<2, 2>(), stream_kernel_ptr<3, 2>(), stream_kernel_ptr<4, 2>()},
-      {stream_kernel_ptr<1, kStreamU>(), stream_kernel_ptr<2, kStreamU>(), stream_kernel_ptr<3, kStreamU>(),
-       stream_kernel_ptr<4, kStreamU>()}};
-  return table[su == 0 ? 0 : (su == 2 ? 1 : 2)][M - 1];
+      {stream_kernel_ptr<1, 2, false>(), stream_kernel_ptr<2, 2, false>(), stream_kernel_ptr<3, 2, false>(),
+       stream_kernel_ptr<4, 2, false>()},
+      {stream_kernel_ptr<1, kStreamU, false>(), stream_kernel_ptr<2, kStreamU, false>(),
+       stream_kernel_ptr<3, kStreamU, false>(), stream_kernel_ptr<4, kStreamU, false>()},
+      {stream_kernel_ptr<1, 2, true>(), stream_kernel_ptr<2, 2, true>(), stream_kernel_ptr<3, 2, true>(),
+       stream_kernel_ptr<4, 2, true>()},
+      {stream_kernel_ptr<1, kStreamU, true>(), stream_kernel_ptr<2, kStreamU, true>(),
+       stream_kernel_ptr<3, kStreamU, true>(), stream_kernel_ptr<4, kStreamU, true>()}};
+  const int row = su == 0 ? 0 : (su == 2 ? 1 : 2) + (nv ? 2 : 0);
+  return table[row][M - 1];
 }
 
 // su: stream mode with stages of su chunks (weights + activation slice of M
@@ -742,7 +749,9 @@ int create_persistent(const q4_stack_entry* entries, int n, int M, int su, const
   if (err == cudaSuccess)
     err = cudaMemcpy(st->entries_dev, host.data(), sizeof(q4k::StackEntryDev) * host.size(), cudaMemcpyHostToDevice);
   if (err != cudaSuccess) return cuda_fail(err, "layer_stack_create: allocation");
-  st->fn = select_stack_kernel(M, su);
+  bool nv = false;
+  for (int i = 0; i < n; ++i) nv = nv || entries[i].bits == Q4_FMT_NVFP4;
+  st->fn = select_stack_kernel(M, su, nv);
   st->smem = stack_smem_bytes(su, M);
   st->block = kStackNW * 32;
   st->grid = dev.sms;

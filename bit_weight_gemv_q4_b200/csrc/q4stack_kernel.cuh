@@ -634,8 +634,10 @@ __device__ __forceinline__ bool stream_segment(const StackParams& sp, const Stac
 }
 
 // SU: chunks per stage and per stream-K block (2 or 4; every product's
-// chunks per tile is a multiple of SU, checked on the host).
-template <int M, int NW, int D, int SU>
+// chunks per tile is a multiple of SU, checked on the host).  NV: the list
+// holds NVFP4 products (their segment is compiled only into this instance,
+// so lists of q4 / q8 products run the code without it).
+template <int M, int NW, int D, int SU, bool NV>
 __global__ void __launch_bounds__(NW * 32, 1) stream_kernel(const StackParams sp) {
   constexpr int SLOT = StreamSlot<SU, M>::kBytes;
   extern __shared__ __align__(128) unsigned char smem[];
@@ -701,7 +703,7 @@ __global__ void __launch_bounds__(NW * 32, 1) stream_kernel(const StackParams sp
     const long long n = in_entry < left ? in_entry : left;
     const XInfo xi = *ep->xinfo;  // written by xprep_kernel, complete once griddepcontrol.wait returned
     scale = xi.ok ? xi.scale : 1.f;
-    if (ep->bits == kFmtNvfp4) {
+    if (NV && ep->bits == kFmtNvfp4) {
       scale *= *reinterpret_cast<const float*>(ep->packed + ep->TC * Format<4>::kChunkBytes);  // t
       ok = xi.ok ? stream_segment<kFmtNvfp4, M, D, SU, true>(sp, ep, e, lb, n, gb, rg, pr, policy, scale, acc, pw,
                                                              e_first, r_first, r, c, lane)

@@ -19,7 +19,10 @@ the sensitive projections and the output head (bs178.com llamAmpere post,
 the symmetric [-8, 7] / [-127, 127] ranges are the plain reading the pages leave
 open; ``layout.py`` decodes the kernel-native packed layout from its written
 specification, and ``quantize.py`` is the offline quantiser (bf16 weights to
-codes and fp16 scales) with every rounding step fixed.
+codes and fp16 scales) with every rounding step fixed.  ``chain.py`` holds the
+steps between the products of a dependent decode chain, ``nvfp4.py`` the NVFP4
+weight format, and ``spec.py`` the MTP draft / verify step (rejection sampling
+over the draft head's mapped vocabulary).
 """
 from __future__ import annotations
 

@@ -23,10 +23,11 @@ INCLUDE = os.path.join(os.path.dirname(HERE), "include")
 GEMV_LIB = os.path.join(HERE, "libq4gemv.so")
 SYNTH_LIB = os.path.join(HERE, "libq4synth.so")
 
-GEMV_SOURCES = [os.path.join(CSRC, "q4gemv.cu"), os.path.join(CSRC, "pack.cpp"), os.path.join(CSRC, "quantize.cu")]
+GEMV_SOURCES = [os.path.join(CSRC, "q4gemv.cu"), os.path.join(CSRC, "pack.cpp"), os.path.join(CSRC, "quantize.cu"),
+                os.path.join(CSRC, "spec.cu")]
 GEMV_DEPS = GEMV_SOURCES + [os.path.join(INCLUDE, "q4gemv.h"), os.path.join(CSRC, "q4gemv_kernels.cuh"),
                             os.path.join(CSRC, "q4stack_kernel.cuh"), os.path.join(CSRC, "q4chain_kernel.cuh"),
-                            os.path.join(CSRC, "q4nvfp4_kernel.cuh")]
+                            os.path.join(CSRC, "q4nvfp4_kernel.cuh"), os.path.join(CSRC, "q4spec_kernel.cuh")]
 SYNTH_SOURCES = [os.path.join(CSRC, "synth.cu")]
 SYNTH_DEPS = SYNTH_SOURCES + [os.path.join(CSRC, "synth_core.h")]
 

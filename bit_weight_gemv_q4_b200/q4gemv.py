@@ -35,6 +35,7 @@ Q4_OP_PRODUCT = 0
 Q4_OP_RESIDUAL_RMSNORM = 1
 Q4_OP_SWIGLU = 2
 Q4_FMT_NVFP4 = 16
+Q4_SPEC_MAX_DRAFT = 15
 
 ERROR_NAMES = {
     Q4_ERR_INVALID_ARG: "INVALID_ARG",
@@ -54,7 +55,7 @@ EXPORTED = [
     "q4_selftest_wait_timeout", "layer_stack_create", "layer_stack_run", "layer_stack_check",
     "layer_stack_launches", "layer_stack_destroy", "q4_quantize", "q4_quantize_device", "layer_chain_create",
     "q4_residual_rmsnorm", "q4_swiglu", "q4_nvfp4_packed_bytes", "q4_pack_nvfp4", "q4_unpack_nvfp4",
-    "q4_pack_nvfp4_device", "q4_nvfp4_dequant_device",
+    "q4_pack_nvfp4_device", "q4_nvfp4_dequant_device", "q4_gather_rows_device", "q4_spec_draft", "q4_spec_verify",
 ]
 
 
@@ -126,6 +127,9 @@ def _load() -> ctypes.CDLL:
         "q4_unpack_nvfp4": ([vp, sz, i64, i64, vp, vp, ctypes.POINTER(ctypes.c_float)], i32),
         "q4_pack_nvfp4_device": ([vp, vp, ctypes.c_float, i64, i64, vp, sz, vp], i32),
         "q4_nvfp4_dequant_device": ([vp, i64, i64, vp, vp], i32),
+        "q4_gather_rows_device": ([vp, i64, i64, vp, i64, vp, vp], i32),
+        "q4_spec_draft": ([vp, i64, vp, ctypes.c_float, vp, vp, vp, vp, vp], i32),
+        "q4_spec_verify": ([vp, i64, vp, i64, vp, vp, vp, i32, ctypes.c_float, vp, vp, vp], i32),
     }
     for name, (args, res) in sig.items():
         f = getattr(L, name)
@@ -244,6 +248,28 @@ def q4_pack_nvfp4_device(codes, scales, tensor_scale: float, N: int, K: int, out
 def q4_nvfp4_dequant_device(packed, N: int, K: int, w_out, stream=None) -> None:
     """Debug decoder: the fp32 weights [N][K] the product kernels multiply."""
     _check(_lib.q4_nvfp4_dequant_device(_dev_ptr(packed), N, K, _dev_ptr(w_out), _stream(stream)))
+
+
+def q4_gather_rows_device(src, row_bytes: int, n_src: int, rows, n_rows: int, dst, stream=None) -> None:
+    """dst row r = src row rows[r] (row_bytes bytes each), device tensors."""
+    _check(_lib.q4_gather_rows_device(_dev_ptr(src), row_bytes, n_src, _dev_ptr(rows), n_rows, _dev_ptr(dst),
+                                      _stream(stream)))
+
+
+def q4_spec_draft(z, n_map: int, vmap, temperature: float, u, row_out, token_out, q_out, stream=None) -> None:
+    """One draft token from the draft head's mapped logits z (device tensors)."""
+    _check(_lib.q4_spec_draft(_dev_ptr(z), n_map, _dev_ptr(vmap), float(temperature), _dev_ptr(u),
+                              _dev_ptr(row_out), _dev_ptr(token_out), _dev_ptr(q_out), _stream(stream)))
+
+
+def q4_spec_verify(target, V: int, drafts, n_map: int, vmap, inv_map, rows, n_draft: int, temperature: float, u,
+                   out, stream=None) -> None:
+    """Keep / reject n_draft drafted tokens against the main model's logits;
+    out (int32, 3 n_draft + 3) receives the kept count, the emitted tokens and
+    the per-position decisions (see include/q4gemv.h)."""
+    opt = lambda t: 0 if t is None else _dev_ptr(t)  # noqa: E731
+    _check(_lib.q4_spec_verify(_dev_ptr(target), V, opt(drafts), n_map, opt(vmap), opt(inv_map), opt(rows), n_draft,
+                               float(temperature), _dev_ptr(u), _dev_ptr(out), _stream(stream)))
 
 
 def q4_quantize(bits: int, mode: int, w_bf16: np.ndarray) -> tuple[np.ndarray, np.ndarray]:
@@ -396,5 +422,6 @@ __all__ = [
     "q4_quantize", "q4_quantize_device", "Q4_QUANT_ABSMAX", "Q4_QUANT_SIGNED_MAX",
     "layer_chain_create", "ChainOp", "Q4_OP_PRODUCT", "Q4_OP_RESIDUAL_RMSNORM", "Q4_OP_SWIGLU",
     "q4_residual_rmsnorm", "q4_swiglu", "Q4_FMT_NVFP4", "q4_nvfp4_packed_bytes", "q4_pack_nvfp4", "q4_unpack_nvfp4",
-    "q4_pack_nvfp4_device", "q4_nvfp4_dequant_device",
+    "q4_pack_nvfp4_device", "q4_nvfp4_dequant_device", "Q4_SPEC_MAX_DRAFT", "q4_gather_rows_device",
+    "q4_spec_draft", "q4_spec_verify",
 ]

@@ -210,6 +210,73 @@ Q4_API int q4_pack_nvfp4_device(const uint8_t* codes, const uint8_t* scales, flo
  * CUDA. */
 Q4_API int q4_nvfp4_dequant_device(const void* packed, int64_t N, int64_t K, float* w_out, void* stream);
 
+/* ---------------------------------------------------------------------------
+ * Speculative decoding around the M = 4 product (MTP draft / verify).  The
+ * bs178.com llamAmpere post ("Why it is this fast", part four) drafts three
+ * tokens with the model's multi-token-prediction head, checks them with one
+ * pass of the main model, and keeps each drafted token with probability
+ * min(1, p/q) (p the main model's probability of the token, q the draft
+ * head's), so the output is distributed as plain generation; the draft head
+ * projects onto a vocabulary map of 65,536 of the ~248K tokens, the main model
+ * onto all of them.  At the first rejected position the emitted token is drawn
+ * from max(0, p - q) normalised; when every draft is kept one more token is
+ * drawn from the main model's next distribution (the standard speculative
+ * sampling step the post's equivalence claim needs).
+ *   dist(l, T) = softmax(l / T) (T > 0), computed in fp32 on the device;
+ *   a draw from weights w with a uniform u in [0, 1) is the first index whose
+ *   running sum exceeds u * sum(w).
+ *   T = 0 is greedy: a draft is kept iff it is the first maximum of the main
+ *   model's logits, and the emitted correction / bonus is that maximum.
+ * The random numbers are inputs (device arrays of uniforms in [0, 1)), so a
+ * step is reproducible and can be captured in a CUDA graph.  Logits may hold
+ * -inf (masked tokens, probability 0); every row needs one finite logit, and
+ * NaN logits give undefined tokens.  Results are bitwise reproducible run to
+ * run (fixed reduction orders).  All pointers are device memory, 4-byte
+ * aligned; calls are asynchronous on `stream`.
+ * -------------------------------------------------------------------------*/
+#define Q4_SPEC_MAX_DRAFT 15
+
+/* Row gather (vocabulary-mapped draft head): dst row r = src row rows[r],
+ * row_bytes bytes each (e.g. canonical q4 codes K/2, q8 codes K, fp16 scales
+ * K/16), for r < n_rows; a rows[r] outside [0, n_src) gives a zero row.  Pack
+ * the gathered codes and scales with q4_pack_weights_device.  Errors: SHAPE,
+ * INVALID_ARG, ALIGN (rows), UNSUPPORTED, CUDA. */
+Q4_API int q4_gather_rows_device(const void* src, int64_t row_bytes, int64_t n_src, const int32_t* rows,
+                                 int64_t n_rows, void* dst, void* stream);
+
+/* One draft token: z fp32 [n_map] (the draft head's logits over the mapped
+ * rows), vmap int32 [n_map] (mapped row -> token id), u [1].  Writes the drawn
+ * mapped row, its token vmap[row] and q = dist(z, T)[row] (1 when greedy).
+ * Errors: SHAPE (n_map < 1), INVALID_ARG (T < 0, NaN or inf; null), ALIGN,
+ * UNSUPPORTED, CUDA. */
+Q4_API int q4_spec_draft(const float* z, int64_t n_map, const int32_t* vmap, float temperature, const float* u,
+                         int32_t* row_out, int32_t* token_out, float* q_out, void* stream);
+
+/* Verify n_draft drafted tokens (0..Q4_SPEC_MAX_DRAFT).
+ *   target  fp32 [n_draft + 1][V]: the main model's logits at the drafted
+ *           positions and the one after them (the M = n_draft + 1 product of
+ *           the output head);
+ *   drafts  fp32 [n_draft][n_map]: the draft head's logits of each draft;
+ *   vmap    int32 [n_map], inv_map int32 [V] (token -> mapped row, -1 if
+ *           unmapped; entries outside [0, n_map) count as unmapped);
+ *   rows    int32 [n_draft]: the drafted mapped rows (from q4_spec_draft);
+ *   u       fp32 [2 n_draft + 1]: keep uniforms, correction uniforms, bonus
+ *           uniform;
+ *   out     int32 [3 n_draft + 3]: out[0] = a, the number of leading drafts
+ *           kept; out[1 .. a] their tokens; out[a + 1] the correction (a <
+ *           n_draft) or bonus token; out[a + 2 .. n_draft + 1] = -1.  Then,
+ *           per position j: out[n_draft + 2 + j] = 1 if draft j passed its
+ *           own test (j < n_draft), and out[2 n_draft + 2 + j] = the draw of
+ *           position j (correction or bonus; -1 where the draft was kept).
+ *           Positions after the first rejection are evaluated too; only the
+ *           first a + 1 tokens are the step's output.
+ * Two launches: one cluster of 8 CTAs per position, then one small kernel.
+ * Errors: INVALID_ARG (n_draft, temperature, null), SHAPE, ALIGN,
+ * UNSUPPORTED, CUDA. */
+Q4_API int q4_spec_verify(const float* target, int64_t V, const float* drafts, int64_t n_map, const int32_t* vmap,
+                          const int32_t* inv_map, const int32_t* rows, int n_draft, float temperature,
+                          const float* u, int32_t* out, void* stream);
+
 /* Bytes of device workspace q4_gemv / q8_gemv need for this shape on the
  * current device.  The workspace holds a status word, the per-warp partial
  * sums of tiles split between warps (a region of fixed size per device) and

@@ -137,3 +137,300 @@ def test_stops_at_the_first_rejection():
 def test_inverse_map():
     inv = OS.inverse_map(np.array([3, 0, 7]), 9)
     assert inv.tolist() == [1, -1, -1, 0, -1, -1, -1, 2, -1]
+
+
+# ---------------------------------------------------------------- device (GPU)
+# fp32 on the device vs fp64 here: a draw or a keep decision may differ only
+# where the oracle's margin to the decision boundary is below the fp32 error
+# bound of the device's sums; elsewhere every integer result must match
+# exactly.  A device running sum at any index is a chain of at most
+# 7 (CTAs) + 31 (warps) + 31 (steps of 32) + 5 (scan levels) = 74 fp32
+# additions of positive terms, so its relative error is below 74 * 2^-24 =
+# 4.4e-6 of the total; expf adds 2 ulp per term.  Hence CDF_TOL = 5e-6 of the
+# total mass for draws from p or q.  A residual weight max(0, p - q) carries
+# the errors of both p and q (each normalised by such a sum): up to 1e-5 of
+# the whole probability mass, plus its own sum's 5e-6 of R.  A keep decision
+# u q < p compares two such quotients: KEEP_TOL = 2e-5 relative.
+CDF_TOL = 5e-6
+KEEP_TOL = 2e-5
+
+
+def _torch():
+    import torch
+
+    return torch
+
+
+def _dev(a, dtype):
+    torch = _torch()
+    return torch.from_numpy(np.ascontiguousarray(a, dtype=dtype)).cuda()
+
+
+def _check_draw(w, u, got, what, tol=None):
+    """got must be a valid inverse-CDF draw of weights w at u (within `tol`,
+    in the units of w; default CDF_TOL of the total), and equal to the
+    oracle's unless u * total lies within tol of a boundary.  Returns whether
+    the exact comparison applied."""
+    w = np.asarray(w, dtype=np.float64)
+    c = np.cumsum(w)
+    total = c[-1]
+    tol = CDF_TOL * total if tol is None else tol
+    t = u * total
+    want = OS.sample(w, u)
+    lo = c[got - 1] if got > 0 else 0.0
+    assert w[got] > 0, f"{what}: drew a zero-weight index {got}"
+    assert lo - tol <= t <= c[got] + tol, f"{what}: {got} is not a valid draw (oracle {want})"
+    lo_w = c[want - 1] if want > 0 else 0.0
+    if min(t - lo_w, c[want] - t) > tol:
+        assert got == want, f"{what}: {got} != oracle {want}"
+        return True
+    return False
+
+
+def _synthetic_map(rng, V, n_map):
+    return np.sort(rng.choice(V, n_map, replace=False)).astype(np.int32)
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("n_map,T", [(65536, 1.0), (65536, 0.6), (1000, 2.0), (37, 1.0), (1, 1.0)])
+def test_draft_parity(cuda_device, n_map, T):
+    import bit_weight_gemv_q4_b200 as q4
+
+    torch = _torch()
+    rng = np.random.default_rng(n_map)
+    V = max(248320, n_map)
+    vmap = _synthetic_map(rng, V, n_map)
+    z = rng.normal(0, 2.0, n_map).astype(np.float32)
+    zd, md = _dev(z, np.float32), _dev(vmap, np.int32)
+    row = torch.empty(1, dtype=torch.int32, device="cuda")
+    tok = torch.empty_like(row)
+    q = torch.empty(1, dtype=torch.float32, device="cuda")
+    qref = OS.dist(z, T)
+    exact = 0
+    for u in list(rng.random(40)) + [0.0, 0.999999]:
+        q4.q4_spec_draft(zd, n_map, md, T, _dev([u], np.float32), row, tok, q)
+        torch.cuda.synchronize()
+        r = int(row.item())
+        exact += _check_draw(qref, float(np.float32(u)), r, f"draft u={u}")
+        assert int(tok.item()) == vmap[r]
+        assert abs(float(q.item()) - qref[r]) <= 1e-4 * qref[r] + 1e-12
+    assert exact >= 25  # of 42: ~80 % of these draws lie farther than CDF_TOL from a boundary
+
+
+@pytest.mark.gpu
+def test_draft_greedy_is_first_maximum(cuda_device):
+    import bit_weight_gemv_q4_b200 as q4
+
+    torch = _torch()
+    n_map = 65536
+    z = np.random.default_rng(3).normal(0, 1, n_map).astype(np.float32)
+    for pos in (0, 12345, 40000, n_map - 1):
+        zz = z.copy()
+        zz[pos] = 10.0
+        zz[(pos + 7777) % n_map] = 10.0  # a tie: the lower index wins
+        vmap = np.arange(n_map, dtype=np.int32) * 3
+        row = torch.empty(1, dtype=torch.int32, device="cuda")
+        tok, q = torch.empty_like(row), torch.empty(1, dtype=torch.float32, device="cuda")
+        q4.q4_spec_draft(_dev(zz, np.float32), n_map, _dev(vmap, np.int32), 0.0, _dev([0.5], np.float32), row, tok, q)
+        torch.cuda.synchronize()
+        want = min(pos, (pos + 7777) % n_map)
+        assert (int(row.item()), int(tok.item()), float(q.item())) == (want, 3 * want, 1.0)
+
+
+def _run_verify(q4, target, drafts, vmap, rows, u, T, V):
+    torch = _torch()
+    n = len(rows)
+    inv = OS.inverse_map(vmap, V)
+    out = torch.full((3 * n + 3,), -7, dtype=torch.int32, device="cuda")
+    q4.q4_spec_verify(_dev(target, np.float32), V, _dev(drafts, np.float32) if n else None, len(vmap),
+                      _dev(vmap, np.int32), _dev(inv, np.int32), _dev(rows, np.int32) if n else None, n, T,
+                      _dev(u, np.float32), out)
+    torch.cuda.synchronize()
+    return out.cpu().numpy()
+
+
+def _check_verify(target, drafts, vmap, rows, u, T, out):
+    """Per position: the keep decision (exact unless within KEEP_TOL of the
+    boundary) and the draw (a valid draw, exact away from boundaries); then
+    the assembled output from the per-position results."""
+    n, V = len(rows), target.shape[1]
+    t64 = target.astype(np.float64)
+    keep = out[n + 2: 2 * n + 2]
+    draw = out[2 * n + 2: 3 * n + 3]
+    exact, n_exact, n_checks = True, 0, 0
+    for j in range(n):
+        d = int(vmap[rows[j]])
+        p = OS.dist(t64[j], T)
+        q = np.zeros(V)
+        q[vmap] = OS.dist(drafts[j].astype(np.float64), T)
+        uq, pd = float(np.float32(u[j])) * q[d], p[d]
+        want = uq < pd
+        n_checks += 1
+        if abs(uq - pd) > KEEP_TOL * max(uq, pd):
+            assert bool(keep[j]) == want, f"position {j}: keep {keep[j]} vs oracle {want} (u q = {uq}, p = {pd})"
+            n_exact += 1
+        else:
+            exact = False
+        if keep[j]:
+            assert draw[j] == -1
+        else:
+            r = np.maximum(p - q, 0.0)
+            if r.sum() > 0:
+                e = _check_draw(r, float(np.float32(u[n + j])), int(draw[j]), f"correction {j}",
+                                tol=1e-5 + CDF_TOL * r.sum())
+            else:
+                e = _check_draw(p, float(np.float32(u[n + j])), int(draw[j]), f"correction {j}")
+            exact &= e
+            n_exact += e
+            n_checks += 1
+    e = _check_draw(OS.dist(t64[n], T), float(np.float32(u[2 * n])), int(draw[n]), "bonus")
+    exact &= e
+    n_exact += e
+    n_checks += 1
+    a = 0
+    while a < n and keep[a]:
+        a += 1
+    assert out[0] == a
+    assert list(out[1: a + 1]) == [int(vmap[r]) for r in rows[:a]]
+    assert out[a + 1] == draw[a] and all(out[a + 2: n + 2] == -1)
+    if exact:  # no boundary case anywhere: the whole step equals the oracle's
+        a_ref, toks = OS.verify(t64, drafts, vmap, rows, np.float32(u).astype(np.float64), T)
+        assert a_ref == a and toks == list(out[1: a + 2])
+    return n_exact, n_checks
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("T", [1.0, 1.7])
+def test_verify_parity_full_vocabulary(cuda_device, T):
+    """V = 248,320, a synthetic map of 65,536 tokens, three drafts whose
+    logits follow the target's with noise (so p/q spans both sides of 1)."""
+    import bit_weight_gemv_q4_b200 as q4
+
+    rng = np.random.default_rng(int(T * 10))
+    V, n_map, n = 248320, 65536, 3
+    vmap = _synthetic_map(rng, V, n_map)
+    n_exact = n_checks = 0
+    for trial in range(12):
+        target = rng.normal(0, 3.0, (n + 1, V)).astype(np.float32)
+        target[:, vmap] += 2.0  # the mapped tokens carry most of the mass
+        drafts = (target[:n][:, vmap] + rng.normal(0, 0.7, (n, n_map))).astype(np.float32)
+        rows = np.array([OS.draft(drafts[j].astype(np.float64), vmap, T, rng.random())[1] for j in range(n)],
+                        dtype=np.int32)
+        u = rng.random(2 * n + 1).astype(np.float32)
+        out = _run_verify(q4, target, drafts, vmap, rows, u, T, V)
+        e, c = _check_verify(target, drafts, vmap, rows, u, T, out)
+        n_exact, n_checks = n_exact + e, n_checks + c
+        out2 = _run_verify(q4, target, drafts, vmap, rows, u, T, V)
+        assert np.array_equal(out, out2)  # bitwise reproducible
+    assert n_exact >= 0.6 * n_checks
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("V,n_map,n", [(100, 10, 1), (1000, 1000, 3), (5000, 64, 15), (70, 3, 0), (1, 1, 2)])
+def test_verify_small_and_edge_shapes(cuda_device, V, n_map, n):
+    """Vocabularies smaller than a cluster's warps (empty slices), the
+    identity map, the most drafts, no draft (a plain draw), one token."""
+    import bit_weight_gemv_q4_b200 as q4
+
+    rng = np.random.default_rng(V + n)
+    vmap = _synthetic_map(rng, V, n_map)
+    for trial in range(6):
+        target = rng.normal(0, 1.5, (n + 1, V)).astype(np.float32)
+        drafts = (target[:n][:, vmap] + rng.normal(0, 0.5, (n, n_map))).astype(np.float32)
+        rows = np.array([OS.draft(drafts[j].astype(np.float64), vmap, 1.0, rng.random())[1] for j in range(n)],
+                        dtype=np.int32)
+        u = rng.random(2 * n + 1).astype(np.float32)
+        out = _run_verify(q4, target, drafts, vmap, rows, u, 1.0, V)
+        _check_verify(target, drafts, vmap, rows, u, 1.0, out)
+
+
+@pytest.mark.gpu
+def test_verify_greedy_exact(cuda_device):
+    import bit_weight_gemv_q4_b200 as q4
+
+    rng = np.random.default_rng(17)
+    V, n_map, n = 248320, 65536, 3
+    vmap = _synthetic_map(rng, V, n_map)
+    for trial in range(8):
+        target = rng.normal(0, 1, (n + 1, V)).astype(np.float32)
+        rows = rng.integers(0, n_map, n).astype(np.int32)
+        for j in range(n):
+            if rng.random() < 0.7:  # this draft is the target's maximum (with a tie after it)
+                target[j, vmap[rows[j]]] = 9.0
+                target[j, V - 1 - j] = 9.0 if vmap[rows[j]] < V - 1 - j else 0.0
+        drafts = rng.normal(0, 1, (n, n_map)).astype(np.float32)
+        out = _run_verify(q4, target, drafts, vmap, rows, np.zeros(2 * n + 1, np.float32), 0.0, V)
+        a, toks = OS.verify(target.astype(np.float64), drafts, vmap, rows, np.zeros(2 * n + 1), 0.0)
+        assert out[0] == a and list(out[1: a + 2]) == toks
+
+
+@pytest.mark.gpu
+def test_verify_keeps_every_draft_of_an_exact_draft_head(cuda_device):
+    import bit_weight_gemv_q4_b200 as q4
+
+    rng = np.random.default_rng(23)
+    V, n = 4096, 3
+    vmap = np.arange(V, dtype=np.int32)
+    target = rng.normal(0, 2, (n + 1, V)).astype(np.float32)
+    for trial in range(6):
+        rows = np.array([OS.draft(target[j].astype(np.float64), vmap, 1.0, rng.random())[1] for j in range(n)],
+                        dtype=np.int32)
+        u = (rng.random(2 * n + 1) * 0.99).astype(np.float32)
+        out = _run_verify(q4, target, target[:n], vmap, rows, u, 1.0, V)
+        assert out[0] == n and list(out[1: n + 1]) == list(rows)
+        _check_draw(OS.dist(target[n].astype(np.float64), 1.0), float(u[2 * n]), int(out[n + 1]), "bonus")
+
+
+@pytest.mark.gpu
+def test_masked_tokens_are_never_emitted(cuda_device):
+    import bit_weight_gemv_q4_b200 as q4
+
+    rng = np.random.default_rng(29)
+    V, n_map, n = 20000, 2000, 2
+    vmap = _synthetic_map(rng, V, n_map)
+    for trial in range(10):
+        target = rng.normal(0, 1, (n + 1, V)).astype(np.float32)
+        mask = rng.random(V) < 0.5
+        target[:, mask] = -np.inf
+        drafts = rng.normal(0, 1, (n, n_map)).astype(np.float32)
+        rows = rng.integers(0, n_map, n).astype(np.int32)
+        u = rng.random(2 * n + 1).astype(np.float32)
+        out = _run_verify(q4, target, drafts, vmap, rows, u, 1.0, V)
+        a = out[0]
+        for t in out[1: a + 2]:
+            assert not mask[t]
+        _check_verify(target, drafts, vmap, rows, u, 1.0, out)
+
+
+@pytest.mark.gpu
+def test_mapped_draft_head_by_row_gather(cuda_device):
+    """The vocabulary-mapped draft head: gather the mapped rows of the q8
+    head's canonical codes and scales on the device, pack them, and its
+    product equals the oracle's product of those rows."""
+    import bit_weight_gemv_q4_b200 as q4
+    import gpu_helpers as H
+    from bit_weight_gemv_q4_b200 import synth
+
+    torch = _torch()
+    N, K, n_map = 6000, 1024, 1000
+    rng = np.random.default_rng(31)
+    vmap = _synthetic_map(rng, N, n_map)
+    qh, sh = synth.tensor(8, 2, 77, N, K)
+    rows_bad = np.concatenate([vmap, [-1, N]]).astype(np.int32)  # two rows out of range: zero rows
+    qd, sd = _dev(qh.view(np.uint8), np.uint8), _dev(sh.view(np.uint16).view(np.int16), np.int16)
+    gq = torch.empty((n_map + 2) * K, dtype=torch.uint8, device="cuda")
+    gs = torch.empty((n_map + 2) * (K // 32), dtype=torch.int16, device="cuda")
+    rd = _dev(rows_bad, np.int32)
+    q4.q4_gather_rows_device(qd, K, N, rd, n_map + 2, gq)
+    q4.q4_gather_rows_device(sd, 2 * (K // 32), N, rd, n_map + 2, gs)
+    torch.cuda.synchronize()
+    gqn = gq.cpu().numpy().reshape(n_map + 2, K)
+    gsn = gs.cpu().numpy().view(np.uint16).reshape(n_map + 2, K // 32)
+    assert np.array_equal(gqn[:n_map], qh.view(np.uint8)[vmap]) and np.array_equal(gsn[:n_map], sh[vmap])
+    assert not gqn[n_map:].any() and not gsn[n_map:].any()
+    packed = torch.empty(q4.q4_packed_bytes(8, n_map, K), dtype=torch.uint8, device="cuda")
+    q4.q4_pack_weights_device(8, gq[: n_map * K], gs[: n_map * (K // 32)], n_map, K, packed)
+    x = synth.activations(2, synth.act_stream(5), 1, K)
+    y, ok = H.run_gemv(8, packed, n_map, K, H.to_device_x(x), 1)
+    assert ok
+    H.assert_parity(y, qh[vmap], sh[vmap], x, 8)

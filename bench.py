@@ -14,7 +14,9 @@ through the public API ("e2e"), the roofline of the dominant kernel, the CPU
 oracle's rate ("cpu_baseline"), the SM clock under load, "chain" (the same
 products as a dependent chain with the residual + RMSNorm and SwiGLU steps
 between them, M = 1 and 4), "nvfp4" (the same stream with its 4-bit tensors
-in NVFP4, the same bytes, M = 1 and 4), and "per_config":
+in NVFP4, the same bytes, M = 1 and 4), "spec" (one MTP speculative step:
+three mapped-vocabulary drafts, the M = 4 pass and the keep / reject step),
+and "per_config":
 microseconds per product of the single-tensor configurations (q4 4096 x 4096,
 each projection of one layer at M = 1 and 4, the q8 vocabulary heads).
 
@@ -323,6 +325,51 @@ def per_config(args, d: Dist, torch, q4, workloads, peak):
     return res
 
 
+def spec_step(args, d: Dist, torch, q4, workloads, stream, peak):
+    """One MTP speculative step (3 drafts): each draft is the mapped draft
+    head's product (65,536 x 5120 q8, M = 1) and a draw; then the decode
+    stream at M = 4 and the keep / reject kernels.  Device time of the step
+    and of its parts.  How many tokens a step yields depends on how often the
+    drafts are kept, which needs trained weights; the step emits 1 to 4."""
+    sp = workloads.DeviceSpec(seed=args.seed, temperature=1.0)
+    n_it = max(3, args.steps // 4)
+
+    def timed(fn, n):
+        for _ in range(3):
+            fn()
+        return d.max(time_region(torch, fn, n, stream) / n)
+
+    ms_step = timed(sp.run, n_it)
+    ms_head = timed(lambda: q4.layer_stack_run(sp.draft_stacks[0]), 4 * n_it)
+    ms_draft = timed(lambda: sp.draft(0), 4 * n_it)
+    ms_pass = timed(sp.verify_stream.run, n_it)
+    ms_verify = timed(sp.verify, 4 * n_it)
+    sp.check()
+    head_bytes = workloads.weight_bytes(8, sp.n_map, sp.K)
+    step_bytes = sp.verify_stream.weight_bytes + sp.n * head_bytes
+    # bytes the keep / reject kernels read: the target logits, the draft
+    # logits and the inverse map (their floor; the kernels re-read from L2)
+    verify_bytes = 4 * ((sp.n + 1) * sp.V + sp.n * sp.n_map + sp.V)
+    out = {
+        "drafts": sp.n, "vocab": sp.V, "mapped_vocab": sp.n_map, "temperature": sp.T,
+        "step_ms": round(ms_step, 5),
+        "step_weight_bytes": step_bytes,
+        "step_GBps": round(step_bytes / (ms_step * 1e6), 1),
+        "pct_of_hbm_peak": round(100 * step_bytes / (ms_step * 1e6) / peak, 2),
+        "draft_head_us": round(ms_head * 1e3, 2),
+        "draft_head_GBps": round(head_bytes / (ms_head * 1e6), 1),
+        "draft_draw_us": round((ms_draft - ms_head) * 1e3, 2),
+        "verify_pass_ms": round(ms_pass, 5),
+        "verify_us": round(ms_verify * 1e3, 2),
+        "verify_bytes": verify_bytes,
+        "launches_per_step": sp.n * 3 + sp.verify_stream.stack.launches() + 2,
+    }
+    sp.close()
+    del sp
+    torch.cuda.empty_cache()
+    return out
+
+
 def quantize_rates(args, d: Dist, torch, q4, peak):
     """The offline quantiser on the device: bf16 weights of a gate|up-sized
     tensor (q4) and of the full vocabulary head (q8) to codes and scales; GB/s
@@ -472,6 +519,8 @@ def run_ours(args, d: Dist):
         del ch
         torch.cuda.empty_cache()
 
+    spec = spec_step(args, d, torch, q4, workloads, stream, peak)
+
     configs = None if args.no_configs else per_config(args, d, torch, q4, workloads, peak)
 
     cpu = None
@@ -540,6 +589,7 @@ def run_ours(args, d: Dist):
         },
         "chain": chain,
         "nvfp4": nvfp4,
+        "spec": spec,
         "per_config": configs,
         "gpu_launches": n_launch * args.steps,
         "clocks": clocks,
@@ -607,12 +657,37 @@ def run_profile_case(args):
     larger than L2), `--profile-launches` launches at M = args.m.  With
     --profile-layers L: the first L layers of the decode stream (about 0.2 GB
     per layer) as one stream-mode stack launch; --profile-nvfp4 puts their
-    4-bit tensors in NVFP4."""
+    4-bit tensors in NVFP4.  --profile-spec: the keep / reject kernels of a
+    speculative step on seeded logits."""
     import torch
 
     import bit_weight_gemv_q4_b200 as q4
     from bit_weight_gemv_q4_b200 import workloads
 
+    if args.profile_spec:
+        # the keep / reject kernels alone on seeded logits (248,320 vocabulary,
+        # 65,536 mapped, 3 drafts); drafts follow the target with noise
+        import numpy as np
+
+        rng = np.random.default_rng(args.seed)
+        V, n = workloads.VOCAB, workloads.SPEC_DRAFTS
+        vmap = workloads.vocab_map(args.seed, V)
+        n_map = len(vmap)
+        target = rng.normal(0, 3.0, (n + 1, V)).astype(np.float32)
+        drafts = (target[:n][:, vmap] + rng.normal(0, 0.7, (n, n_map))).astype(np.float32)
+        inv = np.full(V, -1, dtype=np.int32)
+        inv[vmap] = np.arange(n_map, dtype=np.int32)
+        dev = lambda a: torch.from_numpy(np.ascontiguousarray(a)).cuda()  # noqa: E731
+        td, zd, md, invd = dev(target), dev(drafts), dev(vmap), dev(inv)
+        rows = dev(rng.integers(0, n_map, n).astype(np.int32))
+        u = dev(workloads.spec_uniforms(args.seed, 2 * n + 1))
+        out = torch.zeros(3 * n + 3, dtype=torch.int32, device="cuda")
+        for _ in range(args.profile_launches):
+            q4.q4_spec_verify(td, V, zd, n_map, md, invd, rows, n, 1.0, u, out)
+        torch.cuda.synchronize()
+        print(json.dumps({"profile_case": "spec verify", "V": V, "n_map": n_map, "drafts": n,
+                          "launches": args.profile_launches, "out": out.cpu().tolist()}))
+        return
     if args.profile_layers > 0:
         tensors = workloads.decode_stream(fused=True)[: 4 * args.profile_layers]
         if args.profile_nvfp4:
@@ -656,6 +731,7 @@ def main():
     ap.add_argument("--profile-launches", type=int, default=3)
     ap.add_argument("--profile-layers", type=int, default=0)
     ap.add_argument("--profile-nvfp4", action="store_true")
+    ap.add_argument("--profile-spec", action="store_true", help="profile case: the keep / reject kernels")
     ap.add_argument("--m", type=int, default=1)
     args = ap.parse_args()
     if args.warmup < 3 and not args.profile_case:

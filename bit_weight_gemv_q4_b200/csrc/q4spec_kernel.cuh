@@ -7,13 +7,16 @@
 //
 // One thread-block cluster of kSpecCtas CTAs per logits row: each CTA takes a
 // contiguous slice of the row, and the CTAs exchange their partial maxima,
-// sums and running totals through distributed shared memory, so every
-// reduction has one fixed order (results are bitwise reproducible) and no
-// global atomics or zero-filled workspace are needed.  Within a CTA each warp
-// takes a contiguous sub-slice and walks it in steps of 32 values; a step's
-// sum is a fixed shuffle tree, the warp's running sum adds the steps in order.
-// A draw finds the CTA, then the warp, then the step, then the lane whose
-// running sum first exceeds u * total, re-walking only that warp's sub-slice.
+// sums and totals through distributed shared memory, so every reduction has
+// one fixed order (results are bitwise reproducible) and no global atomics or
+// zero-filled workspace are needed.  A CTA walks its slice in tiles of
+// kSpecTile values; in a tile thread t sums the kSpecRun consecutive values
+// at kSpecRun * t sequentially (the warp reads one contiguous kilobyte), and a
+// block scan of those sums (in thread order) gives each thread its range
+// [lower, upper) of the tile's running total, consecutive threads sharing a
+// bound, so the ranges tile the tile's total without gaps.  Tiles add up in
+// order.  A draw finds the CTA, then the tile, then the thread whose range
+// holds u * total, and that thread walks its run.
 #pragma once
 
 #include <cooperative_groups.h>
@@ -23,87 +26,45 @@ namespace q4k {
 
 namespace cg = cooperative_groups;
 
-constexpr int kSpecCtas = 8;        // CTAs per cluster (one cluster per logits row)
+// Tunables (measured on B200 for a 248,320-token row: runs of 8 beat runs
+// of 16 by ~30 %; 16-CTA clusters, above the portable size, saved ~12 % on
+// the verify kernel and cost ~25 % on the draft kernel).
+#ifndef Q4_TUNE_SPEC_CTAS
+#define Q4_TUNE_SPEC_CTAS 8
+#endif
+#ifndef Q4_TUNE_SPEC_RUN
+#define Q4_TUNE_SPEC_RUN 8
+#endif
+constexpr int kSpecCtas = Q4_TUNE_SPEC_CTAS;  // CTAs per cluster (one cluster per logits row)
 constexpr int kSpecThreads = 1024;  // 32 warps per CTA
 constexpr int kSpecWarps = kSpecThreads / 32;
-constexpr int kSpecUnroll = 8;      // steps of 32 values loaded ahead
+constexpr int kSpecUnroll = 8;      // loads in flight per thread in the strided max pass
+constexpr int kSpecRun = Q4_TUNE_SPEC_RUN;  // consecutive values a thread sums in a tile
+constexpr int kSpecMaxTiles = 64;   // tile totals a CTA keeps for its draw (more: recomputed)
+constexpr int kSpecTile = kSpecRun * kSpecThreads;
 constexpr unsigned kFull = 0xFFFFFFFFu;
 
-// The slice of a row of n values that CTA `rank` takes, and warp w's part of
-// it (a multiple of 32 values, so the steps of every warp start aligned).
+// The slice of a row of n values that CTA `rank` takes.
 struct SpecSlice {
-  long long lo, hi;  // CTA slice
-  long long per_warp;
+  long long lo, hi;
   __device__ SpecSlice(long long n, int rank) {
     const long long per = (n + kSpecCtas - 1) / kSpecCtas;
     lo = rank * per < n ? rank * per : n;
     hi = lo + per < n ? lo + per : n;
-    per_warp = ((hi - lo + kSpecWarps - 1) / kSpecWarps + 31) / 32 * 32;
   }
-  __device__ long long wlo(int w) const { return lo + w * per_warp < hi ? lo + w * per_warp : hi; }
-  __device__ long long whi(int w) const { return lo + (w + 1) * per_warp < hi ? lo + (w + 1) * per_warp : hi; }
 };
 
-// Sum of a warp's 32 values by a fixed tree, the same in every lane.
-__device__ __forceinline__ float warp_tree_sum(float v) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v += __shfl_down_sync(kFull, v, o);
-  return __shfl_sync(kFull, v, 0);
-}
-
-// The running sum of weight(v) over [lo, hi) in steps of 32 (every lane
-// returns it).
+// This thread's run in the tile starting at tb: the weights (0 past hi) and
+// their sequential sum.
 template <class W>
-__device__ __forceinline__ float warp_walk_sum(long long lo, long long hi, const W& weight, int lane) {
-  float run = 0.f;
-  for (long long base = lo; base < hi; base += 32 * kSpecUnroll) {
-    float w[kSpecUnroll];
+__device__ __forceinline__ float run_weights(long long tb, long long hi, const W& weight, float (&w)[kSpecRun]) {
+  const long long a = tb + static_cast<long long>(kSpecRun) * threadIdx.x;
 #pragma unroll
-    for (int k = 0; k < kSpecUnroll; ++k) {
-      const long long v = base + 32 * k + lane;
-      w[k] = v < hi ? weight(v) : 0.f;
-    }
+  for (int k = 0; k < kSpecRun; ++k) w[k] = a + k < hi ? weight(a + k) : 0.f;
+  float s = 0.f;
 #pragma unroll
-    for (int k = 0; k < kSpecUnroll; ++k) run += warp_tree_sum(w[k]);
-  }
-  return run;
-}
-
-// The first v in [lo, hi) where the warp's running sum (as warp_walk_sum
-// forms it) exceeds t; if rounding leaves none, the last v with a positive
-// weight; -1 if all weights are zero.
-template <class W>
-__device__ __forceinline__ long long warp_walk_find(long long lo, long long hi, const W& weight, float t, int lane) {
-  float run = 0.f;
-  long long last_pos = -1;
-  for (long long base = lo; base < hi; base += 32 * kSpecUnroll) {
-    float w[kSpecUnroll];
-#pragma unroll
-    for (int k = 0; k < kSpecUnroll; ++k) {
-      const long long v = base + 32 * k + lane;
-      w[k] = v < hi ? weight(v) : 0.f;
-    }
-#pragma unroll
-    for (int k = 0; k < kSpecUnroll; ++k) {
-      const float step = warp_tree_sum(w[k]);
-      const unsigned pos = __ballot_sync(kFull, w[k] > 0.f);
-      if (pos) last_pos = base + 32 * k + 31 - __clz(pos);
-      if (run + step > t) {
-        // inclusive scan of the step's 32 weights, in lane order
-        float s = w[k];
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-          const float y = __shfl_up_sync(kFull, s, o);
-          if (lane >= o) s += y;
-        }
-        const unsigned hit = __ballot_sync(kFull, run + s > t && w[k] > 0.f);
-        if (hit) return base + 32 * k + __ffs(hit) - 1;
-        return last_pos;  // t fell in the step's rounding gap
-      }
-      run += step;
-    }
-  }
-  return last_pos;
+  for (int k = 0; k < kSpecRun; ++k) s += w[k];
+  return s;
 }
 
 // Per-CTA values exchanged through distributed shared memory.
@@ -114,10 +75,13 @@ struct SpecXch {
 
 struct SpecShared {
   SpecXch x;
-  float warp_p[kSpecWarps];  // warps' running totals of exp((l - max) / T)
-  float warp_r[kSpecWarps];  // warps' running totals of the residual weights
   float red[kSpecWarps];
   int redi[kSpecWarps];
+  float woff[kSpecWarps + 1];  // warps' offsets in a block scan, then the block total
+  float tiles_p[kSpecMaxTiles];  // tile totals of exp((l - max) / T)
+  float tiles_r[kSpecMaxTiles];  // tile totals of the residual weights
+  int found;
+  long long found_index;
 };
 
 __device__ __forceinline__ float block_max(float v, SpecShared& sh) {
@@ -127,8 +91,9 @@ __device__ __forceinline__ float block_max(float v, SpecShared& sh) {
   __syncthreads();
   if (lane == 0) sh.red[warp] = v;
   __syncthreads();
-  float m = sh.red[0];
-  for (int w = 1; w < kSpecWarps; ++w) m = fmaxf(m, sh.red[w]);
+  float m = sh.red[lane];  // every warp reduces the 32 warp maxima
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(kFull, m, o));
   return m;
 }
 
@@ -150,34 +115,158 @@ __device__ __forceinline__ void block_argmax(float& v, int& i, SpecShared& sh) {
     sh.redi[warp] = i;
   }
   __syncthreads();
-  v = sh.red[0];
-  i = sh.redi[0];
-  for (int w = 1; w < kSpecWarps; ++w)
-    if (sh.red[w] > v || (sh.red[w] == v && sh.redi[w] < i)) {
-      v = sh.red[w];
-      i = sh.redi[w];
+  v = sh.red[lane];  // every warp reduces the 32 warp results
+  i = sh.redi[lane];
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    const float v2 = __shfl_xor_sync(kFull, v, o);
+    const int i2 = __shfl_xor_sync(kFull, i, o);
+    if (v2 > v || (v2 == v && i2 < i)) {
+      v = v2;
+      i = i2;
     }
+  }
 }
 
-// Warp totals of a walk -> the CTA total (warps in order); each warp's total
-// is stored in `tot`.
-__device__ __forceinline__ float block_walk_total(float warp_total, float* tot) {
+// This thread's range [lower, upper) of the block's running total of the
+// threads' sums s, in thread order (an inclusive warp scan, warp offsets
+// added in warp order).  upper of thread i is bitwise lower of thread i + 1.
+// Returns the block total.
+struct SpecRange {
+  float lower, upper;
+};
+__device__ __forceinline__ float block_scan(float s, SpecRange& r, SpecShared& sh) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  float incl = s;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const float y = __shfl_up_sync(kFull, incl, o);
+    if (lane >= o) incl += y;
+  }
+  const float excl = __shfl_up_sync(kFull, incl, 1);
   __syncthreads();
-  if (lane == 0) tot[warp] = warp_total;
+  if (lane == 31) sh.red[warp] = incl;
   __syncthreads();
-  float s = 0.f;
-  for (int w = 0; w < kSpecWarps; ++w) s += tot[w];
-  return s;
+  if (warp == 0) {  // the warps' offsets: an inclusive scan of their totals, in warp order
+    const float t = sh.red[lane];
+    float x = t;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const float y = __shfl_up_sync(kFull, x, o);
+      if (lane >= o) x += y;
+    }
+    const float before = __shfl_up_sync(kFull, x, 1);
+    sh.woff[lane] = lane == 0 ? 0.f : before;
+    if (lane == 31) sh.woff[kSpecWarps] = x;
+  }
+  __syncthreads();
+  r.lower = lane == 0 ? sh.woff[warp] : sh.woff[warp] + excl;
+  r.upper = lane == 31 ? sh.woff[warp + 1] : sh.woff[warp] + incl;
+  return sh.woff[kSpecWarps];
+}
+
+// In a tile whose thread ranges r hold t (relative to the tile's start): the
+// thread whose range holds t (if rounding leaves none, the last non-empty
+// thread) walks its run.  Every thread returns the index.
+__device__ __forceinline__ long long tile_find(long long tb, const float (&w)[kSpecRun], const SpecRange& r, float t,
+                                               SpecShared& sh) {
+  const bool nonempty = r.upper > r.lower;
+  if (threadIdx.x == 0) sh.found = -1;
+  __syncthreads();
+  if (nonempty && r.lower <= t && t < r.upper) atomicMax(&sh.found, kSpecThreads + static_cast<int>(threadIdx.x));
+  __syncthreads();
+  if (sh.found < kSpecThreads && nonempty) atomicMax(&sh.found, static_cast<int>(threadIdx.x));
+  __syncthreads();
+  const int f = sh.found;
+  const int owner = f >= kSpecThreads ? f - kSpecThreads : f;
+  if (static_cast<int>(threadIdx.x) == owner) {
+    const long long a = tb + static_cast<long long>(kSpecRun) * threadIdx.x;
+    long long idx = -1;
+    float run = r.lower;
+#pragma unroll
+    for (int k = 0; k < kSpecRun; ++k) {
+      if (w[k] > 0.f && idx < 0) {
+        if (run + w[k] > t) idx = a + k;
+      }
+      run += w[k];
+    }
+    if (idx < 0)  // rounding gap: the run's last positive weight
+      for (int k = kSpecRun - 1; k >= 0 && idx < 0; --k)
+        if (w[k] > 0.f) idx = a + k;
+    sh.found_index = idx;
+  }
+  __syncthreads();
+  const long long res = sh.found_index;
+  __syncthreads();
+  return res;
+}
+
+// The total of weight over the CTA slice: tiles in order, each tile's total
+// from the block scan of its threads' run sums.  The first kSpecMaxTiles tile
+// totals are kept in `tiles` (if given) for slice_find.
+template <class W>
+__device__ float slice_total(const SpecSlice& sl, const W& weight, SpecShared& sh, float* tiles) {
+  float total = 0.f;
+  int k = 0;
+  for (long long tb = sl.lo; tb < sl.hi; tb += kSpecTile, ++k) {
+    float w[kSpecRun];
+    SpecRange r;
+    const float tt = block_scan(run_weights(tb, sl.hi, weight, w), r, sh);
+    if (tiles && k < kSpecMaxTiles && threadIdx.x == 0) tiles[k] = tt;
+    total += tt;
+  }
+  return total;
+}
+
+// The first index of the CTA slice whose running total (tiles in order, then
+// threads, then the run) exceeds t, with the same sums as slice_total; if
+// rounding leaves none, the last index with a positive weight.  With the
+// tile totals kept by slice_total only the chosen tile is recomputed.  Every
+// thread returns it.
+template <class W>
+__device__ long long slice_find(const SpecSlice& sl, const W& weight, float t, SpecShared& sh, const float* tiles) {
+  const long long ntiles = (sl.hi - sl.lo + kSpecTile - 1) / kSpecTile;
+  float run = 0.f;
+  long long sel = -1, last = -1;
+  float t_sel = INFINITY;
+  if (tiles && ntiles <= kSpecMaxTiles) {
+    for (int k = 0; k < ntiles; ++k) {
+      const float tt = tiles[k];
+      if (tt > 0.f) last = k;
+      if (tt > 0.f && run + tt > t) {
+        sel = k;
+        t_sel = t - run;
+        break;
+      }
+      run += tt;
+    }
+  } else {
+    for (long long tb = sl.lo; tb < sl.hi; tb += kSpecTile) {
+      float w[kSpecRun];
+      SpecRange r;
+      const float tt = block_scan(run_weights(tb, sl.hi, weight, w), r, sh);
+      const long long k = (tb - sl.lo) / kSpecTile;
+      if (tt > 0.f) last = k;
+      if (tt > 0.f && run + tt > t) return tile_find(tb, w, r, t - run, sh);
+      run += tt;
+    }
+  }
+  if (sel < 0) sel = last;  // t beyond the slice (rounding): its last positive weight
+  if (sel < 0) return -1;
+  const long long tb = sl.lo + sel * kSpecTile;
+  float w[kSpecRun];
+  SpecRange r;
+  block_scan(run_weights(tb, sl.hi, weight, w), r, sh);
+  return tile_find(tb, w, r, t_sel, sh);
 }
 
 // The draw of one row: the first index whose running total (CTAs in rank
-// order, then warps, then steps, then lanes) exceeds u * total.  cta_tot[c]
-// are the CTAs' totals (the same array in every CTA), warp_tot this CTA's
-// warps' totals.  Returns the index in the CTA that holds it, -1 elsewhere.
+// order, then the CTA's own order) exceeds u * total.  cta_tot[c]: the CTAs'
+// totals (the same array in every CTA).  Returns the index in the CTA that
+// holds it, -1 in the others.
 template <class W>
-__device__ long long cluster_draw(const float* cta_tot, const float* warp_tot, const SpecSlice& sl, int rank, float u,
-                                  const W& weight) {
+__device__ long long cluster_draw(const float* cta_tot, const SpecSlice& sl, int rank, float u, const W& weight,
+                                  SpecShared& sh, const float* tiles) {
   float total = 0.f;
   for (int c = 0; c < kSpecCtas; ++c) total += cta_tot[c];
   const float t = u * total;
@@ -195,29 +284,7 @@ __device__ long long cluster_draw(const float* cta_tot, const float* warp_tot, c
     for (int c = 0; c < last; ++c) run += cta_tot[c];
   }
   if (cta != rank) return -1;
-  float t_in = t - run;
-  // the warp, likewise
-  float wrun = 0.f;
-  int wsel = -1, wlast = -1;
-  for (int w = 0; w < kSpecWarps; ++w) {
-    if (warp_tot[w] > 0.f) wlast = w;
-    if (wsel < 0 && warp_tot[w] > 0.f && wrun + warp_tot[w] > t_in) wsel = w;
-    if (wsel < 0) wrun += warp_tot[w];
-  }
-  if (wsel < 0) {
-    wsel = wlast;
-    wrun = 0.f;
-    for (int w = 0; w < wlast; ++w) wrun += warp_tot[w];
-  }
-  if (wsel < 0) return -1;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  __shared__ long long s_found;
-  if (warp == wsel) {
-    const long long v = warp_walk_find(sl.wlo(warp), sl.whi(warp), weight, t_in - wrun, lane);
-    if (lane == 0) s_found = v;
-  }
-  __syncthreads();
-  return s_found;
+  return slice_find(sl, weight, t - run, sh, tiles);
 }
 
 // Reads field F of every CTA's exchange record, in rank order.
@@ -238,23 +305,39 @@ struct SpecDraftParams {
   float* q_out;
 };
 
+// (max, first index of the max) of a[v] over this thread's share of the CTA
+// slice: strided by the block (coalesced loads, kSpecUnroll in flight); the
+// maximum and its first index do not depend on the visiting order.
+__device__ __forceinline__ void slice_argmax(const float* a, const SpecSlice& sl, float& m, int& mi) {
+  m = -INFINITY;
+  mi = 0x7FFFFFFF;
+  for (long long base = sl.lo + threadIdx.x; base < sl.hi; base += kSpecThreads * kSpecUnroll) {
+    float x[kSpecUnroll];
+#pragma unroll
+    for (int k = 0; k < kSpecUnroll; ++k) {
+      const long long v = base + static_cast<long long>(k) * kSpecThreads;
+      x[k] = v < sl.hi ? a[v] : -INFINITY;
+    }
+#pragma unroll
+    for (int k = 0; k < kSpecUnroll; ++k) {
+      if (x[k] > m) {  // visited in increasing index: the first maximum stays
+        m = x[k];
+        mi = static_cast<int>(base + static_cast<long long>(k) * kSpecThreads);
+      }
+    }
+  }
+}
+
 // One cluster: the draft token from softmax(z / T) over the mapped rows.
 __global__ void __launch_bounds__(kSpecThreads) spec_draft_kernel(const SpecDraftParams P) {
   cg::cluster_group cl = cg::this_cluster();
   __shared__ SpecShared sh;
   const int rank = static_cast<int>(cl.block_rank());
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const SpecSlice sl(P.n_map, rank);
   asm volatile("griddepcontrol.wait;" ::: "memory");
-  float m = -INFINITY;
-  int mi = 0x7FFFFFFF;
-  for (long long v = sl.lo + threadIdx.x; v < sl.hi; v += kSpecThreads) {
-    const float x = P.z[v];
-    if (x > m) {
-      m = x;
-      mi = static_cast<int>(v);
-    }
-  }
+  float m;
+  int mi;
+  slice_argmax(P.z, sl, m, mi);
   block_argmax(m, mi, sh);
   if (threadIdx.x == 0) {
     sh.x.max_q = m;
@@ -282,13 +365,12 @@ __global__ void __launch_bounds__(kSpecThreads) spec_draft_kernel(const SpecDraf
   const float inv_t = P.inv_t;
   const float* z = P.z;
   auto e = [=](long long v) { return expf((z[v] - gm) * inv_t); };
-  const float wsum = warp_walk_sum(sl.wlo(warp), sl.whi(warp), e, lane);
-  const float ctot = block_walk_total(wsum, sh.warp_p);
+  const float ctot = slice_total(sl, e, sh, sh.tiles_p);
   if (threadIdx.x == 0) sh.x.sum_q = ctot;
   cl.sync();
   float tots[kSpecCtas];
   gather_xch(cl, sh, tots, [](const SpecXch& o) { return o.sum_q; });
-  const long long i = cluster_draw(tots, sh.warp_p, sl, rank, *P.u, e);
+  const long long i = cluster_draw(tots, sl, rank, *P.u, e, sh, sh.tiles_p);
   if (i >= 0 && threadIdx.x == 0) {
     float total = 0.f;
     for (int c = 0; c < kSpecCtas; ++c) total += tots[c];
@@ -323,7 +405,6 @@ __global__ void __launch_bounds__(kSpecThreads) spec_verify_kernel(const SpecVer
   cg::cluster_group cl = cg::this_cluster();
   __shared__ SpecShared sh;
   const int rank = static_cast<int>(cl.block_rank());
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int j = blockIdx.y;
   const bool is_draft = j < P.n;
   const float* l = P.target + static_cast<long long>(j) * P.V;
@@ -339,19 +420,14 @@ __global__ void __launch_bounds__(kSpecThreads) spec_verify_kernel(const SpecVer
   }
 
   // maxima (and, greedy, the first index of the maximum) of l_j and z_j
-  float m = -INFINITY;
-  int mi = 0x7FFFFFFF;
-  for (long long v = sl.lo + threadIdx.x; v < sl.hi; v += kSpecThreads) {
-    const float x = l[v];
-    if (x > m) {
-      m = x;
-      mi = static_cast<int>(v);
-    }
-  }
+  float m;
+  int mi;
+  slice_argmax(l, sl, m, mi);
   block_argmax(m, mi, sh);
   float mq = -INFINITY;
   if (is_draft && !P.greedy) {
-    for (long long v = slq.lo + threadIdx.x; v < slq.hi; v += kSpecThreads) mq = fmaxf(mq, z[v]);
+    int unused;
+    slice_argmax(z, slq, mq, unused);
     mq = block_max(mq, sh);
   }
   if (threadIdx.x == 0) {
@@ -389,14 +465,11 @@ __global__ void __launch_bounds__(kSpecThreads) spec_verify_kernel(const SpecVer
   // totals of exp((l - max) / T) and of exp((z - max) / T)
   const float inv_t = P.inv_t;
   auto ep = [=](long long v) { return expf((l[v] - gm) * inv_t); };
-  const float cp = block_walk_total(warp_walk_sum(sl.wlo(warp), sl.whi(warp), ep, lane), sh.warp_p);
+  const float cp = slice_total(sl, ep, sh, sh.tiles_p);
   float cq = 0.f;
   if (is_draft) {
     auto eq = [=](long long v) { return expf((z[v] - gmq) * inv_t); };
-    // these sums only normalise q: a plain strided sum, reduced in a fixed order
-    float s = 0.f;
-    for (long long v = slq.lo + threadIdx.x; v < slq.hi; v += kSpecThreads) s += eq(v);
-    cq = block_walk_total(warp_tree_sum(s), sh.red);
+    cq = slice_total(slq, eq, sh, nullptr);
   }
   if (threadIdx.x == 0) {
     sh.x.sum_p = cp;
@@ -413,7 +486,7 @@ __global__ void __launch_bounds__(kSpecThreads) spec_verify_kernel(const SpecVer
   }
 
   if (!is_draft) {  // the bonus token, from p
-    const long long i = cluster_draw(tot_p, sh.warp_p, sl, rank, P.u[2 * P.n], ep);
+    const long long i = cluster_draw(tot_p, sl, rank, P.u[2 * P.n], ep, sh, sh.tiles_p);
     if (i >= 0 && threadIdx.x == 0) draw_out[j] = static_cast<int32_t>(i);
     cl.sync();
     asm volatile("griddepcontrol.launch_dependents;");
@@ -441,7 +514,7 @@ __global__ void __launch_bounds__(kSpecThreads) spec_verify_kernel(const SpecVer
     const float qv = (r >= 0 && r < n_map) ? expf((z[r] - gmq) * inv_t) * inv_sq : 0.f;
     return fmaxf(expf((l[v] - gm) * inv_t) * inv_sp - qv, 0.f);
   };
-  const float cr = block_walk_total(warp_walk_sum(sl.wlo(warp), sl.whi(warp), er, lane), sh.warp_r);
+  const float cr = slice_total(sl, er, sh, sh.tiles_r);
   if (threadIdx.x == 0) sh.x.sum_r = cr;
   cl.sync();
   float tot_r[kSpecCtas];
@@ -450,9 +523,9 @@ __global__ void __launch_bounds__(kSpecThreads) spec_verify_kernel(const SpecVer
   for (int c = 0; c < kSpecCtas; ++c) sr += tot_r[c];
   long long i;
   if (sr > 0.f)
-    i = cluster_draw(tot_r, sh.warp_r, sl, rank, P.u[P.n + j], er);
+    i = cluster_draw(tot_r, sl, rank, P.u[P.n + j], er, sh, sh.tiles_r);
   else  // p and q agree to rounding: draw from p
-    i = cluster_draw(tot_p, sh.warp_p, sl, rank, P.u[P.n + j], ep);
+    i = cluster_draw(tot_p, sl, rank, P.u[P.n + j], ep, sh, sh.tiles_p);
   if (i >= 0 && threadIdx.x == 0) draw_out[j] = static_cast<int32_t>(i);
   cl.sync();
   asm volatile("griddepcontrol.launch_dependents;");

@@ -38,6 +38,10 @@ int check_device(const char* who) {
 // reading their inputs).
 template <class P>
 int launch_cluster(void (*kernel)(P), const P& params, unsigned rows, cudaStream_t stream, const char* who) {
+  if (q4k::kSpecCtas > 8) {  // clusters above the portable size must be allowed per kernel
+    const cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    if (e != cudaSuccess) return sfail(Q4_ERR_CUDA, std::string(who) + ": cluster size: " + cudaGetErrorString(e));
+  }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(q4k::kSpecCtas, rows, 1);
   cfg.blockDim = dim3(q4k::kSpecThreads, 1, 1);

@@ -344,3 +344,132 @@ class DeviceChain:
     def close(self) -> None:
         self.stack.close()
         self.w.close()
+
+
+# ----------------------------------------------------------------------------
+# One speculative decoding step around the M = 4 pass (bs178.com llamAmpere
+# post, "Why it is this fast", part four): three draft tokens, each from the
+# draft head's projection onto a vocabulary map of 65,536 tokens followed by a
+# draw, then one pass of the main model's stream at M = 4 (the three drafts
+# plus one), whose output head gives the target logits, then the keep /
+# reject step.  The MTP layer that turns a drafted token into the next draft
+# hidden state needs trained weights and is not computed: each draft's hidden
+# state is a seeded input.
+# ----------------------------------------------------------------------------
+SPEC_DRAFTS = 3
+SPEC_INPUT_BASE = 1 << 25  # generator streams of the step's own inputs
+
+
+def vocab_map(seed: int, V: int = VOCAB, n_map: int = DRAFT_VOCAB):
+    """A synthetic vocabulary map (the pages' map file is not available):
+    n_map distinct token ids, ascending, chosen by seeded random keys."""
+    import numpy as np
+
+    from . import synth
+
+    keys = synth.words(seed, synth.act_stream(SPEC_INPUT_BASE), 0, V)
+    return np.sort(np.argsort(keys, kind="stable")[:n_map]).astype(np.int32)
+
+
+def spec_uniforms(seed: int, count: int):
+    """Seeded uniforms in [0, 1) (fp32) for the draws of a step."""
+    import numpy as np
+
+    from . import synth
+
+    w = synth.words(seed, synth.act_stream(SPEC_INPUT_BASE + 1), 0, count)
+    return ((w >> np.uint64(40)).astype(np.float64) / float(1 << 24)).astype(np.float32)
+
+
+class DeviceSpec:
+    """The speculative step on the current CUDA device: the verify stream
+    (DeviceStream of the decode stream at M = n + 1), the mapped draft head
+    (the head's rows at the map's tokens, gathered and packed on the device),
+    one single-product stack per draft, the draft hidden states, logits,
+    drawn rows, uniforms and the verify output."""
+
+    def __init__(self, seed: int = 0, temperature: float = 1.0, n_draft: int = SPEC_DRAFTS):
+        import torch
+
+        import bit_weight_gemv_q4_b200 as q4
+
+        from . import synth
+
+        self.seed, self.T, self.n = seed, float(temperature), n_draft
+        dev = torch.device("cuda")
+        tensors = decode_stream(fused=True)
+        head = tensors[-1]
+        self.V, self.K = head.N, head.K
+        self.verify_stream = DeviceStream(tensors, n_draft + 1, seed=seed, flags=q4.Q4_STACK_INDEPENDENT)
+        self.vmap_host = vocab_map(seed, self.V)
+        self.n_map = len(self.vmap_host)
+        self.vmap = torch.from_numpy(self.vmap_host).to(dev)
+        inv = torch.full((self.V,), -1, dtype=torch.int32)
+        inv[torch.from_numpy(self.vmap_host).long()] = torch.arange(self.n_map, dtype=torch.int32)
+        self.inv_map = inv.to(dev)
+        # the mapped draft head: the head's canonical rows at the map's tokens
+        canon = torch.empty(self.V * self.K, dtype=torch.uint8, device=dev)
+        scales = torch.empty(self.V * (self.K // 32), dtype=torch.int16, device=dev)
+        synth.weights_device(8, seed, synth.weight_stream(head.tensor_id), self.K, 0, self.V, canon)
+        synth.scales_device(seed, synth.scale_stream(head.tensor_id), self.K, 0, self.V, scales)
+        gq = torch.empty(self.n_map * self.K, dtype=torch.uint8, device=dev)
+        gs = torch.empty(self.n_map * (self.K // 32), dtype=torch.int16, device=dev)
+        q4.q4_gather_rows_device(canon, self.K, self.V, self.vmap, self.n_map, gq)
+        q4.q4_gather_rows_device(scales, 2 * (self.K // 32), self.V, self.vmap, self.n_map, gs)
+        self.draft_packed = torch.empty(q4.q4_packed_bytes(8, self.n_map, self.K), dtype=torch.uint8, device=dev)
+        q4.q4_pack_weights_device(8, gq, gs, self.n_map, self.K, self.draft_packed)
+        del canon, scales, gq, gs
+        self.x_draft = []
+        for j in range(n_draft):
+            xj = torch.empty(self.K, dtype=torch.int16, device=dev)
+            synth.activations_device(seed, synth.act_stream(SPEC_INPUT_BASE + 2 + j), 1, self.K, xj)
+            self.x_draft.append(xj)
+        self.z = torch.empty(max(n_draft, 1) * self.n_map, dtype=torch.float32, device=dev)
+        self.draft_stacks = [
+            q4.layer_stack_create([(8, self.n_map, self.K, self.draft_packed, self.x_draft[j],
+                                    self.z[j * self.n_map:(j + 1) * self.n_map])], 1, q4.Q4_STACK_INDEPENDENT)
+            for j in range(n_draft)]
+        self.u_host = spec_uniforms(seed, 3 * n_draft + 1)
+        self.u = torch.from_numpy(self.u_host).to(dev)
+        self.rows = torch.zeros(max(n_draft, 1), dtype=torch.int32, device=dev)
+        self.tokens = torch.zeros(max(n_draft, 1), dtype=torch.int32, device=dev)
+        self.q = torch.zeros(max(n_draft, 1), dtype=torch.float32, device=dev)
+        self.out = torch.zeros(3 * n_draft + 3, dtype=torch.int32, device=dev)
+        torch.cuda.synchronize()
+
+    @property
+    def target_logits(self):
+        return self.verify_stream.y[-1]  # [n + 1][V]
+
+    def draft(self, j: int, stream=None) -> None:
+        import bit_weight_gemv_q4_b200 as q4
+
+        q4.layer_stack_run(self.draft_stacks[j], stream)
+        q4.q4_spec_draft(self.z[j * self.n_map:(j + 1) * self.n_map], self.n_map, self.vmap, self.T,
+                         self.u[j:j + 1], self.rows[j:j + 1], self.tokens[j:j + 1], self.q[j:j + 1], stream)
+
+    def verify(self, stream=None) -> None:
+        import bit_weight_gemv_q4_b200 as q4
+
+        q4.q4_spec_verify(self.target_logits, self.V, self.z, self.n_map, self.vmap, self.inv_map, self.rows,
+                          self.n, self.T, self.u[self.n:], self.out, stream)
+
+    def run(self, stream=None) -> None:
+        """One step: the drafts, the M = n + 1 pass, the keep / reject step."""
+        for j in range(self.n):
+            self.draft(j, stream)
+        self.verify_stream.run(stream)
+        self.verify(stream)
+
+    def check(self, stream=None) -> None:
+        import bit_weight_gemv_q4_b200 as q4
+
+        for st in self.draft_stacks:
+            q4.layer_stack_check(st, stream)
+        self.verify_stream.check(stream)
+
+    def close(self) -> None:
+        for st in self.draft_stacks:
+            st.close()
+        self.draft_stacks.clear()
+        self.verify_stream.close()

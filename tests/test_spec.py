@@ -434,3 +434,42 @@ def test_mapped_draft_head_by_row_gather(cuda_device):
     y, ok = H.run_gemv(8, packed, n_map, K, H.to_device_x(x), 1)
     assert ok
     H.assert_parity(y, qh[vmap], sh[vmap], x, 8)
+
+
+@pytest.mark.gpu
+def test_speculative_step_end_to_end(cuda_device):
+    """The whole step on the device (the mapped draft head gathered from the
+    q8 output head, three drafts, the 257-product stream at M = 4, the keep /
+    reject step): the draws checked against the oracle on the device's own
+    logits.  The synthetic head's logits spread over ~+-300, so T = 60 keeps
+    the distributions wide."""
+    from bit_weight_gemv_q4_b200 import workloads
+
+    torch = _torch()
+    sp = workloads.DeviceSpec(seed=0, temperature=60.0)
+    try:
+        sp.run()
+        sp.check()
+        torch.cuda.synchronize()
+        n, n_map, V = sp.n, sp.n_map, sp.V
+        z = sp.z.cpu().numpy().reshape(n, n_map)
+        rows = sp.rows.cpu().numpy()
+        u = sp.u_host
+        for j in range(n):
+            _check_draw(OS.dist(z[j].astype(np.float64), sp.T), float(u[j]), int(rows[j]), f"draft {j}")
+        assert np.array_equal(sp.tokens.cpu().numpy(), sp.vmap_host[rows])
+        target = sp.target_logits.cpu().numpy().reshape(n + 1, V)
+        out = sp.out.cpu().numpy()
+        _check_verify(target, z, sp.vmap_host, rows, u[n:], sp.T, out)
+        # the mapped head's outputs: row r is the output head's row at token vmap[r]
+        from bit_weight_gemv_q4_b200 import synth
+        import gpu_helpers as H
+
+        rs = np.random.default_rng(1).integers(0, n_map, 6)
+        for r in rs:
+            qh, sh = synth.tensor(8, 0, 1023, V, sp.K, row0=int(sp.vmap_host[r]), nrows=1)
+            x = sp.x_draft[0].cpu().numpy().view(np.uint16).reshape(1, sp.K)
+            H.assert_parity(z[0:1, r:r + 1], qh, sh, x, 8)
+    finally:
+        sp.close()
+        torch.cuda.empty_cache()

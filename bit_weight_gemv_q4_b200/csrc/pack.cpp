@@ -27,18 +27,41 @@ struct Geometry {
 };
 
 bool geometry(int bits, int64_t N, int64_t K, Geometry* g) {
-  if ((bits != 4 && bits != 8) || N < 0 || K < 0 || K % 32 != 0) return false;
+  if ((bits < 4 || bits > 6) && bits != 8) return false;
+  if (N < 0 || K < 0 || K % 32 != 0 || ((bits == 5 || bits == 6) && K % 64 != 0)) return false;
   // keep every offset and index comfortably inside int64 / int32 tile counts
   if (N > (int64_t(1) << 34) || K > (int64_t(1) << 30)) return false;
   g->bits = bits;
   g->N = N;
   g->K = K;
   g->T = (N + kTileRows - 1) / kTileRows;
-  g->k_per_chunk = bits == 4 ? 64 : 32;
+  g->k_per_chunk = bits == 8 ? 32 : 64;
   g->C = (K + g->k_per_chunk - 1) / g->k_per_chunk;
-  g->chunk_bytes = bits == 4 ? 1152 : 1088;
+  g->chunk_bytes = bits == 4 ? 1152 : bits == 5 ? 1408 : bits == 6 ? 1664 : 1088;
   return true;
 }
+
+// q5 / q6: the q4 chunk's code blocks hold the low nibble of u = q + 16 (q5)
+// or q + 32 (q6); the high bits of lane L sit in a plane after them (q5: 8
+// bytes at 1024 + 8L, word h; q6: 16 bytes at 1024 + 16L, word 2h + (j >> 1)),
+// at the positions below, then the scales (q4 placement) at 1024 + 256 (q5)
+// or 1024 + 512 (q6).  Nibble i of code word j belongs to tensor-core register
+// r = i & 3, half-word el = i >> 2.
+constexpr int kWideShift5[8] = {-4, -3, -2, -1, 4, 5, 6, 7};  // by 2j + (r >> 1)
+constexpr int kWideShift6[4] = {-4, -2, 4, 6};                 // by 2 (j & 1) + (r >> 1)
+
+inline int wide_hi_pos(int bits, int j, int i) {
+  const int r = i & 3, el = i >> 2;
+  const int target = (r & 1) ? 8 : 4;
+  const int sh = bits == 5 ? kWideShift5[2 * j + (r >> 1)] : kWideShift6[2 * (j & 1) + (r >> 1)];
+  return 16 * el + sh + target;
+}
+
+inline int64_t wide_hi_offset(int bits, int h, int lane, int j) {
+  return bits == 5 ? 1024 + 8 * lane + 4 * h : 1024 + 16 * lane + 8 * h + 4 * (j >> 1);
+}
+
+inline int64_t wide_scale_base(int bits) { return bits == 5 ? 1024 + 256 : 1024 + 512; }
 
 // Row and column of nibble i of word j in slot (gi, ti) of half h of q4
 // chunk (t, c).
@@ -64,6 +87,93 @@ inline int canon_q4(const uint8_t* q, int64_t K, int64_t row, int64_t col) {
   return nib >= 8 ? nib - 16 : nib;
 }
 
+inline uint32_t load32(const uint8_t* p) {
+  uint32_t v;
+  std::memcpy(&v, p, 4);
+  return v;
+}
+
+inline void store32(uint8_t* p, uint32_t v) { std::memcpy(p, &v, 4); }
+
+// q5 / q6 codes (canonical int8 [N][K], q in [-16, 15] or [-32, 31]) into
+// the packed chunks (K % 64 == 0; see wide_hi_pos).
+void pack_wide(const Geometry& g, const int8_t* q, const uint16_t* scales, uint8_t* dst) {
+  const int bits = g.bits, off = bits == 5 ? 16 : 32;
+  const int64_t hi_bytes = bits == 5 ? 256 : 512, sbase = wide_scale_base(bits), G = g.K / 32;
+#pragma omp parallel for schedule(static)
+  for (int64_t t = 0; t < g.T; ++t) {
+    for (int64_t c = 0; c < g.C; ++c) {
+      uint8_t* chunk = dst + (t * g.C + c) * g.chunk_bytes;
+      std::memset(chunk + 1024, 0, hi_bytes);
+      for (int h = 0; h < 2; ++h)
+        for (int gi = 0; gi < 8; ++gi)
+          for (int ti = 0; ti < 4; ++ti) {
+            const int lane = 4 * gi + ti;
+            uint32_t words[4] = {0, 0, 0, 0};
+            for (int j = 0; j < 4; ++j)
+              for (int i = 0; i < 8; ++i) {
+                int64_t row, col;
+                q4_coord(t, c, h, gi, ti, j, i, &row, &col);
+                const int u = (row < g.N ? q[row * g.K + col] : 0) + off;
+                words[j] |= static_cast<uint32_t>(u & 15) << (4 * i);
+                uint8_t* hp = chunk + wide_hi_offset(bits, h, lane, j);
+                store32(hp, load32(hp) | (static_cast<uint32_t>(u >> 4) << wide_hi_pos(bits, j, i)));
+              }
+            std::memcpy(chunk + 512 * h + 16 * lane, words, 16);
+          }
+      for (int gi = 0; gi < 8; ++gi) {
+        uint16_t s8[8];
+        for (int h = 0; h < 2; ++h)
+          for (int up = 0; up < 2; ++up)
+            for (int gg = 0; gg < 2; ++gg) {
+              const int64_t row = scale_row(t, h, gi, up), grp = 2 * c + gg;
+              s8[4 * h + 2 * up + gg] = row < g.N ? scales[row * G + grp] : 0;
+            }
+        std::memcpy(chunk + sbase + 16 * gi, s8, 16);
+      }
+    }
+  }
+}
+
+void unpack_wide(const Geometry& g, const uint8_t* src, int8_t* q, uint16_t* scales) {
+  const int bits = g.bits, off = bits == 5 ? 16 : 32;
+  const int64_t sbase = wide_scale_base(bits), G = g.K / 32;
+#pragma omp parallel for schedule(static)
+  for (int64_t t = 0; t < g.T; ++t) {
+    for (int64_t c = 0; c < g.C; ++c) {
+      const uint8_t* chunk = src + (t * g.C + c) * g.chunk_bytes;
+      for (int h = 0; h < 2; ++h)
+        for (int gi = 0; gi < 8; ++gi)
+          for (int ti = 0; ti < 4; ++ti) {
+            const int lane = 4 * gi + ti;
+            for (int j = 0; j < 4; ++j) {
+              const uint32_t w = load32(chunk + 512 * h + 16 * lane + 4 * j);
+              const uint32_t hw = load32(chunk + wide_hi_offset(bits, h, lane, j));
+              for (int i = 0; i < 8; ++i) {
+                int64_t row, col;
+                q4_coord(t, c, h, gi, ti, j, i, &row, &col);
+                if (row >= g.N) continue;
+                const int hi = static_cast<int>((hw >> wide_hi_pos(bits, j, i)) & (bits == 5 ? 1u : 3u));
+                const int u = static_cast<int>((w >> (4 * i)) & 15u) + 16 * hi;
+                q[row * g.K + col] = static_cast<int8_t>(u - off);
+              }
+            }
+          }
+      for (int gi = 0; gi < 8; ++gi)
+        for (int h = 0; h < 2; ++h)
+          for (int up = 0; up < 2; ++up)
+            for (int gg = 0; gg < 2; ++gg) {
+              const int64_t row = scale_row(t, h, gi, up), grp = 2 * c + gg;
+              if (row < g.N) {
+                uint16_t v;
+                std::memcpy(&v, chunk + sbase + 16 * gi + 2 * (4 * h + 2 * up + gg), 2);
+                scales[row * G + grp] = v;
+              }
+            }
+    }
+  }
+}
+
 }  // namespace
 
 extern "C" Q4_API size_t q4_packed_bytes(int bits, int64_t N, int64_t K) {
@@ -75,12 +185,13 @@ extern "C" Q4_API size_t q4_packed_bytes(int bits, int64_t N, int64_t K) {
 extern "C" Q4_API int q4_pack_weights(int bits, const void* canon_q, const uint16_t* scales, int64_t N, int64_t K,
                                       void* out, size_t out_bytes) {
   Geometry g;
-  if (bits != 4 && bits != 8) {
-    q4::set_error("q4_pack_weights: bits must be 4 or 8");
+  if (bits != 4 && bits != 5 && bits != 6 && bits != 8) {
+    q4::set_error("q4_pack_weights: bits must be 4, 5, 6 or 8");
     return Q4_ERR_INVALID_ARG;
   }
   if (!geometry(bits, N, K, &g)) {
-    q4::set_error("q4_pack_weights: need N >= 0, K >= 0, K % 32 == 0 (and sizes below 2^34 x 2^30)");
+    q4::set_error("q4_pack_weights: need N >= 0, K >= 0, K % 32 == 0 (K % 64 == 0 for 5 and 6 bits; "
+                  "sizes below 2^34 x 2^30)");
     return Q4_ERR_SHAPE;
   }
   const size_t need = static_cast<size_t>(g.T * g.C * g.chunk_bytes);
@@ -92,6 +203,18 @@ extern "C" Q4_API int q4_pack_weights(int bits, const void* canon_q, const uint1
   if (out_bytes < need) {
     q4::set_error("q4_pack_weights: out_bytes " + std::to_string(out_bytes) + " < " + std::to_string(need));
     return Q4_ERR_BUFFER_TOO_SMALL;
+  }
+  if (bits == 5 || bits == 6) {
+    const int8_t* q = static_cast<const int8_t*>(canon_q);
+    const int lim = bits == 5 ? 16 : 32;
+    for (int64_t e = 0; e < N * K; ++e)
+      if (q[e] < -lim || q[e] >= lim) {
+        q4::set_error("q4_pack_weights: a code outside [" + std::to_string(-lim) + ", " + std::to_string(lim - 1) +
+                      "] for " + std::to_string(bits) + " bits");
+        return Q4_ERR_INVALID_ARG;
+      }
+    pack_wide(g, q, scales, static_cast<uint8_t*>(out));
+    return Q4_OK;
   }
   const int64_t G = K / 32;
   uint8_t* dst = static_cast<uint8_t*>(out);
@@ -157,8 +280,8 @@ extern "C" Q4_API int q4_pack_weights(int bits, const void* canon_q, const uint1
 extern "C" Q4_API int q4_unpack_weights(int bits, const void* packed, size_t packed_bytes, int64_t N, int64_t K,
                                         void* canon_q_out, uint16_t* scales_out) {
   Geometry g;
-  if (bits != 4 && bits != 8) {
-    q4::set_error("q4_unpack_weights: bits must be 4 or 8");
+  if (bits != 4 && bits != 5 && bits != 6 && bits != 8) {
+    q4::set_error("q4_unpack_weights: bits must be 4, 5, 6 or 8");
     return Q4_ERR_INVALID_ARG;
   }
   if (!geometry(bits, N, K, &g)) {
@@ -174,6 +297,10 @@ extern "C" Q4_API int q4_unpack_weights(int bits, const void* packed, size_t pac
   if (packed_bytes < need) {
     q4::set_error("q4_unpack_weights: packed_bytes too small");
     return Q4_ERR_BUFFER_TOO_SMALL;
+  }
+  if (bits == 5 || bits == 6) {
+    unpack_wide(g, static_cast<const uint8_t*>(packed), static_cast<int8_t*>(canon_q_out), scales_out);
+    return Q4_OK;
   }
   const int64_t G = K / 32;
   const uint8_t* src = static_cast<const uint8_t*>(packed);

@@ -148,15 +148,25 @@ int make_shape(int bits, int64_t N, int64_t K, Shape* s, const char* who) {
   return Q4_OK;
 }
 
-// A stack entry's shape: bits 4 or 8, or Q4_FMT_NVFP4 (the q4 chunk geometry,
-// K a multiple of 64).
+// A stack entry's shape: bits 4 or 8, or 5, 6 or Q4_FMT_NVFP4 (the q4 chunk
+// geometry, K a multiple of 64).
 int entry_shape(int bits, int64_t N, int64_t K, Shape* s, const char* who) {
-  if (bits != Q4_FMT_NVFP4) return make_shape(bits, N, K, s, who);
+  if (bits != Q4_FMT_NVFP4 && bits != 5 && bits != 6) return make_shape(bits, N, K, s, who);
   const int rc = make_shape(4, N, K, s, who);
   if (rc) return rc;
-  if (K % 64 != 0) return fail(Q4_ERR_SHAPE, "%s: NVFP4 needs K %% 64 == 0 (K=%lld)", who, (long long)K);
-  s->bits = Q4_FMT_NVFP4;
+  if (K % 64 != 0) return fail(Q4_ERR_SHAPE, "%s: %d-bit formats need K %% 64 == 0 (K=%lld)", who, bits, (long long)K);
+  s->bits = bits;
   return Q4_OK;
+}
+
+// Formats that run in stream mode only.
+bool stream_only(int bits) { return bits == Q4_FMT_NVFP4 || bits == 5 || bits == 6; }
+
+// Chunk bytes of a stack entry's format.
+int chunk_bytes_of(int bits) {
+  return bits == 8 ? q4k::Format<8>::kChunkBytes
+                   : bits == 5 ? q4k::Wide<5>::kChunkBytes : bits == 6 ? q4k::Wide<6>::kChunkBytes
+                                                                       : q4k::Format<4>::kChunkBytes;
 }
 
 long long max_warps(const DeviceInfo& dev) { return static_cast<long long>(dev.sms) * kCtasPerSm * kNW; }
@@ -381,7 +391,8 @@ extern "C" Q4_API int q4_set_wait_timeout_ns(uint64_t ns) {
 extern "C" Q4_API int q4_unpack_device(int bits, const void* packed, int64_t N, int64_t K, int8_t* q_out,
                                        uint16_t* scales_out, void* stream) {
   Shape s;
-  int rc = make_shape(bits, N, K, &s, "q4_unpack_device");
+  if (bits == Q4_FMT_NVFP4) return fail(Q4_ERR_INVALID_ARG, "q4_unpack_device: bits must be 4, 5, 6 or 8");
+  int rc = entry_shape(bits, N, K, &s, "q4_unpack_device");
   if (rc) return rc;
   if (s.TC == 0) return Q4_OK;
   if (!packed || !q_out || !scales_out) return fail(Q4_ERR_INVALID_ARG, "q4_unpack_device: null pointer");
@@ -393,7 +404,13 @@ extern "C" Q4_API int q4_unpack_device(int bits, const void* packed, int64_t N, 
   const long long blocks = (s.TC + warps - 1) / warps;
   if (blocks > 0x7FFFFFFFLL) return fail(Q4_ERR_SHAPE, "q4_unpack_device: tensor too large");
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (bits == 4)
+  if (bits == 5)
+    q4k::unpack_wide_kernel<5><<<static_cast<unsigned>(blocks), warps * 32, 0, st>>>(
+        static_cast<const uint8_t*>(packed), s.N, s.K, s.T, s.C, q_out, scales_out);
+  else if (bits == 6)
+    q4k::unpack_wide_kernel<6><<<static_cast<unsigned>(blocks), warps * 32, 0, st>>>(
+        static_cast<const uint8_t*>(packed), s.N, s.K, s.T, s.C, q_out, scales_out);
+  else if (bits == 4)
     q4k::unpack_kernel<4><<<static_cast<unsigned>(blocks), warps * 32, 0, st>>>(
         static_cast<const uint8_t*>(packed), s.N, s.K, s.T, s.C, q_out, scales_out);
   else
@@ -406,9 +423,10 @@ extern "C" Q4_API int q4_unpack_device(int bits, const void* packed, int64_t N, 
 extern "C" Q4_API int q4_pack_weights_device(int bits, const void* canon_q, const uint16_t* scales_fp16, int64_t N,
                                              int64_t K, void* out, size_t out_bytes, void* stream) {
   Shape s;
-  int rc = make_shape(bits, N, K, &s, "q4_pack_weights_device");
+  if (bits == Q4_FMT_NVFP4) return fail(Q4_ERR_INVALID_ARG, "q4_pack_weights_device: bits must be 4, 5, 6 or 8");
+  int rc = entry_shape(bits, N, K, &s, "q4_pack_weights_device");
   if (rc) return rc;
-  const size_t need = static_cast<size_t>(s.TC) * (bits == 4 ? q4k::Format<4>::kChunkBytes : q4k::Format<8>::kChunkBytes);
+  const size_t need = static_cast<size_t>(s.TC) * chunk_bytes_of(bits);
   if (need == 0) return Q4_OK;
   if (!canon_q || !scales_fp16 || !out) return fail(Q4_ERR_INVALID_ARG, "q4_pack_weights_device: null pointer");
   if (reinterpret_cast<uintptr_t>(out) % 16)
@@ -424,7 +442,13 @@ extern "C" Q4_API int q4_pack_weights_device(int bits, const void* canon_q, cons
   if (blocks > 0x7FFFFFFFLL) return fail(Q4_ERR_SHAPE, "q4_pack_weights_device: tensor too large");
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const uint8_t* q = static_cast<const uint8_t*>(canon_q);
-  if (bits == 4)
+  if (bits == 5)
+    q4k::pack_wide_kernel<5><<<static_cast<unsigned>(blocks), 256, 0, st>>>(
+        reinterpret_cast<const int8_t*>(q), scales_fp16, s.N, s.K, s.T, s.C, static_cast<uint8_t*>(out));
+  else if (bits == 6)
+    q4k::pack_wide_kernel<6><<<static_cast<unsigned>(blocks), 256, 0, st>>>(
+        reinterpret_cast<const int8_t*>(q), scales_fp16, s.N, s.K, s.T, s.C, static_cast<uint8_t*>(out));
+  else if (bits == 4)
     q4k::pack_kernel<4><<<static_cast<unsigned>(blocks), 256, 0, st>>>(q, scales_fp16, s.N, s.K, s.T, s.C,
                                                                         static_cast<uint8_t*>(out));
   else
@@ -599,33 +623,40 @@ void* stack_kernel_ptr() {
   return reinterpret_cast<void*>(&q4k::stack_kernel<M, kStackNW, kStackD, kStackPF>);
 }
 
-template <int M, int SU, bool NV>
+template <int M, int SU, int FC>
 void* stream_kernel_ptr() {
-  return reinterpret_cast<void*>(&q4k::stream_kernel<M, kStackNW, kStackD, SU, NV>);
+  return reinterpret_cast<void*>(&q4k::stream_kernel<M, kStackNW, kStackD, SU, FC>);
 }
 
-// su: chunks per stage of the stream-mode kernel (0 = ordered mode); nv: the
-// list holds NVFP4 products
-void* select_stack_kernel(int M, int su, bool nv) {
-  static void* const table[5][4] = {
-      {stack_kernel_ptr<1>(), stack_kernel_ptr<2>(), stack_kernel_ptr<3>(), stack_kernel_ptr<4>()},
-      {stream_kernel_ptr<1, 2, false>(), stream_kernel_ptr<2, 2, false>(), stream_kernel_ptr<3, 2, false>(),
-       stream_kernel_ptr<4, 2, false>()},
-      {stream_kernel_ptr<1, kStreamU, false>(), stream_kernel_ptr<2, kStreamU, false>(),
-       stream_kernel_ptr<3, kStreamU, false>(), stream_kernel_ptr<4, kStreamU, false>()},
-      {stream_kernel_ptr<1, 2, true>(), stream_kernel_ptr<2, 2, true>(), stream_kernel_ptr<3, 2, true>(),
-       stream_kernel_ptr<4, 2, true>()},
-      {stream_kernel_ptr<1, kStreamU, true>(), stream_kernel_ptr<2, kStreamU, true>(),
-       stream_kernel_ptr<3, kStreamU, true>(), stream_kernel_ptr<4, kStreamU, true>()}};
-  const int row = su == 0 ? 0 : (su == 2 ? 1 : 2) + (nv ? 2 : 0);
-  return table[row][M - 1];
+template <int SU, int FC>
+struct StreamRow {
+  static void* at(int M) {
+    static void* const row[4] = {stream_kernel_ptr<1, SU, FC>(), stream_kernel_ptr<2, SU, FC>(),
+                                 stream_kernel_ptr<3, SU, FC>(), stream_kernel_ptr<4, SU, FC>()};
+    return row[M - 1];
+  }
+};
+
+// su: chunks per stage of the stream-mode kernel (0 = ordered mode); fc: the
+// list's format class (0 q4 / q8, 1 also NVFP4, 2 also q5 / q6).  Class 2 with
+// stages of four chunks exists for M = 1 only (its slots fit shared memory
+// there; create_persistent picks stages of two otherwise).
+void* select_stack_kernel(int M, int su, int fc) {
+  static void* const ordered[4] = {stack_kernel_ptr<1>(), stack_kernel_ptr<2>(), stack_kernel_ptr<3>(),
+                                   stack_kernel_ptr<4>()};
+  if (su == 0) return ordered[M - 1];
+  if (fc == 0) return su == 2 ? StreamRow<2, 0>::at(M) : StreamRow<kStreamU, 0>::at(M);
+  if (fc == 1) return su == 2 ? StreamRow<2, 1>::at(M) : StreamRow<kStreamU, 1>::at(M);
+  if (su != 2 && M == 1) return stream_kernel_ptr<1, kStreamU, 2>();
+  return StreamRow<2, 2>::at(M);
 }
 
 // su: stream mode with stages of su chunks (weights + activation slice of M
 // rows), or 0 for ordered mode (weights only, stages of kStackU chunks).
-int stack_smem_bytes(int su, int M) {
+int stack_smem_bytes(int su, int M, int fc) {
+  const int cb = fc == 2 ? q4k::Wide<6>::kChunkBytes : q4k::Format<4>::kChunkBytes;
   const int slot = su == 0 ? q4k::kStackU * q4k::Format<4>::kChunkBytes
-                           : su * (q4k::Format<4>::kChunkBytes + M * q4k::Format<4>::kKPerChunk * 2);
+                           : su * (cb + M * q4k::Format<4>::kKPerChunk * 2);
   return kStackNW * kStackD * slot + kStackNW * kStackD * 8;
 }
 
@@ -653,6 +684,13 @@ bool stack_eligible(const q4_stack_entry* entries, int n) {
 // su: stream mode with stages of su chunks (every product's C a multiple of
 // su), or 0 for ordered mode.
 int create_persistent(const q4_stack_entry* entries, int n, int M, int su, const DeviceInfo& dev, q4_stack* st) {
+  int fc = 0;
+  for (int i = 0; i < n; ++i) {
+    if (entries[i].bits == Q4_FMT_NVFP4) fc = std::max(fc, 1);
+    if (entries[i].bits == 5 || entries[i].bits == 6) fc = 2;
+  }
+  // stages of four chunks of the widest formats fit shared memory at M = 1 only
+  if (su != 0 && fc == 2 && M > 1) su = 2;
   const bool independent = su != 0;
   const long long blk = independent ? su : q4k::kStackU;  // chunks per stream-K block
   long long max_t = 1, total_blocks = 0, total_tiles = 0;
@@ -699,7 +737,7 @@ int create_persistent(const q4_stack_entry* entries, int n, int M, int su, const
   size_t prep_bytes = 0;
   if (independent) {
     for (int i = 0; i < n; ++i) {
-      const int KC = entries[i].bits == 8 ? q4k::Format<8>::kKPerChunk : q4k::Format<4>::kKPerChunk;
+      const int KC = entries[i].bits == 8 ? q4k::Format<8>::kKPerChunk : q4k::Format<4>::kKPerChunk;  // 64: q4-geometry formats
       size_t jdx = jobs.size();
       for (size_t k = 0; k < jobs.size(); ++k)
         if (jobs[k].x == entries[i].x && jobs[k].K == entries[i].K && jobs[k].KC == KC) jdx = k;
@@ -749,10 +787,8 @@ int create_persistent(const q4_stack_entry* entries, int n, int M, int su, const
   if (err == cudaSuccess)
     err = cudaMemcpy(st->entries_dev, host.data(), sizeof(q4k::StackEntryDev) * host.size(), cudaMemcpyHostToDevice);
   if (err != cudaSuccess) return cuda_fail(err, "layer_stack_create: allocation");
-  bool nv = false;
-  for (int i = 0; i < n; ++i) nv = nv || entries[i].bits == Q4_FMT_NVFP4;
-  st->fn = select_stack_kernel(M, su, nv);
-  st->smem = stack_smem_bytes(su, M);
+  st->fn = select_stack_kernel(M, su, fc);
+  st->smem = stack_smem_bytes(su, M, fc);
   st->block = kStackNW * 32;
   st->grid = dev.sms;
   err = cudaFuncSetAttribute(st->fn, cudaFuncAttributeMaxDynamicSharedMemorySize, st->smem);
@@ -843,17 +879,18 @@ extern "C" Q4_API int layer_stack_create(const q4_stack_entry* entries, int n_en
   DeviceInfo dev;
   int rc = device_info(&dev);
   if (rc) return rc;
-  // NVFP4 products run in stream mode only
+  // NVFP4, q5 and q6 products run in stream mode only
   for (int i = 0; i < n_entries; ++i) {
-    if (entries[i].bits != Q4_FMT_NVFP4) continue;
+    if (!stream_only(entries[i].bits)) continue;
     char who[64];
     snprintf(who, sizeof(who), "layer_stack_create entry %d", i);
     Shape s;
     if ((rc = entry_shape(entries[i].bits, entries[i].N, entries[i].K, &s, who))) return rc;
     if ((flags & Q4_STACK_INDEPENDENT) == 0 || (flags & (Q4_STACK_GRAPH | Q4_STACK_NO_PDL)) != 0)
-      return fail(Q4_ERR_UNSUPPORTED, "%s: NVFP4 products need stream mode (Q4_STACK_INDEPENDENT alone)", who);
+      return fail(Q4_ERR_UNSUPPORTED, "%s: NVFP4, q5 and q6 products need stream mode (Q4_STACK_INDEPENDENT alone)",
+                  who);
     if (!stack_eligible(entries, n_entries))
-      return fail(Q4_ERR_UNSUPPORTED, "%s: NVFP4 needs every product non-empty with an even chunk count", who);
+      return fail(Q4_ERR_UNSUPPORTED, "%s: stream mode needs every product non-empty with an even chunk count", who);
   }
   q4_stack* st = new q4_stack();
   cudaGetDevice(&st->device);
@@ -872,10 +909,10 @@ extern "C" Q4_API int layer_stack_create(const q4_stack_entry* entries, int n_en
     }
   }
   for (int i = 0; i < n_entries; ++i)
-    if (entries[i].bits == Q4_FMT_NVFP4 && su == 0) {
+    if (stream_only(entries[i].bits) && su == 0) {
       free_stack(st);
-      return fail(Q4_ERR_UNSUPPORTED, "layer_stack_create: NVFP4 products need stream mode, and a q4 product "
-                                      "with K %% 64 != 0 rules it out");
+      return fail(Q4_ERR_UNSUPPORTED, "layer_stack_create: NVFP4, q5 and q6 products need stream mode, and a q4 "
+                                      "product with K %% 64 != 0 rules it out");
     }
   rc = graph ? create_graph(entries, n_entries, M, flags, dev, st)
              : create_persistent(entries, n_entries, M, su, dev, st);

@@ -24,6 +24,7 @@
 
 #include "q4gemv_kernels.cuh"
 #include "q4nvfp4_kernel.cuh"
+#include "q4wide_kernel.cuh"
 
 namespace q4k {
 
@@ -471,16 +472,30 @@ __device__ __forceinline__ int entry_of_block(const StackParams& sp, long long g
 // A stage is SU chunks of weights followed, in the same slot and on the same
 // mbarrier, by the matching activation slice (SU chunks x M rows x KC
 // values, one contiguous copy from the chunk-major xc).
-template <int SU, int M>
+// Format classes of a stream-mode list: 0 = q4 / q8, 1 = also NVFP4, 2 = also
+// q5 / q6.  A class's kernel carries only its formats' segments, and its slot
+// fits the largest chunk among them.
+template <int FC>
+struct FormatClass {
+  static constexpr int kMaxChunkBytes = FC == 2 ? Wide<6>::kChunkBytes : Format<4>::kChunkBytes;
+};
+
+// Chunk bytes of a stack entry's format.
+__device__ __forceinline__ int entry_chunk_bytes(int bits) {
+  return bits == 8 ? Format<8>::kChunkBytes
+                   : bits == 5 ? Wide<5>::kChunkBytes : bits == 6 ? Wide<6>::kChunkBytes : Format<4>::kChunkBytes;
+}
+
+template <int SU, int M, int FC>
 struct StreamSlot {
-  static constexpr int kWeightBytes = SU * Format<4>::kChunkBytes;  // the larger of the two formats
+  static constexpr int kWeightBytes = SU * FormatClass<FC>::kMaxChunkBytes;
   static constexpr int kXBytes = SU * M * Format<4>::kKPerChunk * 2;
   static constexpr int kBytes = kWeightBytes + kXBytes;
 };
 
 // The producer side of a warp's ring in stream mode: the next stage (SU
 // chunks) to copy in the warp's range, crossing products.  Warp-uniform state.
-template <int SU, int M>
+template <int SU, int M, int FC>
 struct StreamProducer {
   int e = 0;                 // product of the next stage
   int left_entry = 0;        // stages left in that product
@@ -493,7 +508,9 @@ struct StreamProducer {
 
   __device__ __forceinline__ void enter(const StackParams& sp, int entry, long long lb) {
     const StackEntryDev& en = sp.entries[entry];
-    const int CB = en.bits == 8 ? Format<8>::kChunkBytes : Format<4>::kChunkBytes;  // NVFP4: the q4 geometry
+    // NVFP4, q5 and q6 have the q4 geometry; only class 2 lists hold q5 / q6
+    const int CB = FC == 2 ? entry_chunk_bytes(en.bits)
+                           : (en.bits == 8 ? Format<8>::kChunkBytes : Format<4>::kChunkBytes);
     e = entry;
     bytes = static_cast<uint32_t>(SU * CB);
     src = en.packed + lb * SU * CB;
@@ -516,7 +533,7 @@ struct StreamProducer {
     if (left_total == 0) return false;
     if (left_entry == 0) enter(sp, e + 1, 0);
     const uint32_t xb = x_bytes();
-    bulk_copy_g2s_x_if(lane == 0, dst, src, bytes, dst + StreamSlot<SU, M>::kWeightBytes, x_src(), xb, with_x,
+    bulk_copy_g2s_x_if(lane == 0, dst, src, bytes, dst + StreamSlot<SU, M, FC>::kWeightBytes, x_src(), xb, with_x,
                        bar, policy);
     if (!with_x) {
       *x_later = x_src();
@@ -555,25 +572,26 @@ struct StreamRing {
 // in acc with (r, c).  Returns false if a ring wait gave up.
 // F16: the activations are used in fp16 (en.x16).  Finished tile sums are
 // multiplied by `scale` (2^sigma when F16, times t for NVFP4).
-template <int BITS, int M, int D, int SU, bool F16>
+template <int BITS, int M, int D, int SU, bool F16, int FC>
 __device__ __forceinline__ bool stream_segment(const StackParams& sp, const StackEntryDev* __restrict__ ep, int e,
                                                long long lb0,
                                                long long nblk, long long gb, StreamRing& rg,
-                                               StreamProducer<SU, M>& pr, uint64_t policy, float scale,
+                                               StreamProducer<SU, M, FC>& pr, uint64_t policy, float scale,
                                                float (&acc)[2][4], int pw, int& e_first, int& r_first, int& r,
                                                int& c, int lane) {
   constexpr int U = SU;
-  constexpr int SLOT = StreamSlot<SU, M>::kBytes;
+  constexpr int SLOT = StreamSlot<SU, M, FC>::kBytes;
   constexpr bool NV = BITS == kFmtNvfp4;
-  constexpr int FB = BITS == 8 ? 8 : 4;  // NVFP4 chunks have the q4 geometry
-  constexpr int CB = Format<FB>::kChunkBytes;
+  constexpr bool WIDE = BITS == 5 || BITS == 6;
+  constexpr int FB = BITS == 8 ? 8 : 4;  // NVFP4, q5 and q6 chunks have the q4 geometry
+  constexpr int CB = WIDE ? Wide<WIDE ? BITS : 5>::kChunkBytes : Format<FB>::kChunkBytes;
   constexpr int KC = Format<FB>::kKPerChunk;
   const int gi = lane >> 2, ti = lane & 3;
   const int C = ep->C;  // the entry's other fields are read where they are used, not held in registers
   const int bpt = C / U;
   // this lane's B fragment in the slot's activation slice: row min(gi, M-1)
   // (columns >= M only feed outputs that are never stored), 8 values at 8 ti
-  const uint32_t xlane = StreamSlot<SU, M>::kWeightBytes + ((gi < M ? gi : M - 1) * KC + 8 * ti) * 2;
+  const uint32_t xlane = StreamSlot<SU, M, FC>::kWeightBytes + ((gi < M ? gi : M - 1) * KC + 8 * ti) * 2;
   r = static_cast<int>(floor_div(lb0, bpt));
   c = static_cast<int>(lb0 - static_cast<long long>(r) * bpt) * U;
   for (long long i = 0; i < nblk; ++i) {
@@ -587,9 +605,13 @@ __device__ __forceinline__ bool stream_segment(const StackParams& sp, const Stac
       const uint4 xb = FB == 4 ? lds128(stage + xlane + j * M * KC * 2 + 64) : make_uint4(0, 0, 0, 0);
       cr.codes[0] = lds128(stage + j * CB + 16 * lane);
       cr.codes[1] = lds128(stage + j * CB + kHalfBytes + 16 * lane);
+      uint4 hi = make_uint4(0u, 0u, 0u, 0u);
       if (NV) {
         const uint2 s2 = lds64(stage + j * CB + kCodeBytes + 8 * (2 * gi + (ti >> 1)));
         cr.scales = make_uint4(s2.x, s2.y, 0u, 0u);
+      } else if (WIDE) {
+        hi = wide_load_hi<WIDE ? BITS : 5>(stage + j * CB, lane);
+        cr.scales = lds128(stage + j * CB + Wide<WIDE ? BITS : 5>::kScaleBase + 16 * gi);
       } else if (BITS == 4) {
         cr.scales = lds128(stage + j * CB + kCodeBytes + 16 * gi);
       } else {
@@ -607,6 +629,8 @@ __device__ __forceinline__ bool stream_segment(const StackParams& sp, const Stac
       }
       if (NV) {
         nvfp4_chunk_mac<F16>(acc, cr.codes, make_uint2(cr.scales.x, cr.scales.y), xa, xb);
+      } else if (WIDE) {
+        wide_chunk_mac<WIDE ? BITS : 5, F16>(acc, cr.codes, hi, cr.scales, xa, xb);
       } else if (BITS == 4) {  // stream mode has whole q4 chunks only (K % 64 == 0, checked on the host)
         q4_chunk_mac<F16>(acc, cr, xa, xb);
       } else {
@@ -634,12 +658,13 @@ __device__ __forceinline__ bool stream_segment(const StackParams& sp, const Stac
 }
 
 // SU: chunks per stage and per stream-K block (2 or 4; every product's
-// chunks per tile is a multiple of SU, checked on the host).  NV: the list
-// holds NVFP4 products (their segment is compiled only into this instance,
-// so lists of q4 / q8 products run the code without it).
-template <int M, int NW, int D, int SU, bool NV>
+// chunks per tile is a multiple of SU, checked on the host).  FC: the list's
+// format class (FormatClass): the NVFP4 and q5 / q6 segments are compiled
+// only into the instances whose lists hold them, so lists of q4 / q8 products
+// run the code without them.
+template <int M, int NW, int D, int SU, int FC>
 __global__ void __launch_bounds__(NW * 32, 1) stream_kernel(const StackParams sp) {
-  constexpr int SLOT = StreamSlot<SU, M>::kBytes;
+  constexpr int SLOT = StreamSlot<SU, M, FC>::kBytes;
   extern __shared__ __align__(128) unsigned char smem[];
 
   const int lane = threadIdx.x & 31;
@@ -667,7 +692,7 @@ __global__ void __launch_bounds__(NW * 32, 1) stream_kernel(const StackParams sp
     return;
   }
   const int e0 = entry_of_block(sp, gb);
-  StreamProducer<SU, M> pr;
+  StreamProducer<SU, M, FC> pr;
   pr.left_total = ge - gb;
   pr.enter(sp, e0, gb - sp.entries[e0].blk_off);
   // the first stages' weights now; their activation slices once the
@@ -685,8 +710,8 @@ __global__ void __launch_bounds__(NW * 32, 1) stream_kernel(const StackParams sp
 #pragma unroll
   for (int s = 0; s < D; ++s) {
     if (s < rg.in_flight)
-      bulk_copy_x_if(lane == 0, rg.ring + s * SLOT + StreamSlot<SU, M>::kWeightBytes, x_later[s], x_later_bytes[s],
-                     rg.bars + 8 * s);
+      bulk_copy_x_if(lane == 0, rg.ring + s * SLOT + StreamSlot<SU, M, FC>::kWeightBytes, x_later[s],
+                     x_later_bytes[s], rg.bars + 8 * s);
   }
 
   float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
@@ -703,22 +728,32 @@ __global__ void __launch_bounds__(NW * 32, 1) stream_kernel(const StackParams sp
     const long long n = in_entry < left ? in_entry : left;
     const XInfo xi = *ep->xinfo;  // written by xprep_kernel, complete once griddepcontrol.wait returned
     scale = xi.ok ? xi.scale : 1.f;
-    if (NV && ep->bits == kFmtNvfp4) {
+    if (FC >= 1 && ep->bits == kFmtNvfp4) {
       scale *= *reinterpret_cast<const float*>(ep->packed + ep->TC * Format<4>::kChunkBytes);  // t
-      ok = xi.ok ? stream_segment<kFmtNvfp4, M, D, SU, true>(sp, ep, e, lb, n, gb, rg, pr, policy, scale, acc, pw,
-                                                             e_first, r_first, r, c, lane)
-                 : stream_segment<kFmtNvfp4, M, D, SU, false>(sp, ep, e, lb, n, gb, rg, pr, policy, scale, acc, pw,
-                                                              e_first, r_first, r, c, lane);
+      ok = xi.ok ? stream_segment<kFmtNvfp4, M, D, SU, true, FC>(sp, ep, e, lb, n, gb, rg, pr, policy, scale, acc,
+                                                                 pw, e_first, r_first, r, c, lane)
+                 : stream_segment<kFmtNvfp4, M, D, SU, false, FC>(sp, ep, e, lb, n, gb, rg, pr, policy, scale, acc,
+                                                                  pw, e_first, r_first, r, c, lane);
+    } else if (FC == 2 && ep->bits == 5) {
+      ok = xi.ok ? stream_segment<5, M, D, SU, true, FC>(sp, ep, e, lb, n, gb, rg, pr, policy, scale, acc, pw,
+                                                         e_first, r_first, r, c, lane)
+                 : stream_segment<5, M, D, SU, false, FC>(sp, ep, e, lb, n, gb, rg, pr, policy, scale, acc, pw,
+                                                          e_first, r_first, r, c, lane);
+    } else if (FC == 2 && ep->bits == 6) {
+      ok = xi.ok ? stream_segment<6, M, D, SU, true, FC>(sp, ep, e, lb, n, gb, rg, pr, policy, scale, acc, pw,
+                                                         e_first, r_first, r, c, lane)
+                 : stream_segment<6, M, D, SU, false, FC>(sp, ep, e, lb, n, gb, rg, pr, policy, scale, acc, pw,
+                                                          e_first, r_first, r, c, lane);
     } else if (ep->bits == 4) {
-      ok = xi.ok ? stream_segment<4, M, D, SU, true>(sp, ep, e, lb, n, gb, rg, pr, policy, scale, acc, pw, e_first,
-                                                     r_first, r, c, lane)
-                 : stream_segment<4, M, D, SU, false>(sp, ep, e, lb, n, gb, rg, pr, policy, scale, acc, pw,
-                                                      e_first, r_first, r, c, lane);
+      ok = xi.ok ? stream_segment<4, M, D, SU, true, FC>(sp, ep, e, lb, n, gb, rg, pr, policy, scale, acc, pw,
+                                                         e_first, r_first, r, c, lane)
+                 : stream_segment<4, M, D, SU, false, FC>(sp, ep, e, lb, n, gb, rg, pr, policy, scale, acc, pw,
+                                                          e_first, r_first, r, c, lane);
     } else {
-      ok = xi.ok ? stream_segment<8, M, D, SU, true>(sp, ep, e, lb, n, gb, rg, pr, policy, scale, acc, pw, e_first,
-                                                     r_first, r, c, lane)
-                 : stream_segment<8, M, D, SU, false>(sp, ep, e, lb, n, gb, rg, pr, policy, scale, acc, pw,
-                                                      e_first, r_first, r, c, lane);
+      ok = xi.ok ? stream_segment<8, M, D, SU, true, FC>(sp, ep, e, lb, n, gb, rg, pr, policy, scale, acc, pw,
+                                                         e_first, r_first, r, c, lane)
+                 : stream_segment<8, M, D, SU, false, FC>(sp, ep, e, lb, n, gb, rg, pr, policy, scale, acc, pw,
+                                                          e_first, r_first, r, c, lane);
     }
     if (!ok) break;
     left -= n;

@@ -65,7 +65,11 @@ def _ptr(a: np.ndarray) -> int:
 
 
 def weights(bits: int, seed: int, stream: int, K: int, row0: int, nrows: int) -> np.ndarray:
-    """Canonical quantised weights for rows [row0, row0+nrows) of a tensor with K columns."""
+    """Canonical quantised weights for rows [row0, row0+nrows) of a tensor with K columns.
+    q5 / q6 (int8 [nrows][K] in [-16, 15] / [-32, 31]): the q8 codes of the
+    same stream shifted right by 3 / 2 (arithmetic)."""
+    if bits in (5, 6):
+        return weights(8, seed, stream, K, row0, nrows) >> np.int8(8 - bits)
     if bits == 4:
         out = np.empty((nrows, K // 2), dtype=np.uint8)
         rc = lib().synth_q4(seed, stream, K, row0, nrows, _ptr(out))
@@ -204,6 +208,14 @@ def _stream(stream) -> int:
     return stream if isinstance(stream, int) else stream.cuda_stream
 
 
+class _null_ctx:
+    def __enter__(self):
+        return None
+
+    def __exit__(self, *a):
+        return False
+
+
 def _dev_check(rc: int, what: str) -> None:
     if rc != 0:
         raise RuntimeError(f"synth {what}: {'bad arguments' if rc == -1 else 'CUDA launch failed'}")
@@ -216,6 +228,12 @@ def weights_device(bits: int, seed: int, stream_id: int, K: int, row0: int, nrow
         raise ValueError("output tensor too small")
     fn = lib().synth_q4_device if bits == 4 else lib().synth_q8_device
     _dev_check(fn(seed, stream_id, K, row0, nrows, _dev(out), _stream(stream)), "weights")
+    if bits in (5, 6):  # the q8 codes shifted right (arithmetic), as weights() does on the host
+        import torch
+
+        with torch.cuda.stream(stream) if stream is not None else _null_ctx():
+            v = out.view(torch.int8)[:expect]
+            v.copy_(torch.bitwise_right_shift(v, 8 - bits))
 
 
 def scales_device(seed: int, stream_id: int, K: int, row0: int, nrows: int, out, std: float = SCALE_STD,

@@ -14,7 +14,8 @@ post, part four).
 Algorithmic weight bytes per tensor: N*K/2 + 2*N*K/32 (q4) and
 N*K + 2*N*K/32 (q8): the integer codes plus one fp16 scale per group of 32.
 NVFP4 tensors (bits = NVFP4) hold N*K/2 code bytes plus one E4M3 byte per 16
-values, N*K/16: the same 4.5 bits per weight as q4.
+values, N*K/16: the same 4.5 bits per weight as q4.  q5 and q6 tensors hold
+N*K*5/8 or N*K*6/8 code bytes plus the fp16 scales.
 """
 from __future__ import annotations
 
@@ -33,7 +34,7 @@ def weight_bytes(bits: int, N: int, K: int) -> int:
     """Algorithmic bytes of one N x K tensor (codes + scales)."""
     if bits == NVFP4:
         return N * K // 2 + N * (K // 16)
-    codes = N * K // 2 if bits == 4 else N * K
+    codes = N * K * bits // 8  # q4, q5, q6, q8
     return codes + 2 * N * (K // 32)
 
 
@@ -100,6 +101,12 @@ def decode_stream(fused: bool = True) -> list[Tensor]:
     return out
 
 
+def as_width(tensors: list[Tensor], bits: int) -> list[Tensor]:
+    """The same list with every q4 tensor at another width (5 or 6 bits; the
+    q8 tensors kept)."""
+    return [Tensor(t.name, bits, t.N, t.K, t.tensor_id) if t.bits == 4 else t for t in tensors]
+
+
 def as_nvfp4(tensors: list[Tensor]) -> list[Tensor]:
     """The same list with every q4 tensor in NVFP4 instead (q8 tensors kept):
     the same shapes and the same weight bytes."""
@@ -138,13 +145,13 @@ class DeviceStream:
         self.M = M
         self.seed = seed
         dev = torch.device("cuda")
-        max_canon = max((t.N * (t.K if t.bits == 8 else t.K // 2) for t in self.tensors), default=0)
+        max_canon = max((t.N * (t.K // 2 if t.bits in (4, NVFP4) else t.K) for t in self.tensors), default=0)
         max_scales = max((t.N * (t.K // 16 if t.bits == NVFP4 else t.K // 32 * 2) for t in self.tensors), default=0)
         canon = torch.empty(max(max_canon, 16), dtype=torch.uint8, device=dev)
         scales = torch.empty(max(max_scales, 16), dtype=torch.uint8, device=dev)
         self.packed = []
         for t in self.tensors:
-            nq = t.N * (t.K if t.bits == 8 else t.K // 2)
+            nq = t.N * (t.K // 2 if t.bits in (4, NVFP4) else t.K)
             if t.bits == NVFP4:  # codes from the q4 code stream, E4M3 scales from the scale stream
                 ns = t.N * (t.K // 16)
                 synth.weights_device(4, seed, synth.weight_stream(t.tensor_id), t.K, 0, t.N, canon[:nq])

@@ -66,6 +66,22 @@
  *       u = q + 128 of row (b odd ? R' : R), column 32c + 8ti + 4e + 2f + (b>>1).
  *       Scales (at byte 1024): 8 entries of 8 bytes; entry gi holds s(r, c)
  *       at position 2h + up for r = 32t + 16h + gi + 8up.
+ *   q5 / q6 (bits = 5, 6; K % 64 == 0; canonical codes int8 [N][K] with q in
+ *       [-16, 15] / [-32, 31]; a width between q4 and q8 for tensors that
+ *       need more precision, as the bs178 post's recipe upgrades some tensors
+ *       to 5 and 6 bits): the q4 chunk geometry, CB = 1408 (q5) or 1664 (q6).
+ *       u = q + 16 (q5) or q + 32 (q6).  The code blocks hold the low nibble
+ *       u & 15 at the q4 nibble's place.  The high bits u >> 4 of lane L's
+ *       values follow at byte 1024: q5, 8 bytes at 1024 + 8L (32-bit word h
+ *       for half h); q6, 16 bytes at 1024 + 16L (word 2h + (j >> 1)).  The
+ *       value in nibble i of code word j (tensor-core register r = i & 3,
+ *       half-word e = i >> 2) has its high bit(s) at bit
+ *         16e + S + (r odd ? 8 : 4),
+ *       S = {-4, -3, -2, -1, 4, 5, 6, 7}[2j + (r >> 1)] (q5, one bit) or
+ *       S = {-4, -2, 4, 6}[2 (j & 1) + (r >> 1)] (q6, two bits), so one shift
+ *       of the word by S brings a register pair's bits to the mantissa bits
+ *       the decode needs.  Scales: the q4 placement, at byte 1280 (q5) or 1536
+ *       (q6).  q5 / q6 products run in stream-mode stacks.
  *   Padding rows (>= N) and padding groups (>= K/32) hold q = 0 and scale 0.
  *   This places, for one warp, exactly the operands of bf16 m16n8k16 tensor-core
  *   products: slot L of block h is lane L's A fragment for the 16-row half h,
@@ -101,8 +117,9 @@ extern "C" {
 /* Message of the last failing call on this thread ("" if none). */
 Q4_API const char* q4_last_error(void);
 
-/* Bytes of the packed layout for an N x K tensor of `bits` (4 or 8); 0 when
- * bits is not 4 or 8, N or K is negative, or K % 32 != 0.
+/* Bytes of the packed layout for an N x K tensor of `bits` (4, 5, 6 or 8); 0
+ * when bits is not one of them, N or K is negative, K % 32 != 0, or (5 and 6
+ * bits) K % 64 != 0.
  * Weight-stream bytes are the algorithmic N*K/2 + N*K/16 (q4) or
  * N*K + N*K/16 (q8); the packed size adds only the row and group padding. */
 Q4_API size_t q4_packed_bytes(int bits, int64_t N, int64_t K);
@@ -112,7 +129,9 @@ Q4_API size_t q4_packed_bytes(int bits, int64_t N, int64_t K);
  * scales [N][K/32]; writes the packed layout into `out` (out_bytes >=
  * q4_packed_bytes).  A pure byte and bit permutation plus the q -> q+8 / q+128
  * offset; bit-exact inverse: q4_unpack_weights.  The same call packs q8
- * (bits = 8).  Errors: INVALID_ARG, SHAPE, BUFFER_TOO_SMALL. */
+ * (bits = 8) and q5 / q6 (bits = 5, 6: canonical int8 [N][K]; a code outside
+ * the width's range is INVALID_ARG).  Errors: INVALID_ARG, SHAPE,
+ * BUFFER_TOO_SMALL. */
 Q4_API int q4_pack_weights(int bits, const void* canon_q, const uint16_t* scales_fp16, int64_t N, int64_t K,
                            void* out, size_t out_bytes);
 

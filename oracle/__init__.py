@@ -76,9 +76,25 @@ def _c(a: np.ndarray, dtype) -> np.ndarray:
     return np.ascontiguousarray(a, dtype=dtype)
 
 
+_WIDE_RANGE = {5: 16, 6: 32}  # q5 / q6: int8 codes in [-r, r - 1]
+
+
+def _narrow(bits: int, q: np.ndarray) -> int:
+    """q5 and q6 codes are int8 [N][K] like q8's, in a narrower range; the
+    definition (s * q * x summed) is the same, so they take the q8 routine."""
+    if bits in _WIDE_RANGE:
+        r = _WIDE_RANGE[bits]
+        qa = np.asarray(q)
+        if qa.size and (qa.min() < -r or qa.max() > r - 1):
+            raise ValueError(f"q{bits} codes must lie in [{-r}, {r - 1}]")
+        return 8
+    return bits
+
+
 def gemv(bits: int, q: np.ndarray, s: np.ndarray, x: np.ndarray) -> tuple[np.ndarray, np.ndarray]:
     """(y, B) in fp64, each [M][N], for canonical q ([N][K/2] uint8 or [N][K] int8),
     fp16-bit scales s [N][K/32] and bf16-bit activations x [M][K]."""
+    bits = _narrow(bits, q)
     x = _c(np.atleast_2d(x), np.uint16)
     M, K = x.shape
     N = q.shape[0]
@@ -100,6 +116,7 @@ def gemv(bits: int, q: np.ndarray, s: np.ndarray, x: np.ndarray) -> tuple[np.nda
 
 def dequantize(bits: int, q: np.ndarray, s: np.ndarray) -> np.ndarray:
     """Dense W[n][k] = s[n][k/32] * q[n][k] as fp64."""
+    bits = _narrow(bits, q)
     N = q.shape[0]
     K = s.shape[1] * 32
     q = _c(q, np.uint8 if bits == 4 else np.int8)

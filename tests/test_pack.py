@@ -61,14 +61,15 @@ def test_sizes_equal_algorithmic_bytes_without_padding():
 
 
 def test_invalid_arguments():
-    assert q4.q4_packed_bytes(5, 16, 32) == 0
+    assert q4.q4_packed_bytes(5, 16, 32) == 0  # 5 bits need K % 64 == 0
+    assert q4.q4_packed_bytes(7, 16, 64) == 0
     assert q4.q4_packed_bytes(4, 16, 48) == 0
     assert q4.q4_packed_bytes(4, -1, 32) == 0
     q, s = synth.tensor(4, 0, 1, 16, 64)
     lib = q4.lib()
     out = np.zeros(100, dtype=np.uint8)
     assert lib.q4_pack_weights(4, q.ctypes.data, s.ctypes.data, 16, 64, out.ctypes.data, out.size) == q4.Q4_ERR_BUFFER_TOO_SMALL
-    assert lib.q4_pack_weights(6, q.ctypes.data, s.ctypes.data, 16, 64, out.ctypes.data, out.size) == q4.Q4_ERR_INVALID_ARG
+    assert lib.q4_pack_weights(7, q.ctypes.data, s.ctypes.data, 16, 64, out.ctypes.data, out.size) == q4.Q4_ERR_INVALID_ARG
     assert lib.q4_pack_weights(4, q.ctypes.data, s.ctypes.data, 16, 40, out.ctypes.data, out.size) == q4.Q4_ERR_SHAPE
     assert lib.q4_pack_weights(4, None, s.ctypes.data, 16, 64, out.ctypes.data, out.size) == q4.Q4_ERR_INVALID_ARG
     assert "null" in q4.q4_last_error()

@@ -14,7 +14,8 @@ through the public API ("e2e"), the roofline of the dominant kernel, the CPU
 oracle's rate ("cpu_baseline"), the SM clock under load, "chain" (the same
 products as a dependent chain with the residual + RMSNorm and SwiGLU steps
 between them, M = 1 and 4), "nvfp4" (the same stream with its 4-bit tensors
-in NVFP4, the same bytes, M = 1 and 4), "spec" (one MTP speculative step:
+in NVFP4, the same bytes, M = 1 and 4), "widths" (the same with its 4-bit
+tensors at 5 and 6 bits), "spec" (one MTP speculative step:
 three mapped-vocabulary drafts, the M = 4 pass and the keep / reject step),
 and "per_config":
 microseconds per product of the single-tensor configurations (q4 4096 x 4096,
@@ -482,25 +483,32 @@ def run_ours(args, d: Dist):
     del st4
     torch.cuda.empty_cache()
 
-    # the same stream with its 4-bit tensors in NVFP4 (E2M1 codes, E4M3 block
-    # scales of 16, fp32 tensor scale): the same shapes and weight bytes
-    nvfp4 = {}
+    # the same stream with its 4-bit tensors in other formats: NVFP4 (E2M1
+    # codes, E4M3 block scales of 16, fp32 tensor scale; the same bytes) and
+    # q5 / q6 (more bytes per weight)
+    def format_stream(fmt_tensors):
+        fb = workloads.total_bytes(fmt_tensors)
+        res = {"weight_bytes_per_step": fb}
+        for M in (1, 4):
+            sn = workloads.DeviceStream(fmt_tensors, M, seed=args.seed, flags=q4.Q4_STACK_INDEPENDENT)
+            for _ in range(args.warmup):
+                sn.run()
+            d.barrier()
+            n_f = max(3, args.steps // 2)
+            ms_f = d.max(time_region(torch, sn.run, n_f, stream) / n_f)
+            sn.check()
+            res[f"M{M}"] = {"value": round(fb * d.world / (ms_f * 1e6), 1), "unit": UNIT,
+                            "ms_per_step": round(ms_f, 5), "pct_of_hbm_peak": round(100 * fb / (ms_f * 1e6) / peak, 2),
+                            "tok_per_s": round(1000.0 / ms_f, 1), "launches": sn.stack.launches()}
+            sn.close()
+            del sn
+            torch.cuda.empty_cache()
+        return res
+
     nv_tensors = workloads.as_nvfp4(tensors)
     assert workloads.total_bytes(nv_tensors) == wbytes
-    for M in (1, 4):
-        sn = workloads.DeviceStream(nv_tensors, M, seed=args.seed, flags=q4.Q4_STACK_INDEPENDENT)
-        for _ in range(args.warmup):
-            sn.run()
-        d.barrier()
-        n_nv = max(3, args.steps // 2)
-        ms_nv = d.max(time_region(torch, sn.run, n_nv, stream) / n_nv)
-        sn.check()
-        nvfp4[f"M{M}"] = {"value": round(wbytes * d.world / (ms_nv * 1e6), 1), "unit": UNIT,
-                          "ms_per_step": round(ms_nv, 5), "pct_of_hbm_peak": round(100 * wbytes / (ms_nv * 1e6) / peak, 2),
-                          "tok_per_s": round(1000.0 / ms_nv, 1), "launches": sn.stack.launches()}
-        sn.close()
-        del sn
-        torch.cuda.empty_cache()
+    nvfp4 = format_stream(nv_tensors)
+    widths = {f"q{b}": format_stream(workloads.as_width(tensors, b)) for b in (5, 6)}
 
     # the dependent chain: the same products with the steps between them
     # (residual + RMSNorm, SwiGLU), one CUDA graph with programmatic dependent launch
@@ -589,6 +597,7 @@ def run_ours(args, d: Dist):
         },
         "chain": chain,
         "nvfp4": nvfp4,
+        "widths": widths,
         "spec": spec,
         "per_config": configs,
         "gpu_launches": n_launch * args.steps,

@@ -287,8 +287,8 @@ def test_unsupported_modes_are_refused(q4, cuda_device):
 @pytest.mark.gpu
 @pytest.mark.parametrize("bits,M", [(5, 1), (6, 1), (6, 4)])
 def test_full_decode_stream_at_other_widths_sampled(q4, cuda_device, bits, M):
-    """The 64-layer decode stream with its q4 tensors at 5 or 6 bits (15.5 /
-    17.4 GB) in one stream-mode launch; sampled rows against the oracle."""
+    """The 64-layer decode stream with its q4 tensors at 5 or 6 bits (16.3 /
+    18.8 GB) in one stream-mode launch; sampled rows against the oracle."""
     torch = _torch()
     import gpu_helpers as H
 

@@ -44,6 +44,17 @@ std::atomic<unsigned long long> g_timeout_ns{kDefaultTimeoutNs};
 #ifndef Q4_TUNE_RING_CHUNKS
 #define Q4_TUNE_RING_CHUNKS 4
 #endif
+// Split-tile width of a single product: each warp takes at least
+// Q4_TUNE_MIN_BLOCKS stream-K blocks (fewer warps share each tile, so the
+// split-tile fix-up reduces fewer partials) as long as that still leaves
+// Q4_TUNE_MIN_WARPS_PER_SM warps per SM; smaller products keep one block per
+// warp and their parallelism.
+#ifndef Q4_TUNE_MIN_BLOCKS
+#define Q4_TUNE_MIN_BLOCKS 4
+#endif
+#ifndef Q4_TUNE_MIN_WARPS_PER_SM
+#define Q4_TUNE_MIN_WARPS_PER_SM 8
+#endif
 #ifndef Q4_TUNE_MAX_U
 #define Q4_TUNE_MAX_U 2
 #endif
@@ -171,6 +182,15 @@ int chunk_bytes_of(int bits) {
 
 long long max_warps(const DeviceInfo& dev) { return static_cast<long long>(dev.sms) * kCtasPerSm * kNW; }
 
+// Warps that split one product of TB stream-K blocks (the single-product
+// kernel and, per product, the ordered persistent kernel, so their outputs
+// stay bitwise equal): at most `most`, at least Q4_TUNE_MIN_BLOCKS blocks per
+// warp while that leaves Q4_TUNE_MIN_WARPS_PER_SM warps per SM.
+long long product_warps(long long TB, long long most, const DeviceInfo& dev) {
+  const long long floor_warps = std::min(TB, static_cast<long long>(dev.sms) * Q4_TUNE_MIN_WARPS_PER_SM);
+  return std::min(most, std::max(TB / Q4_TUNE_MIN_BLOCKS, floor_warps));
+}
+
 // Workspace layout: [status word | partial sums | tile counters].  The
 // partial-sum region has one fixed size per device (M = 4 worst case), so the
 // counters sit at the same offset for every shape and M: one zero-filled
@@ -264,8 +284,7 @@ int prepare(int bits, const void* packed, int64_t N, int64_t K, const uint16_t* 
 
   const int U = pick_u(s.C);
   const bool xs = stage_x(bits, U, M, s.K);
-  long long P = max_warps(dev);
-  if (P > s.TC / U) P = s.TC / U;
+  const long long P = product_warps(s.TC / U, max_warps(dev), dev);
   const int G = static_cast<int>((P + kNW - 1) / kNW);
   unsigned char* ws = static_cast<unsigned char*>(workspace);
 
@@ -707,8 +726,7 @@ int create_persistent(const q4_stack_entry* entries, int n, int M, int su, const
     if (reinterpret_cast<uintptr_t>(en.packed) % 16 || reinterpret_cast<uintptr_t>(en.x) % 16 ||
         reinterpret_cast<uintptr_t>(en.y) % 4)
       return fail(Q4_ERR_ALIGN, "%s: packed and x must be 16-byte aligned, y 4-byte aligned", who);
-    long long P = warps;
-    if (P > s.TC / q4k::kStackU) P = s.TC / q4k::kStackU;
+    const long long P = product_warps(s.TC / q4k::kStackU, warps, dev);
     q4k::StackEntryDev& d = host[static_cast<size_t>(i)];
     d.packed = static_cast<const uint8_t*>(en.packed);
     d.x = en.x;

@@ -240,8 +240,12 @@ int smem_bytes(int bits, int U, int M, long long K, bool xs) {
   return base + (xs ? static_cast<int>(M * q4k::x_row_stride_bytes(K)) : 0);
 }
 
+#ifndef Q4_TUNE_STAGE_X
+#define Q4_TUNE_STAGE_X 1
+#endif
 bool stage_x(int bits, int U, int M, long long K) {
-  return static_cast<long long>(smem_bytes(bits, U, M, 0, false)) + M * q4k::x_row_stride_bytes(K) <= kSmemLimit;
+  return Q4_TUNE_STAGE_X &&
+         static_cast<long long>(smem_bytes(bits, U, M, 0, false)) + M * q4k::x_row_stride_bytes(K) <= kSmemLimit;
 }
 
 struct Launch {

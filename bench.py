@@ -3,8 +3,9 @@
 One step = one pass of the whole hot path over one decode token's weights:
 the 257 group-quantised products of a dense 27B-shaped hybrid model (64 layers
 of fused q|k|v, o, gate|up, down; the 16 attention layers' q|k|v|o and the
-output head in q8 g32, everything else q4 g32), replayed as one captured
-layer stack.  13.7 GB of packed weights are resident in HBM; x and y are small.
+output head in q8 g32, everything else q4 g32), run as one stream-mode layer
+stack: the activation preparation and one persistent kernel over all 257
+products.  13.7 GB of packed weights are resident in HBM; x and y are small.
 
 Metric: weight-stream GB/s (algorithmic weight bytes / device time per step)
 at M = 1, with % of the measured HBM peak and the implied decode tok/s; the

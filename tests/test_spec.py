@@ -473,3 +473,40 @@ def test_speculative_step_end_to_end(cuda_device):
     finally:
         sp.close()
         torch.cuda.empty_cache()
+
+
+# ---------------------------------------------------------------- C-ABI argument checks (CPU)
+def test_argument_errors_are_reported_before_any_device_work():
+    """Invalid arguments are refused by the C ABI itself (no device call):
+    draft count, temperature, sizes, null and misaligned pointers."""
+    import ctypes
+
+    import bit_weight_gemv_q4_b200 as q4
+
+    L = q4.lib()
+    buf = ctypes.create_string_buffer(64)
+    p = ctypes.addressof(buf)
+    p16 = (p + 15) // 16 * 16
+    rc = L.q4_spec_verify(p16, 100, p16, 10, p16, p16, p16, 16, 1.0, p16, p16, None)
+    assert rc == q4.Q4_ERR_INVALID_ARG and "n_draft" in q4.q4_last_error()
+    rc = L.q4_spec_verify(p16, 100, p16, 10, p16, p16, p16, 3, -1.0, p16, p16, None)
+    assert rc == q4.Q4_ERR_INVALID_ARG and "temperature" in q4.q4_last_error()
+    rc = L.q4_spec_verify(p16, 100, p16, 10, p16, p16, p16, 3, float("nan"), p16, p16, None)
+    assert rc == q4.Q4_ERR_INVALID_ARG
+    rc = L.q4_spec_verify(p16, 0, p16, 10, p16, p16, p16, 3, 1.0, p16, p16, None)
+    assert rc == q4.Q4_ERR_SHAPE
+    rc = L.q4_spec_verify(p16, 100, p16, 200, p16, p16, p16, 3, 1.0, p16, p16, None)  # n_map > V
+    assert rc == q4.Q4_ERR_SHAPE
+    rc = L.q4_spec_verify(p16, 100, None, 10, p16, p16, p16, 3, 1.0, p16, p16, None)
+    assert rc == q4.Q4_ERR_INVALID_ARG and "null" in q4.q4_last_error()
+    rc = L.q4_spec_verify(p16 + 2, 100, p16, 10, p16, p16, p16, 3, 1.0, p16, p16, None)
+    assert rc == q4.Q4_ERR_ALIGN
+    rc = L.q4_spec_draft(p16, 0, p16, 1.0, p16, p16, p16, p16, None)
+    assert rc == q4.Q4_ERR_SHAPE
+    rc = L.q4_spec_draft(p16, 10, p16, float("inf"), p16, p16, p16, p16, None)
+    assert rc == q4.Q4_ERR_INVALID_ARG
+    rc = L.q4_gather_rows_device(p16, -1, 10, p16, 5, p16, None)
+    assert rc == q4.Q4_ERR_SHAPE
+    assert L.q4_gather_rows_device(p16, 16, 10, p16, 0, p16, None) == q4.Q4_OK  # nothing to copy
+    rc = L.q4_gather_rows_device(p16, 16, 10, p16 + 1, 5, p16, None)
+    assert rc == q4.Q4_ERR_ALIGN

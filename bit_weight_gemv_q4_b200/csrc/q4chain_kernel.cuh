@@ -21,7 +21,27 @@ constexpr int kNormThreads = 1024;
 
 // One CTA per activation row m.  The sum of squares is reduced in a fixed
 // order (per-thread strided sums, a shuffle tree per warp, warps in order), so
-// it is bitwise reproducible.
+// it is bitwise reproducible.  Rows of up to kNormThreads * kNormPer values
+// keep each thread's values in registers: every load (h, y, gamma) is issued
+// at once and h is not read back, so the step costs one memory round trip
+// instead of one per value; longer rows take the same arithmetic in loops.
+constexpr int kNormPer = 8;
+
+__device__ __forceinline__ float norm_block_reduce(float ss) {
+  __shared__ float s_part[32];
+  __shared__ float s_t;
+  for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xFFFFFFFFu, ss, o);
+  if ((threadIdx.x & 31) == 0) s_part[threadIdx.x >> 5] = ss;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float t = 0.f;
+    for (int w = 0; w < static_cast<int>(blockDim.x >> 5); ++w) t += s_part[w];
+    s_t = t;
+  }
+  __syncthreads();
+  return s_t;
+}
+
 __global__ void __launch_bounds__(kNormThreads) residual_rmsnorm_kernel(float* __restrict__ h,
                                                                        const float* __restrict__ y,
                                                                        const uint16_t* __restrict__ gamma,
@@ -29,9 +49,42 @@ __global__ void __launch_bounds__(kNormThreads) residual_rmsnorm_kernel(float* _
                                                                        int set) {
   asm volatile("griddepcontrol.wait;" ::: "memory");
   asm volatile("griddepcontrol.launch_dependents;");
-  __shared__ float s_part[32];
-  __shared__ float s_r;
   const long long row = static_cast<long long>(blockIdx.x) * N;
+  if (N <= kNormThreads * kNormPer) {
+    float v[kNormPer], g[kNormPer];
+#pragma unroll
+    for (int j = 0; j < kNormPer; ++j) {
+      const int k = threadIdx.x + j * kNormThreads;
+      v[j] = 0.f;
+      g[j] = 1.f;
+      if (k < N) {
+        const float hv = set ? 0.f : h[row + k];
+        const float yv = y ? y[row + k] : 0.f;
+        v[j] = set ? yv : (y ? hv + yv : hv);
+        if (gamma) g[j] = __uint_as_float(static_cast<uint32_t>(gamma[k]) << 16);
+      }
+    }
+    float ss = 0.f;
+#pragma unroll
+    for (int j = 0; j < kNormPer; ++j) {
+      const int k = threadIdx.x + j * kNormThreads;
+      if (k < N) {
+        h[row + k] = v[j];
+        ss = fmaf(v[j], v[j], ss);
+      }
+    }
+    const float r = 1.f / sqrtf(norm_block_reduce(ss) / static_cast<float>(N) + eps);
+#pragma unroll
+    for (int j = 0; j < kNormPer; ++j) {
+      const int k = threadIdx.x + j * kNormThreads;
+      if (k < N) {
+        float o = v[j] * r;
+        if (gamma) o *= g[j];
+        x[row + k] = __bfloat16_as_ushort(__float2bfloat16_rn(o));
+      }
+    }
+    return;
+  }
   float ss = 0.f;
   for (int k = threadIdx.x; k < N; k += blockDim.x) {
     float v = set ? y[row + k] : h[row + k];
@@ -39,16 +92,7 @@ __global__ void __launch_bounds__(kNormThreads) residual_rmsnorm_kernel(float* _
     h[row + k] = v;
     ss = fmaf(v, v, ss);
   }
-  for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xFFFFFFFFu, ss, o);
-  if ((threadIdx.x & 31) == 0) s_part[threadIdx.x >> 5] = ss;
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    float t = 0.f;
-    for (int w = 0; w < static_cast<int>(blockDim.x >> 5); ++w) t += s_part[w];
-    s_r = 1.f / sqrtf(t / static_cast<float>(N) + eps);
-  }
-  __syncthreads();
-  const float r = s_r;
+  const float r = 1.f / sqrtf(norm_block_reduce(ss) / static_cast<float>(N) + eps);
   for (int k = threadIdx.x; k < N; k += blockDim.x) {
     float v = h[row + k] * r;
     if (gamma) v *= __uint_as_float(static_cast<uint32_t>(gamma[k]) << 16);

@@ -508,13 +508,17 @@ def run_ours(args, d: Dist):
 
     nv_tensors = workloads.as_nvfp4(tensors)
     assert workloads.total_bytes(nv_tensors) == wbytes
-    nvfp4 = format_stream(nv_tensors)
-    widths = {f"q{b}": format_stream(workloads.as_width(tensors, b)) for b in (5, 6)}
+    # the secondary sections run at N = 1 only: with N > 1 the line reports the
+    # headline step, M = 4, the other stack modes and e2e (replicas scale the same)
+    secondary = d.world == 1 and not args.headline_only
+    skipped = {"skipped": "measured at N = 1 only" if d.world > 1 else "--headline-only"}
+    nvfp4 = format_stream(nv_tensors) if secondary else skipped
+    widths = ({f"q{b}": format_stream(workloads.as_width(tensors, b)) for b in (5, 6)} if secondary else skipped)
 
     # the dependent chain: the same products with the steps between them
     # (residual + RMSNorm, SwiGLU), one CUDA graph with programmatic dependent launch
-    chain = {}
-    for M in (1, 4):
+    chain = {} if secondary else skipped
+    for M in ((1, 4) if secondary else ()):
         ch = workloads.DeviceChain(workloads.ChainShape(), M, seed=args.seed)
         for _ in range(3):
             ch.run()
@@ -528,12 +532,12 @@ def run_ours(args, d: Dist):
         del ch
         torch.cuda.empty_cache()
 
-    spec = spec_step(args, d, torch, q4, workloads, stream, peak)
+    spec = spec_step(args, d, torch, q4, workloads, stream, peak) if secondary else skipped
 
-    configs = None if args.no_configs else per_config(args, d, torch, q4, workloads, peak)
+    configs = None if args.no_configs or not secondary else per_config(args, d, torch, q4, workloads, peak)
 
     cpu = None
-    if d.rank == 0 and not args.no_cpu_baseline:
+    if d.rank == 0 and d.world == 1 and not args.no_cpu_baseline:  # the oracle is timed at N = 1 only
         rate, threads, desc, _ = oracle_sample_rate(args.cpu_seconds, args.seed)
         cpu = {"value": round(rate, 4), "unit": UNIT, "cores": threads, "kind": "oracle", "sample": desc}
 
@@ -735,6 +739,8 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU time of the oracle sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-configs", action="store_true", help="skip the per-configuration product timings")
+    ap.add_argument("--headline-only", action="store_true",
+                    help="skip the format, width, chain and speculative sections (as every N > 1 run does)")
     ap.add_argument("--reference-rows", type=int, default=8, help="rows per tensor per reference step")
     ap.add_argument("--profile-case", action="store_true", help="run the small ncu case and exit")
     ap.add_argument("--profile-bits", type=int, default=4)

@@ -632,6 +632,7 @@ struct q4_stack {
   q4k::XPrepJob* xprep_dev = nullptr;
   int xprep_jobs = 0;
   int xprep_ctas = 1;  // CTAs per job
+  int rx_bytes = 0;    // stream mode: resident activations' bytes (0: slices through the rings)
   int M = 1;
   void* workspace = nullptr;
   size_t workspace_bytes = 0;
@@ -668,6 +669,8 @@ void* select_stack_kernel(int M, int su, int fc) {
   static void* const ordered[4] = {stack_kernel_ptr<1>(), stack_kernel_ptr<2>(), stack_kernel_ptr<3>(),
                                    stack_kernel_ptr<4>()};
   if (su == 0) return ordered[M - 1];
+  if (fc >= 3)  // resident activations: M = 1, stages of kStreamU chunks only
+    return fc == 3 ? stream_kernel_ptr<1, kStreamU, 3>() : stream_kernel_ptr<1, kStreamU, 4>();
   if (fc == 0) return su == 2 ? StreamRow<2, 0>::at(M) : StreamRow<kStreamU, 0>::at(M);
   if (fc == 1) return su == 2 ? StreamRow<2, 1>::at(M) : StreamRow<kStreamU, 1>::at(M);
   if (su != 2 && M == 1) return stream_kernel_ptr<1, kStreamU, 2>();
@@ -676,8 +679,14 @@ void* select_stack_kernel(int M, int su, int fc) {
 
 // su: stream mode with stages of su chunks (weights + activation slice of M
 // rows), or 0 for ordered mode (weights only, stages of kStackU chunks).
-int stack_smem_bytes(int su, int M, int fc) {
+// fc 3 / 4 (resident activations): weights-only slots, one more barrier, and
+// the activation copies (rx_bytes) from the next 128-byte boundary.
+int stack_smem_bytes(int su, int M, int fc, int rx_bytes = 0) {
   const int cb = fc == 2 ? q4k::Wide<6>::kChunkBytes : q4k::Format<4>::kChunkBytes;
+  if (su != 0 && fc >= 3) {
+    const int rings = kStackNW * kStackD * su * q4k::Format<4>::kChunkBytes;
+    return (rings + kStackNW * kStackD * 8 + 8 + 127) / 128 * 128 + rx_bytes;
+  }
   const int slot = su == 0 ? q4k::kStackU * q4k::Format<4>::kChunkBytes
                            : su * (cb + M * q4k::Format<4>::kKPerChunk * 2);
   return kStackNW * kStackD * slot + kStackNW * kStackD * 8;
@@ -753,6 +762,7 @@ int create_persistent(const q4_stack_entry* entries, int n, int M, int su, const
   // ordered mode re-uses one counter per tile of the largest product; stream
   // mode keeps one per tile of every product
   const size_t counters = (static_cast<size_t>(independent ? total_tiles : max_t) * 4 + 255) / 256 * 256;
+  int rx_bytes = 0;  // stream mode with resident activations: their bytes in shared memory
   // stream mode: per distinct (x, K, format) a chunk-major copy of x and its XInfo
   std::vector<q4k::XPrepJob> jobs;
   std::vector<size_t> job_of(static_cast<size_t>(n), 0), x16_off, info_off;
@@ -792,15 +802,27 @@ int create_persistent(const q4_stack_entry* entries, int n, int M, int su, const
       jobs[k].xc = reinterpret_cast<uint16_t*>(base + x16_off[k]);
       jobs[k].info = reinterpret_cast<q4k::XInfo*>(base + info_off[k]);
     }
+    // resident activations (M = 1, classes 0 / 1, stages of kStreamU): every
+    // CTA keeps each prepared tensor in shared memory when they all fit
+    if (M == 1 && su == kStreamU && fc <= 1) {
+      int off = 0;
+      for (auto& j : jobs) {
+        j.rx_off = off;
+        off += static_cast<int>((j.K * 2 + 127) / 128 * 128);
+      }
+      if (stack_smem_bytes(su, M, fc + 3, off) <= kSmemLimit) rx_bytes = off;
+    }
     for (int i = 0; i < n; ++i) {
       const q4k::XPrepJob& j = jobs[job_of[static_cast<size_t>(i)]];
       host[static_cast<size_t>(i)].xc = j.xc;
       host[static_cast<size_t>(i)].xinfo = j.info;
+      host[static_cast<size_t>(i)].rx_off = j.rx_off;
     }
     err = cudaMalloc(&st->xprep_dev, sizeof(q4k::XPrepJob) * jobs.size());
     if (err == cudaSuccess)
       err = cudaMemcpy(st->xprep_dev, jobs.data(), sizeof(q4k::XPrepJob) * jobs.size(), cudaMemcpyHostToDevice);
     st->xprep_jobs = static_cast<int>(jobs.size());
+    st->rx_bytes = rx_bytes;
     long long most = 0;
     for (const auto& j : jobs) most = std::max(most, static_cast<long long>(M) * j.K / 8);
     st->xprep_ctas = static_cast<int>(std::max(1LL, (most + q4k::kXPrepThreads - 1) / q4k::kXPrepThreads));
@@ -809,8 +831,9 @@ int create_persistent(const q4_stack_entry* entries, int n, int M, int su, const
   if (err == cudaSuccess)
     err = cudaMemcpy(st->entries_dev, host.data(), sizeof(q4k::StackEntryDev) * host.size(), cudaMemcpyHostToDevice);
   if (err != cudaSuccess) return cuda_fail(err, "layer_stack_create: allocation");
-  st->fn = select_stack_kernel(M, su, fc);
-  st->smem = stack_smem_bytes(su, M, fc);
+  const int fc_sel = rx_bytes > 0 ? fc + 3 : fc;
+  st->fn = select_stack_kernel(M, su, fc_sel);
+  st->smem = stack_smem_bytes(su, M, fc_sel, rx_bytes);
   st->block = kStackNW * 32;
   st->grid = dev.sms;
   err = cudaFuncSetAttribute(st->fn, cudaFuncAttributeMaxDynamicSharedMemorySize, st->smem);
@@ -831,6 +854,9 @@ int create_persistent(const q4_stack_entry* entries, int n, int M, int su, const
   p.timeout_ns = g_timeout_ns.load();
   p.TBg = total_blocks;
   p.Pg = static_cast<int>(total_blocks < warps ? total_blocks : warps);
+  p.jobs = st->xprep_dev;
+  p.n_jobs = st->xprep_jobs;
+  p.rx_bytes = rx_bytes;
   st->persistent = true;
   st->launches = independent ? 2 : 1;  // stream mode: xprep_kernel + stream_kernel
   return Q4_OK;

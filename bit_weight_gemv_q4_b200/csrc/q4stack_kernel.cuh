@@ -50,6 +50,7 @@ struct XPrepJob {
   XInfo* info;
   long long K;
   int KC;
+  int rx_off;         // stream mode with resident activations: offset of xc's copy in shared memory
 };
 
 struct StackEntryDev {
@@ -62,6 +63,7 @@ struct StackEntryDev {
   long long blk_off;  // first block of this product in the concatenated sequence (stream mode)
   int T, C, bits, P, khalf;
   int tile_off;       // first counter of this product (stream mode)
+  int rx_off;         // stream mode with resident activations: its activations' offset in shared memory
 };
 
 struct StackParams {
@@ -75,6 +77,9 @@ struct StackParams {
   unsigned long long timeout_ns;
   long long TBg;        // stream mode: blocks of all products, concatenated
   int Pg;               // stream mode: warps with work
+  const XPrepJob* jobs; // stream mode with resident activations: the prepared activations to stage
+  int n_jobs;
+  int rx_bytes;         // their bytes in shared memory
 };
 
 constexpr int kStackU = 2;                                   // chunks per stage
@@ -477,7 +482,12 @@ __device__ __forceinline__ int entry_of_block(const StackParams& sp, long long g
 // fits the largest chunk among them.
 template <int FC>
 struct FormatClass {
-  static constexpr int kMaxChunkBytes = FC == 2 ? Wide<6>::kChunkBytes : Format<4>::kChunkBytes;
+  // classes 3 and 4 are classes 0 and 1 with resident activations: every CTA
+  // copies each prepared activation tensor into shared memory once, and the
+  // stages carry weights only
+  static constexpr bool kResidentX = FC >= 3;
+  static constexpr int kClass = FC >= 3 ? FC - 3 : FC;
+  static constexpr int kMaxChunkBytes = kClass == 2 ? Wide<6>::kChunkBytes : Format<4>::kChunkBytes;
 };
 
 // Chunk bytes of a stack entry's format.
@@ -489,7 +499,7 @@ __device__ __forceinline__ int entry_chunk_bytes(int bits) {
 template <int SU, int M, int FC>
 struct StreamSlot {
   static constexpr int kWeightBytes = SU * FormatClass<FC>::kMaxChunkBytes;
-  static constexpr int kXBytes = SU * M * Format<4>::kKPerChunk * 2;
+  static constexpr int kXBytes = FormatClass<FC>::kResidentX ? 0 : SU * M * Format<4>::kKPerChunk * 2;
   static constexpr int kBytes = kWeightBytes + kXBytes;
 };
 
@@ -509,8 +519,8 @@ struct StreamProducer {
   __device__ __forceinline__ void enter(const StackParams& sp, int entry, long long lb) {
     const StackEntryDev& en = sp.entries[entry];
     // NVFP4, q5 and q6 have the q4 geometry; only class 2 lists hold q5 / q6
-    const int CB = FC == 2 ? entry_chunk_bytes(en.bits)
-                           : (en.bits == 8 ? Format<8>::kChunkBytes : Format<4>::kChunkBytes);
+    const int CB = FormatClass<FC>::kClass == 2 ? entry_chunk_bytes(en.bits)
+                                                : (en.bits == 8 ? Format<8>::kChunkBytes : Format<4>::kChunkBytes);
     e = entry;
     bytes = static_cast<uint32_t>(SU * CB);
     src = en.packed + lb * SU * CB;
@@ -532,9 +542,9 @@ struct StreamProducer {
                                         int lane, bool with_x, const uint16_t** x_later, uint32_t* x_later_bytes) {
     if (left_total == 0) return false;
     if (left_entry == 0) enter(sp, e + 1, 0);
-    const uint32_t xb = x_bytes();
-    bulk_copy_g2s_x_if(lane == 0, dst, src, bytes, dst + StreamSlot<SU, M, FC>::kWeightBytes, x_src(), xb, with_x,
-                       bar, policy);
+    const uint32_t xb = FormatClass<FC>::kResidentX ? 0u : x_bytes();
+    bulk_copy_g2s_x_if(lane == 0, dst, src, bytes, dst + StreamSlot<SU, M, FC>::kWeightBytes, x_src(), xb,
+                       FormatClass<FC>::kResidentX ? false : with_x, bar, policy);
     if (!with_x) {
       *x_later = x_src();
       *x_later_bytes = xb;
@@ -556,9 +566,10 @@ __device__ __forceinline__ void scale_acc(float (&acc)[2][4], float scale) {
     for (int q = 0; q < 4; ++q) acc[h][q] *= scale;
 }
 
-// The warp's ring: D slots of one stage each, and the stage counters.
+// The warp's ring: D slots of one stage each, and the stage counters; rx:
+// the resident activations (classes 3 and 4).
 struct StreamRing {
-  uint32_t ring, bars;
+  uint32_t ring, bars, rx;
   int slot = 0;          // slot of the next stage to consume
   uint32_t phase = 0;
   int in_flight = 0;     // stages issued and not yet consumed
@@ -589,9 +600,13 @@ __device__ __forceinline__ bool stream_segment(const StackParams& sp, const Stac
   const int gi = lane >> 2, ti = lane & 3;
   const int C = ep->C;  // the entry's other fields are read where they are used, not held in registers
   const int bpt = C / U;
-  // this lane's B fragment in the slot's activation slice: row min(gi, M-1)
-  // (columns >= M only feed outputs that are never stored), 8 values at 8 ti
-  const uint32_t xlane = StreamSlot<SU, M, FC>::kWeightBytes + ((gi < M ? gi : M - 1) * KC + 8 * ti) * 2;
+  // this lane's B fragment in the slot's activation slice (or, resident, in
+  // the chunk's slice of the tensor's copy): row min(gi, M-1) (columns >= M
+  // only feed outputs that are never stored), 8 values at 8 ti
+  constexpr bool RX = FormatClass<FC>::kResidentX;
+  const uint32_t xrow = ((gi < M ? gi : M - 1) * KC + 8 * ti) * 2;
+  const uint32_t xlane = StreamSlot<SU, M, FC>::kWeightBytes + xrow;
+  const uint32_t xres = RX ? rg.rx + static_cast<uint32_t>(ep->rx_off) + xrow : 0u;
   r = static_cast<int>(floor_div(lb0, bpt));
   c = static_cast<int>(lb0 - static_cast<long long>(r) * bpt) * U;
   for (long long i = 0; i < nblk; ++i) {
@@ -601,8 +616,9 @@ __device__ __forceinline__ bool stream_segment(const StackParams& sp, const Stac
 #pragma unroll
     for (int j = 0; j < U; ++j) {
       ChunkRegs cr;
-      const uint4 xa = lds128(stage + xlane + j * M * KC * 2);
-      const uint4 xb = FB == 4 ? lds128(stage + xlane + j * M * KC * 2 + 64) : make_uint4(0, 0, 0, 0);
+      const uint32_t xaddr = RX ? xres + static_cast<uint32_t>(c + j) * (M * KC * 2) : stage + xlane + j * M * KC * 2;
+      const uint4 xa = lds128(xaddr);
+      const uint4 xb = FB == 4 ? lds128(xaddr + 64) : make_uint4(0, 0, 0, 0);
       cr.codes[0] = lds128(stage + j * CB + 16 * lane);
       cr.codes[1] = lds128(stage + j * CB + kHalfBytes + 16 * lane);
       uint4 hi = make_uint4(0u, 0u, 0u, 0u);
@@ -657,6 +673,18 @@ __device__ __forceinline__ bool stream_segment(const StackParams& sp, const Stac
   return true;
 }
 
+// Thread 0 of a CTA: every prepared activation tensor of the list into its
+// place in shared memory, completing on xbar (armed for all their bytes).
+// Called after griddepcontrol.wait (the preparation kernel has completed).
+__device__ __forceinline__ void stage_resident_x(const StackParams& sp, uint32_t rx, uint32_t xbar) {
+  mbar_arrive_expect_tx(xbar, static_cast<uint32_t>(sp.rx_bytes));
+  for (int k = 0; k < sp.n_jobs; ++k) {
+    const XPrepJob& j = sp.jobs[k];
+    const uint32_t bytes = static_cast<uint32_t>(j.K * 2);  // M = 1: K values
+    bulk_copy_x_if(true, rx + static_cast<uint32_t>(j.rx_off), j.xc, bytes, xbar);
+  }
+}
+
 // SU: chunks per stage and per stream-K block (2 or 4; every product's
 // chunks per tile is a multiple of SU, checked on the host).  FC: the list's
 // format class (FormatClass): the NVFP4 and q5 / q6 segments are compiled
@@ -665,6 +693,8 @@ __device__ __forceinline__ bool stream_segment(const StackParams& sp, const Stac
 template <int M, int NW, int D, int SU, int FC>
 __global__ void __launch_bounds__(NW * 32, 1) stream_kernel(const StackParams sp) {
   constexpr int SLOT = StreamSlot<SU, M, FC>::kBytes;
+  constexpr bool RX = FormatClass<FC>::kResidentX;
+  static_assert(!RX || M == 1, "resident activations are staged for M = 1");
   extern __shared__ __align__(128) unsigned char smem[];
 
   const int lane = threadIdx.x & 31;
@@ -673,12 +703,19 @@ __global__ void __launch_bounds__(NW * 32, 1) stream_kernel(const StackParams sp
   StreamRing rg;
   rg.ring = smem_addr(smem + warp * D * SLOT);
   rg.bars = smem_addr(smem + NW * D * SLOT) + warp * D * 8;
+  // resident activations: one barrier after the warps' ones, the copies at the next 128-byte boundary
+  const uint32_t xbar = smem_addr(smem + NW * D * SLOT) + NW * D * 8;
+  rg.rx = smem_addr(smem) + ((NW * D * SLOT + NW * D * 8 + 8 + 127) / 128) * 128;
 
   if (lane == 0) {
     for (int s = 0; s < D; ++s) mbar_init(rg.bars + 8 * s, 1);
+    if (RX && warp == 0) mbar_init(xbar, 1);
     fence_barrier_init();
   }
-  __syncwarp();
+  if (RX)
+    __syncthreads();  // every warp waits on the activation barrier warp 0 set up
+  else
+    __syncwarp();
   const uint64_t policy = l2_evict_first_policy();
 
   long long gb = 0, ge = 0;
@@ -689,6 +726,13 @@ __global__ void __launch_bounds__(NW * 32, 1) stream_kernel(const StackParams sp
   if (ge <= gb) {
     grid_dependency_wait();
     grid_dependents_launch();
+    if (RX && warp == 0) {
+      // the copies of the resident activations are this warp's: issue them for
+      // the CTA's other warps and wait (bounded) before leaving
+      if (lane == 0) stage_resident_x(sp, rg.rx, xbar);
+      __syncwarp();
+      if (!mbar_wait_bounded(xbar, 0, sp.timeout_ns) && lane == 0) atomicOr(sp.status, kStatusTimeout);
+    }
     return;
   }
   const int e0 = entry_of_block(sp, gb);
@@ -707,11 +751,15 @@ __global__ void __launch_bounds__(NW * 32, 1) stream_kernel(const StackParams sp
 
   grid_dependency_wait();
   grid_dependents_launch();
+  if constexpr (RX) {
+    if (threadIdx.x == 0) stage_resident_x(sp, rg.rx, xbar);
+  } else {
 #pragma unroll
-  for (int s = 0; s < D; ++s) {
-    if (s < rg.in_flight)
-      bulk_copy_x_if(lane == 0, rg.ring + s * SLOT + StreamSlot<SU, M, FC>::kWeightBytes, x_later[s],
-                     x_later_bytes[s], rg.bars + 8 * s);
+    for (int s = 0; s < D; ++s) {
+      if (s < rg.in_flight)
+        bulk_copy_x_if(lane == 0, rg.ring + s * SLOT + StreamSlot<SU, M, FC>::kWeightBytes, x_later[s],
+                       x_later_bytes[s], rg.bars + 8 * s);
+    }
   }
 
   float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
@@ -723,23 +771,24 @@ __global__ void __launch_bounds__(NW * 32, 1) stream_kernel(const StackParams sp
   const StackEntryDev* __restrict__ ep = sp.entries + e;
   bool ok = true;
   float scale = 1.f;
-  while (left > 0) {
+  if (RX) ok = mbar_wait_bounded(xbar, 0, sp.timeout_ns);  // the resident activations have landed
+  while ((!RX || ok) && left > 0) {
     const long long in_entry = ep->TC / SU - lb;
     const long long n = in_entry < left ? in_entry : left;
     const XInfo xi = *ep->xinfo;  // written by xprep_kernel, complete once griddepcontrol.wait returned
     scale = xi.ok ? xi.scale : 1.f;
-    if (FC >= 1 && ep->bits == kFmtNvfp4) {
+    if (FormatClass<FC>::kClass >= 1 && ep->bits == kFmtNvfp4) {
       scale *= *reinterpret_cast<const float*>(ep->packed + ep->TC * Format<4>::kChunkBytes);  // t
       ok = xi.ok ? stream_segment<kFmtNvfp4, M, D, SU, true, FC>(sp, ep, e, lb, n, gb, rg, pr, policy, scale, acc,
                                                                  pw, e_first, r_first, r, c, lane)
                  : stream_segment<kFmtNvfp4, M, D, SU, false, FC>(sp, ep, e, lb, n, gb, rg, pr, policy, scale, acc,
                                                                   pw, e_first, r_first, r, c, lane);
-    } else if (FC == 2 && ep->bits == 5) {
+    } else if (FormatClass<FC>::kClass == 2 && ep->bits == 5) {
       ok = xi.ok ? stream_segment<5, M, D, SU, true, FC>(sp, ep, e, lb, n, gb, rg, pr, policy, scale, acc, pw,
                                                          e_first, r_first, r, c, lane)
                  : stream_segment<5, M, D, SU, false, FC>(sp, ep, e, lb, n, gb, rg, pr, policy, scale, acc, pw,
                                                           e_first, r_first, r, c, lane);
-    } else if (FC == 2 && ep->bits == 6) {
+    } else if (FormatClass<FC>::kClass == 2 && ep->bits == 6) {
       ok = xi.ok ? stream_segment<6, M, D, SU, true, FC>(sp, ep, e, lb, n, gb, rg, pr, policy, scale, acc, pw,
                                                          e_first, r_first, r, c, lane)
                  : stream_segment<6, M, D, SU, false, FC>(sp, ep, e, lb, n, gb, rg, pr, policy, scale, acc, pw,

@@ -14,7 +14,8 @@ line also reports the ordered and graph stack modes, the end-to-end step
 through the public API ("e2e"), the roofline of the dominant kernel, the CPU
 oracle's rate ("cpu_baseline"), the SM clock under load, "chain" (the same
 products as a dependent chain with the residual + RMSNorm and SwiGLU steps
-between them, M = 1 and 4), "nvfp4" (the same stream with its 4-bit tensors
+between them, M = 1 and 4 as a CUDA graph, M = 1 also as one persistent
+launch), "nvfp4" (the same stream with its 4-bit tensors
 in NVFP4, the same bytes, M = 1 and 4), "widths" (the same with its 4-bit
 tensors at 5 and 6 bits), "spec" (one MTP speculative step:
 three mapped-vocabulary drafts, the M = 4 pass and the keep / reject step),
@@ -516,16 +517,18 @@ def run_ours(args, d: Dist):
     widths = ({f"q{b}": format_stream(workloads.as_width(tensors, b)) for b in (5, 6)} if secondary else skipped)
 
     # the dependent chain: the same products with the steps between them
-    # (residual + RMSNorm, SwiGLU), one CUDA graph with programmatic dependent launch
+    # (residual + RMSNorm, SwiGLU), one CUDA graph with programmatic dependent
+    # launch (M1, M4), and at M = 1 as one persistent cooperative launch
     chain = {} if secondary else skipped
-    for M in ((1, 4) if secondary else ()):
-        ch = workloads.DeviceChain(workloads.ChainShape(), M, seed=args.seed)
+    for key, M, flags in ((("M1", 1, 0), ("M4", 4, 0), ("M1_persistent", 1, q4.Q4_CHAIN_PERSISTENT))
+                          if secondary else ()):
+        ch = workloads.DeviceChain(workloads.ChainShape(), M, seed=args.seed, flags=flags)
         for _ in range(3):
             ch.run()
         n_ch = max(3, args.steps // 4)
         ms_ch = d.max(time_region(torch, ch.run, n_ch, stream) / n_ch)
         ch.check()
-        chain[f"M{M}"] = {"value": round(wbytes * d.world / (ms_ch * 1e6), 1), "unit": UNIT,
+        chain[key] = {"value": round(wbytes * d.world / (ms_ch * 1e6), 1), "unit": UNIT,
                           "ms_per_step": round(ms_ch, 5), "pct_of_hbm_peak": round(100 * wbytes / (ms_ch * 1e6) / peak, 2),
                           "tok_per_s": round(1000.0 / ms_ch, 1), "launches": ch.stack.launches()}
         ch.close()

@@ -27,7 +27,8 @@ GEMV_SOURCES = [os.path.join(CSRC, "q4gemv.cu"), os.path.join(CSRC, "pack.cpp"),
                 os.path.join(CSRC, "spec.cu")]
 GEMV_DEPS = GEMV_SOURCES + [os.path.join(INCLUDE, "q4gemv.h"), os.path.join(CSRC, "q4gemv_kernels.cuh"),
                             os.path.join(CSRC, "q4stack_kernel.cuh"), os.path.join(CSRC, "q4chain_kernel.cuh"),
-                            os.path.join(CSRC, "q4nvfp4_kernel.cuh"), os.path.join(CSRC, "q4spec_kernel.cuh")]
+                            os.path.join(CSRC, "q4nvfp4_kernel.cuh"), os.path.join(CSRC, "q4spec_kernel.cuh"),
+                            os.path.join(CSRC, "q4wide_kernel.cuh"), os.path.join(CSRC, "q4chainp_kernel.cuh")]
 SYNTH_SOURCES = [os.path.join(CSRC, "synth.cu")]
 SYNTH_DEPS = SYNTH_SOURCES + [os.path.join(CSRC, "synth_core.h")]
 

@@ -17,6 +17,7 @@
 #include "q4gemv_kernels.cuh"
 #include "q4chain_kernel.cuh"
 #include "q4stack_kernel.cuh"
+#include "q4chainp_kernel.cuh"
 
 namespace q4 {
 
@@ -633,6 +634,11 @@ struct q4_stack {
   int xprep_jobs = 0;
   int xprep_ctas = 1;  // CTAs per job
   int rx_bytes = 0;    // stream mode: resident activations' bytes (0: slices through the rings)
+  // persistent chain (Q4_CHAIN_PERSISTENT): one cooperative chain_kernel launch
+  bool chain = false;
+  q4k::ChainParams chain_params{};
+  q4k::ChainOpDev* chain_ops_dev = nullptr;
+  q4k::ChainResid* chain_resids_dev = nullptr;
   int M = 1;
   void* workspace = nullptr;
   size_t workspace_bytes = 0;
@@ -697,6 +703,8 @@ void free_stack(q4_stack* st) {
   if (st->graph) cudaGraphDestroy(st->graph);
   if (st->entries_dev) cudaFree(st->entries_dev);
   if (st->xprep_dev) cudaFree(st->xprep_dev);
+  if (st->chain_ops_dev) cudaFree(st->chain_ops_dev);
+  if (st->chain_resids_dev) cudaFree(st->chain_resids_dev);
   if (st->workspace) cudaFree(st->workspace);
   delete st;
 }
@@ -1052,6 +1060,230 @@ extern "C" Q4_API int q4_swiglu(const float* y_gu, uint16_t* x, int64_t N, int M
                     dim3(256), args, static_cast<cudaStream_t>(stream), true, "q4_swiglu: launch");
 }
 
+namespace {
+
+// A byte range an op reads or writes (empty for a null buffer).
+struct Span {
+  uintptr_t lo = 0, hi = 0;
+  bool overlaps(const Span& o) const { return lo < hi && o.lo < o.hi && lo < o.hi && o.lo < hi; }
+};
+
+Span span_of(const void* p, long long bytes) {
+  Span sp;
+  if (p) {
+    sp.lo = reinterpret_cast<uintptr_t>(p);
+    sp.hi = sp.lo + static_cast<uintptr_t>(bytes);
+  }
+  return sp;
+}
+
+// The persistent chain: one cooperative chain_kernel launch over the whole op
+// list (M = 1).  Eligible when every product is q4 or q8 with stages of
+// kStreamU whole chunks, each step's row fits the kernel's vector passes, no
+// op overwrites a buffer an earlier op reads, no two ops write the same bytes
+// (except the residual stream, shared by RMSNorm ops), and the activation
+// buffer and the residual streams fit shared memory beside the rings.  A
+// grid barrier goes before every op that reads bytes another CTA wrote since
+// the last barrier; a product whose activations are those the CTA itself
+// just computed (the preceding step's output) or already holds reads them
+// from shared memory.  Consecutive products without a barrier alternate
+// between two split-tile partial buffers, so a barrier also goes before a
+// third.
+int create_chain_persistent(const q4_chain_op* ops, int n, int M, const DeviceInfo& dev, q4_stack* st) {
+  const char* who = "layer_chain_create (persistent)";
+  if (M != 1) return fail(Q4_ERR_UNSUPPORTED, "%s: the persistent chain runs M = 1 only", who);
+  const int G = dev.sms;
+  if (G > 32 * q4k::kChainFlagsPerLane) return fail(Q4_ERR_UNSUPPORTED, "%s: more SMs than its barrier polls", who);
+  constexpr int SU = kStreamU;
+  const long long warps = static_cast<long long>(G) * kStackNW;
+  struct Access {
+    Span r[2], w;
+    Span resid;
+  };
+  std::vector<Access> acc(static_cast<size_t>(n));
+  std::vector<q4k::StackEntryDev> entries;
+  std::vector<q4k::ChainOpDev> dops(static_cast<size_t>(n));
+  std::vector<q4k::ChainResid> resids;
+  long long total_tiles = 0;
+  long long x_max = 0;
+  int h_floats = 0;
+  for (int i = 0; i < n; ++i) {
+    const q4_chain_op& op = ops[i];
+    q4k::ChainOpDev& d = dops[static_cast<size_t>(i)];
+    d = q4k::ChainOpDev{};
+    Access& a = acc[static_cast<size_t>(i)];
+    if (op.kind == Q4_OP_PRODUCT) {
+      Shape s;
+      make_shape(op.bits, op.N, op.K, &s, who);
+      const long long need = static_cast<long long>(SU) * (op.bits == 4 ? 64 : 32);
+      if (s.N == 0 || s.K == 0 || s.K % need != 0)
+        return fail(Q4_ERR_UNSUPPORTED, "%s: op %d: products need N > 0 and K a multiple of %lld", who, i, need);
+      if (!op.packed || !op.in || !op.out || misaligned(op.packed, 16) || misaligned(op.in, 16) ||
+          misaligned(op.out, 4))
+        return fail(Q4_ERR_ALIGN, "%s: op %d: packed and in must be 16-byte aligned, out 4-byte", who, i);
+      q4k::StackEntryDev e{};
+      e.packed = static_cast<const uint8_t*>(op.packed);
+      e.x = static_cast<const uint16_t*>(op.in);
+      e.y = static_cast<float*>(op.out);
+      e.N = s.N;
+      e.K = s.K;
+      e.TC = s.TC;
+      e.T = s.T;
+      e.C = s.C;
+      e.bits = op.bits;
+      const long long TB = s.TC / SU;
+      e.P = static_cast<int>(TB < warps ? TB : warps);  // the split of a one-product stream-mode stack
+      e.tile_off = static_cast<int>(total_tiles);
+      total_tiles += s.T;
+      d.kind = q4k::kChainProduct;
+      d.entry = static_cast<int>(entries.size());
+      d.x = e.x;
+      entries.push_back(e);
+      a.r[0] = span_of(op.in, s.K * 2);
+      a.w = span_of(op.out, s.N * 4);
+      x_max = std::max(x_max, s.K);
+    } else {
+      if (op.N % 8 != 0) return fail(Q4_ERR_UNSUPPORTED, "%s: op %d: step rows must be a multiple of 8", who, i);
+      d.N = static_cast<int>(op.N);
+      d.out = static_cast<uint16_t*>(op.out);
+      d.y = static_cast<const float*>(op.in);
+      a.w = span_of(op.out, op.N * 2);
+      x_max = std::max(x_max, static_cast<long long>(op.N));
+      if (op.kind == Q4_OP_SWIGLU) {
+        d.kind = q4k::kChainSwiglu;
+        a.r[0] = span_of(op.in, op.N * 8);
+      } else {
+        d.kind = q4k::kChainRmsnorm;
+        d.set = op.bits == 1 ? 1 : 0;
+        d.gamma = static_cast<const uint16_t*>(op.packed);
+        d.resid = op.resid;
+        a.r[0] = span_of(op.in, op.N * 4);
+        a.r[1] = span_of(op.packed, op.N * 2);
+        a.resid = span_of(op.resid, op.N * 4);
+        int slot = -1;
+        for (size_t k = 0; k < resids.size(); ++k)
+          if (resids[k].h == op.resid) slot = static_cast<int>(k);
+        if (slot >= 0 && resids[static_cast<size_t>(slot)].N != op.N)
+          return fail(Q4_ERR_UNSUPPORTED, "%s: op %d: one residual stream with two lengths", who, i);
+        if (slot < 0) {
+          resids.push_back(q4k::ChainResid{op.resid, static_cast<int>(op.N), h_floats});
+          h_floats += static_cast<int>((op.N + 3) / 4 * 4);
+          slot = static_cast<int>(resids.size()) - 1;
+        }
+        d.h_off = resids[static_cast<size_t>(slot)].h_off;
+      }
+    }
+  }
+  if (entries.empty()) return fail(Q4_ERR_UNSUPPORTED, "%s: no product", who);
+  // hazards the kernel does not order
+  for (int j = 0; j < n; ++j) {
+    const Access& aj = acc[static_cast<size_t>(j)];
+    for (int i = 0; i < n; ++i) {
+      const Access& ai = acc[static_cast<size_t>(i)];
+      if (i <= j && (aj.w.overlaps(ai.r[0]) || aj.w.overlaps(ai.r[1]) || aj.resid.overlaps(ai.r[0]) ||
+                     aj.resid.overlaps(ai.r[1])))
+        return fail(Q4_ERR_UNSUPPORTED, "%s: op %d writes bytes op %d reads", who, j, i);
+      if (aj.r[0].overlaps(ai.resid) || aj.r[1].overlaps(ai.resid))
+        return fail(Q4_ERR_UNSUPPORTED, "%s: op %d reads a residual stream", who, j);
+      if (i != j && (aj.w.overlaps(ai.w) || aj.w.overlaps(ai.resid) ||
+                     (aj.resid.overlaps(ai.resid) && (aj.resid.lo != ai.resid.lo || aj.resid.hi != ai.resid.hi))))
+        return fail(Q4_ERR_UNSUPPORTED, "%s: ops %d and %d write the same bytes", who, i, j);
+    }
+  }
+  // barriers, activation sources, partial buffers
+  std::vector<Span> since;  // bytes written since the last barrier
+  const void* tag = nullptr;
+  long long tag_n = 0;
+  int products_since = 0;
+  for (int j = 0; j < n; ++j) {
+    const q4_chain_op& op = ops[j];
+    q4k::ChainOpDev& d = dops[static_cast<size_t>(j)];
+    const Access& aj = acc[static_cast<size_t>(j)];
+    const bool resident = op.kind == Q4_OP_PRODUCT && op.in == tag && op.K == tag_n;
+    bool need = false;
+    for (const Span& w : since)
+      if ((!resident && aj.r[0].overlaps(w)) || aj.r[1].overlaps(w)) need = true;
+    if (op.kind == Q4_OP_PRODUCT && products_since == 2) need = true;
+    if (need) {
+      d.barrier = 1;
+      since.clear();
+      products_since = 0;
+    }
+    if (op.kind == Q4_OP_PRODUCT) {
+      d.stage_x = resident ? 0 : 1;
+      d.pbuf = products_since;
+      ++products_since;
+      tag = op.in;
+      tag_n = op.K;
+    } else {
+      tag = op.out;
+      tag_n = op.N;
+    }
+    since.push_back(aj.w);
+  }
+  const int rings = kStackNW * kStackD * q4k::StreamSlot<SU, 1, 3>::kBytes;
+  const int x_off = (rings + kStackNW * kStackD * 8 + 127) / 128 * 128;
+  const long long h_base = x_off + (x_max * 2 + 127) / 128 * 128;
+  const long long smem = h_base + static_cast<long long>(h_floats) * 4;
+  if (smem > kSmemLimit - 1024)
+    return fail(Q4_ERR_UNSUPPORTED, "%s: activations (%lld values) and residual streams (%d floats) exceed shared "
+                                    "memory", who, x_max, h_floats);
+  // workspace: [status | partials: 2 buffers of [warps][2][32] | tile counters | barrier flags]
+  const long long pbuf_floats = warps * 2 * q4k::kTileRows;
+  const size_t partials_at = kWsHeader;
+  const size_t counters_at = partials_at + static_cast<size_t>(2 * pbuf_floats) * 4;
+  const size_t flags_at = counters_at + (static_cast<size_t>(total_tiles) * 4 + 255) / 256 * 256;
+  st->workspace_bytes = flags_at + (static_cast<size_t>(G) * 4 + 255) / 256 * 256;
+  cudaError_t err = cudaMalloc(&st->workspace, st->workspace_bytes);
+  if (err == cudaSuccess) err = cudaMemset(st->workspace, 0, st->workspace_bytes);
+  if (err == cudaSuccess) err = cudaMalloc(&st->entries_dev, sizeof(q4k::StackEntryDev) * entries.size());
+  if (err == cudaSuccess)
+    err = cudaMemcpy(st->entries_dev, entries.data(), sizeof(q4k::StackEntryDev) * entries.size(),
+                     cudaMemcpyHostToDevice);
+  if (err == cudaSuccess) err = cudaMalloc(&st->chain_ops_dev, sizeof(q4k::ChainOpDev) * dops.size());
+  if (err == cudaSuccess)
+    err = cudaMemcpy(st->chain_ops_dev, dops.data(), sizeof(q4k::ChainOpDev) * dops.size(), cudaMemcpyHostToDevice);
+  if (err == cudaSuccess && !resids.empty())
+    err = cudaMalloc(&st->chain_resids_dev, sizeof(q4k::ChainResid) * resids.size());
+  if (err == cudaSuccess && !resids.empty())
+    err = cudaMemcpy(st->chain_resids_dev, resids.data(), sizeof(q4k::ChainResid) * resids.size(),
+                     cudaMemcpyHostToDevice);
+  if (err != cudaSuccess) return cuda_fail(err, "layer_chain_create: allocation");
+  st->fn = reinterpret_cast<void*>(&q4k::chain_kernel<kStackNW, kStackD, SU>);
+  st->smem = static_cast<int>(smem);
+  st->block = kStackNW * 32;
+  st->grid = G;
+  err = cudaFuncSetAttribute(st->fn, cudaFuncAttributeMaxDynamicSharedMemorySize, st->smem);
+  if (err != cudaSuccess) return cuda_fail(err, "layer_chain_create: cudaFuncSetAttribute");
+  int per_sm = 0;
+  err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, st->fn, st->block, st->smem);
+  if (err != cudaSuccess) return cuda_fail(err, "layer_chain_create: occupancy query");
+  if (per_sm < 1) return fail(Q4_ERR_UNSUPPORTED, "%s: the chain kernel does not fit on an SM", who);
+  unsigned char* ws = static_cast<unsigned char*>(st->workspace);
+  q4k::ChainParams& p = st->chain_params;
+  p.ops = st->chain_ops_dev;
+  p.n_ops = n;
+  p.entries = st->entries_dev;
+  p.E = static_cast<int>(entries.size());
+  p.resids = st->chain_resids_dev;
+  p.n_resids = static_cast<int>(resids.size());
+  p.partials = reinterpret_cast<float*>(ws + partials_at);
+  p.pbuf_floats = pbuf_floats;
+  p.counters = reinterpret_cast<unsigned*>(ws + counters_at);
+  p.status = reinterpret_cast<unsigned*>(ws);
+  p.bar_flags = reinterpret_cast<unsigned*>(ws + flags_at);
+  p.G = G;
+  p.x_off = x_off;
+  p.h_base = static_cast<int>(h_base);
+  p.timeout_ns = g_timeout_ns.load();
+  st->chain = true;
+  st->M = 1;
+  st->launches = 1;
+  return Q4_OK;
+}
+
+}  // namespace
+
 extern "C" Q4_API int layer_chain_create(const q4_chain_op* ops, int n_ops, int M, int flags, q4_stack** out) {
   if (!out) return fail(Q4_ERR_INVALID_ARG, "layer_chain_create: out is null");
   *out = nullptr;
@@ -1068,6 +1300,17 @@ extern "C" Q4_API int layer_chain_create(const q4_chain_op* ops, int n_ops, int 
       make_shape(ops[i].bits, ops[i].N, ops[i].K, &s, "layer_chain_create");
       ws = std::max(ws, workspace_bytes(s, M, dev));
     }
+  }
+  if (flags & Q4_CHAIN_PERSISTENT) {
+    q4_stack* st = new q4_stack();
+    cudaGetDevice(&st->device);
+    rc = create_chain_persistent(ops, n_ops, M, dev, st);
+    if (rc) {
+      free_stack(st);
+      return rc;
+    }
+    *out = st;
+    return Q4_OK;
   }
   q4_stack* st = new q4_stack();
   cudaGetDevice(&st->device);
@@ -1149,6 +1392,21 @@ extern "C" Q4_API int layer_chain_create(const q4_chain_op* ops, int n_ops, int 
 extern "C" Q4_API int layer_stack_run(q4_stack* st, void* stream) {
   if (!st) return fail(Q4_ERR_INVALID_ARG, "layer_stack_run: null stack");
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (st->chain) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(st->grid);
+    cfg.blockDim = dim3(st->block);
+    cfg.dynamicSmemBytes = static_cast<size_t>(st->smem);
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeCooperative;  // its grid barriers need every CTA resident
+    attr[0].val.cooperative = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    void* args[] = {&st->chain_params};
+    cudaError_t err = cudaLaunchKernelExC(&cfg, st->fn, args);
+    return err == cudaSuccess ? Q4_OK : cuda_fail(err, "layer_stack_run: chain launch");
+  }
   if (st->persistent) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(st->grid);

@@ -583,11 +583,14 @@ struct StreamRing {
 // in acc with (r, c).  Returns false if a ring wait gave up.
 // F16: the activations are used in fp16 (en.x16).  Finished tile sums are
 // multiplied by `scale` (2^sigma when F16, times t for NVFP4).
-template <int BITS, int M, int D, int SU, bool F16, int FC>
-__device__ __forceinline__ bool stream_segment(const StackParams& sp, const StackEntryDev* __restrict__ ep, int e,
+// SP supplies timeout_ns and partials; PR refills the ring (issue), so the
+// persistent chain kernel runs the same loop with its own per-product ranges.
+template <int BITS, int M, int D, int SU, bool F16, int FC, class SP = StackParams,
+          class PR = StreamProducer<SU, M, FC>>
+__device__ __forceinline__ bool stream_segment(const SP& sp, const StackEntryDev* __restrict__ ep, int e,
                                                long long lb0,
                                                long long nblk, long long gb, StreamRing& rg,
-                                               StreamProducer<SU, M, FC>& pr, uint64_t policy, float scale,
+                                               PR& pr, uint64_t policy, float scale,
                                                float (&acc)[2][4], int pw, int& e_first, int& r_first, int& r,
                                                int& c, int lane) {
   constexpr int U = SU;

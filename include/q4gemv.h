@@ -470,8 +470,32 @@ typedef struct q4_chain_op {
   float* resid;        /* RMSNORM: residual stream h (fp32 [M][N], device); else NULL */
 } q4_chain_op;
 
+/* Q4_CHAIN_PERSISTENT (M = 1): the whole chain as ONE cooperative kernel
+ * launch instead of a graph of one kernel per op.  Every product is split
+ * between all warps of the GPU exactly as a one-product stream-mode stack
+ * splits it (its output is bitwise that stack's on the same activations);
+ * each CTA computes every step itself into its own shared-memory copy of the
+ * next product's activations, keeps the residual streams in shared memory,
+ * and writes its slice of each step's outputs; a bounded grid barrier goes
+ * before each op that reads another CTA's writes; the weight copies run
+ * ahead across ops.  The steps' outputs are bitwise those of
+ * q4_residual_rmsnorm / q4_swiglu on the same inputs.  Needs: M = 1;
+ * products q4 (K % 256 == 0) or q8 (K % 128 == 0), N > 0; steps with N % 8
+ * == 0; no op writing bytes that an earlier (or the same) op reads, no two
+ * ops writing the same bytes except RMSNorm ops sharing one residual stream
+ * (same pointer and N), no op reading a residual stream through `in`; the
+ * largest activation row and the residual streams within shared memory
+ * beside the weight rings (about 84 KB: a 17,408-value row and a 5,120-value
+ * stream fit).  Otherwise Q4_ERR_UNSUPPORTED with the reason.  A grid
+ * barrier whose wait gives up sets the status word (layer_stack_check
+ * returns Q4_ERR_TIMEOUT).  On the 64-layer decode chain it measured slower
+ * than the graph (each CTA recomputes every step over the whole row, and
+ * every step waits at a grid barrier for the slowest CTA). */
+#define Q4_CHAIN_PERSISTENT 8
+
 /* Validates the ops and captures them, in order, on the current device.
- * flags: Q4_STACK_NO_PDL launches without programmatic dependent launch.
+ * flags: Q4_STACK_NO_PDL launches without programmatic dependent launch;
+ * Q4_CHAIN_PERSISTENT as above.
  * The returned stack runs with layer_stack_run, is checked with
  * layer_stack_check and freed with layer_stack_destroy.  Errors: as
  * layer_stack_create (INVALID_ARG for an unknown kind, a null or misaligned

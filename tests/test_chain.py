@@ -221,13 +221,15 @@ def test_chain_equals_its_steps_called_one_by_one(cuda_device, M):
 
 
 @pytest.mark.gpu
-@pytest.mark.parametrize("M", [1, 2])
-def test_chain_against_the_oracle_chain(cuda_device, M):
+@pytest.mark.parametrize("M,mode", [(1, "graph"), (2, "graph"), (1, "persistent")])
+def test_chain_against_the_oracle_chain(cuda_device, M, mode):
     """A two-layer chain against the oracle's chain computed alone: the first
     activations equal the oracle's away from rounding ties, the first product
     is within the product tolerance, and the end (after nine dependent steps)
     stays within 1e-3 in relative norm."""
-    ch = workloads.DeviceChain(SMALL, M, seed=6)
+    import bit_weight_gemv_q4_b200 as q4
+
+    ch = workloads.DeviceChain(SMALL, M, seed=6, flags=q4.Q4_CHAIN_PERSISTENT if mode == "persistent" else 0)
     ch.run()
     ch.check()
     got = _outputs(ch)
@@ -265,3 +267,110 @@ def test_full_chain_runs_and_is_reproducible(cuda_device, M):
     assert np.all(np.isfinite(a)) and np.array_equal(a, b)
     ch.close()
     torch.cuda.empty_cache()
+
+
+# ---------------------------------------------------------- the one-launch chain
+@pytest.mark.gpu
+def test_persistent_chain_equals_its_ops_called_one_by_one(cuda_device):
+    """The chain as one cooperative launch (M = 1) is bitwise the same ops run
+    one call at a time on the same buffers: each product as a one-product
+    stream-mode stack (the same split and decode), each step as
+    q4_residual_rmsnorm / q4_swiglu; and two runs agree bitwise."""
+    import bit_weight_gemv_q4_b200 as q4
+
+    torch = _torch()
+    ch = workloads.DeviceChain(SMALL, 1, seed=7, flags=q4.Q4_CHAIN_PERSISTENT)
+    assert ch.stack.launches() == 1
+    ch.run()
+    ch.check()
+    one = _outputs(ch)
+    ch.run()
+    ch.check()
+    again = _outputs(ch)
+    for key in ("y", "x"):
+        assert all(np.array_equal(a, b) for a, b in zip(one[key], again[key]))
+    assert np.array_equal(one["h"], again["h"])
+    for y in ch.w.y:
+        y.fill_(float("nan"))
+    for x in ch.x_qkv + ch.x_gu + ch.x_down + [ch.x_head]:
+        x.fill_(-1)
+    ch.h.fill_(float("nan"))
+    for kind, bits, N, K, packed, inp, out, resid in ch.ops:
+        if kind == q4.Q4_OP_PRODUCT:
+            st = q4.layer_stack_create([(bits, N, K, packed, inp, out)], 1, q4.Q4_STACK_INDEPENDENT)
+            q4.layer_stack_run(st)
+            q4.layer_stack_check(st)
+            st.close()
+        elif kind == q4.Q4_OP_RESIDUAL_RMSNORM:
+            q4.q4_residual_rmsnorm(resid, inp, packed, out, N, 1, bits == 1)
+        else:
+            q4.q4_swiglu(inp, out, N, 1)
+    torch.cuda.synchronize()
+    single = _outputs(ch)
+    for i, (a, b) in enumerate(zip(one["y"], single["y"])):
+        assert np.array_equal(a, b), workloads.chain_tensors(SMALL)[i].name
+    for a, b in zip(one["x"], single["x"]):
+        assert np.array_equal(a, b)
+    assert np.array_equal(one["h"], single["h"])
+    ch.close()
+
+
+@pytest.mark.gpu
+def test_full_persistent_chain_against_the_graph_chain(cuda_device):
+    """The 64-layer chain as one launch: reproducible bitwise, and its first
+    product and its logits agree with the captured graph's (the two split and
+    decode the products differently, so they agree within rounding)."""
+    import bit_weight_gemv_q4_b200 as q4
+
+    torch = _torch()
+    ch = workloads.DeviceChain(workloads.ChainShape(), 1, flags=q4.Q4_CHAIN_PERSISTENT)
+    ch.run()
+    ch.check()
+    a = ch.logits.cpu().numpy().copy()
+    y0 = ch.w.y[0].cpu().numpy().copy()
+    ch.run()
+    ch.check()
+    assert np.all(np.isfinite(a)) and np.array_equal(a, ch.logits.cpu().numpy())
+    graph = q4.layer_chain_create(ch.ops, 1, 0)
+    q4.layer_stack_run(graph)
+    q4.layer_stack_check(graph)
+    torch.cuda.synchronize()
+    g = ch.logits.cpu().numpy().copy()
+    g0 = ch.w.y[0].cpu().numpy().copy()
+    graph.close()
+    assert np.linalg.norm(y0 - g0) <= 1e-5 * np.linalg.norm(g0)
+    rel = np.linalg.norm(a - g) / np.linalg.norm(g)
+    print("persistent vs graph logits, relative norm", rel)
+    assert rel <= 2e-2
+    ch.close()
+    torch.cuda.empty_cache()
+
+
+@pytest.mark.gpu
+def test_persistent_chain_rejects_what_it_cannot_order(cuda_device):
+    import bit_weight_gemv_q4_b200 as q4
+
+    torch = _torch()
+    ch = workloads.DeviceChain(SMALL, 1, seed=8)
+    P = q4.Q4_CHAIN_PERSISTENT
+    with pytest.raises(q4.Q4Error) as e:
+        q4.layer_chain_create(ch.ops, 2, P)
+    assert e.value.code == q4.Q4_ERR_UNSUPPORTED
+    # two ops writing one buffer
+    ops = list(ch.ops)
+    k = next(i for i, op in enumerate(ops) if op[0] == q4.Q4_OP_PRODUCT)
+    k2 = next(i for i, op in enumerate(ops) if op[0] == q4.Q4_OP_PRODUCT and i > k)
+    op2 = list(ops[k2])
+    op2[6] = ops[k][6]
+    bad = ops[:k2] + [tuple(op2)] + ops[k2 + 1:]
+    with pytest.raises(q4.Q4Error) as e:
+        q4.layer_chain_create(bad, 1, P)
+    assert e.value.code == q4.Q4_ERR_UNSUPPORTED
+    # a q4 product whose K is not a multiple of 256
+    w = torch.zeros(q4.q4_packed_bytes(4, 32, 96), dtype=torch.uint8, device="cuda")
+    x = torch.zeros(96, dtype=torch.int16, device="cuda")
+    y = torch.zeros(32, dtype=torch.float32, device="cuda")
+    with pytest.raises(q4.Q4Error) as e:
+        q4.layer_chain_create([(q4.Q4_OP_PRODUCT, 4, 32, 96, w, x, y, None)], 1, P)
+    assert e.value.code == q4.Q4_ERR_UNSUPPORTED
+    ch.close()

@@ -542,16 +542,21 @@ struct StreamProducer {
                                         int lane, bool with_x, const uint16_t** x_later, uint32_t* x_later_bytes) {
     if (left_total == 0) return false;
     if (left_entry == 0) enter(sp, e + 1, 0);
-    const uint32_t xb = FormatClass<FC>::kResidentX ? 0u : x_bytes();
-    bulk_copy_g2s_x_if(lane == 0, dst, src, bytes, dst + StreamSlot<SU, M, FC>::kWeightBytes, x_src(), xb,
-                       FormatClass<FC>::kResidentX ? false : with_x, bar, policy);
-    if (!with_x) {
-      *x_later = x_src();
-      *x_later_bytes = xb;
+    if constexpr (FormatClass<FC>::kResidentX) {
+      // the slots carry weights only; the activations are already resident
+      bulk_copy_g2s_if(lane == 0, dst, src, bytes, bar, policy);
+    } else {
+      const uint32_t xb = x_bytes();
+      bulk_copy_g2s_x_if(lane == 0, dst, src, bytes, dst + StreamSlot<SU, M, FC>::kWeightBytes, x_src(), xb, with_x,
+                         bar, policy);
+      if (!with_x) {
+        *x_later = x_src();
+        *x_later_bytes = xb;
+      }
+      cpos += SU;
+      if (cpos == C) cpos = 0;
     }
     src += bytes;
-    cpos += SU;
-    if (cpos == C) cpos = 0;
     --left_entry;
     --left_total;
     return true;
@@ -612,7 +617,8 @@ __device__ __forceinline__ bool stream_segment(const SP& sp, const StackEntryDev
   const uint32_t xres = RX ? rg.rx + static_cast<uint32_t>(ep->rx_off) + xrow : 0u;
   r = static_cast<int>(floor_div(lb0, bpt));
   c = static_cast<int>(lb0 - static_cast<long long>(r) * bpt) * U;
-  for (long long i = 0; i < nblk; ++i) {
+  const int n_stages = static_cast<int>(nblk);  // a warp's range is far below 2^31 stages
+  for (int i = 0; i < n_stages; ++i) {
     const uint32_t bar = rg.bars + 8 * rg.slot;
     if (!mbar_wait_bounded(bar, rg.phase, sp.timeout_ns)) return false;
     const uint32_t stage = rg.ring + rg.slot * SLOT;

@@ -374,3 +374,54 @@ def test_persistent_chain_rejects_what_it_cannot_order(cuda_device):
         q4.layer_chain_create([(q4.Q4_OP_PRODUCT, 4, 32, 96, w, x, y, None)], 1, P)
     assert e.value.code == q4.Q4_ERR_UNSUPPORTED
     ch.close()
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("case", ["wide_range", "huge", "zeros"])
+def test_persistent_chain_activation_ranges(cuda_device, case):
+    """Products of the one-launch chain on activations staged from global
+    memory: beyond fp16's range after any power-of-two scaling (the bf16
+    decode), far above it (scaled in exactly), all zero.  The second product
+    reads the same activations and takes them from shared memory without
+    staging them again.  Each output is within the tolerance of the oracle
+    and bitwise the one-product stream-mode stack's."""
+    import bit_weight_gemv_q4_b200 as q4
+    import gpu_helpers as H
+
+    torch = _torch()
+    K = 5120
+    x = synth.activations(6, synth.act_stream(44), 1, K)
+    xf = (x.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    if case == "wide_range":
+        xf[:, ::7] *= 2.0 ** 60
+        xf[:, 3::11] *= 2.0 ** -60
+    elif case == "huge":
+        xf *= 2.0 ** 100
+    else:
+        xf[:] = 0.0
+    x = synth.f64_to_bf16_bits(xf.ravel()).reshape(1, K)
+    x_dev = H.to_device_x(x)
+    ops, hosts, ys = [], [], []
+    for bits, N, tid in ((4, 160, 53), (8, 96, 54)):
+        q, s = synth.tensor(bits, 6, tid, N, K)
+        packed = H.to_device_packed(bits, q, s, N, K)
+        y = torch.full((N,), float("nan"), dtype=torch.float32, device="cuda")
+        ops.append((q4.Q4_OP_PRODUCT, bits, N, K, packed, x_dev, y, None))
+        hosts.append((bits, N, q, s, packed))
+        ys.append(y)
+    ch = q4.layer_chain_create(ops, 1, q4.Q4_CHAIN_PERSISTENT)
+    q4.layer_stack_run(ch)
+    q4.layer_stack_check(ch)
+    torch.cuda.synchronize()
+    for (bits, N, q, s, packed), y in zip(hosts, ys):
+        yy = y.cpu().numpy().reshape(1, N).copy()
+        if case == "zeros":
+            assert np.all(yy == 0.0)
+        H.assert_parity(yy, q, s, x, bits)
+        y2 = torch.full((N,), float("nan"), dtype=torch.float32, device="cuda")
+        st = q4.layer_stack_create([(bits, N, K, packed, x_dev, y2)], 1, q4.Q4_STACK_INDEPENDENT)
+        q4.layer_stack_run(st)
+        q4.layer_stack_check(st)
+        assert np.array_equal(yy.ravel(), y2.cpu().numpy())
+        st.close()
+    ch.close()

@@ -39,7 +39,9 @@ namespace q4k {
 constexpr int kChainProduct = 0;
 constexpr int kChainRmsnorm = 1;
 constexpr int kChainSwiglu = 2;
-constexpr int kChainFlagsPerLane = 8;  // grid barrier: one polling warp reads up to 32 x 8 CTA flags
+// The host admits grids of up to 32 x kChainFlagsPerLane CTAs (one polling
+// warp, a few flags per lane per poll; B200 has 148 SMs).
+constexpr int kChainFlagsPerLane = 8;
 
 struct ChainOpDev {
   int kind;      // kChainProduct / kChainRmsnorm / kChainSwiglu
@@ -121,18 +123,13 @@ struct ChainProducer {
   }
 };
 
-__device__ __forceinline__ unsigned ld_relaxed_gpu(const unsigned* p) {
-  unsigned v;
-  asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-  return v;
-}
-
 // Grid-wide barrier of the G resident CTAs (all threads call it).  CTA b
 // publishes `epoch` in its own flag (release store after a fence), and one
-// warp polls every flag with relaxed loads, all in flight at once; the fence
-// after the last poll makes the other CTAs' released writes visible (the
-// relaxed-load-then-fence acquire pattern).  Bounded by timeout_ns.  Returns
-// false when this CTA is aborting.
+// warp polls every flag with acquire loads.  The acquire loads of a poll
+// complete one after another, which keeps the polling rate low: the 148
+// flags share five cache lines, and polling them with every load in flight
+// at once delayed the late CTAs' arrival stores (9 % slower on the 64-layer
+// chain).  Bounded by timeout_ns.  Returns false when this CTA is aborting.
 __device__ __forceinline__ bool chain_barrier(const ChainParams& cp, unsigned epoch, volatile int* s_abort) {
   __syncthreads();
   if (threadIdx.x < 32 && !*s_abort) {
@@ -144,15 +141,8 @@ __device__ __forceinline__ bool chain_barrier(const ChainParams& cp, unsigned ep
     __syncwarp();
     const unsigned long long t0 = global_timer_ns();
     while (true) {
-      unsigned v[kChainFlagsPerLane];
-#pragma unroll
-      for (int q = 0; q < kChainFlagsPerLane; ++q) {
-        const int i = lane + 32 * q;
-        v[q] = i < cp.G ? ld_relaxed_gpu(cp.bar_flags + i) : epoch;
-      }
       bool here = true;
-#pragma unroll
-      for (int q = 0; q < kChainFlagsPerLane; ++q) here &= static_cast<int>(v[q] - epoch) >= 0;
+      for (int i = lane; i < cp.G; i += 32) here &= static_cast<int>(ld_acquire_gpu(cp.bar_flags + i) - epoch) >= 0;
       if (__all_sync(0xFFFFFFFFu, here)) break;
       const unsigned long long waited = __shfl_sync(0xFFFFFFFFu, global_timer_ns() - t0, 0);
       if (waited > cp.timeout_ns) {

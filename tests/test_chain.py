@@ -73,6 +73,22 @@ def test_chain_shape_of_the_decode_stream():
     assert workloads.chain_tensors(workloads.ChainShape()) == workloads.decode_stream(fused=True)
 
 
+def test_chain_shapes_meet_the_one_launch_conditions():
+    """The conditions include/q4gemv.h states for Q4_CHAIN_PERSISTENT (q4
+    products K % 256 == 0, q8 K % 128 == 0, step rows N % 8 == 0, the largest
+    activation row and the residual stream within the ~84 KB of shared
+    memory beside the rings) hold for the decode chain and the small one."""
+    for shape in (workloads.ChainShape(), SMALL):
+        tensors = workloads.chain_tensors(shape)
+        for t in tensors:
+            assert t.bits in (4, 8) and t.N > 0
+            assert t.K % (256 if t.bits == 4 else 128) == 0, t.name
+        assert shape.hidden % 8 == 0 and shape.ffn % 8 == 0
+        x_bytes = -(-2 * max(max(t.K for t in tensors), shape.hidden, shape.ffn) // 128) * 128
+        rings = -(-(16 * 2 * 4 * 1152 + 16 * 2 * 8) // 128) * 128  # 16 warps x 2 stages x 4 chunks, barriers
+        assert x_bytes + 4 * shape.hidden <= 227 * 1024 - 1024 - rings  # 83,712 bytes
+
+
 # ---------------------------------------------------------------- oracle chain
 def oracle_chain(shape, M, seed):
     """Every intermediate of the chain from the oracle alone (inputs from the

@@ -95,3 +95,23 @@ def test_reference_arm_runs_on_rank_zero_only():
 def test_warmup_below_three_is_refused():
     r = _run_bench(["--impl", "reference", "--steps", "1", "--warmup", "2"])
     assert r.returncode != 0
+
+
+def test_traffic_comes_only_from_a_capture_of_the_current_kernel_source(monkeypatch):
+    """roofline.traffic is the committed ncu figure while the capture's
+    source fingerprint equals the kernel sources' one, and null otherwise
+    (the figure no longer describes the kernel that runs)."""
+    import re
+
+    sys.path.insert(0, ROOT)
+    import bench
+
+    text = open(os.path.join(ROOT, "profiles", "gemv_q4_traffic.md")).read()
+    sha = re.search(r"kernel_source_sha:\s*([0-9a-f]+)", text).group(1)
+    per = int(re.search(r"dram_bytes_per_full_launch:\s*([0-9]+)", text).group(1))
+    assert per >= 13_745_029_120  # DRAM traffic cannot be below the weight bytes the launch streams
+    assert re.fullmatch(r"[0-9a-f]{16}", bench.kernel_source_sha())
+    monkeypatch.setattr(bench, "kernel_source_sha", lambda: sha)
+    assert bench.profiled_traffic() == per
+    monkeypatch.setattr(bench, "kernel_source_sha", lambda: "f" * 16 if sha != "f" * 16 else "0" * 16)
+    assert bench.profiled_traffic() is None

@@ -94,3 +94,39 @@ def test_without_a_device_gpu_calls_fail_loudly():
     with pytest.raises(q4.Q4Error):
         q4.q4_gemv_workspace_bytes(4, 16, 64, 1)
     _ = np  # numpy imported for parity with other test modules
+
+
+def test_binding_structs_match_the_c_layout(tmp_path):
+    """The ctypes structures the binding passes by pointer (q4_stack_entry,
+    q4_chain_op) have the sizes and field offsets the C compiler gives the
+    header's declarations (compiled here as C99 with gcc)."""
+    import ctypes
+    import shutil
+    import subprocess
+
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("gcc is not available")
+    cases = [
+        ("q4_stack_entry", q4.StackEntry, {"bits": "bits", "N": "N", "K": "K", "packed": "packed", "x": "x", "y": "y"}),
+        ("q4_chain_op", q4.ChainOp, {"kind": "kind", "bits": "bits", "N": "N", "K": "K", "packed": "packed",
+                                     "inp": "in", "out": "out", "resid": "resid"}),
+    ]
+    lines = ["#include <stdio.h>", "#include <stddef.h>", '#include "q4gemv.h"', "int main(void) {"]
+    for cname, _, fields in cases:
+        lines.append(f'  printf("{cname} size %zu\\n", sizeof({cname}));')
+        for cfield in fields.values():
+            lines.append(f'  printf("{cname} {cfield} %zu\\n", offsetof({cname}, {cfield}));')
+    lines += ["  return 0;", "}"]
+    src = tmp_path / "layout.c"
+    src.write_text("\n".join(lines) + "\n")
+    exe = tmp_path / "layout"
+    subprocess.run([gcc, "-std=c99", "-Wall", "-Werror", "-I", os.path.dirname(HEADER), str(src), "-o", str(exe)], check=True)
+    got = {}
+    for line in subprocess.run([str(exe)], check=True, capture_output=True, text=True).stdout.splitlines():
+        name, field, value = line.split()
+        got[(name, field)] = int(value)
+    for cname, cls, fields in cases:
+        assert ctypes.sizeof(cls) == got[(cname, "size")], cname
+        for pyfield, cfield in fields.items():
+            assert getattr(cls, pyfield).offset == got[(cname, cfield)], (cname, cfield)

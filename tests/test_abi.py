@@ -130,3 +130,42 @@ def test_binding_structs_match_the_c_layout(tmp_path):
         assert ctypes.sizeof(cls) == got[(cname, "size")], cname
         for pyfield, cfield in fields.items():
             assert getattr(cls, pyfield).offset == got[(cname, cfield)], (cname, cfield)
+
+
+def _c_category(decl: str) -> str:
+    decl = " ".join(decl.split())
+    if "*" in decl:
+        return "ptr"
+    words = [w for w in decl.split() if w != "const"]
+    if len(words) > 1 and words[-1] not in ("int", "long", "float", "double", "void"):
+        words = words[:-1]  # drop the parameter name
+    t = " ".join(words)
+    return {"int": "int", "int64_t": "i64", "uint64_t": "u64", "size_t": "u64", "unsigned long long": "u64",
+            "float": "float", "void": "void"}[t]
+
+
+def _ctypes_category(t) -> str:
+    import ctypes
+
+    if t is None:
+        return "void"
+    if t in (ctypes.c_void_p, ctypes.c_char_p) or hasattr(t, "_type_") and isinstance(t._type_, type):
+        return "ptr"
+    return {ctypes.c_int: "int", ctypes.c_int64: "i64", ctypes.c_uint64: "u64", ctypes.c_size_t: "u64",
+            ctypes.c_float: "float"}[t]
+
+
+def test_binding_signatures_match_the_c_prototypes():
+    """Every declared entry point is called through ctypes with the argument
+    and return types of its C prototype (int, int64_t, 64-bit unsigned,
+    float, pointer), in order."""
+    text = re.sub(r"/\*.*?\*/", " ", open(HEADER).read(), flags=re.S)
+    protos = re.findall(r"Q4_API\s+([\w\s\*]+?)\b(\w+)\s*\(([^)]*)\)\s*;", text)
+    assert sorted(name for _, name, _ in protos) == declared_symbols()
+    L = q4.lib()
+    for ret, name, params in protos:
+        params = params.strip()
+        c_args = [] if params in ("", "void") else [_c_category(p) for p in params.split(",")]
+        f = getattr(L, name)
+        assert [_ctypes_category(a) for a in f.argtypes] == c_args, name
+        assert _ctypes_category(f.restype) == _c_category(ret), name

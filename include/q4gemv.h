@@ -484,9 +484,10 @@ typedef struct q4_chain_op {
  * == 0; no op writing bytes that an earlier (or the same) op reads, no two
  * ops writing the same bytes except RMSNorm ops sharing one residual stream
  * (same pointer and N), no op reading a residual stream through `in`; the
- * largest activation row and the residual streams within shared memory
- * beside the weight rings (about 84 KB: a 17,408-value row and a 5,120-value
- * stream fit).  Otherwise Q4_ERR_UNSUPPORTED with the reason.  A grid
+ * largest activation row (2 bytes a value, rounded up to 128) and the
+ * residual streams (4 bytes a value) within the 83,712 bytes of shared
+ * memory beside the weight rings (a 17,408-value row and a 5,120-value
+ * stream take 55,296).  Otherwise Q4_ERR_UNSUPPORTED with the reason.  A grid
  * barrier whose wait gives up sets the status word (layer_stack_check
  * returns Q4_ERR_TIMEOUT).  On the 64-layer decode chain it measured slower
  * than the graph (each CTA recomputes every step over the whole row, and

@@ -76,7 +76,7 @@ def test_chain_shape_of_the_decode_stream():
 def test_chain_shapes_meet_the_one_launch_conditions():
     """The conditions include/q4gemv.h states for Q4_CHAIN_PERSISTENT (q4
     products K % 256 == 0, q8 K % 128 == 0, step rows N % 8 == 0, the largest
-    activation row and the residual stream within the ~84 KB of shared
+    activation row and the residual stream within the 83,712 bytes of shared
     memory beside the rings) hold for the decode chain and the small one."""
     for shape in (workloads.ChainShape(), SMALL):
         tensors = workloads.chain_tensors(shape)

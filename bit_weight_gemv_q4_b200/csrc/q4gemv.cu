@@ -546,11 +546,10 @@ extern "C" Q4_API int q4_selftest_wait_timeout(uint64_t timeout_ns, int* status_
 
 // ----------------------------------------------------------------------------
 // q4 product without a caller-provided workspace.  Some callers cannot
-// allocate device memory at the point where they run the product: code inside
-// an open stream capture (cudaMalloc is not a stream operation and is not
-// allowed while a global or thread-local capture is open), plug-ins that run
-// under a host application's memory budget or allocator they do not own, and
-// latency-critical loops that must not take the driver's allocation path.
+// allocate device memory at the point where they run the product: plug-ins
+// that run inside a host application which owns the device memory budget (its
+// own pool or allocator, none of it handed to them), and latency-critical
+// loops that must not call cudaMalloc, which can synchronise the whole device.
 // For them the split-tile scratch lives in this file-scope device array
 // instead.  Every GPU that loads the library holds it until the process exits.
 // ----------------------------------------------------------------------------
@@ -592,12 +591,17 @@ extern "C" Q4_API int q4_gemv_noalloc(const void* packed, int64_t N, int64_t K, 
   DeviceInfo dev;
   if ((rc = device_info(&dev))) return rc;
   const size_t need = workspace_bytes(s, M, dev);
-  if (need > kNoAllocWorkspaceBytes)
+  if (need > kNoAllocWorkspaceBytes) {
+    // rows whose tile counters fit beside the header and the partial sums
+    // (counters take whole 256-byte blocks of 64 tiles, 32 rows each)
+    const size_t fixed = kWsHeader + partials_bytes(dev);
+    const long long max_rows =
+        fixed >= kNoAllocWorkspaceBytes ? 0 : static_cast<long long>((kNoAllocWorkspaceBytes - fixed) / 256 * 64 * 32);
     return fail(Q4_ERR_UNSUPPORTED,
                 "%s: this shape needs %zu bytes of scratch, more than the %zu-byte static array "
                 "(at most %lld rows on this device); use q4_gemv with a workspace",
-                who, need, kNoAllocWorkspaceBytes,
-                static_cast<long long>((kNoAllocWorkspaceBytes - kWsHeader - partials_bytes(dev)) / 4 * 32));
+                who, need, kNoAllocWorkspaceBytes, max_rows);
+  }
   void* ws = nullptr;
   if ((rc = noalloc_workspace(&ws))) return rc;
   Launch L;

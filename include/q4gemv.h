@@ -320,22 +320,24 @@ Q4_API int q8_gemv(const void* packed, int64_t N, int64_t K, const uint16_t* x, 
                    size_t workspace_bytes, void* stream);
 
 /* q4_gemv for callers that cannot allocate device memory where they run the
- * product: code inside an open stream capture (cudaMalloc is not allowed
- * there), plug-ins that run under a host application's memory budget or
- * allocator, and loops that must not take the driver's allocation path.  The
- * pages describe no such entry point; it has no counterpart there.
+ * product: plug-ins inside a host application that owns the device memory
+ * budget (its own pool or allocator, none of it handed to them), and
+ * latency-critical loops that must not call cudaMalloc, which can synchronise
+ * the whole device.  The pages describe no such entry point; it has no
+ * counterpart there.
  * Same product, arguments and errors as q4_gemv, without the workspace: the
  * split-tile scratch is a file-scope device array of 4 MiB that every GPU
  * loading the library holds until the process exits.  Shapes whose scratch
  * does not fit (more than about 14 million rows on a 148-SM device) are
- * rejected with Q4_ERR_UNSUPPORTED.  Allocates and frees nothing.  The first
- * call on a device looks up the array's device address
- * (cudaGetSymbolAddress); make that first call before any stream capture.
- * Each call clears the array's status word and counters with two
- * asynchronous memsets on `stream` before its kernel.  All calls share the
- * one array: calls that may overlap on the GPU (different streams without
- * ordering between them) race and give undefined results.  A device wait that
- * gives up is not reported by this entry point. */
+ * rejected with Q4_ERR_UNSUPPORTED before any device work.  Allocates and
+ * frees nothing.  The first call on a device looks up the array's device
+ * address (cudaGetSymbolAddress, with that device current); make that first
+ * call before any stream capture.  Each call clears the array's status word
+ * and the counters it uses with two asynchronous memsets on `stream` before
+ * its kernel.  All calls share the one array, which keeps the last call's
+ * contents: calls that may overlap on the GPU (different streams without
+ * ordering between them) race and give undefined results.  A device wait
+ * that gives up is not reported by this entry point. */
 Q4_API int q4_gemv_noalloc(const void* packed, int64_t N, int64_t K, const uint16_t* x, int M, float* y,
                            void* stream);
 

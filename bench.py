@@ -517,11 +517,12 @@ def run_ours(args, d: Dist):
     widths = ({f"q{b}": format_stream(workloads.as_width(tensors, b)) for b in (5, 6)} if secondary else skipped)
 
     # the dependent chain: the same products with the steps between them
-    # (residual + RMSNorm, SwiGLU), one CUDA graph with programmatic dependent
-    # launch (M1, M4), and at M = 1 as one persistent cooperative launch
+    # (residual + RMSNorm, SwiGLU), in the form layer_chain_create picks by
+    # default (M1: one cooperative launch; M4: one CUDA graph with programmatic
+    # dependent launch) and in the other form
     chain = {} if secondary else skipped
-    for key, M, flags in ((("M1", 1, 0), ("M4", 4, 0), ("M1_persistent", 1, q4.Q4_CHAIN_PERSISTENT))
-                          if secondary else ()):
+    for key, M, flags in ((("M1", 1, 0), ("M4", 4, 0), ("M1_graph", 1, q4.Q4_CHAIN_GRAPH),
+                           ("M4_persistent", 4, q4.Q4_CHAIN_PERSISTENT)) if secondary else ()):
         ch = workloads.DeviceChain(workloads.ChainShape(), M, seed=args.seed, flags=flags)
         try:
             for _ in range(3):

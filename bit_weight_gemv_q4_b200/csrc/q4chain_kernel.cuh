@@ -19,24 +19,32 @@ namespace q4k {
 
 constexpr int kNormThreads = 1024;
 
-// One CTA per activation row m.  The sum of squares is reduced in a fixed
-// order (per-thread strided sums, a shuffle tree per warp, warps in order), so
-// it is bitwise reproducible.  Rows of up to kNormThreads * kNormPer values
-// keep each thread's values in registers: every load (h, y, gamma) is issued
-// at once and h is not read back, so the step costs one memory round trip
-// instead of one per value; longer rows take the same arithmetic in loops.
+// One CTA per activation row m.  The sum of squares has one fixed
+// association, shared with the one-launch chain kernel: fp32 squares, a
+// butterfly (xor-shuffle) sum over each tile of 32 consecutive values, the
+// tile sums t = w, w + 32, w + 64, ... added in order (warp w of the 32 warps
+// holds exactly those tiles, since thread t takes k = t + 1024 j), and a
+// butterfly over the 32 warps' sums; so the two give bitwise the same
+// activations.  Rows of up to kNormThreads * kNormPer values keep each
+// thread's values in registers: every load (h, y, gamma) is issued at once
+// and h is not read back; longer rows take the same arithmetic in loops.
 constexpr int kNormPer = 8;
 
-__device__ __forceinline__ float norm_block_reduce(float ss) {
+__device__ __forceinline__ float norm_warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, o);
+  return v;
+}
+
+// Every thread: the row's sum of squares from its warp's running tile sum.
+__device__ __forceinline__ float norm_block_total(float warp_tiles) {
   __shared__ float s_part[32];
   __shared__ float s_t;
-  for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xFFFFFFFFu, ss, o);
-  if ((threadIdx.x & 31) == 0) s_part[threadIdx.x >> 5] = ss;
+  if ((threadIdx.x & 31) == 0) s_part[threadIdx.x >> 5] = warp_tiles;
   __syncthreads();
-  if (threadIdx.x == 0) {
-    float t = 0.f;
-    for (int w = 0; w < static_cast<int>(blockDim.x >> 5); ++w) t += s_part[w];
-    s_t = t;
+  if (threadIdx.x < 32) {
+    const float t = norm_warp_sum(s_part[threadIdx.x]);
+    if (threadIdx.x == 0) s_t = t;
   }
   __syncthreads();
   return s_t;
@@ -64,38 +72,40 @@ __global__ void __launch_bounds__(kNormThreads) residual_rmsnorm_kernel(float* _
         if (gamma) g[j] = __uint_as_float(static_cast<uint32_t>(gamma[k]) << 16);
       }
     }
-    float ss = 0.f;
+    float tiles = 0.f;
 #pragma unroll
     for (int j = 0; j < kNormPer; ++j) {
       const int k = threadIdx.x + j * kNormThreads;
-      if (k < N) {
-        h[row + k] = v[j];
-        ss = fmaf(v[j], v[j], ss);
-      }
+      if (k < N) h[row + k] = v[j];
+      if (j * kNormThreads < N) tiles += norm_warp_sum(__fmul_rn(v[j], v[j]));
     }
-    const float r = 1.f / sqrtf(norm_block_reduce(ss) / static_cast<float>(N) + eps);
+    const float r = 1.f / sqrtf(norm_block_total(tiles) / static_cast<float>(N) + eps);
 #pragma unroll
     for (int j = 0; j < kNormPer; ++j) {
       const int k = threadIdx.x + j * kNormThreads;
       if (k < N) {
-        float o = v[j] * r;
-        if (gamma) o *= g[j];
+        float o = __fmul_rn(v[j], r);
+        if (gamma) o = __fmul_rn(o, g[j]);
         x[row + k] = __bfloat16_as_ushort(__float2bfloat16_rn(o));
       }
     }
     return;
   }
-  float ss = 0.f;
-  for (int k = threadIdx.x; k < N; k += blockDim.x) {
-    float v = set ? y[row + k] : h[row + k];
-    if (y && !set) v += y[row + k];
-    h[row + k] = v;
-    ss = fmaf(v, v, ss);
+  float tiles = 0.f;
+  for (int base = 0; base < N; base += kNormThreads) {
+    const int k = base + threadIdx.x;
+    float v = 0.f;
+    if (k < N) {
+      v = set ? y[row + k] : h[row + k];
+      if (y && !set) v += y[row + k];
+      h[row + k] = v;
+    }
+    tiles += norm_warp_sum(__fmul_rn(v, v));
   }
-  const float r = 1.f / sqrtf(norm_block_reduce(ss) / static_cast<float>(N) + eps);
+  const float r = 1.f / sqrtf(norm_block_total(tiles) / static_cast<float>(N) + eps);
   for (int k = threadIdx.x; k < N; k += blockDim.x) {
-    float v = h[row + k] * r;
-    if (gamma) v *= __uint_as_float(static_cast<uint32_t>(gamma[k]) << 16);
+    float v = __fmul_rn(h[row + k], r);
+    if (gamma) v = __fmul_rn(v, __uint_as_float(static_cast<uint32_t>(gamma[k]) << 16));
     x[row + k] = __bfloat16_as_ushort(__float2bfloat16_rn(v));
   }
 }

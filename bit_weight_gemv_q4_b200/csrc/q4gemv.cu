@@ -80,6 +80,10 @@ constexpr int kStackD = Q4_TUNE_STACK_D;    // stages per warp in the persistent
 constexpr int kStackPF = Q4_TUNE_STACK_PF;  // further stages prefetched into L2 (ordered mode)
 constexpr int kStreamU = Q4_TUNE_STREAM_U;  // chunks per stage in stream mode, when the shapes allow
 constexpr int kStackNW = Q4_TUNE_STACK_NW;  // warps per CTA of the persistent kernels (one CTA per SM)
+#ifndef Q4_TUNE_CHAIN_PF
+#define Q4_TUNE_CHAIN_PF 0
+#endif
+constexpr int kChainPF = Q4_TUNE_CHAIN_PF;  // one-launch chain: stages prefetched into L2 beyond each ring
 // shared memory a CTA may use (B200: 227 KB per CTA)
 constexpr int kSmemLimit = 227 * 1024 / kCtasPerSm;
 constexpr size_t kWsHeader = 256;
@@ -642,7 +646,6 @@ struct q4_stack {
   bool chain = false;
   q4k::ChainParams chain_params{};
   q4k::ChainOpDev* chain_ops_dev = nullptr;
-  q4k::ChainResid* chain_resids_dev = nullptr;
   int M = 1;
   void* workspace = nullptr;
   size_t workspace_bytes = 0;
@@ -708,7 +711,6 @@ void free_stack(q4_stack* st) {
   if (st->entries_dev) cudaFree(st->entries_dev);
   if (st->xprep_dev) cudaFree(st->xprep_dev);
   if (st->chain_ops_dev) cudaFree(st->chain_ops_dev);
-  if (st->chain_resids_dev) cudaFree(st->chain_resids_dev);
   if (st->workspace) cudaFree(st->workspace);
   delete st;
 }
@@ -1082,23 +1084,45 @@ Span span_of(const void* p, long long bytes) {
 }
 
 // The persistent chain: one cooperative chain_kernel launch over the whole op
-// list (M = 1).  Eligible when every product is q4 or q8 with stages of
-// kStreamU whole chunks, each step's row fits the kernel's vector passes, no
-// op overwrites a buffer an earlier op reads, no two ops write the same bytes
-// (except the residual stream, shared by RMSNorm ops), and the activation
-// buffer and the residual streams fit shared memory beside the rings.  A
-// grid barrier goes before every op that reads bytes another CTA wrote since
-// the last barrier; a product whose activations are those the CTA itself
-// just computed (the preceding step's output) or already holds reads them
-// from shared memory.  Consecutive products without a barrier alternate
-// between two split-tile partial buffers, so a barrier also goes before a
-// third.
+// list (M = 1..4).  Eligible when every product is q4 or q8 with stages of
+// chain_su(M) whole chunks, each step's row length is a multiple of 8, no op
+// overwrites a buffer an earlier op reads, no two ops write the same bytes
+// (except the residual stream, shared by RMSNorm ops), and the largest
+// activation tensor fits shared memory beside the rings.
+//  * A step directly after the product whose output it reads runs its
+//    elementwise part in that product's tile finishers (RMSNorm: the product's
+//    N is the norm's; SwiGLU: the product's N is twice the step's, a multiple
+//    of 64); other steps split it between the CTAs and add a barrier.
+//  * A grid barrier goes before every op that reads bytes another CTA wrote
+//    since the last barrier; a product whose activations are those the CTA
+//    itself just computed (the preceding step's output) or already holds, in
+//    the same chunk layout, reads them from shared memory.  Consecutive
+//    products without a barrier alternate between two split-tile partial
+//    buffers, so a barrier also goes before a third.
+//  * The RMSNorm ops of one residual stream R read and write it in turn
+//    through two workspace buffers: the i-th of c reads R (i = 0) or buffer
+//    (i - 1) % 2 and writes buffer i % 2, the last one R.
+int chain_su(int M) { return M <= 2 ? 4 : 2; }
+
+template <int M, int SU>
+void* chain_kernel_ptr() {
+  return reinterpret_cast<void*>(&q4k::chain_kernel<M, kStackNW, kStackD, SU, kChainPF>);
+}
+
+void* chain_kernel_for(int M) {
+  switch (M) {
+    case 1: return chain_kernel_ptr<1, 4>();
+    case 2: return chain_kernel_ptr<2, 4>();
+    case 3: return chain_kernel_ptr<3, 2>();
+    default: return chain_kernel_ptr<4, 2>();
+  }
+}
+
 int create_chain_persistent(const q4_chain_op* ops, int n, int M, const DeviceInfo& dev, q4_stack* st) {
   const char* who = "layer_chain_create (persistent)";
-  if (M != 1) return fail(Q4_ERR_UNSUPPORTED, "%s: the persistent chain runs M = 1 only", who);
+  if (M < 1 || M > 4) return fail(Q4_ERR_INVALID_ARG, "%s: M must be in 1..4", who);
   const int G = dev.sms;
-  if (G > 32 * q4k::kChainFlagsPerLane) return fail(Q4_ERR_UNSUPPORTED, "%s: more SMs than its barrier polls", who);
-  constexpr int SU = kStreamU;
+  const int SU = chain_su(M);
   const long long warps = static_cast<long long>(G) * kStackNW;
   struct Access {
     Span r[2], w;
@@ -1107,21 +1131,25 @@ int create_chain_persistent(const q4_chain_op* ops, int n, int M, const DeviceIn
   std::vector<Access> acc(static_cast<size_t>(n));
   std::vector<q4k::StackEntryDev> entries;
   std::vector<q4k::ChainOpDev> dops(static_cast<size_t>(n));
-  std::vector<q4k::ChainResid> resids;
-  long long total_tiles = 0;
+  std::vector<int> kc_of(static_cast<size_t>(n), 64);  // products: values per chunk
   long long x_max = 0;
-  int h_floats = 0;
   for (int i = 0; i < n; ++i) {
     const q4_chain_op& op = ops[i];
     q4k::ChainOpDev& d = dops[static_cast<size_t>(i)];
     d = q4k::ChainOpDev{};
+    d.pre_next = -1;
+    d.pre_off = -1;
+    d.src_op = -1;
+    d.prep = -1;
     Access& a = acc[static_cast<size_t>(i)];
     if (op.kind == Q4_OP_PRODUCT) {
       Shape s;
       make_shape(op.bits, op.N, op.K, &s, who);
-      const long long need = static_cast<long long>(SU) * (op.bits == 4 ? 64 : 32);
+      const int KC = op.bits == 4 ? 64 : 32;
+      const long long need = static_cast<long long>(SU) * KC;
       if (s.N == 0 || s.K == 0 || s.K % need != 0)
-        return fail(Q4_ERR_UNSUPPORTED, "%s: op %d: products need N > 0 and K a multiple of %lld", who, i, need);
+        return fail(Q4_ERR_UNSUPPORTED, "%s: op %d: products need N > 0 and K a multiple of %lld at M = %d", who, i,
+                    need, M);
       if (!op.packed || !op.in || !op.out || misaligned(op.packed, 16) || misaligned(op.in, 16) ||
           misaligned(op.out, 4))
         return fail(Q4_ERR_ALIGN, "%s: op %d: packed and in must be 16-byte aligned, out 4-byte", who, i);
@@ -1137,44 +1165,36 @@ int create_chain_persistent(const q4_chain_op* ops, int n, int M, const DeviceIn
       e.bits = op.bits;
       const long long TB = s.TC / SU;
       e.P = static_cast<int>(TB < warps ? TB : warps);  // the split of a one-product stream-mode stack
-      e.tile_off = static_cast<int>(total_tiles);
-      total_tiles += s.T;
       d.kind = q4k::kChainProduct;
       d.entry = static_cast<int>(entries.size());
       d.x = e.x;
+      d.kc = KC;
+      kc_of[static_cast<size_t>(i)] = KC;
       entries.push_back(e);
-      a.r[0] = span_of(op.in, s.K * 2);
-      a.w = span_of(op.out, s.N * 4);
+      a.r[0] = span_of(op.in, static_cast<long long>(M) * s.K * 2);
+      a.w = span_of(op.out, static_cast<long long>(M) * s.N * 4);
       x_max = std::max(x_max, s.K);
     } else {
       if (op.N % 8 != 0) return fail(Q4_ERR_UNSUPPORTED, "%s: op %d: step rows must be a multiple of 8", who, i);
+      if (op.N > (int64_t(1) << 24)) return fail(Q4_ERR_UNSUPPORTED, "%s: op %d: step row too long", who, i);
+      if (misaligned(op.out, 16))  // its outputs are read back 16 bytes at a time
+        return fail(Q4_ERR_ALIGN, "%s: op %d: a step's out must be 16-byte aligned", who, i);
+      d.kc = 8;  // the activation buffer's layout when no product reads this output from it
       d.N = static_cast<int>(op.N);
       d.out = static_cast<uint16_t*>(op.out);
       d.y = static_cast<const float*>(op.in);
-      a.w = span_of(op.out, op.N * 2);
+      a.w = span_of(op.out, static_cast<long long>(M) * op.N * 2);
       x_max = std::max(x_max, static_cast<long long>(op.N));
       if (op.kind == Q4_OP_SWIGLU) {
         d.kind = q4k::kChainSwiglu;
-        a.r[0] = span_of(op.in, op.N * 8);
+        a.r[0] = span_of(op.in, static_cast<long long>(M) * op.N * 8);
       } else {
         d.kind = q4k::kChainRmsnorm;
         d.set = op.bits == 1 ? 1 : 0;
         d.gamma = static_cast<const uint16_t*>(op.packed);
-        d.resid = op.resid;
-        a.r[0] = span_of(op.in, op.N * 4);
+        a.r[0] = span_of(op.in, static_cast<long long>(M) * op.N * 4);
         a.r[1] = span_of(op.packed, op.N * 2);
-        a.resid = span_of(op.resid, op.N * 4);
-        int slot = -1;
-        for (size_t k = 0; k < resids.size(); ++k)
-          if (resids[k].h == op.resid) slot = static_cast<int>(k);
-        if (slot >= 0 && resids[static_cast<size_t>(slot)].N != op.N)
-          return fail(Q4_ERR_UNSUPPORTED, "%s: op %d: one residual stream with two lengths", who, i);
-        if (slot < 0) {
-          resids.push_back(q4k::ChainResid{op.resid, static_cast<int>(op.N), h_floats});
-          h_floats += static_cast<int>((op.N + 3) / 4 * 4);
-          slot = static_cast<int>(resids.size()) - 1;
-        }
-        d.h_off = resids[static_cast<size_t>(slot)].h_off;
+        a.resid = span_of(op.resid, static_cast<long long>(M) * op.N * 4);
       }
     }
   }
@@ -1194,66 +1214,207 @@ int create_chain_persistent(const q4_chain_op* ops, int n, int M, const DeviceIn
         return fail(Q4_ERR_UNSUPPORTED, "%s: ops %d and %d write the same bytes", who, i, j);
     }
   }
-  // barriers, activation sources, partial buffers
+  // the residual streams: norms per stream, in order
+  struct Stream {
+    float* R;
+    long long N;
+    std::vector<int> norms;
+  };
+  std::vector<Stream> streams;
+  for (int i = 0; i < n; ++i) {
+    if (ops[i].kind != Q4_OP_RESIDUAL_RMSNORM) continue;
+    size_t k = 0;
+    while (k < streams.size() && streams[k].R != ops[i].resid) ++k;
+    if (k == streams.size()) streams.push_back(Stream{ops[i].resid, ops[i].N, {}});
+    if (streams[k].N != ops[i].N)
+      return fail(Q4_ERR_UNSUPPORTED, "%s: op %d: one residual stream with two lengths", who, i);
+    streams[k].norms.push_back(i);
+  }
+  // fused steps, epilogues, chunk layouts of the activation buffer, tagged words
+  long long n_words = 0;
+  auto words = [&](long long count) {
+    const long long at = n_words;
+    n_words += (count + 31) / 32 * 32;
+    return at;
+  };
+  for (int j = 0; j < n; ++j) {
+    const q4_chain_op& op = ops[j];
+    if (op.kind == Q4_OP_PRODUCT) continue;
+    q4k::ChainOpDev& d = dops[static_cast<size_t>(j)];
+    if (j + 1 < n && ops[j + 1].kind == Q4_OP_PRODUCT && ops[j + 1].in == op.out && ops[j + 1].K == op.N)
+      d.kc = kc_of[static_cast<size_t>(j + 1)];
+    const bool after_product = j > 0 && ops[j - 1].kind == Q4_OP_PRODUCT && op.in && ops[j - 1].out == op.in;
+    const long long tiles = (op.N + q4k::kTileRows - 1) / q4k::kTileRows;
+    if (op.kind == Q4_OP_RESIDUAL_RMSNORM) {
+      // its tile sums of squares go to the warps' scratch, one float per tile and row
+      if (tiles * M > static_cast<long long>(kStackNW) * M * q4k::kTileRows)
+        return fail(Q4_ERR_UNSUPPORTED, "%s: op %d: a norm row of more than %d values", who, j,
+                    kStackNW * q4k::kTileRows * q4k::kTileRows);
+      d.tw = static_cast<int>(words(M * op.N));
+      d.epi = after_product && ops[j - 1].N == op.N ? 1 : 0;
+    } else {
+      d.tw = static_cast<int>(words(M * op.N / 2));
+      d.epi = after_product && ops[j - 1].N == 2 * op.N && op.N % q4k::kTileRows == 0 ? 1 : 0;
+      if (d.epi) d.uw = static_cast<int>(words(M * op.N));
+    }
+    if (d.epi) {
+      q4k::ChainOpDev& pd = dops[static_cast<size_t>(j - 1)];
+      pd.epi = op.kind == Q4_OP_RESIDUAL_RMSNORM ? q4k::kEpiResid : q4k::kEpiSwiglu;
+      pd.step = j;
+    }
+  }
+  if (n_words > (1LL << 31) - 1) return fail(Q4_ERR_UNSUPPORTED, "%s: the steps' words exceed 2^31", who);
+  // Products whose activations are not in the CTA's buffer (the op before
+  // them neither computed nor read them in the same layout) stage them.  A
+  // staged product whose activations no op writes, right after an op that
+  // leaves the buffer's tail free, gets a prepared copy: the launch converts
+  // it first, and the op before copies it into the tail, where it is read in
+  // place.
+  {
+    const void* t = nullptr;
+    long long tn = 0;
+    int tk = 0;
+    for (int j = 0; j < n; ++j) {
+      const q4_chain_op& op = ops[j];
+      q4k::ChainOpDev& d = dops[static_cast<size_t>(j)];
+      if (op.kind == Q4_OP_PRODUCT) {
+        d.stage_x = (op.in == t && op.K == tn && d.kc == tk) ? 0 : 1;
+        t = op.in;
+        tn = op.K;
+      } else {
+        t = op.out;
+        tn = op.N;
+      }
+      tk = d.kc;
+    }
+  }
+  const long long X = static_cast<long long>(M) * x_max * 2;  // the activation buffer's bytes
+  std::vector<int> prep_ops;
+  long long prep_values = 0;
+  for (int p = 1; p < n; ++p) {
+    q4k::ChainOpDev& d = dops[static_cast<size_t>(p)];
+    if (ops[p].kind != Q4_OP_PRODUCT || !d.stage_x || dops[static_cast<size_t>(p - 1)].pre_off >= 0) continue;
+    bool written = false;
+    for (int i = 0; i < n; ++i)
+      if (acc[static_cast<size_t>(i)].w.overlaps(acc[static_cast<size_t>(p)].r[0]) ||
+          acc[static_cast<size_t>(i)].resid.overlaps(acc[static_cast<size_t>(p)].r[0]))
+        written = true;
+    const long long used = static_cast<long long>(M) * (ops[p - 1].kind == Q4_OP_PRODUCT ? ops[p - 1].K : ops[p - 1].N) * 2;
+    const long long need = static_cast<long long>(M) * ops[p].K * 2;
+    if (written || used + need > X) continue;
+    d.pre_off = static_cast<int>(X - need);
+    d.prep = static_cast<int>(prep_ops.size());
+    d.prep_at = prep_values;
+    prep_values += static_cast<long long>(M) * ops[p].K;
+    prep_ops.push_back(p);
+    dops[static_cast<size_t>(p - 1)].pre_next = p;
+    entries[static_cast<size_t>(d.entry)].rx_off = d.pre_off;  // the product reads the copy in place
+  }
+  // a product after a prepared one reads its activations from the start of
+  // the buffer, not from the tail: it stages them itself
+  for (int p = 1; p < n; ++p)
+    if (ops[p].kind == Q4_OP_PRODUCT && !dops[static_cast<size_t>(p)].stage_x &&
+        dops[static_cast<size_t>(p - 1)].prep >= 0)
+      dops[static_cast<size_t>(p)].stage_x = 1;
+  // Grid barriers (the fallback): a product that stages its activations from
+  // global memory itself, or a step not fed by the product before it, reads
+  // bytes that other CTAs write with plain stores, so it needs a barrier when
+  // it reads bytes written since the last one.  A product reusing a partial
+  // buffer needs one unless, since the buffer's last user, a step has waited
+  // for every tile of a product to which every warp contributes (so every
+  // warp has finished the last user).
   std::vector<Span> since;  // bytes written since the last barrier
   const void* tag = nullptr;
   long long tag_n = 0;
-  int products_since = 0;
+  int tag_kc = 0;
+  int n_products = 0;
+  std::vector<int> pbuf_user(q4k::kChainPartialBufs, -1);  // product index of each buffer's last user
+  int last_completion = -1;                                 // product index of the last awaited full product
   for (int j = 0; j < n; ++j) {
     const q4_chain_op& op = ops[j];
     q4k::ChainOpDev& d = dops[static_cast<size_t>(j)];
     const Access& aj = acc[static_cast<size_t>(j)];
-    const bool resident = op.kind == Q4_OP_PRODUCT && op.in == tag && op.K == tag_n;
+    const bool resident = op.kind == Q4_OP_PRODUCT && op.in == tag && op.K == tag_n && d.kc == tag_kc;
+    const bool reads_plain = (op.kind == Q4_OP_PRODUCT && !resident && d.prep < 0) ||
+                             (op.kind != Q4_OP_PRODUCT && !d.epi);
     bool need = false;
-    for (const Span& w : since)
-      if ((!resident && aj.r[0].overlaps(w)) || aj.r[1].overlaps(w)) need = true;
-    if (op.kind == Q4_OP_PRODUCT && products_since == 2) need = true;
+    if (reads_plain)
+      for (const Span& w : since)
+        if (aj.r[0].overlaps(w) || aj.r[1].overlaps(w) || aj.resid.overlaps(w)) need = true;
+    if (op.kind == Q4_OP_PRODUCT) {
+      const int pb = n_products % q4k::kChainPartialBufs;
+      if (pbuf_user[static_cast<size_t>(pb)] >= 0 && last_completion <= pbuf_user[static_cast<size_t>(pb)]) need = true;
+    }
     if (need) {
       d.barrier = 1;
       since.clear();
-      products_since = 0;
+      last_completion = n_products - 1;  // every product so far is complete
     }
     if (op.kind == Q4_OP_PRODUCT) {
-      d.stage_x = resident ? 0 : 1;
-      d.pbuf = products_since;
-      ++products_since;
+      d.pbuf = n_products % q4k::kChainPartialBufs;
+      pbuf_user[static_cast<size_t>(d.pbuf)] = n_products;
+      ++n_products;
       tag = op.in;
       tag_n = op.K;
+      tag_kc = d.kc;
+      since.push_back(aj.w);
     } else {
+      if (d.epi && entries[static_cast<size_t>(dops[static_cast<size_t>(j - 1)].entry)].P == warps)
+        last_completion = n_products - 1;
       tag = op.out;
       tag_n = op.N;
+      tag_kc = d.kc;
+      since.push_back(aj.w);
+      since.push_back(aj.resid);
     }
-    since.push_back(aj.w);
   }
-  const int rings = kStackNW * kStackD * q4k::StreamSlot<SU, 1, 3>::kBytes;
-  const int x_off = (rings + kStackNW * kStackD * 8 + 127) / 128 * 128;
-  const long long h_base = x_off + (x_max * 2 + 127) / 128 * 128;
-  const long long smem = h_base + static_cast<long long>(h_floats) * 4;
+  long long max_tiles = 0;  // of a norm row
+  for (int j = 0; j < n; ++j)
+    if (ops[j].kind == Q4_OP_RESIDUAL_RMSNORM) max_tiles = std::max<long long>(max_tiles, (ops[j].N + 31) / 32);
+  const int rings = kStackNW * kStackD * SU * q4k::Format<4>::kChunkBytes;
+  const long long x_off = (rings + kStackNW * kStackD * 8 + 127) / 128 * 128;
+  const long long scr_off = x_off + (X + 127) / 128 * 128;
+  const long long tiles_off = scr_off + static_cast<long long>(kStackNW) * M * q4k::kTileRows * 4;
+  const long long smem = tiles_off + (M * max_tiles * 4 + 127) / 128 * 128;
   if (smem > kSmemLimit - 1024)
-    return fail(Q4_ERR_UNSUPPORTED, "%s: activations (%lld values) and residual streams (%d floats) exceed shared "
-                                    "memory", who, x_max, h_floats);
-  // workspace: [status | partials: 2 buffers of [warps][2][32] | tile counters | barrier flags]
-  const long long pbuf_floats = warps * 2 * q4k::kTileRows;
-  const size_t partials_at = kWsHeader;
-  const size_t counters_at = partials_at + static_cast<size_t>(2 * pbuf_floats) * 4;
-  const size_t flags_at = counters_at + (static_cast<size_t>(total_tiles) * 4 + 255) / 256 * 256;
-  st->workspace_bytes = flags_at + (static_cast<size_t>(G) * 4 + 255) / 256 * 256;
+    return fail(Q4_ERR_UNSUPPORTED, "%s: activations of %lld values x M = %d exceed shared memory", who, x_max, M);
+  // workspace: [status | partial buffers | tagged words | per-CTA run counters | barrier counter]
+  auto up256 = [](size_t v) { return (v + 255) / 256 * 256; };
+  const long long pbuf_words = warps * M * q4k::kTileRows;
+  const size_t parts_at = kWsHeader;
+  const size_t words_at = parts_at + up256(static_cast<size_t>(q4k::kChainPartialBufs * pbuf_words) * 8);
+  const size_t run_at = words_at + up256(static_cast<size_t>(n_words) * 8);
+  const size_t bar_at = run_at + up256(static_cast<size_t>(G) * 4);
+  const size_t prep_at = bar_at + 256;
+  const size_t prep_info_at = prep_at + up256(static_cast<size_t>(prep_values) * 2);
+  const size_t prep_ops_at = prep_info_at + up256(prep_ops.size() * 8);
+  st->workspace_bytes = prep_ops_at + up256(prep_ops.size() * 4);
   cudaError_t err = cudaMalloc(&st->workspace, st->workspace_bytes);
   if (err == cudaSuccess) err = cudaMemset(st->workspace, 0, st->workspace_bytes);
-  if (err == cudaSuccess) err = cudaMalloc(&st->entries_dev, sizeof(q4k::StackEntryDev) * entries.size());
+  if (err != cudaSuccess) return cuda_fail(err, "layer_chain_create: workspace");
+  unsigned char* ws = static_cast<unsigned char*>(st->workspace);
+  // the norms of a stream: each adds to the previous one's tagged h; the
+  // first reads the caller's buffer (unless it sets h), the last writes it
+  for (const Stream& sr : streams) {
+    const size_t c = sr.norms.size();
+    for (size_t i = 0; i < c; ++i) {
+      q4k::ChainOpDev& d = dops[static_cast<size_t>(sr.norms[i])];
+      d.src_op = i == 0 ? -1 : sr.norms[i - 1];
+      d.h_src = i == 0 ? sr.R : nullptr;
+      d.h_dst = i + 1 == c ? sr.R : nullptr;
+    }
+  }
+  err = cudaMalloc(&st->entries_dev, sizeof(q4k::StackEntryDev) * entries.size());
   if (err == cudaSuccess)
     err = cudaMemcpy(st->entries_dev, entries.data(), sizeof(q4k::StackEntryDev) * entries.size(),
                      cudaMemcpyHostToDevice);
+  if (err == cudaSuccess && !prep_ops.empty())
+    err = cudaMemcpy(ws + prep_ops_at, prep_ops.data(), prep_ops.size() * 4, cudaMemcpyHostToDevice);
   if (err == cudaSuccess) err = cudaMalloc(&st->chain_ops_dev, sizeof(q4k::ChainOpDev) * dops.size());
   if (err == cudaSuccess)
     err = cudaMemcpy(st->chain_ops_dev, dops.data(), sizeof(q4k::ChainOpDev) * dops.size(), cudaMemcpyHostToDevice);
-  if (err == cudaSuccess && !resids.empty())
-    err = cudaMalloc(&st->chain_resids_dev, sizeof(q4k::ChainResid) * resids.size());
-  if (err == cudaSuccess && !resids.empty())
-    err = cudaMemcpy(st->chain_resids_dev, resids.data(), sizeof(q4k::ChainResid) * resids.size(),
-                     cudaMemcpyHostToDevice);
   if (err != cudaSuccess) return cuda_fail(err, "layer_chain_create: allocation");
-  st->fn = reinterpret_cast<void*>(&q4k::chain_kernel<kStackNW, kStackD, SU>);
+  st->fn = chain_kernel_for(M);
   st->smem = static_cast<int>(smem);
   st->block = kStackNW * 32;
   st->grid = G;
@@ -1263,25 +1424,28 @@ int create_chain_persistent(const q4_chain_op* ops, int n, int M, const DeviceIn
   err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, st->fn, st->block, st->smem);
   if (err != cudaSuccess) return cuda_fail(err, "layer_chain_create: occupancy query");
   if (per_sm < 1) return fail(Q4_ERR_UNSUPPORTED, "%s: the chain kernel does not fit on an SM", who);
-  unsigned char* ws = static_cast<unsigned char*>(st->workspace);
   q4k::ChainParams& p = st->chain_params;
   p.ops = st->chain_ops_dev;
   p.n_ops = n;
   p.entries = st->entries_dev;
   p.E = static_cast<int>(entries.size());
-  p.resids = st->chain_resids_dev;
-  p.n_resids = static_cast<int>(resids.size());
-  p.partials = reinterpret_cast<float*>(ws + partials_at);
-  p.pbuf_floats = pbuf_floats;
-  p.counters = reinterpret_cast<unsigned*>(ws + counters_at);
+  p.parts = reinterpret_cast<unsigned long long*>(ws + parts_at);
+  p.pbuf_words = pbuf_words;
+  p.words = reinterpret_cast<unsigned long long*>(ws + words_at);
+  p.run_ctr = reinterpret_cast<unsigned*>(ws + run_at);
+  p.bar_count = reinterpret_cast<unsigned long long*>(ws + bar_at);
+  p.prep = reinterpret_cast<uint16_t*>(ws + prep_at);
+  p.prep_info = reinterpret_cast<int*>(ws + prep_info_at);
+  p.prep_ops = reinterpret_cast<const int*>(ws + prep_ops_at);
+  p.n_prep = static_cast<int>(prep_ops.size());
+  p.tiles_off = static_cast<int>(tiles_off);
   p.status = reinterpret_cast<unsigned*>(ws);
-  p.bar_flags = reinterpret_cast<unsigned*>(ws + flags_at);
   p.G = G;
-  p.x_off = x_off;
-  p.h_base = static_cast<int>(h_base);
+  p.x_off = static_cast<int>(x_off);
+  p.scr_off = static_cast<int>(scr_off);
   p.timeout_ns = g_timeout_ns.load();
   st->chain = true;
-  st->M = 1;
+  st->M = M;
   st->launches = 1;
   return Q4_OK;
 }
@@ -1305,16 +1469,22 @@ extern "C" Q4_API int layer_chain_create(const q4_chain_op* ops, int n_ops, int 
       ws = std::max(ws, workspace_bytes(s, M, dev));
     }
   }
-  if (flags & Q4_CHAIN_PERSISTENT) {
+  if ((flags & Q4_CHAIN_PERSISTENT) && (flags & (Q4_CHAIN_GRAPH | Q4_STACK_NO_PDL)))
+    return fail(Q4_ERR_INVALID_ARG, "layer_chain_create: Q4_CHAIN_PERSISTENT with a graph flag");
+  // without a form named: the single launch at M = 1 (measured faster on the
+  // 64-layer decode chain), the graph otherwise or when the list is not eligible
+  const bool named = (flags & (Q4_CHAIN_PERSISTENT | Q4_CHAIN_GRAPH | Q4_STACK_NO_PDL)) != 0;
+  if ((flags & Q4_CHAIN_PERSISTENT) || (!named && M == 1)) {
     q4_stack* st = new q4_stack();
     cudaGetDevice(&st->device);
     rc = create_chain_persistent(ops, n_ops, M, dev, st);
-    if (rc) {
-      free_stack(st);
-      return rc;
+    if (rc == Q4_OK) {
+      *out = st;
+      return Q4_OK;
     }
-    *out = st;
-    return Q4_OK;
+    free_stack(st);
+    if (flags & Q4_CHAIN_PERSISTENT) return rc;
+    if (rc != Q4_ERR_UNSUPPORTED) return rc;
   }
   q4_stack* st = new q4_stack();
   cudaGetDevice(&st->device);

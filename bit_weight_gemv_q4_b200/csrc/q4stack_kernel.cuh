@@ -589,15 +589,30 @@ struct StreamRing {
 // F16: the activations are used in fp16 (en.x16).  Finished tile sums are
 // multiplied by `scale` (2^sigma when F16, times t for NVFP4).
 // SP supplies timeout_ns and partials; PR refills the ring (issue), so the
-// persistent chain kernel runs the same loop with its own per-product ranges.
+// persistent chain kernel runs the same loop with its own per-product ranges;
+// TS stores a tile finished inside the range (the chain adds its step's
+// elementwise part there) and the partial of a tile that began in an earlier
+// warp's range (the chain writes it with a tag).
+struct TileStoreY {
+  template <int M>
+  __device__ __forceinline__ void store(const StackEntryDev* __restrict__ ep, int r, const float (&acc)[2][4],
+                                        int lane) const {
+    store_tile<M>(ep->y, ep->N, r, acc, lane);
+  }
+  template <int M, class SP>
+  __device__ __forceinline__ void first_partial(const SP& sp, int pw, const float (&acc)[2][4], int lane) const {
+    write_partial<M>(sp.partials, pw, 0, acc, lane);
+  }
+};
+
 template <int BITS, int M, int D, int SU, bool F16, int FC, class SP = StackParams,
-          class PR = StreamProducer<SU, M, FC>>
+          class PR = StreamProducer<SU, M, FC>, class TS = TileStoreY>
 __device__ __forceinline__ bool stream_segment(const SP& sp, const StackEntryDev* __restrict__ ep, int e,
                                                long long lb0,
                                                long long nblk, long long gb, StreamRing& rg,
                                                PR& pr, uint64_t policy, float scale,
                                                float (&acc)[2][4], int pw, int& e_first, int& r_first, int& r,
-                                               int& c, int lane) {
+                                               int& c, int lane, const TS& ts = TS()) {
   constexpr int U = SU;
   constexpr int SLOT = StreamSlot<SU, M, FC>::kBytes;
   constexpr bool NV = BITS == kFmtNvfp4;
@@ -667,11 +682,11 @@ __device__ __forceinline__ bool stream_segment(const SP& sp, const StackEntryDev
       if (F16 || NV) scale_acc(acc, scale);
       const long long tile_g = ep->blk_off + static_cast<long long>(r) * bpt;  // the tile's first block
       if (tile_g < gb) {  // began in an earlier warp's range: its partial goes to slot 0 now
-        write_partial<M>(sp.partials, pw, 0, acc, lane);
+        ts.template first_partial<M>(sp, pw, acc, lane);
         e_first = e;
         r_first = r;
       } else {
-        store_tile<M>(ep->y, ep->N, r, acc, lane);
+        ts.template store<M>(ep, r, acc, lane);
       }
       ++r;
       c = 0;

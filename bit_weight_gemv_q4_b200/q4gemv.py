@@ -30,6 +30,7 @@ Q4_STACK_NO_PDL = 1
 Q4_STACK_GRAPH = 2
 Q4_STACK_INDEPENDENT = 4
 Q4_CHAIN_PERSISTENT = 8
+Q4_CHAIN_GRAPH = 16
 Q4_QUANT_ABSMAX = 0
 Q4_QUANT_SIGNED_MAX = 1
 Q4_OP_PRODUCT = 0
@@ -421,7 +422,7 @@ __all__ = [
     "q4_workspace_check", "q4_set_wait_timeout_ns", "q4_unpack_device", "q4_selftest_wait_timeout",
     "layer_stack_create", "layer_stack_run", "layer_stack_check", "layer_stack_destroy",
     "q4_quantize", "q4_quantize_device", "Q4_QUANT_ABSMAX", "Q4_QUANT_SIGNED_MAX",
-    "layer_chain_create", "Q4_CHAIN_PERSISTENT", "ChainOp", "Q4_OP_PRODUCT", "Q4_OP_RESIDUAL_RMSNORM", "Q4_OP_SWIGLU",
+    "layer_chain_create", "Q4_CHAIN_PERSISTENT", "Q4_CHAIN_GRAPH", "ChainOp", "Q4_OP_PRODUCT", "Q4_OP_RESIDUAL_RMSNORM", "Q4_OP_SWIGLU",
     "q4_residual_rmsnorm", "q4_swiglu", "Q4_FMT_NVFP4", "q4_nvfp4_packed_bytes", "q4_pack_nvfp4", "q4_unpack_nvfp4",
     "q4_pack_nvfp4_device", "q4_nvfp4_dequant_device", "Q4_SPEC_MAX_DRAFT", "q4_gather_rows_device",
     "q4_spec_draft", "q4_spec_verify",

@@ -472,33 +472,42 @@ typedef struct q4_chain_op {
   float* resid;        /* RMSNORM: residual stream h (fp32 [M][N], device); else NULL */
 } q4_chain_op;
 
-/* Q4_CHAIN_PERSISTENT (M = 1): the whole chain as ONE cooperative kernel
- * launch instead of a graph of one kernel per op.  Every product is split
- * between all warps of the GPU exactly as a one-product stream-mode stack
- * splits it (its output is bitwise that stack's on the same activations);
- * each CTA computes every step itself into its own shared-memory copy of the
- * next product's activations, keeps the residual streams in shared memory,
- * and writes its slice of each step's outputs; a bounded grid barrier goes
- * before each op that reads another CTA's writes; the weight copies run
- * ahead across ops.  The steps' outputs are bitwise those of
- * q4_residual_rmsnorm / q4_swiglu on the same inputs.  Needs: M = 1;
- * products q4 (K % 256 == 0) or q8 (K % 128 == 0), N > 0; steps with N % 8
- * == 0; no op writing bytes that an earlier (or the same) op reads, no two
- * ops writing the same bytes except RMSNorm ops sharing one residual stream
- * (same pointer and N), no op reading a residual stream through `in`; the
- * largest activation row (2 bytes a value, rounded up to 128) and the
- * residual streams (4 bytes a value) within the 83,712 bytes of shared
- * memory beside the weight rings (a 17,408-value row and a 5,120-value
- * stream take 55,296).  Otherwise Q4_ERR_UNSUPPORTED with the reason.  A grid
- * barrier whose wait gives up sets the status word (layer_stack_check
- * returns Q4_ERR_TIMEOUT).  On the 64-layer decode chain it measured slower
- * than the graph (each CTA recomputes every step over the whole row, and
- * every step waits at a grid barrier for the slowest CTA). */
+/* Q4_CHAIN_PERSISTENT: the whole chain as ONE cooperative kernel launch
+ * instead of a graph of one kernel per op.  Every product is split between
+ * all warps of the GPU as a one-product stream-mode stack splits it (at
+ * M <= 2 its output is bitwise that stack's on the same activations); the
+ * weight copies run ahead across ops.  No fence, atomic or grid barrier sits
+ * between one product and the next: every value another warp reads is
+ * written as a 64-bit word holding it and a tag (run, op), which the reader
+ * polls (bounded).  A split tile is summed by the warp holding its first
+ * chunk; a step's elementwise part (residual add; silu(gate) * up) runs in
+ * the owners of the product before it, and every CTA then finishes the step
+ * for itself (mean square, bf16 activations, fp16 when exact) into its
+ * shared-memory copy of the next product's activations.  Activations of a
+ * product that no op writes (the mixer outputs) are prepared once at the
+ * start of the launch and copied into shared memory while the op before runs.
+ * The steps' outputs are bitwise those of q4_residual_rmsnorm / q4_swiglu on
+ * the same inputs.  Needs: M in 1..4; products q4 or q8 with K a multiple of
+ * 256 / 128 (M <= 2) or 128 / 64 (M >= 3), N > 0; steps with N % 8 == 0 and a
+ * 16-byte aligned out, RMSNorm rows of at most 16,384 values; no op writing
+ * bytes that an earlier (or the same) op reads, no two ops writing the same
+ * bytes except RMSNorm ops sharing one residual stream (same pointer and N),
+ * no op reading a residual stream through `in`; M rows of the largest
+ * activation tensor (2 bytes a value) within the shared memory beside the
+ * weight rings (M = 4: 139,264 bytes, a 17,408-value row).  Otherwise
+ * Q4_ERR_UNSUPPORTED with the reason.  A wait that gives up sets the status
+ * word (layer_stack_check returns Q4_ERR_TIMEOUT and clears the workspace). */
 #define Q4_CHAIN_PERSISTENT 8
+/* Q4_CHAIN_GRAPH: the graph of one kernel per op (programmatic dependent
+ * launch).  Without either flag, layer_chain_create takes the form measured
+ * faster on the 64-layer decode chain for that M: the single launch at
+ * M = 1, the graph at M >= 2; an op list the single launch cannot run takes
+ * the graph. */
+#define Q4_CHAIN_GRAPH 16
 
 /* Validates the ops and captures them, in order, on the current device.
- * flags: Q4_STACK_NO_PDL launches without programmatic dependent launch;
- * Q4_CHAIN_PERSISTENT as above.
+ * flags: Q4_STACK_NO_PDL launches the graph without programmatic dependent
+ * launch; Q4_CHAIN_PERSISTENT, Q4_CHAIN_GRAPH as above.
  * The returned stack runs with layer_stack_run, is checked with
  * layer_stack_check and freed with layer_stack_destroy.  Errors: as
  * layer_stack_create (INVALID_ARG for an unknown kind, a null or misaligned

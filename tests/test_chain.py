@@ -1,12 +1,14 @@
 """The dependent decode chain: the oracle's steps pinned by closed forms and
 identities (CPU); each step kernel against the oracle, the captured chain
-against the same steps called one by one, and a short chain against the
-oracle's own chain (GPU)."""
+against the same steps called one by one, and every op of the two-layer and
+of the 64-layer chain, in both chain forms, against the oracle element by
+element on the GPU's own inputs (GPU)."""
 import numpy as np
 import pytest
 
 from oracle import chain as OC
 import oracle
+import chain_check
 from bit_weight_gemv_q4_b200 import synth, workloads
 
 SMALL = workloads.ChainShape(layers=2, hidden=1024, ffn=2048, kv=256, vocab=4096)
@@ -74,19 +76,24 @@ def test_chain_shape_of_the_decode_stream():
 
 
 def test_chain_shapes_meet_the_one_launch_conditions():
-    """The conditions include/q4gemv.h states for Q4_CHAIN_PERSISTENT (q4
-    products K % 256 == 0, q8 K % 128 == 0, step rows N % 8 == 0, the largest
-    activation row and the residual stream within the 83,712 bytes of shared
-    memory beside the rings) hold for the decode chain and the small one."""
+    """The conditions include/q4gemv.h states for Q4_CHAIN_PERSISTENT hold for
+    the decode chain and the small one at every M: stages of four chunks at
+    M <= 2 and of two at M >= 3 (q4 K a multiple of 256 / 128, q8 K of 128 /
+    64), step rows N % 8 == 0, and the rings, the activation buffer (M rows
+    of the largest K or step row, bf16) and the per-warp tile scratch within
+    227 KB of shared memory less 1 KB."""
     for shape in (workloads.ChainShape(), SMALL):
         tensors = workloads.chain_tensors(shape)
-        for t in tensors:
-            assert t.bits in (4, 8) and t.N > 0
-            assert t.K % (256 if t.bits == 4 else 128) == 0, t.name
         assert shape.hidden % 8 == 0 and shape.ffn % 8 == 0
-        x_bytes = -(-2 * max(max(t.K for t in tensors), shape.hidden, shape.ffn) // 128) * 128
-        rings = -(-(16 * 2 * 4 * 1152 + 16 * 2 * 8) // 128) * 128  # 16 warps x 2 stages x 4 chunks, barriers
-        assert x_bytes + 4 * shape.hidden <= 227 * 1024 - 1024 - rings  # 83,712 bytes
+        for M in (1, 2, 3, 4):
+            su = 4 if M <= 2 else 2
+            for t in tensors:
+                assert t.bits in (4, 8) and t.N > 0
+                assert t.K % (su * (64 if t.bits == 4 else 32)) == 0, t.name
+            x_max = max(max(t.K for t in tensors), shape.hidden, shape.ffn)
+            rings = -(-(16 * 2 * su * 1152 + 16 * 2 * 8) // 128) * 128  # 16 warps x 2 stages, barriers
+            x_bytes = -(-2 * M * x_max // 128) * 128
+            assert rings + x_bytes + 16 * M * 32 * 4 <= 227 * 1024 - 1024, (M, rings, x_bytes)
 
 
 # ---------------------------------------------------------------- oracle chain
@@ -204,7 +211,8 @@ def test_chain_equals_its_steps_called_one_by_one(cuda_device, M):
     import bit_weight_gemv_q4_b200 as q4
 
     torch = _torch()
-    ch = workloads.DeviceChain(SMALL, M, seed=5)
+    ch = workloads.DeviceChain(SMALL, M, seed=5, flags=q4.Q4_CHAIN_GRAPH)
+    assert ch.stack.launches() == 7 * SMALL.layers + 2
     ch.run()
     ch.check()
     graph = _outputs(ch)
@@ -237,65 +245,44 @@ def test_chain_equals_its_steps_called_one_by_one(cuda_device, M):
 
 
 @pytest.mark.gpu
-@pytest.mark.parametrize("M,mode", [(1, "graph"), (2, "graph"), (1, "persistent")])
-def test_chain_against_the_oracle_chain(cuda_device, M, mode):
-    """A two-layer chain against the oracle's chain computed alone: the first
-    activations equal the oracle's away from rounding ties, the first product
-    is within the product tolerance, and the end (after nine dependent steps)
-    stays within 1e-3 in relative norm."""
+@pytest.mark.parametrize("mode", ["graph", "persistent"])
+@pytest.mark.parametrize("M", [1, 2, 4])
+def test_chain_ops_against_the_oracle(cuda_device, M, mode):
+    """Every op of the two-layer chain on the GPU's own inputs: every output
+    of every product within the product tolerance, every activation of every
+    step equal to the oracle's outside the rounding-tie window, the residual
+    stream equal to its fp32 replay.  The first activations (the norm of the
+    embedding) also equal those of the oracle's own chain, computed from the
+    seeded inputs alone."""
     import bit_weight_gemv_q4_b200 as q4
 
-    ch = workloads.DeviceChain(SMALL, M, seed=6, flags=q4.Q4_CHAIN_PERSISTENT if mode == "persistent" else 0)
+    ch = workloads.DeviceChain(SMALL, M, seed=6,
+                               flags=q4.Q4_CHAIN_PERSISTENT if mode == "persistent" else q4.Q4_CHAIN_GRAPH)
     ch.run()
     ch.check()
-    got = _outputs(ch)
+    stats = chain_check.check(ch)
+    assert stats["products"] == 4 * SMALL.layers + 1 and stats["norms"] == 2 * SMALL.layers + 1
+    assert stats["tie_diffs"] <= 1e-3 * stats["values"]
     ref = oracle_chain(SMALL, M, 6)
-    x0 = got["x"][0].view(np.uint16).reshape(M, SMALL.hidden)
-    z0 = ref["z"][("qkv", 0)]
+    x0 = ch.x_qkv[0].cpu().numpy().view(np.uint16).reshape(M, SMALL.hidden)
     diff = x0 != ref["x"][("qkv", 0)]
-    assert not (diff & ~OC.near_bf16_tie(z0, 2.0 ** -17)).any()
-    t0 = workloads.chain_tensors(SMALL)[0]
-    y0 = got["y"][0].reshape(M, t0.N).astype(np.float64)
-    if not diff.any():
-        ok, _, _ = oracle.within_tolerance(y0, ref["y"][0], ref["B"][0])
-        assert ok.all()
-    for i in range(len(got["y"])):
-        t = workloads.chain_tensors(SMALL)[i]
-        y = got["y"][i].reshape(M, t.N).astype(np.float64)
-        r = ref["y"][i]
-        assert np.all(np.isfinite(y))
-        assert np.linalg.norm(y - r) <= 1e-3 * np.linalg.norm(r) + 1e-6, t.name
+    assert not (diff & ~OC.near_bf16_tie(ref["z"][("qkv", 0)], 2.0 ** -17)).any()
     ch.close()
-
-
-@pytest.mark.gpu
-@pytest.mark.parametrize("M", [1, 4])
-def test_full_chain_runs_and_is_reproducible(cuda_device, M):
-    torch = _torch()
-    ch = workloads.DeviceChain(workloads.ChainShape(), M)
-    assert ch.stack.launches() == 64 * 7 + 2
-    ch.run()
-    ch.check()
-    a = ch.logits.cpu().numpy().copy()
-    ch.run()
-    ch.check()
-    b = ch.logits.cpu().numpy().copy()
-    assert np.all(np.isfinite(a)) and np.array_equal(a, b)
-    ch.close()
-    torch.cuda.empty_cache()
 
 
 # ---------------------------------------------------------- the one-launch chain
 @pytest.mark.gpu
-def test_persistent_chain_equals_its_ops_called_one_by_one(cuda_device):
-    """The chain as one cooperative launch (M = 1) is bitwise the same ops run
-    one call at a time on the same buffers: each product as a one-product
-    stream-mode stack (the same split and decode), each step as
-    q4_residual_rmsnorm / q4_swiglu; and two runs agree bitwise."""
+@pytest.mark.parametrize("M", [1, 2])
+def test_persistent_chain_equals_its_ops_called_one_by_one(cuda_device, M):
+    """The chain as one cooperative launch is bitwise the same ops run one
+    call at a time on the same buffers: each product as a one-product
+    stream-mode stack (the same split and decode: stages of four chunks at
+    M <= 2), each step as q4_residual_rmsnorm / q4_swiglu (the same sum of
+    squares); and two runs agree bitwise."""
     import bit_weight_gemv_q4_b200 as q4
 
     torch = _torch()
-    ch = workloads.DeviceChain(SMALL, 1, seed=7, flags=q4.Q4_CHAIN_PERSISTENT)
+    ch = workloads.DeviceChain(SMALL, M, seed=7, flags=q4.Q4_CHAIN_PERSISTENT)
     assert ch.stack.launches() == 1
     ch.run()
     ch.check()
@@ -313,14 +300,14 @@ def test_persistent_chain_equals_its_ops_called_one_by_one(cuda_device):
     ch.h.fill_(float("nan"))
     for kind, bits, N, K, packed, inp, out, resid in ch.ops:
         if kind == q4.Q4_OP_PRODUCT:
-            st = q4.layer_stack_create([(bits, N, K, packed, inp, out)], 1, q4.Q4_STACK_INDEPENDENT)
+            st = q4.layer_stack_create([(bits, N, K, packed, inp, out)], M, q4.Q4_STACK_INDEPENDENT)
             q4.layer_stack_run(st)
             q4.layer_stack_check(st)
             st.close()
         elif kind == q4.Q4_OP_RESIDUAL_RMSNORM:
-            q4.q4_residual_rmsnorm(resid, inp, packed, out, N, 1, bits == 1)
+            q4.q4_residual_rmsnorm(resid, inp, packed, out, N, M, bits == 1)
         else:
-            q4.q4_swiglu(inp, out, N, 1)
+            q4.q4_swiglu(inp, out, N, M)
     torch.cuda.synchronize()
     single = _outputs(ch)
     for i, (a, b) in enumerate(zip(one["y"], single["y"])):
@@ -332,34 +319,53 @@ def test_persistent_chain_equals_its_ops_called_one_by_one(cuda_device):
 
 
 @pytest.mark.gpu
-def test_full_persistent_chain_against_the_graph_chain(cuda_device):
-    """The 64-layer chain as one launch: reproducible bitwise, and its first
-    product and its logits agree with the captured graph's (the two split and
-    decode the products differently, so they agree within rounding)."""
+@pytest.mark.parametrize("M", [1, 4])
+def test_full_chain_ops_against_the_oracle(cuda_device, M):
+    """The 64-layer chain with the output head, captured (one kernel per op)
+    and as one launch: both reproducible bitwise run to run, and every op of
+    each checked on that run's own inputs: 16 rows of every product
+    (including the 248,320-row head) within the product tolerance, every
+    activation of every step outside the rounding-tie window, the final
+    residual stream equal to its fp32 replay."""
     import bit_weight_gemv_q4_b200 as q4
 
     torch = _torch()
-    ch = workloads.DeviceChain(workloads.ChainShape(), 1, flags=q4.Q4_CHAIN_PERSISTENT)
-    ch.run()
-    ch.check()
-    a = ch.logits.cpu().numpy().copy()
-    y0 = ch.w.y[0].cpu().numpy().copy()
-    ch.run()
-    ch.check()
-    assert np.all(np.isfinite(a)) and np.array_equal(a, ch.logits.cpu().numpy())
-    graph = q4.layer_chain_create(ch.ops, 1, 0)
-    q4.layer_stack_run(graph)
-    q4.layer_stack_check(graph)
-    torch.cuda.synchronize()
-    g = ch.logits.cpu().numpy().copy()
-    g0 = ch.w.y[0].cpu().numpy().copy()
-    graph.close()
-    assert np.linalg.norm(y0 - g0) <= 1e-5 * np.linalg.norm(g0)
-    rel = np.linalg.norm(a - g) / np.linalg.norm(g)
-    print("persistent vs graph logits, relative norm", rel)
-    assert rel <= 2e-2
+    ch = workloads.DeviceChain(workloads.ChainShape(), M, flags=q4.Q4_CHAIN_GRAPH)
+    assert ch.stack.launches() == 64 * 7 + 2
+    persistent = q4.layer_chain_create(ch.ops, M, q4.Q4_CHAIN_PERSISTENT)
+    assert persistent.launches() == 1
+    try:
+        for name, stack in (("graph", ch.stack), ("persistent", persistent)):
+            q4.layer_stack_run(stack)
+            q4.layer_stack_check(stack)
+            a = ch.logits.cpu().numpy().copy()
+            q4.layer_stack_run(stack)
+            q4.layer_stack_check(stack)
+            assert np.all(np.isfinite(a)) and np.array_equal(a, ch.logits.cpu().numpy()), name
+            stats = chain_check.check(ch, sample_rows=16)
+            assert stats["products"] == 257 and stats["norms"] == 129 and stats["swiglus"] == 64, name
+            assert stats["tie_diffs"] <= 1e-3 * stats["values"], name
+    finally:
+        persistent.close()
+        ch.close()
+        torch.cuda.empty_cache()
+
+
+@pytest.mark.gpu
+def test_chain_form_chosen_by_default(cuda_device):
+    """Without a form named, the chain runs as one launch at M = 1 and as the
+    graph at M >= 2; naming both forms is an argument error."""
+    import bit_weight_gemv_q4_b200 as q4
+
+    for M, launches in ((1, 1), (2, 7 * SMALL.layers + 2)):
+        ch = workloads.DeviceChain(SMALL, M, seed=9)
+        assert ch.stack.launches() == launches
+        ch.close()
+    ch = workloads.DeviceChain(SMALL, 1, seed=9, flags=q4.Q4_CHAIN_GRAPH)
+    with pytest.raises(q4.Q4Error) as e:
+        q4.layer_chain_create(ch.ops, 1, q4.Q4_CHAIN_PERSISTENT | q4.Q4_CHAIN_GRAPH)
+    assert e.value.code == q4.Q4_ERR_INVALID_ARG
     ch.close()
-    torch.cuda.empty_cache()
 
 
 @pytest.mark.gpu
@@ -369,9 +375,6 @@ def test_persistent_chain_rejects_what_it_cannot_order(cuda_device):
     torch = _torch()
     ch = workloads.DeviceChain(SMALL, 1, seed=8)
     P = q4.Q4_CHAIN_PERSISTENT
-    with pytest.raises(q4.Q4Error) as e:
-        q4.layer_chain_create(ch.ops, 2, P)
-    assert e.value.code == q4.Q4_ERR_UNSUPPORTED
     # two ops writing one buffer
     ops = list(ch.ops)
     k = next(i for i, op in enumerate(ops) if op[0] == q4.Q4_OP_PRODUCT)
@@ -389,6 +392,17 @@ def test_persistent_chain_rejects_what_it_cannot_order(cuda_device):
     with pytest.raises(q4.Q4Error) as e:
         q4.layer_chain_create([(q4.Q4_OP_PRODUCT, 4, 32, 96, w, x, y, None)], 1, P)
     assert e.value.code == q4.Q4_ERR_UNSUPPORTED
+    # at M = 4 (stages of two chunks) a q4 K must be a multiple of 128
+    y4 = torch.zeros(4 * 32, dtype=torch.float32, device="cuda")
+    for K, ok in ((192, False), (256, True)):
+        w = torch.zeros(q4.q4_packed_bytes(4, 32, K), dtype=torch.uint8, device="cuda")
+        x = torch.zeros(4 * K, dtype=torch.int16, device="cuda")
+        if ok:
+            q4.layer_chain_create([(q4.Q4_OP_PRODUCT, 4, 32, K, w, x, y4, None)], 4, P).close()
+        else:
+            with pytest.raises(q4.Q4Error) as e:
+                q4.layer_chain_create([(q4.Q4_OP_PRODUCT, 4, 32, K, w, x, y4, None)], 4, P)
+            assert e.value.code == q4.Q4_ERR_UNSUPPORTED
     ch.close()
 
 

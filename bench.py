@@ -162,43 +162,104 @@ def nvml_index(local_rank: int) -> int:
 # ----------------------------------------------------------------------------
 # CPU oracle on a bounded sample of the workload
 # ----------------------------------------------------------------------------
+def _sample_inputs(tensors, rows_per_tensor, seed, M=1):
+    """(tensor, q, s) of evenly strided whole rows of each tensor, and the
+    activations per distinct K."""
+    import numpy as np
+
+    from bit_weight_gemv_q4_b200 import synth, workloads
+
+    x = {K: synth.activations(seed, synth.act_stream(workloads.activation_stream_id(K)), M, K)
+         for K in workloads.distinct_k(tensors)}
+    inputs = []
+    for t in tensors:
+        n = min(rows_per_tensor, t.N)
+        if n == t.N:
+            q, s = synth.tensor(t.bits, seed, t.tensor_id, t.N, t.K)
+        else:
+            stride = t.N // n
+            r0 = (seed * 7919) % stride
+            qs = [synth.tensor(t.bits, seed, t.tensor_id, t.N, t.K, row0=r, nrows=1)
+                  for r in range(r0, t.N, stride)[:n]]
+            q, s = np.concatenate([a for a, _ in qs]), np.concatenate([b for _, b in qs])
+        inputs.append((t, q, s))
+    return inputs, x
+
+
+def _oracle_pass(inputs, x):
+    import oracle
+
+    for t, q, s in inputs:
+        oracle.gemv(t.bits, q, s, x[t.K])
+
+
+def _sampled_rate(tensors, target_s, seed, M=1, max_rows=4096):
+    """Grows whole-row samples of every tensor until one oracle pass takes
+    about target_s (or the tensors are whole); returns (GB/s of weights,
+    seconds, rows per tensor, sampled bytes)."""
+    from bit_weight_gemv_q4_b200 import workloads
+
+    rows = 2
+    while True:
+        inputs, x = _sample_inputs(tensors, rows, seed, M)
+        nbytes = sum(workloads.weight_bytes(t.bits, q.shape[0], t.K) for t, q, _ in inputs)
+        t0 = time.perf_counter()
+        _oracle_pass(inputs, x)
+        dt = time.perf_counter() - t0
+        whole = all(q.shape[0] == t.N for t, q, _ in inputs)
+        if dt >= 0.7 * target_s or whole or rows >= max_rows:
+            return nbytes / dt / 1e9, dt, rows, nbytes
+        rows = min(max_rows, max(2 * rows, int(rows * target_s / max(dt, 1e-3))))
+
+
 def oracle_sample_rate(target_s: float = 12.0, seed: int = 0):
     """Times the CPU oracle on whole rows spread over every tensor of the decode
     stream; returns (GB/s of weights, threads, sample description, seconds)."""
-    import numpy as np
-
     import oracle
-    from bit_weight_gemv_q4_b200 import synth, workloads
+    from bit_weight_gemv_q4_b200 import workloads
 
     tensors = workloads.decode_stream(fused=True)
-    x = {K: synth.activations(seed, synth.act_stream(workloads.activation_stream_id(K)), 1, K)
-         for K in workloads.distinct_k(tensors)}
-
-    def run(rows_per_tensor):
-        inputs = []
-        for t in tensors:
-            stride = max(1, t.N // rows_per_tensor)
-            r0 = (seed * 7919) % stride
-            rows = list(range(r0, t.N, stride))[:rows_per_tensor]
-            # contiguous blocks of 1 row each: generate them on the host
-            qs = [synth.tensor(t.bits, seed, t.tensor_id, t.N, t.K, row0=r, nrows=1) for r in rows]
-            q = np.concatenate([a for a, _ in qs])
-            s = np.concatenate([b for _, b in qs])
-            inputs.append((t, q, s))
-        nbytes = sum(workloads.weight_bytes(t.bits, q.shape[0], t.K) for t, q, _ in inputs)
-        t0 = time.perf_counter()
-        for t, q, s in inputs:
-            oracle.gemv(t.bits, q, s, x[t.K])
-        return nbytes, time.perf_counter() - t0
-
-    rows = 2
-    nb, dt = run(rows)
-    while dt < 0.7 * target_s and rows < 4096:  # grow the sample until it takes about target_s
-        rows = min(4096, max(2 * rows, int(rows * target_s / max(dt, 1e-3))))
-        nb, dt = run(rows)
+    rate, dt, rows, nbytes = _sampled_rate(tensors, target_s, seed)
     desc = (f"{rows} whole rows (evenly strided) of each of the 257 tensors of the M=1 decode stream, "
-            f"{nb / 1e6:.1f} MB of weights, fp64 oracle, {dt:.1f} s")
-    return nb / dt / 1e9, oracle.threads(), desc, dt
+            f"{nbytes / 1e6:.1f} MB of weights, fp64 oracle, {dt:.1f} s")
+    return rate, oracle.threads(), desc, dt
+
+
+def oracle_config_rates(budget_s: float, seed: int = 0):
+    """The CPU oracle on each single-tensor configuration (q4 4096 x 4096, one
+    27B-shaped q4 layer at M = 1 and 4, the q8 heads of 65,536 and 248,320
+    rows, K = 5120), whole when that fits the budget per configuration, else on
+    whole-row samples; GB/s of weights and the implied microseconds for the
+    whole configuration, with the threads the oracle used."""
+    import oracle
+    from bit_weight_gemv_q4_b200 import workloads
+
+    cases = [("q4_4096x4096_M1", [workloads.Tensor("w", 4, 4096, 4096, 3000)], 1),
+             ("layer_q4_M1", workloads.layer_q4(), 1), ("layer_q4_M4", workloads.layer_q4(), 4)]
+    cases += [(f"{h.name}_q8_{h.N}x{h.K}_M1", [h], 1) for h in workloads.draft_heads()]
+    out = {"threads": oracle.threads()}
+    for name, tensors, M in cases:
+        rate, dt, rows, nbytes = _sampled_rate(tensors, budget_s, seed, M, max_rows=1 << 20)
+        total = workloads.total_bytes(tensors)
+        out[name] = {"GBps": round(rate, 4), "us": round(total / (rate * 1e3), 1),
+                     "sample": "whole" if nbytes == total else f"{nbytes / 1e6:.1f} of {total / 1e6:.1f} MB",
+                     "seconds": round(dt, 2)}
+    return out
+
+
+def oracle_config_rates_in(threads: int, budget_s: float, seed: int = 0):
+    """oracle_config_rates in a fresh process whose OpenMP runtime uses
+    `threads` threads (the oracle as it stands; the thread count is the
+    runtime's environment variable)."""
+    import subprocess
+
+    env = dict(os.environ, OMP_NUM_THREADS=str(threads))
+    cmd = [sys.executable, os.path.abspath(__file__), "--oracle-configs", "--cpu-seconds", str(budget_s),
+           "--seed", str(seed)]
+    proc = subprocess.run(cmd, env=env, stdout=subprocess.PIPE, stderr=subprocess.PIPE, text=True, timeout=900)
+    if proc.returncode != 0:
+        return {"error": proc.stderr.strip().splitlines()[-1:] or ["failed"]}
+    return json.loads(proc.stdout.strip().splitlines()[-1])
 
 
 # ----------------------------------------------------------------------------
@@ -438,7 +499,7 @@ def run_ours(args, d: Dist):
     # product's outputs complete before the next reads its activations), as
     # one ordered persistent launch and as a graph of one launch per product
     other = {}
-    for flags, name in ((0, "ordered"), (q4.Q4_STACK_GRAPH, "graph")):
+    for flags, name in ((q4.Q4_STACK_ORDERED, "ordered"), (q4.Q4_STACK_GRAPH, "graph")):
         alt = st.make_stack(flags)
         run_alt = lambda: q4.layer_stack_run(alt)  # noqa: E731
         for _ in range(max(3, args.warmup // 2)):
@@ -550,7 +611,9 @@ def run_ours(args, d: Dist):
     cpu = None
     if d.rank == 0 and d.world == 1 and not args.no_cpu_baseline:  # the oracle is timed at N = 1 only
         rate, threads, desc, _ = oracle_sample_rate(args.cpu_seconds, args.seed)
-        cpu = {"value": round(rate, 4), "unit": UNIT, "cores": threads, "kind": "oracle", "sample": desc}
+        cpu = {"value": round(rate, 4), "unit": UNIT, "cores": threads, "kind": "oracle", "sample": desc,
+               "per_config_all_cores": oracle_config_rates(args.cpu_seconds / 12, args.seed),
+               "per_config_one_core": oracle_config_rates_in(1, args.cpu_seconds / 12, args.seed)}
 
     traffic = profiled_traffic()
     clocks = sampler.summary()
@@ -623,39 +686,29 @@ def run_ours(args, d: Dist):
 
 
 def run_reference(args, d: Dist):
-    """The CPU oracle on the host cores: each step is a bounded sample of the
-    same workload; value = sampled weight bytes / time, same metric."""
+    """The CPU oracle on the host cores: each step is one pass of the oracle
+    over the same bounded sample of the workload as cpu_baseline (whole rows
+    of every tensor of the decode stream), sized so the whole --steps K
+    --warmup W run takes about --reference-seconds; value = sampled weight
+    bytes / time, same metric."""
     if d.rank != 0:
         return None
-    import numpy as np
-
     import oracle
-    from bit_weight_gemv_q4_b200 import synth, workloads
+    from bit_weight_gemv_q4_b200 import workloads
 
     tensors = workloads.decode_stream(fused=True)
-    x = {K: synth.activations(args.seed, synth.act_stream(workloads.activation_stream_id(K)), 1, K)
-         for K in workloads.distinct_k(tensors)}
-    rows = args.reference_rows
-    inputs = []
-    for t in tensors:
-        stride = max(1, t.N // rows)
-        qs = [synth.tensor(t.bits, args.seed, t.tensor_id, t.N, t.K, row0=r, nrows=1) for r in range(0, t.N, stride)[:rows]]
-        inputs.append((t, np.concatenate([a for a, _ in qs]), np.concatenate([b for _, b in qs])))
-    nbytes = sum(workloads.weight_bytes(t.bits, q.shape[0], t.K) for t, q, _ in inputs)
-
-    def step():
-        for t, q, s in inputs:
-            oracle.gemv(t.bits, q, s, x[t.K])
-
+    per_step = max(0.05, args.reference_seconds / (args.steps + args.warmup))
+    _, _, rows, nbytes = _sampled_rate(tensors, per_step, args.seed)
+    inputs, x = _sample_inputs(tensors, rows, args.seed)
     for _ in range(args.warmup):
-        step()
+        _oracle_pass(inputs, x)
     t0 = time.perf_counter()
     for _ in range(args.steps):
-        step()
+        _oracle_pass(inputs, x)
     dt = (time.perf_counter() - t0) / args.steps
     value = nbytes / dt / 1e9
     desc = (f"{rows} whole rows (evenly strided) of each of the 257 tensors of the M=1 decode stream per step, "
-            f"{nbytes / 1e6:.1f} MB of weights")
+            f"{nbytes / 1e6:.1f} MB of weights, fp64 oracle")
     return {
         "impl": "reference",
         "metric": METRIC,
@@ -752,7 +805,10 @@ def main():
     ap.add_argument("--no-configs", action="store_true", help="skip the per-configuration product timings")
     ap.add_argument("--headline-only", action="store_true",
                     help="skip the format, width, chain and speculative sections (as every N > 1 run does)")
-    ap.add_argument("--reference-rows", type=int, default=8, help="rows per tensor per reference step")
+    ap.add_argument("--reference-seconds", type=float, default=150.0,
+                    help="CPU time of the whole reference run (its per-step sample is sized from it)")
+    ap.add_argument("--oracle-configs", action="store_true",
+                    help="print the CPU oracle's per-configuration rates as one JSON line and exit")
     ap.add_argument("--profile-case", action="store_true", help="run the small ncu case and exit")
     ap.add_argument("--profile-bits", type=int, default=4)
     ap.add_argument("--profile-launches", type=int, default=3)
@@ -766,6 +822,9 @@ def main():
 
     if args.profile_case:
         run_profile_case(args)
+        return
+    if args.oracle_configs:  # host only: no CUDA
+        print(json.dumps(oracle_config_rates(args.cpu_seconds, args.seed)), flush=True)
         return
 
     if args.impl == "reference" and int(os.environ.get("RANK", "0")) != 0:

@@ -956,7 +956,9 @@ extern "C" Q4_API int layer_stack_create(const q4_stack_entry* entries, int n_en
   }
   q4_stack* st = new q4_stack();
   cudaGetDevice(&st->device);
-  const bool graph = (flags & (Q4_STACK_GRAPH | Q4_STACK_NO_PDL)) != 0 || !stack_eligible(entries, n_entries);
+  // graph mode unless a persistent mode is asked for (and the list is eligible)
+  const bool graph = (flags & (Q4_STACK_GRAPH | Q4_STACK_NO_PDL)) != 0 ||
+                     (flags & (Q4_STACK_INDEPENDENT | Q4_STACK_ORDERED)) == 0 || !stack_eligible(entries, n_entries);
   // stream mode also needs whole q4 chunks (K a multiple of 64); else ordered.
   // Its stages hold kStreamU chunks when every product's chunks per tile is a
   // multiple of kStreamU, else 2.

@@ -29,6 +29,7 @@ Q4_ERR_UNSUPPORTED = -7
 Q4_STACK_NO_PDL = 1
 Q4_STACK_GRAPH = 2
 Q4_STACK_INDEPENDENT = 4
+Q4_STACK_ORDERED = 32
 Q4_CHAIN_PERSISTENT = 8
 Q4_CHAIN_GRAPH = 16
 Q4_QUANT_ABSMAX = 0

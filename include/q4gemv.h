@@ -388,9 +388,12 @@ typedef struct q4_stack q4_stack;
 #define Q4_STACK_NO_PDL 1 /* graph mode, launched without programmatic dependent launch */
 #define Q4_STACK_GRAPH 2  /* graph mode: one kernel per product, captured as a CUDA graph */
 #define Q4_STACK_INDEPENDENT 4 /* stream mode: the caller asserts no product reads another's output */
+#define Q4_STACK_ORDERED 32    /* ordered persistent mode */
 
 /* Validates every entry and prepares the stack on the current device.
- * Default (ordered persistent) mode: one cooperative kernel, one CTA per SM,
+ * flags == 0 is graph mode (measured faster than the ordered mode on the
+ * 257-product decode stream: 3.87 against 5.74 ms).
+ * Ordered mode (Q4_STACK_ORDERED): one cooperative kernel, one CTA per SM,
  * runs the whole list; each product's weights are streamed exactly as by
  * q4_gemv / q8_gemv (bitwise-equal outputs), the bulk-copy rings prefetch the
  * next product's weights while the current one finishes, and a grid-wide
@@ -410,7 +413,8 @@ typedef struct q4_stack q4_stack;
  * (tiles may be split at other places, and fp16 sums round differently).
  * Both persistent modes need every product non-empty with an even number of
  * chunks per tile; other lists use graph mode.  Stream mode also needs every
- * q4 K to be a multiple of 64; otherwise the ordered mode is used.
+ * q4 K to be a multiple of 64; otherwise the ordered mode is used.  A list
+ * not eligible for the persistent modes takes graph mode.
  * NVFP4 products (bits = Q4_FMT_NVFP4) run in stream mode only: a list holding
  * one needs flags == Q4_STACK_INDEPENDENT and every product eligible for it,
  * else UNSUPPORTED.  They decode each code byte and scale pair in one

@@ -68,7 +68,7 @@ def _run_bench(args, env_extra=None):
 
 
 def test_reference_arm_prints_the_contract_line():
-    r = _run_bench(["--impl", "reference", "--steps", "1", "--warmup", "3", "--reference-rows", "1"])
+    r = _run_bench(["--impl", "reference", "--steps", "1", "--warmup", "3", "--reference-seconds", "0.2"])
     assert r.returncode == 0, r.stderr[-2000:]
     lines = [l for l in r.stdout.splitlines() if l.startswith("{")]
     assert len(lines) == 1
@@ -86,7 +86,7 @@ def test_reference_arm_prints_the_contract_line():
 
 
 def test_reference_arm_runs_on_rank_zero_only():
-    r = _run_bench(["--impl", "reference", "--gpus", "2", "--steps", "1", "--warmup", "3", "--reference-rows", "1"],
+    r = _run_bench(["--impl", "reference", "--gpus", "2", "--steps", "1", "--warmup", "3", "--reference-seconds", "0.2"],
                    {"RANK": "1", "LOCAL_RANK": "1", "WORLD_SIZE": "2"})
     assert r.returncode == 0, r.stderr[-2000:]
     assert r.stdout.strip() == ""

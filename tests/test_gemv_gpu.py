@@ -146,8 +146,9 @@ def sampled_rows(N, count=8, seed=0):
 
 @pytest.mark.parametrize("head", workloads.draft_heads(), ids=lambda h: h.name)
 def test_q8_vocab_heads(q4, head):
-    """Draft-head projections K=5120 q8 at M=1: the mapped head whole, the full
-    vocabulary on sampled rows (generated on the device; the oracle's rows are
+    """Draft-head projections K=5120 q8 at M=1, the mapped (65,536 rows) and the
+    full vocabulary (248,320 rows): every output within the tolerance of the
+    oracle (the weights are generated on the device, the oracle's copy is
     regenerated on the host)."""
     t = T()
     seed = 0
@@ -155,15 +156,10 @@ def test_q8_vocab_heads(q4, head):
     x = synth.activations(seed, synth.act_stream(head.tensor_id), 1, head.K)
     y, guards = H.run_gemv(8, packed, head.N, head.K, H.to_device_x(x), 1)
     assert guards
-    if head.N <= 65536:
-        q, s = synth.tensor(8, seed, head.tensor_id, head.N, head.K)
-        H.assert_parity(y, q, s, x, 8)
-    else:
-        for r in sampled_rows(head.N, 64):
-            q, s = synth.tensor(8, seed, head.tensor_id, head.N, head.K, row0=r, nrows=1)
-            H.assert_parity(y[:, r:r + 1], q, s, x, 8)
     del packed
     t.cuda.empty_cache()
+    q, s = synth.tensor(8, seed, head.tensor_id, head.N, head.K)
+    H.assert_parity(y, q, s, x, 8)
 
 
 # --------------------------------------------------------------- edge cases

@@ -1,7 +1,10 @@
 """The captured layer stack: same results as one call per product, oracle parity,
-and the full 64-layer decode stream (13.7 GB) checked on sampled rows."""
+and the full 64-layer decode stream (13.7 GB) checked on sampled rows and, in
+every mode, on every output."""
 import numpy as np
 import pytest
+
+import oracle
 
 from bit_weight_gemv_q4_b200 import synth, workloads
 from bit_weight_gemv_q4_b200.workloads import Tensor
@@ -79,7 +82,7 @@ def _check_stack(q4, tensors, M, flags, expect_launches):
 
 @pytest.mark.parametrize("M", [1, 4])
 def test_stack_modes_equal_single_calls_and_oracle(q4, M):
-    persistent = _check_stack(q4, MIXED, M, 0, 1)
+    persistent = _check_stack(q4, MIXED, M, q4.Q4_STACK_ORDERED, 1)
     graph = _check_stack(q4, MIXED, M, q4.Q4_STACK_GRAPH, len(MIXED))
     nopdl = _check_stack(q4, MIXED, M, q4.Q4_STACK_NO_PDL, len(MIXED))
     for a, b, c in zip(persistent, graph, nopdl):
@@ -134,7 +137,7 @@ def test_full_decode_stream_sampled(q4, M, mode):
     persistent kernel; sampled rows of several tensors against the oracle."""
     torch = H.torch()
     tensors = workloads.decode_stream(fused=True)
-    st = workloads.DeviceStream(tensors, M, flags=0 if mode == "ordered" else q4.Q4_STACK_INDEPENDENT)
+    st = workloads.DeviceStream(tensors, M, flags=q4.Q4_STACK_ORDERED if mode == "ordered" else q4.Q4_STACK_INDEPENDENT)
     # one persistent kernel for the 257 products (stream mode: after xprep_kernel)
     assert st.stack.launches() == (1 if mode == "ordered" else 2)
     st.run()
@@ -155,6 +158,48 @@ def test_full_decode_stream_sampled(q4, M, mode):
     torch.cuda.empty_cache()
 
 
+@pytest.mark.parametrize("M", [1, 4])
+def test_full_decode_stream_every_output(q4, M):
+    """Every output of all 257 products of one decode step (64 layers + the
+    248,320-row q8 head: 13.7 GB of weights), in stream, ordered and graph
+    mode, within the product tolerance of the fp64 oracle, which is
+    regenerated tensor by tensor on the host (13.7 GB of codes per M).  The
+    modes split the products differently (stream mode: one stream-K range over
+    all of them, across product boundaries), so this also covers every place a
+    split falls at full size."""
+    torch = H.torch()
+    tensors = workloads.decode_stream(fused=True)
+    st = workloads.DeviceStream(tensors, M, flags=q4.Q4_STACK_INDEPENDENT)
+    got = {}
+    for mode, flags in (("stream", None), ("ordered", q4.Q4_STACK_ORDERED), ("graph", q4.Q4_STACK_GRAPH)):
+        stack = st.stack if flags is None else st.make_stack(flags)
+        for y in st.y:
+            y.fill_(float("nan"))
+        q4.layer_stack_run(stack)
+        q4.layer_stack_check(stack)
+        torch.cuda.synchronize()
+        got[mode] = [_y(st, i).copy() for i in range(len(tensors))]
+        if flags is not None:
+            stack.close()
+    x = {K: synth.activations(st.seed, synth.act_stream(workloads.activation_stream_id(K)), M, K)
+         for K in workloads.distinct_k(tensors)}
+    st.close()
+    torch.cuda.empty_cache()
+    worst = 0.0
+    for i, t in enumerate(tensors):
+        q, s = synth.tensor(t.bits, 0, t.tensor_id, t.N, t.K)
+        y_ref, B = oracle.gemv(t.bits, q, s, x[t.K])
+        del q, s
+        for mode, ys in got.items():
+            ok, err, bound = oracle.within_tolerance(ys[i], y_ref, B)
+            if not ok.all():
+                m, r = np.argwhere(~ok)[0]
+                raise AssertionError(f"{mode} {t.name}: {(~ok).sum()} of {ok.size} outside tolerance, first row {r} "
+                                     f"m {m}: {ys[i][m, r]} vs {y_ref[m, r]}")
+            worst = max(worst, float((err / np.maximum(B, 1e-30)).max()))
+    print(f"M={M}: worst |y - y_ref| / sum|w x| over all outputs and modes: {worst:.3g}")
+
+
 @pytest.mark.parametrize("mode", ["ordered", "stream", "graph"])
 @pytest.mark.parametrize("M", [1, 3])
 def test_degenerate_rows_in_stacks(q4, mode, M):
@@ -172,7 +217,7 @@ def test_degenerate_rows_in_stacks(q4, mode, M):
         entries.append((bits, N, K, H.to_device_packed(bits, q, s, N, K), x_dev, y))
         hosts.append((q, s))
         ys.append(y)
-    flags = {"ordered": 0, "stream": q4.Q4_STACK_INDEPENDENT, "graph": q4.Q4_STACK_GRAPH}[mode]
+    flags = {"ordered": q4.Q4_STACK_ORDERED, "stream": q4.Q4_STACK_INDEPENDENT, "graph": q4.Q4_STACK_GRAPH}[mode]
     st = q4.layer_stack_create(entries, M, flags)
     q4.layer_stack_run(st)
     q4.layer_stack_check(st)

@@ -766,6 +766,25 @@ def run_profile_case(args):
         print(json.dumps({"profile_case": "spec verify", "V": V, "n_map": n_map, "drafts": n,
                           "launches": args.profile_launches, "out": out.cpu().tolist()}))
         return
+    if args.profile_shape:
+        # single products (one gemv_kernel launch each) in copies rotated so
+        # that no launch finds its weights in L2 (the per_config section's
+        # "graph" figures)
+        bits, N, K = (int(v) for v in args.profile_shape.split(","))
+        one = workloads.weight_bytes(bits, N, K)
+        l2 = torch.cuda.get_device_properties(0).L2_cache_size
+        copies = max(2, -(-2 * l2 // one))
+        tensors = [workloads.Tensor(f"shape.{i}", bits, N, K, 3000 + i) for i in range(copies)]
+        st = workloads.DeviceStream(tensors, args.m, seed=args.seed, flags=q4.Q4_STACK_GRAPH)
+        for _ in range(args.profile_launches):
+            st.run()
+        torch.cuda.synchronize()
+        st.check()
+        print(json.dumps({"profile_case": f"single products {bits},{N},{K} x {copies} copies, graph mode",
+                          "M": args.m, "runs": args.profile_launches, "launches_per_run": copies,
+                          "kernel_source_sha": kernel_source_sha()}))
+        st.close()
+        return
     if args.profile_layers > 0:
         tensors = workloads.decode_stream(fused=True)[: 4 * args.profile_layers]
         if args.profile_nvfp4:
@@ -815,6 +834,8 @@ def main():
     ap.add_argument("--profile-layers", type=int, default=0)
     ap.add_argument("--profile-nvfp4", action="store_true")
     ap.add_argument("--profile-spec", action="store_true", help="profile case: the keep / reject kernels")
+    ap.add_argument("--profile-shape", default="",
+                    help="profile case: bits,N,K of single products, in rotating copies (graph mode)")
     ap.add_argument("--m", type=int, default=1)
     args = ap.parse_args()
     if args.warmup < 3 and not args.profile_case:

@@ -71,6 +71,7 @@ struct GemvParams {
   int T, C;                  // tiles, chunks per tile
   int P;                     // warps with work (P <= TC / U)
   int khalf;                 // q4 with K % 64 == 32: the last chunk of a tile holds one group
+  int interleave;            // warp p of the split runs as warp p / gridDim.x of CTA p % gridDim.x
   unsigned long long timeout_ns;
 };
 
@@ -517,8 +518,14 @@ __device__ __forceinline__ unsigned tile_contributors(const Partition& pt, const
 
 // Last arrival on a split tile: sum the partials of its contributing warps in
 // warp order (one row per lane) and store the tile; then re-zero its counter.
+// The partials' loads go out 32 at a time (contributors x rows) before any is
+// added, so a tile split between many warps costs a few round trips to L2, not
+// one per contributor; the additions keep warp order.  Out of line: its
+// registers do not weigh on the streaming loop.
+constexpr int kReduceBatch = 32;
+
 template <int M>
-__device__ __forceinline__ void reduce_tile(const Partition& pt, const SplitTile& st, int lane) {
+__device__ __noinline__ void reduce_tile(const Partition& pt, const SplitTile& st, int lane) {
   const int p_lo = owner_of(st.blo, pt.TB, pt.P);
   const int p_hi = owner_of(st.bhi - 1, pt.TB, pt.P);
   const long long row = static_cast<long long>(st.r) * kTileRows + lane;
@@ -527,14 +534,29 @@ __device__ __forceinline__ void reduce_tile(const Partition& pt, const SplitTile
   // begins inside the tile, so the tile is its first: slot 0.
   const int slot_lo = (range_begin(p_lo, pt.TB, pt.P) == st.blo) ? 0 : 1;
   const float* base = pt.partials + lane;
+  float sum[M];
 #pragma unroll
-  for (int m = 0; m < M; ++m) {
-    float sum = __ldcg(base + (static_cast<long long>(p_lo) * 2 + slot_lo) * (M * kTileRows) + m * kTileRows);
-#pragma unroll 4
-    for (int q = p_lo + 1; q <= p_hi; ++q)
-      sum += __ldcg(base + (static_cast<long long>(q) * 2) * (M * kTileRows) + m * kTileRows);
-    if (row < st.N) st.y[m * st.N + row] = sum;
+  for (int m = 0; m < M; ++m)
+    sum[m] = __ldcg(base + (static_cast<long long>(p_lo) * 2 + slot_lo) * (M * kTileRows) + m * kTileRows);
+  // word j of the rest: contributor p_lo + 1 + j / M, row m = j % M
+  const int rest = (p_hi - p_lo) * M;
+  for (int j0 = 0; j0 < rest; j0 += kReduceBatch) {
+    float v[kReduceBatch];
+#pragma unroll
+    for (int k = 0; k < kReduceBatch; ++k) {
+      const int j = j0 + k;
+      const int q = p_lo + 1 + j / M, m = j % M;
+      v[k] = j < rest ? __ldcg(base + (static_cast<long long>(q) * 2) * (M * kTileRows) + m * kTileRows) : 0.f;
+    }
+#pragma unroll
+    for (int k = 0; k < kReduceBatch; ++k) {
+      const int j = j0 + k;
+      if (j < rest) sum[j % M] += v[k];
+    }
   }
+#pragma unroll
+  for (int m = 0; m < M; ++m)
+    if (row < st.N) st.y[m * st.N + row] = sum[m];
   if (lane == 0) *st.counter = 0u;
 }
 
@@ -600,7 +622,11 @@ __global__ void __launch_bounds__(NW * 32, 1) gemv_kernel(const GemvParams p) {
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
   const int gi = lane >> 2, ti = lane & 3;
-  const int pw = blockIdx.x * NW + warp;
+  // warp index in the split: consecutive within a CTA, or, for a product
+  // split between fewer warps than the GPU holds, interleaved over one CTA per
+  // SM so that every SM streams (p.interleave)
+  const int pw = p.interleave ? warp * static_cast<int>(gridDim.x) + static_cast<int>(blockIdx.x)
+                              : static_cast<int>(blockIdx.x) * NW + warp;
 
   const uint32_t ring = smem_addr(smem + warp * Cfg::kRingBytes);
   const uint32_t bars = smem_addr(smem + Cfg::kBarOffset) + warp * D * 8;

@@ -181,7 +181,9 @@ __global__ void __launch_bounds__(NW * 32, 1) stack_kernel(const StackParams sp)
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
   const int gi = lane >> 2, ti = lane & 3;
-  const int pw = blockIdx.x * NW + warp;
+  // interleaved over the CTAs, as in gemv_kernel: a product split between
+  // fewer warps than the grid holds spreads them over every SM
+  const int pw = warp * static_cast<int>(gridDim.x) + static_cast<int>(blockIdx.x);
   const uint32_t ring = smem_addr(smem + warp * D * SLOT);
   const uint32_t bars = smem_addr(smem + NW * D * SLOT) + warp * D * 8;
 

@@ -766,6 +766,18 @@ def run_profile_case(args):
         print(json.dumps({"profile_case": "spec verify", "V": V, "n_map": n_map, "drafts": n,
                           "launches": args.profile_launches, "out": out.cpu().tolist()}))
         return
+    if args.profile_chain_layers > 0:
+        shape = workloads.ChainShape(layers=args.profile_chain_layers)
+        ch = workloads.DeviceChain(shape, args.m, seed=args.seed, flags=q4.Q4_CHAIN_PERSISTENT)
+        for _ in range(args.profile_launches):
+            ch.run()
+        torch.cuda.synchronize()
+        ch.check()
+        print(json.dumps({"profile_case": f"dependent chain of {args.profile_chain_layers} layers, one launch",
+                          "M": args.m, "launches": args.profile_launches, "weight_bytes": ch.weight_bytes,
+                          "kernel_source_sha": kernel_source_sha()}))
+        ch.close()
+        return
     if args.profile_shape:
         # single products (one gemv_kernel launch each) in copies rotated so
         # that no launch finds its weights in L2 (the per_config section's
@@ -834,6 +846,8 @@ def main():
     ap.add_argument("--profile-layers", type=int, default=0)
     ap.add_argument("--profile-nvfp4", action="store_true")
     ap.add_argument("--profile-spec", action="store_true", help="profile case: the keep / reject kernels")
+    ap.add_argument("--profile-chain-layers", type=int, default=0,
+                    help="profile case: the dependent chain of this many layers as one launch (M = --m)")
     ap.add_argument("--profile-shape", default="",
                     help="profile case: bits,N,K of single products, in rotating copies (graph mode)")
     ap.add_argument("--m", type=int, default=1)

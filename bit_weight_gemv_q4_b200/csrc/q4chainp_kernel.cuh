@@ -606,7 +606,7 @@ __device__ __forceinline__ bool chain_finish_product(const ChainParams& cp, cons
   float sum[M];
   tile_rows<M>(acc, warp_scratch<M>(cp), lane, sum);
   const int p_hi = owner_of(tg + bpt - 1, TB, ep->P);
-  constexpr int GQ = M <= 2 ? 8 / M : 2;  // contributors whose words one round trip loads
+  constexpr int GQ = 16 / M;  // contributors whose words one round trip loads (16 words)
   bool got = true;
   for (int q0 = pw + 1; q0 <= p_hi; q0 += GQ) {
     const int nq = min(GQ, p_hi - q0 + 1);

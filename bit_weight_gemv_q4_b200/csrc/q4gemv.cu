@@ -64,6 +64,9 @@ constexpr int kCtasPerSm = Q4_TUNE_CTAS_PER_SM;
 constexpr int kRingChunks = Q4_TUNE_RING_CHUNKS;
 constexpr int kMaxU = Q4_TUNE_MAX_U;
 static_assert(kRingChunks % 2 == 0 && kRingChunks >= 4, "ring must hold two stages of two chunks");
+#ifndef Q4_TUNE_STREAM_MIXED  // 0: M = 2..4 stream lists carry every activation slice in the slots
+#define Q4_TUNE_STREAM_MIXED 1
+#endif
 #ifndef Q4_TUNE_STACK_D
 #define Q4_TUNE_STACK_D 2
 #endif
@@ -690,6 +693,8 @@ void* select_stack_kernel(int M, int su, int fc) {
   static void* const ordered[4] = {stack_kernel_ptr<1>(), stack_kernel_ptr<2>(), stack_kernel_ptr<3>(),
                                    stack_kernel_ptr<4>()};
   if (su == 0) return ordered[M - 1];
+  if (fc == 5)  // some tensors resident: M = 2 / 3, stages of kStreamU chunks only
+    return M == 2 ? stream_kernel_ptr<2, kStreamU, 5>() : stream_kernel_ptr<3, kStreamU, 5>();
   if (fc >= 3)  // resident activations: M = 1, stages of kStreamU chunks only
     return fc == 3 ? stream_kernel_ptr<1, kStreamU, 3>() : stream_kernel_ptr<1, kStreamU, 4>();
   if (fc == 0) return su == 2 ? StreamRow<2, 0>::at(M) : StreamRow<kStreamU, 0>::at(M);
@@ -701,16 +706,16 @@ void* select_stack_kernel(int M, int su, int fc) {
 // su: stream mode with stages of su chunks (weights + activation slice of M
 // rows), or 0 for ordered mode (weights only, stages of kStackU chunks).
 // fc 3 / 4 (resident activations): weights-only slots, one more barrier, and
-// the activation copies (rx_bytes) from the next 128-byte boundary.
+// the activation copies (rx_bytes) from the next 128-byte boundary; fc 5:
+// the same with slots that also hold a slice.
 int stack_smem_bytes(int su, int M, int fc, int rx_bytes = 0) {
+  constexpr int nw = kStackNW;
+  if (su == 0) return nw * kStackD * q4k::kStackU * q4k::Format<4>::kChunkBytes + nw * kStackD * 8;
   const int cb = fc == 2 ? q4k::Wide<6>::kChunkBytes : q4k::Format<4>::kChunkBytes;
-  if (su != 0 && fc >= 3) {
-    const int rings = kStackNW * kStackD * su * q4k::Format<4>::kChunkBytes;
-    return (rings + kStackNW * kStackD * 8 + 8 + 127) / 128 * 128 + rx_bytes;
-  }
-  const int slot = su == 0 ? q4k::kStackU * q4k::Format<4>::kChunkBytes
-                           : su * (cb + M * q4k::Format<4>::kKPerChunk * 2);
-  return kStackNW * kStackD * slot + kStackNW * kStackD * 8;
+  const int xb = fc == 3 || fc == 4 ? 0 : M * q4k::Format<4>::kKPerChunk * 2;
+  const int rings = nw * kStackD * su * (cb + xb);
+  if (fc >= 3) return (rings + nw * kStackD * 8 + 8 + 127) / 128 * 128 + rx_bytes;
+  return rings + nw * kStackD * 8;
 }
 
 void free_stack(q4_stack* st) {
@@ -785,6 +790,7 @@ int create_persistent(const q4_stack_entry* entries, int n, int M, int su, const
   // mode keeps one per tile of every product
   const size_t counters = (static_cast<size_t>(independent ? total_tiles : max_t) * 4 + 255) / 256 * 256;
   int rx_bytes = 0;  // stream mode with resident activations: their bytes in shared memory
+  int fc_sel = fc;   // the kernel's class: fc, or 3 + fc (all resident), or 5 (some resident)
   // stream mode: per distinct (x, K, format) a chunk-major copy of x and its XInfo
   std::vector<q4k::XPrepJob> jobs;
   std::vector<size_t> job_of(static_cast<size_t>(n), 0), x16_off, info_off;
@@ -824,21 +830,52 @@ int create_persistent(const q4_stack_entry* entries, int n, int M, int su, const
       jobs[k].xc = reinterpret_cast<uint16_t*>(base + x16_off[k]);
       jobs[k].info = reinterpret_cast<q4k::XInfo*>(base + info_off[k]);
     }
-    // resident activations (M = 1, classes 0 / 1, stages of kStreamU): every
-    // CTA keeps each prepared tensor in shared memory when they all fit
+    // resident activations (stages of kStreamU).  M = 1, classes 0 / 1:
+    // every CTA keeps each prepared tensor in shared memory when they all
+    // fit.  M = 2 / 3, class 0 (class 5): the tensors in the q4 geometry that
+    // fit beside the slots, narrowest first; a q8 product whose activations
+    // have such a copy reads it (half a chunk of it per q8 chunk); the other
+    // products' slices stay in the slots.  (At M = 4 the slots leave no room
+    // for 5120 values per row; with 14 warps per CTA instead of 16 there is,
+    // but the decode stream ran 5 % slower than with every slice in the slots.)
+    for (auto& j : jobs) j.rx_off = -1;
     if (M == 1 && su == kStreamU && fc <= 1) {
       int off = 0;
       for (auto& j : jobs) {
         j.rx_off = off;
         off += static_cast<int>((j.K * 2 + 127) / 128 * 128);
       }
-      if (stack_smem_bytes(su, M, fc + 3, off) <= kSmemLimit) rx_bytes = off;
+      if (stack_smem_bytes(su, M, fc + 3, off) <= kSmemLimit) {
+        rx_bytes = off;
+        fc_sel = fc + 3;
+      }
+    } else if (Q4_TUNE_STREAM_MIXED && (M == 2 || M == 3) && su == kStreamU && fc == 0) {
+      std::vector<size_t> order;
+      for (size_t k = 0; k < jobs.size(); ++k)
+        if (jobs[k].KC == q4k::Format<4>::kKPerChunk) order.push_back(k);
+      std::stable_sort(order.begin(), order.end(), [&](size_t a, size_t b) { return jobs[a].K < jobs[b].K; });
+      int off = 0;
+      for (size_t k : order) {
+        const long long bytes = static_cast<long long>(M) * jobs[k].K * 2;  // a multiple of 128: K % 64 == 0
+        if (stack_smem_bytes(su, M, 5, static_cast<int>(std::min<long long>(off + bytes, 1 << 30))) > kSmemLimit)
+          continue;
+        jobs[k].rx_off = off;
+        off += static_cast<int>(bytes);
+      }
+      if (off > 0) {
+        rx_bytes = off;
+        fc_sel = 5;
+      }
     }
     for (int i = 0; i < n; ++i) {
-      const q4k::XPrepJob& j = jobs[job_of[static_cast<size_t>(i)]];
-      host[static_cast<size_t>(i)].xc = j.xc;
-      host[static_cast<size_t>(i)].xinfo = j.info;
-      host[static_cast<size_t>(i)].rx_off = j.rx_off;
+      const q4k::XPrepJob* j = &jobs[job_of[static_cast<size_t>(i)]];
+      host[static_cast<size_t>(i)].xc = j->xc;
+      if (fc_sel == 5 && j->rx_off < 0 && entries[i].bits == 8) {
+        for (const auto& r : jobs)  // the q4-geometry copy of the same activations, if resident
+          if (r.rx_off >= 0 && r.x == j->x && r.K == j->K) j = &r;
+      }
+      host[static_cast<size_t>(i)].xinfo = j->info;
+      host[static_cast<size_t>(i)].rx_off = j->rx_off;
     }
     err = cudaMalloc(&st->xprep_dev, sizeof(q4k::XPrepJob) * jobs.size());
     if (err == cudaSuccess)
@@ -853,7 +890,6 @@ int create_persistent(const q4_stack_entry* entries, int n, int M, int su, const
   if (err == cudaSuccess)
     err = cudaMemcpy(st->entries_dev, host.data(), sizeof(q4k::StackEntryDev) * host.size(), cudaMemcpyHostToDevice);
   if (err != cudaSuccess) return cuda_fail(err, "layer_stack_create: allocation");
-  const int fc_sel = rx_bytes > 0 ? fc + 3 : fc;
   st->fn = select_stack_kernel(M, su, fc_sel);
   st->smem = stack_smem_bytes(su, M, fc_sel, rx_bytes);
   st->block = kStackNW * 32;

@@ -370,9 +370,34 @@ struct ChunkRegs {
   uint4 scales;    // q4: (R0: 2c, 2c+1) (R0+8) (R1) (R1+8);  q8: .x = (R0, R0+8), .y = (R1, R1+8)
 };
 
+// acc[0..1] += s d[0..1] and acc[2..3] += s8 d[2..3], each a fused fp32
+// multiply-add rounded once.  X2 issues them as two paired fp32 FMAs
+// (fma.rn.f32x2, the same two roundings per element): for products whose
+// odd columns are stored (M >= 2).  With one token column the odd outputs are
+// dead and the compiler drops their FMAs, so the scalar form is the cheaper.
+__device__ __forceinline__ void fma_f32x2(float& a0, float& a1, float s, float d0, float d1) {
+  asm("{\n\t.reg .b64 pa, ps, pd;\n\t"
+      "mov.b64 pa, {%0, %1};\n\tmov.b64 ps, {%2, %2};\n\tmov.b64 pd, {%3, %4};\n\t"
+      "fma.rn.f32x2 pa, ps, pd, pa;\n\tmov.b64 {%0, %1}, pa;\n\t}"
+      : "+f"(a0), "+f"(a1)
+      : "f"(s), "f"(d0), "f"(d1));
+}
+template <bool X2>
+__device__ __forceinline__ void scale_fma(float (&acc)[4], float s, float s8, const float (&d)[4]) {
+  if constexpr (X2) {
+    fma_f32x2(acc[0], acc[1], s, d[0], d[1]);
+    fma_f32x2(acc[2], acc[3], s8, d[2], d[3]);
+  } else {
+    acc[0] = fmaf(s, d[0], acc[0]);
+    acc[1] = fmaf(s, d[1], acc[1]);
+    acc[2] = fmaf(s8, d[2], acc[2]);
+    acc[3] = fmaf(s8, d[3], acc[3]);
+  }
+}
+
 // F16: activations and codes in fp16 (xprep_kernel made x fp16-exact),
-// else bf16.
-template <bool F16 = false>
+// else bf16.  X2: see scale_fma.
+template <bool F16 = false, bool X2 = false>
 __device__ __forceinline__ void q4_chunk_mac(float (&acc)[2][4], const ChunkRegs& r, const uint4& xa,
                                              const uint4& xb) {
   const uint32_t sc[4] = {r.scales.x, r.scales.y, r.scales.z, r.scales.w};
@@ -390,17 +415,12 @@ __device__ __forceinline__ void q4_chunk_mac(float (&acc)[2][4], const ChunkRegs
       mma_m16n8k16<F16>(d, a, xg.z, xg.w);
       const float2 s_r = half2_bits_to_float2(sc[2 * h]);       // row 16h + gi: groups 2c, 2c+1
       const float2 s_r8 = half2_bits_to_float2(sc[2 * h + 1]);  // row 16h + gi + 8
-      const float sr = G ? s_r.y : s_r.x;
-      const float sr8 = G ? s_r8.y : s_r8.x;
-      acc[h][0] = fmaf(sr, d[0], acc[h][0]);
-      acc[h][1] = fmaf(sr, d[1], acc[h][1]);
-      acc[h][2] = fmaf(sr8, d[2], acc[h][2]);
-      acc[h][3] = fmaf(sr8, d[3], acc[h][3]);
+      scale_fma<X2>(acc[h], G ? s_r.y : s_r.x, G ? s_r8.y : s_r8.x, d);
     }
   }
 }
 
-template <bool F16 = false>
+template <bool F16 = false, bool X2 = false>
 __device__ __forceinline__ void q8_chunk_mac(float (&acc)[2][4], const ChunkRegs& r, const uint4& xa) {
 #pragma unroll
   for (int h = 0; h < 2; ++h) {
@@ -422,10 +442,7 @@ __device__ __forceinline__ void q8_chunk_mac(float (&acc)[2][4], const ChunkRegs
       mma_m16n8k16<false>(d, lo, xa.z, xa.w);
     }
     const float2 s = half2_bits_to_float2(h ? r.scales.y : r.scales.x);  // rows 16h + gi, 16h + gi + 8
-    acc[h][0] = fmaf(s.x, d[0], acc[h][0]);
-    acc[h][1] = fmaf(s.x, d[1], acc[h][1]);
-    acc[h][2] = fmaf(s.y, d[2], acc[h][2]);
-    acc[h][3] = fmaf(s.y, d[3], acc[h][3]);
+    scale_fma<X2>(acc[h], s.x, s.y, d);
   }
 }
 
@@ -744,9 +761,9 @@ __global__ void __launch_bounds__(NW * 32, 1) gemv_kernel(const GemvParams p) {
         }
       }
       if (BITS == 4)
-        q4_chunk_mac(acc, regs[j], xa, xb);
+        q4_chunk_mac<false, (M > 1)>(acc, regs[j], xa, xb);
       else
-        q8_chunk_mac(acc, regs[j], xa);
+        q8_chunk_mac<false, (M > 1)>(acc, regs[j], xa);
     }
     c += U;
     if (c == p.C) {

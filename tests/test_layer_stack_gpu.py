@@ -89,13 +89,17 @@ def test_stack_modes_equal_single_calls_and_oracle(q4, M):
         assert np.array_equal(a, b) and np.array_equal(a, c)
 
 
-@pytest.mark.parametrize("M", [1, 2, 4])
+@pytest.mark.parametrize("M", [1, 2, 3, 4])
 @pytest.mark.parametrize("tensors", [MIXED, MIXED4], ids=["stages2", "stages4"])
 def test_stream_mode_of_independent_products(q4, M, tensors):
     """Stream mode splits the concatenated products between warps differently
     from one call per product: the outputs are compared with the oracle (every
     row) and with single calls within the product tolerance, and two runs are
-    bitwise identical."""
+    bitwise identical.  With stages of four chunks at M = 2 and 3 the
+    activations of K 256 and 5120 stay resident in shared memory (q8 products
+    with K 5120 and 256 read the q4 layout's copy), while those of K 17408 and
+    of the q8 product with K 128 (no q4 product shares them) travel with the
+    weights; at M = 1 every tensor is resident, at M = 4 none."""
     torch = H.torch()
     st = workloads.DeviceStream(tensors, M, flags=q4.Q4_STACK_INDEPENDENT)
     assert st.stack.launches() == 2  # activation preparation + stream kernel

@@ -579,10 +579,10 @@ def run_ours(args, d: Dist):
 
     # the dependent chain: the same products with the steps between them
     # (residual + RMSNorm, SwiGLU), in the form layer_chain_create picks by
-    # default (M1: one cooperative launch; M4: one CUDA graph with programmatic
-    # dependent launch) and in the other form
+    # default (one CUDA graph with programmatic dependent launch) and as one
+    # cooperative launch
     chain = {} if secondary else skipped
-    for key, M, flags in ((("M1", 1, 0), ("M4", 4, 0), ("M1_graph", 1, q4.Q4_CHAIN_GRAPH),
+    for key, M, flags in ((("M1", 1, 0), ("M4", 4, 0), ("M1_persistent", 1, q4.Q4_CHAIN_PERSISTENT),
                            ("M4_persistent", 4, q4.Q4_CHAIN_PERSISTENT)) if secondary else ()):
         ch = workloads.DeviceChain(workloads.ChainShape(), M, seed=args.seed, flags=flags)
         try:

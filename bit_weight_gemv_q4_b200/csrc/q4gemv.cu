@@ -88,7 +88,8 @@ constexpr int kStackNW = Q4_TUNE_STACK_NW;  // warps per CTA of the persistent k
 #endif
 constexpr int kChainPF = Q4_TUNE_CHAIN_PF;  // one-launch chain: stages prefetched into L2 beyond each ring
 // shared memory a CTA may use (B200: 227 KB per CTA)
-constexpr int kSmemLimit = 227 * 1024 / kCtasPerSm;
+constexpr int kSmemLimit = 227 * 1024 / kCtasPerSm;  // single-product kernel, per CTA
+constexpr int kStackSmemLimit = 227 * 1024;           // persistent kernels: one CTA per SM
 constexpr size_t kWsHeader = 256;
 
 int fail(int code, const char* fmt, ...) {
@@ -188,7 +189,13 @@ int chunk_bytes_of(int bits) {
                                                                        : q4k::Format<4>::kChunkBytes;
 }
 
-long long max_warps(const DeviceInfo& dev) { return static_cast<long long>(dev.sms) * kCtasPerSm * kNW; }
+// CTAs per SM a single product's grid fills at most (kCtasPerSm: fits; fewer
+// leaves room for the next kernel's CTAs)
+#ifndef Q4_TUNE_GRID_PER_SM
+#define Q4_TUNE_GRID_PER_SM Q4_TUNE_CTAS_PER_SM
+#endif
+constexpr int kGridPerSm = Q4_TUNE_GRID_PER_SM;
+long long max_warps(const DeviceInfo& dev) { return static_cast<long long>(dev.sms) * kGridPerSm * kNW; }
 
 // Warps that split one product of TB stream-K blocks (the single-product
 // kernel and, per product, the ordered persistent kernel, so their outputs
@@ -197,6 +204,20 @@ long long max_warps(const DeviceInfo& dev) { return static_cast<long long>(dev.s
 long long product_warps(long long TB, long long most, const DeviceInfo& dev) {
   const long long floor_warps = std::min(TB, static_cast<long long>(dev.sms) * Q4_TUNE_MIN_WARPS_PER_SM);
   return std::min(most, std::max(TB / Q4_TUNE_MIN_BLOCKS, floor_warps));
+}
+
+// Warps a single product (or a product of an ordered stack, which splits it
+// the same way) is split between, in blocks of U chunks.  A product with
+// fewer than 4 blocks per warp is bound by its split tiles' fix-up more than
+// by streaming: at most kPartBatch / M contributors per tile there, so that
+// each tile's owner collects their words in one batch of loads (measured on
+// the 1024 x 5120 product at M = 4: 5.1 us instead of 10.3; on the
+// 5120 x 17408 one, 9 blocks per warp, the cap cost 19 %).
+long long split_warps(const Shape& s, int U, int M, long long most, const DeviceInfo& dev) {
+  long long P = product_warps(s.TC / U, most, dev);
+  if (s.TC / U < 4 * P)
+    P = std::max<long long>(1, std::min(P, static_cast<long long>(s.T) * std::max(1, q4k::kPartBatch / std::max(M, 1))));
+  return P;
 }
 
 // Workspace layout: [status word | partial sums | tile counters].  The
@@ -296,14 +317,14 @@ int prepare(int bits, const void* packed, int64_t N, int64_t K, const uint16_t* 
 
   const int U = pick_u(s.C);
   const bool xs = stage_x(bits, U, M, s.K);
-  const long long P = product_warps(s.TC / U, max_warps(dev), dev);
+  const long long P = split_warps(s, U, M, max_warps(dev), dev);
   // Split between every warp the GPU holds: consecutive warps per CTA (the
   // contributors of a split tile mostly share an SM: measured 10 % faster on
   // the 17,408 x 5120 products).  Between fewer: one CTA per SM with the warps
   // interleaved over them, so every SM streams (measured 8-10 % faster on the
   // 4096- and 5120-row products than filling half the SMs).
   const bool interleave = P < max_warps(dev);
-  const int G = interleave ? static_cast<int>(std::min<long long>(P, static_cast<long long>(dev.sms) * kCtasPerSm))
+  const int G = interleave ? static_cast<int>(std::min<long long>(P, static_cast<long long>(dev.sms) * kGridPerSm))
                            : static_cast<int>((P + kNW - 1) / kNW);
   unsigned char* ws = static_cast<unsigned char*>(workspace);
 
@@ -622,13 +643,15 @@ extern "C" Q4_API int q4_gemv_noalloc(const void* packed, int64_t N, int64_t K, 
   Launch L;
   if ((rc = prepare(4, packed, N, K, x, M, y, ws, kNoAllocWorkspaceBytes, who, &L))) return rc;
   L.params.y = y;
-  // The array keeps whatever the last call left: clear the status word and
-  // this shape's tile counters, which must start at zero.
+  // The array keeps whatever the last call left (a call whose wait gave up
+  // leaves words set): clear the status word and the split-tile words this
+  // launch's warps use, which must start at zero.
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   unsigned char* base = static_cast<unsigned char*>(ws);
   cudaError_t err = cudaMemsetAsync(base, 0, kWsHeader, st);
   if (err == cudaSuccess)
-    err = cudaMemsetAsync(base + kWsHeader + partials_bytes(dev), 0, static_cast<size_t>(s.T) * 4, st);
+    err = cudaMemsetAsync(base + kWsHeader, 0,
+                          static_cast<size_t>(L.params.P) * M * q4k::kTileRows * sizeof(unsigned long long), st);
   if (err != cudaSuccess) return cuda_fail(err, "q4_gemv_noalloc: cudaMemsetAsync");
   return launch(L, st, true);
 }
@@ -766,7 +789,8 @@ int create_persistent(const q4_stack_entry* entries, int n, int M, int su, const
     if (reinterpret_cast<uintptr_t>(en.packed) % 16 || reinterpret_cast<uintptr_t>(en.x) % 16 ||
         reinterpret_cast<uintptr_t>(en.y) % 4)
       return fail(Q4_ERR_ALIGN, "%s: packed and x must be 16-byte aligned, y 4-byte aligned", who);
-    const long long P = product_warps(s.TC / q4k::kStackU, warps, dev);
+    // ordered mode splits each product as a single call does (bitwise the same y)
+    const long long P = split_warps(s, q4k::kStackU, M, warps, dev);
     q4k::StackEntryDev& d = host[static_cast<size_t>(i)];
     d.packed = static_cast<const uint8_t*>(en.packed);
     d.x = en.x;
@@ -845,7 +869,7 @@ int create_persistent(const q4_stack_entry* entries, int n, int M, int su, const
         j.rx_off = off;
         off += static_cast<int>((j.K * 2 + 127) / 128 * 128);
       }
-      if (stack_smem_bytes(su, M, fc + 3, off) <= kSmemLimit) {
+      if (stack_smem_bytes(su, M, fc + 3, off) <= kStackSmemLimit) {
         rx_bytes = off;
         fc_sel = fc + 3;
       }
@@ -857,7 +881,7 @@ int create_persistent(const q4_stack_entry* entries, int n, int M, int su, const
       int off = 0;
       for (size_t k : order) {
         const long long bytes = static_cast<long long>(M) * jobs[k].K * 2;  // a multiple of 128: K % 64 == 0
-        if (stack_smem_bytes(su, M, 5, static_cast<int>(std::min<long long>(off + bytes, 1 << 30))) > kSmemLimit)
+        if (stack_smem_bytes(su, M, 5, static_cast<int>(std::min<long long>(off + bytes, 1 << 30))) > kStackSmemLimit)
           continue;
         jobs[k].rx_off = off;
         off += static_cast<int>(bytes);
@@ -1422,7 +1446,7 @@ int create_chain_persistent(const q4_chain_op* ops, int n, int M, const DeviceIn
   const long long scr_off = x_off + (X + 127) / 128 * 128;
   const long long tiles_off = scr_off + static_cast<long long>(kStackNW) * M * q4k::kTileRows * 4;
   const long long smem = tiles_off + (M * max_tiles * 4 + 127) / 128 * 128;
-  if (smem > kSmemLimit - 1024)
+  if (smem > kStackSmemLimit - 1024)
     return fail(Q4_ERR_UNSUPPORTED, "%s: activations of %lld values x M = %d exceed shared memory", who, x_max, M);
   // workspace: [status | partial buffers | tagged words | per-CTA run counters | barrier counter]
   auto up256 = [](size_t v) { return (v + 255) / 256 * 256; };
@@ -1517,10 +1541,9 @@ extern "C" Q4_API int layer_chain_create(const q4_chain_op* ops, int n_ops, int 
   }
   if ((flags & Q4_CHAIN_PERSISTENT) && (flags & (Q4_CHAIN_GRAPH | Q4_STACK_NO_PDL)))
     return fail(Q4_ERR_INVALID_ARG, "layer_chain_create: Q4_CHAIN_PERSISTENT with a graph flag");
-  // without a form named: the single launch at M = 1 (measured faster on the
-  // 64-layer decode chain), the graph otherwise or when the list is not eligible
-  const bool named = (flags & (Q4_CHAIN_PERSISTENT | Q4_CHAIN_GRAPH | Q4_STACK_NO_PDL)) != 0;
-  if ((flags & Q4_CHAIN_PERSISTENT) || (!named && M == 1)) {
+  // without a form named: the graph (measured faster on the 64-layer decode
+  // chain at M = 1 and 4); the single launch only when asked for
+  if (flags & Q4_CHAIN_PERSISTENT) {
     q4_stack* st = new q4_stack();
     cudaGetDevice(&st->device);
     rc = create_chain_persistent(ops, n_ops, M, dev, st);
@@ -1529,8 +1552,7 @@ extern "C" Q4_API int layer_chain_create(const q4_chain_op* ops, int n_ops, int 
       return Q4_OK;
     }
     free_stack(st);
-    if (flags & Q4_CHAIN_PERSISTENT) return rc;
-    if (rc != Q4_ERR_UNSUPPORTED) return rc;
+    return rc;
   }
   q4_stack* st = new q4_stack();
   cudaGetDevice(&st->device);

@@ -39,6 +39,16 @@
 #include <cuda_fp16.h>
 #include <stdint.h>
 
+// Single-product kernel: CTAs per SM it is compiled for, and whether it
+// lets the next kernel launch (programmatic dependent launch) at its start
+// rather than after its own dependency wait.
+#ifndef Q4_TUNE_CTAS_PER_SM
+#define Q4_TUNE_CTAS_PER_SM 1
+#endif
+#ifndef Q4_TUNE_EARLY_TRIGGER
+#define Q4_TUNE_EARLY_TRIGGER 0
+#endif
+
 namespace q4k {
 
 constexpr int kTileRows = 32;        // rows per tile: two m16 tensor-core tiles
@@ -63,8 +73,8 @@ struct GemvParams {
   const uint8_t* packed;     // packed chunks, 16-byte aligned
   const uint16_t* x;         // bf16 bits [M][K]
   float* y;                  // [M][N]
-  float* partials;           // [P][2][M][32] split-tile partial sums
-  unsigned* counters;        // [T] arrival counters, zero between launches
+  float* partials;           // split-tile words, [P][M][32] tagged 64-bit (zero between launches)
+  unsigned* counters;        // unused by gemv_kernel (the workspace keeps the region)
   unsigned* status;          // status word
   long long N, K;
   long long TC;              // T * C, the number of chunks
@@ -616,6 +626,98 @@ __device__ __forceinline__ void finish_split_tiles(const Partition& pt, int pw, 
 // ----------------------------------------------------------------------------
 constexpr int kXPadBytes = 64;
 
+// ----------------------------------------------------------------------------
+// Split tiles of the single-product kernel.  A warp whose range begins inside
+// a tile publishes its part of the tile as tagged 64-bit words (the float's
+// bits, tag kPartTag in the high half; one word per token row and tile row):
+// a 64-bit store is single-copy atomic, so a reader that sees the tag sees the
+// value, and no fence or counter is needed.  The warp holding the tile's
+// first block (its owner) polls its contributors' words, adds the parts in
+// warp order, stores the tile and writes the words back to zero, so every
+// completed launch leaves them zero for the next (which reads none of them
+// before griddepcontrol.wait has seen this one complete).  Words: [warp][M][32].
+// ----------------------------------------------------------------------------
+constexpr unsigned long long kPartTag = 1ull << 32;
+constexpr int kPartBatch = 32;  // words a lane keeps in flight while polling
+
+__device__ __forceinline__ void part_store(unsigned long long* p, unsigned long long v) {
+  asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+}
+__device__ __forceinline__ unsigned long long part_load(const unsigned long long* p) {
+  unsigned long long v;
+  asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+  return v;
+}
+
+// The tile's values by row: lane l gets row l of every token column m < M
+// from the mma accumulator layout (half h: rows 16h + gi and 16h + gi + 8,
+// columns 2ti and 2ti + 1).
+template <int M>
+__device__ __forceinline__ void tile_rows_shfl(const float (&acc)[2][4], int lane, float (&out)[M]) {
+  const int h = lane >> 4, hi = (lane >> 3) & 1, g = lane & 7;
+#pragma unroll
+  for (int m = 0; m < M; ++m) {
+    const int src = g * 4 + (m >> 1);
+    const float v00 = __shfl_sync(0xFFFFFFFFu, acc[0][m & 1], src);
+    const float v01 = __shfl_sync(0xFFFFFFFFu, acc[0][2 + (m & 1)], src);
+    const float v10 = __shfl_sync(0xFFFFFFFFu, acc[1][m & 1], src);
+    const float v11 = __shfl_sync(0xFFFFFFFFu, acc[1][2 + (m & 1)], src);
+    out[m] = h ? (hi ? v11 : v10) : (hi ? v01 : v00);
+  }
+}
+
+// A contributor's part of the tile that began before its range.
+template <int M>
+__device__ __forceinline__ void publish_part(unsigned long long* words, int pw, const float (&acc)[2][4], int lane) {
+  float v[M];
+  tile_rows_shfl<M>(acc, lane, v);
+#pragma unroll
+  for (int m = 0; m < M; ++m)
+    part_store(words + (static_cast<long long>(pw) * M + m) * kTileRows + lane, kPartTag | __float_as_uint(v[m]));
+}
+
+// The owner (warp pw) of tile r: its own part (acc) plus contributors
+// pw + 1 .. p_hi, in warp order, into y; false when a wait gave up.
+template <int M>
+__device__ __noinline__ bool own_tile(unsigned long long* words, float* y, long long N, int r, int pw, int p_hi,
+                                      const float (&acc)[2][4], int lane, unsigned long long timeout_ns) {
+  float sum[M];
+  tile_rows_shfl<M>(acc, lane, sum);
+  constexpr int GQ = kPartBatch / M;  // contributors per round trip
+  unsigned long long t0 = 0;
+  for (int q0 = pw + 1; q0 <= p_hi; q0 += GQ) {
+    const int nq = min(GQ, p_hi - q0 + 1);
+    unsigned long long* base = words + static_cast<long long>(q0) * M * kTileRows + lane;
+    unsigned long long w[kPartBatch];
+#pragma unroll
+    for (int k = 0; k < kPartBatch; ++k) w[k] = k < nq * M ? part_load(base + k * kTileRows) : kPartTag;
+    while (true) {
+      bool mine = true;
+#pragma unroll
+      for (int k = 0; k < kPartBatch; ++k) mine = mine && (w[k] >> 32) == 1u;
+      if (__all_sync(0xFFFFFFFFu, mine)) break;
+      if (t0 == 0) t0 = global_timer_ns();
+      const unsigned long long waited = __shfl_sync(0xFFFFFFFFu, global_timer_ns() - t0, 0);
+      if (waited > timeout_ns) return false;
+#pragma unroll
+      for (int k = 0; k < kPartBatch; ++k)
+        if (k < nq * M && (w[k] >> 32) != 1u) w[k] = part_load(base + k * kTileRows);
+    }
+#pragma unroll
+    for (int k = 0; k < kPartBatch; ++k) {
+      if (k < nq * M) {
+        sum[k % M] += __uint_as_float(static_cast<unsigned>(w[k]));
+        part_store(base + k * kTileRows, 0ull);
+      }
+    }
+  }
+  const long long row = static_cast<long long>(r) * kTileRows + lane;
+#pragma unroll
+  for (int m = 0; m < M; ++m)
+    if (row < N) y[m * N + row] = sum[m];
+  return true;
+}
+
 template <int BITS, int NW, int D, int U>
 struct GemvConfig {
   static constexpr int kChunkBytes = Format<BITS>::kChunkBytes;
@@ -630,7 +732,7 @@ struct GemvConfig {
 __host__ __device__ constexpr long long x_row_stride_bytes(long long K) { return 2 * K + kXPadBytes; }
 
 template <int BITS, int M, int NW, int D, int U, bool XS>
-__global__ void __launch_bounds__(NW * 32, 1) gemv_kernel(const GemvParams p) {
+__global__ void __launch_bounds__(NW * 32, Q4_TUNE_CTAS_PER_SM) gemv_kernel(const GemvParams p) {
   using Cfg = GemvConfig<BITS, NW, D, U>;
   constexpr int CB = Cfg::kChunkBytes;
   constexpr int KC = Format<BITS>::kKPerChunk;
@@ -660,6 +762,7 @@ __global__ void __launch_bounds__(NW * 32, 1) gemv_kernel(const GemvParams p) {
   }
   const int nst = static_cast<int>((e - b) / U);
 
+  if (Q4_TUNE_EARLY_TRIGGER) grid_dependents_launch();
   if (lane == 0) {
     for (int s = 0; s < D; ++s) mbar_init(bars + 8 * s, 1);
     if (XS && warp == 0) mbar_init(xbar, 1);
@@ -689,7 +792,7 @@ __global__ void __launch_bounds__(NW * 32, 1) gemv_kernel(const GemvParams p) {
 
   // The weights do not depend on the previous kernel; x, y and the workspace may.
   grid_dependency_wait();
-  grid_dependents_launch();
+  if (!Q4_TUNE_EARLY_TRIGGER) grid_dependents_launch();
 
   if (XS && threadIdx.x == 0) {
     mbar_arrive_expect_tx(xbar, static_cast<uint32_t>(M * 2 * p.K));
@@ -709,8 +812,7 @@ __global__ void __launch_bounds__(NW * 32, 1) gemv_kernel(const GemvParams p) {
   const uint32_t xs_lane = xsm + (x_lane ? gi : 0) * xstride + 16 * ti;
   const uint16_t* xrow = p.x + static_cast<long long>(x_lane ? gi : 0) * p.K + 8 * ti;
   float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-  float acc_first[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-  int r_first = -1;  // split first tile, finished after the last chunk
+  unsigned long long* words = reinterpret_cast<unsigned long long*>(p.partials);
   uint4 xa = make_uint4(0, 0, 0, 0), xb = make_uint4(0, 0, 0, 0);
 
   bool ok = true;
@@ -768,15 +870,10 @@ __global__ void __launch_bounds__(NW * 32, 1) gemv_kernel(const GemvParams p) {
     c += U;
     if (c == p.C) {
       const long long tile_lo = static_cast<long long>(r) * p.C;
-      if (tile_lo < b) {  // the first tile began in an earlier warp's range
-        r_first = r;
-#pragma unroll
-        for (int h = 0; h < 2; ++h)
-#pragma unroll
-          for (int q = 0; q < 4; ++q) acc_first[h][q] = acc[h][q];
-      } else {
+      if (tile_lo < b)  // the first tile began in an earlier warp's range: its owner adds this part
+        publish_part<M>(words, pw, acc, lane);
+      else
         store_tile<M>(p.y, p.N, r, acc, lane);
-      }
       ++r;
       c = 0;
 #pragma unroll
@@ -796,21 +893,17 @@ __global__ void __launch_bounds__(NW * 32, 1) gemv_kernel(const GemvParams p) {
     if (XS) (void)mbar_wait_bounded(xbar, 0, p.timeout_ns);
     return;
   }
-  if (nst == 0) return;
-  // the range may end inside a tile: that tile's partial goes to slot 0 when
-  // it is also the tile the range began in, else to slot 1
-  int r_last = -1, slot_last = 1;
-  if (c != 0) {
-    r_last = r;
-    slot_last = (static_cast<long long>(r) * p.C <= b) ? 0 : 1;
+  if (nst == 0 || c == 0) return;
+  // the range ends inside tile r: its part, if the tile began in an earlier
+  // range; else this warp owns the tile
+  if (static_cast<long long>(r) * p.C < b) {
+    publish_part<M>(words, pw, acc, lane);
+    return;
   }
-  const Partition pt{TB, p.P, p.partials};
-  const int bpt = p.C / U;  // blocks per tile
-  const SplitTile first{p.y, p.N, r_first, p.counters + (r_first < 0 ? 0 : r_first),
-                        static_cast<long long>(r_first) * bpt, static_cast<long long>(r_first + 1) * bpt};
-  const SplitTile last{p.y, p.N, r_last, p.counters + (r_last < 0 ? 0 : r_last),
-                       static_cast<long long>(r_last) * bpt, static_cast<long long>(r_last + 1) * bpt};
-  finish_split_tiles<M>(pt, pw, first, acc_first, last, slot_last, acc, lane);
+  const long long bpt = p.C / U;  // blocks per tile
+  const int p_hi = owner_of((static_cast<long long>(r) + 1) * bpt - 1, TB, p.P);
+  if (!own_tile<M>(words, p.y, p.N, r, pw, p_hi, acc, lane, p.timeout_ns) && lane == 0)
+    atomicOr(p.status, kStatusTimeout);
 }
 
 // ----------------------------------------------------------------------------

@@ -353,11 +353,11 @@ def test_full_chain_ops_against_the_oracle(cuda_device, M):
 
 @pytest.mark.gpu
 def test_chain_form_chosen_by_default(cuda_device):
-    """Without a form named, the chain runs as one launch at M = 1 and as the
-    graph at M >= 2; naming both forms is an argument error."""
+    """Without a form named, the chain runs as the graph at every M; naming
+    both forms is an argument error."""
     import bit_weight_gemv_q4_b200 as q4
 
-    for M, launches in ((1, 1), (2, 7 * SMALL.layers + 2)):
+    for M, launches in ((1, 7 * SMALL.layers + 2), (2, 7 * SMALL.layers + 2)):
         ch = workloads.DeviceChain(SMALL, M, seed=9)
         assert ch.stack.launches() == launches
         ch.close()

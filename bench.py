@@ -226,17 +226,19 @@ def oracle_sample_rate(target_s: float = 12.0, seed: int = 0):
 
 
 def oracle_config_rates(budget_s: float, seed: int = 0):
-    """The CPU oracle on each single-tensor configuration (q4 4096 x 4096, one
-    27B-shaped q4 layer at M = 1 and 4, the q8 heads of 65,536 and 248,320
-    rows, K = 5120), whole when that fits the budget per configuration, else on
-    whole-row samples; GB/s of weights and the implied microseconds for the
-    whole configuration, with the threads the oracle used."""
+    """The CPU oracle on each configuration (q4 4096 x 4096, one 27B-shaped q4
+    layer at M = 1 and 4, the q8 heads of 65,536 and 248,320 rows, K = 5120,
+    and the 257-product decode stream at M = 1), whole when that fits the
+    budget per configuration, else on whole-row samples; GB/s of weights and
+    the implied microseconds for the whole configuration, with the threads the
+    oracle used."""
     import oracle
     from bit_weight_gemv_q4_b200 import workloads
 
     cases = [("q4_4096x4096_M1", [workloads.Tensor("w", 4, 4096, 4096, 3000)], 1),
              ("layer_q4_M1", workloads.layer_q4(), 1), ("layer_q4_M4", workloads.layer_q4(), 4)]
     cases += [(f"{h.name}_q8_{h.N}x{h.K}_M1", [h], 1) for h in workloads.draft_heads()]
+    cases.append(("decode_stream_M1", workloads.decode_stream(fused=True), 1))
     out = {"threads": oracle.threads()}
     for name, tensors, M in cases:
         rate, dt, rows, nbytes = _sampled_rate(tensors, budget_s, seed, M, max_rows=1 << 20)

@@ -64,8 +64,8 @@ constexpr int kCtasPerSm = Q4_TUNE_CTAS_PER_SM;
 constexpr int kRingChunks = Q4_TUNE_RING_CHUNKS;
 constexpr int kMaxU = Q4_TUNE_MAX_U;
 static_assert(kRingChunks % 2 == 0 && kRingChunks >= 4, "ring must hold two stages of two chunks");
-#ifndef Q4_TUNE_STREAM_MIXED  // 0: M = 2..4 stream lists carry every activation slice in the slots
-#define Q4_TUNE_STREAM_MIXED 1
+#ifndef Q4_TUNE_STREAM_GROUPS  // 0: M >= 2 stream lists run as one launch
+#define Q4_TUNE_STREAM_GROUPS 1
 #endif
 #ifndef Q4_TUNE_STACK_D
 #define Q4_TUNE_STACK_D 2
@@ -676,6 +676,15 @@ struct q4_stack {
   int xprep_jobs = 0;
   int xprep_ctas = 1;  // CTAs per job
   int rx_bytes = 0;    // stream mode: resident activations' bytes (0: slices through the rings)
+  // stream mode split into groups (M >= 2): one stream_kernel launch per
+  // group after the preparation, each with its own entries, stages and
+  // resident activations; empty when the list runs as one launch (fn, params)
+  struct Group {
+    void* fn = nullptr;
+    int smem = 0;
+    q4k::StackParams params{};
+  };
+  std::vector<Group> groups;
   // persistent chain (Q4_CHAIN_PERSISTENT): one cooperative chain_kernel launch
   bool chain = false;
   q4k::ChainParams chain_params{};
@@ -716,8 +725,11 @@ void* select_stack_kernel(int M, int su, int fc) {
   static void* const ordered[4] = {stack_kernel_ptr<1>(), stack_kernel_ptr<2>(), stack_kernel_ptr<3>(),
                                    stack_kernel_ptr<4>()};
   if (su == 0) return ordered[M - 1];
-  if (fc == 5)  // some tensors resident: M = 2 / 3, stages of kStreamU chunks only
-    return M == 2 ? stream_kernel_ptr<2, kStreamU, 5>() : stream_kernel_ptr<3, kStreamU, 5>();
+  if (fc == 3 && M >= 2) {  // a group of a stream list with its activations resident (M = 2..4)
+    static void* const row[3] = {stream_kernel_ptr<2, kStreamU, 3>(), stream_kernel_ptr<3, kStreamU, 3>(),
+                                 stream_kernel_ptr<4, kStreamU, 3>()};
+    return row[M - 2];
+  }
   if (fc >= 3)  // resident activations: M = 1, stages of kStreamU chunks only
     return fc == 3 ? stream_kernel_ptr<1, kStreamU, 3>() : stream_kernel_ptr<1, kStreamU, 4>();
   if (fc == 0) return su == 2 ? StreamRow<2, 0>::at(M) : StreamRow<kStreamU, 0>::at(M);
@@ -729,23 +741,33 @@ void* select_stack_kernel(int M, int su, int fc) {
 // su: stream mode with stages of su chunks (weights + activation slice of M
 // rows), or 0 for ordered mode (weights only, stages of kStackU chunks).
 // fc 3 / 4 (resident activations): weights-only slots, one more barrier, and
-// the activation copies (rx_bytes) from the next 128-byte boundary; fc 5:
-// the same with slots that also hold a slice.
+// the activation copies (rx_bytes) from the next 128-byte boundary.
 int stack_smem_bytes(int su, int M, int fc, int rx_bytes = 0) {
   constexpr int nw = kStackNW;
   if (su == 0) return nw * kStackD * q4k::kStackU * q4k::Format<4>::kChunkBytes + nw * kStackD * 8;
   const int cb = fc == 2 ? q4k::Wide<6>::kChunkBytes : q4k::Format<4>::kChunkBytes;
-  const int xb = fc == 3 || fc == 4 ? 0 : M * q4k::Format<4>::kKPerChunk * 2;
+  const int xb = fc >= 3 ? 0 : M * q4k::Format<4>::kKPerChunk * 2;
   const int rings = nw * kStackD * su * (cb + xb);
   if (fc >= 3) return (rings + nw * kStackD * 8 + 8 + 127) / 128 * 128 + rx_bytes;
   return rings + nw * kStackD * 8;
+}
+
+// A persistent kernel's dynamic shared-memory limit is a property of the
+// function, shared by every stack that launches it with its own size: allow
+// the most one CTA per SM can take beside the function's static shared memory.
+cudaError_t allow_dynamic_smem(void* fn) {
+  cudaFuncAttributes a{};
+  cudaError_t err = cudaFuncGetAttributes(&a, fn);
+  if (err != cudaSuccess) return err;
+  return cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              kStackSmemLimit - static_cast<int>(a.sharedSizeBytes));
 }
 
 void free_stack(q4_stack* st) {
   if (st->exec) cudaGraphExecDestroy(st->exec);
   if (st->graph) cudaGraphDestroy(st->graph);
   if (st->entries_dev) cudaFree(st->entries_dev);
-  if (st->xprep_dev) cudaFree(st->xprep_dev);
+  if (st->xprep_dev) cudaFree(st->xprep_dev);  // also holds the groups' job tables
   if (st->chain_ops_dev) cudaFree(st->chain_ops_dev);
   if (st->workspace) cudaFree(st->workspace);
   delete st;
@@ -814,7 +836,7 @@ int create_persistent(const q4_stack_entry* entries, int n, int M, int su, const
   // mode keeps one per tile of every product
   const size_t counters = (static_cast<size_t>(independent ? total_tiles : max_t) * 4 + 255) / 256 * 256;
   int rx_bytes = 0;  // stream mode with resident activations: their bytes in shared memory
-  int fc_sel = fc;   // the kernel's class: fc, or 3 + fc (all resident), or 5 (some resident)
+  int fc_sel = fc;   // the kernel's class: fc, or 3 + fc (activations resident)
   // stream mode: per distinct (x, K, format) a chunk-major copy of x and its XInfo
   std::vector<q4k::XPrepJob> jobs;
   std::vector<size_t> job_of(static_cast<size_t>(n), 0), x16_off, info_off;
@@ -839,6 +861,15 @@ int create_persistent(const q4_stack_entry* entries, int n, int M, int su, const
       job_of[static_cast<size_t>(i)] = jdx;
     }
   }
+  // stream-mode groups (see below)
+  struct GroupPlan {
+    int su, fc;
+    long long rx;
+  };
+  std::vector<GroupPlan> plan;
+  std::vector<std::vector<int>> group_rx;  // per group and job: the job's offset in shared memory, or -1
+  std::vector<int> job_group(jobs.size(), -1);
+  const bool grouped = independent && Q4_TUNE_STREAM_GROUPS && M >= 2 && su == kStreamU && fc == 0;
   // ordered mode: one barrier flag per CTA
   const size_t flags_bytes = independent ? 0 : (static_cast<size_t>(dev.sms) * 4 + 255) / 256 * 256;
   const size_t flags_base = kWsHeader + partials_bytes(dev) + counters;
@@ -856,14 +887,52 @@ int create_persistent(const q4_stack_entry* entries, int n, int M, int su, const
     }
     // resident activations (stages of kStreamU).  M = 1, classes 0 / 1:
     // every CTA keeps each prepared tensor in shared memory when they all
-    // fit.  M = 2 / 3, class 0 (class 5): the tensors in the q4 geometry that
-    // fit beside the slots, narrowest first; a q8 product whose activations
-    // have such a copy reads it (half a chunk of it per q8 chunk); the other
-    // products' slices stay in the slots.  (At M = 4 the slots leave no room
-    // for 5120 values per row; with 14 warps per CTA instead of 16 there is,
-    // but the decode stream ran 5 % slower than with every slice in the slots.)
+    // fit, and the stages carry weights only.
     for (auto& j : jobs) j.rx_off = -1;
-    if (M == 1 && su == kStreamU && fc <= 1) {
+    // M >= 2, q4 / q8 lists with stages of kStreamU: the list runs as groups,
+    // one launch each.  The prepared tensors, narrowest first, join the first
+    // group whose resident activations they fit beside the weights-only
+    // stages; a tensor that fits no group leaves its products to one group
+    // whose stages carry the activation slices.  Every CTA of a resident group
+    // copies the group's tensors into shared memory once.  (On the decode
+    // stream, interleaved on one box: M = 4 5,302 GB/s at 1,530 MHz against
+    // 5,124 at 1,552 as one launch with every slice in the slots; M = 2 and 3
+    // +3 % and +2 % against one launch that kept only the 5120-value inputs
+    // resident beside slots with room for slices.  A resident 17,408-value
+    // group with stages of two chunks streamed no faster than its slices in
+    // stages of four and executed 146 instead of ~127 warp instructions per
+    // chunk.)
+    if (grouped) {
+      std::vector<size_t> order(jobs.size());
+      for (size_t k = 0; k < jobs.size(); ++k) order[k] = k;
+      std::stable_sort(order.begin(), order.end(), [&](size_t a, size_t b) { return jobs[a].K < jobs[b].K; });
+      int ring_group = -1;
+      auto fits = [&](int gsu, long long rx) {
+        return rx < (1LL << 30) && stack_smem_bytes(gsu, M, 3, static_cast<int>(rx)) <= kStackSmemLimit;
+      };
+      for (size_t k : order) {
+        // the copy's bytes, resident only when a whole number of 128-byte
+        // blocks (always, with stages of four chunks: K % 128 == 0)
+        const long long bytes = static_cast<long long>(M) * jobs[k].K * 2;
+        int g = -1;
+        for (size_t q = 0; q < plan.size() && g < 0; ++q)
+          if (plan[q].fc == 3 && bytes % 128 == 0 && fits(plan[q].su, plan[q].rx + bytes)) g = static_cast<int>(q);
+        if (g < 0) {
+          const int gsu = bytes % 128 == 0 && fits(kStreamU, bytes) ? kStreamU : 0;
+          if (gsu != 0 || ring_group < 0) {
+            plan.push_back(GroupPlan{gsu != 0 ? gsu : kStreamU, gsu != 0 ? 3 : 0, 0});
+            group_rx.emplace_back(jobs.size(), -1);
+            if (gsu == 0) ring_group = static_cast<int>(plan.size()) - 1;
+          }
+          g = gsu != 0 ? static_cast<int>(plan.size()) - 1 : ring_group;
+        }
+        if (plan[static_cast<size_t>(g)].fc == 3) {
+          group_rx[static_cast<size_t>(g)][k] = static_cast<int>(plan[static_cast<size_t>(g)].rx);
+          plan[static_cast<size_t>(g)].rx += bytes;
+        }
+        job_group[k] = g;
+      }
+    } else if (M == 1 && su == kStreamU && fc <= 1) {
       int off = 0;
       for (auto& j : jobs) {
         j.rx_off = off;
@@ -873,42 +942,50 @@ int create_persistent(const q4_stack_entry* entries, int n, int M, int su, const
         rx_bytes = off;
         fc_sel = fc + 3;
       }
-    } else if (Q4_TUNE_STREAM_MIXED && (M == 2 || M == 3) && su == kStreamU && fc == 0) {
-      std::vector<size_t> order;
-      for (size_t k = 0; k < jobs.size(); ++k)
-        if (jobs[k].KC == q4k::Format<4>::kKPerChunk) order.push_back(k);
-      std::stable_sort(order.begin(), order.end(), [&](size_t a, size_t b) { return jobs[a].K < jobs[b].K; });
-      int off = 0;
-      for (size_t k : order) {
-        const long long bytes = static_cast<long long>(M) * jobs[k].K * 2;  // a multiple of 128: K % 64 == 0
-        if (stack_smem_bytes(su, M, 5, static_cast<int>(std::min<long long>(off + bytes, 1 << 30))) > kStackSmemLimit)
-          continue;
-        jobs[k].rx_off = off;
-        off += static_cast<int>(bytes);
-      }
-      if (off > 0) {
-        rx_bytes = off;
-        fc_sel = 5;
-      }
     }
     for (int i = 0; i < n; ++i) {
-      const q4k::XPrepJob* j = &jobs[job_of[static_cast<size_t>(i)]];
+      const size_t jk = job_of[static_cast<size_t>(i)];
+      const q4k::XPrepJob* j = &jobs[jk];
       host[static_cast<size_t>(i)].xc = j->xc;
-      if (fc_sel == 5 && j->rx_off < 0 && entries[i].bits == 8) {
-        for (const auto& r : jobs)  // the q4-geometry copy of the same activations, if resident
-          if (r.rx_off >= 0 && r.x == j->x && r.K == j->K) j = &r;
-      }
       host[static_cast<size_t>(i)].xinfo = j->info;
-      host[static_cast<size_t>(i)].rx_off = j->rx_off;
+      host[static_cast<size_t>(i)].rx_off =
+          grouped ? group_rx[static_cast<size_t>(job_group[jk])][jk] : j->rx_off;
     }
-    err = cudaMalloc(&st->xprep_dev, sizeof(q4k::XPrepJob) * jobs.size());
+    // the preparation's job table, then per group a copy with that group's
+    // shared-memory offsets (the tensors it stages)
+    std::vector<q4k::XPrepJob> tables(jobs);
+    for (size_t g = 0; g < plan.size(); ++g)
+      for (size_t k = 0; k < jobs.size(); ++k) {
+        tables.push_back(jobs[k]);
+        tables.back().rx_off = group_rx[g][k];
+      }
+    err = cudaMalloc(&st->xprep_dev, sizeof(q4k::XPrepJob) * tables.size());
     if (err == cudaSuccess)
-      err = cudaMemcpy(st->xprep_dev, jobs.data(), sizeof(q4k::XPrepJob) * jobs.size(), cudaMemcpyHostToDevice);
+      err = cudaMemcpy(st->xprep_dev, tables.data(), sizeof(q4k::XPrepJob) * tables.size(), cudaMemcpyHostToDevice);
     st->xprep_jobs = static_cast<int>(jobs.size());
     st->rx_bytes = rx_bytes;
     long long most = 0;
     for (const auto& j : jobs) most = std::max(most, static_cast<long long>(M) * j.K / 8);
     st->xprep_ctas = static_cast<int>(std::max(1LL, (most + q4k::kXPrepThreads - 1) / q4k::kXPrepThreads));
+  }
+  // groups: the entries ordered by group, each group's blocks (of its own
+  // stage size) numbered from 0
+  std::vector<size_t> group_first(plan.size() + 1, 0);
+  std::vector<long long> group_blocks(plan.size(), 0);
+  if (grouped) {
+    std::vector<q4k::StackEntryDev> sorted;
+    for (size_t g = 0; g < plan.size(); ++g) {
+      group_first[g] = sorted.size();
+      for (int i = 0; i < n; ++i) {
+        if (job_group[job_of[static_cast<size_t>(i)]] != static_cast<int>(g)) continue;
+        q4k::StackEntryDev d = host[static_cast<size_t>(i)];
+        d.blk_off = group_blocks[g];
+        group_blocks[g] += d.TC / plan[g].su;
+        sorted.push_back(d);
+      }
+    }
+    group_first[plan.size()] = sorted.size();
+    host.swap(sorted);
   }
   if (err == cudaSuccess) err = cudaMalloc(&st->entries_dev, sizeof(q4k::StackEntryDev) * host.size());
   if (err == cudaSuccess)
@@ -918,7 +995,7 @@ int create_persistent(const q4_stack_entry* entries, int n, int M, int su, const
   st->smem = stack_smem_bytes(su, M, fc_sel, rx_bytes);
   st->block = kStackNW * 32;
   st->grid = dev.sms;
-  err = cudaFuncSetAttribute(st->fn, cudaFuncAttributeMaxDynamicSharedMemorySize, st->smem);
+  err = allow_dynamic_smem(st->fn);
   if (err != cudaSuccess) return cuda_fail(err, "layer_stack_create: cudaFuncSetAttribute");
   int per_sm = 0;
   err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, st->fn, st->block, st->smem);
@@ -941,6 +1018,25 @@ int create_persistent(const q4_stack_entry* entries, int n, int M, int su, const
   p.rx_bytes = rx_bytes;
   st->persistent = true;
   st->launches = independent ? 2 : 1;  // stream mode: xprep_kernel + stream_kernel
+  for (size_t g = 0; grouped && g < plan.size(); ++g) {
+    q4_stack::Group grp;
+    grp.fn = select_stack_kernel(M, plan[g].su, plan[g].fc);
+    grp.smem = stack_smem_bytes(plan[g].su, M, plan[g].fc, static_cast<int>(plan[g].rx));
+    err = allow_dynamic_smem(grp.fn);
+    if (err != cudaSuccess) return cuda_fail(err, "layer_stack_create: cudaFuncSetAttribute");
+    err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, grp.fn, st->block, grp.smem);
+    if (err != cudaSuccess) return cuda_fail(err, "layer_stack_create: occupancy query");
+    if (per_sm < 1) return fail(Q4_ERR_UNSUPPORTED, "layer_stack_create: a stream kernel does not fit on an SM");
+    grp.params = p;
+    grp.params.entries = st->entries_dev + group_first[g];
+    grp.params.E = static_cast<int>(group_first[g + 1] - group_first[g]);
+    grp.params.TBg = group_blocks[g];
+    grp.params.Pg = static_cast<int>(group_blocks[g] < warps ? group_blocks[g] : warps);
+    grp.params.jobs = st->xprep_dev + (g + 1) * jobs.size();
+    grp.params.rx_bytes = static_cast<int>(plan[g].rx);
+    st->groups.push_back(grp);
+  }
+  if (grouped) st->launches = 1 + static_cast<int>(st->groups.size());
   return Q4_OK;
 }
 
@@ -1488,7 +1584,7 @@ int create_chain_persistent(const q4_chain_op* ops, int n, int M, const DeviceIn
   st->smem = static_cast<int>(smem);
   st->block = kStackNW * 32;
   st->grid = G;
-  err = cudaFuncSetAttribute(st->fn, cudaFuncAttributeMaxDynamicSharedMemorySize, st->smem);
+  err = allow_dynamic_smem(st->fn);
   if (err != cudaSuccess) return cuda_fail(err, "layer_chain_create: cudaFuncSetAttribute");
   int per_sm = 0;
   err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, st->fn, st->block, st->smem);
@@ -1672,6 +1768,17 @@ extern "C" Q4_API int layer_stack_run(q4_stack* st, void* stream) {
     }
     cfg.attrs = attr;
     cfg.numAttrs = 1;
+    // groups: one launch each, every one after the one before (programmatic
+    // dependent launch: a group starts its weight copies while the one before
+    // finishes, and waits for it before it reads an activation or the
+    // workspace)
+    for (auto& grp : st->groups) {
+      cfg.dynamicSmemBytes = static_cast<size_t>(grp.smem);
+      void* gargs[] = {&grp.params};
+      cudaError_t err = cudaLaunchKernelExC(&cfg, grp.fn, gargs);
+      if (err != cudaSuccess) return cuda_fail(err, "layer_stack_run: stream group launch");
+    }
+    if (!st->groups.empty()) return Q4_OK;
     void* args[] = {&st->params};
     cudaError_t err = cudaLaunchKernelExC(&cfg, st->fn, args);
     return err == cudaSuccess ? Q4_OK : cuda_fail(err, "layer_stack_run: persistent launch");

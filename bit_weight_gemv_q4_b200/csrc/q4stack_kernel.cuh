@@ -50,7 +50,7 @@ struct XPrepJob {
   XInfo* info;
   long long K;
   int KC;
-  int rx_off;         // stream mode: offset of xc's copy in shared memory, or -1 (not resident)
+  int rx_off;         // stream mode: offset of xc's copy in a group's shared memory, or -1 (not that group's)
 };
 
 struct StackEntryDev {
@@ -63,7 +63,7 @@ struct StackEntryDev {
   long long blk_off;  // first block of this product in the concatenated sequence (stream mode)
   int T, C, bits, P, khalf;
   int tile_off;       // first counter of this product (stream mode)
-  int rx_off;         // stream mode: its resident activations' offset in shared memory, or -1 (in the slots)
+  int rx_off;         // stream mode with resident activations: their offset in shared memory
 };
 
 struct StackParams {
@@ -486,14 +486,9 @@ template <int FC>
 struct FormatClass {
   // classes 3 and 4 are classes 0 and 1 with resident activations: every CTA
   // copies each prepared activation tensor into shared memory once, and the
-  // stages carry weights only.  Class 5 is class 0 with the activation
-  // tensors that fit resident (in the q4 geometry: 64 values per row per
-  // chunk, which a q8 chunk reads half of) and the others carried through the
-  // slots (rx_off < 0).
-  static constexpr bool kResidentX = FC == 3 || FC == 4;
-  static constexpr bool kMixedX = FC == 5;
-  static constexpr bool kStagedX = FC >= 3;  // some tensor is copied in at the start
-  static constexpr int kClass = FC == 5 ? 0 : FC >= 3 ? FC - 3 : FC;
+  // stages carry weights only
+  static constexpr bool kResidentX = FC >= 3;
+  static constexpr int kClass = FC >= 3 ? FC - 3 : FC;
   static constexpr int kMaxChunkBytes = kClass == 2 ? Wide<6>::kChunkBytes : Format<4>::kChunkBytes;
 };
 
@@ -522,7 +517,6 @@ struct StreamProducer {
   const uint16_t* xc = nullptr;  // the product's chunk-major activations
   int cpos = 0;                  // chunk of the tile where the next stage starts
   int C = 0, KC = 0;
-  bool rx = false;               // class 5: the product's activations are resident (the slots carry weights only)
 
   __device__ __forceinline__ void enter(const StackParams& sp, int entry, long long lb) {
     const StackEntryDev& en = sp.entries[entry];
@@ -535,7 +529,6 @@ struct StreamProducer {
     const long long in_entry = en.TC / SU - lb;
     left_entry = static_cast<int>(in_entry < left_total ? in_entry : left_total);
     xc = en.xc;
-    rx = FormatClass<FC>::kMixedX && en.rx_off >= 0;
     C = en.C;
     KC = en.bits == 8 ? Format<8>::kKPerChunk : Format<4>::kKPerChunk;
     const int bpt = en.C / SU;
@@ -555,9 +548,9 @@ struct StreamProducer {
       // the slots carry weights only; the activations are already resident
       bulk_copy_g2s_if(lane == 0, dst, src, bytes, bar, policy);
     } else {
-      const uint32_t xb = rx ? 0u : x_bytes();
-      bulk_copy_g2s_x_if(lane == 0, dst, src, bytes, dst + StreamSlot<SU, M, FC>::kWeightBytes, x_src(), xb,
-                         with_x && !rx, bar, policy);
+      const uint32_t xb = x_bytes();
+      bulk_copy_g2s_x_if(lane == 0, dst, src, bytes, dst + StreamSlot<SU, M, FC>::kWeightBytes, x_src(), xb, with_x,
+                         bar, policy);
       if (!with_x) {
         *x_later = x_src();
         *x_later_bytes = xb;
@@ -636,16 +629,9 @@ __device__ __forceinline__ bool stream_segment(const SP& sp, const StackEntryDev
   // the chunk's slice of the tensor's copy): row min(gi, M-1) (columns >= M
   // only feed outputs that are never stored), 8 values at 8 ti
   constexpr bool RX = FormatClass<FC>::kResidentX;
-  constexpr bool MX = FormatClass<FC>::kMixedX;
-  const bool rxe = RX || (MX && ep->rx_off >= 0);  // this product's activations are resident
-  // a resident copy has the product's own chunk layout (RX: KC values per row
-  // per chunk) or the q4 geometry (MX: 64 per row; q8 chunk c is half
-  // (c & 1) of chunk c / 2)
-  constexpr int RKC = MX ? Format<4>::kKPerChunk : KC;
   const uint32_t xrow = ((gi < M ? gi : M - 1) * KC + 8 * ti) * 2;
   const uint32_t xlane = StreamSlot<SU, M, FC>::kWeightBytes + xrow;
-  const uint32_t xres = rxe ? rg.rx + static_cast<uint32_t>(ep->rx_off) + ((gi < M ? gi : M - 1) * RKC + 8 * ti) * 2
-                            : 0u;
+  const uint32_t xres = RX ? rg.rx + static_cast<uint32_t>(ep->rx_off) + xrow : 0u;
   r = static_cast<int>(floor_div(lb0, bpt));
   c = static_cast<int>(lb0 - static_cast<long long>(r) * bpt) * U;
   const int n_stages = static_cast<int>(nblk);  // a warp's range is far below 2^31 stages
@@ -653,18 +639,10 @@ __device__ __forceinline__ bool stream_segment(const SP& sp, const StackEntryDev
     const uint32_t bar = rg.bars + 8 * rg.slot;
     if (!mbar_wait_bounded(bar, rg.phase, sp.timeout_ns)) return false;
     const uint32_t stage = rg.ring + rg.slot * SLOT;
-    // the stage's first activation fragment (c is a multiple of U, so even)
-    const uint32_t xst = RX    ? xres + static_cast<uint32_t>(c) * (M * KC * 2)
-                         : !MX ? stage + xlane
-                         : rxe ? xres + static_cast<uint32_t>(FB == 8 ? c >> 1 : c) * (M * RKC * 2)
-                               : stage + xlane;
 #pragma unroll
     for (int j = 0; j < U; ++j) {
       ChunkRegs cr;
-      constexpr int kRowBytes = M * KC * 2;
-      uint32_t xaddr = xst + j * kRowBytes;
-      if (MX && FB == 8 && j > 0)  // resident q8: chunk j is half (j & 1) of q4-geometry chunk j / 2
-        xaddr = xst + (rxe ? (j >> 1) * (M * RKC * 2) + (j & 1) * KC * 2 : j * kRowBytes);
+      const uint32_t xaddr = RX ? xres + static_cast<uint32_t>(c + j) * (M * KC * 2) : stage + xlane + j * M * KC * 2;
       const uint4 xa = lds128(xaddr);
       const uint4 xb = FB == 4 ? lds128(xaddr + 64) : make_uint4(0, 0, 0, 0);
       cr.codes[0] = lds128(stage + j * CB + 16 * lane);
@@ -744,7 +722,7 @@ __device__ __forceinline__ void stage_resident_x(const StackParams& sp, uint32_t
 template <int M, int NW, int D, int SU, int FC>
 __global__ void __launch_bounds__(NW * 32, 1) stream_kernel(const StackParams sp) {
   constexpr int SLOT = StreamSlot<SU, M, FC>::kBytes;
-  constexpr bool RX = FormatClass<FC>::kStagedX;  // some activation tensor is resident
+  constexpr bool RX = FormatClass<FC>::kResidentX;
   extern __shared__ __align__(128) unsigned char smem[];
 
   const int lane = threadIdx.x & 31;
@@ -803,13 +781,12 @@ __global__ void __launch_bounds__(NW * 32, 1) stream_kernel(const StackParams sp
   grid_dependents_launch();
   if constexpr (RX) {
     if (threadIdx.x == 0) stage_resident_x<M>(sp, rg.rx, xbar);
-  }
-  if constexpr (!FormatClass<FC>::kResidentX) {
+  } else {
 #pragma unroll
     for (int s = 0; s < D; ++s) {
-      if (s < rg.in_flight)  // a slice of 0 bytes: a resident product's stage (class 5)
-        bulk_copy_x_if(lane == 0 && x_later_bytes[s] != 0, rg.ring + s * SLOT + StreamSlot<SU, M, FC>::kWeightBytes,
-                       x_later[s], x_later_bytes[s], rg.bars + 8 * s);
+      if (s < rg.in_flight)
+        bulk_copy_x_if(lane == 0, rg.ring + s * SLOT + StreamSlot<SU, M, FC>::kWeightBytes, x_later[s],
+                       x_later_bytes[s], rg.bars + 8 * s);
     }
   }
 

@@ -95,14 +95,17 @@ def test_stream_mode_of_independent_products(q4, M, tensors):
     """Stream mode splits the concatenated products between warps differently
     from one call per product: the outputs are compared with the oracle (every
     row) and with single calls within the product tolerance, and two runs are
-    bitwise identical.  With stages of four chunks at M = 2 and 3 the
-    activations of K 256 and 5120 stay resident in shared memory (q8 products
-    with K 5120 and 256 read the q4 layout's copy), while those of K 17408 and
-    of the q8 product with K 128 (no q4 product shares them) travel with the
-    weights; at M = 1 every tensor is resident, at M = 4 none."""
+    bitwise identical."""
     torch = H.torch()
     st = workloads.DeviceStream(tensors, M, flags=q4.Q4_STACK_INDEPENDENT)
-    assert st.stack.launches() == 2  # activation preparation + stream kernel
+    # activation preparation + one stream kernel per group: at M = 1 one group
+    # (every activation resident); with stages of four chunks at M >= 2 the
+    # products are grouped so that each group's activations stay resident
+    # (K 128 / 256 / 5120 together and K 17408 apart, resident at M = 2, with
+    # its slices in the stages at M = 3 and 4; at M = 4 the q8 copy of the
+    # 5120-value input needs a group of its own)
+    expect = 2 if M == 1 or tensors is MIXED else {2: 3, 3: 3, 4: 4}[M]
+    assert st.stack.launches() == expect
     st.run()
     st.check()
     first = [_y(st, i).copy() for i in range(len(tensors))]
@@ -142,8 +145,9 @@ def test_full_decode_stream_sampled(q4, M, mode):
     torch = H.torch()
     tensors = workloads.decode_stream(fused=True)
     st = workloads.DeviceStream(tensors, M, flags=q4.Q4_STACK_ORDERED if mode == "ordered" else q4.Q4_STACK_INDEPENDENT)
-    # one persistent kernel for the 257 products (stream mode: after xprep_kernel)
-    assert st.stack.launches() == (1 if mode == "ordered" else 2)
+    # one persistent kernel for the 257 products (stream mode: after xprep_kernel;
+    # at M = 4 two groups, the products of the 5120- and the 17,408-value inputs)
+    assert st.stack.launches() == (1 if mode == "ordered" else 2 if M == 1 else 3)
     st.run()
     st.run()
     st.check()

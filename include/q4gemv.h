@@ -405,7 +405,11 @@ typedef struct q4_stack q4_stack;
  * earlier product).  One kernel treats the concatenated products
  * as a single work-split problem: every warp streams one contiguous range
  * across product boundaries with no synchronisation, so the HBM stream never
- * pauses between products.  Before it, a small kernel prepares each distinct
+ * pauses between products.  At M >= 2 (q4 / q8 lists with four chunks per
+ * stage) the products are run in groups, one such launch each, formed so
+ * that every group's activations fit in shared memory beside its weight
+ * stages (products whose activations fit nowhere form one group that
+ * carries them with the weights); layer_stack_launches counts them.  Before it, a small kernel prepares each distinct
  * activation tensor: when a power of two 2^s makes every x * 2^-s exactly
  * representable in fp16, the products of that tensor run on that fp16 copy
  * (a shorter decode; outputs scaled back by 2^s, exactly), otherwise on x in

@@ -115,3 +115,21 @@ def test_traffic_comes_only_from_a_capture_of_the_current_kernel_source(monkeypa
     assert bench.profiled_traffic() == per
     monkeypatch.setattr(bench, "kernel_source_sha", lambda: "f" * 16 if sha != "f" * 16 else "0" * 16)
     assert bench.profiled_traffic() is None
+
+
+def test_oracle_timing_per_configuration_on_one_core():
+    """The CPU baseline's per-configuration oracle timing, as the bench runs
+    it for its one-core figures: a fresh process whose OpenMP runtime has one
+    thread, every configuration (1-4 and the decode stream) with its rate,
+    the implied time for the whole configuration and the sample it timed."""
+    r = _run_bench(["--oracle-configs", "--cpu-seconds", "0.1"], {"OMP_NUM_THREADS": "1"})
+    assert r.returncode == 0, r.stderr[-2000:]
+    out = json.loads(r.stdout.strip().splitlines()[-1])
+    assert out["threads"] == 1
+    names = {"q4_4096x4096_M1", "layer_q4_M1", "layer_q4_M4", "head.mapped_q8_65536x5120_M1",
+             "head.full_q8_248320x5120_M1", "decode_stream_M1"}
+    assert names <= set(out)
+    for name in names:
+        c = out[name]
+        assert c["GBps"] > 0 and c["us"] > 0 and c["seconds"] > 0, name
+        assert c["sample"] == "whole" or " of " in c["sample"], name

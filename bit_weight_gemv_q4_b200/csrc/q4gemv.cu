@@ -895,7 +895,7 @@ int create_persistent(const q4_stack_entry* entries, int n, int M, int su, const
     // stages; a tensor that fits no group leaves its products to one group
     // whose stages carry the activation slices.  Every CTA of a resident group
     // copies the group's tensors into shared memory once.  (On the decode
-    // stream, interleaved on one box: M = 4 5,302 GB/s at 1,530 MHz against
+    // stream, interleaved on one B200: M = 4 5,302 GB/s at 1,530 MHz against
     // 5,124 at 1,552 as one launch with every slice in the slots; M = 2 and 3
     // +3 % and +2 % against one launch that kept only the 5120-value inputs
     // resident beside slots with room for slices.  A resident 17,408-value

@@ -112,7 +112,7 @@ extern "C" {
 #define Q4_ERR_BUFFER_TOO_SMALL (-4) /* output or workspace smaller than required */
 #define Q4_ERR_CUDA (-5)             /* a CUDA call failed (message has the CUDA error) */
 #define Q4_ERR_TIMEOUT (-6)          /* a bounded device wait gave up (see q4_workspace_check) */
-#define Q4_ERR_UNSUPPORTED (-7)      /* no sm_100 device, or a request this build does not serve */
+#define Q4_ERR_UNSUPPORTED (-7)      /* no sm_100 device, or a request this library does not serve */
 
 /* Message of the last failing call on this thread ("" if none). */
 Q4_API const char* q4_last_error(void);

@@ -657,7 +657,7 @@ def run_ours(args, d: Dist):
         },
         "roofline": {
             "bound": "hbm",
-            "kernel": "stream_kernel<M=1> (the whole decode stream in one launch; timed as the step, which also holds the activation preparation xprep_kernel, 0.5 % of its serialised time under ncu)",
+            "kernel": "stream_kernel<M=1> (the whole decode stream in one launch; timed as the step, which also holds the activation preparation xprep_kernel, 0.4 % of its serialised time under ncu)",
             "achieved": round(achieved, 1),
             "peak": peak,
             "unit": "GB/s",
